@@ -1,0 +1,136 @@
+"""CPU oracle for the block selected inverse -- TEST INFRASTRUCTURE ONLY.
+
+Plain double-precision C (``selinv_oracle.c``) behind a NumPy front end.
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+and reference legs may import this package; the product path never does, and
+the oracle shares no code with the CUDA library.
+
+What it computes follows gabp-sparse-inv 0.3.2 (PyPI page), "Implemented and
+tested kernels" -> Chain and Tree, and the "Quickstart" conventions: the
+on-pattern blocks of A^-1 (G_diag, G_lower / G_edge), log det A from the same
+factorisation, and the chain solve x = A^-1 r.  The C file's header states the
+recursion and every reading taken where the pages are silent.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "selinv_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB = os.path.join(_BUILD, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/_build/liboracle.so`` with gcc."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        os.makedirs(_BUILD, exist_ok=True)
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c99", "-fopenmp", "-fPIC", "-shared",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _bind(path):
+    """Load an oracle shared library and declare its signatures."""
+    lib = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    I64 = ctypes.c_int64
+    lib.oracle_chain.argtypes = [P, P, I64, I64, ctypes.c_int, P, P, P, P, P, P, P]
+    lib.oracle_chain.restype = ctypes.c_int
+    lib.oracle_tree.argtypes = [P, I64, I64, ctypes.c_int, P, P, P, P, P, P]
+    lib.oracle_tree.restype = ctypes.c_int
+    lib.oracle_threads.argtypes = []
+    lib.oracle_threads.restype = ctypes.c_int
+    return lib
+
+
+def _load(lib=None):
+    global _lib
+    if lib is not None:
+        return lib
+    if _lib is None:
+        _lib = _bind(build())
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f64(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float64)
+
+
+def threads() -> int:
+    """Number of OpenMP threads the oracle's batch loop runs on."""
+    return int(_load().oracle_threads())
+
+
+def chain(diag, lower, rhs=None, want_g=True, lib=None):
+    """Selected inverse of block-tridiagonal SPD chains.
+
+    diag [..., L, b, b] (lower triangle read), lower [..., L-1, b, b] with
+    lower[i] = A_{i+1,i}; optional rhs [..., L, b].
+    Returns dict with G_diag [..., L, b, b], G_lower [..., L-1, b, b],
+    logdet [...], x [..., L, b] (if rhs), info [...] (-1 ok, else the first
+    block whose Schur complement is not positive definite) and asym [...]
+    (largest |G - G^T| of a diagonal block before symmetrisation).
+    """
+    diag = _f64(diag)
+    lead = diag.shape[:-3]
+    L, b = diag.shape[-3], diag.shape[-1]
+    batch = int(np.prod(lead)) if lead else 1
+    if lower is None or L == 1:
+        lower = np.zeros(lead + (max(L - 1, 0), b, b))
+    lower = _f64(lower)
+    assert lower.shape == lead + (L - 1, b, b)
+    G_diag = np.empty(lead + (L, b, b)) if want_g else None
+    G_lower = np.empty(lead + (L - 1, b, b)) if want_g else None
+    logdet = np.empty(lead)
+    info = np.empty(lead, dtype=np.int32)
+    asym = np.zeros(lead)
+    x = None
+    if rhs is not None:
+        rhs = _f64(rhs)
+        assert rhs.shape == lead + (L, b)
+        x = np.empty(lead + (L, b))
+    rc = _load(lib).oracle_chain(_ptr(diag), _ptr(lower) if L > 1 else None, batch, L, b,
+                              _ptr(G_diag), _ptr(G_lower), _ptr(logdet), _ptr(rhs), _ptr(x),
+                              _ptr(info), _ptr(asym))
+    if rc != 0:
+        raise ValueError("oracle_chain: invalid arguments")
+    return {"G_diag": G_diag, "G_lower": G_lower, "logdet": logdet, "x": x,
+            "info": info, "asym": asym}
+
+
+def tree(parent, diag, edge, lib=None):
+    """Selected inverse of block-tree SPD matrices.
+
+    parent [..., n] int (root = -1), diag [..., n, b, b], edge [..., n, b, b]
+    with edge[v] = A_{parent(v),v} (root slot ignored).  Returns dict with
+    G_diag, G_edge (root slot 0), logdet [...] and info [...] (-1 ok, node of
+    a failing pivot, or -2 for a parent array that is not one rooted tree).
+    """
+    diag = _f64(diag)
+    edge = _f64(edge)
+    parent = np.ascontiguousarray(parent, dtype=np.int32)
+    lead = parent.shape[:-1]
+    n, b = diag.shape[-3], diag.shape[-1]
+    trees = int(np.prod(lead)) if lead else 1
+    assert diag.shape == lead + (n, b, b) and edge.shape == diag.shape
+    G_diag = np.empty_like(diag)
+    G_edge = np.empty_like(diag)
+    logdet = np.empty(lead)
+    info = np.empty(lead, dtype=np.int32)
+    rc = _load(lib).oracle_tree(_ptr(parent), trees, n, b, _ptr(diag), _ptr(edge),
+                             _ptr(G_diag), _ptr(G_edge), _ptr(logdet), _ptr(info))
+    if rc != 0:
+        raise ValueError("oracle_tree: invalid arguments")
+    return {"G_diag": G_diag, "G_edge": G_edge, "logdet": logdet, "info": info}

@@ -1,0 +1,373 @@
+/*
+ * Oracle for the block selected inverse -- TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, obviously-correct CPU implementation in double precision of
+ * what the GPU library computes.  Only the tests, the smoke check and the
+ * bench's CPU-baseline / reference arm may load it; the product path never
+ * does.  It shares no code, header or table with the CUDA library.
+ *
+ * Sources (gabp-sparse-inv 0.3.2, PyPI page):
+ *   - "Implemented and tested kernels" -> Chain: block LDL^T factorisation of
+ *     a block-tridiagonal SPD matrix followed by the Takahashi back-recursion,
+ *     returning the diagonal blocks and the first sub-diagonal blocks of A^-1.
+ *   - "Implemented and tested kernels" -> Tree: parent array, one edge block
+ *     per non-root node with edge[v] = A_{parent(v), v}; collect from the
+ *     leaves to the root, then distribute from the root to the leaves.
+ *   - "Quickstart": inputs diag [L,b,b], lower [L-1,b,b]; G_diag[v] = (A^-1)_vv,
+ *     G_edge[v] = (A^-1)_{parent(v),v}, root slot zero.
+ *   - "Gaussian sampling" / "junction_logdet": log det A from the same
+ *     LDL^T factorisation; "junction_solve": x = A^-1 r sharing that factor.
+ * (sparsax, PyPI page, "Features": a matrix that is not positive definite is
+ *  an error, reported here through info[] as the first failing block.)
+ *
+ * The recursion, in the pages' notation (S = Schur complement, B_i = lower[i]
+ * = A_{i+1,i}):
+ *   collect     S_0 = D_0,  S_{i+1} = D_{i+1} - B_i S_i^-1 B_i^T
+ *   log-det     log|A| = sum_i log det S_i
+ *   distribute  G_{L-1,L-1} = S_{L-1}^-1,
+ *               G_{i+1,i} = -G_{i+1,i+1} B_i S_i^-1,
+ *               G_ii      = S_i^-1 - S_i^-1 B_i^T G_{i+1,i}
+ *   solve       y_0 = r_0, y_{i+1} = r_{i+1} - B_i S_i^-1 y_i,
+ *               x_{L-1} = S_{L-1}^-1 y_{L-1}, x_i = S_i^-1 (y_i - B_i^T x_{i+1})
+ * Each S_i^-1 is formed from a textbook Cholesky factor S = R R^T (R lower):
+ * S^-1 = R^-T R^-1, and log det S = 2 sum_k log R_kk.
+ *
+ * Readings where the pages are silent: only the lower triangle of a diagonal
+ * block is read (the upper one is taken as its mirror); the returned G_ii is
+ * symmetrised as (G + G^T)/2 and the largest |G - G^T| before that is
+ * reported; a non-positive (or NaN) Cholesky pivot in block i stops that
+ * batch element with info = i (else info = -1).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---------- small dense helpers (row-major b x b, naive loops) ---------- */
+
+/* R := lower Cholesky factor of the symmetric matrix S (only S's lower
+ * triangle is read).  Returns 0, or -1 if a pivot is not > 0. */
+static int cholesky_lower(int b, const double *S, double *R)
+{
+    for (int i = 0; i < b * b; ++i) R[i] = 0.0;
+    for (int j = 0; j < b; ++j) {
+        double d = S[j * b + j];
+        for (int k = 0; k < j; ++k) d -= R[j * b + k] * R[j * b + k];
+        if (!(d > 0.0)) return -1;             /* also catches NaN */
+        double rjj = sqrt(d);
+        R[j * b + j] = rjj;
+        for (int i = j + 1; i < b; ++i) {
+            double s = S[i * b + j];
+            for (int k = 0; k < j; ++k) s -= R[i * b + k] * R[j * b + k];
+            R[i * b + j] = s / rjj;
+        }
+    }
+    return 0;
+}
+
+/* Rinv := R^-1 for lower-triangular R (column-by-column forward substitution). */
+static void lower_inverse(int b, const double *R, double *Rinv)
+{
+    for (int i = 0; i < b * b; ++i) Rinv[i] = 0.0;
+    for (int j = 0; j < b; ++j) {
+        Rinv[j * b + j] = 1.0 / R[j * b + j];
+        for (int i = j + 1; i < b; ++i) {
+            double s = 0.0;
+            for (int k = j; k < i; ++k) s += R[i * b + k] * Rinv[k * b + j];
+            Rinv[i * b + j] = -s / R[i * b + i];
+        }
+    }
+}
+
+/* C := op(A) * op(B), op = identity or transpose; all b x b. */
+static void matmul(int b, const double *A, int ta, const double *B, int tb, double *C)
+{
+    for (int i = 0; i < b; ++i)
+        for (int j = 0; j < b; ++j) {
+            double s = 0.0;
+            for (int k = 0; k < b; ++k) {
+                double a = ta ? A[k * b + i] : A[i * b + k];
+                double c = tb ? B[j * b + k] : B[k * b + j];
+                s += a * c;
+            }
+            C[i * b + j] = s;
+        }
+}
+
+/* y := op(A) x for a b x b matrix and a length-b vector. */
+static void matvec(int b, const double *A, int ta, const double *x, double *y)
+{
+    for (int i = 0; i < b; ++i) {
+        double s = 0.0;
+        for (int k = 0; k < b; ++k) s += (ta ? A[k * b + i] : A[i * b + k]) * x[k];
+        y[i] = s;
+    }
+}
+
+/* Full symmetric copy of a block from its lower triangle. */
+static void sym_from_lower(int b, const double *D, double *S)
+{
+    for (int i = 0; i < b; ++i)
+        for (int j = 0; j < b; ++j)
+            S[i * b + j] = (j <= i) ? D[i * b + j] : D[j * b + i];
+}
+
+/* Factor S, form S^-1 = R^-T R^-1, return log det S (2 sum log R_kk).
+ * Returns 0 or -1 (not positive definite).  work holds 2 b*b doubles. */
+static int spd_inverse_logdet(int b, const double *S, double *Sinv, double *logdet, double *work)
+{
+    double *R = work, *Rinv = work + (size_t)b * b;
+    if (cholesky_lower(b, S, R) != 0) return -1;
+    double ld = 0.0;
+    for (int k = 0; k < b; ++k) ld += 2.0 * log(R[k * b + k]);
+    *logdet = ld;
+    lower_inverse(b, R, Rinv);
+    matmul(b, Rinv, 1, Rinv, 0, Sinv);         /* R^-T R^-1 */
+    return 0;
+}
+
+/* G := (G + G^T)/2, returning the largest |G - G^T| seen before. */
+static double symmetrise(int b, double *G)
+{
+    double worst = 0.0;
+    for (int i = 0; i < b; ++i)
+        for (int j = 0; j < i; ++j) {
+            double d = fabs(G[i * b + j] - G[j * b + i]);
+            if (d > worst) worst = d;
+            double m = 0.5 * (G[i * b + j] + G[j * b + i]);
+            G[i * b + j] = m;
+            G[j * b + i] = m;
+        }
+    return worst;
+}
+
+/* ------------------------------- chain ---------------------------------- */
+
+/* One block-tridiagonal chain.  Returns info (-1 ok, else failing block). */
+static int chain_one(int64_t L, int b, const double *diag, const double *lower,
+                     double *G_diag, double *G_lower, double *logdet_out,
+                     const double *rhs, double *x, double *asym_out)
+{
+    const size_t bb = (size_t)b * b;
+    double *Sinv = malloc(sizeof(double) * bb * (size_t)L);  /* S_i^-1, all i */
+    double *S = malloc(sizeof(double) * bb);
+    double *T1 = malloc(sizeof(double) * bb);
+    double *T2 = malloc(sizeof(double) * bb);
+    double *work = malloc(sizeof(double) * 2 * bb);
+    double *y = rhs ? malloc(sizeof(double) * (size_t)b * (size_t)L) : NULL;
+    double *v1 = malloc(sizeof(double) * (size_t)b);
+    double *v2 = malloc(sizeof(double) * (size_t)b);
+    int info = -1;
+    double logdet = 0.0, asym = 0.0;
+
+    /* collect: S_0 = D_0; S_{i+1} = D_{i+1} - B_i S_i^-1 B_i^T */
+    sym_from_lower(b, diag, S);
+    for (int64_t i = 0; i < L; ++i) {
+        double ld;
+        if (spd_inverse_logdet(b, S, Sinv + bb * i, &ld, work) != 0) { info = (int)i; goto done; }
+        logdet += ld;
+        if (i + 1 < L) {
+            const double *Bi = lower + bb * i;
+            matmul(b, Bi, 0, Sinv + bb * i, 0, T1);          /* B_i S_i^-1 */
+            matmul(b, T1, 0, Bi, 1, T2);                      /* B_i S_i^-1 B_i^T */
+            sym_from_lower(b, diag + bb * (i + 1), S);
+            for (size_t k = 0; k < bb; ++k) S[k] -= T2[k];
+        }
+    }
+    if (logdet_out) *logdet_out = logdet;
+
+    /* distribute: G_{L-1} = S_{L-1}^-1, then the Takahashi back-recursion */
+    if (G_diag) {
+        memcpy(G_diag + bb * (L - 1), Sinv + bb * (L - 1), sizeof(double) * bb);
+        double a = symmetrise(b, G_diag + bb * (L - 1));
+        if (a > asym) asym = a;
+        for (int64_t i = L - 2; i >= 0; --i) {
+            const double *Bi = lower + bb * i;
+            double *Gl = G_lower + bb * i;
+            double *Gii = G_diag + bb * i;
+            const double *Gn = G_diag + bb * (i + 1);
+            /* G_{i+1,i} = -G_{i+1,i+1} B_i S_i^-1 */
+            matmul(b, Gn, 0, Bi, 0, T1);
+            matmul(b, T1, 0, Sinv + bb * i, 0, T2);
+            for (size_t k = 0; k < bb; ++k) Gl[k] = -T2[k];
+            /* G_ii = S_i^-1 - S_i^-1 B_i^T G_{i+1,i} */
+            matmul(b, Sinv + bb * i, 0, Bi, 1, T1);
+            matmul(b, T1, 0, Gl, 0, T2);
+            for (size_t k = 0; k < bb; ++k) Gii[k] = Sinv[bb * i + k] - T2[k];
+            a = symmetrise(b, Gii);
+            if (a > asym) asym = a;
+        }
+    }
+
+    /* solve with the same factor */
+    if (rhs && x) {
+        memcpy(y, rhs, sizeof(double) * (size_t)b);
+        for (int64_t i = 0; i + 1 < L; ++i) {
+            /* y_{i+1} = r_{i+1} - B_i S_i^-1 y_i */
+            matvec(b, Sinv + bb * i, 0, y + b * i, v1);
+            matvec(b, lower + bb * i, 0, v1, v2);
+            for (int k = 0; k < b; ++k) y[b * (i + 1) + k] = rhs[b * (i + 1) + k] - v2[k];
+        }
+        matvec(b, Sinv + bb * (L - 1), 0, y + b * (L - 1), x + b * (L - 1));
+        for (int64_t i = L - 2; i >= 0; --i) {
+            /* x_i = S_i^-1 (y_i - B_i^T x_{i+1}) */
+            matvec(b, lower + bb * i, 1, x + b * (i + 1), v1);
+            for (int k = 0; k < b; ++k) v2[k] = y[b * i + k] - v1[k];
+            matvec(b, Sinv + bb * i, 0, v2, x + b * i);
+        }
+    }
+done:
+    if (asym_out) *asym_out = asym;
+    free(Sinv); free(S); free(T1); free(T2); free(work); free(y); free(v1); free(v2);
+    return info;
+}
+
+/*
+ * Batched chain.  diag [batch,L,b,b], lower [batch,L-1,b,b] (row-major,
+ * contiguous).  Any of G_diag/G_lower (given together), logdet, rhs/x
+ * (given together), asym may be NULL.  info [batch] is required.
+ * Batch elements are independent; they are spread over OpenMP threads.
+ */
+int oracle_chain(const double *diag, const double *lower, int64_t batch, int64_t L, int b,
+                 double *G_diag, double *G_lower, double *logdet,
+                 const double *rhs, double *x, int32_t *info, double *asym)
+{
+    if (batch < 0 || L < 1 || b < 1 || !diag || !info || (L > 1 && !lower)) return 1;
+    const size_t bb = (size_t)b * b;
+    int64_t e;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (e = 0; e < batch; ++e) {
+        info[e] = chain_one(L, b, diag + bb * L * e, lower ? lower + bb * (L - 1) * e : NULL,
+                            G_diag ? G_diag + bb * L * e : NULL,
+                            G_lower ? G_lower + bb * (L - 1) * e : NULL,
+                            logdet ? logdet + e : NULL,
+                            rhs ? rhs + (size_t)b * L * e : NULL,
+                            x ? x + (size_t)b * L * e : NULL,
+                            asym ? asym + e : NULL);
+    }
+    return 0;
+}
+
+/* -------------------------------- tree ---------------------------------- */
+
+/* One rooted tree (parent[root] = -1).  Collect in reverse breadth-first
+ * order (every child before its parent; children summed in ascending
+ * index), distribute in breadth-first order.  Returns info, or -2 if the
+ * parent array is not a single rooted tree. */
+static int tree_one(int64_t n, int b, const int32_t *parent, const double *diag,
+                    const double *edge, double *G_diag, double *G_edge, double *logdet_out)
+{
+    const size_t bb = (size_t)b * b;
+    int info = -1;
+    int64_t root = -1;
+    for (int64_t v = 0; v < n; ++v) {
+        if (parent[v] == -1) { if (root >= 0) return -2; root = v; }
+        else if (parent[v] < 0 || parent[v] >= n || parent[v] == v) return -2;
+    }
+    if (root < 0) return -2;
+
+    /* children lists (ascending, since v is visited in increasing order) */
+    int64_t *count = calloc((size_t)n + 1, sizeof(int64_t));
+    int64_t *child = malloc(sizeof(int64_t) * (size_t)(n > 0 ? n : 1));
+    int64_t *order = malloc(sizeof(int64_t) * (size_t)n);
+    for (int64_t v = 0; v < n; ++v) if (parent[v] >= 0) count[parent[v] + 1]++;
+    for (int64_t v = 0; v < n; ++v) count[v + 1] += count[v];
+    int64_t *fill = malloc(sizeof(int64_t) * (size_t)n);
+    for (int64_t v = 0; v < n; ++v) fill[v] = count[v];
+    for (int64_t v = 0; v < n; ++v) if (parent[v] >= 0) child[fill[parent[v]]++] = v;
+
+    /* breadth-first order from the root; a cycle leaves nodes unreached */
+    int64_t head = 0, tail = 0;
+    order[tail++] = root;
+    while (head < tail) {
+        int64_t v = order[head++];
+        for (int64_t k = count[v]; k < count[v + 1]; ++k) order[tail++] = child[k];
+    }
+    double *Sinv = NULL, *S = NULL, *T1 = NULL, *T2 = NULL, *work = NULL;
+    if (tail != n) { info = -2; goto done; }
+
+    Sinv = malloc(sizeof(double) * bb * (size_t)n);
+    S = malloc(sizeof(double) * bb);
+    T1 = malloc(sizeof(double) * bb);
+    T2 = malloc(sizeof(double) * bb);
+    work = malloc(sizeof(double) * 2 * bb);
+    double logdet = 0.0;
+
+    /* collect: S_v = D_v - sum_{c in ch(v)} E_c S_c^-1 E_c^T, E_c = edge[c] */
+    for (int64_t t = n - 1; t >= 0; --t) {
+        int64_t v = order[t];
+        sym_from_lower(b, diag + bb * v, S);
+        for (int64_t k = count[v]; k < count[v + 1]; ++k) {
+            int64_t c = child[k];
+            matmul(b, edge + bb * c, 0, Sinv + bb * c, 0, T1);
+            matmul(b, T1, 0, edge + bb * c, 1, T2);
+            for (size_t q = 0; q < bb; ++q) S[q] -= T2[q];
+        }
+        double ld;
+        if (spd_inverse_logdet(b, S, Sinv + bb * v, &ld, work) != 0) { info = (int)v; goto done; }
+        logdet += ld;
+    }
+    if (logdet_out) *logdet_out = logdet;
+
+    /* distribute: G_root = S_root^-1; G_edge[v] = -G_p E_v S_v^-1;
+     * G_vv = S_v^-1 - S_v^-1 E_v^T G_edge[v] */
+    if (G_diag) {
+        memcpy(G_diag + bb * root, Sinv + bb * root, sizeof(double) * bb);
+        symmetrise(b, G_diag + bb * root);
+        memset(G_edge + bb * root, 0, sizeof(double) * bb);
+        for (int64_t t = 1; t < n; ++t) {
+            int64_t v = order[t], p = parent[v];
+            matmul(b, G_diag + bb * p, 0, edge + bb * v, 0, T1);
+            matmul(b, T1, 0, Sinv + bb * v, 0, T2);
+            for (size_t q = 0; q < bb; ++q) G_edge[bb * v + q] = -T2[q];
+            matmul(b, Sinv + bb * v, 0, edge + bb * v, 1, T1);
+            matmul(b, T1, 0, G_edge + bb * v, 0, T2);
+            for (size_t q = 0; q < bb; ++q) G_diag[bb * v + q] = Sinv[bb * v + q] - T2[q];
+            symmetrise(b, G_diag + bb * v);
+        }
+    }
+done:
+    free(count); free(child); free(order); free(fill);
+    free(Sinv); free(S); free(T1); free(T2); free(work);
+    return info;
+}
+
+/*
+ * Batched trees: parent [trees,n] (int32, root = -1), diag/edge
+ * [trees,n,b,b] (edge root slot ignored), outputs G_diag/G_edge
+ * [trees,n,b,b] (G_edge root slot set to 0), logdet [trees], info [trees]
+ * (-1 ok, node index of a failing pivot, or -2 for a malformed tree).
+ */
+int oracle_tree(const int32_t *parent, int64_t trees, int64_t n, int b,
+                const double *diag, const double *edge,
+                double *G_diag, double *G_edge, double *logdet, int32_t *info)
+{
+    if (trees < 0 || n < 1 || b < 1 || !parent || !diag || !edge || !info) return 1;
+    const size_t bb = (size_t)b * b;
+    int64_t t;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (t = 0; t < trees; ++t) {
+        info[t] = tree_one(n, b, parent + n * t, diag + bb * n * t, edge + bb * n * t,
+                           G_diag ? G_diag + bb * n * t : NULL,
+                           G_edge ? G_edge + bb * n * t : NULL,
+                           logdet ? logdet + t : NULL);
+    }
+    return 0;
+}
+
+/* Threads an OpenMP parallel region will use (for reporting core counts). */
+int oracle_threads(void)
+{
+    int n = 1;
+#pragma omp parallel
+    {
+#pragma omp single
+        {
+#ifdef _OPENMP
+            extern int omp_get_num_threads(void);
+            n = omp_get_num_threads();
+#endif
+        }
+    }
+    return n;
+}

@@ -1,0 +1,342 @@
+"""Pins of the CPU oracle to facts outside itself (tests only).
+
+Each pin returns an error that must stay below its tolerance.  They are
+written so that a plausible slip in the oracle (a dropped term, a wrong sign
+or index, a transposed operand) breaks at least one of them; the mutant test
+plants such slips in copies of the oracle's C source and checks exactly that.
+
+Sources:
+  gabp-sparse-inv 0.3.2 (PyPI page)
+    "Quickstart": G_diag[0] equals inv(A)[0:4,0:4] to 1e-10 for 8 blocks of
+      size 4 with diag_load 2.0; tree G_diag[0] likewise; the path tree
+      reproduces the chain block-for-block (the chain roots the path at its
+      last node, the tree at node 0).
+    "junction_solve" / "junction_logdet": solve and log det equal the dense
+      ones.
+    "Tests": every kernel against a dense fp64 oracle, symmetry / SPD
+      properties, independent residuals, leading batch dimensions.
+  sparsax (PyPI page) "Quick start": the 3 x 3 SPD example.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+
+import oracle
+from sparse_spd_selected_b200 import inputs
+from tests.dense import (balanced_parent, blk, chain_dense, path_parent, rel,
+                         star_parent, tree_dense)
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _chain_vs_dense(diag, lower, rhs, lib):
+    """Max relative error of every oracle output against the dense route."""
+    out = oracle.chain(diag, lower, rhs, lib=lib)
+    lead = diag.shape[:-3]
+    L, b = diag.shape[-3], diag.shape[-1]
+    worst = 0.0
+    for idx in np.ndindex(*lead) if lead else [()]:
+        if out["info"][idx] != -1:
+            return math.inf
+        A = chain_dense(diag[idx], lower[idx])
+        inv = np.linalg.inv(A)
+        for i in range(L):
+            worst = max(worst, rel(out["G_diag"][idx][i], blk(inv, i, i, b)))
+        for i in range(L - 1):
+            worst = max(worst, rel(out["G_lower"][idx][i], blk(inv, i + 1, i, b)))
+        sign, ld = np.linalg.slogdet(A)
+        worst = max(worst, abs(out["logdet"][idx] - ld) / max(1.0, abs(ld)), 0.0 if sign > 0 else math.inf)
+        if rhs is not None:
+            worst = max(worst, rel(out["x"][idx].ravel(), np.linalg.solve(A, rhs[idx].ravel())))
+    return worst
+
+
+def pin_tiny_chains_dense(lib=None):
+    """Brute force: tiny random chains (with leading batch dims) vs dense inverse/slogdet/solve."""
+    worst = 0.0
+    for (L, b, lead) in [(1, 1, ()), (1, 3, (2,)), (2, 1, (3,)), (2, 2, ()), (3, 3, (2, 3)),
+                         (5, 2, (2,)), (6, 4, ()), (4, 5, (2,))]:
+        E = int(np.prod(lead)) if lead else 1
+        d, l, r = inputs.chain_inputs(E, L, b, seed=100 + L * 10 + b, load=0.3, with_rhs=True)
+        d = d.reshape(lead + d.shape[1:]) if lead else d[0]
+        l = l.reshape(lead + l.shape[1:]) if lead else l[0]
+        r = r.reshape(lead + r.shape[1:]) if lead else r[0]
+        worst = max(worst, _chain_vs_dense(d, l, r, lib))
+    return worst
+
+
+def pin_quickstart(lib=None):
+    """Quickstart fact: G_diag[0] == inv(A)[0:4,0:4] (atol 1e-10) on 8 blocks of 4, load 2.0."""
+    w = inputs.WORKLOADS["chain_1x8_b4"]
+    g = inputs.generate(w)
+    out = oracle.chain(g["diag"], g["lower"], g["rhs"], lib=lib)
+    inv = np.linalg.inv(chain_dense(g["diag"][0], g["lower"][0]))
+    return float(np.abs(out["G_diag"][0, 0] - inv[0:4, 0:4]).max())
+
+
+def _frac_inverse(M):
+    """Exact inverse and determinant of a small rational matrix (Gauss-Jordan in Fractions)."""
+    n = len(M)
+    A = [[Fraction(x) for x in row] + [Fraction(int(i == j)) for j in range(n)]
+         for i, row in enumerate(M)]
+    det = Fraction(1)
+    for k in range(n):
+        p = next(i for i in range(k, n) if A[i][k] != 0)
+        if p != k:
+            A[k], A[p] = A[p], A[k]
+            det = -det
+        det *= A[k][k]
+        piv = A[k][k]
+        A[k] = [x / piv for x in A[k]]
+        for i in range(n):
+            if i != k and A[i][k] != 0:
+                f = A[i][k]
+                A[i] = [x - f * y for x, y in zip(A[i], A[k])]
+    return [row[n:] for row in A], det
+
+
+def pin_sparsax_3x3(lib=None):
+    """sparsax 'Quick start' 3x3 SPD matrix as a b=1, L=3 chain vs exact rational arithmetic."""
+    g = json.load(open(os.path.join(GOLDEN, "sparsax_quickstart_3x3.json")))
+    n = g["n"]
+    A = [[0.0] * n for _ in range(n)]
+    for i, j, v in zip(g["Ai"], g["Aj"], g["Ax"]):
+        if i <= j:                        # the page: entries with Ai <= Aj are used
+            A[i][j] = v
+            A[j][i] = v
+    inv, det = _frac_inverse(A)
+    bvec = [Fraction(x) for x in g["b"]]
+    xs = [sum(inv[i][k] * bvec[k] for k in range(n)) for i in range(n)]
+    diag = np.array([[[A[i][i]]] for i in range(n)])
+    lower = np.array([[[A[i + 1][i]]] for i in range(n - 1)])
+    out = oracle.chain(diag, lower, np.array(g["b"]).reshape(n, 1), lib=lib)
+    errs = [abs(out["G_diag"][i, 0, 0] - float(inv[i][i])) for i in range(n)]
+    errs += [abs(out["G_lower"][i, 0, 0] - float(inv[i + 1][i])) for i in range(n - 1)]
+    errs += [abs(out["x"][i, 0] - float(xs[i])) for i in range(n)]
+    errs += [abs(out["logdet"] - math.log(det))]
+    return float(max(errs))
+
+
+def _laplacian_inverse(m):
+    """(T^-1)_{ij} = min(i,j) (m+1-max(i,j)) / (m+1), 1-based, for T = tridiag(-1,2,-1)."""
+    i = np.arange(1, m + 1)
+    return np.minimum.outer(i, i) * (m + 1 - np.maximum.outer(i, i)) / (m + 1)
+
+
+def pin_laplacian_closed_form(lib=None):
+    """b=1 1-D Laplacian and its rotated block version vs the closed-form inverse and det = m+1."""
+    worst = 0.0
+    for m in [1, 2, 3, 7, 30]:
+        Tinv = _laplacian_inverse(m)
+        out = oracle.chain(np.full((m, 1, 1), 2.0), np.full((m - 1, 1, 1), -1.0), lib=lib)
+        worst = max(worst, rel(out["G_diag"][:, 0, 0], np.diag(Tinv)))
+        if m > 1:
+            worst = max(worst, rel(out["G_lower"][:, 0, 0], np.diag(Tinv, -1)))
+        worst = max(worst, abs(out["logdet"] - math.log(m + 1)))
+    # Rotated block Laplacian: D_i = 2I, B_i = -Q_i with Q_i = U_{i+1} U_i^T (U_i orthogonal).
+    # Then A = U (T kron I) U^T, so G_ii = (T^-1)_ii I, G_{i+1,i} = (T^-1)_{i+1,i} Q_i,
+    # log det A = b log(m+1) and x = U (T^-1 kron I) U^T r.
+    rng = np.random.default_rng(7)
+    for m, b in [(5, 3), (9, 4)]:
+        U = np.stack([np.linalg.qr(rng.standard_normal((b, b)))[0] for _ in range(m)])
+        Q = np.matmul(U[1:], np.swapaxes(U[:-1], 1, 2))
+        r = rng.standard_normal((m, b))
+        Tinv = _laplacian_inverse(m)
+        out = oracle.chain(np.broadcast_to(2 * np.eye(b), (m, b, b)).copy(), -Q, r, lib=lib)
+        for i in range(m):
+            worst = max(worst, rel(out["G_diag"][i], Tinv[i, i] * np.eye(b)))
+        for i in range(m - 1):
+            worst = max(worst, rel(out["G_lower"][i], Tinv[i + 1, i] * Q[i]))
+        worst = max(worst, abs(out["logdet"] - b * math.log(m + 1)))
+        Ur = np.einsum("iba,ib->ia", U, r)                # U_i^T r_i
+        x = np.einsum("iab,ib->ia", U, Tinv @ Ur)         # U_i sum_j T^-1_ij U_j^T r_j
+        worst = max(worst, rel(out["x"], x))
+    return worst
+
+
+def pin_decoupled(lib=None):
+    """B = 0: G_ii = D_i^-1, G_lower = 0, log det = sum log det D_i, x_i = D_i^-1 r_i."""
+    d, _, r = inputs.chain_inputs(2, 6, 5, seed=11, load=0.5, with_rhs=True)
+    lower = np.zeros((2, 5, 5, 5))
+    out = oracle.chain(d, lower, r, lib=lib)
+    worst = float(np.abs(out["G_lower"]).max())
+    for e in range(2):
+        for i in range(6):
+            worst = max(worst, rel(out["G_diag"][e, i], np.linalg.inv(d[e, i])))
+            worst = max(worst, rel(out["x"][e, i], np.linalg.solve(d[e, i], r[e, i])))
+        ld = sum(np.linalg.slogdet(d[e, i])[1] for i in range(6))
+        worst = max(worst, abs(out["logdet"][e] - ld) / abs(ld))
+    return worst
+
+
+def grid_closed_form(m, tau, r=None, rows=None):
+    """Spectral closed form of the m x m grid precision T kron I + I kron T + tau I.
+
+    With T = S diag(mu) S^T, s_j(i) = sqrt(2/(m+1)) sin(j pi (i+1)/(m+1)),
+    lambda_jk = tau + mu_j + mu_k:
+      G_ii      = S diag_k( sum_j s_j(i)^2        / lambda_jk ) S^T
+      G_{i+1,i} = S diag_k( sum_j s_j(i+1) s_j(i) / lambda_jk ) S^T
+      log det   = sum_jk log lambda_jk,   X = S ((S^T R S) / lambda) S^T.
+    Returns (G_diag [rows], G_lower [rows], logdet, x) for the requested block rows.
+    """
+    j = np.arange(1, m + 1)
+    i = np.arange(m)
+    S = math.sqrt(2.0 / (m + 1)) * np.sin(np.outer(i + 1, j) * math.pi / (m + 1))
+    mu = 4.0 * np.sin(j * math.pi / (2 * (m + 1))) ** 2
+    lam = tau + mu[:, None] + mu[None, :]
+    rows = range(m) if rows is None else rows
+    Gd, Gl = {}, {}
+    for row in rows:
+        wk = (S[row] ** 2) @ (1.0 / lam)
+        Gd[row] = (S * wk) @ S.T
+        if row + 1 < m:
+            wk = (S[row + 1] * S[row]) @ (1.0 / lam)
+            Gl[row] = (S * wk) @ S.T
+    x = None
+    if r is not None:
+        x = S @ ((S.T @ r @ S) / lam) @ S.T
+    return Gd, Gl, float(np.log(lam).sum()), x
+
+
+def pin_grid_closed_form(lib=None, m=12):
+    """Grid precision chain (D = tridiag(-1,4+tau,-1), B = -I) vs its spectral closed form."""
+    diag, lower, rhs, tau = inputs.grid_inputs(2, m, seed=21)
+    out = oracle.chain(diag, lower, rhs, lib=lib)
+    worst = 0.0
+    for e in range(2):
+        Gd, Gl, ld, x = grid_closed_form(m, tau[e], rhs[e])
+        for i in range(m):
+            worst = max(worst, rel(out["G_diag"][e, i], Gd[i]))
+        for i in range(m - 1):
+            worst = max(worst, rel(out["G_lower"][e, i], Gl[i]))
+        worst = max(worst, abs(out["logdet"][e] - ld) / abs(ld), rel(out["x"][e], x))
+    return worst
+
+
+def block_row_residual(diag, lower, G_diag, G_lower):
+    """max_v || A_vv G_vv + sum_u A_vu G_uv - I ||_F for a chain, from on-pattern blocks only."""
+    L, b = diag.shape[0], diag.shape[-1]
+    D = np.tril(diag) + np.swapaxes(np.tril(diag, -1), -1, -2)
+    worst = 0.0
+    for v in range(L):
+        R = D[v] @ G_diag[v] - np.eye(b)
+        if v > 0:    # A_{v,v-1} = B_{v-1}, G_{v-1,v} = G_lower[v-1]^T
+            R += lower[v - 1] @ G_lower[v - 1].T
+        if v + 1 < L:  # A_{v,v+1} = B_v^T, G_{v+1,v} = G_lower[v]
+            R += lower[v].T @ G_lower[v]
+        worst = max(worst, np.linalg.norm(R))
+    return worst
+
+
+def pin_block_row_identity(lib=None):
+    """A G = I restricted to block rows (on-pattern blocks suffice) at b=16, L=64, plus solve residual."""
+    d, l, r = inputs.chain_inputs(2, 64, 16, seed=31, load=2.0, with_rhs=True)
+    out = oracle.chain(d, l, r, lib=lib)
+    worst = 0.0
+    for e in range(2):
+        worst = max(worst, block_row_residual(d[e], l[e], out["G_diag"][e], out["G_lower"][e]))
+        A = chain_dense(d[e], l[e])
+        worst = max(worst, np.linalg.norm(A @ out["x"][e].ravel() - r[e].ravel()) / np.linalg.norm(r[e]))
+        # G_ii symmetric positive definite (Cholesky succeeds)
+        for i in range(64):
+            np.linalg.cholesky(out["G_diag"][e, i])
+    return worst
+
+
+def _tree_vs_dense(parent, diag, edge, lib):
+    out = oracle.tree(parent, diag, edge, lib=lib)
+    worst = 0.0
+    E, n, b = diag.shape[0], diag.shape[1], diag.shape[-1]
+    for e in range(E):
+        if out["info"][e] != -1:
+            return math.inf
+        A = tree_dense(parent[e], diag[e], edge[e])
+        inv = np.linalg.inv(A)
+        for v in range(n):
+            worst = max(worst, rel(out["G_diag"][e, v], blk(inv, v, v, b)))
+            p = parent[e, v]
+            if p >= 0:
+                worst = max(worst, rel(out["G_edge"][e, v], blk(inv, p, v, b)))
+            else:
+                worst = max(worst, float(np.abs(out["G_edge"][e, v]).max()))
+        ld = np.linalg.slogdet(A)[1]
+        worst = max(worst, abs(out["logdet"][e] - ld) / max(1.0, abs(ld)))
+    return worst
+
+
+def pin_tiny_trees_dense(lib=None):
+    """Brute force: random / path / star / balanced / re-rooted trees vs the dense inverse."""
+    worst = 0.0
+    for n, b in [(1, 2), (2, 1), (5, 2), (12, 3), (17, 2)]:
+        rng = np.random.default_rng(n * 100 + b)
+        parents = [inputs.random_parent(rng, n), path_parent(n), star_parent(n),
+                   balanced_parent(n, 2), balanced_parent(n, 3)]
+        # a tree rooted at its last node, with parents drawn among later indices
+        pr = np.full(n, -1, dtype=np.int32)
+        for v in range(n - 1):
+            pr[v] = rng.integers(v + 1, n)
+        parents.append(pr)
+        P = np.stack(parents)
+        diag, edge = inputs.tree_inputs_from_parent(P, b, seed=n + b, load=0.3)
+        worst = max(worst, _tree_vs_dense(P, diag, edge, lib))
+    return worst
+
+
+def pin_tree_quickstart(lib=None):
+    """Tree quickstart shape (12 nodes, b=3, random kind): G_diag[0] == inv[0:3,0:3] to 1e-10."""
+    P, diag, edge = inputs.tree_inputs(1, 12, 3, seed=0, load=2.0)
+    out = oracle.tree(P, diag, edge, lib=lib)
+    inv = np.linalg.inv(tree_dense(P[0], diag[0], edge[0]))
+    return float(np.abs(out["G_diag"][0, 0] - inv[0:3, 0:3]).max())
+
+
+def pin_root_invariance(lib=None):
+    """Path tree rooted at node 0 (eliminated in the reverse order) == chain rooted at its last node."""
+    L, b = 40, 6
+    d, l, _ = inputs.chain_inputs(1, L, b, seed=41, load=0.5, with_rhs=False)
+    ch = oracle.chain(d, l, lib=lib)
+    parent = path_parent(L)[None]
+    edge = np.zeros((1, L, b, b))
+    edge[0, 1:] = np.swapaxes(l[0], 1, 2)       # edge[v] = A_{v-1,v} = lower[v-1]^T
+    tr = oracle.tree(parent, d, edge, lib=lib)
+    worst = max(rel(tr["G_diag"][0, i], ch["G_diag"][0, i]) for i in range(L))
+    worst = max(worst, max(rel(tr["G_edge"][0, v].T, ch["G_lower"][0, v - 1]) for v in range(1, L)))
+    worst = max(worst, abs(tr["logdet"][0] - ch["logdet"][0]) / abs(ch["logdet"][0]))
+    return worst
+
+
+def pin_not_spd(lib=None):
+    """A non-positive-definite Schur complement is reported at the first failing block."""
+    d, l, _ = inputs.chain_inputs(3, 7, 3, seed=51, load=1.0, with_rhs=False)
+    d[1, 4] = -np.eye(3)
+    d[2, 0, 1, 1] = np.nan
+    out = oracle.chain(d, l, lib=lib)
+    ok = list(out["info"]) == [-1, 4, 0]
+    P, td, te = inputs.tree_inputs(2, 9, 2, seed=52, load=1.0)
+    td[1, 5] = -np.eye(2)
+    tout = oracle.tree(P, td, te, lib=lib)
+    ok = ok and tout["info"][0] == -1 and tout["info"][1] >= 0
+    bad = P.copy()
+    bad[0, 3] = -1                               # two roots
+    bad[1, 2] = 2                                # self loop
+    ok = ok and list(oracle.tree(bad, td, te, lib=lib)["info"]) == [-2, -2]
+    return 0.0 if ok else 1.0
+
+
+# name -> (function, tolerance)
+PINS = {
+    "tiny_chains_dense": (pin_tiny_chains_dense, 1e-12),
+    "quickstart": (pin_quickstart, 1e-10),
+    "sparsax_3x3": (pin_sparsax_3x3, 1e-14),
+    "laplacian_closed_form": (pin_laplacian_closed_form, 1e-12),
+    "decoupled": (pin_decoupled, 1e-12),
+    "grid_closed_form": (pin_grid_closed_form, 1e-12),
+    "block_row_identity": (pin_block_row_identity, 1e-12),
+    "tiny_trees_dense": (pin_tiny_trees_dense, 1e-12),
+    "tree_quickstart": (pin_tree_quickstart, 1e-10),
+    "root_invariance": (pin_root_invariance, 1e-11),
+    "not_spd": (pin_not_spd, 0.5),
+}

@@ -1,0 +1,66 @@
+"""Planted slips in copies of the oracle's C source must break at least one pin.
+
+This checks the pins themselves: a dropped term, a wrong sign or index, or a
+transposed operand anywhere in the oracle is caught.  Mutants are compiled
+from the source text into a temporary directory; the oracle in the tree is
+untouched.
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests.pins import PINS
+
+SRC = open(os.path.join(os.path.dirname(oracle.__file__), "selinv_oracle.c")).read()
+
+MUTANTS = {
+    "schur_sign": ("for (size_t k = 0; k < bb; ++k) S[k] -= T2[k];",
+                   "for (size_t k = 0; k < bb; ++k) S[k] += T2[k];"),
+    "schur_transposed_B": ("matmul(b, T1, 0, Bi, 1, T2);", "matmul(b, T1, 0, Bi, 0, T2);"),
+    "g_lower_sign": ("Gl[k] = -T2[k];", "Gl[k] = T2[k];"),
+    "g_lower_transposed_B": ("matmul(b, Gn, 0, Bi, 0, T1);", "matmul(b, Gn, 0, Bi, 1, T1);"),
+    "g_diag_transposed_B": ("matmul(b, Sinv + bb * i, 0, Bi, 1, T1);",
+                            "matmul(b, Sinv + bb * i, 0, Bi, 0, T1);"),
+    "g_diag_sign": ("Gii[k] = Sinv[bb * i + k] - T2[k];", "Gii[k] = Sinv[bb * i + k] + T2[k];"),
+    "logdet_half": ("ld += 2.0 * log(R[k * b + k]);", "ld += log(R[k * b + k]);"),
+    "cholesky_index": ("s -= R[i * b + k] * R[j * b + k];", "s -= R[i * b + k] * R[k * b + j];"),
+    "tri_inverse_pivot": ("Rinv[i * b + j] = -s / R[i * b + i];", "Rinv[i * b + j] = -s / R[j * b + j];"),
+    "sinv_order": ("matmul(b, Rinv, 1, Rinv, 0, Sinv);", "matmul(b, Rinv, 0, Rinv, 1, Sinv);"),
+    "solve_forward_transposed": ("matvec(b, lower + bb * i, 0, v1, v2);",
+                                 "matvec(b, lower + bb * i, 1, v1, v2);"),
+    "solve_backward_transposed": ("matvec(b, lower + bb * i, 1, x + b * (i + 1), v1);",
+                                  "matvec(b, lower + bb * i, 0, x + b * (i + 1), v1);"),
+    "solve_rhs_index": ("y[b * (i + 1) + k] = rhs[b * (i + 1) + k] - v2[k];",
+                        "y[b * (i + 1) + k] = rhs[b * i + k] - v2[k];"),
+    "tree_child_transposed": ("matmul(b, T1, 0, edge + bb * c, 1, T2);",
+                              "matmul(b, T1, 0, edge + bb * c, 0, T2);"),
+    "tree_child_skipped": ("for (int64_t k = count[v]; k < count[v + 1]; ++k) {",
+                           "for (int64_t k = count[v] + 1; k < count[v + 1]; ++k) {"),
+    "tree_edge_transposed": ("matmul(b, G_diag + bb * p, 0, edge + bb * v, 0, T1);",
+                             "matmul(b, G_diag + bb * p, 0, edge + bb * v, 1, T1);"),
+    "tree_g_diag_transposed": ("matmul(b, Sinv + bb * v, 0, edge + bb * v, 1, T1);",
+                               "matmul(b, Sinv + bb * v, 0, edge + bb * v, 0, T1);"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    assert SRC.count(old) == 1, f"mutation site for {name} is not unique"
+    src = tmp_path / "mutant.c"
+    src.write_text(SRC.replace(old, new))
+    so = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c99", "-fopenmp", "-fPIC", "-shared",
+                           "-o", str(so), str(src), "-lm"])
+    lib = oracle._bind(str(so))
+    failed = []
+    for pin, (fn, tol) in PINS.items():
+        try:
+            err = fn(lib=lib)
+        except Exception:                      # a crash in the pin also counts as caught
+            err = float("inf")
+        if not err <= tol:
+            failed.append(pin)
+    assert failed, f"mutant {name} passed every pin"
