@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Throughput of the batched block selected inverse (libselinv) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one call of the library's public entry point over one batch of
+synthetic input (selected inverse + log det + the solve where the workload
+asks for it), all of it on the device.  Default workload: 4096 independent
+chains of 64 blocks of 16 (float64, diag load 2.0, one right-hand side).
+The metric is b x b blocks per second (value = all ranks' blocks / time).
+
+Under torchrun each rank owns its own slice of chains (batch elements are
+independent, so there is no data-path collective: weak scaling); a barrier and
+a max-over-ranks of the device-timed region are the only cross-rank steps.
+Inputs (> 2 GB) are larger than L2, so no flush is needed between steps.
+
+``--impl reference`` times the CPU oracle (the plain C implementation the
+tests check against) on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_spd_selected_b200 import inputs  # noqa: E402
+
+PROFILES = os.path.join(ROOT, "profiles")
+KERNEL_SOURCES = {
+    "chain_small_kernel": ["chain_small.cu", "warp16.cuh", "common.cuh"],
+    "chain_large_kernel": ["chain_large.cu", "common.cuh"],
+    "tree_collect_kernel": ["tree.cu", "warp16.cuh", "common.cuh"],
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="chain_4096x64_b16", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--dtype", default="f64", choices=["f64", "f32"])
+    ap.add_argument("--batch", type=int, default=None, help="override the per-GPU batch (profiling runs)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+
+def source_hash(kernel: str) -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES.get(kernel, []):
+        with open(os.path.join(ROOT, "sparse_spd_selected_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged since."""
+    path = os.path.join(PROFILES, f"{kernel}__{workload}.md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    s = re.search(r"source_sha256_16:\s*([0-9a-f]+)", txt)
+    if not m or not s or s.group(1) != source_hash(kernel):
+        return None
+    return float(m.group(1))
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.dev = device_index
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (getattr(self, "out", "") or "").strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_baseline(w, dtype_name, budget_s=10.0):
+    """The oracle, as it stands, on a bounded sample of the same workload (host cores)."""
+    import oracle
+    oracle.build()
+    n_probe = 32 if w.kind != "grid" else 1
+    elems = list(range(min(n_probe, w.batch)))
+    g = inputs.generate(w, elements=elems)
+
+    def run(gg):
+        if w.kind == "tree":
+            oracle.tree(gg["parent"], gg["diag"], gg["edge"])
+        else:
+            oracle.chain(gg["diag"], gg["lower"], gg.get("rhs"))
+
+    t0 = time.perf_counter()
+    run(g)
+    dt = time.perf_counter() - t0
+    n = int(min(w.batch, max(len(elems), len(elems) * budget_s / max(dt, 1e-6))))
+    if n > len(elems):
+        elems = list(range(n))
+        g = inputs.generate(w, elements=elems)
+        t0 = time.perf_counter()
+        run(g)
+        dt = time.perf_counter() - t0
+    blocks = len(elems) * w.L
+    unit_name = "trees" if w.kind == "tree" else "chains"
+    return {"value": blocks / dt, "unit": "blocks/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{len(elems)} of {w.batch} {unit_name} ({w.name}, float64), {dt:.2f} s"}
+
+
+def algorithmic_bytes(w, es, batch):
+    """Bytes the method must move: read D and B (or edge) blocks, write G_diag and G_lower
+    (or G_edge) blocks, plus the right-hand side and solution when solving."""
+    b2 = w.b * w.b
+    if w.kind == "tree":
+        n = batch * w.L
+        return es * (b2 * n + b2 * (n - batch) + b2 * n + b2 * (n - batch))
+    nodes, edges = batch * w.L, batch * (w.L - 1)
+    byt = es * (b2 * nodes + b2 * edges + b2 * nodes + b2 * edges)
+    if w.solve:
+        byt += es * 2 * w.b * nodes
+    return byt
+
+
+def algorithmic_flops(w, batch):
+    """Nominal 7 b^3 flops per block: collect (Cholesky b^3/3 + trsm b^3 + syrk b^3) and
+    distribute (inverse 2b^3/3 + trmm b^3 + gemm 2b^3 + symmetric half-gemm b^3)."""
+    return 7.0 * w.b ** 3 * batch * w.L
+
+
+def fp64_peak_tflops(torch):
+    """cuBLAS DGEMM 8192^3 (FP64 tensor cores), best of 5."""
+    a = torch.randn(8192, 8192, dtype=torch.float64, device="cuda")
+    b = torch.randn_like(a)
+    for _ in range(2):
+        a @ b
+    best = 0.0
+    for _ in range(5):
+        s, e = torch.cuda.Event(True), torch.cuda.Event(True)
+        s.record()
+        a @ b
+        e.record()
+        torch.cuda.synchronize()
+        best = max(best, 2 * 8192 ** 3 / (s.elapsed_time(e) / 1e3) / 1e12)
+    del a, b
+    return best
+
+
+# ------------------------------------------------------------------ arms
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = inputs.WORKLOADS[args.workload]
+    import oracle
+    oracle.build()
+    n_per_step = {"chain": 64, "tree": 1, "grid": 1}[w.kind]
+    if w.kind == "chain" and w.L * w.b ** 3 > 64 * 16 ** 3 * 64:
+        n_per_step = 2
+    elems = list(range(min(n_per_step, w.batch)))
+    g = inputs.generate(w, elements=elems)
+    times = []
+    for it in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        if w.kind == "tree":
+            oracle.tree(g["parent"], g["diag"], g["edge"])
+        else:
+            oracle.chain(g["diag"], g["lower"], g.get("rhs"))
+        if it >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    blocks = len(elems) * w.L
+    value = blocks * len(times) / sum(times)
+    sample = f"{len(elems)} of {w.batch} {'trees' if w.kind == 'tree' else 'chains'} per step"
+    line = {
+        "impl": "reference", "metric": "selinv blocks/s (fp64)", "value": value, "unit": "blocks/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": w.batch * args.gpus, "block": w.b, "L": w.L},
+        "cpu_baseline": {"value": value, "unit": "blocks/s", "cores": oracle.threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "blocks/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from sparse_spd_selected_b200 import selinv
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    w = inputs.WORKLOADS[args.workload]
+    batch = args.batch or w.batch
+    tdt = torch.float64 if args.dtype == "f64" else torch.float32
+    es = 8 if args.dtype == "f64" else 4
+    # cpu baseline first (host only), so nothing forks after CUDA work starts
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.dtype)
+
+    elems = list(range(rank * batch, (rank + 1) * batch))
+    stream = torch.cuda.current_stream()
+    if w.kind == "grid":
+        diag, lower, rhs, _ = inputs.grid_inputs_torch(batch, w.b, w.seed, "cuda", tdt, w.solve)
+        host_in = None
+    else:
+        g = inputs.generate(w, elements=elems)   # per-element seeds: rank r owns its own slice
+        host_in = {k: torch.from_numpy(v).to(tdt).pin_memory() for k, v in g.items()
+                   if v is not None and k != "parent"}
+        dev_in = {k: v.to("cuda", non_blocking=True) for k, v in host_in.items()}
+        torch.cuda.synchronize()
+
+    if w.kind == "tree":
+        plan = selinv.TreePlan(g["parent"])
+        n_collect, n_dist = plan.levels()
+        launches_per_step = 2 + n_collect + max(n_dist - 1, 0)
+        out = {"G_diag": torch.empty_like(dev_in["diag"]), "G_edge": torch.empty_like(dev_in["diag"]),
+               "logdet": torch.empty(batch, dtype=torch.float64, device="cuda"),
+               "info": torch.empty(batch, dtype=torch.int32, device="cuda")}
+        ws = torch.empty(plan.workspace_size(tdt, w.b), dtype=torch.uint8, device="cuda")
+        kernel = "tree_collect_kernel"
+
+        def step():
+            selinv.selinv_tree(plan, dev_in["diag"], dev_in["edge"], check=False, out=out, workspace=ws)
+    else:
+        if w.kind == "grid":
+            dev_in = {"diag": diag, "lower": lower}
+            if rhs is not None:
+                dev_in["rhs"] = rhs
+        L, b = w.L, w.b
+        out = {"G_diag": torch.empty((batch, L, b, b), dtype=tdt, device="cuda"),
+               "G_lower": torch.empty((batch, L - 1, b, b), dtype=tdt, device="cuda"),
+               "logdet": torch.empty(batch, dtype=torch.float64, device="cuda"),
+               "info": torch.empty(batch, dtype=torch.int32, device="cuda")}
+        if "rhs" in dev_in:
+            out["x"] = torch.empty((batch, L, b), dtype=tdt, device="cuda")
+        ws = torch.empty(max(selinv.chain_workspace_size(tdt, batch, L, b, True, "rhs" in dev_in), 1),
+                         dtype=torch.uint8, device="cuda")
+        launches_per_step = 1
+        kernel = "chain_small_kernel" if b <= 16 else "chain_large_kernel"
+
+        def step():
+            selinv.selinv_chain(dev_in["diag"], dev_in["lower"], dev_in.get("rhs"), check=False, out=out,
+                                workspace=ws)
+
+    # correctness guard: the last warm-up step must report every element SPD
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if bool((out["info"] != -1).any()):
+        raise SystemExit("bench input reported not SPD")
+
+    K = args.steps
+    k_start = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    k_end = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dev_index = torch.cuda.current_device()
+    try:
+        dev_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[local])
+    except Exception:
+        pass
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev_index) as clk:
+        t_start.record(stream)
+        for i in range(K):
+            k_start[i].record(stream)
+            step()
+            k_end[i].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    kernel_ms = sum(a.elapsed_time(b_) for a, b_ in zip(k_start, k_end)) / K
+    if world > 1:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    nodes_per_rank = batch * w.L
+    value = world * nodes_per_rank * K / (elapsed_ms / 1e3)
+
+    # end to end through the same call, inputs from pinned host memory, outputs read back
+    e2e = None
+    if not args.no_e2e and host_in is not None:
+        host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()}
+        Ke = max(1, min(3, K))
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(Ke):
+            for k, v in host_in.items():
+                dev_in[k].copy_(v, non_blocking=True)
+            step()
+            for k, v in out.items():
+                host_out[k].copy_(v, non_blocking=True)
+        e.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = s.elapsed_time(e)
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+        d2h = sum(v.numel() * v.element_size() for v in out.values())
+        e2e = {"value": world * nodes_per_rank * Ke / (e2e_ms / 1e3), "unit": "blocks/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if w.b >= 64:
+        peak = fp64_peak_tflops(torch)
+        flops = algorithmic_flops(w, batch)
+        roof = {"bound": "tensor", "achieved": flops / (kernel_ms / 1e3) / 1e12, "peak": peak,
+                "unit": "TFLOP/s", "peak_source": "measured in this run: cuBLAS DGEMM 8192^3 (FP64 tensor cores)"}
+        roof["frac"] = roof["achieved"] / peak
+        roof["traffic"] = profiled_traffic(kernel, w.name)
+    else:
+        peak, src = hbm_peak()
+        byt = algorithmic_bytes(w, es, batch)
+        achieved = byt / (kernel_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": profiled_traffic(kernel, w.name) if batch == w.batch else None,
+                "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback 6650 GB/s",
+                "algorithmic_bytes_per_launch": byt, "kernel": kernel}
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": "selinv blocks/s (fp64)" if args.dtype == "f64" else "selinv blocks/s (fp32)",
+        "value": value, "unit": "blocks/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": args.dtype, "data": "synthetic",
+        "config": {"workload": w.name if batch == w.batch else f"{w.name} (batch {batch} per GPU)",
+                   "global_batch": batch * world, "block": w.b, "L_or_n": w.L,
+                   "solve": bool(w.solve), "parallelism": f"dp{world} (independent chains per GPU)",
+                   "l2": "inputs larger than L2 (no flush)"},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": K * launches_per_step,
+        "clocks": clk.summary(),
+        "kernel_ms": kernel_ms,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

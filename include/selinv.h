@@ -1,0 +1,160 @@
+/*
+ * libselinv -- batched block selected inverse of sparse SPD matrices whose
+ * block graph is a chain (block tridiagonal) or a tree, on NVIDIA B200
+ * (sm_100a).
+ *
+ * The problem (gabp-sparse-inv 0.3.2, PyPI page, "Implemented and tested
+ * kernels" -> Chain and Tree; "Quickstart"): for an SPD matrix A made of
+ * b x b blocks, return only the blocks of A^-1 on A's own pattern -- the
+ * diagonal blocks G_vv = (A^-1)_vv and one off-diagonal block per edge --
+ * never the dense inverse.  The same block LDL^T factorisation also gives
+ * log det A and the solve x = A^-1 r ("junction_solve", "junction_logdet";
+ * sparsax, PyPI page, "Factor once, do everything").
+ *
+ * Method: a collect sweep of Schur complements
+ *     S_0 = D_0,  S_{i+1} = D_{i+1} - B_i S_i^-1 B_i^T
+ * (tree: S_v = D_v - sum_{c child of v} E_c S_c^-1 E_c^T, leaves to root),
+ * log det A = sum_v log det S_v, then the distribute sweep (the Takahashi
+ * back-recursion)
+ *     G_{L-1,L-1} = S_{L-1}^-1,
+ *     G_{i+1,i} = -G_{i+1,i+1} B_i S_i^-1,  G_ii = S_i^-1 - S_i^-1 B_i^T G_{i+1,i}
+ * (tree: G_edge[v] = -G_{p(v)} E_v S_v^-1, G_vv = S_v^-1 - S_v^-1 E_v^T G_edge[v],
+ * root to leaves).
+ *
+ * Conventions shared by every entry point
+ *   - All block arrays are dense, contiguous, row-major b x b blocks in
+ *     DEVICE memory, in the precision named by `dtype` (float64 or float32).
+ *     Leading batch dimensions are flattened into `batch` by the caller.
+ *   - Only the lower triangle of each diagonal block D is read; the upper
+ *     triangle is taken as its mirror.  Every G_vv is written in full and
+ *     exactly symmetric.
+ *   - log-determinants are always written as float64 (natural log).
+ *   - info[e] (int32, device) is written for every batch element: -1 when
+ *     all Schur complements were positive definite, else the index of the
+ *     first block (chain) or node (tree) whose pivot was not > 0 (or NaN).
+ *     The outputs of such an element are unspecified.  Kernels never trap.
+ *   - The caller owns every buffer, including the workspace, whose size the
+ *     *_workspace_size functions give (0 means none is needed; the pointer
+ *     may then be NULL).  Workspace and outputs must not overlap inputs.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and returns without synchronising.  Argument errors are
+ *     reported synchronously, before anything is launched.
+ *   - Supported block sizes: 1 <= b <= selinv_max_block().
+ *   - Device pointers must be aligned to their element size; 16-byte
+ *     alignment of every array enables the vectorised paths.
+ */
+#ifndef SELINV_H
+#define SELINV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SELINV_OK = 0,
+    SELINV_ERR_INVALID_ARG = 1,   /* bad size, NULL or misaligned pointer, bad dtype */
+    SELINV_ERR_NOT_SPD = 2,       /* returned by bindings that read info[] back */
+    SELINV_ERR_BAD_TREE = 3,      /* parent array is not one rooted tree per slot */
+    SELINV_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    SELINV_ERR_WORKSPACE = 5,     /* workspace smaller than *_workspace_size */
+    SELINV_ERR_UNSUPPORTED = 6    /* block size beyond selinv_max_block() */
+} selinv_status;
+
+typedef enum { SELINV_F64 = 0, SELINV_F32 = 1 } selinv_dtype;
+
+/* Human-readable name of a status code (static string). */
+const char *selinv_status_string(selinv_status s);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int32_t selinv_version(void);
+
+/* Largest supported block size b. */
+int32_t selinv_max_block(void);
+
+/*
+ * Workspace bytes selinv_chain / chain_solve need for these sizes and
+ * outputs (want_g: G_diag/G_lower requested; want_x: a solve requested).
+ */
+size_t selinv_chain_workspace_size(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b,
+                                   int32_t want_g, int32_t want_x);
+
+/*
+ * Selected inverse, log-determinant and (optionally) solve of `batch`
+ * independent block-tridiagonal SPD chains of L blocks of size b.
+ * (gabp-sparse-inv, "Implemented and tested kernels" -> Chain, and the
+ * "Quickstart" call selected_inverse_chain(diag, lower).)
+ *
+ *   diag    [batch, L, b, b]    D_i = A_{i,i} (lower triangle read)
+ *   lower   [batch, L-1, b, b]  B_i = A_{i+1,i}; may be NULL when L == 1
+ *   G_diag  [batch, L, b, b]    out: (A^-1)_{i,i}          } both NULL, or
+ *   G_lower [batch, L-1, b, b]  out: (A^-1)_{i+1,i}        } both given
+ *   logdet  [batch] float64     out: log det A; may be NULL
+ *   rhs     [batch, L, b]       right-hand side r; NULL for no solve
+ *   x       [batch, L, b]       out: A^-1 r; given iff rhs is given
+ *   info    [batch] int32       out: see the conventions above (required)
+ * Returns SELINV_OK once the work is enqueued.
+ */
+selinv_status selinv_chain(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b,
+                           const void *diag, const void *lower,
+                           void *G_diag, void *G_lower, double *logdet,
+                           const void *rhs, void *x, int32_t *info,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Solve only: x = A^-1 r for each chain, from the same block LDL^T factor,
+ * without forming any block of A^-1 (sparsax, "Features": solve, and
+ * gabp-sparse-inv "junction_solve").  Arguments as in selinv_chain; logdet
+ * may be NULL; rhs, x and info are required.
+ */
+selinv_status chain_solve(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b,
+                          const void *diag, const void *lower, const void *rhs, void *x,
+                          double *logdet, int32_t *info,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Tree plan: validates `trees` parent arrays of n nodes each (HOST memory,
+ * parent [trees, n] int32, exactly one root per tree with parent = -1, no
+ * cycles, indices in [0, n)), builds the level-set schedule -- nodes grouped
+ * by height for the collect sweep and by depth for the distribute sweep,
+ * children in ascending index -- and copies it to the current device.
+ * (gabp-sparse-inv, "Implemented and tested kernels" -> Tree, and the
+ * level-set batched path of "General sparse selected inverse": one batched
+ * step per elimination level.)  The plan is owned by the library until
+ * selinv_tree_plan_free.  Synchronous.  Returns SELINV_ERR_BAD_TREE for a
+ * malformed parent array.
+ */
+typedef struct selinv_tree_plan_s selinv_tree_plan_t;
+
+selinv_status selinv_tree_plan(const int32_t *parent, int64_t trees, int64_t n,
+                               selinv_tree_plan_t **out);
+
+void selinv_tree_plan_free(selinv_tree_plan_t *plan);
+
+/* Levels of a plan: *collect = max height + 1, *distribute = max depth + 1. */
+selinv_status selinv_tree_plan_levels(const selinv_tree_plan_t *plan, int32_t *collect,
+                                      int32_t *distribute);
+
+size_t selinv_tree_workspace_size(const selinv_tree_plan_t *plan, selinv_dtype dtype, int32_t b);
+
+/*
+ * Selected inverse and log-determinant of block-tree SPD matrices.
+ *   diag   [trees, n, b, b]  D_v (lower triangle read)
+ *   edge   [trees, n, b, b]  edge[v] = A_{parent(v), v}; root slot ignored
+ *   G_diag [trees, n, b, b]  out: (A^-1)_{v,v}
+ *   G_edge [trees, n, b, b]  out: (A^-1)_{parent(v), v}; root slot written 0
+ *   logdet [trees] float64   out; may be NULL
+ *   info   [trees] int32     out: -1, or a node whose pivot failed
+ */
+selinv_status selinv_tree(const selinv_tree_plan_t *plan, selinv_dtype dtype, int32_t b,
+                          const void *diag, const void *edge,
+                          void *G_diag, void *G_edge, double *logdet, int32_t *info,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SELINV_H */

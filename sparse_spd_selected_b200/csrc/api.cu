@@ -1,0 +1,135 @@
+// C ABI of libselinv: argument validation, workspace sizing and kernel
+// dispatch.  Declarations and the full contract are in include/selinv.h.
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace selinv;
+
+namespace {
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t elem_size(selinv_dtype d) { return d == SELINV_F64 ? 8 : 4; }
+
+bool valid_dtype(selinv_dtype d) { return d == SELINV_F64 || d == SELINV_F32; }
+
+constexpr int32_t MAX_BLOCK = 128;
+constexpr size_t WS_ALIGN = 256;
+
+size_t round_up(size_t x) { return (x + WS_ALIGN - 1) / WS_ALIGN * WS_ALIGN; }
+
+selinv_status chain_check(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b, const void *diag,
+                          const void *lower, int32_t *info)
+{
+    if (!valid_dtype(dtype) || batch < 0 || L < 1 || b < 1) return SELINV_ERR_INVALID_ARG;
+    if (b > MAX_BLOCK) return SELINV_ERR_UNSUPPORTED;
+    if (batch > 0 && (!diag || !info || (L > 1 && !lower))) return SELINV_ERR_INVALID_ARG;
+    const size_t es = elem_size(dtype);
+    if (!aligned(diag, es) || !aligned(lower, es) || !aligned(info, 4)) return SELINV_ERR_INVALID_ARG;
+    return SELINV_OK;
+}
+
+selinv_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SELINV_OK : SELINV_ERR_CUDA; }
+
+template <class T>
+selinv_status run_chain(int64_t batch, int64_t L, int32_t b, const void *diag, const void *lower,
+                        void *G_diag, void *G_lower, double *logdet, const void *rhs, void *x,
+                        int32_t *info, void *ws, cudaStream_t s)
+{
+    ChainArgs<T> a;
+    a.diag = static_cast<const T *>(diag);
+    a.lower = static_cast<const T *>(lower);
+    a.G_diag = static_cast<T *>(G_diag);
+    a.G_lower = static_cast<T *>(G_lower);
+    a.logdet = logdet;
+    a.rhs = static_cast<const T *>(rhs);
+    a.x = static_cast<T *>(x);
+    a.info = info;
+    a.ws = static_cast<T *>(ws);
+    a.batch = batch;
+    a.L = L;
+    a.b = b;
+    if (b <= 16) {
+        const bool al = aligned(diag, 16) && aligned(lower, 16) && aligned(G_diag, 16) &&
+                        aligned(G_lower, 16) && aligned(ws, 16);
+        return from_cuda(chain_small_launch<T>(a, al, s));
+    }
+    return from_cuda(chain_large_launch<T>(a, s));
+}
+
+size_t chain_ws(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b, bool want_g, bool want_x)
+{
+    if (!want_g && !want_x) return 0;
+    const size_t es = elem_size(dtype);
+    if (b <= 16) return round_up(chain_small_workspace(es, batch, L));
+    return round_up(chain_large_workspace(es, batch, L, b));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *selinv_status_string(selinv_status s)
+{
+    switch (s) {
+    case SELINV_OK: return "ok";
+    case SELINV_ERR_INVALID_ARG: return "invalid argument";
+    case SELINV_ERR_NOT_SPD: return "matrix not positive definite";
+    case SELINV_ERR_BAD_TREE: return "parent array is not one rooted tree per slot";
+    case SELINV_ERR_CUDA: return "CUDA error";
+    case SELINV_ERR_WORKSPACE: return "workspace too small";
+    case SELINV_ERR_UNSUPPORTED: return "block size not supported";
+    }
+    return "unknown status";
+}
+
+int32_t selinv_version(void) { return 100; }
+
+int32_t selinv_max_block(void) { return MAX_BLOCK; }
+
+size_t selinv_chain_workspace_size(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b,
+                                   int32_t want_g, int32_t want_x)
+{
+    if (!valid_dtype(dtype) || batch < 0 || L < 1 || b < 1 || b > MAX_BLOCK) return 0;
+    return chain_ws(dtype, batch, L, b, want_g != 0, want_x != 0);
+}
+
+selinv_status selinv_chain(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b, const void *diag,
+                           const void *lower, void *G_diag, void *G_lower, double *logdet,
+                           const void *rhs, void *x, int32_t *info, void *workspace,
+                           size_t workspace_bytes, void *stream)
+{
+    selinv_status st = chain_check(dtype, batch, L, b, diag, lower, info);
+    if (st != SELINV_OK) return st;
+    const size_t es = elem_size(dtype);
+    const bool want_g = G_diag != nullptr;
+    const bool want_x = rhs != nullptr;
+    if (want_g && L > 1 && G_lower == nullptr) return SELINV_ERR_INVALID_ARG;
+    if (!want_g && G_lower != nullptr) return SELINV_ERR_INVALID_ARG;
+    if ((rhs == nullptr) != (x == nullptr)) return SELINV_ERR_INVALID_ARG;
+    if (!aligned(G_diag, es) || !aligned(G_lower, es) || !aligned(rhs, es) || !aligned(x, es) ||
+        !aligned(logdet, 8) || !aligned(workspace, 16))
+        return SELINV_ERR_INVALID_ARG;
+    const size_t need = chain_ws(dtype, batch, L, b, want_g, want_x);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return SELINV_ERR_WORKSPACE;
+    if (batch == 0) return SELINV_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dtype == SELINV_F64)
+        return run_chain<double>(batch, L, b, diag, lower, G_diag, G_lower, logdet, rhs, x, info,
+                                 workspace, s);
+    return run_chain<float>(batch, L, b, diag, lower, G_diag, G_lower, logdet, rhs, x, info,
+                            workspace, s);
+}
+
+selinv_status chain_solve(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b, const void *diag,
+                          const void *lower, const void *rhs, void *x, double *logdet, int32_t *info,
+                          void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (rhs == nullptr || x == nullptr) return batch == 0 ? SELINV_OK : SELINV_ERR_INVALID_ARG;
+    return selinv_chain(dtype, batch, L, b, diag, lower, nullptr, nullptr, logdet, rhs, x, info,
+                        workspace, workspace_bytes, stream);
+}
+
+}  // extern "C"

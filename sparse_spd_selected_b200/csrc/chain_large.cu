@@ -1,0 +1,641 @@
+// Block-tridiagonal chains with 16 < b <= 128: one CTA per chain.
+//
+// gabp-sparse-inv 0.3.2 (PyPI page), "Implemented and tested kernels" ->
+// Chain.  Same recursion as the b <= 16 kernel, scaled up: blocks are padded
+// to BP in {32, 64, 128} (identity / zero pad), and a CTA of (BP/32)^2 warps
+// holds the current BP x BP block as a register tile, each warp a 32 x 32
+// quadrant laid out as 4 x 4 accumulator tiles of the m8n8k4 FP64 tensor-core
+// instruction.
+//
+// Per block i:
+//   collect     S_i^-1 by a CTA-wide symmetric Gauss-Jordan sweep in registers
+//               (one column broadcast through shared memory per pivot; the
+//               pivots give log det S_i);
+//               W_i = B_i S_i^-1 and S_{i+1} = D_{i+1} - W_i B_i^T on the
+//               tensor cores, one operand resident in shared memory and the
+//               other (B_i) streamed through 16-wide K panels (cp.async,
+//               double-buffered);
+//   distribute  G_{i+1,i} = -G_{i+1,i+1} W_i and G_ii = S_i^-1 - W_i^T G_{i+1,i}
+//               with G_{i+1,i+1} / G_{i+1,i} resident and W_i streamed from
+//               the workspace.
+// S_i^-1 and W_i are kept in the caller's workspace between the sweeps (at
+// these sizes the products dominate and storing W_i saves recomputing it).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace selinv {
+
+namespace {
+
+template <int BP> struct Geo {
+    static constexpr int RW = BP / 32;       // warps per row (and per column) of the block
+    static constexpr int NW = RW * RW;
+    static constexpr int NT = NW * 32;
+    static constexpr int NP = BP / 16;       // K panels of width 16
+};
+
+// Shared-memory image of a row-major matrix of pitch P (a multiple of 16).
+//  double: XOR swizzle of 16-byte chunks inside each 128-byte row segment,
+//          chunk ^= f(r), f(r) = ((r & 1) << 2) | ((r >> 1) & 3): conflict-free
+//          tensor-core fragment reads (8 rows x 4 columns, 4 rows x 8 columns).
+//  float:  4-float row padding.
+template <class T> struct SW;
+template <> struct SW<double> {
+    static constexpr int PAD = 0;
+    SELINV_DEVINL static int idx(int r, int c, int P)
+    {
+        const int f = ((r & 1) << 2) | ((r >> 1) & 3);
+        return r * P + (c & ~15) + ((((c >> 1) & 7) ^ f) << 1) + (c & 1);
+    }
+};
+template <> struct SW<float> {
+    static constexpr int PAD = 4;
+    SELINV_DEVINL static int idx(int r, int c, int P) { return r * (P + 4) + c; }
+};
+
+template <class T> struct V2;
+template <> struct V2<double> { using type = double2; };
+template <> struct V2<float> { using type = float2; };
+
+template <class T> struct Big {
+    T v[4][4][2];    // [mi][ni][j]: row R(mi) = 32 rw + 8 mi + g, col C(ni, j) = 32 cw + 8 ni + 2 t + j
+};
+
+template <class T, int BP> struct Ctx {
+    static constexpr int RW = Geo<BP>::RW;
+    static constexpr int NT = Geo<BP>::NT;
+    static constexpr int BIG = BP * (BP + SW<T>::PAD);           // resident matrix
+    static constexpr int PANEL = 16 * (BP + SW<T>::PAD) > BP * (16 + SW<T>::PAD)
+                                     ? 16 * (BP + SW<T>::PAD) : BP * (16 + SW<T>::PAD);
+    int tid, lane, g, t, rw, cw;
+    SELINV_DEVINL void init()
+    {
+        tid = threadIdx.x;
+        lane = tid & 31;
+        g = lane >> 2;
+        t = lane & 3;
+        const int w = tid >> 5;
+        rw = w / RW;
+        cw = w % RW;
+    }
+    SELINV_DEVINL int R(int mi) const { return 32 * rw + 8 * mi + g; }
+    SELINV_DEVINL int C(int ni, int j) const { return 32 * cw + 8 * ni + 2 * t + j; }
+};
+
+template <class T, int BP> constexpr size_t smem_elems()
+{
+    using X = Ctx<T, BP>;
+    return (size_t)X::BIG + 2 * X::PANEL + 2 * BP /*colbuf*/ + 4 * BP /*y, x*/ + 2 * X::RW * BP /*red*/;
+}
+
+template <class T> SELINV_DEVINL void zero(Big<T> &a)
+{
+#pragma unroll
+    for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni) a.v[mi][ni][0] = a.v[mi][ni][1] = T(0);
+}
+
+SELINV_DEVINL void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
+
+// ---- register tile <-> shared / global -----------------------------------------
+
+template <class T, int BP>
+SELINV_DEVINL void to_smem(T *S, const Big<T> &a, const Ctx<T, BP> &x)
+{
+    using V = typename V2<T>::type;
+#pragma unroll
+    for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni) {
+            V v;
+            v.x = a.v[mi][ni][0];
+            v.y = a.v[mi][ni][1];
+            *reinterpret_cast<V *>(S + SW<T>::idx(x.R(mi), x.C(ni, 0), BP)) = v;
+        }
+}
+
+template <class T, int BP>
+SELINV_DEVINL void from_smem(Big<T> &a, const T *S, const Ctx<T, BP> &x)
+{
+    using V = typename V2<T>::type;
+#pragma unroll
+    for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni) {
+            V v = *reinterpret_cast<const V *>(S + SW<T>::idx(x.R(mi), x.C(ni, 0), BP));
+            a.v[mi][ni][0] = v.x;
+            a.v[mi][ni][1] = v.y;
+        }
+}
+
+// lower triangle and its mirror: an exactly symmetric image, every entry written once
+template <class T, int BP>
+SELINV_DEVINL void to_smem_sym(T *S, const Big<T> &a, const Ctx<T, BP> &x)
+{
+#pragma unroll
+    for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int r = x.R(mi), c = x.C(ni, j);
+                if (c <= r) S[SW<T>::idx(r, c, BP)] = a.v[mi][ni][j];
+                if (c < r) S[SW<T>::idx(c, r, BP)] = a.v[mi][ni][j];
+            }
+}
+
+// diagonal block (row-major b x b, lower triangle read), identity pad
+template <class T, int BP>
+SELINV_DEVINL void load_sym(Big<T> &a, const T *D, int b, const Ctx<T, BP> &x)
+{
+#pragma unroll
+    for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int r = x.R(mi), c = x.C(ni, j);
+                const int rr = c <= r ? r : c, cc = c <= r ? c : r;
+                a.v[mi][ni][j] = (r < b && c < b) ? __ldg(D + (int64_t)rr * b + cc) : (r == c ? T(1) : T(0));
+            }
+}
+
+template <class T, int BP, bool FULL>
+SELINV_DEVINL void store_block(T *G, const Big<T> &a, int b, const Ctx<T, BP> &x)
+{
+    using V = typename V2<T>::type;
+#pragma unroll
+    for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni) {
+            const int r = x.R(mi), c = x.C(ni, 0);
+            if (FULL) {
+                V v;
+                v.x = a.v[mi][ni][0];
+                v.y = a.v[mi][ni][1];
+                __stcs(reinterpret_cast<V *>(G + r * BP + c), v);
+            } else {
+                if (r < b && c < b) G[(int64_t)r * b + c] = a.v[mi][ni][0];
+                if (r < b && c + 1 < b) G[(int64_t)r * b + c + 1] = a.v[mi][ni][1];
+            }
+        }
+}
+
+// workspace blocks are always BP x BP row-major
+template <class T, int BP>
+SELINV_DEVINL void store_ws(T *W, const Big<T> &a, const Ctx<T, BP> &x)
+{
+    using V = typename V2<T>::type;
+#pragma unroll
+    for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni) {
+            V v;
+            v.x = a.v[mi][ni][0];
+            v.y = a.v[mi][ni][1];
+            *reinterpret_cast<V *>(W + x.R(mi) * BP + x.C(ni, 0)) = v;
+        }
+}
+
+template <class T, int BP>
+SELINV_DEVINL void load_ws(Big<T> &a, const T *W, const Ctx<T, BP> &x)
+{
+    using V = typename V2<T>::type;
+#pragma unroll
+    for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni) {
+            V v = *reinterpret_cast<const V *>(W + x.R(mi) * BP + x.C(ni, 0));
+            a.v[mi][ni][0] = v.x;
+            a.v[mi][ni][1] = v.y;
+        }
+}
+
+// ---- K panels -------------------------------------------------------------------
+
+// Column panel: rows 0..BP-1, columns k0..k0+15 of a row-major b x b input block.
+template <class T, int BP, bool FULL>
+SELINV_DEVINL void load_colpanel(T *P, const T *M, int b, int k0, const Ctx<T, BP> &x)
+{
+    constexpr int CH = 16 / sizeof(T);
+    if (FULL) {
+        for (int j = x.tid; j < BP * (16 / CH); j += Ctx<T, BP>::NT) {
+            const int r = j / (16 / CH), c = (j % (16 / CH)) * CH;
+            cp_async16(P + SW<T>::idx(r, c, 16), M + r * BP + k0 + c);
+        }
+    } else {
+        for (int j = x.tid; j < BP * 16; j += Ctx<T, BP>::NT) {
+            const int r = j >> 4, c = j & 15;
+            P[SW<T>::idx(r, c, 16)] = (r < b && k0 + c < b) ? __ldg(M + (int64_t)r * b + k0 + c) : T(0);
+        }
+    }
+}
+
+// Row panel: rows k0..k0+15 of a BP x BP workspace block.
+template <class T, int BP>
+SELINV_DEVINL void load_rowpanel(T *P, const T *M, int k0, const Ctx<T, BP> &x)
+{
+    constexpr int CH = 16 / sizeof(T);
+    for (int j = x.tid; j < 16 * (BP / CH); j += Ctx<T, BP>::NT) {
+        const int r = j / (BP / CH), c = (j % (BP / CH)) * CH;
+        cp_async16(P + SW<T>::idx(r, c, BP), M + (k0 + r) * BP + c);
+    }
+}
+
+enum { OP_BIG = 0, OP_COLPANEL = 1, OP_ROWPANEL = 2 };
+
+// acc += (NEG ? -1 : 1) * A B over k = 0..BP-1.  One operand is the resident
+// matrix `big` (row-major, A[m][k] or B[k][n]); the other is streamed in
+// panels from global memory:
+//   A = OP_COLPANEL: A[m][k] = M[m][k] (column panels of M)
+//   A = OP_ROWPANEL: A[m][k] = M[k][m] (row panels of M, i.e. M^T)
+//   B = OP_COLPANEL: B[k][n] = M[n][k] (column panels of M, i.e. M^T)
+//   B = OP_ROWPANEL: B[k][n] = M[k][n] (row panels of M)
+template <class T, int BP, int AOP, int BOP, bool NEG, bool FULL>
+SELINV_DEVINL void gemm(Big<T> &acc, const T *big, T *pbuf, const T *M, int b, const Ctx<T, BP> &x)
+{
+    constexpr int NP = Geo<BP>::NP;
+    constexpr int PANEL = Ctx<T, BP>::PANEL;
+    constexpr int STREAM = AOP != OP_BIG ? AOP : BOP;
+    auto issue = [&](int p) {
+        T *dst = pbuf + (p & 1) * PANEL;
+        if (STREAM == OP_COLPANEL) load_colpanel<T, BP, FULL>(dst, M, b, 16 * p, x);
+        else load_rowpanel<T, BP>(dst, M, 16 * p, x);
+        cp_async_commit();
+    };
+    issue(0);
+    for (int p = 0; p < NP; ++p) {
+        if (p + 1 < NP) {
+            issue(p + 1);
+            cp_async_wait_one();
+        } else {
+            cp_async_wait_all();
+        }
+        __syncthreads();
+        const T *P = pbuf + (p & 1) * PANEL;
+        const int k0 = 16 * p;
+        if constexpr (sizeof(T) == 8) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                double a[4], bf[4];
+                const int kl = 4 * kk + x.t;        // k within the panel for this lane's fragment
+#pragma unroll
+                for (int mi = 0; mi < 4; ++mi) {
+                    const int m = 32 * x.rw + 8 * mi + x.g;
+                    double v;
+                    if (AOP == OP_BIG) v = big[SW<T>::idx(m, k0 + kl, BP)];
+                    else if (AOP == OP_COLPANEL) v = P[SW<T>::idx(m, kl, 16)];
+                    else v = P[SW<T>::idx(kl, m, BP)];
+                    a[mi] = NEG ? -v : v;
+                }
+#pragma unroll
+                for (int ni = 0; ni < 4; ++ni) {
+                    const int n = 32 * x.cw + 8 * ni + x.g;
+                    if (BOP == OP_BIG) bf[ni] = big[SW<T>::idx(k0 + kl, n, BP)];
+                    else if (BOP == OP_COLPANEL) bf[ni] = P[SW<T>::idx(n, kl, 16)];
+                    else bf[ni] = P[SW<T>::idx(kl, n, BP)];
+                }
+#pragma unroll
+                for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+                    for (int ni = 0; ni < 4; ++ni)
+                        dmma_8x8x4(acc.v[mi][ni][0], acc.v[mi][ni][1], a[mi], bf[ni]);
+            }
+        } else {
+#pragma unroll 4
+            for (int kl = 0; kl < 16; ++kl) {
+                float a[4], bf[4][2];
+#pragma unroll
+                for (int mi = 0; mi < 4; ++mi) {
+                    const int m = x.R(mi);
+                    float v;
+                    if (AOP == OP_BIG) v = big[SW<T>::idx(m, k0 + kl, BP)];
+                    else if (AOP == OP_COLPANEL) v = P[SW<T>::idx(m, kl, 16)];
+                    else v = P[SW<T>::idx(kl, m, BP)];
+                    a[mi] = NEG ? -v : v;
+                }
+#pragma unroll
+                for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int n = x.C(ni, j);
+                        if (BOP == OP_BIG) bf[ni][j] = big[SW<T>::idx(k0 + kl, n, BP)];
+                        else if (BOP == OP_COLPANEL) bf[ni][j] = P[SW<T>::idx(n, kl, 16)];
+                        else bf[ni][j] = P[SW<T>::idx(kl, n, BP)];
+                    }
+#pragma unroll
+                for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+                    for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) acc.v[mi][ni][j] = fmaf(a[mi], bf[ni][j], acc.v[mi][ni][j]);
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// CTA-wide in-register inverse of a symmetric positive definite block by the
+// symmetric Gauss-Jordan sweep: for each pivot k (d = A_kk),
+// A_ij -= A_ik A_kj / d, A_ik /= d, A_kj /= d, A_kk = -1/d; the result is
+// -A^-1 and is negated.  Column k is broadcast through shared memory (row k
+// equals it by symmetry).  The product of the pivots is det A.
+template <class T, int BP>
+SELINV_DEVINL void spd_inverse(Big<T> &a, T *colbuf, const Ctx<T, BP> &x, LogAcc &det, bool &bad)
+{
+    constexpr int RW = Geo<BP>::RW;
+    for (int kb = 0; kb < RW; ++kb) {
+#pragma unroll
+        for (int kc = 0; kc < 32; ++kc) {
+            const int k = 32 * kb + kc;
+            const int nik = kc >> 3, tk = (kc & 7) >> 1, jk = kc & 1;
+            T *cb = colbuf + (kc & 1) * BP;
+            const bool owner = (x.cw == kb) && (x.t == tk);
+            if (owner) {
+#pragma unroll
+                for (int mi = 0; mi < 4; ++mi) cb[x.R(mi)] = a.v[mi][nik][jk];
+            }
+            __syncthreads();
+            const T d = cb[k];
+            bad |= !(d > T(0));
+            if (x.tid == 0) det.mul((double)d);
+            const T p = T(1) / d;
+            T cr[4], cc[4][2];
+#pragma unroll
+            for (int mi = 0; mi < 4; ++mi) cr[mi] = cb[x.R(mi)] * p;
+#pragma unroll
+            for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) cc[ni][j] = cb[x.C(ni, j)];
+#pragma unroll
+            for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+                for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) a.v[mi][ni][j] = fma(-cr[mi], cc[ni][j], a.v[mi][ni][j]);
+#pragma unroll
+            for (int mi = 0; mi < 4; ++mi) {
+                if (x.R(mi) == k) {
+#pragma unroll
+                    for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) a.v[mi][ni][j] = (x.C(ni, j) == k) ? -p : cc[ni][j] * p;
+                } else if (owner) {
+                    a.v[mi][nik][jk] = cr[mi];
+                }
+            }
+        }
+        if (x.tid == 0) det.renorm();
+    }
+#pragma unroll
+    for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni) a.v[mi][ni][0] = -a.v[mi][ni][0], a.v[mi][ni][1] = -a.v[mi][ni][1];
+}
+
+// Row sums (over this thread's columns) of a tile times the vector v, reduced
+// over the 4 lanes of a row group: the per-warp partial for rows R(mi).
+template <class T, int BP>
+SELINV_DEVINL void row_partial(T s[4], const Big<T> &a, const T *v, const Ctx<T, BP> &x)
+{
+#pragma unroll
+    for (int mi = 0; mi < 4; ++mi) {
+        T acc = T(0);
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) acc = fma(a.v[mi][ni][j], v[x.C(ni, j)], acc);
+        acc += shfl_xor(acc, 1);
+        acc += shfl_xor(acc, 2);
+        s[mi] = acc;
+    }
+}
+
+// Column sums (over this thread's rows) of a tile weighted by v, reduced over
+// the 8 row groups of the warp: the per-warp partial of (A^T v) for cols C.
+template <class T, int BP>
+SELINV_DEVINL void col_partial(T s[4][2], const Big<T> &a, const T *v, const Ctx<T, BP> &x)
+{
+#pragma unroll
+    for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            T acc = T(0);
+#pragma unroll
+            for (int mi = 0; mi < 4; ++mi) acc = fma(a.v[mi][ni][j], v[x.R(mi)], acc);
+            acc += shfl_xor(acc, 4);
+            acc += shfl_xor(acc, 8);
+            acc += shfl_xor(acc, 16);
+            s[ni][j] = acc;
+        }
+}
+
+template <class T, int BP, bool FULL, bool WANT_G, bool WANT_X>
+__global__ void __launch_bounds__(Geo<BP>::NT) chain_large_kernel(ChainArgs<T> p)
+{
+    using X = Ctx<T, BP>;
+    constexpr int RW = X::RW;
+    constexpr int64_t BB = (int64_t)BP * BP;
+    X x;
+    x.init();
+    const int64_t e = blockIdx.x;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    T *big = reinterpret_cast<T *>(smem_raw);
+    T *pbuf = big + X::BIG;
+    T *colbuf = pbuf + 2 * X::PANEL;
+    T *ybuf = colbuf + 2 * BP;     // two buffers
+    T *xbuf = ybuf + 2 * BP;       // two buffers
+    T *red1 = xbuf + 2 * BP;       // [RW][BP]
+    T *red2 = red1 + RW * BP;      // [RW][BP]
+
+    const int b = p.b;
+    const int64_t L = p.L;
+    const int64_t bb = (int64_t)b * b;
+    const T *D = p.diag + e * L * bb;
+    const T *Bl = p.lower + e * (L - 1) * bb;
+    T *ws = p.ws + e * (L - 1) * 2 * BB;
+    const T *Rv = WANT_X ? p.rhs + e * L * b : nullptr;
+    T *Xv = WANT_X ? p.x + e * L * b : nullptr;
+    constexpr bool KEEP = WANT_G || WANT_X;
+
+    LogAcc det;
+    det.init();
+    int fail = -1;
+
+    if (WANT_X && x.tid < BP) {
+        const T r0 = x.tid < b ? Rv[x.tid] : T(0);
+        ybuf[x.tid] = r0;
+        if (x.tid < b) Xv[x.tid] = r0;            // y_0 kept in x until the distribute sweep
+    }
+    Big<T> a;
+    load_sym<T, BP>(a, D, b, x);
+    __syncthreads();
+
+    // ---------------- collect sweep ----------------
+    for (int64_t i = 0; i < L; ++i) {
+        bool bad = false;
+        spd_inverse<T, BP>(a, colbuf, x, det, bad);
+        if (bad && fail < 0) fail = (int)i;
+        if (i == L - 1) break;
+        if (KEEP) store_ws<T, BP>(ws + (2 * i) * BB, a, x);
+        __syncthreads();
+        to_smem<T, BP>(big, a, x);
+        __syncthreads();
+        zero(a);
+        gemm<T, BP, OP_COLPANEL, OP_BIG, false, FULL>(a, big, pbuf, Bl + i * bb, b, x);   // W_i = B_i S_i^-1
+        if (KEEP) store_ws<T, BP>(ws + (2 * i + 1) * BB, a, x);
+        if (WANT_X) {                              // y_{i+1} = r_{i+1} - W_i y_i
+            T s[4];
+            row_partial<T, BP>(s, a, ybuf + BP * (i & 1), x);
+            if (x.t == 0) {
+#pragma unroll
+                for (int mi = 0; mi < 4; ++mi) red1[x.cw * BP + x.R(mi)] = s[mi];
+            }
+        }
+        to_smem<T, BP>(big, a, x);                 // big: S_i^-1 no longer read after the gemm
+        __syncthreads();
+        if (WANT_X && x.tid < BP) {
+            T s = T(0);
+            for (int c = 0; c < RW; ++c) s += red1[c * BP + x.tid];
+            const T r = x.tid < b ? Rv[(i + 1) * b + x.tid] : T(0);
+            const T yv = r - s;
+            ybuf[BP * ((i + 1) & 1) + x.tid] = yv;
+            if (x.tid < b) Xv[(i + 1) * b + x.tid] = yv;
+        }
+        load_sym<T, BP>(a, D + (i + 1) * bb, b, x);
+        gemm<T, BP, OP_BIG, OP_COLPANEL, true, FULL>(a, big, pbuf, Bl + i * bb, b, x);     // S_{i+1} = D_{i+1} - W_i B_i^T
+    }
+    if (x.tid == 0) {
+        if (p.logdet) p.logdet[e] = det.log_value();
+        p.info[e] = fail;
+    }
+    if (!KEEP) return;
+
+    // ---------------- distribute sweep ----------------
+    __syncthreads();
+    to_smem_sym<T, BP>(big, a, x);                 // G_{L-1,L-1} = S_{L-1}^-1, exactly symmetric
+    __syncthreads();
+    from_smem<T, BP>(a, big, x);
+    const int64_t last = L - 1;
+    if (WANT_G) store_block<T, BP, FULL>(p.G_diag + e * L * bb + last * bb, a, b, x);
+    if (WANT_X) {                                  // x_{L-1} = S_{L-1}^-1 y_{L-1}
+        T s[4];
+        row_partial<T, BP>(s, a, ybuf + BP * (last & 1), x);
+        if (x.t == 0) {
+#pragma unroll
+            for (int mi = 0; mi < 4; ++mi) red1[x.cw * BP + x.R(mi)] = s[mi];
+        }
+        __syncthreads();
+        if (x.tid < BP) {
+            T v = T(0);
+            for (int c = 0; c < RW; ++c) v += red1[c * BP + x.tid];
+            xbuf[BP * (last & 1) + x.tid] = v;
+            if (x.tid < b) Xv[last * b + x.tid] = v;
+        }
+        __syncthreads();
+    }
+
+    for (int64_t i = L - 2; i >= 0; --i) {
+        const T *Sinv = ws + (2 * i) * BB;
+        const T *W = ws + (2 * i + 1) * BB;
+        if (WANT_G) {
+            zero(a);
+            gemm<T, BP, OP_BIG, OP_ROWPANEL, true, FULL>(a, big, pbuf, W, b, x);          // G_{i+1,i} = -G_{i+1,i+1} W_i
+            store_block<T, BP, FULL>(p.G_lower + e * (L - 1) * bb + i * bb, a, b, x);
+            to_smem<T, BP>(big, a, x);             // all reads of G_{i+1,i+1} ended at the gemm's last barrier
+            __syncthreads();
+        }
+        load_ws<T, BP>(a, Sinv, x);
+        if (WANT_X) {                              // x_i = S_i^-1 y_i - W_i^T x_{i+1}; first half
+            if (x.tid < BP) ybuf[x.tid] = x.tid < b ? Xv[i * b + x.tid] : T(0);
+            __syncthreads();
+            T s[4];
+            row_partial<T, BP>(s, a, ybuf, x);
+            if (x.t == 0) {
+#pragma unroll
+                for (int mi = 0; mi < 4; ++mi) red1[x.cw * BP + x.R(mi)] = s[mi];
+            }
+        }
+        if (WANT_G) {
+            gemm<T, BP, OP_ROWPANEL, OP_BIG, true, FULL>(a, big, pbuf, W, b, x);          // G_ii = S_i^-1 - W_i^T G_{i+1,i}
+            to_smem_sym<T, BP>(big, a, x);
+            __syncthreads();
+            from_smem<T, BP>(a, big, x);
+            store_block<T, BP, FULL>(p.G_diag + e * L * bb + i * bb, a, b, x);
+        }
+        if (WANT_X) {                              // second half: W_i^T x_{i+1}
+            load_ws<T, BP>(a, W, x);
+            T s[4][2];
+            col_partial<T, BP>(s, a, xbuf + BP * ((i + 1) & 1), x);
+            if (x.g == 0) {
+#pragma unroll
+                for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) red2[x.rw * BP + x.C(ni, j)] = s[ni][j];
+            }
+            __syncthreads();
+            if (x.tid < BP) {
+                T v = T(0);
+                for (int c = 0; c < RW; ++c) v += red1[c * BP + x.tid] - red2[c * BP + x.tid];
+                xbuf[BP * (i & 1) + x.tid] = v;
+                if (x.tid < b) Xv[i * b + x.tid] = v;
+            }
+            __syncthreads();
+        }
+    }
+}
+
+template <class T, int BP, bool FULL, bool G, bool Xs>
+cudaError_t launch_t(const ChainArgs<T> &a, cudaStream_t s)
+{
+    const size_t smem = sizeof(T) * smem_elems<T, BP>();
+    auto k = chain_large_kernel<T, BP, FULL, G, Xs>;
+    cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    k<<<(unsigned)a.batch, Geo<BP>::NT, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <class T, int BP, bool FULL>
+cudaError_t launch_flags(const ChainArgs<T> &a, cudaStream_t s)
+{
+    const bool G = a.G_diag != nullptr, Xs = a.x != nullptr;
+    if (G && Xs) return launch_t<T, BP, FULL, true, true>(a, s);
+    if (G) return launch_t<T, BP, FULL, true, false>(a, s);
+    if (Xs) return launch_t<T, BP, FULL, false, true>(a, s);
+    return launch_t<T, BP, FULL, false, false>(a, s);
+}
+
+template <class T, int BP>
+cudaError_t launch_bp(const ChainArgs<T> &a, bool full, cudaStream_t s)
+{
+    return full ? launch_flags<T, BP, true>(a, s) : launch_flags<T, BP, false>(a, s);
+}
+
+int padded(int b) { return b <= 32 ? 32 : (b <= 64 ? 64 : 128); }
+
+bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+}  // namespace
+
+size_t chain_large_workspace(size_t elem, int64_t batch, int64_t L, int b)
+{
+    const size_t bp = (size_t)padded(b);
+    return (size_t)batch * (size_t)(L > 1 ? L - 1 : 0) * 2 * bp * bp * elem;
+}
+
+template <class T> cudaError_t chain_large_launch(const ChainArgs<T> &a, cudaStream_t s)
+{
+    if (a.batch == 0) return cudaSuccess;
+    const int bp = padded(a.b);
+    const bool full = a.b == bp && al16(a.diag) && al16(a.lower) && al16(a.G_diag) && al16(a.G_lower);
+    if (bp == 32) return launch_bp<T, 32>(a, full, s);
+    if (bp == 64) return launch_bp<T, 64>(a, full, s);
+    return launch_bp<T, 128>(a, full, s);
+}
+
+template cudaError_t chain_large_launch<double>(const ChainArgs<double> &, cudaStream_t);
+template cudaError_t chain_large_launch<float>(const ChainArgs<float> &, cudaStream_t);
+
+}  // namespace selinv

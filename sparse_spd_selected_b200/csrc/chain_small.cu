@@ -1,0 +1,282 @@
+// Block-tridiagonal chains with b <= 16: one warp per chain.
+//
+// gabp-sparse-inv 0.3.2 (PyPI page), "Implemented and tested kernels" ->
+// Chain: block LDL^T of the chain, then the Takahashi back-recursion.  The
+// whole per-chain computation is one fused kernel: the collect sweep
+// (Schur complements, the log-determinant and the forward half of the
+// solve) runs i = 0..L-1 keeping S_i in registers; the distribute sweep
+// (G blocks and the backward half of the solve) runs i = L-2..0.
+//
+// Per block i the warp holds S_i as a register tile, inverts it in
+// registers (symmetric Gauss-Jordan sweep, pivots -> log det), and forms
+//   W_i = B_i S_i^-1,  S_{i+1} = D_{i+1} - W_i B_i^T          (collect)
+//   G_{i+1,i} = -G_{i+1,i+1} W_i,  G_ii = S_i^-1 - W_i^T G_{i+1,i}  (distribute)
+// (G_ii = S_i^-1 - S_i^-1 B_i^T G_{i+1,i} with S_i^-1 B_i^T = W_i^T).  The
+// products run on the FP64 tensor cores (m8n8k4) from shared memory.
+// Between the sweeps only the lower triangle of each S_i^-1 is kept, in the
+// caller's workspace; W_i is recomputed from B_i in the distribute sweep,
+// which moves fewer bytes than storing it.
+#include "kernels.h"
+#include "warp16.cuh"
+
+namespace selinv {
+
+namespace {
+
+constexpr int WARPS = 4;
+
+template <class T> __host__ __device__ constexpr int warp_smem_elems() { return 4 * w16::SL<T>::ELEMS + 64; }
+
+template <class T, bool FULL, bool WANT_G, bool WANT_X>
+__global__ void __launch_bounds__(WARPS * 32) chain_small_kernel(ChainArgs<T> p)
+{
+    using namespace w16;
+    constexpr int E = SL<T>::ELEMS;
+    const int lane = threadIdx.x & 31;
+    const int wid = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int64_t e = (int64_t)blockIdx.x * WARPS + wid;
+    if (e >= p.batch) return;
+
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    T *sbase = reinterpret_cast<T *>(smem_raw) + wid * warp_smem_elems<T>();
+    T *sS = sbase;             // S_i^-1 (operand), later G_{i+1,i}
+    T *sW = sS + E;            // W_i
+    T *sB = sW + E;            // B_i
+    T *sG = sB + E;            // G_{i+1,i+1}
+    T *sy = sG + E;            // y vectors, two buffers of 16
+    T *sx = sy + 32;           // x vectors, two buffers of 16
+
+    const int b = p.b;
+    const int64_t L = p.L;
+    const int64_t bb = (int64_t)b * b;
+    const T *D = p.diag + e * L * bb;
+    const T *Bl = p.lower + e * (L - 1) * bb;
+    T *ws = p.ws + e * (L - 1) * SLOT_ELEMS;
+    const T *R = WANT_X ? p.rhs + e * L * b : nullptr;
+    T *X = WANT_X ? p.x + e * L * b : nullptr;
+
+    LogAcc det;
+    det.init();
+    int fail = -1;
+
+    Tile<T> a, dn, w;
+    load_sym<T, FULL>(a, D, b, g, t);
+    if (L > 1) {
+        load_block_async<T, FULL>(sB, Bl, b, lane);
+        cp_async_commit();
+        load_sym<T, FULL>(dn, D + bb, b, g, t);
+    }
+    T rn[2] = {T(0), T(0)};    // r_{i+1} at rows g, g+8 (lanes with t == 0)
+    if (WANT_X) {
+        if (lane < 16) {
+            const T r0 = lane < b ? R[lane] : T(0);
+            sy[lane] = r0;
+            if (lane < b) X[lane] = r0;        // y_0 kept in x until the distribute sweep
+        }
+        if (L > 1 && t == 0) {
+            rn[0] = g < b ? R[b + g] : T(0);
+            rn[1] = g + 8 < b ? R[b + g + 8] : T(0);
+        }
+    }
+    __syncwarp();
+
+    // ---------------- collect sweep ----------------
+    for (int64_t i = 0; i < L; ++i) {
+        bool bad = false;
+        spd_inverse<T>(a, lane, g, t, det, bad);
+        det.renorm();
+        if (bad && fail < 0) fail = (int)i;
+        if (i == L - 1) break;
+
+        if (WANT_G || WANT_X) store_lower_slot<T>(ws + i * SLOT_ELEMS, a, lane, g, t);
+        to_smem<T>(sS, a, g, t);
+        cp_async_wait_all();
+        __syncwarp();
+
+        zero(w);
+        gemm<0, 0, false>(w, sB, sS, g, t);          // W_i = B_i S_i^-1
+        to_smem<T>(sW, w, g, t);
+        __syncwarp();
+
+        a = dn;
+        gemm<0, 1, true>(a, sW, sB, g, t);           // S_{i+1} = D_{i+1} - W_i B_i^T
+
+        if (WANT_X) {                                 // y_{i+1} = r_{i+1} - W_i y_i
+            T s[2];
+            row_matvec<T>(s, w, sy + 16 * (i & 1), t);
+            if (t == 0) {
+                T *ynext = sy + 16 * ((i + 1) & 1);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int r = g + 8 * h;
+                    const T yv = rn[h] - s[h];
+                    ynext[r] = yv;
+                    if (r < b) X[(i + 1) * b + r] = yv;
+                }
+            }
+        }
+        __syncwarp();
+        if (i + 1 < L - 1) {
+            load_block_async<T, FULL>(sB, Bl + (i + 1) * bb, b, lane);
+            cp_async_commit();
+        }
+        if (i + 2 < L) {
+            load_sym<T, FULL>(dn, D + (i + 2) * bb, b, g, t);
+            if (WANT_X && t == 0) {
+                rn[0] = g < b ? R[(i + 2) * b + g] : T(0);
+                rn[1] = g + 8 < b ? R[(i + 2) * b + g + 8] : T(0);
+            }
+        }
+    }
+    if (lane == 0) {
+        if (p.logdet) p.logdet[e] = det.log_value();
+        p.info[e] = fail;
+    }
+    if (!(WANT_G || WANT_X)) return;
+
+    // ---------------- distribute sweep ----------------
+    // a = S_{L-1}^-1 = G_{L-1,L-1}; make it exactly symmetric.
+    __syncwarp();
+    to_smem_sym<T>(sG, a, g, t);
+    __syncwarp();
+    from_smem<T>(a, sG, g, t);
+    if (WANT_G) store_block<T, FULL>(p.G_diag + e * L * bb + (L - 1) * bb, a, b, g, t);
+
+    const int64_t last = L - 1;
+    T yp[2] = {T(0), T(0)};     // y_i at rows g, g+8
+    if (WANT_X) {               // x_{L-1} = S_{L-1}^-1 y_{L-1}
+        const T *y = sy + 16 * (last & 1);
+        T part[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) part[q] = a.v[0][q] * y[g] + a.v[1][q] * y[g + 8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            part[q] += shfl_xor(part[q], 4);
+            part[q] += shfl_xor(part[q], 8);
+            part[q] += shfl_xor(part[q], 16);
+        }
+        if (g == 0) {
+            T *xs = sx + 16 * (last & 1);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int c = tcol(t, q);
+                xs[c] = part[q];
+                if (c < b) X[last * b + c] = part[q];
+            }
+        }
+        if (L > 1) {
+            yp[0] = g < b ? X[(last - 1) * b + g] : T(0);
+            yp[1] = g + 8 < b ? X[(last - 1) * b + g + 8] : T(0);
+        }
+    }
+    Tile<T> pre;
+    if (L > 1) {
+        load_block_async<T, FULL>(sB, Bl + (L - 2) * bb, b, lane);
+        cp_async_commit();
+        load_lower_slot<T>(pre, ws + (L - 2) * SLOT_ELEMS, lane, g, t);
+    }
+    __syncwarp();
+
+    for (int64_t i = L - 2; i >= 0; --i) {
+        to_smem_sym<T>(sS, pre, g, t);               // S_i^-1, full and symmetric
+        const T yi[2] = {yp[0], yp[1]};
+        cp_async_wait_all();
+        __syncwarp();
+
+        zero(w);
+        gemm<0, 0, false>(w, sB, sS, g, t);          // W_i = B_i S_i^-1
+        from_smem<T>(a, sS, g, t);                   // S_i^-1 in registers
+        to_smem<T>(sW, w, g, t);
+        __syncwarp();
+        if (i > 0) {
+            load_block_async<T, FULL>(sB, Bl + (i - 1) * bb, b, lane);
+            cp_async_commit();
+            load_lower_slot<T>(pre, ws + (i - 1) * SLOT_ELEMS, lane, g, t);
+            if (WANT_X) {
+                yp[0] = g < b ? X[(i - 1) * b + g] : T(0);
+                yp[1] = g + 8 < b ? X[(i - 1) * b + g + 8] : T(0);
+            }
+        }
+
+        if (WANT_G) {
+            Tile<T> gl;
+            zero(gl);
+            gemm<0, 0, true>(gl, sG, sW, g, t);      // G_{i+1,i} = -G_{i+1,i+1} W_i
+            store_block<T, FULL>(p.G_lower + e * (L - 1) * bb + i * bb, gl, b, g, t);
+            to_smem<T>(sS, gl, g, t);
+            __syncwarp();
+            Tile<T> gd = a;
+            gemm<1, 0, true>(gd, sW, sS, g, t);      // G_ii = S_i^-1 - W_i^T G_{i+1,i}
+            to_smem_sym<T>(sG, gd, g, t);
+            __syncwarp();
+            from_smem<T>(gd, sG, g, t);
+            store_block<T, FULL>(p.G_diag + e * L * bb + i * bb, gd, b, g, t);
+        }
+        if (WANT_X) {                                 // x_i = S_i^-1 y_i - W_i^T x_{i+1}
+            const T *xn = sx + 16 * ((i + 1) & 1);
+            const T x0 = xn[g], x1 = xn[g + 8];
+            T part[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                part[q] = a.v[0][q] * yi[0] + a.v[1][q] * yi[1] - w.v[0][q] * x0 - w.v[1][q] * x1;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                part[q] += shfl_xor(part[q], 4);
+                part[q] += shfl_xor(part[q], 8);
+                part[q] += shfl_xor(part[q], 16);
+            }
+            if (g == 0) {
+                T *xs = sx + 16 * (i & 1);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int c = tcol(t, q);
+                    xs[c] = part[q];
+                    if (c < b) X[i * b + c] = part[q];
+                }
+            }
+        }
+        __syncwarp();
+    }
+}
+
+template <class T, bool FULL, bool G, bool X>
+cudaError_t launch_t(const ChainArgs<T> &a, cudaStream_t s)
+{
+    const size_t smem = sizeof(T) * warp_smem_elems<T>() * WARPS;
+    auto k = chain_small_kernel<T, FULL, G, X>;
+    cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    const int64_t blocks = ceil_div(a.batch, WARPS);
+    k<<<(unsigned)blocks, WARPS * 32, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <class T, bool FULL>
+cudaError_t launch_full(const ChainArgs<T> &a, cudaStream_t s)
+{
+    const bool G = a.G_diag != nullptr, X = a.x != nullptr;
+    if (G && X) return launch_t<T, FULL, true, true>(a, s);
+    if (G) return launch_t<T, FULL, true, false>(a, s);
+    if (X) return launch_t<T, FULL, false, true>(a, s);
+    return launch_t<T, FULL, false, false>(a, s);
+}
+
+}  // namespace
+
+size_t chain_small_workspace(size_t elem, int64_t batch, int64_t L)
+{
+    return (size_t)batch * (size_t)(L > 1 ? L - 1 : 0) * w16::SLOT_ELEMS * elem;
+}
+
+template <class T> cudaError_t chain_small_launch(const ChainArgs<T> &a, bool aligned16, cudaStream_t s)
+{
+    if (a.batch == 0) return cudaSuccess;
+    if (a.b == 16 && aligned16) return launch_full<T, true>(a, s);
+    return launch_full<T, false>(a, s);
+}
+
+template cudaError_t chain_small_launch<double>(const ChainArgs<double> &, bool, cudaStream_t);
+template cudaError_t chain_small_launch<float>(const ChainArgs<float> &, bool, cudaStream_t);
+
+}  // namespace selinv

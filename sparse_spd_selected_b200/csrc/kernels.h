@@ -1,0 +1,34 @@
+// Internal interface between the C ABI (api.cu) and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace selinv {
+
+// One batched chain call: all arrays device, row-major, contiguous.
+template <class T> struct ChainArgs {
+    const T *diag;      // [batch, L, b, b]
+    const T *lower;     // [batch, L-1, b, b]
+    T *G_diag;          // [batch, L, b, b] or null
+    T *G_lower;         // [batch, L-1, b, b] or null (with G_diag)
+    double *logdet;     // [batch] or null
+    const T *rhs;       // [batch, L, b] or null
+    T *x;               // [batch, L, b] or null (with rhs)
+    int32_t *info;      // [batch]
+    T *ws;              // workspace
+    int64_t batch;
+    int64_t L;
+    int b;
+};
+
+// b <= 16: one warp per chain.
+size_t chain_small_workspace(size_t elem, int64_t batch, int64_t L);
+template <class T> cudaError_t chain_small_launch(const ChainArgs<T> &a, bool aligned16, cudaStream_t s);
+
+// 16 < b <= 128: one CTA per chain.
+size_t chain_large_workspace(size_t elem, int64_t batch, int64_t L, int b);
+template <class T> cudaError_t chain_large_launch(const ChainArgs<T> &a, cudaStream_t s);
+
+}  // namespace selinv

@@ -1,0 +1,427 @@
+// Block trees: plan (host) and level-set kernels (b <= 16, one warp per node).
+//
+// gabp-sparse-inv 0.3.2 (PyPI page), "Implemented and tested kernels" ->
+// Tree: a parent array and one edge block per non-root node,
+// edge[v] = A_{parent(v), v}; collect from the leaves to the root, then
+// distribute from the root to the leaves.  The level-set batching follows the
+// package's batched path ("General sparse selected inverse": one batched step
+// per elimination level instead of per node): every node of one height is
+// independent in the collect sweep, every node of one depth in the distribute
+// sweep, so each level is one kernel launch over all trees of the batch.
+//
+// Collect, node v (all children already done):
+//   S_v = D_v - sum_{c in ch(v)} U_c,        U_c = E_c S_c^-1 E_c^T
+//   S_v^-1 and log det S_v; if v is not a root, U_v = W_v E_v^T with
+//   W_v = E_v S_v^-1 is left in the workspace for the parent.
+// Distribute, node v with parent p (G_pp already written):
+//   G_edge[v] = -G_pp W_v,   G_vv = S_v^-1 - W_v^T G_edge[v]
+// (S_v^-1 E_v^T G_edge[v] = W_v^T G_edge[v]).  Roots get G = S^-1 in collect.
+#include <algorithm>
+#include <climits>
+#include <new>
+#include <vector>
+
+#include "kernels.h"
+#include "warp16.cuh"
+
+struct selinv_tree_plan_s {
+    int64_t trees = 0, n = 0;
+    int device = 0;
+    std::vector<int64_t> collect_off;      // [H + 1] into collect_nodes
+    std::vector<int64_t> dist_off;         // [Dm + 1] into dist_nodes (depth >= 1)
+    int32_t *d_collect_nodes = nullptr;    // global node ids by (height, id)
+    int32_t *d_dist_nodes = nullptr;       // non-root global ids by (depth, id)
+    int32_t *d_child_ptr = nullptr;        // [trees*n + 1]
+    int32_t *d_child_idx = nullptr;        // global ids, ascending per parent
+    int32_t *d_parent = nullptr;           // global parent id or -1
+};
+
+namespace selinv {
+
+namespace {
+
+constexpr int TWARPS = 4;
+
+template <class T> __host__ __device__ constexpr int tree_smem_elems() { return 4 * w16::SL<T>::ELEMS; }
+
+struct TreeDev {
+    const int32_t *child_ptr;
+    const int32_t *child_idx;
+    const int32_t *parent;
+    int64_t n;
+};
+
+template <class T> struct TreeBufs {
+    const T *diag, *edge;
+    T *G_diag, *G_edge;
+    T *ws_sinv, *ws_u;       // per node lower slots
+    double *ws_ld;           // per node log det S_v
+    int32_t *info;           // per tree, INT_MAX = ok until finalised
+    int b;
+};
+
+template <class T, bool FULL>
+__global__ void __launch_bounds__(TWARPS * 32)
+tree_collect_kernel(TreeBufs<T> p, TreeDev td, const int32_t *nodes, int64_t count)
+{
+    using namespace w16;
+    constexpr int E = SL<T>::ELEMS;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int64_t k = (int64_t)blockIdx.x * TWARPS + wid;
+    if (k >= count) return;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    T *sS = reinterpret_cast<T *>(smem_raw) + wid * tree_smem_elems<T>();
+    T *sW = sS + E, *sB = sW + E, *sT = sB + E;
+
+    const int b = p.b;
+    const int64_t bb = (int64_t)b * b;
+    const int32_t v = nodes[k];
+    const int32_t par = td.parent[v];
+    if (par >= 0) {                               // E_v -> shared memory, early
+        load_block_async<T, FULL>(sB, p.edge + v * bb, b, lane);
+        cp_async_commit();
+    }
+    Tile<T> a;
+    load_sym<T, FULL>(a, p.diag + v * bb, b, g, t);
+
+    // sum of the children's U_c (lower slots), then mirrored once
+    const int32_t c0 = td.child_ptr[v], c1 = td.child_ptr[v + 1];
+    if (c1 > c0) {
+        Tile<T> acc, u;
+        zero(acc);
+        for (int32_t c = c0; c < c1; ++c) {
+            load_lower_slot<T>(u, p.ws_u + (int64_t)td.child_idx[c] * SLOT_ELEMS, lane, g, t);
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc.v[h][q] += u.v[h][q];
+        }
+        to_smem_sym<T>(sT, acc, g, t);
+        __syncwarp();
+        from_smem<T>(acc, sT, g, t);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) a.v[h][q] -= acc.v[h][q];
+    }
+
+    LogAcc det;
+    det.init();
+    bool bad = false;
+    spd_inverse<T>(a, lane, g, t, det, bad);
+    if (lane == 0) {
+        p.ws_ld[v] = det.log_value();
+        if (bad) atomicMin(p.info + v / td.n, (int32_t)(v % td.n));
+    }
+    if (par < 0) {                                // root: G = S^-1, G_edge = 0
+        __syncwarp();
+        to_smem_sym<T>(sT, a, g, t);
+        __syncwarp();
+        from_smem<T>(a, sT, g, t);
+        store_block<T, FULL>(p.G_diag + v * bb, a, b, g, t);
+        Tile<T> z;
+        zero(z);
+        store_block<T, FULL>(p.G_edge + v * bb, z, b, g, t);
+        return;
+    }
+    store_lower_slot<T>(p.ws_sinv + (int64_t)v * SLOT_ELEMS, a, lane, g, t);
+    to_smem<T>(sS, a, g, t);
+    cp_async_wait_all();
+    __syncwarp();
+    Tile<T> w;
+    zero(w);
+    gemm<0, 0, false>(w, sB, sS, g, t);           // W_v = E_v S_v^-1
+    to_smem<T>(sW, w, g, t);
+    __syncwarp();
+    Tile<T> u;
+    zero(u);
+    gemm<0, 1, false>(u, sW, sB, g, t);           // U_v = W_v E_v^T
+    store_lower_slot<T>(p.ws_u + (int64_t)v * SLOT_ELEMS, u, lane, g, t);
+}
+
+template <class T, bool FULL>
+__global__ void __launch_bounds__(TWARPS * 32)
+tree_distribute_kernel(TreeBufs<T> p, TreeDev td, const int32_t *nodes, int64_t count)
+{
+    using namespace w16;
+    constexpr int E = SL<T>::ELEMS;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int64_t k = (int64_t)blockIdx.x * TWARPS + wid;
+    if (k >= count) return;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    T *sS = reinterpret_cast<T *>(smem_raw) + wid * tree_smem_elems<T>();
+    T *sW = sS + E, *sB = sW + E, *sG = sB + E;
+
+    const int b = p.b;
+    const int64_t bb = (int64_t)b * b;
+    const int32_t v = nodes[k];
+    const int32_t par = td.parent[v];
+    load_block_async<T, FULL>(sB, p.edge + v * bb, b, lane);
+    load_block_async<T, FULL>(sG, p.G_diag + (int64_t)par * bb, b, lane);   // G_pp (symmetric)
+    cp_async_commit();
+    Tile<T> a;
+    load_lower_slot<T>(a, p.ws_sinv + (int64_t)v * SLOT_ELEMS, lane, g, t);
+    to_smem_sym<T>(sS, a, g, t);
+    cp_async_wait_all();
+    __syncwarp();
+    Tile<T> w;
+    zero(w);
+    gemm<0, 0, false>(w, sB, sS, g, t);           // W_v = E_v S_v^-1
+    from_smem<T>(a, sS, g, t);
+    to_smem<T>(sW, w, g, t);
+    __syncwarp();
+    Tile<T> ge;
+    zero(ge);
+    gemm<0, 0, true>(ge, sG, sW, g, t);           // G_edge[v] = -G_pp W_v
+    store_block<T, FULL>(p.G_edge + v * bb, ge, b, g, t);
+    to_smem<T>(sS, ge, g, t);
+    __syncwarp();
+    gemm<1, 0, true>(a, sW, sS, g, t);            // G_vv = S_v^-1 - W_v^T G_edge[v]
+    __syncwarp();
+    to_smem_sym<T>(sB, a, g, t);
+    __syncwarp();
+    from_smem<T>(a, sB, g, t);
+    store_block<T, FULL>(p.G_diag + v * bb, a, b, g, t);
+}
+
+__global__ void tree_info_init(int32_t *info, int64_t trees)
+{
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < trees) info[i] = INT_MAX;
+}
+
+// log det per tree = sum of its nodes' log det S_v in a fixed order
+// (deterministic); info INT_MAX -> -1.
+__global__ void tree_finalize(const double *ws_ld, int64_t n, double *logdet, int32_t *info)
+{
+    __shared__ double part[256];
+    const int64_t tr = blockIdx.x;
+    double s = 0.0;
+    for (int64_t v = threadIdx.x; v < n; v += blockDim.x) s += ws_ld[tr * n + v];
+    part[threadIdx.x] = s;
+    __syncthreads();
+    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+        if ((int)threadIdx.x < w) part[threadIdx.x] += part[threadIdx.x + w];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        if (logdet) logdet[tr] = part[0];
+        if (info[tr] == INT_MAX) info[tr] = -1;
+    }
+}
+
+template <class T> size_t slot_bytes() { return sizeof(T) * w16::SLOT_ELEMS; }
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+template <class T>
+cudaError_t run_tree(const selinv_tree_plan_s *pl, int b, const T *diag, const T *edge, T *G_diag, T *G_edge,
+                     double *logdet, int32_t *info, void *ws, bool full, cudaStream_t s)
+{
+    const int64_t N = pl->trees * pl->n;
+    char *w = static_cast<char *>(ws);
+    TreeBufs<T> p;
+    p.diag = diag;
+    p.edge = edge;
+    p.G_diag = G_diag;
+    p.G_edge = G_edge;
+    p.ws_sinv = reinterpret_cast<T *>(w);
+    w += align256(N * slot_bytes<T>());
+    p.ws_u = reinterpret_cast<T *>(w);
+    w += align256(N * slot_bytes<T>());
+    p.ws_ld = reinterpret_cast<double *>(w);
+    p.info = info;
+    p.b = b;
+    TreeDev td{pl->d_child_ptr, pl->d_child_idx, pl->d_parent, pl->n};
+
+    tree_info_init<<<(unsigned)ceil_div(pl->trees, 256), 256, 0, s>>>(info, pl->trees);
+    const size_t smem = sizeof(T) * tree_smem_elems<T>() * TWARPS;
+    auto kc = full ? tree_collect_kernel<T, true> : tree_collect_kernel<T, false>;
+    auto kd = full ? tree_distribute_kernel<T, true> : tree_distribute_kernel<T, false>;
+    cudaError_t err = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err == cudaSuccess) err = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    for (size_t h = 0; h + 1 < pl->collect_off.size(); ++h) {
+        const int64_t cnt = pl->collect_off[h + 1] - pl->collect_off[h];
+        if (cnt == 0) continue;
+        kc<<<(unsigned)ceil_div(cnt, TWARPS), TWARPS * 32, smem, s>>>(p, td, pl->d_collect_nodes + pl->collect_off[h], cnt);
+    }
+    for (size_t d = 0; d + 1 < pl->dist_off.size(); ++d) {
+        const int64_t cnt = pl->dist_off[d + 1] - pl->dist_off[d];
+        if (cnt == 0) continue;
+        kd<<<(unsigned)ceil_div(cnt, TWARPS), TWARPS * 32, smem, s>>>(p, td, pl->d_dist_nodes + pl->dist_off[d], cnt);
+    }
+    tree_finalize<<<(unsigned)pl->trees, 256, 0, s>>>(p.ws_ld, pl->n, logdet, info);
+    return cudaGetLastError();
+}
+
+bool is_aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+
+size_t tree_workspace(const selinv_tree_plan_s *pl, size_t elem)
+{
+    const int64_t N = pl->trees * pl->n;
+    return 2 * align256((size_t)N * elem * w16::SLOT_ELEMS) + align256((size_t)N * sizeof(double));
+}
+
+}  // namespace selinv
+
+using namespace selinv;
+
+extern "C" {
+
+selinv_status selinv_tree_plan(const int32_t *parent, int64_t trees, int64_t n, selinv_tree_plan_t **out)
+{
+    if (!out) return SELINV_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!parent || trees < 1 || n < 1 || trees * n >= (int64_t)INT32_MAX) return SELINV_ERR_INVALID_ARG;
+    const int64_t N = trees * n;
+    std::vector<int32_t> gparent(N), cnt(N + 1, 0), height(N, 0), depth(N, 0), order;
+    order.reserve(N);
+    for (int64_t tr = 0; tr < trees; ++tr) {
+        int64_t root = -1;
+        for (int64_t v = 0; v < n; ++v) {
+            const int32_t p = parent[tr * n + v];
+            if (p == -1) {
+                if (root >= 0) return SELINV_ERR_BAD_TREE;
+                root = v;
+                gparent[tr * n + v] = -1;
+            } else {
+                if (p < 0 || p >= n || p == v) return SELINV_ERR_BAD_TREE;
+                gparent[tr * n + v] = (int32_t)(tr * n + p);
+                cnt[tr * n + p + 1]++;
+            }
+        }
+        if (root < 0) return SELINV_ERR_BAD_TREE;
+    }
+    for (int64_t v = 0; v < N; ++v) cnt[v + 1] += cnt[v];
+    std::vector<int32_t> child(std::max<int64_t>(cnt[N], 1)), fill(cnt.begin(), cnt.end() - 1);
+    for (int64_t v = 0; v < N; ++v)
+        if (gparent[v] >= 0) child[fill[gparent[v]]++] = (int32_t)v;   // ascending per parent
+    // breadth-first order per tree from its root; a cycle leaves nodes unreached
+    for (int64_t tr = 0; tr < trees; ++tr) {
+        const size_t start = order.size();
+        for (int64_t v = 0; v < n; ++v)
+            if (gparent[tr * n + v] < 0) order.push_back((int32_t)(tr * n + v));
+        for (size_t h = start; h < order.size(); ++h) {
+            const int32_t v = order[h];
+            for (int32_t c = cnt[v]; c < cnt[v + 1]; ++c) {
+                depth[child[c]] = depth[v] + 1;
+                order.push_back(child[c]);
+            }
+        }
+        if ((int64_t)(order.size() - start) != n) return SELINV_ERR_BAD_TREE;
+    }
+    for (int64_t i = N - 1; i >= 0; --i) {
+        const int32_t v = order[i];
+        if (gparent[v] >= 0) height[gparent[v]] = std::max(height[gparent[v]], height[v] + 1);
+    }
+    int32_t H = 0, Dm = 0;
+    for (int64_t v = 0; v < N; ++v) {
+        H = std::max(H, height[v]);
+        Dm = std::max(Dm, depth[v]);
+    }
+    auto *pl = new (std::nothrow) selinv_tree_plan_s();
+    if (!pl) return SELINV_ERR_INVALID_ARG;
+    pl->trees = trees;
+    pl->n = n;
+    cudaGetDevice(&pl->device);
+    // counting sort by level keeps ascending ids within a level
+    std::vector<int32_t> cnodes(N), dnodes;
+    pl->collect_off.assign(H + 2, 0);
+    for (int64_t v = 0; v < N; ++v) pl->collect_off[height[v] + 1]++;
+    for (int32_t h = 0; h <= H; ++h) pl->collect_off[h + 1] += pl->collect_off[h];
+    {
+        std::vector<int64_t> pos(pl->collect_off.begin(), pl->collect_off.end() - 1);
+        for (int64_t v = 0; v < N; ++v) cnodes[pos[height[v]]++] = (int32_t)v;
+    }
+    pl->dist_off.assign(Dm + 1, 0);     // depths 1..Dm
+    for (int64_t v = 0; v < N; ++v)
+        if (depth[v] >= 1) pl->dist_off[depth[v]]++;
+    for (int32_t d = 1; d <= Dm; ++d) pl->dist_off[d] += pl->dist_off[d - 1];
+    dnodes.assign(std::max<int64_t>(pl->dist_off[Dm], 1), 0);
+    {
+        std::vector<int64_t> pos(Dm + 1, 0);
+        for (int32_t d = 1; d <= Dm; ++d) pos[d] = pl->dist_off[d - 1];
+        for (int64_t v = 0; v < N; ++v)
+            if (depth[v] >= 1) dnodes[pos[depth[v]]++] = (int32_t)v;
+    }
+    bool ok = true;
+    auto up = [&](int32_t **dst, const std::vector<int32_t> &src) {
+        if (!ok) return;
+        ok = cudaMalloc(dst, src.size() * sizeof(int32_t)) == cudaSuccess &&
+             cudaMemcpy(*dst, src.data(), src.size() * sizeof(int32_t), cudaMemcpyHostToDevice) == cudaSuccess;
+    };
+    up(&pl->d_collect_nodes, cnodes);
+    up(&pl->d_dist_nodes, dnodes);
+    up(&pl->d_child_ptr, cnt);
+    up(&pl->d_child_idx, child);
+    up(&pl->d_parent, gparent);
+    if (!ok) {
+        selinv_tree_plan_free(pl);
+        return SELINV_ERR_CUDA;
+    }
+    *out = pl;
+    return SELINV_OK;
+}
+
+void selinv_tree_plan_free(selinv_tree_plan_t *pl)
+{
+    if (!pl) return;
+    cudaFree(pl->d_collect_nodes);
+    cudaFree(pl->d_dist_nodes);
+    cudaFree(pl->d_child_ptr);
+    cudaFree(pl->d_child_idx);
+    cudaFree(pl->d_parent);
+    delete pl;
+}
+
+selinv_status selinv_tree_plan_levels(const selinv_tree_plan_t *pl, int32_t *collect, int32_t *distribute)
+{
+    if (!pl || !collect || !distribute) return SELINV_ERR_INVALID_ARG;
+    *collect = (int32_t)pl->collect_off.size() - 1;
+    *distribute = (int32_t)pl->dist_off.size();
+    return SELINV_OK;
+}
+
+size_t selinv_tree_workspace_size(const selinv_tree_plan_t *pl, selinv_dtype dtype, int32_t b)
+{
+    if (!pl || (dtype != SELINV_F64 && dtype != SELINV_F32) || b < 1 || b > 16) return 0;
+    return tree_workspace(pl, dtype == SELINV_F64 ? 8 : 4);
+}
+
+selinv_status selinv_tree(const selinv_tree_plan_t *pl, selinv_dtype dtype, int32_t b, const void *diag,
+                          const void *edge, void *G_diag, void *G_edge, double *logdet, int32_t *info,
+                          void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!pl || (dtype != SELINV_F64 && dtype != SELINV_F32) || b < 1) return SELINV_ERR_INVALID_ARG;
+    if (b > 16) return SELINV_ERR_UNSUPPORTED;
+    if (!diag || !edge || !G_diag || !G_edge || !info) return SELINV_ERR_INVALID_ARG;
+    const size_t es = dtype == SELINV_F64 ? 8 : 4;
+    if (!is_aligned(diag, es) || !is_aligned(edge, es) || !is_aligned(G_diag, es) || !is_aligned(G_edge, es) ||
+        !is_aligned(logdet, 8) || !is_aligned(info, 4) || !is_aligned(workspace, 256))
+        return SELINV_ERR_INVALID_ARG;
+    const size_t need = tree_workspace(pl, es);
+    if (!workspace || workspace_bytes < need) return SELINV_ERR_WORKSPACE;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev != pl->device) return SELINV_ERR_INVALID_ARG;
+    const bool full = b == 16 && is_aligned(diag, 16) && is_aligned(edge, 16) && is_aligned(G_diag, 16) &&
+                      is_aligned(G_edge, 16);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t err;
+    if (dtype == SELINV_F64)
+        err = run_tree<double>(pl, b, static_cast<const double *>(diag), static_cast<const double *>(edge),
+                               static_cast<double *>(G_diag), static_cast<double *>(G_edge), logdet, info,
+                               workspace, full, s);
+    else
+        err = run_tree<float>(pl, b, static_cast<const float *>(diag), static_cast<const float *>(edge),
+                              static_cast<float *>(G_diag), static_cast<float *>(G_edge), logdet, info,
+                              workspace, full, s);
+    return err == cudaSuccess ? SELINV_OK : SELINV_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,314 @@
+// Warp-level toolkit for blocks of size b <= 16: one warp owns one padded
+// 16 x 16 block at a time.  Blocks smaller than 16 are embedded with an
+// identity (diagonal blocks) or zero (off-diagonal blocks) pad, which leaves
+// the unpadded part of every Schur complement and inverse unchanged and adds
+// log 1 = 0 to the log-determinant.
+#pragma once
+
+#include "common.cuh"
+
+namespace selinv {
+namespace w16 {
+
+// Register tile.  Lane = 4 g + t holds rows g + 8 h (h = 0, 1) and columns
+// tcol(t, q) = 2 t + (q & 1) + 8 (q >> 1) (q = 0..3): the accumulator layout of
+// the m8n8k4 FP64 tensor-core instruction, four of whose 8 x 8 tiles cover the
+// 16 x 16 block (tile (h, q >> 1)).
+template <class T> struct Tile {
+    T v[2][4];
+};
+
+SELINV_DEVINL int tcol(int t, int q) { return 2 * t + (q & 1) + 8 * (q >> 1); }
+
+// Shared-memory image of a 16 x 16 block.
+//  double: 16 doubles per row (8 chunks of 16 B) with chunk index XOR f(r),
+//          f(r) = ((r & 1) << 2) | ((r >> 1) & 3).  Conflict-free for the
+//          tensor-core fragment reads (8 rows x 4 columns and 4 rows x 8
+//          columns) and for the tile's own 16-byte pair accesses.
+//  float:  row pitch 20 floats (8-byte pairs stay aligned; column reads of 8
+//          rows hit distinct banks).
+template <class T> struct SL;
+template <> struct SL<double> {
+    static constexpr int ELEMS = 256;
+    SELINV_DEVINL static int idx(int r, int c)
+    {
+        const int f = ((r & 1) << 2) | ((r >> 1) & 3);
+        return (r << 4) | ((((c >> 1) ^ f) << 1) | (c & 1));
+    }
+};
+template <> struct SL<float> {
+    static constexpr int ELEMS = 16 * 20;
+    SELINV_DEVINL static int idx(int r, int c) { return r * 20 + c; }
+};
+
+template <class T> struct Vec2;
+template <> struct Vec2<double> { using type = double2; };
+template <> struct Vec2<float> { using type = float2; };
+
+template <class T> SELINV_DEVINL void zero(Tile<T> &a)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) a.v[h][q] = T(0);
+}
+
+// ---- shared memory <-> registers -------------------------------------------
+
+template <class T> SELINV_DEVINL void to_smem(T *s, const Tile<T> &a, int g, int t)
+{
+    using V = typename Vec2<T>::type;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            V v;
+            v.x = a.v[h][2 * p];
+            v.y = a.v[h][2 * p + 1];
+            *reinterpret_cast<V *>(s + SL<T>::idx(g + 8 * h, 2 * t + 8 * p)) = v;
+        }
+}
+
+template <class T> SELINV_DEVINL void from_smem(Tile<T> &a, const T *s, int g, int t)
+{
+    using V = typename Vec2<T>::type;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            V v = *reinterpret_cast<const V *>(s + SL<T>::idx(g + 8 * h, 2 * t + 8 * p));
+            a.v[h][2 * p] = v.x;
+            a.v[h][2 * p + 1] = v.y;
+        }
+}
+
+// Writes the lower triangle (c <= r) of the tile and its mirror, so the
+// shared image is exactly symmetric and every entry is written once.
+template <class T> SELINV_DEVINL void to_smem_sym(T *s, const Tile<T> &a, int g, int t)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = g + 8 * h, c = tcol(t, q);
+            if (c <= r) s[SL<T>::idx(r, c)] = a.v[h][q];
+            if (c < r) s[SL<T>::idx(c, r)] = a.v[h][q];
+        }
+}
+
+// ---- global memory -----------------------------------------------------------
+
+// Diagonal block D (row-major b x b) into a tile, reading only D's lower
+// triangle (upper entries come from their mirror); identity pad beyond b.
+template <class T, bool FULL> SELINV_DEVINL void load_sym(Tile<T> &a, const T *D, int b, int g, int t)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = g + 8 * h, c = tcol(t, q);
+            const int rr = c <= r ? r : c, cc = c <= r ? c : r;
+            if (FULL) {
+                a.v[h][q] = __ldg(D + rr * 16 + cc);
+            } else {
+                a.v[h][q] = (r < b && c < b) ? __ldg(D + rr * b + cc) : (r == c ? T(1) : T(0));
+            }
+        }
+}
+
+// Off-diagonal block (row-major b x b) into shared memory, zero pad beyond b.
+// FULL: 16-byte cp.async chunks (caller commits / waits); else plain loads.
+template <class T, bool FULL> SELINV_DEVINL void load_block_async(T *s, const T *B, int b, int lane)
+{
+    if (FULL) {
+        constexpr int CH = 16 / sizeof(T);          // elements per chunk
+        constexpr int PER_ROW = 16 / CH;
+#pragma unroll
+        for (int j = lane; j < 16 * PER_ROW; j += 32) {
+            const int r = j / PER_ROW, c = (j % PER_ROW) * CH;
+            cp_async16(s + SL<T>::idx(r, c), B + r * 16 + c);
+        }
+    } else {
+        for (int j = lane; j < 256; j += 32) {
+            const int r = j >> 4, c = j & 15;
+            s[SL<T>::idx(r, c)] = (r < b && c < b) ? __ldg(B + r * b + c) : T(0);
+        }
+    }
+}
+
+// Full tile to a row-major b x b block in global memory.
+template <class T, bool FULL> SELINV_DEVINL void store_block(T *G, const Tile<T> &a, int b, int g, int t)
+{
+    using V = typename Vec2<T>::type;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const int r = g + 8 * h, c = 2 * t + 8 * p;
+            if (FULL) {
+                V v;
+                v.x = a.v[h][2 * p];
+                v.y = a.v[h][2 * p + 1];
+                __stcs(reinterpret_cast<V *>(G + r * 16 + c), v);
+            } else {
+                if (r < b && c < b) G[r * b + c] = a.v[h][2 * p];
+                if (r < b && c + 1 < b) G[r * b + c + 1] = a.v[h][2 * p + 1];
+            }
+        }
+}
+
+// Lower-triangle slot of a symmetric tile in workspace memory (192 elements):
+// [0, 64): rows 8..15 x cols 0..7, two entries per lane;
+// [64, 192): the two diagonal 8 x 8 tiles' entries of lanes with 2t <= g,
+// four per lane.  Exactly the entries with c <= r (plus four on the
+// diagonal pairs) are kept; to_smem_sym rebuilds the full block.
+constexpr int SLOT_ELEMS = 192;
+
+template <class T> SELINV_DEVINL void store_lower_slot(T *slot, const Tile<T> &a, int lane, int g, int t)
+{
+    using V = typename Vec2<T>::type;
+    V v;
+    v.x = a.v[1][0];
+    v.y = a.v[1][1];
+    *reinterpret_cast<V *>(slot + 2 * lane) = v;
+    if (2 * t <= g) {
+        V u, w;
+        u.x = a.v[0][0];
+        u.y = a.v[0][1];
+        w.x = a.v[1][2];
+        w.y = a.v[1][3];
+        *reinterpret_cast<V *>(slot + 64 + 4 * lane) = u;
+        *reinterpret_cast<V *>(slot + 64 + 4 * lane + 2) = w;
+    }
+}
+
+template <class T> SELINV_DEVINL void load_lower_slot(Tile<T> &a, const T *slot, int lane, int g, int t)
+{
+    using V = typename Vec2<T>::type;
+    V v = __ldcs(reinterpret_cast<const V *>(slot + 2 * lane));
+    a.v[1][0] = v.x;
+    a.v[1][1] = v.y;
+    a.v[0][2] = a.v[0][3] = T(0);
+    if (2 * t <= g) {
+        V u = __ldcs(reinterpret_cast<const V *>(slot + 64 + 4 * lane));
+        V w = __ldcs(reinterpret_cast<const V *>(slot + 64 + 4 * lane + 2));
+        a.v[0][0] = u.x;
+        a.v[0][1] = u.y;
+        a.v[1][2] = w.x;
+        a.v[1][3] = w.y;
+    } else {
+        a.v[0][0] = a.v[0][1] = a.v[1][2] = a.v[1][3] = T(0);
+    }
+}
+
+// ---- arithmetic --------------------------------------------------------------
+
+// acc += (NEG ? -1 : 1) * op(A) op(B), with A and B 16 x 16 in shared memory;
+// OPA / OPB = 1 means transposed.
+template <int OPA, int OPB, bool NEG>
+SELINV_DEVINL void gemm(Tile<double> &acc, const double *sA, const double *sB, int g, int t)
+{
+    using L = SL<double>;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+        double a[2], b[2];
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            a[m] = OPA == 0 ? sA[L::idx(8 * m + g, 4 * kk + t)] : sA[L::idx(4 * kk + t, 8 * m + g)];
+            if (NEG) a[m] = -a[m];
+        }
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+            b[n] = OPB == 0 ? sB[L::idx(4 * kk + t, 8 * n + g)] : sB[L::idx(8 * n + g, 4 * kk + t)];
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int n = 0; n < 2; ++n) dmma_8x8x4(acc.v[m][2 * n], acc.v[m][2 * n + 1], a[m], b[n]);
+    }
+}
+
+template <int OPA, int OPB, bool NEG>
+SELINV_DEVINL void gemm(Tile<float> &acc, const float *sA, const float *sB, int g, int t)
+{
+    using L = SL<float>;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        float a[2], b[4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            a[h] = OPA == 0 ? sA[L::idx(g + 8 * h, k)] : sA[L::idx(k, g + 8 * h)];
+            if (NEG) a[h] = -a[h];
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) b[q] = OPB == 0 ? sB[L::idx(k, tcol(t, q))] : sB[L::idx(tcol(t, q), k)];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc.v[h][q] = fmaf(a[h], b[q], acc.v[h][q]);
+    }
+}
+
+// In-register inverse of a symmetric positive definite tile by the symmetric
+// sweep form of Gauss-Jordan elimination (no pivoting): for k = 0..15,
+// with d = A_kk,  A_ij -= A_ik A_kj / d (i, j != k),  A_ik /= d,  A_kj /= d,
+// A_kk = -1/d; after all k the tile holds -A^-1, which is negated.  The
+// pivots d are the successive Schur-complement pivots, so their product is
+// det A (multiplied into `det`); a pivot that is not > 0 sets `bad`.
+template <class T>
+SELINV_DEVINL void spd_inverse(Tile<T> &a, int lane, int g, int t, LogAcc &det, bool &bad)
+{
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const int kg = k & 7, kh = k >> 3, kt = (k & 7) >> 1, kq = (k & 1) | ((k >> 3) << 1);
+        const int src_col = (lane & ~3) | kt;     // owner of A[g + 8h][k]
+        const int src_row = (kg << 2) | t;        // owner of A[k][tcol(t, q)]
+        T col[2], row[4];
+        col[0] = shfl(a.v[0][kq], src_col);
+        col[1] = shfl(a.v[1][kq], src_col);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) row[q] = shfl(a.v[kh][q], src_row);
+        const T d = shfl(a.v[kh][kq], (kg << 2) | kt);
+        bad |= !(d > T(0));
+        det.mul((double)d);
+        const T p = T(1) / d;
+        T tc[2];
+        tc[0] = col[0] * p;
+        tc[1] = col[1] * p;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) a.v[h][q] = fma(-tc[h], row[q], a.v[h][q]);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const bool in_row = (g + 8 * h) == k;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const bool in_col = (t == kt) && (q == kq);
+                if (in_row) a.v[h][q] = in_col ? -p : row[q] * p;
+                else if (in_col) a.v[h][q] = tc[h];
+            }
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) a.v[h][q] = -a.v[h][q];
+}
+
+// y_r = sum_c A[r][c] x[c] for the lane's rows g, g + 8 (x in shared memory);
+// every lane of a row group ends with the full sums.
+template <class T> SELINV_DEVINL void row_matvec(T out[2], const Tile<T> &a, const T *x, int t)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        T s = T(0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) s = fma(a.v[h][q], x[tcol(t, q)], s);
+        s += shfl_xor(s, 1);
+        s += shfl_xor(s, 2);
+        out[h] = s;
+    }
+}
+
+}  // namespace w16
+}  // namespace selinv

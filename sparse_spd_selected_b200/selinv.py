@@ -1,0 +1,291 @@
+"""ctypes binding of libselinv (the C ABI in include/selinv.h).
+
+Argument marshalling only: tensors are checked for device, dtype and
+contiguity, outputs and the workspace are allocated with torch, and every
+step of the computation runs in the library's CUDA kernels on the current
+torch stream.  There is no CPU fallback: if ``libselinv.so`` is missing or no
+CUDA device is present, calls raise.
+
+The calls follow the problem statement of gabp-sparse-inv 0.3.2 (PyPI page,
+"Quickstart"): inputs ``[..., L, b, b]`` with optional leading batch
+dimensions, outputs only the on-pattern blocks of A^-1 (never the dense
+inverse), plus log det A and A^-1 r from the same factorisation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libselinv.so")
+
+OK, ERR_INVALID_ARG, ERR_NOT_SPD, ERR_BAD_TREE, ERR_CUDA, ERR_WORKSPACE, ERR_UNSUPPORTED = range(7)
+F64, F32 = 0, 1
+
+_lib = None
+
+
+class SelinvError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+class NotSPDError(SelinvError):
+    def __init__(self, info):
+        self.info = info
+        super().__init__(ERR_NOT_SPD, f"first failing block per batch element: {info}")
+
+
+def lib():
+    """The loaded libselinv.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m sparse_spd_selected_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+        L.selinv_status_string.argtypes = [ctypes.c_int]
+        L.selinv_status_string.restype = ctypes.c_char_p
+        L.selinv_version.restype = I32
+        L.selinv_max_block.restype = I32
+        L.selinv_chain_workspace_size.argtypes = [ctypes.c_int, I64, I64, I32, I32, I32]
+        L.selinv_chain_workspace_size.restype = SZ
+        L.selinv_chain.argtypes = [ctypes.c_int, I64, I64, I32, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.selinv_chain.restype = ctypes.c_int
+        L.chain_solve.argtypes = [ctypes.c_int, I64, I64, I32, P, P, P, P, P, P, P, SZ, P]
+        L.chain_solve.restype = ctypes.c_int
+        L.selinv_tree_plan.argtypes = [P, I64, I64, ctypes.POINTER(P)]
+        L.selinv_tree_plan.restype = ctypes.c_int
+        L.selinv_tree_plan_free.argtypes = [P]
+        L.selinv_tree_plan_free.restype = None
+        L.selinv_tree_plan_levels.argtypes = [P, ctypes.POINTER(I32), ctypes.POINTER(I32)]
+        L.selinv_tree_plan_levels.restype = ctypes.c_int
+        L.selinv_tree_workspace_size.argtypes = [P, ctypes.c_int, I32]
+        L.selinv_tree_workspace_size.restype = SZ
+        L.selinv_tree.argtypes = [P, ctypes.c_int, I32, P, P, P, P, P, P, P, SZ, P]
+        L.selinv_tree.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().selinv_status_string(int(status)).decode()
+
+
+def max_block() -> int:
+    return int(lib().selinv_max_block())
+
+
+def _code(dtype) -> int:
+    if dtype == torch.float64:
+        return F64
+    if dtype == torch.float32:
+        return F32
+    raise TypeError(f"libselinv computes in float64 or float32, not {dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _cuda_contig(name, t, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _stream_handle(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status, what):
+    if status != OK:
+        raise SelinvError(status, what)
+
+
+def chain_workspace_size(dtype, batch, L, b, want_g=True, want_x=False) -> int:
+    return int(lib().selinv_chain_workspace_size(_code(dtype), batch, L, b, int(want_g), int(want_x)))
+
+
+def _workspace(nbytes, device, workspace):
+    if nbytes == 0:
+        return None
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise ValueError(f"workspace needs {nbytes} bytes")
+        return workspace
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def _raise_on_info(info, check):
+    if check:
+        host = info.cpu()
+        if bool((host >= 0).any()):
+            raise NotSPDError(host.tolist())
+
+
+def selinv_chain(diag: torch.Tensor, lower: Optional[torch.Tensor] = None, rhs: Optional[torch.Tensor] = None,
+                 *, want_g: bool = True, check: bool = True, out=None, workspace=None, stream=None):
+    """Selected inverse (+ log det, + optional solve) of block-tridiagonal SPD chains.
+
+    diag [..., L, b, b], lower [..., L-1, b, b] (lower[i] = A_{i+1,i}),
+    rhs [..., L, b] optional.  Returns a dict with G_diag, G_lower, logdet
+    (float64), x (if rhs) and info (int32, -1 = ok).  With check=True the
+    call synchronises once to read info and raises NotSPDError on failure.
+    ``out`` may hold preallocated output tensors under the same keys.
+    """
+    _cuda_contig("diag", diag)
+    dt = diag.dtype
+    code = _code(dt)
+    if diag.dim() < 3 or diag.shape[-1] != diag.shape[-2]:
+        raise ValueError("diag must be [..., L, b, b]")
+    lead = tuple(diag.shape[:-3])
+    L, b = int(diag.shape[-3]), int(diag.shape[-1])
+    batch = 1
+    for d in lead:
+        batch *= int(d)
+    if L > 1:
+        if lower is None:
+            raise ValueError("lower is required when L > 1")
+        _cuda_contig("lower", lower, dt)
+        if tuple(lower.shape) != lead + (L - 1, b, b):
+            raise ValueError(f"lower must be {lead + (L - 1, b, b)}, got {tuple(lower.shape)}")
+    else:
+        lower = None
+    if rhs is not None:
+        _cuda_contig("rhs", rhs, dt)
+        if tuple(rhs.shape) != lead + (L, b):
+            raise ValueError(f"rhs must be {lead + (L, b)}")
+    dev = diag.device
+    out = dict(out or {})
+    G_diag = G_lower = x = None
+    if want_g:
+        G_diag = out.get("G_diag")
+        if G_diag is None:
+            G_diag = torch.empty(lead + (L, b, b), dtype=dt, device=dev)
+        G_lower = out.get("G_lower")
+        if G_lower is None:
+            G_lower = torch.empty(lead + (max(L - 1, 0), b, b), dtype=dt, device=dev)
+    if rhs is not None:
+        x = out.get("x")
+        if x is None:
+            x = torch.empty(lead + (L, b), dtype=dt, device=dev)
+    logdet = out.get("logdet")
+    if logdet is None:
+        logdet = torch.empty(lead, dtype=torch.float64, device=dev)
+    info = out.get("info")
+    if info is None:
+        info = torch.empty(lead, dtype=torch.int32, device=dev)
+    nbytes = chain_workspace_size(dt, batch, L, b, want_g, rhs is not None)
+    ws = _workspace(nbytes, dev, workspace)
+    with torch.cuda.device(dev):
+        st = lib().selinv_chain(code, batch, L, b, _ptr(diag), _ptr(lower),
+                                _ptr(G_diag), _ptr(G_lower if L > 1 else None), _ptr(logdet),
+                                _ptr(rhs), _ptr(x), _ptr(info), _ptr(ws), nbytes,
+                                _stream_handle(stream))
+    _check(st, "selinv_chain")
+    _raise_on_info(info, check)
+    return {"G_diag": G_diag, "G_lower": G_lower, "logdet": logdet, "x": x, "info": info}
+
+
+def chain_solve(diag, lower, rhs, *, check=True, workspace=None, stream=None):
+    """x = A^-1 r for block-tridiagonal SPD chains (no G blocks formed); returns (x, logdet, info)."""
+    r = selinv_chain(diag, lower, rhs, want_g=False, check=False, workspace=workspace, stream=stream)
+    _raise_on_info(r["info"], check)
+    return r["x"], r["logdet"], r["info"]
+
+
+class TreePlan:
+    """Validated level-set schedule of `trees` parent arrays of n nodes each (cached on the device)."""
+
+    def __init__(self, parent):
+        import numpy as np
+        p = np.ascontiguousarray(np.asarray(parent, dtype=np.int32))
+        if p.ndim == 1:
+            p = p[None]
+        if p.ndim != 2:
+            raise ValueError("parent must be [n] or [trees, n]")
+        self.trees, self.n = int(p.shape[0]), int(p.shape[1])
+        h = ctypes.c_void_p()
+        st = lib().selinv_tree_plan(p.ctypes.data_as(ctypes.c_void_p), self.trees, self.n, ctypes.byref(h))
+        _check(st, "selinv_tree_plan")
+        self._h = h
+
+    @property
+    def handle(self):
+        return self._h
+
+    def levels(self):
+        c, d = ctypes.c_int32(), ctypes.c_int32()
+        _check(lib().selinv_tree_plan_levels(self._h, ctypes.byref(c), ctypes.byref(d)), "levels")
+        return c.value, d.value
+
+    def workspace_size(self, dtype, b) -> int:
+        return int(lib().selinv_tree_workspace_size(self._h, _code(dtype), b))
+
+    def close(self):
+        if getattr(self, "_h", None) and _lib is not None:
+            _lib.selinv_tree_plan_free(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def selinv_tree(plan: TreePlan, diag: torch.Tensor, edge: torch.Tensor, *, check=True, out=None,
+                workspace=None, stream=None):
+    """Selected inverse and log det of block-tree SPD matrices.
+
+    diag, edge [trees, n, b, b] (or [n, b, b] for one tree) with
+    edge[v] = A_{parent(v), v}.  Returns dict with G_diag, G_edge (root slot
+    zero), logdet [trees] float64 and info [trees].
+    """
+    _cuda_contig("diag", diag)
+    dt = diag.dtype
+    code = _code(dt)
+    _cuda_contig("edge", edge, dt)
+    single = diag.dim() == 3
+    d4 = diag[None] if single else diag
+    e4 = edge[None] if single else edge
+    if d4.dim() != 4 or tuple(d4.shape[:2]) != (plan.trees, plan.n) or d4.shape[-1] != d4.shape[-2]:
+        raise ValueError(f"diag must be [{plan.trees}, {plan.n}, b, b]")
+    if e4.shape != d4.shape:
+        raise ValueError("edge must have diag's shape")
+    b = int(d4.shape[-1])
+    dev = diag.device
+    out = dict(out or {})
+    G_diag = out.get("G_diag")
+    if G_diag is None:
+        G_diag = torch.empty_like(d4)
+    G_edge = out.get("G_edge")
+    if G_edge is None:
+        G_edge = torch.empty_like(d4)
+    logdet = out.get("logdet")
+    if logdet is None:
+        logdet = torch.empty(plan.trees, dtype=torch.float64, device=dev)
+    info = out.get("info")
+    if info is None:
+        info = torch.empty(plan.trees, dtype=torch.int32, device=dev)
+    nbytes = plan.workspace_size(dt, b)
+    ws = _workspace(nbytes, dev, workspace)
+    with torch.cuda.device(dev):
+        st = lib().selinv_tree(plan.handle, code, b, _ptr(d4), _ptr(e4), _ptr(G_diag), _ptr(G_edge),
+                               _ptr(logdet), _ptr(info), _ptr(ws), nbytes, _stream_handle(stream))
+    _check(st, "selinv_tree")
+    _raise_on_info(info, check)
+    if single:
+        G_diag, G_edge = G_diag[0], G_edge[0]
+    return {"G_diag": G_diag, "G_edge": G_edge, "logdet": logdet, "info": info}

@@ -1,0 +1,88 @@
+"""The C-ABI library loads, exports every entry point include/selinv.h declares,
+and rejects bad arguments synchronously (no GPU needed: nothing is launched)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from sparse_spd_selected_b200 import build, selinv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return selinv.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "selinv.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", src)
+    keywords = {"if", "sizeof", "while", "for", "return"}
+    return sorted({n for n in names if n not in keywords and n.startswith(("selinv_", "chain_"))})
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert "selinv_chain" in names and "chain_solve" in names and "selinv_tree" in names
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings_and_limits(lib):
+    for code in range(7):
+        assert selinv.status_string(code)
+    assert selinv.max_block() == 128
+    assert lib.selinv_version() >= 100
+
+
+FAKE = ctypes.c_void_p(1 << 20)     # never dereferenced: validation fails first
+
+
+def call_chain(lib, dtype=0, batch=1, L=4, b=4, diag=FAKE, lower=FAKE, G=FAKE, Gl=FAKE, ld=None,
+               rhs=None, x=None, info=FAKE, ws=FAKE, ws_bytes=1 << 30):
+    return lib.selinv_chain(dtype, batch, L, b, diag, lower, G, Gl, ld, rhs, x, info, ws, ws_bytes, None)
+
+
+def test_chain_argument_errors(lib):
+    assert call_chain(lib, dtype=7) == selinv.ERR_INVALID_ARG
+    assert call_chain(lib, L=0) == selinv.ERR_INVALID_ARG
+    assert call_chain(lib, b=0) == selinv.ERR_INVALID_ARG
+    assert call_chain(lib, batch=-1) == selinv.ERR_INVALID_ARG
+    assert call_chain(lib, b=129) == selinv.ERR_UNSUPPORTED
+    assert call_chain(lib, diag=None) == selinv.ERR_INVALID_ARG
+    assert call_chain(lib, lower=None) == selinv.ERR_INVALID_ARG
+    assert call_chain(lib, info=None) == selinv.ERR_INVALID_ARG
+    assert call_chain(lib, diag=ctypes.c_void_p((1 << 20) + 4)) == selinv.ERR_INVALID_ARG   # misaligned f64
+    assert call_chain(lib, Gl=None) == selinv.ERR_INVALID_ARG                              # G_diag without G_lower
+    assert call_chain(lib, rhs=FAKE) == selinv.ERR_INVALID_ARG                              # rhs without x
+    assert call_chain(lib, ws=None) == selinv.ERR_WORKSPACE
+    assert call_chain(lib, ws_bytes=16) == selinv.ERR_WORKSPACE
+    assert call_chain(lib, batch=0) == selinv.OK                                            # nothing to do
+
+
+def test_workspace_sizes(lib):
+    f = lib.selinv_chain_workspace_size
+    assert f(0, 10, 8, 16, 0, 0) == 0                       # log det only: no workspace
+    small = f(0, 10, 8, 16, 1, 0)
+    assert small >= 10 * 7 * 192 * 8 and small % 256 == 0
+    assert f(1, 10, 8, 16, 1, 0) < small                     # float32 slots are half the size
+    assert f(0, 10, 1, 16, 1, 1) == 0                        # one block: nothing kept between sweeps
+
+
+def test_tree_plan_rejects_malformed_parents(lib):
+    def plan(parent):
+        p = np.ascontiguousarray(np.asarray(parent, dtype=np.int32))
+        h = ctypes.c_void_p()
+        trees, n = (1, p.size) if p.ndim == 1 else p.shape
+        return lib.selinv_tree_plan(p.ctypes.data_as(ctypes.c_void_p), trees, n, ctypes.byref(h))
+    assert plan([-1, 0, -1]) == selinv.ERR_BAD_TREE          # two roots
+    assert plan([0, 0, 1]) == selinv.ERR_BAD_TREE            # no root (self loop at 0)
+    assert plan([1, 2, 0, -1]) == selinv.ERR_BAD_TREE        # cycle 0 -> 1 -> 2 -> 0
+    assert plan([-1, 5, 0]) == selinv.ERR_BAD_TREE           # out of range
+    assert plan([[-1, 0, 1], [-1, -1, 0]]) == selinv.ERR_BAD_TREE   # second tree has two roots
+    assert lib.selinv_tree_plan(None, 1, 3, ctypes.byref(ctypes.c_void_p())) == selinv.ERR_INVALID_ARG

@@ -1,0 +1,207 @@
+"""GPU chain kernels vs the CPU oracle, called through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_spd_selected_b200 import inputs, selinv
+from tests.parity import TOL, host, logdet_err, to_dev, worst
+
+pytestmark = pytest.mark.gpu
+
+
+def run_both(diag, lower, rhs, dtype, lead_ndim=1):
+    """GPU (inputs rounded to dtype) vs oracle on the same rounded inputs."""
+    d_dev, l_dev = to_dev(diag, dtype), to_dev(lower, dtype)
+    r_dev = to_dev(rhs, dtype) if rhs is not None else None
+    out = selinv.selinv_chain(d_dev, l_dev, r_dev)
+    ref = oracle.chain(host(d_dev), host(l_dev), host(r_dev) if rhs is not None else None)
+    assert (ref["info"] == -1).all()
+    errs = {
+        "G_diag": worst(host(out["G_diag"]), ref["G_diag"], lead_ndim),
+        "G_lower": worst(host(out["G_lower"]), ref["G_lower"], lead_ndim) if diag.shape[-3] > 1 else 0.0,
+        "logdet": logdet_err(host(out["logdet"]), ref["logdet"]),
+    }
+    if rhs is not None:
+        errs["x"] = worst(host(out["x"]), ref["x"], lead_ndim)
+    assert (host(out["info"]) == -1).all()
+    return errs, out
+
+
+@pytest.mark.parametrize("b", [1, 2, 3, 4, 5, 7, 8, 9, 12, 15, 16])
+@pytest.mark.parametrize("L", [1, 2, 3, 5, 17])
+def test_small_blocks_f64(cuda_ok, b, L):
+    diag, lower, rhs = inputs.chain_inputs(6, L, b, seed=1000 + 17 * b + L, load=0.5)
+    errs, _ = run_both(diag, lower, rhs, torch.float64)
+    assert max(errs.values()) <= TOL[torch.float64], errs
+
+
+@pytest.mark.parametrize("b,L", [(4, 9), (16, 33), (11, 6)])
+def test_small_blocks_f32(cuda_ok, b, L):
+    diag, lower, rhs = inputs.chain_inputs(5, L, b, seed=2000 + b, load=2.0)
+    errs, _ = run_both(diag, lower, rhs, torch.float32)
+    assert max(errs.values()) <= TOL[torch.float32], errs
+
+
+def test_leading_batch_dims(cuda_ok):
+    diag, lower, rhs = inputs.chain_inputs(6, 7, 16, seed=3001, load=1.0)
+    shp = (2, 3)
+    errs, out = run_both(diag.reshape(shp + diag.shape[1:]), lower.reshape(shp + lower.shape[1:]),
+                         rhs.reshape(shp + rhs.shape[1:]), torch.float64, lead_ndim=2)
+    assert out["G_diag"].shape == (2, 3, 7, 16, 16) and out["logdet"].shape == (2, 3)
+    assert max(errs.values()) <= 1e-9, errs
+
+
+def test_quickstart_fact(cuda_ok):
+    """G_diag[0] == inv(A)[0:4, 0:4] to 1e-10 on 8 blocks of 4 with diag_load 2.0."""
+    w = inputs.WORKLOADS["chain_1x8_b4"]
+    g = inputs.generate(w)
+    out = selinv.selinv_chain(to_dev(g["diag"][0], torch.float64), to_dev(g["lower"][0], torch.float64),
+                              to_dev(g["rhs"][0], torch.float64))
+    from tests.dense import chain_dense
+    inv = np.linalg.inv(chain_dense(g["diag"][0], g["lower"][0]))
+    assert np.abs(host(out["G_diag"])[0] - inv[0:4, 0:4]).max() <= 1e-10
+    errs, _ = run_both(g["diag"], g["lower"], g["rhs"], torch.float64)
+    assert max(errs.values()) <= 1e-9, errs
+
+
+def test_full_size_b16_sampled(cuda_ok):
+    """4096 chains x 64 blocks of 16 (the benchmark launch), checked on sampled chains."""
+    w = inputs.WORKLOADS["chain_4096x64_b16"]
+    g = inputs.generate(w)
+    d, l, r = (to_dev(g[k], torch.float64) for k in ("diag", "lower", "rhs"))
+    out = selinv.selinv_chain(d, l, r)
+    pick = [0, 1, 2, 777, 2048, 4094, 4095]
+    ref = oracle.chain(g["diag"][pick], g["lower"][pick], g["rhs"][pick])
+    assert worst(host(out["G_diag"][pick]), ref["G_diag"]) <= 1e-9
+    assert worst(host(out["G_lower"][pick]), ref["G_lower"]) <= 1e-9
+    assert worst(host(out["x"][pick]), ref["x"]) <= 1e-9
+    assert logdet_err(host(out["logdet"][pick]), ref["logdet"]) <= 1e-9
+    # properties that hold for every chain: exact symmetry of G_ii, positive diagonal
+    Gd = out["G_diag"]
+    assert torch.equal(Gd, Gd.transpose(-1, -2))
+    assert bool((torch.diagonal(Gd, dim1=-2, dim2=-1) > 0).all())
+
+
+def test_upper_triangle_of_diag_is_not_read(cuda_ok):
+    diag, lower, rhs = inputs.chain_inputs(3, 6, 16, seed=3100, load=1.0)
+    d_dev = to_dev(diag, torch.float64)
+    ref = selinv.selinv_chain(d_dev, to_dev(lower, torch.float64), to_dev(rhs, torch.float64))
+    junk = d_dev.clone()
+    iu = torch.triu_indices(16, 16, 1)
+    junk[..., iu[0], iu[1]] = float("nan")
+    out = selinv.selinv_chain(junk, to_dev(lower, torch.float64), to_dev(rhs, torch.float64))
+    for k in ("G_diag", "G_lower", "logdet", "x"):
+        assert torch.equal(out[k], ref[k]), k
+
+
+def test_not_spd_reports_first_failing_block(cuda_ok):
+    diag, lower, _ = inputs.chain_inputs(3, 7, 16, seed=3200, load=1.0)
+    diag[1, 4] = -np.eye(16)
+    diag[2, 0, 3, 3] = np.nan
+    with pytest.raises(selinv.NotSPDError) as ei:
+        selinv.selinv_chain(to_dev(diag, torch.float64), to_dev(lower, torch.float64))
+    assert ei.value.info == [-1, 4, 0]
+    out = selinv.selinv_chain(to_dev(diag, torch.float64), to_dev(lower, torch.float64), check=False)
+    assert host(out["info"]).tolist() == [-1, 4, 0]
+
+
+def test_deterministic(cuda_ok):
+    diag, lower, rhs = inputs.chain_inputs(64, 20, 16, seed=3300, load=1.0)
+    args = [to_dev(a, torch.float64) for a in (diag, lower, rhs)]
+    a = selinv.selinv_chain(*args)
+    b = selinv.selinv_chain(*args)
+    for k in ("G_diag", "G_lower", "logdet", "x"):
+        assert torch.equal(a[k], b[k]), k
+
+
+def test_solve_only_and_logdet_only(cuda_ok):
+    diag, lower, rhs = inputs.chain_inputs(9, 12, 16, seed=3400, load=1.0)
+    d, l, r = (to_dev(a, torch.float64) for a in (diag, lower, rhs))
+    full = selinv.selinv_chain(d, l, r)
+    x, ld, info = selinv.chain_solve(d, l, r)
+    assert torch.equal(x, full["x"]) and torch.equal(ld, full["logdet"])
+    only = selinv.selinv_chain(d, l, want_g=False)
+    assert torch.equal(only["logdet"], full["logdet"]) and only["G_diag"] is None
+
+
+def test_workspace_too_small_is_rejected(cuda_ok):
+    diag, lower, _ = inputs.chain_inputs(2, 5, 16, seed=3500, load=1.0)
+    ws = torch.empty(64, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ValueError):
+        selinv.selinv_chain(to_dev(diag, torch.float64), to_dev(lower, torch.float64), workspace=ws)
+
+
+def test_empty_batch(cuda_ok):
+    d = torch.empty((0, 5, 16, 16), dtype=torch.float64, device="cuda")
+    l = torch.empty((0, 4, 16, 16), dtype=torch.float64, device="cuda")
+    out = selinv.selinv_chain(d, l)
+    assert out["G_diag"].shape == (0, 5, 16, 16)
+
+
+# ---------------- 16 < b <= 128: one CTA per chain ----------------
+
+@pytest.mark.parametrize("b", [17, 24, 32, 33, 48, 64, 65, 100, 128])
+@pytest.mark.parametrize("L", [1, 2, 5])
+def test_large_blocks_f64(cuda_ok, b, L):
+    diag, lower, rhs = inputs.chain_inputs(3, L, b, seed=4000 + 7 * b + L, load=0.5)
+    errs, _ = run_both(diag, lower, rhs, torch.float64)
+    assert max(errs.values()) <= TOL[torch.float64], errs
+
+
+@pytest.mark.parametrize("b,L", [(32, 20), (64, 6), (128, 4), (40, 7)])
+def test_large_blocks_f32(cuda_ok, b, L):
+    diag, lower, rhs = inputs.chain_inputs(3, L, b, seed=5000 + b, load=2.0)
+    errs, _ = run_both(diag, lower, rhs, torch.float32)
+    assert max(errs.values()) <= TOL[torch.float32], errs
+
+
+def test_large_solve_only_and_logdet_only(cuda_ok):
+    diag, lower, rhs = inputs.chain_inputs(4, 9, 64, seed=5100, load=1.0)
+    d, l, r = (to_dev(a, torch.float64) for a in (diag, lower, rhs))
+    full = selinv.selinv_chain(d, l, r)
+    x, ld, _ = selinv.chain_solve(d, l, r)
+    assert torch.equal(x, full["x"]) and torch.equal(ld, full["logdet"])
+    only = selinv.selinv_chain(d, l, want_g=False)
+    assert torch.equal(only["logdet"], full["logdet"])
+    Gd = full["G_diag"]
+    assert torch.equal(Gd, Gd.transpose(-1, -2))
+
+
+def test_grid_full_size_sampled(cuda_ok):
+    """256 grid precisions (128 x 128 grid as 128 blocks of 128), checked on two elements
+    against the oracle and against the spectral closed form."""
+    from tests.pins import grid_closed_form
+    w = inputs.WORKLOADS["grid_256x128_b128"]
+    diag, lower, rhs, taus = inputs.grid_inputs_torch(w.batch, w.b, w.seed, "cuda")
+    out = selinv.selinv_chain(diag, lower, rhs)
+    pick = [0, 255]
+    g = inputs.generate(w, elements=pick)
+    ref = oracle.chain(g["diag"], g["lower"], g["rhs"])
+    assert worst(host(out["G_diag"][pick]), ref["G_diag"]) <= 1e-9
+    assert worst(host(out["G_lower"][pick]), ref["G_lower"]) <= 1e-9
+    assert worst(host(out["x"][pick]), ref["x"]) <= 1e-9
+    assert logdet_err(host(out["logdet"][pick]), ref["logdet"]) <= 1e-9
+    for k, e in enumerate(pick):
+        Gd, Gl, ld, x = grid_closed_form(w.b, g["tau"][k], g["rhs"][k], rows=[0, 63, 127])
+        for i in (0, 63, 127):
+            assert worst(host(out["G_diag"][e, i])[None], Gd[i][None]) <= 1e-9
+        for i in (0, 63):
+            assert worst(host(out["G_lower"][e, i])[None], Gl[i][None]) <= 1e-9
+        assert abs(host(out["logdet"][e]) - ld) / abs(ld) <= 1e-9
+        assert worst(host(out["x"][e])[None], x[None]) <= 1e-9
+
+
+@pytest.mark.parametrize("dtype", [torch.float64, torch.float32])
+def test_long_chains_full_size_sampled(cuda_ok, dtype):
+    """64 chains of 4096 blocks of 32 (diag load 0.5), float64 and float32, sampled chains."""
+    w = inputs.WORKLOADS["chain_64x4096_b32"]
+    g = inputs.generate(w)
+    d, l = to_dev(g["diag"], dtype), to_dev(g["lower"], dtype)
+    out = selinv.selinv_chain(d, l)
+    pick = [0, 63]
+    ref = oracle.chain(host(d[pick]), host(l[pick]))
+    tol = TOL[dtype]
+    assert worst(host(out["G_diag"][pick]), ref["G_diag"]) <= tol
+    assert worst(host(out["G_lower"][pick]), ref["G_lower"]) <= tol
+    assert logdet_err(host(out["logdet"][pick]), ref["logdet"]) <= tol
