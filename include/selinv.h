@@ -115,6 +115,34 @@ selinv_status chain_solve(selinv_dtype dtype, int64_t batch, int64_t L, int32_t 
                           void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Same computation as selinv_chain for b <= 16, with no workspace argument
+ * and no allocation of any kind.  The pages have no counterpart: this entry
+ * point exists for callers that cannot allocate device memory -- code running
+ * inside another framework's execution hook (an inference-engine plugin's
+ * enqueue, a compiler runtime's custom call, a fixed-budget real-time loop),
+ * where the framework owns all device memory and a cudaMalloc is forbidden,
+ * fails, or would synchronise the device.  Such callers pass inputs and
+ * outputs only (arguments and layouts as in selinv_chain).
+ *
+ * The scratch is a library-owned device array of SELINV_CHAIN_NOALLOC_MAX_BYTES
+ * (16 MiB) that every GPU loading the library keeps until the process
+ * exits.  Requests needing more -- batch * (L-1) * 192 * sizeof(element) bytes
+ * when G or x is asked for -- return SELINV_ERR_WORKSPACE before anything is
+ * launched.  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  All calls share the one array and it keeps the
+ * last call's contents; nothing needs clearing, because every slot a call
+ * reads is written earlier in the same call.  Calls whose executions overlap
+ * on the GPU (different streams, or different host threads) race on it.
+ */
+#define SELINV_CHAIN_NOALLOC_MAX_BYTES ((size_t)16 << 20)
+
+selinv_status selinv_chain_noalloc(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b,
+                                   const void *diag, const void *lower,
+                                   void *G_diag, void *G_lower, double *logdet,
+                                   const void *rhs, void *x, int32_t *info, void *stream);
+
+/*
  * Tree plan: validates `trees` parent arrays of n nodes each (HOST memory,
  * parent [trees, n] int32, exactly one root per tree with parent = -1, no
  * cycles, indices in [0, n)), builds the level-set schedule -- nodes grouped
