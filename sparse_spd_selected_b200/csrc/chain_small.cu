@@ -25,10 +25,18 @@ namespace {
 
 constexpr int WARPS = 4;
 
-template <class T> __host__ __device__ constexpr int warp_smem_elems() { return 4 * w16::SL<T>::ELEMS + 64; }
+// Resident CTAs per SM the register allocation is sized for (4 warps each).
+#ifndef SELINV_CHAIN_MINB
+#define SELINV_CHAIN_MINB 4
+#endif
+
+template <class T> __host__ __device__ constexpr int warp_smem_elems()
+{
+    return 4 * w16::SL<T>::ELEMS + w16::SLOT_ELEMS + 96;
+}
 
 template <class T, bool FULL, bool WANT_G, bool WANT_X>
-__global__ void __launch_bounds__(WARPS * 32) chain_small_kernel(ChainArgs<T> p)
+__global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_kernel(ChainArgs<T> p)
 {
     using namespace w16;
     constexpr int E = SL<T>::ELEMS;
@@ -43,16 +51,19 @@ __global__ void __launch_bounds__(WARPS * 32) chain_small_kernel(ChainArgs<T> p)
     T *sS = sbase;             // S_i^-1 (operand), later G_{i+1,i}
     T *sW = sS + E;            // W_i
     T *sB = sW + E;            // B_i
-    T *sG = sB + E;            // G_{i+1,i+1}
-    T *sy = sG + E;            // y vectors, two buffers of 16
+    T *sD = sB + E;            // D_{i+1} (lower triangle); G_{i+1,i+1} in the distribute sweep
+    T *sG = sD;
+    T *stg = sD + E;           // staged S_i^-1 slot (distribute sweep)
+    T *sy = stg + SLOT_ELEMS;  // y vectors, two buffers of 16
     T *sx = sy + 32;           // x vectors, two buffers of 16
+    T *cb = sx + 32;           // pivot-column broadcast, two buffers of 16
 
     const int b = p.b;
     const int64_t L = p.L;
     const int64_t bb = (int64_t)b * b;
     const T *D = p.diag + e * L * bb;
     const T *Bl = p.lower + e * (L - 1) * bb;
-    T *ws = p.ws + e * (L - 1) * SLOT_ELEMS;
+    T *ws = (WANT_G || WANT_X) ? p.ws + e * (L - 1) * SLOT_ELEMS : nullptr;
     const T *R = WANT_X ? p.rhs + e * L * b : nullptr;
     T *X = WANT_X ? p.x + e * L * b : nullptr;
 
@@ -60,12 +71,17 @@ __global__ void __launch_bounds__(WARPS * 32) chain_small_kernel(ChainArgs<T> p)
     det.init();
     int fail = -1;
 
-    Tile<T> a, dn, w;
-    load_sym<T, FULL>(a, D, b, g, t);
+    Tile<T> a, w;
+    load_lower_async<T, FULL>(sD, D, b, lane);
+    cp_async_commit();
+    cp_async_wait_all();
+    __syncwarp();
+    from_smem_lower<T>(a, sD, g, t);
+    __syncwarp();
     if (L > 1) {
         load_block_async<T, FULL>(sB, Bl, b, lane);
+        load_lower_async<T, FULL>(sD, D + bb, b, lane);
         cp_async_commit();
-        load_sym<T, FULL>(dn, D + bb, b, g, t);
     }
     T rn[2] = {T(0), T(0)};    // r_{i+1} at rows g, g+8 (lanes with t == 0)
     if (WANT_X) {
@@ -84,7 +100,7 @@ __global__ void __launch_bounds__(WARPS * 32) chain_small_kernel(ChainArgs<T> p)
     // ---------------- collect sweep ----------------
     for (int64_t i = 0; i < L; ++i) {
         bool bad = false;
-        spd_inverse<T>(a, lane, g, t, det, bad);
+        spd_inverse<T>(a, cb, g, t, det, bad);
         det.renorm();
         if (bad && fail < 0) fail = (int)i;
         if (i == L - 1) break;
@@ -96,21 +112,21 @@ __global__ void __launch_bounds__(WARPS * 32) chain_small_kernel(ChainArgs<T> p)
 
         zero(w);
         gemm<0, 0, false>(w, sB, sS, g, t);          // W_i = B_i S_i^-1
+        from_smem_lower<T>(a, sD, g, t);             // D_{i+1}
         to_smem<T>(sW, w, g, t);
         __syncwarp();
 
-        a = dn;
         gemm<0, 1, true>(a, sW, sB, g, t);           // S_{i+1} = D_{i+1} - W_i B_i^T
 
         if (WANT_X) {                                 // y_{i+1} = r_{i+1} - W_i y_i
-            T s[2];
-            row_matvec<T>(s, w, sy + 16 * (i & 1), t);
+            T s2[2];
+            row_matvec<T>(s2, w, sy + 16 * (i & 1), t);
             if (t == 0) {
                 T *ynext = sy + 16 * ((i + 1) & 1);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int r = g + 8 * h;
-                    const T yv = rn[h] - s[h];
+                    const T yv = rn[h] - s2[h];
                     ynext[r] = yv;
                     if (r < b) X[(i + 1) * b + r] = yv;
                 }
@@ -119,10 +135,8 @@ __global__ void __launch_bounds__(WARPS * 32) chain_small_kernel(ChainArgs<T> p)
         __syncwarp();
         if (i + 1 < L - 1) {
             load_block_async<T, FULL>(sB, Bl + (i + 1) * bb, b, lane);
+            load_lower_async<T, FULL>(sD, D + (i + 2) * bb, b, lane);
             cp_async_commit();
-        }
-        if (i + 2 < L) {
-            load_sym<T, FULL>(dn, D + (i + 2) * bb, b, g, t);
             if (WANT_X && t == 0) {
                 rn[0] = g < b ? R[(i + 2) * b + g] : T(0);
                 rn[1] = g + 8 < b ? R[(i + 2) * b + g + 8] : T(0);
@@ -170,18 +184,18 @@ __global__ void __launch_bounds__(WARPS * 32) chain_small_kernel(ChainArgs<T> p)
             yp[1] = g + 8 < b ? X[(last - 1) * b + g + 8] : T(0);
         }
     }
-    Tile<T> pre;
     if (L > 1) {
         load_block_async<T, FULL>(sB, Bl + (L - 2) * bb, b, lane);
+        stage_lower_slot<T>(stg, ws + (L - 2) * SLOT_ELEMS, lane, g, t);
         cp_async_commit();
-        load_lower_slot<T>(pre, ws + (L - 2) * SLOT_ELEMS, lane, g, t);
     }
     __syncwarp();
 
     for (int64_t i = L - 2; i >= 0; --i) {
-        to_smem_sym<T>(sS, pre, g, t);               // S_i^-1, full and symmetric
         const T yi[2] = {yp[0], yp[1]};
         cp_async_wait_all();
+        unstage_lower_slot<T>(a, stg, lane, g, t);
+        to_smem_sym<T>(sS, a, g, t);                 // S_i^-1, full and symmetric
         __syncwarp();
 
         zero(w);
@@ -191,8 +205,8 @@ __global__ void __launch_bounds__(WARPS * 32) chain_small_kernel(ChainArgs<T> p)
         __syncwarp();
         if (i > 0) {
             load_block_async<T, FULL>(sB, Bl + (i - 1) * bb, b, lane);
+            stage_lower_slot<T>(stg, ws + (i - 1) * SLOT_ELEMS, lane, g, t);
             cp_async_commit();
-            load_lower_slot<T>(pre, ws + (i - 1) * SLOT_ELEMS, lane, g, t);
             if (WANT_X) {
                 yp[0] = g < b ? X[(i - 1) * b + g] : T(0);
                 yp[1] = g + 8 < b ? X[(i - 1) * b + g + 8] : T(0);
@@ -207,7 +221,7 @@ __global__ void __launch_bounds__(WARPS * 32) chain_small_kernel(ChainArgs<T> p)
             to_smem<T>(sS, gl, g, t);
             __syncwarp();
             Tile<T> gd = a;
-            gemm<1, 0, true>(gd, sW, sS, g, t);      // G_ii = S_i^-1 - W_i^T G_{i+1,i}
+            gemm<1, 0, true, true>(gd, sW, sS, g, t);   // G_ii = S_i^-1 - W_i^T G_{i+1,i} (lower tiles)
             to_smem_sym<T>(sG, gd, g, t);
             __syncwarp();
             from_smem<T>(gd, sG, g, t);

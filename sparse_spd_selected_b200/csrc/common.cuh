@@ -33,6 +33,20 @@ SELINV_DEVINL void dmma_8x8x4(double &d0, double &d1, double a, double b)
                  : "d"(a), "d"(b));
 }
 
+// Reciprocal of a positive normal d: the hardware approximation refined by one
+// cubic Newton-Raphson step, r <- r (1 + e + e^2) with e = 1 - d r, which
+// triples the number of correct bits of the estimate (about 20 -> full
+// precision).  Not for zero, negative, subnormal or non-finite d (the callers
+// flag such pivots as failures and do not use the result).
+SELINV_DEVINL double recip(double d)
+{
+    double r;
+    asm("rcp.approx.ftz.f64 %0, %1;\n" : "=d"(r) : "d"(d));
+    const double e = fma(-d, r, 1.0);
+    return fma(r, fma(e, e, e), r);
+}
+SELINV_DEVINL float recip(float d) { return __frcp_rn(d); }
+
 template <class T> SELINV_DEVINL T shfl(T v, int src) { return __shfl_sync(FULL_MASK, v, src); }
 template <class T> SELINV_DEVINL T shfl_xor(T v, int m) { return __shfl_xor_sync(FULL_MASK, v, m); }
 

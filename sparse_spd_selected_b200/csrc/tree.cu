@@ -42,7 +42,7 @@ namespace {
 
 constexpr int TWARPS = 4;
 
-template <class T> __host__ __device__ constexpr int tree_smem_elems() { return 4 * w16::SL<T>::ELEMS; }
+template <class T> __host__ __device__ constexpr int tree_smem_elems() { return 4 * w16::SL<T>::ELEMS + 64; }
 
 struct TreeDev {
     const int32_t *child_ptr;
@@ -72,7 +72,7 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, const int32_t *nodes, int64_t cou
     if (k >= count) return;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     T *sS = reinterpret_cast<T *>(smem_raw) + wid * tree_smem_elems<T>();
-    T *sW = sS + E, *sB = sW + E, *sT = sB + E;
+    T *sW = sS + E, *sB = sW + E, *sT = sB + E, *cb = sT + E;
 
     const int b = p.b;
     const int64_t bb = (int64_t)b * b;
@@ -109,7 +109,7 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, const int32_t *nodes, int64_t cou
     LogAcc det;
     det.init();
     bool bad = false;
-    spd_inverse<T>(a, lane, g, t, det, bad);
+    spd_inverse<T>(a, cb, g, t, det, bad);
     if (lane == 0) {
         p.ws_ld[v] = det.log_value();
         if (bad) atomicMin(p.info + v / td.n, (int32_t)(v % td.n));
@@ -136,7 +136,7 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, const int32_t *nodes, int64_t cou
     __syncwarp();
     Tile<T> u;
     zero(u);
-    gemm<0, 1, false>(u, sW, sB, g, t);           // U_v = W_v E_v^T
+    gemm<0, 1, false, true>(u, sW, sB, g, t);     // U_v = W_v E_v^T (lower tiles)
     store_lower_slot<T>(p.ws_u + (int64_t)v * SLOT_ELEMS, u, lane, g, t);
 }
 
@@ -178,7 +178,7 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, const int32_t *nodes, int64_t 
     store_block<T, FULL>(p.G_edge + v * bb, ge, b, g, t);
     to_smem<T>(sS, ge, g, t);
     __syncwarp();
-    gemm<1, 0, true>(a, sW, sS, g, t);            // G_vv = S_v^-1 - W_v^T G_edge[v]
+    gemm<1, 0, true, true>(a, sW, sS, g, t);      // G_vv = S_v^-1 - W_v^T G_edge[v] (lower tiles)
     __syncwarp();
     to_smem_sym<T>(sB, a, g, t);
     __syncwarp();

@@ -116,6 +116,39 @@ template <class T, bool FULL> SELINV_DEVINL void load_sym(Tile<T> &a, const T *D
         }
 }
 
+// Lower triangle of a diagonal block D (row-major b x b) into shared memory
+// (entries with c <= r; identity pad beyond b).  FULL: 16-byte cp.async
+// chunks that touch the lower triangle only (caller commits / waits).
+template <class T, bool FULL> SELINV_DEVINL void load_lower_async(T *s, const T *D, int b, int lane)
+{
+    if (FULL) {
+        constexpr int CH = 16 / sizeof(T);
+        constexpr int PER_ROW = 16 / CH;
+#pragma unroll
+        for (int j = lane; j < 16 * PER_ROW; j += 32) {
+            const int r = j / PER_ROW, c = (j % PER_ROW) * CH;
+            if (c <= r) cp_async16(s + SL<T>::idx(r, c), D + r * 16 + c);
+        }
+    } else {
+        for (int j = lane; j < 256; j += 32) {
+            const int r = j >> 4, c = j & 15;
+            if (c <= r) s[SL<T>::idx(r, c)] = (r < b && c < b) ? __ldg(D + r * b + c) : (r == c ? T(1) : T(0));
+        }
+    }
+}
+
+// Tile from a shared image of which only the lower triangle is valid.
+template <class T> SELINV_DEVINL void from_smem_lower(Tile<T> &a, const T *s, int g, int t)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = g + 8 * h, c = tcol(t, q);
+            a.v[h][q] = c <= r ? s[SL<T>::idx(r, c)] : s[SL<T>::idx(c, r)];
+        }
+}
+
 // Off-diagonal block (row-major b x b) into shared memory, zero pad beyond b.
 // FULL: 16-byte cp.async chunks (caller commits / waits); else plain loads.
 template <class T, bool FULL> SELINV_DEVINL void load_block_async(T *s, const T *B, int b, int lane)
@@ -201,11 +234,55 @@ template <class T> SELINV_DEVINL void load_lower_slot(Tile<T> &a, const T *slot,
     }
 }
 
+// The same slot copied to shared memory by each lane for itself (cp.async;
+// the caller commits / waits), then read back by the same lane.
+template <class T> SELINV_DEVINL void stage_lower_slot(T *stg, const T *slot, int lane, int g, int t)
+{
+    constexpr int CH = 16 / sizeof(T);          // elements per 16-byte chunk
+    if (CH == 2) {
+        cp_async16(stg + 2 * lane, slot + 2 * lane);
+        if (2 * t <= g) {
+            cp_async16(stg + 64 + 4 * lane, slot + 64 + 4 * lane);
+            cp_async16(stg + 64 + 4 * lane + 2, slot + 64 + 4 * lane + 2);
+        }
+    } else {                                    // float: 8-byte pairs, plain loads
+        *reinterpret_cast<typename Vec2<T>::type *>(stg + 2 * lane) =
+            *reinterpret_cast<const typename Vec2<T>::type *>(slot + 2 * lane);
+        if (2 * t <= g) {
+            *reinterpret_cast<typename Vec2<T>::type *>(stg + 64 + 4 * lane) =
+                *reinterpret_cast<const typename Vec2<T>::type *>(slot + 64 + 4 * lane);
+            *reinterpret_cast<typename Vec2<T>::type *>(stg + 64 + 4 * lane + 2) =
+                *reinterpret_cast<const typename Vec2<T>::type *>(slot + 64 + 4 * lane + 2);
+        }
+    }
+}
+
+template <class T> SELINV_DEVINL void unstage_lower_slot(Tile<T> &a, const T *stg, int lane, int g, int t)
+{
+    using V = typename Vec2<T>::type;
+    V v = *reinterpret_cast<const V *>(stg + 2 * lane);
+    a.v[1][0] = v.x;
+    a.v[1][1] = v.y;
+    a.v[0][2] = a.v[0][3] = T(0);
+    if (2 * t <= g) {
+        V u = *reinterpret_cast<const V *>(stg + 64 + 4 * lane);
+        V w = *reinterpret_cast<const V *>(stg + 64 + 4 * lane + 2);
+        a.v[0][0] = u.x;
+        a.v[0][1] = u.y;
+        a.v[1][2] = w.x;
+        a.v[1][3] = w.y;
+    } else {
+        a.v[0][0] = a.v[0][1] = a.v[1][2] = a.v[1][3] = T(0);
+    }
+}
+
 // ---- arithmetic --------------------------------------------------------------
 
 // acc += (NEG ? -1 : 1) * op(A) op(B), with A and B 16 x 16 in shared memory;
-// OPA / OPB = 1 means transposed.
-template <int OPA, int OPB, bool NEG>
+// OPA / OPB = 1 means transposed.  LOWER skips the upper-right 8 x 8 tile of
+// the result (rows 0..7, cols 8..15), for products known to be symmetric whose
+// upper triangle is rebuilt from the lower one afterwards.
+template <int OPA, int OPB, bool NEG, bool LOWER = false>
 SELINV_DEVINL void gemm(Tile<double> &acc, const double *sA, const double *sB, int g, int t)
 {
     using L = SL<double>;
@@ -223,11 +300,12 @@ SELINV_DEVINL void gemm(Tile<double> &acc, const double *sA, const double *sB, i
 #pragma unroll
         for (int m = 0; m < 2; ++m)
 #pragma unroll
-            for (int n = 0; n < 2; ++n) dmma_8x8x4(acc.v[m][2 * n], acc.v[m][2 * n + 1], a[m], b[n]);
+            for (int n = 0; n < 2; ++n)
+                if (!(LOWER && m == 0 && n == 1)) dmma_8x8x4(acc.v[m][2 * n], acc.v[m][2 * n + 1], a[m], b[n]);
     }
 }
 
-template <int OPA, int OPB, bool NEG>
+template <int OPA, int OPB, bool NEG, bool LOWER = false>
 SELINV_DEVINL void gemm(Tile<float> &acc, const float *sA, const float *sB, int g, int t)
 {
     using L = SL<float>;
@@ -254,39 +332,43 @@ SELINV_DEVINL void gemm(Tile<float> &acc, const float *sA, const float *sB, int 
 // A_kk = -1/d; after all k the tile holds -A^-1, which is negated.  The
 // pivots d are the successive Schur-complement pivots, so their product is
 // det A (multiplied into `det`); a pivot that is not > 0 sets `bad`.
+// Column k is broadcast through `cbuf` (2 x 16 elements of shared memory,
+// alternating per step so one __syncwarp per step suffices); row k is read
+// from the same buffer, the matrix being symmetric.
 template <class T>
-SELINV_DEVINL void spd_inverse(Tile<T> &a, int lane, int g, int t, LogAcc &det, bool &bad)
+SELINV_DEVINL void spd_inverse(Tile<T> &a, T *cbuf, int g, int t, LogAcc &det, bool &bad)
 {
+    using V = typename Vec2<T>::type;
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
-        const int kg = k & 7, kh = k >> 3, kt = (k & 7) >> 1, kq = (k & 1) | ((k >> 3) << 1);
-        const int src_col = (lane & ~3) | kt;     // owner of A[g + 8h][k]
-        const int src_row = (kg << 2) | t;        // owner of A[k][tcol(t, q)]
-        T col[2], row[4];
-        col[0] = shfl(a.v[0][kq], src_col);
-        col[1] = shfl(a.v[1][kq], src_col);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) row[q] = shfl(a.v[kh][q], src_row);
-        const T d = shfl(a.v[kh][kq], (kg << 2) | kt);
+        const int kh = k >> 3, kt = (k & 7) >> 1, kq = (k & 1) | ((k >> 3) << 1);
+        T *cb = cbuf + 16 * (k & 1);
+        if (t == kt) {                      // the 8 lanes owning column k publish it
+            cb[g] = a.v[0][kq];
+            cb[g + 8] = a.v[1][kq];
+        }
+        __syncwarp();
+        const T d = cb[k];
+        const T c0 = cb[g], c1 = cb[g + 8];
+        const V r01 = *reinterpret_cast<const V *>(cb + 2 * t);
+        const V r23 = *reinterpret_cast<const V *>(cb + 2 * t + 8);
+        const T row[4] = {r01.x, r01.y, r23.x, r23.y};
         bad |= !(d > T(0));
         det.mul((double)d);
-        const T p = T(1) / d;
-        T tc[2];
-        tc[0] = col[0] * p;
-        tc[1] = col[1] * p;
+        const T p = recip(d);
+        const T tc[2] = {c0 * p, c1 * p};
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
             for (int q = 0; q < 4; ++q) a.v[h][q] = fma(-tc[h], row[q], a.v[h][q]);
+        if (t == kt) {                      // column k: A_ik / d
+            a.v[0][kq] = tc[0];
+            a.v[1][kq] = tc[1];
+        }
+        if (g == (k & 7)) {                 // row k: A_kj / d, and A_kk = -1/d
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const bool in_row = (g + 8 * h) == k;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const bool in_col = (t == kt) && (q == kq);
-                if (in_row) a.v[h][q] = in_col ? -p : row[q] * p;
-                else if (in_col) a.v[h][q] = tc[h];
-            }
+            for (int q = 0; q < 4; ++q) a.v[kh][q] = row[q] * p;
+            if (t == kt) a.v[kh][kq] = -p;
         }
     }
 #pragma unroll

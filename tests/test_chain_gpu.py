@@ -205,3 +205,17 @@ def test_long_chains_full_size_sampled(cuda_ok, dtype):
     assert worst(host(out["G_diag"][pick]), ref["G_diag"]) <= tol
     assert worst(host(out["G_lower"][pick]), ref["G_lower"]) <= tol
     assert logdet_err(host(out["logdet"][pick]), ref["logdet"]) <= tol
+
+
+def test_pivot_reciprocal_against_cuda_division(cuda_ok):
+    """A 1 x 1 block's inverse is the kernel's pivot reciprocal (Newton-refined
+    hardware estimate): it must agree with CUDA's IEEE division to a few ulp
+    over a wide range of magnitudes, and log det with log."""
+    rng = np.random.default_rng(123)
+    d = np.exp(rng.uniform(-40.0, 40.0, size=200_000))
+    dev = torch.from_numpy(d).cuda().reshape(-1, 1, 1, 1)
+    out = selinv.selinv_chain(dev, None)
+    ref = 1.0 / dev
+    ulp = torch.abs(out["G_diag"] - ref) / (torch.finfo(torch.float64).eps * torch.abs(ref))
+    assert float(ulp.max()) <= 4.0
+    assert float(torch.max(torch.abs(out["logdet"] - torch.log(dev.reshape(-1))))) <= 1e-12
