@@ -12,7 +12,9 @@
 //   W_i = B_i S_i^-1,  S_{i+1} = D_{i+1} - W_i B_i^T          (collect)
 //   G_{i+1,i} = -G_{i+1,i+1} W_i,  G_ii = S_i^-1 - W_i^T G_{i+1,i}  (distribute)
 // (G_ii = S_i^-1 - S_i^-1 B_i^T G_{i+1,i} with S_i^-1 B_i^T = W_i^T).  The
-// products run on the FP64 tensor cores (m8n8k4) from shared memory.
+// products run on the FP64 tensor cores (m8n8k4) straight from registers;
+// only W_i and G_{i+1,i} pass through shared memory once each, to be
+// transposed.
 // Between the sweeps only the lower triangle of each S_i^-1 is kept, in the
 // caller's workspace; W_i is recomputed from B_i in the distribute sweep,
 // which moves fewer bytes than storing it.
@@ -48,12 +50,11 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
 
     extern __shared__ __align__(16) unsigned char smem_raw[];
     T *sbase = reinterpret_cast<T *>(smem_raw) + wid * warp_smem_elems<T>();
-    T *sS = sbase;             // S_i^-1 (operand), later G_{i+1,i}
-    T *sW = sS + E;            // W_i
-    T *sB = sW + E;            // B_i
-    T *sD = sB + E;            // D_{i+1} (lower triangle); G_{i+1,i+1} in the distribute sweep
-    T *sG = sD;
-    T *stg = sD + E;           // staged S_i^-1 slot (distribute sweep)
+    T *sB = sbase;             // B_i
+    T *sD = sB + E;            // D_{i+1} (lower triangle)
+    T *sT = sD + E;            // transposes / mirrors
+    T *sT2 = sT + E;           // second transpose buffer
+    T *stg = sT2 + E;          // staged S_i^-1 slot (distribute sweep)
     T *sy = stg + SLOT_ELEMS;  // y vectors, two buffers of 16
     T *sx = sy + 32;           // x vectors, two buffers of 16
     T *cb = sx + 32;           // pivot-column broadcast, two buffers of 16
@@ -71,7 +72,7 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
     det.init();
     int fail = -1;
 
-    Tile<T> a, w;
+    Tile<T> a, w, bt;
     load_lower_async<T, FULL>(sD, D, b, lane);
     cp_async_commit();
     cp_async_wait_all();
@@ -100,23 +101,21 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
     // ---------------- collect sweep ----------------
     for (int64_t i = 0; i < L; ++i) {
         bool bad = false;
-        spd_inverse<T>(a, cb, g, t, det, bad);
+        spd_inverse<T>(a, cb, g, t, det, bad);        // a = S_i^-1
         det.renorm();
         if (bad && fail < 0) fail = (int)i;
         if (i == L - 1) break;
 
         if (WANT_G || WANT_X) store_lower_slot<T>(ws + i * SLOT_ELEMS, a, lane, g, t);
-        to_smem<T>(sS, a, g, t);
         cp_async_wait_all();
         __syncwarp();
-
+        from_smem<T>(bt, sB, g, t);                   // B_i
+        Tile<T> dn;
+        from_smem_lower<T>(dn, sD, g, t);             // D_{i+1}
         zero(w);
-        gemm<0, 0, false>(w, sB, sS, g, t);          // W_i = B_i S_i^-1
-        from_smem_lower<T>(a, sD, g, t);             // D_{i+1}
-        to_smem<T>(sW, w, g, t);
-        __syncwarp();
-
-        gemm<0, 1, true>(a, sW, sB, g, t);           // S_{i+1} = D_{i+1} - W_i B_i^T
+        gemm_nt<false>(w, bt, a, sT, sT2, g, t);      // W_i = B_i S_i^-1  (S_i^-1 symmetric)
+        gemm_nt<true>(dn, w, bt, sT, sT2, g, t);      // S_{i+1} = D_{i+1} - W_i B_i^T
+        a = dn;
 
         if (WANT_X) {                                 // y_{i+1} = r_{i+1} - W_i y_i
             T s2[2];
@@ -150,12 +149,13 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
     if (!(WANT_G || WANT_X)) return;
 
     // ---------------- distribute sweep ----------------
-    // a = S_{L-1}^-1 = G_{L-1,L-1}; make it exactly symmetric.
+    // G = S_{L-1}^-1 = G_{L-1,L-1}, made exactly symmetric; kept in registers.
+    Tile<T> G;
     __syncwarp();
-    to_smem_sym<T>(sG, a, g, t);
+    to_smem<T>(sT, a, g, t);
     __syncwarp();
-    from_smem<T>(a, sG, g, t);
-    if (WANT_G) store_block<T, FULL>(p.G_diag + e * L * bb + (L - 1) * bb, a, b, g, t);
+    from_smem_lower<T>(G, sT, g, t);
+    if (WANT_G) store_block<T, FULL>(p.G_diag + e * L * bb + (L - 1) * bb, G, b, g, t);
 
     const int64_t last = L - 1;
     T yp[2] = {T(0), T(0)};     // y_i at rows g, g+8
@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
         const T *y = sy + 16 * (last & 1);
         T part[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) part[q] = a.v[0][q] * y[g] + a.v[1][q] * y[g + 8];
+        for (int q = 0; q < 4; ++q) part[q] = G.v[0][q] * y[g] + G.v[1][q] * y[g + 8];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             part[q] += shfl_xor(part[q], 4);
@@ -184,24 +184,21 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
             yp[1] = g + 8 < b ? X[(last - 1) * b + g + 8] : T(0);
         }
     }
+    __syncwarp();
     if (L > 1) {
         load_block_async<T, FULL>(sB, Bl + (L - 2) * bb, b, lane);
         stage_lower_slot<T>(stg, ws + (L - 2) * SLOT_ELEMS, lane, g, t);
         cp_async_commit();
     }
-    __syncwarp();
 
     for (int64_t i = L - 2; i >= 0; --i) {
         const T yi[2] = {yp[0], yp[1]};
         cp_async_wait_all();
         unstage_lower_slot<T>(a, stg, lane, g, t);
-        to_smem_sym<T>(sS, a, g, t);                 // S_i^-1, full and symmetric
+        to_smem<T>(sT, a, g, t);                      // lower entries valid
         __syncwarp();
-
-        zero(w);
-        gemm<0, 0, false>(w, sB, sS, g, t);          // W_i = B_i S_i^-1
-        from_smem<T>(a, sS, g, t);                   // S_i^-1 in registers
-        to_smem<T>(sW, w, g, t);
+        from_smem_lower<T>(a, sT, g, t);              // S_i^-1, full and symmetric
+        from_smem<T>(bt, sB, g, t);                   // B_i
         __syncwarp();
         if (i > 0) {
             load_block_async<T, FULL>(sB, Bl + (i - 1) * bb, b, lane);
@@ -212,21 +209,9 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
                 yp[1] = g + 8 < b ? X[(i - 1) * b + g + 8] : T(0);
             }
         }
+        zero(w);
+        gemm_nt<false>(w, bt, a, sT, sT2, g, t);      // W_i = B_i S_i^-1
 
-        if (WANT_G) {
-            Tile<T> gl;
-            zero(gl);
-            gemm<0, 0, true>(gl, sG, sW, g, t);      // G_{i+1,i} = -G_{i+1,i+1} W_i
-            store_block<T, FULL>(p.G_lower + e * (L - 1) * bb + i * bb, gl, b, g, t);
-            to_smem<T>(sS, gl, g, t);
-            __syncwarp();
-            Tile<T> gd = a;
-            gemm<1, 0, true, true>(gd, sW, sS, g, t);   // G_ii = S_i^-1 - W_i^T G_{i+1,i} (lower tiles)
-            to_smem_sym<T>(sG, gd, g, t);
-            __syncwarp();
-            from_smem<T>(gd, sG, g, t);
-            store_block<T, FULL>(p.G_diag + e * L * bb + i * bb, gd, b, g, t);
-        }
         if (WANT_X) {                                 // x_i = S_i^-1 y_i - W_i^T x_{i+1}
             const T *xn = sx + 16 * ((i + 1) & 1);
             const T x0 = xn[g], x1 = xn[g + 8];
@@ -249,6 +234,26 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
                     if (c < b) X[i * b + c] = part[q];
                 }
             }
+        }
+        if (WANT_G) {
+            Tile<T> wt, gl, glt;
+            __syncwarp();
+            to_smem<T>(sT, w, g, t);
+            __syncwarp();
+            from_smem_T<T>(wt, sT, g, t);             // W_i^T
+            zero(gl);
+            gemm_nt<true>(gl, G, wt, sT, sT2, g, t);  // G_{i+1,i} = -G_{i+1,i+1} W_i
+            store_block<T, FULL>(p.G_lower + e * (L - 1) * bb + i * bb, gl, b, g, t);
+            __syncwarp();
+            to_smem<T>(sT2, gl, g, t);
+            __syncwarp();
+            from_smem_T<T>(glt, sT2, g, t);           // G_{i+1,i}^T
+            gemm_nt<true, true>(a, wt, glt, sT, sT2, g, t);   // G_ii = S_i^-1 - W_i^T G_{i+1,i} (lower tiles)
+            __syncwarp();
+            to_smem<T>(sT, a, g, t);
+            __syncwarp();
+            from_smem_lower<T>(G, sT, g, t);          // exactly symmetric G_ii, next step's G_{i+1,i+1}
+            store_block<T, FULL>(p.G_diag + e * L * bb + i * bb, G, b, g, t);
         }
         __syncwarp();
     }

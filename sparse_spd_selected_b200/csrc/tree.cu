@@ -1,13 +1,20 @@
-// Block trees: plan (host) and level-set kernels (b <= 16, one warp per node).
+// Block trees: plan (host) and the collect / distribute kernels (b <= 16,
+// one warp per node at a time).
 //
 // gabp-sparse-inv 0.3.2 (PyPI page), "Implemented and tested kernels" ->
 // Tree: a parent array and one edge block per non-root node,
 // edge[v] = A_{parent(v), v}; collect from the leaves to the root, then
-// distribute from the root to the leaves.  The level-set batching follows the
-// package's batched path ("General sparse selected inverse": one batched step
-// per elimination level instead of per node): every node of one height is
-// independent in the collect sweep, every node of one depth in the distribute
-// sweep, so each level is one kernel launch over all trees of the batch.
+// distribute from the root to the leaves.  The package batches its tree
+// kernel by elimination level ("General sparse selected inverse": one batched
+// step per level instead of per node).  Here the level sets order the work
+// but do not separate launches: one launch per sweep over the whole forest.
+//  * collect: warps take leaves; a warp that finishes a node and is the last
+//    of its parent's children to do so (an atomic count) goes on with the
+//    parent, so no warp ever waits;
+//  * distribute: warps take non-root nodes in depth order and wait (bounded)
+//    for their parent's diagonal block to be published; a parent is always
+//    taken before its children by a warp that is already running, so every
+//    wait ends.
 //
 // Collect, node v (all children already done):
 //   S_v = D_v - sum_{c in ch(v)} U_c,        U_c = E_c S_c^-1 E_c^T
@@ -60,136 +67,225 @@ template <class T> struct TreeBufs {
     int b;
 };
 
+struct TreeSync {
+    int32_t *pending;     // [N] children of a node not collected yet
+    int32_t *done;        // [N] 1 once G_vv is written (distribute)
+    unsigned long long *counters;   // [0] leaves taken, [1] distribute nodes taken
+};
+
+constexpr int SPIN_LIMIT = 1 << 22;     // x >= 64 ns per poll: well over a second
+
+SELINV_DEVINL unsigned long long warp_take(unsigned long long *ctr, int lane)
+{
+    unsigned long long k = 0;
+    if (lane == 0) k = atomicAdd(ctr, 1ull);
+    return __shfl_sync(FULL_MASK, k, 0);
+}
+
+SELINV_DEVINL int ld_acquire(const int32_t *p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+SELINV_DEVINL void st_release(int32_t *p, int v)
+{
+    asm volatile("st.release.gpu.global.s32 [%0], %1;\n" ::"l"(p), "r"(v) : "memory");
+}
+
+template <class T> SELINV_DEVINL void load_lower_slot_l2(w16::Tile<T> &a, const T *slot, int lane, int g, int t)
+{
+    using V = typename w16::Vec2<T>::type;
+    V v = __ldcg(reinterpret_cast<const V *>(slot + 2 * lane));
+    a.v[1][0] = v.x;
+    a.v[1][1] = v.y;
+    a.v[0][2] = a.v[0][3] = T(0);
+    if (2 * t <= g) {
+        V u = __ldcg(reinterpret_cast<const V *>(slot + 64 + 4 * lane));
+        V w = __ldcg(reinterpret_cast<const V *>(slot + 64 + 4 * lane + 2));
+        a.v[0][0] = u.x;
+        a.v[0][1] = u.y;
+        a.v[1][2] = w.x;
+        a.v[1][3] = w.y;
+    } else {
+        a.v[0][0] = a.v[0][1] = a.v[1][2] = a.v[1][3] = T(0);
+    }
+}
+
 template <class T, bool FULL>
 __global__ void __launch_bounds__(TWARPS * 32)
-tree_collect_kernel(TreeBufs<T> p, TreeDev td, const int32_t *nodes, int64_t count)
+tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leaves, int64_t nleaves)
 {
     using namespace w16;
     constexpr int E = SL<T>::ELEMS;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
-    const int64_t k = (int64_t)blockIdx.x * TWARPS + wid;
-    if (k >= count) return;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    T *sS = reinterpret_cast<T *>(smem_raw) + wid * tree_smem_elems<T>();
-    T *sW = sS + E, *sB = sW + E, *sT = sB + E, *cb = sT + E;
-
+    T *sB = reinterpret_cast<T *>(smem_raw) + wid * tree_smem_elems<T>();
+    T *sD = sB + E, *sT = sD + E, *sT2 = sT + E, *cb = sT2 + E;
     const int b = p.b;
     const int64_t bb = (int64_t)b * b;
-    const int32_t v = nodes[k];
-    const int32_t par = td.parent[v];
-    if (par >= 0) {                               // E_v -> shared memory, early
-        load_block_async<T, FULL>(sB, p.edge + v * bb, b, lane);
-        cp_async_commit();
-    }
-    Tile<T> a;
-    load_sym<T, FULL>(a, p.diag + v * bb, b, g, t);
 
-    // sum of the children's U_c (lower slots), then mirrored once
-    const int32_t c0 = td.child_ptr[v], c1 = td.child_ptr[v + 1];
-    if (c1 > c0) {
-        Tile<T> acc, u;
-        zero(acc);
-        for (int32_t c = c0; c < c1; ++c) {
-            load_lower_slot<T>(u, p.ws_u + (int64_t)td.child_idx[c] * SLOT_ELEMS, lane, g, t);
+    for (;;) {
+        const unsigned long long k = warp_take(sy.counters, lane);
+        if (k >= (unsigned long long)nleaves) break;
+        int32_t v = leaves[k];
+        for (;;) {                                   // v, then each parent this warp completes last
+            const int32_t par = td.parent[v];
+            if (par >= 0) load_block_async<T, FULL>(sB, p.edge + v * bb, b, lane);   // E_v
+            load_lower_async<T, FULL>(sD, p.diag + v * bb, b, lane);                 // D_v
+            cp_async_commit();
+            Tile<T> acc;                              // sum of the children's U_c (lower slots)
+            zero(acc);
+            const int32_t c0 = td.child_ptr[v], c1 = td.child_ptr[v + 1];
+            for (int32_t c = c0; c < c1; ++c) {
+                Tile<T> u;
+                load_lower_slot_l2<T>(u, p.ws_u + (int64_t)td.child_idx[c] * SLOT_ELEMS, lane, g, t);
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+                for (int h = 0; h < 2; ++h)
 #pragma unroll
-                for (int q = 0; q < 4; ++q) acc.v[h][q] += u.v[h][q];
+                    for (int q = 0; q < 4; ++q) acc.v[h][q] += u.v[h][q];
+            }
+            cp_async_wait_all();
+            __syncwarp();
+            Tile<T> a;
+            from_smem_lower<T>(a, sD, g, t);
+            if (c1 > c0) {                            // S_v = D_v - sum U_c (mirrored from the lower slots)
+                to_smem<T>(sT, acc, g, t);
+                __syncwarp();
+                from_smem_lower<T>(acc, sT, g, t);
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) a.v[h][q] -= acc.v[h][q];
+            }
+            LogAcc det;
+            det.init();
+            bool bad = false;
+            spd_inverse<T>(a, cb, g, t, det, bad);
+            if (lane == 0) {
+                p.ws_ld[v] = det.log_value();
+                if (bad) atomicMin(p.info + v / td.n, (int32_t)(v % td.n));
+            }
+            if (par < 0) {                            // root: G = S^-1, G_edge = 0, published
+                __syncwarp();
+                to_smem<T>(sT, a, g, t);
+                __syncwarp();
+                from_smem_lower<T>(a, sT, g, t);
+                store_block<T, FULL>(p.G_diag + v * bb, a, b, g, t);
+                Tile<T> z;
+                zero(z);
+                store_block<T, FULL>(p.G_edge + v * bb, z, b, g, t);
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) st_release(sy.done + v, 1);
+                __syncwarp();
+                break;
+            }
+            store_lower_slot<T>(p.ws_sinv + (int64_t)v * SLOT_ELEMS, a, lane, g, t);
+            Tile<T> et, w, u;
+            from_smem<T>(et, sB, g, t);               // E_v
+            zero(w);
+            gemm_nt<false>(w, et, a, sT, sT2, g, t);  // W_v = E_v S_v^-1
+            zero(u);
+            gemm_nt<false, true>(u, w, et, sT, sT2, g, t);   // U_v = W_v E_v^T (lower tiles)
+            store_lower_slot<T>(p.ws_u + (int64_t)v * SLOT_ELEMS, u, lane, g, t);
+            __threadfence();                          // U_v visible before the count drops
+            __syncwarp();
+            int old = 0;
+            if (lane == 0) old = atomicSub(sy.pending + par, 1);
+            old = __shfl_sync(FULL_MASK, old, 0);
+            if (old != 1) break;                      // a sibling is still running: it will go on
+            __threadfence();                          // see every sibling's U
+            v = par;
         }
-        to_smem_sym<T>(sT, acc, g, t);
-        __syncwarp();
-        from_smem<T>(acc, sT, g, t);
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) a.v[h][q] -= acc.v[h][q];
     }
-
-    LogAcc det;
-    det.init();
-    bool bad = false;
-    spd_inverse<T>(a, cb, g, t, det, bad);
-    if (lane == 0) {
-        p.ws_ld[v] = det.log_value();
-        if (bad) atomicMin(p.info + v / td.n, (int32_t)(v % td.n));
-    }
-    if (par < 0) {                                // root: G = S^-1, G_edge = 0
-        __syncwarp();
-        to_smem_sym<T>(sT, a, g, t);
-        __syncwarp();
-        from_smem<T>(a, sT, g, t);
-        store_block<T, FULL>(p.G_diag + v * bb, a, b, g, t);
-        Tile<T> z;
-        zero(z);
-        store_block<T, FULL>(p.G_edge + v * bb, z, b, g, t);
-        return;
-    }
-    store_lower_slot<T>(p.ws_sinv + (int64_t)v * SLOT_ELEMS, a, lane, g, t);
-    to_smem<T>(sS, a, g, t);
-    cp_async_wait_all();
-    __syncwarp();
-    Tile<T> w;
-    zero(w);
-    gemm<0, 0, false>(w, sB, sS, g, t);           // W_v = E_v S_v^-1
-    to_smem<T>(sW, w, g, t);
-    __syncwarp();
-    Tile<T> u;
-    zero(u);
-    gemm<0, 1, false, true>(u, sW, sB, g, t);     // U_v = W_v E_v^T (lower tiles)
-    store_lower_slot<T>(p.ws_u + (int64_t)v * SLOT_ELEMS, u, lane, g, t);
 }
 
 template <class T, bool FULL>
 __global__ void __launch_bounds__(TWARPS * 32)
-tree_distribute_kernel(TreeBufs<T> p, TreeDev td, const int32_t *nodes, int64_t count)
+tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *nodes, int64_t count)
 {
     using namespace w16;
     constexpr int E = SL<T>::ELEMS;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
-    const int64_t k = (int64_t)blockIdx.x * TWARPS + wid;
-    if (k >= count) return;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    T *sS = reinterpret_cast<T *>(smem_raw) + wid * tree_smem_elems<T>();
-    T *sW = sS + E, *sB = sW + E, *sG = sB + E;
-
+    T *sB = reinterpret_cast<T *>(smem_raw) + wid * tree_smem_elems<T>();
+    T *sG = sB + E, *sT = sG + E, *sT2 = sT + E;
     const int b = p.b;
     const int64_t bb = (int64_t)b * b;
-    const int32_t v = nodes[k];
-    const int32_t par = td.parent[v];
-    load_block_async<T, FULL>(sB, p.edge + v * bb, b, lane);
-    load_block_async<T, FULL>(sG, p.G_diag + (int64_t)par * bb, b, lane);   // G_pp (symmetric)
-    cp_async_commit();
-    Tile<T> a;
-    load_lower_slot<T>(a, p.ws_sinv + (int64_t)v * SLOT_ELEMS, lane, g, t);
-    to_smem_sym<T>(sS, a, g, t);
-    cp_async_wait_all();
-    __syncwarp();
-    Tile<T> w;
-    zero(w);
-    gemm<0, 0, false>(w, sB, sS, g, t);           // W_v = E_v S_v^-1
-    from_smem<T>(a, sS, g, t);
-    to_smem<T>(sW, w, g, t);
-    __syncwarp();
-    Tile<T> ge;
-    zero(ge);
-    gemm<0, 0, true>(ge, sG, sW, g, t);           // G_edge[v] = -G_pp W_v
-    store_block<T, FULL>(p.G_edge + v * bb, ge, b, g, t);
-    to_smem<T>(sS, ge, g, t);
-    __syncwarp();
-    gemm<1, 0, true, true>(a, sW, sS, g, t);      // G_vv = S_v^-1 - W_v^T G_edge[v] (lower tiles)
-    __syncwarp();
-    to_smem_sym<T>(sB, a, g, t);
-    __syncwarp();
-    from_smem<T>(a, sB, g, t);
-    store_block<T, FULL>(p.G_diag + v * bb, a, b, g, t);
+
+    for (;;) {
+        const unsigned long long k = warp_take(sy.counters + 1, lane);
+        if (k >= (unsigned long long)count) break;
+        const int32_t v = nodes[k];
+        const int32_t par = td.parent[v];
+        load_block_async<T, FULL>(sB, p.edge + v * bb, b, lane);          // E_v
+        cp_async_commit();
+        Tile<T> a;
+        load_lower_slot<T>(a, p.ws_sinv + (int64_t)v * SLOT_ELEMS, lane, g, t);
+        int ok = 1;                                   // wait for G_pp (bounded)
+        if (lane == 0) {
+            int n = 0;
+            while (ld_acquire(sy.done + par) == 0) {
+                if (++n > SPIN_LIMIT) { ok = 0; break; }
+                __nanosleep(64);
+            }
+        }
+        ok = __shfl_sync(FULL_MASK, ok, 0);
+        if (!ok) {                                    // cannot happen for a valid plan: report, move on
+            cp_async_wait_all();
+            if (lane == 0) atomicMin(p.info + v / td.n, -2);
+            continue;
+        }
+        __threadfence();
+        load_lower_async<T, FULL>(sG, p.G_diag + (int64_t)par * bb, b, lane);   // G_pp (lower), from L2
+        cp_async_commit();
+        to_smem<T>(sT, a, g, t);                      // lower entries of S_v^-1 valid
+        cp_async_wait_all();
+        __syncwarp();
+        from_smem_lower<T>(a, sT, g, t);              // S_v^-1, full
+        Tile<T> gp, et, w, wt, ge, get;
+        from_smem_lower<T>(gp, sG, g, t);             // G_pp, full
+        from_smem<T>(et, sB, g, t);                   // E_v
+        zero(w);
+        gemm_nt<false>(w, et, a, sT, sT2, g, t);      // W_v = E_v S_v^-1
+        __syncwarp();
+        to_smem<T>(sT, w, g, t);
+        __syncwarp();
+        from_smem_T<T>(wt, sT, g, t);                 // W_v^T
+        zero(ge);
+        gemm_nt<true>(ge, gp, wt, sT, sT2, g, t);     // G_edge[v] = -G_pp W_v
+        store_block<T, FULL>(p.G_edge + v * bb, ge, b, g, t);
+        __syncwarp();
+        to_smem<T>(sT2, ge, g, t);
+        __syncwarp();
+        from_smem_T<T>(get, sT2, g, t);               // G_edge[v]^T
+        gemm_nt<true, true>(a, wt, get, sT, sT2, g, t);   // G_vv = S_v^-1 - W_v^T G_edge[v] (lower tiles)
+        __syncwarp();
+        to_smem<T>(sT, a, g, t);
+        __syncwarp();
+        from_smem_lower<T>(a, sT, g, t);              // exactly symmetric
+        store_block<T, FULL>(p.G_diag + v * bb, a, b, g, t);
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) st_release(sy.done + v, 1);
+        __syncwarp();
+    }
 }
 
-__global__ void tree_info_init(int32_t *info, int64_t trees)
+__global__ void tree_init(const int32_t *child_ptr, int64_t N, int32_t *pending, int32_t *done,
+                          unsigned long long *counters, int32_t *info, int64_t trees)
 {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < N) {
+        pending[i] = child_ptr[i + 1] - child_ptr[i];
+        done[i] = 0;
+    }
     if (i < trees) info[i] = INT_MAX;
+    if (i < 2) counters[i] = 0;
 }
 
 // log det per tree = sum of its nodes' log det S_v in a fixed order
@@ -232,26 +328,37 @@ cudaError_t run_tree(const selinv_tree_plan_s *pl, int b, const T *diag, const T
     p.ws_u = reinterpret_cast<T *>(w);
     w += align256(N * slot_bytes<T>());
     p.ws_ld = reinterpret_cast<double *>(w);
+    w += align256(N * sizeof(double));
+    TreeSync sy;
+    sy.pending = reinterpret_cast<int32_t *>(w);
+    w += align256(N * sizeof(int32_t));
+    sy.done = reinterpret_cast<int32_t *>(w);
+    w += align256(N * sizeof(int32_t));
+    sy.counters = reinterpret_cast<unsigned long long *>(w);
     p.info = info;
     p.b = b;
     TreeDev td{pl->d_child_ptr, pl->d_child_idx, pl->d_parent, pl->n};
 
-    tree_info_init<<<(unsigned)ceil_div(pl->trees, 256), 256, 0, s>>>(info, pl->trees);
+    const int64_t init_n = std::max<int64_t>(N, pl->trees);
+    tree_init<<<(unsigned)ceil_div(init_n, 256), 256, 0, s>>>(pl->d_child_ptr, N, sy.pending, sy.done, sy.counters,
+                                                               info, pl->trees);
     const size_t smem = sizeof(T) * tree_smem_elems<T>() * TWARPS;
     auto kc = full ? tree_collect_kernel<T, true> : tree_collect_kernel<T, false>;
     auto kd = full ? tree_distribute_kernel<T, true> : tree_distribute_kernel<T, false>;
     cudaError_t err = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err == cudaSuccess) err = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    for (size_t h = 0; h + 1 < pl->collect_off.size(); ++h) {
-        const int64_t cnt = pl->collect_off[h + 1] - pl->collect_off[h];
-        if (cnt == 0) continue;
-        kc<<<(unsigned)ceil_div(cnt, TWARPS), TWARPS * 32, smem, s>>>(p, td, pl->d_collect_nodes + pl->collect_off[h], cnt);
-    }
-    for (size_t d = 0; d + 1 < pl->dist_off.size(); ++d) {
-        const int64_t cnt = pl->dist_off[d + 1] - pl->dist_off[d];
-        if (cnt == 0) continue;
-        kd<<<(unsigned)ceil_div(cnt, TWARPS), TWARPS * 32, smem, s>>>(p, td, pl->d_dist_nodes + pl->dist_off[d], cnt);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t max_blocks = (int64_t)sms * 4;      // about one resident wave of warps
+    const int64_t nleaves = pl->collect_off.size() > 1 ? pl->collect_off[1] - pl->collect_off[0] : 0;
+    const int64_t ndist = pl->dist_off.empty() ? 0 : pl->dist_off.back();
+    const int64_t bc = std::min<int64_t>(max_blocks, std::max<int64_t>(1, ceil_div(nleaves, TWARPS)));
+    kc<<<(unsigned)bc, TWARPS * 32, smem, s>>>(p, td, sy, pl->d_collect_nodes, nleaves);
+    if (ndist > 0) {
+        const int64_t bd = std::min<int64_t>(max_blocks, ceil_div(ndist, TWARPS));
+        kd<<<(unsigned)bd, TWARPS * 32, smem, s>>>(p, td, sy, pl->d_dist_nodes, ndist);
     }
     tree_finalize<<<(unsigned)pl->trees, 256, 0, s>>>(p.ws_ld, pl->n, logdet, info);
     return cudaGetLastError();
@@ -264,7 +371,8 @@ bool is_aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p
 size_t tree_workspace(const selinv_tree_plan_s *pl, size_t elem)
 {
     const int64_t N = pl->trees * pl->n;
-    return 2 * align256((size_t)N * elem * w16::SLOT_ELEMS) + align256((size_t)N * sizeof(double));
+    return 2 * align256((size_t)N * elem * w16::SLOT_ELEMS) + align256((size_t)N * sizeof(double)) +
+           2 * align256((size_t)N * sizeof(int32_t)) + 256;
 }
 
 }  // namespace selinv

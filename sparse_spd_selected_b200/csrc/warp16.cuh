@@ -21,10 +21,11 @@ template <class T> struct Tile {
 SELINV_DEVINL int tcol(int t, int q) { return 2 * t + (q & 1) + 8 * (q >> 1); }
 
 // Shared-memory image of a 16 x 16 block.
-//  double: 16 doubles per row (8 chunks of 16 B) with chunk index XOR f(r),
-//          f(r) = ((r & 1) << 2) | ((r >> 1) & 3).  Conflict-free for the
-//          tensor-core fragment reads (8 rows x 4 columns and 4 rows x 8
-//          columns) and for the tile's own 16-byte pair accesses.
+//  double: 16 doubles per row (8 chunks of 16 B); the chunk index is XORed
+//          with f(r) = 4 ((r ^ (r >> 1)) & 1), which puts rows 2j and 2j+1 in
+//          opposite halves of the banks (conflict-free 16-byte pair accesses
+//          of the register tile) and splits every set of rows {j, j+2, j+4,
+//          j+6} two and two (transposed reads of a tile in two wavefronts).
 //  float:  row pitch 20 floats (8-byte pairs stay aligned; column reads of 8
 //          rows hit distinct banks).
 template <class T> struct SL;
@@ -32,7 +33,7 @@ template <> struct SL<double> {
     static constexpr int ELEMS = 256;
     SELINV_DEVINL static int idx(int r, int c)
     {
-        const int f = ((r & 1) << 2) | ((r >> 1) & 3);
+        const int f = ((r ^ (r >> 1)) & 1) << 2;
         return (r << 4) | ((((c >> 1) ^ f) << 1) | (c & 1));
     }
 };
@@ -278,52 +279,63 @@ template <class T> SELINV_DEVINL void unstage_lower_slot(Tile<T> &a, const T *st
 
 // ---- arithmetic --------------------------------------------------------------
 
-// acc += (NEG ? -1 : 1) * op(A) op(B), with A and B 16 x 16 in shared memory;
-// OPA / OPB = 1 means transposed.  LOWER skips the upper-right 8 x 8 tile of
-// the result (rows 0..7, cols 8..15), for products known to be symmetric whose
-// upper triangle is rebuilt from the lower one afterwards.
-template <int OPA, int OPB, bool NEG, bool LOWER = false>
-SELINV_DEVINL void gemm(Tile<double> &acc, const double *sA, const double *sB, int g, int t)
+// Transposed copy of a tile: out[r][c] = in[c][r], through the shared image s
+// (the caller makes s free before and syncs before reusing it).
+template <class T> SELINV_DEVINL void from_smem_T(Tile<T> &a, const T *s, int g, int t)
 {
-    using L = SL<double>;
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-        double a[2], b[2];
+    for (int h = 0; h < 2; ++h)
 #pragma unroll
-        for (int m = 0; m < 2; ++m) {
-            a[m] = OPA == 0 ? sA[L::idx(8 * m + g, 4 * kk + t)] : sA[L::idx(4 * kk + t, 8 * m + g)];
-            if (NEG) a[m] = -a[m];
-        }
+        for (int q = 0; q < 4; ++q) a.v[h][q] = s[SL<T>::idx(tcol(t, q), g + 8 * h)];
+}
+
+// acc += (NEG ? -1 : 1) X Y^T for register tiles X, Y (16 x 16).
+//
+// double: the FP64 tensor cores.  Each m8n8k4 step s = 0..3 lets lane t carry
+// k = 2t, 2t+1, 8+2t, 9+2t respectively (any assignment of the k index that
+// both operands share gives the same sum), so the A fragment of row tile m is
+// the lane's own X.v[m][s] and the B fragment of column tile n is Y.v[n][s]:
+// no data movement at all.  LOWER skips the upper-right 8 x 8 tile of the
+// result (products known to be symmetric, rebuilt from the lower half).
+// float: plain FMAs from shared copies of X and Y (sX, sY: two free 16 x 16
+// images), X and Y written there first.
+template <bool NEG, bool LOWER = false>
+SELINV_DEVINL void gemm_nt(Tile<double> &acc, const Tile<double> &X, const Tile<double> &Y, double *, double *,
+                           int, int)
+{
 #pragma unroll
-        for (int n = 0; n < 2; ++n)
-            b[n] = OPB == 0 ? sB[L::idx(4 * kk + t, 8 * n + g)] : sB[L::idx(8 * n + g, 4 * kk + t)];
-#pragma unroll
-        for (int m = 0; m < 2; ++m)
-#pragma unroll
-            for (int n = 0; n < 2; ++n)
-                if (!(LOWER && m == 0 && n == 1)) dmma_8x8x4(acc.v[m][2 * n], acc.v[m][2 * n + 1], a[m], b[n]);
+    for (int st = 0; st < 4; ++st) {
+        const double a0 = NEG ? -X.v[0][st] : X.v[0][st];
+        const double a1 = NEG ? -X.v[1][st] : X.v[1][st];
+        dmma_8x8x4(acc.v[0][0], acc.v[0][1], a0, Y.v[0][st]);
+        if (!LOWER) dmma_8x8x4(acc.v[0][2], acc.v[0][3], a0, Y.v[1][st]);
+        dmma_8x8x4(acc.v[1][0], acc.v[1][1], a1, Y.v[0][st]);
+        dmma_8x8x4(acc.v[1][2], acc.v[1][3], a1, Y.v[1][st]);
     }
 }
 
-template <int OPA, int OPB, bool NEG, bool LOWER = false>
-SELINV_DEVINL void gemm(Tile<float> &acc, const float *sA, const float *sB, int g, int t)
+template <bool NEG, bool LOWER = false>
+SELINV_DEVINL void gemm_nt(Tile<float> &acc, const Tile<float> &X, const Tile<float> &Y, float *sX, float *sY,
+                           int g, int t)
 {
     using L = SL<float>;
-#pragma unroll
+    __syncwarp();
+    to_smem<float>(sX, X, g, t);
+    to_smem<float>(sY, Y, g, t);
+    __syncwarp();
+#pragma unroll 4
     for (int k = 0; k < 16; ++k) {
         float a[2], b[4];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            a[h] = OPA == 0 ? sA[L::idx(g + 8 * h, k)] : sA[L::idx(k, g + 8 * h)];
-            if (NEG) a[h] = -a[h];
-        }
+        for (int h = 0; h < 2; ++h) a[h] = NEG ? -sX[L::idx(g + 8 * h, k)] : sX[L::idx(g + 8 * h, k)];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) b[q] = OPB == 0 ? sB[L::idx(k, tcol(t, q))] : sB[L::idx(tcol(t, q), k)];
+        for (int q = 0; q < 4; ++q) b[q] = sY[L::idx(tcol(t, q), k)];
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
             for (int q = 0; q < 4; ++q) acc.v[h][q] = fmaf(a[h], b[q], acc.v[h][q]);
     }
+    __syncwarp();
 }
 
 // In-register inverse of a symmetric positive definite tile by the symmetric
