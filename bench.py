@@ -212,6 +212,33 @@ def fp64_peak_tflops(torch):
     return best
 
 
+# ------------------------------------------------------------------ sharding
+
+def shard_elements(rank: int, batch_per_rank: int):
+    """Batch elements (chains or trees) owned by `rank`: a contiguous slice.
+
+    Elements are independent, so ranks never exchange data; each element's
+    inputs come from its own seeded generator, so the union over ranks is one
+    larger batch of distinct elements (weak scaling)."""
+    return list(range(rank * batch_per_rank, (rank + 1) * batch_per_rank))
+
+
+def max_over_ranks(value_ms: float, world: int, device=None) -> float:
+    """Slowest rank's time (the job's time): an all-reduce MAX when world > 1."""
+    if world <= 1:
+        return value_ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, units_per_rank: int, steps: int, max_ms: float) -> float:
+    """Units processed by all ranks per second of the slowest rank's time."""
+    return world * units_per_rank * steps / (max_ms / 1e3)
+
+
 # ------------------------------------------------------------------ arms
 
 def run_reference(args):
@@ -276,7 +303,7 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.dtype)
 
-    elems = list(range(rank * batch, (rank + 1) * batch))
+    elems = shard_elements(rank, batch)
     stream = torch.cuda.current_stream()
     if w.kind == "grid":
         diag, lower, rhs, _ = inputs.grid_inputs_torch(batch, w.b, w.seed, "cuda", tdt, w.solve)
@@ -352,12 +379,9 @@ def run_ours(args):
         dist.barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
     kernel_ms = sum(a.elapsed_time(b_) for a, b_ in zip(k_start, k_end)) / K
-    if world > 1:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world, "cuda")
     nodes_per_rank = batch * w.L
-    value = world * nodes_per_rank * K / (elapsed_ms / 1e3)
+    value = job_throughput(world, nodes_per_rank, K, elapsed_ms)
 
     # end to end through the same call, inputs from pinned host memory, outputs read back
     e2e = None
@@ -378,13 +402,10 @@ def run_ours(args):
         e.record(stream)
         torch.cuda.synchronize()
         e2e_ms = s.elapsed_time(e)
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e2e_ms, world, "cuda")
         h2d = sum(v.numel() * v.element_size() for v in host_in.values())
         d2h = sum(v.numel() * v.element_size() for v in out.values())
-        e2e = {"value": world * nodes_per_rank * Ke / (e2e_ms / 1e3), "unit": "blocks/s",
+        e2e = {"value": job_throughput(world, nodes_per_rank, Ke, e2e_ms), "unit": "blocks/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     if w.b >= 64:

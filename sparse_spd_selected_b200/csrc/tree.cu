@@ -177,9 +177,11 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leave
                 Tile<T> z;
                 zero(z);
                 store_block<T, FULL>(p.G_edge + v * bb, z, b, g, t);
-                __threadfence();
                 __syncwarp();
-                if (lane == 0) st_release(sy.done + v, 1);
+                if (lane == 0) {
+                    __threadfence();
+                    st_release(sy.done + v, 1);
+                }
                 __syncwarp();
                 break;
             }
@@ -191,13 +193,15 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leave
             zero(u);
             gemm_nt<false, true>(u, w, et, sT, sT2, g, t);   // U_v = W_v E_v^T (lower tiles)
             store_lower_slot<T>(p.ws_u + (int64_t)v * SLOT_ELEMS, u, lane, g, t);
-            __threadfence();                          // U_v visible before the count drops
-            __syncwarp();
+            __syncwarp();                             // the warp's stores are ordered before lane 0's fence
             int old = 0;
-            if (lane == 0) old = atomicSub(sy.pending + par, 1);
+            if (lane == 0) {
+                __threadfence();                      // release U_v before the count drops
+                old = atomicSub(sy.pending + par, 1);
+                if (old == 1) __threadfence();        // acquire every sibling's U
+            }
             old = __shfl_sync(FULL_MASK, old, 0);
             if (old != 1) break;                      // a sibling is still running: it will go on
-            __threadfence();                          // see every sibling's U
             v = par;
         }
     }
@@ -235,12 +239,12 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
             }
         }
         ok = __shfl_sync(FULL_MASK, ok, 0);
+        __syncwarp();                                 // every lane's reads below are ordered after lane 0's acquire
         if (!ok) {                                    // cannot happen for a valid plan: report, move on
             cp_async_wait_all();
             if (lane == 0) atomicMin(p.info + v / td.n, -2);
             continue;
         }
-        __threadfence();
         load_lower_async<T, FULL>(sG, p.G_diag + (int64_t)par * bb, b, lane);   // G_pp (lower), from L2
         cp_async_commit();
         to_smem<T>(sT, a, g, t);                      // lower entries of S_v^-1 valid
@@ -269,9 +273,11 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
         __syncwarp();
         from_smem_lower<T>(a, sT, g, t);              // exactly symmetric
         store_block<T, FULL>(p.G_diag + v * bb, a, b, g, t);
-        __threadfence();
         __syncwarp();
-        if (lane == 0) st_release(sy.done + v, 1);
+        if (lane == 0 && td.child_ptr[v + 1] > td.child_ptr[v]) {   // only parents are waited for
+            __threadfence();
+            st_release(sy.done + v, 1);
+        }
         __syncwarp();
     }
 }
@@ -289,16 +295,29 @@ __global__ void tree_init(const int32_t *child_ptr, int64_t N, int32_t *pending,
 }
 
 // log det per tree = sum of its nodes' log det S_v in a fixed order
-// (deterministic); info INT_MAX -> -1.
-__global__ void tree_finalize(const double *ws_ld, int64_t n, double *logdet, int32_t *info)
+// (deterministic); info INT_MAX -> -1.  1024 threads, each summing a fixed
+// strided subset with four independent partial sums, then a tree in shared
+// memory.
+constexpr int FIN_THREADS = 1024;
+
+__global__ void __launch_bounds__(FIN_THREADS) tree_finalize(const double *ws_ld, int64_t n, double *logdet,
+                                                             int32_t *info)
 {
-    __shared__ double part[256];
+    __shared__ double part[FIN_THREADS];
     const int64_t tr = blockIdx.x;
-    double s = 0.0;
-    for (int64_t v = threadIdx.x; v < n; v += blockDim.x) s += ws_ld[tr * n + v];
-    part[threadIdx.x] = s;
+    const double *x = ws_ld + tr * n;
+    double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+    int64_t v = threadIdx.x;
+    for (; v + 3 * FIN_THREADS < n; v += 4 * FIN_THREADS) {
+        s0 += x[v];
+        s1 += x[v + FIN_THREADS];
+        s2 += x[v + 2 * FIN_THREADS];
+        s3 += x[v + 3 * FIN_THREADS];
+    }
+    for (; v < n; v += FIN_THREADS) s0 += x[v];
+    part[threadIdx.x] = (s0 + s1) + (s2 + s3);
     __syncthreads();
-    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    for (int w = FIN_THREADS / 2; w > 0; w >>= 1) {
         if ((int)threadIdx.x < w) part[threadIdx.x] += part[threadIdx.x + w];
         __syncthreads();
     }
@@ -360,7 +379,7 @@ cudaError_t run_tree(const selinv_tree_plan_s *pl, int b, const T *diag, const T
         const int64_t bd = std::min<int64_t>(max_blocks, ceil_div(ndist, TWARPS));
         kd<<<(unsigned)bd, TWARPS * 32, smem, s>>>(p, td, sy, pl->d_dist_nodes, ndist);
     }
-    tree_finalize<<<(unsigned)pl->trees, 256, 0, s>>>(p.ws_ld, pl->n, logdet, info);
+    tree_finalize<<<(unsigned)pl->trees, FIN_THREADS, 0, s>>>(p.ws_ld, pl->n, logdet, info);
     return cudaGetLastError();
 }
 
