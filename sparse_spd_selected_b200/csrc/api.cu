@@ -56,6 +56,7 @@ selinv_status run_chain(int64_t batch, int64_t L, int32_t b, const void *diag, c
                         aligned(G_lower, 16) && aligned(ws, 16);
         return from_cuda(chain_small_launch<T>(a, al, s));
     }
+    if (b <= 32 && rhs == nullptr) return from_cuda(chain_mid_launch<T>(a, s));
     return from_cuda(chain_large_launch<T>(a, s));
 }
 
@@ -64,6 +65,7 @@ size_t chain_ws(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b, bool wa
     if (!want_g && !want_x) return 0;
     const size_t es = elem_size(dtype);
     if (b <= 16) return round_up(chain_small_workspace(es, batch, L));
+    if (b <= 32 && !want_x) return round_up(chain_mid_workspace(es, batch, L));
     return round_up(chain_large_workspace(es, batch, L, b));
 }
 

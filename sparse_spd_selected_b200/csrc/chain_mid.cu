@@ -1,0 +1,400 @@
+// Block-tridiagonal chains with 16 < b <= 32 (no right-hand side): one CTA
+// of two 4-warp groups per chain, eliminating the chain from both ends.
+//
+// gabp-sparse-inv 0.3.2 (PyPI page), "Implemented and tested kernels" ->
+// Chain and Tree: a chain is a path, and the tree kernel may root it at any
+// node (the Quickstart's root-invariance remark: the chain roots the path at
+// its last node, the tree at node 0).  Rooting it at the middle block m makes
+// the collect sweep two independent half-chains:
+//   top    (group 0)  blocks 0, 1, ..., m-1, coupling C = B_i = A_{i+1,i}
+//   bottom (group 1)  blocks L-1, L-2, ..., m+1, coupling C = B_{i-1}^T = A_{i-1,i}
+// each running S' = D' - C S^-1 C^T toward m; then S_m = D_m - (both
+// contributions), G_mm = S_m^-1, and the two distribute sweeps run outward
+// again with G_{next,j} = -G_{next} W_j, G_jj = S_j^-1 - W_j^T G_{next,j},
+// W_j = C_j S_j^-1.  The two halves run concurrently, halving the
+// sequential length of the long chains.
+//
+// Blocks are padded to 32 (identity / zero pad).  Warp w of a group owns
+// quadrant (I, J) = (w >> 1, w & 1) of every 32 x 32 block as a 16 x 16
+// register tile; products X Y^T are sums of two tile products whose operand
+// quadrants come from shared images, each a register-register FP64
+// tensor-core product; the 32 x 32 inverse is the symmetric Gauss-Jordan
+// sweep over the group (pivot column broadcast through shared memory, one
+// named barrier per pivot).
+#include "kernels.h"
+#include "warp16.cuh"
+
+namespace selinv {
+
+namespace {
+
+constexpr int GW = 4;                  // warps per group
+constexpr int GT = GW * 32;            // threads per group
+
+template <class T> struct Lay {        // per-group shared memory (elements)
+    static constexpr int E = w16::SL<T>::ELEMS;
+    static constexpr int IMG = 4 * E;  // one 32 x 32 block = four quadrant images
+    static constexpr int SCR = sizeof(T) == 4 ? 2 * E * GW : 0;   // float products: per-warp scratch
+    static constexpr int C = 0, D = IMG, X = 2 * IMG, Y = 3 * IMG, Z = 4 * IMG, S = 5 * IMG;
+    static constexpr int CB = S + SCR;
+    static constexpr int GROUP = CB + 64;
+    static constexpr int EXCH = 2 * GROUP;        // exchange image after both groups
+    static constexpr int TOTAL = EXCH + IMG;
+};
+
+SELINV_DEVINL void group_bar(int id) { asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(GT) : "memory"); }
+
+template <class T> SELINV_DEVINL T *quad(T *img, int r, int c) { return img + (2 * r + c) * w16::SL<T>::ELEMS; }
+
+// Quadrant (i, k) of an operand held as four images: TR = false gives
+// M[i][k]; TR = true gives (M^T)[i][k] = M[k][i]^T.
+template <bool TR, class T> SELINV_DEVINL void qget(w16::Tile<T> &o, T *img, int i, int k, int g, int t)
+{
+    if (TR) w16::from_smem_T<T>(o, quad(img, k, i), g, t);
+    else w16::from_smem<T>(o, quad(img, i, k), g, t);
+}
+
+// acc += (NEG ? -1 : 1) (X Y^T)_{IJ} = sum_K X_IK Y_JK^T, operands from images.
+template <bool NEG, bool TX, bool TY, bool LOWER, class T>
+SELINV_DEVINL void qgemm(w16::Tile<T> &acc, T *imgX, T *imgY, int I, int J, T *s1, T *s2, int g, int t)
+{
+#pragma unroll
+    for (int K = 0; K < 2; ++K) {
+        w16::Tile<T> x, y;
+        qget<TX>(x, imgX, I, K, g, t);
+        qget<TY>(y, imgY, J, K, g, t);
+        w16::gemm_nt<NEG, LOWER>(acc, x, y, s1, s2, g, t);
+    }
+}
+
+// Lower triangle of a diagonal block (row-major b x b, identity pad beyond b)
+// into the quadrant images (0,0), (1,0), (1,1); FULL: cp.async chunks.
+template <class T, bool FULL> SELINV_DEVINL void load_diag(T *img, const T *D, int b, int tid)
+{
+    constexpr int CH = 16 / sizeof(T);
+    if (FULL) {
+        for (int j = tid; j < 32 * (32 / CH); j += GT) {
+            const int r = j / (32 / CH), c = (j % (32 / CH)) * CH;
+            if (c <= r) cp_async16(quad(img, r >> 4, c >> 4) + w16::SL<T>::idx(r & 15, c & 15), D + r * 32 + c);
+        }
+    } else {
+        for (int j = tid; j < 1024; j += GT) {
+            const int r = j >> 5, c = j & 31;
+            if (c <= r)
+                quad(img, r >> 4, c >> 4)[w16::SL<T>::idx(r & 15, c & 15)] =
+                    (r < b && c < b) ? __ldg(D + r * b + c) : (r == c ? T(1) : T(0));
+        }
+    }
+}
+
+// A full off-diagonal block (row-major b x b, zero pad) into four images.
+template <class T, bool FULL> SELINV_DEVINL void load_full(T *img, const T *B, int b, int tid)
+{
+    constexpr int CH = 16 / sizeof(T);
+    if (FULL) {
+        for (int j = tid; j < 32 * (32 / CH); j += GT) {
+            const int r = j / (32 / CH), c = (j % (32 / CH)) * CH;
+            cp_async16(quad(img, r >> 4, c >> 4) + w16::SL<T>::idx(r & 15, c & 15), B + r * 32 + c);
+        }
+    } else {
+        for (int j = tid; j < 1024; j += GT) {
+            const int r = j >> 5, c = j & 31;
+            quad(img, r >> 4, c >> 4)[w16::SL<T>::idx(r & 15, c & 15)] = (r < b && c < b) ? __ldg(B + r * b + c) : T(0);
+        }
+    }
+}
+
+// The warp's quadrant of the symmetric block whose lower quadrants are in img.
+template <class T> SELINV_DEVINL void sym_quad(w16::Tile<T> &o, T *img, int I, int J, int g, int t)
+{
+    if (I == J) w16::from_smem_lower<T>(o, quad(img, I, J), g, t);
+    else if (I > J) w16::from_smem<T>(o, quad(img, I, J), g, t);
+    else w16::from_smem_T<T>(o, quad(img, J, I), g, t);
+}
+
+// Store a quadrant tile into a row-major b x b block (TR: transposed position).
+template <class T, bool TR> SELINV_DEVINL void store_quad(T *G, const w16::Tile<T> &a, int b, int I, int J, int g, int t)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            int r = 16 * I + g + 8 * h, c = 16 * J + w16::tcol(t, q);
+            if (TR) {
+                const int tmp = r;
+                r = c;
+                c = tmp;
+            }
+            if (r < b && c < b) G[r * b + c] = a.v[h][q];
+        }
+}
+
+// CTA-group inverse of a symmetric positive definite 32 x 32 block held as
+// quadrant tiles: the symmetric Gauss-Jordan sweep (A_ij -= A_ik A_kj / d,
+// A_ik /= d, A_kj /= d, A_kk = -1/d, then negate); pivots -> det, bad.
+template <class T>
+SELINV_DEVINL void qinverse(w16::Tile<T> &a, T *cbuf, int I, int J, int g, int t, int bar, LogAcc &det, bool &bad)
+{
+    using V = typename w16::Vec2<T>::type;
+    for (int kb = 0; kb < 2; ++kb) {
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+            const int k = 16 * kb + kk;
+            const int kh = kk >> 3, kt = (kk & 7) >> 1, kq = (kk & 1) | ((kk >> 3) << 1);
+            T *cb = cbuf + 32 * (kk & 1);
+            const bool col_owner = (J == kb) && (t == kt);
+            if (col_owner) {
+                cb[16 * I + g] = a.v[0][kq];
+                cb[16 * I + g + 8] = a.v[1][kq];
+            }
+            group_bar(bar);
+            const T d = cb[k];
+            const T c0 = cb[16 * I + g], c1 = cb[16 * I + g + 8];
+            const V r01 = *reinterpret_cast<const V *>(cb + 16 * J + 2 * t);
+            const V r23 = *reinterpret_cast<const V *>(cb + 16 * J + 2 * t + 8);
+            const T row[4] = {r01.x, r01.y, r23.x, r23.y};
+            bad |= !(d > T(0));
+            det.mul((double)d);
+            const T p = recip(d);
+            const T tc[2] = {c0 * p, c1 * p};
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) a.v[h][q] = fma(-tc[h], row[q], a.v[h][q]);
+            if (col_owner) {
+                a.v[0][kq] = tc[0];
+                a.v[1][kq] = tc[1];
+            }
+            if (I == kb && g == (kk & 7)) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) a.v[kh][q] = row[q] * p;
+                if (col_owner) a.v[kh][kq] = -p;
+            }
+        }
+        det.renorm();
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) a.v[h][q] = -a.v[h][q];
+}
+
+template <class T, bool FULL, bool WANT_G>
+__global__ void __launch_bounds__(2 * GT) chain_mid_kernel(ChainArgs<T> p)
+{
+    using namespace w16;
+    using Ly = Lay<T>;
+    constexpr int E = SL<T>::ELEMS;
+    constexpr int64_t SLOT = 3 * 256;                 // S_j^-1 quadrants (0,0), (1,0), (1,1), fragment-major
+    const int tid = threadIdx.x;
+    const int grp = tid / GT;                         // 0: top half, 1: bottom half
+    const int gtid = tid % GT;
+    const int wq = gtid >> 5, lane = tid & 31;
+    const int I = wq >> 1, J = wq & 1;
+    const int g = lane >> 2, t = lane & 3;
+    const int bar = 1 + grp;
+    const bool bottom = grp == 1;
+    const int64_t e = blockIdx.x;
+
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    T *base = reinterpret_cast<T *>(smem_raw);
+    T *gs = base + grp * Ly::GROUP;
+    T *sC = gs + Ly::C, *sD = gs + Ly::D, *sX = gs + Ly::X, *sY = gs + Ly::Y, *sZ = gs + Ly::Z;
+    T *s1 = sizeof(T) == 4 ? gs + Ly::S + wq * 2 * E : nullptr;
+    T *s2 = sizeof(T) == 4 ? s1 + E : nullptr;
+    T *cb = gs + Ly::CB;
+    T *ex = base + Ly::EXCH;
+
+    const int b = p.b;
+    const int64_t L = p.L;
+    const int64_t bb = (int64_t)b * b;
+    const int64_t m = L / 2;
+    const int64_t nh = bottom ? L - 1 - m : m;        // blocks this group eliminates before m
+    const T *Dg = p.diag + e * L * bb;
+    const T *Bg = p.lower + e * (L - 1) * bb;
+    T *ws = p.ws + e * (L > 1 ? L - 1 : 0) * SLOT;    // slots of top block j at j, bottom block L-1-j at L-2-j
+    // j-th block of this half (global index) and the lower block that couples it to the next one
+    auto node = [&](int64_t j) { return bottom ? L - 1 - j : j; };
+    auto cpl = [&](int64_t j) { return bottom ? L - 2 - j : j; };
+    auto slot = [&](int64_t j) { return ws + (bottom ? L - 2 - j : j) * SLOT; };
+
+    LogAcc det;
+    det.init();
+    int fail = -1;
+    Tile<T> a;
+
+    // ---------------- collect sweep, both halves toward m ----------------
+    if (!bottom || nh > 0) {
+        load_diag<T, FULL>(sD, Dg + node(0) * bb, b, gtid);
+        cp_async_commit();
+        cp_async_wait_all();
+        group_bar(bar);
+        sym_quad<T>(a, sD, I, J, g, t);
+        group_bar(bar);
+    } else {
+        zero(a);                                      // no bottom half: contributes nothing to S_m
+    }
+    if (nh > 0) {
+        load_full<T, FULL>(sC, Bg + cpl(0) * bb, b, gtid);
+        if (!bottom || nh > 1) load_diag<T, FULL>(sD, Dg + node(1) * bb, b, gtid);
+        cp_async_commit();
+    }
+    for (int64_t j = 0; j < nh; ++j) {
+        bool bad = false;
+        qinverse<T>(a, cb, I, J, g, t, bar, det, bad);              // a = S_j^-1
+        if (bad && fail < 0) fail = (int)node(j);
+        if (WANT_G && !(I == 0 && J == 1)) {                         // keep the lower quadrants
+            const int qs = I == 0 ? 0 : (J == 0 ? 1 : 2);
+            T *dst = slot(j) + qs * 256 + lane * 8;
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) dst[4 * h + q] = a.v[h][q];
+        }
+        to_smem<T>(quad(sX, I, J), a, g, t);
+        cp_async_wait_all();
+        group_bar(bar);
+        Tile<T> w;
+        zero(w);
+        if (bottom) qgemm<false, true, false, false>(w, sC, sX, I, J, s1, s2, g, t);   // W_j = C_j S_j^-1
+        else qgemm<false, false, false, false>(w, sC, sX, I, J, s1, s2, g, t);
+        to_smem<T>(quad(sY, I, J), w, g, t);
+        group_bar(bar);
+        const bool last = j == nh - 1;
+        if (last && bottom) zero(a);                                  // bottom: only the contribution
+        else sym_quad<T>(a, sD, I, J, g, t);                          // D of the next block (m for the top)
+        if (bottom) qgemm<true, false, true, false>(a, sY, sC, I, J, s1, s2, g, t);    // S' -= W_j C_j^T
+        else qgemm<true, false, false, false>(a, sY, sC, I, J, s1, s2, g, t);
+        group_bar(bar);
+        if (!last) {
+            load_full<T, FULL>(sC, Bg + cpl(j + 1) * bb, b, gtid);
+            if (bottom ? j + 2 < nh : true) load_diag<T, FULL>(sD, Dg + node(j + 2) * bb, b, gtid);
+            cp_async_commit();
+        }
+    }
+
+    // ---------------- middle block m ----------------
+    __syncthreads();
+    if (bottom) to_smem<T>(quad(ex, I, J), a, g, t);
+    __syncthreads();
+    Tile<T> G;
+    if (!bottom) {
+        Tile<T> u;
+        from_smem<T>(u, quad(ex, I, J), g, t);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) a.v[h][q] += u.v[h][q];
+        bool bad = false;
+        qinverse<T>(a, cb, I, J, g, t, bar, det, bad);               // G_mm = S_m^-1
+        if (bad && fail < 0) fail = (int)m;
+    }
+    __syncthreads();
+    if (!bottom) to_smem<T>(quad(ex, I, J), a, g, t);
+    __syncthreads();
+    sym_quad<T>(G, ex, I, J, g, t);                                   // exactly symmetric G_mm, both groups
+    // log det and info: the top group's thread 0 combines both halves
+    double *shd = reinterpret_cast<double *>(base + Ly::D);          // group 0's diagonal images are free here
+    __syncthreads();
+    if (gtid == 0) {
+        shd[2 * grp] = det.log_value();
+        reinterpret_cast<int *>(shd + 4)[grp] = fail;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        if (p.logdet) p.logdet[e] = shd[0] + shd[2];
+        const int f0 = reinterpret_cast<int *>(shd + 4)[0], f1 = reinterpret_cast<int *>(shd + 4)[1];
+        int f = -1;                                                  // first failing block in chain order
+        if (f0 >= 0) f = f0;
+        if (f1 >= 0 && (f < 0 || f1 < f)) f = f1;
+        p.info[e] = f;
+    }
+    __syncthreads();
+    if (!WANT_G) return;
+    if (!bottom) store_quad<T, false>(p.G_diag + e * L * bb + m * bb, G, b, I, J, g, t);
+
+    // ---------------- distribute sweeps, outward from m ----------------
+    if (nh > 0) {
+        load_full<T, FULL>(sC, Bg + cpl(nh - 1) * bb, b, gtid);
+        cp_async_commit();
+    }
+    for (int64_t j = nh - 1; j >= 0; --j) {
+        Tile<T> s;                                                    // S_j^-1
+        if (!(I == 0 && J == 1)) {
+            const int qs = I == 0 ? 0 : (J == 0 ? 1 : 2);
+            const T *src = slot(j) + qs * 256 + lane * 8;
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) s.v[h][q] = src[4 * h + q];
+            to_smem<T>(quad(sX, I, J), s, g, t);
+        }
+        cp_async_wait_all();
+        group_bar(bar);
+        if (I == 0 && J == 1) {
+            from_smem_T<T>(s, quad(sX, 1, 0), g, t);
+            to_smem<T>(quad(sX, 0, 1), s, g, t);
+        }
+        to_smem<T>(quad(sZ, I, J), G, g, t);
+        group_bar(bar);
+        Tile<T> w, gl;
+        zero(w);
+        if (bottom) qgemm<false, true, false, false>(w, sC, sX, I, J, s1, s2, g, t);   // W_j = C_j S_j^-1
+        else qgemm<false, false, false, false>(w, sC, sX, I, J, s1, s2, g, t);
+        to_smem<T>(quad(sY, I, J), w, g, t);
+        group_bar(bar);
+        if (j > 0) {                                                  // next coupling block, early
+            load_full<T, FULL>(sC, Bg + cpl(j - 1) * bb, b, gtid);
+            cp_async_commit();
+        }
+        zero(gl);
+        qgemm<true, false, true, false>(gl, sZ, sY, I, J, s1, s2, g, t);   // G_{next,j} = -G_next W_j
+        T *Gl = p.G_lower + e * (L - 1) * bb + cpl(j) * bb;
+        if (bottom) store_quad<T, true>(Gl, gl, b, I, J, g, t);       // G_lower = G_{next,j}^T below m
+        else store_quad<T, false>(Gl, gl, b, I, J, g, t);
+        group_bar(bar);
+        to_smem<T>(quad(sZ, I, J), gl, g, t);
+        group_bar(bar);
+        qgemm<true, true, true, false>(s, sY, sZ, I, J, s1, s2, g, t);     // G_jj = S_j^-1 - W_j^T G_{next,j}
+        group_bar(bar);
+        to_smem<T>(quad(sZ, I, J), s, g, t);
+        group_bar(bar);
+        sym_quad<T>(G, sZ, I, J, g, t);                               // exactly symmetric G_jj
+        store_quad<T, false>(p.G_diag + e * L * bb + node(j) * bb, G, b, I, J, g, t);
+        group_bar(bar);
+    }
+}
+
+template <class T, bool FULL, bool WANT_G>
+cudaError_t launch_t(const ChainArgs<T> &a, cudaStream_t s)
+{
+    const size_t smem = sizeof(T) * Lay<T>::TOTAL;
+    auto k = chain_mid_kernel<T, FULL, WANT_G>;
+    cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    k<<<(unsigned)a.batch, 2 * GT, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+}  // namespace
+
+size_t chain_mid_workspace(size_t elem, int64_t batch, int64_t L)
+{
+    return (size_t)batch * (size_t)(L > 1 ? L - 1 : 0) * 3 * 256 * elem;
+}
+
+template <class T> cudaError_t chain_mid_launch(const ChainArgs<T> &a, cudaStream_t s)
+{
+    if (a.batch == 0) return cudaSuccess;
+    const bool full = a.b == 32 && al16(a.diag) && al16(a.lower);
+    const bool G = a.G_diag != nullptr;
+    if (full) return G ? launch_t<T, true, true>(a, s) : launch_t<T, true, false>(a, s);
+    return G ? launch_t<T, false, true>(a, s) : launch_t<T, false, false>(a, s);
+}
+
+template cudaError_t chain_mid_launch<double>(const ChainArgs<double> &, cudaStream_t);
+template cudaError_t chain_mid_launch<float>(const ChainArgs<float> &, cudaStream_t);
+
+}  // namespace selinv

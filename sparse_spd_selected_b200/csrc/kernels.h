@@ -27,6 +27,11 @@ template <class T> struct ChainArgs {
 size_t chain_small_workspace(size_t elem, int64_t batch, int64_t L);
 template <class T> cudaError_t chain_small_launch(const ChainArgs<T> &a, bool aligned16, cudaStream_t s);
 
+// 16 < b <= 32, no right-hand side: one CTA of two 4-warp groups per chain,
+// eliminating from both ends toward the middle block.
+size_t chain_mid_workspace(size_t elem, int64_t batch, int64_t L);
+template <class T> cudaError_t chain_mid_launch(const ChainArgs<T> &a, cudaStream_t s);
+
 // 16 < b <= 128: one CTA per chain.
 size_t chain_large_workspace(size_t elem, int64_t batch, int64_t L, int b);
 template <class T> cudaError_t chain_large_launch(const ChainArgs<T> &a, cudaStream_t s);

@@ -219,3 +219,36 @@ def test_pivot_reciprocal_against_cuda_division(cuda_ok):
     ulp = torch.abs(out["G_diag"] - ref) / (torch.finfo(torch.float64).eps * torch.abs(ref))
     assert float(ulp.max()) <= 4.0
     assert float(torch.max(torch.abs(out["logdet"] - torch.log(dev.reshape(-1))))) <= 1e-12
+
+
+# ---------------- 16 < b <= 32 without a right-hand side: two-ended kernel ----------------
+
+@pytest.mark.parametrize("b", [17, 20, 24, 31, 32])
+@pytest.mark.parametrize("L", [1, 2, 3, 4, 5, 8, 33])
+def test_two_ended_blocks_f64(cuda_ok, b, L):
+    diag, lower, _ = inputs.chain_inputs(3, L, b, seed=6000 + 3 * b + L, load=0.5, with_rhs=False)
+    errs, out = run_both(diag, lower, None, torch.float64)
+    assert max(errs.values()) <= TOL[torch.float64], errs
+    Gd = out["G_diag"]
+    assert torch.equal(Gd, Gd.transpose(-1, -2))
+
+
+@pytest.mark.parametrize("b,L", [(32, 40), (24, 9)])
+def test_two_ended_blocks_f32(cuda_ok, b, L):
+    diag, lower, _ = inputs.chain_inputs(3, L, b, seed=6100 + b, load=1.0, with_rhs=False)
+    errs, _ = run_both(diag, lower, None, torch.float32)
+    assert max(errs.values()) <= TOL[torch.float32], errs
+
+
+def test_two_ended_logdet_only_and_not_spd(cuda_ok):
+    diag, lower, _ = inputs.chain_inputs(4, 12, 32, seed=6200, load=1.0, with_rhs=False)
+    d, l = to_dev(diag, torch.float64), to_dev(lower, torch.float64)
+    full = selinv.selinv_chain(d, l)
+    only = selinv.selinv_chain(d, l, want_g=False)
+    assert torch.equal(only["logdet"], full["logdet"])
+    bad = diag.copy()
+    bad[1, 3] = -np.eye(32)          # top half
+    bad[2, 10] = -np.eye(32)         # bottom half
+    out = selinv.selinv_chain(to_dev(bad, torch.float64), l, check=False)
+    info = host(out["info"]).tolist()
+    assert info[0] == -1 and info[3] == -1 and info[1] >= 0 and info[2] >= 0
