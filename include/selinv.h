@@ -30,9 +30,14 @@
  *     exactly symmetric.
  *   - log-determinants are always written as float64 (natural log).
  *   - info[e] (int32, device) is written for every batch element: -1 when
- *     all Schur complements were positive definite, else the index of the
- *     first block (chain) or node (tree) whose pivot was not > 0 (or NaN).
- *     The outputs of such an element are unspecified.  Kernels never trap.
+ *     all Schur complements were positive definite, else the index of a
+ *     block (chain) or node (tree) whose pivot was not > 0 (or NaN): the
+ *     first one in elimination order -- 0 -> L-1 for chains, except that
+ *     chains with 16 < b <= 32 and no right-hand side are eliminated from
+ *     both ends toward the middle block and report the smaller of the two
+ *     halves' first failures.  The outputs of such an element are
+ *     unspecified.  Kernels never trap.  A tree distribute step whose wait
+ *     for its parent timed out (not expected for a valid plan) reports -2.
  *   - The caller owns every buffer, including the workspace, whose size the
  *     *_workspace_size functions give (0 means none is needed; the pointer
  *     may then be NULL).  Workspace and outputs must not overlap inputs.

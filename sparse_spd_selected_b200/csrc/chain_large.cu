@@ -76,8 +76,17 @@ template <class T, int BP> struct Ctx {
         t = lane & 3;
         const int w = tid >> 5;
         rw = w / RW;
-        cw = w % RW;
+        // Quadrants of one row go to four different SM sub-partitions (warp w
+        // runs on sub-partition w % 4), shifted by the row: the lower-triangle
+        // quadrants that the symmetric steps keep busy are then spread evenly.
+#ifndef SELINV_LARGE_ROTATE
+#define SELINV_LARGE_ROTATE 1
+#endif
+        cw = (RW == 4 && SELINV_LARGE_ROTATE) ? (((w & 3) - rw) & 3) : (w % RW);
     }
+    // Tile (mi, ni) of this warp's quadrant lies on or below the block diagonal.
+    SELINV_DEVINL bool tile_lower(int mi, int ni) const { return 32 * rw + 8 * mi >= 32 * cw + 8 * ni; }
+    SELINV_DEVINL bool quad_upper() const { return rw < cw; }
     SELINV_DEVINL int R(int mi) const { return 32 * rw + 8 * mi + g; }
     SELINV_DEVINL int C(int ni, int j) const { return 32 * cw + 8 * ni + 2 * t + j; }
 };
@@ -96,7 +105,6 @@ template <class T> SELINV_DEVINL void zero(Big<T> &a)
         for (int ni = 0; ni < 4; ++ni) a.v[mi][ni][0] = a.v[mi][ni][1] = T(0);
 }
 
-SELINV_DEVINL void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 
 // ---- register tile <-> shared / global -----------------------------------------
 
@@ -252,7 +260,7 @@ enum { OP_BIG = 0, OP_COLPANEL = 1, OP_ROWPANEL = 2 };
 //   A = OP_ROWPANEL: A[m][k] = M[k][m] (row panels of M, i.e. M^T)
 //   B = OP_COLPANEL: B[k][n] = M[n][k] (column panels of M, i.e. M^T)
 //   B = OP_ROWPANEL: B[k][n] = M[k][n] (row panels of M)
-template <class T, int BP, int AOP, int BOP, bool NEG, bool FULL>
+template <class T, int BP, int AOP, int BOP, bool NEG, bool FULL, bool LOWER = false>
 SELINV_DEVINL void gemm(Big<T> &acc, const T *big, T *pbuf, const T *M, int b, const Ctx<T, BP> &x)
 {
     constexpr int NP = Geo<BP>::NP;
@@ -275,7 +283,9 @@ SELINV_DEVINL void gemm(Big<T> &acc, const T *big, T *pbuf, const T *M, int b, c
         __syncthreads();
         const T *P = pbuf + (p & 1) * PANEL;
         const int k0 = 16 * p;
-        if constexpr (sizeof(T) == 8) {
+        if (LOWER && x.quad_upper()) {
+            // nothing to compute above the diagonal
+        } else if constexpr (sizeof(T) == 8) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 double a[4], bf[4];
@@ -300,7 +310,8 @@ SELINV_DEVINL void gemm(Big<T> &acc, const T *big, T *pbuf, const T *M, int b, c
                 for (int mi = 0; mi < 4; ++mi)
 #pragma unroll
                     for (int ni = 0; ni < 4; ++ni)
-                        dmma_8x8x4(acc.v[mi][ni][0], acc.v[mi][ni][1], a[mi], bf[ni]);
+                        if (!LOWER || x.tile_lower(mi, ni))
+                            dmma_8x8x4(acc.v[mi][ni][0], acc.v[mi][ni][1], a[mi], bf[ni]);
             }
         } else {
 #pragma unroll 4
@@ -394,6 +405,146 @@ SELINV_DEVINL void spd_inverse(Big<T> &a, T *colbuf, const Ctx<T, BP> &x, LogAcc
         for (int ni = 0; ni < 4; ++ni) a.v[mi][ni][0] = -a.v[mi][ni][0], a.v[mi][ni][1] = -a.v[mi][ni][1];
 }
 
+// Blocked form of the same sweep for float64: pivots are taken eight at a
+// time (block K = columns 8K..8K+7).  With P = A_KK and T_i = A_iK P^-1, one
+// block step is
+//   A_ij -= T_i A_Kj (i, j not in K),  A_iK = T_i,  A_Kj = T_j^T,  A_KK = -P^-1
+// (equal to eight scalar sweep steps).  Per step: the owners of column block K
+// publish it (BP x 8, shared); every warp inverts the 8 x 8 P in registers (a
+// scalar sweep over one 8 x 8 accumulator tile, so P's eight pivots enter
+// det), forms T for its rows and applies the rank-8 update on the FP64 tensor
+// cores (k permuted to the accumulator layout, as in the 16 x 16 products);
+// T is published for the owners of row block K.  Two barriers per eight
+// pivots instead of eight.
+SELINV_DEVINL void inv8_sweep(double v[2], int lane, int g, int t, LogAcc &det, bool &bad, bool count)
+{
+    // v = P[g][2t], P[g][2t+1] of a symmetric positive definite 8 x 8 P
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int kt = k >> 1, kj = k & 1;
+        const double c = shfl(v[kj], (lane & ~3) | kt);          // P[g][k]
+        double row[2];
+        row[0] = shfl(v[0], (k << 2) | t);                         // P[k][2t]
+        row[1] = shfl(v[1], (k << 2) | t);                         // P[k][2t+1]
+        const double d = shfl(v[kj], (k << 2) | kt);               // P[k][k]
+        bad |= !(d > 0.0);
+        if (count) det.mul(d);
+        const double p = recip(d);
+        const double tc = c * p;
+        v[0] = fma(-tc, row[0], v[0]);
+        v[1] = fma(-tc, row[1], v[1]);
+        if (t == kt) v[kj] = tc;
+        if (g == k) {
+            v[0] = row[0] * p;
+            v[1] = row[1] * p;
+            if (t == kt) v[kj] = -p;
+        }
+    }
+    v[0] = -v[0];
+    v[1] = -v[1];
+}
+
+template <int BP>
+SELINV_DEVINL void spd_inverse_blocked(Big<double> &a, double *cbuf, double *tbuf, const Ctx<double, BP> &x,
+                                       LogAcc &det, bool &bad)
+{
+    constexpr int NB = BP / 8;
+    for (int K = 0; K < NB; ++K) {
+        double *cb = cbuf + (K & 1) * BP * 8;                     // cb[r * 8 + c] = A[r][8K + c]
+        double *tb = tbuf + (K & 1) * BP * 8;                     // tb[r * 8 + c] = T[r][c]
+        const int qK = K >> 2, tK = K & 3;                        // quadrant and tile holding block K
+        if (x.cw == qK) {                                         // publish column block K
+#pragma unroll
+            for (int mi = 0; mi < 4; ++mi) {
+#pragma unroll
+                for (int n = 0; n < 4; ++n)
+                    if (n == tK) {
+                        double2 u;
+                        u.x = a.v[mi][n][0];
+                        u.y = a.v[mi][n][1];
+                        *reinterpret_cast<double2 *>(cb + x.R(mi) * 8 + 2 * x.t) = u;
+                    }
+            }
+        }
+        __syncthreads();
+        // P^-1 in registers (accumulator layout of one 8 x 8 tile; symmetric)
+        double pv[2];
+        {
+            const double2 u = *reinterpret_cast<const double2 *>(cb + (8 * K + x.g) * 8 + 2 * x.t);
+            pv[0] = u.x;
+            pv[1] = u.y;
+        }
+        inv8_sweep(pv, x.lane, x.g, x.t, det, bad, x.tid == 0);
+        // T = A_{rows,K} P^-1 for this warp's rows: 4 m-tiles x 2 k-steps
+        double T[4][2];
+#pragma unroll
+        for (int mi = 0; mi < 4; ++mi) {
+            const double2 arow = *reinterpret_cast<const double2 *>(cb + x.R(mi) * 8 + 2 * x.t);
+            T[mi][0] = T[mi][1] = 0.0;
+            dmma_8x8x4(T[mi][0], T[mi][1], arow.x, pv[0]);
+            dmma_8x8x4(T[mi][0], T[mi][1], arow.y, pv[1]);
+        }
+        if (x.cw == 0) {                                          // publish T (one copy per row)
+#pragma unroll
+            for (int mi = 0; mi < 4; ++mi) {
+                double2 u;
+                u.x = T[mi][0];
+                u.y = T[mi][1];
+                *reinterpret_cast<double2 *>(tb + x.R(mi) * 8 + 2 * x.t) = u;
+            }
+        }
+        // rank-8 update A_ij -= T_i A_Kj, A_Kj = A_jK (symmetric): B fragments from cb
+        double bk[4][2];
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni) {
+            const double2 u = *reinterpret_cast<const double2 *>(cb + (32 * x.cw + 8 * ni + x.g) * 8 + 2 * x.t);
+            bk[ni][0] = u.x;
+            bk[ni][1] = u.y;
+        }
+#pragma unroll
+        for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+            for (int ni = 0; ni < 4; ++ni) {
+                dmma_8x8x4(a.v[mi][ni][0], a.v[mi][ni][1], -T[mi][0], bk[ni][0]);
+                dmma_8x8x4(a.v[mi][ni][0], a.v[mi][ni][1], -T[mi][1], bk[ni][1]);
+            }
+        if (x.cw == qK) {                                         // column block K: T (rows outside K)
+#pragma unroll
+            for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+                for (int n = 0; n < 4; ++n)
+                    if (n == tK) {
+                        a.v[mi][n][0] = T[mi][0];
+                        a.v[mi][n][1] = T[mi][1];
+                    }
+        }
+        __syncthreads();                                          // T published
+        if (x.rw == qK) {                                         // row block K: T_j^T, diagonal block -P^-1
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                if (m == tK) {
+#pragma unroll
+                    for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) a.v[m][ni][j] = tb[x.C(ni, j) * 8 + x.g];
+                    if (x.cw == qK) {
+#pragma unroll
+                        for (int n = 0; n < 4; ++n)
+                            if (n == tK) {
+                                a.v[m][n][0] = -pv[0];
+                                a.v[m][n][1] = -pv[1];
+                            }
+                    }
+                }
+        }
+        if (x.tid == 0) det.renorm();
+    }
+#pragma unroll
+    for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni) a.v[mi][ni][0] = -a.v[mi][ni][0], a.v[mi][ni][1] = -a.v[mi][ni][1];
+}
+
 // Row sums (over this thread's columns) of a tile times the vector v, reduced
 // over the 4 lanes of a row group: the per-warp partial for rows R(mi).
 template <class T, int BP>
@@ -475,7 +626,8 @@ __global__ void __launch_bounds__(Geo<BP>::NT) chain_large_kernel(ChainArgs<T> p
     // ---------------- collect sweep ----------------
     for (int64_t i = 0; i < L; ++i) {
         bool bad = false;
-        spd_inverse<T, BP>(a, colbuf, x, det, bad);
+        if constexpr (sizeof(T) == 8) spd_inverse_blocked<BP>(a, pbuf, pbuf + 2 * BP * 8, x, det, bad);
+        else spd_inverse<T, BP>(a, colbuf, x, det, bad);
         if (bad && fail < 0) fail = (int)i;
         if (i == L - 1) break;
         if (KEEP) store_ws<T, BP>(ws + (2 * i) * BB, a, x);
@@ -504,7 +656,10 @@ __global__ void __launch_bounds__(Geo<BP>::NT) chain_large_kernel(ChainArgs<T> p
             if (x.tid < b) Xv[(i + 1) * b + x.tid] = yv;
         }
         load_sym<T, BP>(a, D + (i + 1) * bb, b, x);
-        gemm<T, BP, OP_BIG, OP_COLPANEL, true, FULL>(a, big, pbuf, Bl + i * bb, b, x);     // S_{i+1} = D_{i+1} - W_i B_i^T
+        gemm<T, BP, OP_BIG, OP_COLPANEL, true, FULL, true>(a, big, pbuf, Bl + i * bb, b, x);   // S_{i+1} = D_{i+1} - W_i B_i^T (lower)
+        to_smem_sym<T, BP>(big, a, x);             // complete the upper triangle (big is free after the gemm)
+        __syncthreads();
+        from_smem<T, BP>(a, big, x);
     }
     if (x.tid == 0) {
         if (p.logdet) p.logdet[e] = det.log_value();
@@ -558,7 +713,7 @@ __global__ void __launch_bounds__(Geo<BP>::NT) chain_large_kernel(ChainArgs<T> p
             }
         }
         if (WANT_G) {
-            gemm<T, BP, OP_ROWPANEL, OP_BIG, true, FULL>(a, big, pbuf, W, b, x);          // G_ii = S_i^-1 - W_i^T G_{i+1,i}
+            gemm<T, BP, OP_ROWPANEL, OP_BIG, true, FULL, true>(a, big, pbuf, W, b, x);    // G_ii = S_i^-1 - W_i^T G_{i+1,i} (lower)
             to_smem_sym<T, BP>(big, a, x);
             __syncthreads();
             from_smem<T, BP>(a, big, x);

@@ -20,6 +20,8 @@ SELINV_DEVINL void cp_async16(void *smem, const void *gmem)
 }
 SELINV_DEVINL void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 SELINV_DEVINL void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+// Wait until at most one committed group (the most recent) is still in flight.
+SELINV_DEVINL void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 
 // Read-only global loads that should not linger in L1.
 template <class T> SELINV_DEVINL T ldg_stream(const T *p) { return __ldcs(p); }

@@ -50,6 +50,12 @@ namespace {
 constexpr int TWARPS = 4;
 
 template <class T> __host__ __device__ constexpr int tree_smem_elems() { return 4 * w16::SL<T>::ELEMS + 64; }
+// distribute: two (edge, S^-1 slot) buffer sets for the node being processed
+// and the next one, plus G_pp and two transpose images
+template <class T> __host__ __device__ constexpr int dist_smem_elems()
+{
+    return 5 * w16::SL<T>::ELEMS + 2 * w16::SLOT_ELEMS;
+}
 
 struct TreeDev {
     const int32_t *child_ptr;
@@ -216,20 +222,30 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    T *sB = reinterpret_cast<T *>(smem_raw) + wid * tree_smem_elems<T>();
-    T *sG = sB + E, *sT = sG + E, *sT2 = sT + E;
+    T *base = reinterpret_cast<T *>(smem_raw) + wid * dist_smem_elems<T>();
+    T *sBuf[2] = {base, base + E};                    // E_v of the current / next node
+    T *sG = base + 2 * E, *sT = sG + E, *sT2 = sT + E;
+    T *stg[2] = {sT2 + E, sT2 + E + SLOT_ELEMS};     // S_v^-1 slots, current / next
     const int b = p.b;
     const int64_t bb = (int64_t)b * b;
+    const unsigned long long cnt = (unsigned long long)count;
 
-    for (;;) {
-        const unsigned long long k = warp_take(sy.counters + 1, lane);
-        if (k >= (unsigned long long)count) break;
+    // Nodes are taken one ahead: the next node's edge block and S^-1 slot
+    // stream in while the current one is computed (its loads are issued after
+    // the current G_pp load, so waiting for "all but the newest group" waits
+    // for exactly the current node's data).
+    unsigned long long k = warp_take(sy.counters + 1, lane);
+    int cur = 0;
+    if (k < cnt) {
+        const int32_t v0 = nodes[k];
+        load_block_async<T, FULL>(sBuf[0], p.edge + v0 * bb, b, lane);
+        stage_lower_slot<T>(stg[0], p.ws_sinv + (int64_t)v0 * SLOT_ELEMS, lane, g, t);
+        cp_async_commit();
+    }
+    while (k < cnt) {
         const int32_t v = nodes[k];
         const int32_t par = td.parent[v];
-        load_block_async<T, FULL>(sB, p.edge + v * bb, b, lane);          // E_v
-        cp_async_commit();
-        Tile<T> a;
-        load_lower_slot<T>(a, p.ws_sinv + (int64_t)v * SLOT_ELEMS, lane, g, t);
+        const unsigned long long kn = warp_take(sy.counters + 1, lane);
         int ok = 1;                                   // wait for G_pp (bounded)
         if (lane == 0) {
             int n = 0;
@@ -240,20 +256,32 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
         }
         ok = __shfl_sync(FULL_MASK, ok, 0);
         __syncwarp();                                 // every lane's reads below are ordered after lane 0's acquire
-        if (!ok) {                                    // cannot happen for a valid plan: report, move on
+        if (ok) load_lower_async<T, FULL>(sG, p.G_diag + (int64_t)par * bb, b, lane);   // G_pp (lower), from L2
+        cp_async_commit();
+        if (kn < cnt) {
+            const int32_t vn = nodes[kn];
+            load_block_async<T, FULL>(sBuf[cur ^ 1], p.edge + vn * bb, b, lane);
+            stage_lower_slot<T>(stg[cur ^ 1], p.ws_sinv + (int64_t)vn * SLOT_ELEMS, lane, g, t);
+            cp_async_commit();
+            cp_async_wait_one();
+        } else {
             cp_async_wait_all();
+        }
+        __syncwarp();
+        if (!ok) {                                    // cannot happen for a valid plan: report, move on
             if (lane == 0) atomicMin(p.info + v / td.n, -2);
+            k = kn;
+            cur ^= 1;
             continue;
         }
-        load_lower_async<T, FULL>(sG, p.G_diag + (int64_t)par * bb, b, lane);   // G_pp (lower), from L2
-        cp_async_commit();
+        Tile<T> a;
+        unstage_lower_slot<T>(a, stg[cur], lane, g, t);
         to_smem<T>(sT, a, g, t);                      // lower entries of S_v^-1 valid
-        cp_async_wait_all();
         __syncwarp();
         from_smem_lower<T>(a, sT, g, t);              // S_v^-1, full
         Tile<T> gp, et, w, wt, ge, get;
         from_smem_lower<T>(gp, sG, g, t);             // G_pp, full
-        from_smem<T>(et, sB, g, t);                   // E_v
+        from_smem<T>(et, sBuf[cur], g, t);            // E_v
         zero(w);
         gemm_nt<false>(w, et, a, sT, sT2, g, t);      // W_v = E_v S_v^-1
         __syncwarp();
@@ -279,6 +307,8 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
             st_release(sy.done + v, 1);
         }
         __syncwarp();
+        k = kn;
+        cur ^= 1;
     }
 }
 
@@ -362,10 +392,11 @@ cudaError_t run_tree(const selinv_tree_plan_s *pl, int b, const T *diag, const T
     tree_init<<<(unsigned)ceil_div(init_n, 256), 256, 0, s>>>(pl->d_child_ptr, N, sy.pending, sy.done, sy.counters,
                                                                info, pl->trees);
     const size_t smem = sizeof(T) * tree_smem_elems<T>() * TWARPS;
+    const size_t smem_d = sizeof(T) * dist_smem_elems<T>() * TWARPS;
     auto kc = full ? tree_collect_kernel<T, true> : tree_collect_kernel<T, false>;
     auto kd = full ? tree_distribute_kernel<T, true> : tree_distribute_kernel<T, false>;
     cudaError_t err = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err == cudaSuccess) err = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err == cudaSuccess) err = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_d);
     if (err != cudaSuccess) return err;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -377,7 +408,7 @@ cudaError_t run_tree(const selinv_tree_plan_s *pl, int b, const T *diag, const T
     kc<<<(unsigned)bc, TWARPS * 32, smem, s>>>(p, td, sy, pl->d_collect_nodes, nleaves);
     if (ndist > 0) {
         const int64_t bd = std::min<int64_t>(max_blocks, ceil_div(ndist, TWARPS));
-        kd<<<(unsigned)bd, TWARPS * 32, smem, s>>>(p, td, sy, pl->d_dist_nodes, ndist);
+        kd<<<(unsigned)bd, TWARPS * 32, smem_d, s>>>(p, td, sy, pl->d_dist_nodes, ndist);
     }
     tree_finalize<<<(unsigned)pl->trees, FIN_THREADS, 0, s>>>(p.ws_ld, pl->n, logdet, info);
     return cudaGetLastError();
