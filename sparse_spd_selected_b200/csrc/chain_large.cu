@@ -416,34 +416,6 @@ SELINV_DEVINL void spd_inverse(Big<T> &a, T *colbuf, const Ctx<T, BP> &x, LogAcc
 // cores (k permuted to the accumulator layout, as in the 16 x 16 products);
 // T is published for the owners of row block K.  Two barriers per eight
 // pivots instead of eight.
-SELINV_DEVINL void inv8_sweep(double v[2], int lane, int g, int t, LogAcc &det, bool &bad, bool count)
-{
-    // v = P[g][2t], P[g][2t+1] of a symmetric positive definite 8 x 8 P
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const int kt = k >> 1, kj = k & 1;
-        const double c = shfl(v[kj], (lane & ~3) | kt);          // P[g][k]
-        double row[2];
-        row[0] = shfl(v[0], (k << 2) | t);                         // P[k][2t]
-        row[1] = shfl(v[1], (k << 2) | t);                         // P[k][2t+1]
-        const double d = shfl(v[kj], (k << 2) | kt);               // P[k][k]
-        bad |= !(d > 0.0);
-        if (count) det.mul(d);
-        const double p = recip(d);
-        const double tc = c * p;
-        v[0] = fma(-tc, row[0], v[0]);
-        v[1] = fma(-tc, row[1], v[1]);
-        if (t == kt) v[kj] = tc;
-        if (g == k) {
-            v[0] = row[0] * p;
-            v[1] = row[1] * p;
-            if (t == kt) v[kj] = -p;
-        }
-    }
-    v[0] = -v[0];
-    v[1] = -v[1];
-}
-
 template <int BP>
 SELINV_DEVINL void spd_inverse_blocked(Big<double> &a, double *cbuf, double *tbuf, const Ctx<double, BP> &x,
                                        LogAcc &det, bool &bad)

@@ -68,6 +68,40 @@ struct LogAcc {
     SELINV_DEVINL double log_value() const { return log(m) + (double)e * 0.69314718055994530942; }
 };
 
+// Inverse of a symmetric positive definite 8 x 8 matrix held by one warp in
+// the m8n8 accumulator layout (lane 4g+t: v = P[g][2t], P[g][2t+1]) by the
+// symmetric Gauss-Jordan sweep: for each pivot k (d = P_kk),
+// P_ij -= P_ik P_kj / d, P_ik /= d, P_kj /= d, P_kk = -1/d, then negated.
+// Row and column k travel by shuffles.  The pivots are multiplied into det
+// (when `count`), a pivot that is not > 0 sets bad.
+SELINV_DEVINL void inv8_sweep(double v[2], int lane, int g, int t, LogAcc &det, bool &bad, bool count)
+{
+    // v = P[g][2t], P[g][2t+1] of a symmetric positive definite 8 x 8 P
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int kt = k >> 1, kj = k & 1;
+        const double c = shfl(v[kj], (lane & ~3) | kt);          // P[g][k]
+        double row[2];
+        row[0] = shfl(v[0], (k << 2) | t);                         // P[k][2t]
+        row[1] = shfl(v[1], (k << 2) | t);                         // P[k][2t+1]
+        const double d = shfl(v[kj], (k << 2) | kt);               // P[k][k]
+        bad |= !(d > 0.0);
+        if (count) det.mul(d);
+        const double p = recip(d);
+        const double tc = c * p;
+        v[0] = fma(-tc, row[0], v[0]);
+        v[1] = fma(-tc, row[1], v[1]);
+        if (t == kt) v[kj] = tc;
+        if (g == k) {
+            v[0] = row[0] * p;
+            v[1] = row[1] * p;
+            if (t == kt) v[kj] = -p;
+        }
+    }
+    v[0] = -v[0];
+    v[1] = -v[1];
+}
+
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 }  // namespace selinv

@@ -347,9 +347,57 @@ SELINV_DEVINL void gemm_nt(Tile<float> &acc, const Tile<float> &X, const Tile<fl
 // Column k is broadcast through `cbuf` (2 x 16 elements of shared memory,
 // alternating per step so one __syncwarp per step suffices); row k is read
 // from the same buffer, the matrix being symmetric.
+// float64 (two block steps of eight pivots):  with K = {8K..8K+7}, H the
+// other half, P = A_KK (the accumulator tile (K, K) itself) and T = A_HK P^-1,
+//   A_HH -= T A_KH,  A_HK = T,  A_KH = T^T,  A_KK = -P^-1,
+// which equals eight scalar sweep steps.  P^-1 is an 8 x 8 register sweep
+// (shuffles only), T and the rank-8 update are FP64 tensor-core MMAs whose
+// k index follows the accumulator layout (P^-1 and A_HK symmetric partners
+// supply the B fragments from the lane's own registers), and T^T is formed
+// by shuffles.  No shared memory, no barrier.
+SELINV_DEVINL void spd_inverse_blocked(Tile<double> &a, int g, int t, LogAcc &det, bool &bad)
+{
+    const int lane = 4 * g + t;
+#pragma unroll
+    for (int K = 0; K < 2; ++K) {
+        const int H = 1 - K;
+        double pv[2] = {a.v[K][2 * K], a.v[K][2 * K + 1]};
+        inv8_sweep(pv, lane, g, t, det, bad, true);
+        double t0 = 0.0, t1 = 0.0;                        // T = A_HK P^-1
+        dmma_8x8x4(t0, t1, a.v[H][2 * K], pv[0]);
+        dmma_8x8x4(t0, t1, a.v[H][2 * K + 1], pv[1]);
+        // A_HH -= T A_KH, with A_KH[k][c] = A_HK[c][k]
+        dmma_8x8x4(a.v[H][2 * H], a.v[H][2 * H + 1], -t0, a.v[H][2 * K]);
+        dmma_8x8x4(a.v[H][2 * H], a.v[H][2 * H + 1], -t1, a.v[H][2 * K + 1]);
+        double tt[2];                                     // T^T: lane (g, t) needs T[2t + j][g]
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int src = ((2 * t + j) << 2) | (g >> 1);
+            const double u0 = shfl(t0, src), u1 = shfl(t1, src);
+            tt[j] = (g & 1) ? u1 : u0;
+        }
+        a.v[H][2 * K] = t0;
+        a.v[H][2 * K + 1] = t1;
+        a.v[K][2 * H] = tt[0];
+        a.v[K][2 * H + 1] = tt[1];
+        a.v[K][2 * K] = -pv[0];
+        a.v[K][2 * K + 1] = -pv[1];
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) a.v[h][q] = -a.v[h][q];
+}
+
 template <class T>
 SELINV_DEVINL void spd_inverse(Tile<T> &a, T *cbuf, int g, int t, LogAcc &det, bool &bad)
 {
+    if constexpr (sizeof(T) == 8) {
+#ifndef SELINV_SCALAR_SWEEP
+        spd_inverse_blocked(a, g, t, det, bad);
+        return;
+#endif
+    }
     using V = typename Vec2<T>::type;
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
