@@ -40,6 +40,7 @@ from sparse_spd_selected_b200 import inputs  # noqa: E402
 PROFILES = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = {
     "chain_small_kernel": ["chain_small.cu", "warp16.cuh", "common.cuh"],
+    "chain_mid_kernel": ["chain_mid.cu", "warp16.cuh", "common.cuh"],
     "chain_large_kernel": ["chain_large.cu", "common.cuh"],
     "tree_collect_kernel": ["tree.cu", "warp16.cuh", "common.cuh"],
 }
@@ -317,8 +318,8 @@ def run_ours(args):
 
     if w.kind == "tree":
         plan = selinv.TreePlan(g["parent"])
-        n_collect, n_dist = plan.levels()
-        launches_per_step = 2 + n_collect + max(n_dist - 1, 0)
+        # init, collect sweep, distribute sweep (trees with more than one node), log-det finalize
+        launches_per_step = 4 if w.L > 1 else 3
         out = {"G_diag": torch.empty_like(dev_in["diag"]), "G_edge": torch.empty_like(dev_in["diag"]),
                "logdet": torch.empty(batch, dtype=torch.float64, device="cuda"),
                "info": torch.empty(batch, dtype=torch.int32, device="cuda")}
@@ -342,7 +343,12 @@ def run_ours(args):
         ws = torch.empty(max(selinv.chain_workspace_size(tdt, batch, L, b, True, "rhs" in dev_in), 1),
                          dtype=torch.uint8, device="cuda")
         launches_per_step = 1
-        kernel = "chain_small_kernel" if b <= 16 else "chain_large_kernel"
+        if b <= 16:
+            kernel = "chain_small_kernel"
+        elif b <= 32 and "rhs" not in dev_in:
+            kernel = "chain_mid_kernel"
+        else:
+            kernel = "chain_large_kernel"
 
         def step():
             selinv.selinv_chain(dev_in["diag"], dev_in["lower"], dev_in.get("rhs"), check=False, out=out,
@@ -408,21 +414,34 @@ def run_ours(args):
         e2e = {"value": job_throughput(world, nodes_per_rank, Ke, e2e_ms), "unit": "blocks/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
-    if w.b >= 64:
+    hbm, src = hbm_peak()
+    byt = algorithmic_bytes(w, es, batch)
+    hbm_achieved = byt / (kernel_ms / 1e3) / 1e9
+    flops = algorithmic_flops(w, batch)
+    flop_rate = flops / (kernel_ms / 1e3) / 1e12
+    traffic = profiled_traffic(kernel, w.name) if batch == w.batch else None
+    hbm_src = f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback 6650 GB/s"
+    if w.b >= 32 and args.dtype == "f64":
+        # arithmetic intensity 7 b^3 / (32 b^2) flop/byte: past the FP64 ridge from b = 32 on
         peak = fp64_peak_tflops(torch)
-        flops = algorithmic_flops(w, batch)
-        roof = {"bound": "tensor", "achieved": flops / (kernel_ms / 1e3) / 1e12, "peak": peak,
-                "unit": "TFLOP/s", "peak_source": "measured in this run: cuBLAS DGEMM 8192^3 (FP64 tensor cores)"}
-        roof["frac"] = roof["achieved"] / peak
-        roof["traffic"] = profiled_traffic(kernel, w.name)
+        roof = {"bound": "tensor", "achieved": flop_rate, "peak": peak, "unit": "TFLOP/s",
+                "frac": flop_rate / peak, "traffic": traffic,
+                "peak_source": "measured in this run: cuBLAS DGEMM 8192^3 (FP64 tensor cores)",
+                "algorithmic_flops_per_launch": flops, "kernel": kernel,
+                "hbm": {"achieved": hbm_achieved, "peak": hbm, "unit": "GB/s", "frac": hbm_achieved / hbm,
+                        "peak_source": hbm_src}}
+    elif w.b >= 32:
+        # fp32 runs on the FP32 pipes: 148 SMs x 128 lanes x 2 flop x 1965 MHz
+        peak = 148 * 128 * 2 * 1.965e9 / 1e12
+        roof = {"bound": "alu", "achieved": flop_rate, "peak": peak, "unit": "TFLOP/s",
+                "frac": flop_rate / peak, "traffic": traffic,
+                "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 flop x 1965 MHz max SM clock",
+                "algorithmic_flops_per_launch": flops, "kernel": kernel,
+                "hbm": {"achieved": hbm_achieved, "peak": hbm, "unit": "GB/s", "frac": hbm_achieved / hbm,
+                        "peak_source": hbm_src}}
     else:
-        peak, src = hbm_peak()
-        byt = algorithmic_bytes(w, es, batch)
-        achieved = byt / (kernel_ms / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "traffic": profiled_traffic(kernel, w.name) if batch == w.batch else None,
-                "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback 6650 GB/s",
-                "algorithmic_bytes_per_launch": byt, "kernel": kernel}
+        roof = {"bound": "hbm", "achieved": hbm_achieved, "peak": hbm, "unit": "GB/s", "frac": hbm_achieved / hbm,
+                "traffic": traffic, "peak_source": hbm_src, "algorithmic_bytes_per_launch": byt, "kernel": kernel}
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
