@@ -308,7 +308,9 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
     if w.kind == "grid":
         diag, lower, rhs, _ = inputs.grid_inputs_torch(batch, w.b, w.seed, "cuda", tdt, w.solve)
-        host_in = None
+        host_in = {"diag": diag.cpu().pin_memory(), "lower": lower.cpu().pin_memory()}
+        if rhs is not None:
+            host_in["rhs"] = rhs.cpu().pin_memory()
     else:
         g = inputs.generate(w, elements=elems)   # per-element seeds: rank r owns its own slice
         host_in = {k: torch.from_numpy(v).to(tdt).pin_memory() for k, v in g.items()

@@ -13,8 +13,8 @@
 //   G_{i+1,i} = -G_{i+1,i+1} W_i,  G_ii = S_i^-1 - W_i^T G_{i+1,i}  (distribute)
 // (G_ii = S_i^-1 - S_i^-1 B_i^T G_{i+1,i} with S_i^-1 B_i^T = W_i^T).  The
 // products run on the FP64 tensor cores (m8n8k4) straight from registers;
-// only W_i and G_{i+1,i} pass through shared memory once each, to be
-// transposed.
+// the distribute sweep forms W_i^T and G_{i+1,i}^T directly, so nothing is
+// transposed (G_{i+1,i} is written out by a transposed store).
 // Between the sweeps only the lower triangle of each S_i^-1 is kept, in the
 // caller's workspace; W_i is recomputed from B_i in the distribute sweep,
 // which moves fewer bytes than storing it.
@@ -158,30 +158,28 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
     if (WANT_G) store_block<T, FULL>(p.G_diag + e * L * bb + (L - 1) * bb, G, b, g, t);
 
     const int64_t last = L - 1;
-    T yp[2] = {T(0), T(0)};     // y_i at rows g, g+8
+    // Backward solve in row form: lane (g, t) keeps x_{i+1} at rows g, g + 8
+    // (xr) and reads y_i at its four columns tcol(t, q) (yc).
+    T xr[2] = {T(0), T(0)};
+    T yc[4] = {T(0), T(0), T(0), T(0)};
     if (WANT_X) {               // x_{L-1} = S_{L-1}^-1 y_{L-1}
         const T *y = sy + 16 * (last & 1);
-        T part[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) part[q] = G.v[0][q] * y[g] + G.v[1][q] * y[g + 8];
+        for (int h = 0; h < 2; ++h) {
+            T s2 = T(0);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            part[q] += shfl_xor(part[q], 4);
-            part[q] += shfl_xor(part[q], 8);
-            part[q] += shfl_xor(part[q], 16);
+            for (int q = 0; q < 4; ++q) s2 = fma(G.v[h][q], y[tcol(t, q)], s2);
+            s2 += shfl_xor(s2, 1);
+            s2 += shfl_xor(s2, 2);
+            xr[h] = s2;
         }
-        if (g == 0) {
-            T *xs = sx + 16 * (last & 1);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int c = tcol(t, q);
-                xs[c] = part[q];
-                if (c < b) X[last * b + c] = part[q];
-            }
+        if (t == 0) {
+            if (g < b) X[last * b + g] = xr[0];
+            if (g + 8 < b) X[last * b + g + 8] = xr[1];
         }
         if (L > 1) {
-            yp[0] = g < b ? X[(last - 1) * b + g] : T(0);
-            yp[1] = g + 8 < b ? X[(last - 1) * b + g + 8] : T(0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) yc[q] = tcol(t, q) < b ? X[(last - 1) * b + tcol(t, q)] : T(0);
         }
     }
     __syncwarp();
@@ -191,8 +189,13 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
         cp_async_commit();
     }
 
+    // W_i^T = S_i^-1 B_i^T and G_{i+1,i}^T = -W_i^T G_{i+1,i+1} are products of
+    // the form X Y^T of register tiles (S_i^-1 and G_{i+1,i+1} symmetric), so no
+    // operand is ever transposed; G_{i+1,i} leaves through a transposed store.
     for (int64_t i = L - 2; i >= 0; --i) {
-        const T yi[2] = {yp[0], yp[1]};
+        T yi[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) yi[q] = yc[q];
         cp_async_wait_all();
         unstage_lower_slot<T>(a, stg, lane, g, t);
         to_smem<T>(sT, a, g, t);                      // lower entries valid
@@ -205,50 +208,40 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
             stage_lower_slot<T>(stg, ws + (i - 1) * SLOT_ELEMS, lane, g, t);
             cp_async_commit();
             if (WANT_X) {
-                yp[0] = g < b ? X[(i - 1) * b + g] : T(0);
-                yp[1] = g + 8 < b ? X[(i - 1) * b + g + 8] : T(0);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) yc[q] = tcol(t, q) < b ? X[(i - 1) * b + tcol(t, q)] : T(0);
             }
         }
-        zero(w);
-        gemm_nt<false>(w, bt, a, sT, sT2, g, t);      // W_i = B_i S_i^-1
+        Tile<T> wt;
+        zero(wt);
+        gemm_nt<false>(wt, a, bt, sT, sT2, g, t);     // W_i^T = S_i^-1 B_i^T
 
         if (WANT_X) {                                 // x_i = S_i^-1 y_i - W_i^T x_{i+1}
-            const T *xn = sx + 16 * ((i + 1) & 1);
-            const T x0 = xn[g], x1 = xn[g + 8];
-            T part[4];
+            T xc[4];                                  // x_{i+1} at the lane's columns
+            xc[0] = shfl(xr[0], (2 * t) << 2);
+            xc[1] = shfl(xr[0], (2 * t + 1) << 2);
+            xc[2] = shfl(xr[1], (2 * t) << 2);
+            xc[3] = shfl(xr[1], (2 * t + 1) << 2);
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                part[q] = a.v[0][q] * yi[0] + a.v[1][q] * yi[1] - w.v[0][q] * x0 - w.v[1][q] * x1;
+            for (int h = 0; h < 2; ++h) {
+                T s2 = T(0);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                part[q] += shfl_xor(part[q], 4);
-                part[q] += shfl_xor(part[q], 8);
-                part[q] += shfl_xor(part[q], 16);
+                for (int q = 0; q < 4; ++q) s2 = fma(a.v[h][q], yi[q], fma(-wt.v[h][q], xc[q], s2));
+                s2 += shfl_xor(s2, 1);
+                s2 += shfl_xor(s2, 2);
+                xr[h] = s2;
             }
-            if (g == 0) {
-                T *xs = sx + 16 * (i & 1);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int c = tcol(t, q);
-                    xs[c] = part[q];
-                    if (c < b) X[i * b + c] = part[q];
-                }
+            if (t == 0) {
+                if (g < b) X[i * b + g] = xr[0];
+                if (g + 8 < b) X[i * b + g + 8] = xr[1];
             }
         }
         if (WANT_G) {
-            Tile<T> wt, gl, glt;
-            __syncwarp();
-            to_smem<T>(sT, w, g, t);
-            __syncwarp();
-            from_smem_T<T>(wt, sT, g, t);             // W_i^T
-            zero(gl);
-            gemm_nt<true>(gl, G, wt, sT, sT2, g, t);  // G_{i+1,i} = -G_{i+1,i+1} W_i
-            store_block<T, FULL>(p.G_lower + e * (L - 1) * bb + i * bb, gl, b, g, t);
-            __syncwarp();
-            to_smem<T>(sT2, gl, g, t);
-            __syncwarp();
-            from_smem_T<T>(glt, sT2, g, t);           // G_{i+1,i}^T
-            gemm_nt<true, true>(a, wt, glt, sT, sT2, g, t);   // G_ii = S_i^-1 - W_i^T G_{i+1,i} (lower tiles)
+            Tile<T> glt;
+            zero(glt);
+            gemm_nt<true>(glt, wt, G, sT, sT2, g, t);          // G_{i+1,i}^T = -W_i^T G_{i+1,i+1}
+            store_block_T<T, FULL>(p.G_lower + e * (L - 1) * bb + i * bb, glt, b, g, t);
+            gemm_nt<true, true>(a, wt, glt, sT, sT2, g, t);    // G_ii = S_i^-1 - W_i^T G_{i+1,i} (lower tiles)
             __syncwarp();
             to_smem<T>(sT, a, g, t);
             __syncwarp();

@@ -191,6 +191,20 @@ template <class T, bool FULL> SELINV_DEVINL void store_block(T *G, const Tile<T>
         }
 }
 
+// Transposed tile to a row-major b x b block: G[c][r] = a[r][c].  For each
+// register the warp writes four runs of eight consecutive elements.
+template <class T, bool FULL> SELINV_DEVINL void store_block_T(T *G, const Tile<T> &a, int b, int g, int t)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = g + 8 * h, c = tcol(t, q);
+            if (FULL) __stcs(G + c * 16 + r, a.v[h][q]);
+            else if (r < b && c < b) G[c * b + r] = a.v[h][q];
+        }
+}
+
 // Lower-triangle slot of a symmetric tile in workspace memory (192 elements):
 // [0, 64): rows 8..15 x cols 0..7, two entries per lane;
 // [64, 192): the two diagonal 8 x 8 tiles' entries of lanes with 2t <= g,
@@ -344,9 +358,9 @@ SELINV_DEVINL void gemm_nt(Tile<float> &acc, const Tile<float> &X, const Tile<fl
 // A_kk = -1/d; after all k the tile holds -A^-1, which is negated.  The
 // pivots d are the successive Schur-complement pivots, so their product is
 // det A (multiplied into `det`); a pivot that is not > 0 sets `bad`.
-// Column k is broadcast through `cbuf` (2 x 16 elements of shared memory,
-// alternating per step so one __syncwarp per step suffices); row k is read
-// from the same buffer, the matrix being symmetric.
+// float32 (one pivot per step): column k is broadcast through `cbuf` (2 x 16
+// elements of shared memory, alternating per step so one __syncwarp per step
+// suffices); row k is read from the same buffer, the matrix being symmetric.
 // float64 (two block steps of eight pivots):  with K = {8K..8K+7}, H the
 // other half, P = A_KK (the accumulator tile (K, K) itself) and T = A_HK P^-1,
 //   A_HH -= T A_KH,  A_HK = T,  A_KH = T^T,  A_KK = -P^-1,
@@ -390,14 +404,8 @@ SELINV_DEVINL void spd_inverse_blocked(Tile<double> &a, int g, int t, LogAcc &de
 }
 
 template <class T>
-SELINV_DEVINL void spd_inverse(Tile<T> &a, T *cbuf, int g, int t, LogAcc &det, bool &bad)
+SELINV_DEVINL void spd_inverse_scalar(Tile<T> &a, T *cbuf, int g, int t, LogAcc &det, bool &bad)
 {
-    if constexpr (sizeof(T) == 8) {
-#ifndef SELINV_SCALAR_SWEEP
-        spd_inverse_blocked(a, g, t, det, bad);
-        return;
-#endif
-    }
     using V = typename Vec2<T>::type;
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
@@ -435,6 +443,13 @@ SELINV_DEVINL void spd_inverse(Tile<T> &a, T *cbuf, int g, int t, LogAcc &det, b
     for (int h = 0; h < 2; ++h)
 #pragma unroll
         for (int q = 0; q < 4; ++q) a.v[h][q] = -a.v[h][q];
+}
+
+// float: one pivot at a time; double: two 8-pivot block steps on the tensor cores.
+template <class T> SELINV_DEVINL void spd_inverse(Tile<T> &a, T *cbuf, int g, int t, LogAcc &det, bool &bad)
+{
+    if constexpr (sizeof(T) == 8) spd_inverse_blocked(a, g, t, det, bad);
+    else spd_inverse_scalar(a, cbuf, g, t, det, bad);
 }
 
 // y_r = sum_c A[r][c] x[c] for the lane's rows g, g + 8 (x in shared memory);
