@@ -19,8 +19,9 @@
 // register tile; products X Y^T are sums of two tile products whose operand
 // quadrants come from shared images, each a register-register FP64
 // tensor-core product; the 32 x 32 inverse is the symmetric Gauss-Jordan
-// sweep over the group (pivot column broadcast through shared memory, one
-// named barrier per pivot).
+// sweep over the group: float64 in four blocks of eight pivots (one named
+// barrier per block, the block updates on the tensor cores), float32 one
+// pivot per barrier.
 #include "kernels.h"
 #include "warp16.cuh"
 
@@ -35,9 +36,10 @@ template <class T> struct Lay {        // per-group shared memory (elements)
     static constexpr int E = w16::SL<T>::ELEMS;
     static constexpr int IMG = 4 * E;  // one 32 x 32 block = four quadrant images
     static constexpr int SCR = sizeof(T) == 4 ? 2 * E * GW : 0;   // float products: per-warp scratch
-    static constexpr int C = 0, D = IMG, X = 2 * IMG, Y = 3 * IMG, Z = 4 * IMG, S = 5 * IMG;
+    static constexpr int C = 0, D = IMG, X = 2 * IMG, Y = 3 * IMG, Z = 4 * IMG, Z2 = 5 * IMG, S = 6 * IMG;
     static constexpr int CB = S + SCR;
-    static constexpr int GROUP = CB + 64;
+    static constexpr int CBN = sizeof(T) == 8 ? 2 * (32 * 8 + 8 * 8) : 64;   // inverse broadcast buffers
+    static constexpr int GROUP = CB + CBN;
     static constexpr int EXCH = 2 * GROUP;        // exchange image after both groups
     static constexpr int TOTAL = EXCH + IMG;
 };
@@ -133,7 +135,8 @@ template <class T, bool TR> SELINV_DEVINL void store_quad(T *G, const w16::Tile<
 // quadrant tiles: the symmetric Gauss-Jordan sweep (A_ij -= A_ik A_kj / d,
 // A_ik /= d, A_kj /= d, A_kk = -1/d, then negate); pivots -> det, bad.
 template <class T>
-SELINV_DEVINL void qinverse(w16::Tile<T> &a, T *cbuf, int I, int J, int g, int t, int bar, LogAcc &det, bool &bad)
+SELINV_DEVINL void qinverse_scalar(w16::Tile<T> &a, T *cbuf, int I, int J, int g, int t, int bar, LogAcc &det,
+                                   bool &bad)
 {
     using V = typename w16::Vec2<T>::type;
     for (int kb = 0; kb < 2; ++kb) {
@@ -179,13 +182,125 @@ SELINV_DEVINL void qinverse(w16::Tile<T> &a, T *cbuf, int I, int J, int g, int t
         for (int q = 0; q < 4; ++q) a.v[h][q] = -a.v[h][q];
 }
 
+// float64: four block steps of eight pivots.  Block K (rows and columns
+// 8K..8K+7) lies in quadrant kq = K >> 1, half kh = K & 1.  The diagonal warp
+// (kq, kq) inverts the pivot block P = A_KK in registers (shuffle-only sweep;
+// pivots -> det, bad) and publishes P^-1; the warps of quadrant column kq
+// publish block column K.  After one group barrier each warp updates its four
+// 8 x 8 subtiles (r, c) on the FP64 tensor cores:
+//   r, c != K:  A_rc -= T_r A_cK^T,  T_r = A_rK P^-1
+//   c == K:     A_rK = T_r;    r == K:  A_Kc = P^-1 A_cK^T;    A_KK = -P^-1
+// (the m8n8k4 k index runs over 2t, 2t + 1 of the block, the accumulator
+// layout itself).  The two broadcast buffers alternate between block steps,
+// so one barrier per step suffices.  Only the diagonal warps see the pivots.
+constexpr int QBUF = 32 * 8 + 8 * 8;
+
+SELINV_DEVINL void qinverse_blocked(w16::Tile<double> &a, double *buf, int I, int J, int g, int t, int bar,
+                                    LogAcc &det, bool &bad)
+{
+    const int lane = 4 * g + t;
+#pragma unroll
+    for (int K = 0; K < 4; ++K) {
+        const int kq = K >> 1, kh = K & 1;
+        double *col = buf + (K & 1) * QBUF;            // block column K, [32][8]
+        double *pin = col + 32 * 8;                     // P^-1, [8][8]
+        if (J == kq) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                *reinterpret_cast<double2 *>(col + (16 * I + g + 8 * h) * 8 + 2 * t) =
+                    make_double2(a.v[h][2 * kh], a.v[h][2 * kh + 1]);
+            if (I == kq) {
+                double pv[2] = {a.v[kh][2 * kh], a.v[kh][2 * kh + 1]};
+                inv8_sweep(pv, lane, g, t, det, bad, true);
+                det.renorm();
+                *reinterpret_cast<double2 *>(pin + g * 8 + 2 * t) = make_double2(pv[0], pv[1]);
+            }
+        }
+        group_bar(bar);
+        const double2 pi = *reinterpret_cast<const double2 *>(pin + g * 8 + 2 * t);
+        double2 ar[2], ac[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            ar[h] = *reinterpret_cast<const double2 *>(col + (16 * I + g + 8 * h) * 8 + 2 * t);
+            ac[h] = *reinterpret_cast<const double2 *>(col + (16 * J + g + 8 * h) * 8 + 2 * t);
+        }
+        double tr[2][2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {                   // T_r = A_rK P^-1
+            tr[h][0] = tr[h][1] = 0.0;
+            dmma_8x8x4(tr[h][0], tr[h][1], ar[h].x, pi.x);
+            dmma_8x8x4(tr[h][0], tr[h][1], ar[h].y, pi.y);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h)                     // A_rc -= T_r A_cK^T
+#pragma unroll
+            for (int n = 0; n < 2; ++n) {
+                dmma_8x8x4(a.v[h][2 * n], a.v[h][2 * n + 1], -tr[h][0], ac[n].x);
+                dmma_8x8x4(a.v[h][2 * n], a.v[h][2 * n + 1], -tr[h][1], ac[n].y);
+            }
+        if (J == kq) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                a.v[h][2 * kh] = tr[h][0];
+                a.v[h][2 * kh + 1] = tr[h][1];
+            }
+        }
+        if (I == kq) {
+#pragma unroll
+            for (int n = 0; n < 2; ++n) {               // A_Kc = P^-1 A_cK^T
+                double u0 = 0.0, u1 = 0.0;
+                dmma_8x8x4(u0, u1, pi.x, ac[n].x);
+                dmma_8x8x4(u0, u1, pi.y, ac[n].y);
+                a.v[kh][2 * n] = u0;
+                a.v[kh][2 * n + 1] = u1;
+            }
+            if (J == kq) {
+                a.v[kh][2 * kh] = -pi.x;
+                a.v[kh][2 * kh + 1] = -pi.y;
+            }
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) a.v[h][q] = -a.v[h][q];
+}
+
+template <class T>
+SELINV_DEVINL void qinverse(w16::Tile<T> &a, T *cbuf, int I, int J, int g, int t, int bar, LogAcc &det, bool &bad)
+{
+    if constexpr (sizeof(T) == 8) qinverse_blocked(a, cbuf, I, J, g, t, bar, det, bad);
+    else qinverse_scalar(a, cbuf, I, J, g, t, bar, det, bad);
+}
+
+// Copy n elements (a multiple of 16 bytes) from shared to global memory, or
+// stage them from global to shared (cp.async; the caller commits / waits).
+template <class T> SELINV_DEVINL void copy_out(T *dst, const T *src, int n, int gtid)
+{
+    using V = typename w16::Vec2<T>::type;
+    constexpr int CH = 16 / sizeof(T);
+    for (int k = gtid; k < n / CH; k += GT) {
+        const V *s4 = reinterpret_cast<const V *>(src + k * CH);
+        V *d4 = reinterpret_cast<V *>(dst + k * CH);
+        d4[0] = s4[0];
+        if (CH == 4) d4[1] = s4[1];
+    }
+}
+template <class T> SELINV_DEVINL void stage_in(T *dst, const T *src, int n, int gtid)
+{
+    constexpr int CH = 16 / sizeof(T);
+    for (int k = gtid; k < n / CH; k += GT) cp_async16(dst + k * CH, src + k * CH);
+}
+
 template <class T, bool FULL, bool WANT_G>
 __global__ void __launch_bounds__(2 * GT) chain_mid_kernel(ChainArgs<T> p)
 {
     using namespace w16;
     using Ly = Lay<T>;
     constexpr int E = SL<T>::ELEMS;
-    constexpr int64_t SLOT = 3 * 256;                 // S_j^-1 quadrants (0,0), (1,0), (1,1), fragment-major
+    // workspace per eliminated block: the lower quadrant images (0,0), (1,0),
+    // (1,1) of S_j^-1, then the four quadrant images of W_j
+    constexpr int64_t SLOT = 7 * E;
     const int tid = threadIdx.x;
     const int grp = tid / GT;                         // 0: top half, 1: bottom half
     const int gtid = tid % GT;
@@ -199,7 +314,7 @@ __global__ void __launch_bounds__(2 * GT) chain_mid_kernel(ChainArgs<T> p)
     extern __shared__ __align__(16) unsigned char smem_raw[];
     T *base = reinterpret_cast<T *>(smem_raw);
     T *gs = base + grp * Ly::GROUP;
-    T *sC = gs + Ly::C, *sD = gs + Ly::D, *sX = gs + Ly::X, *sY = gs + Ly::Y, *sZ = gs + Ly::Z;
+    T *sC = gs + Ly::C, *sD = gs + Ly::D, *sX = gs + Ly::X, *sY = gs + Ly::Y, *sZ = gs + Ly::Z, *sZ2 = gs + Ly::Z2;
     T *s1 = sizeof(T) == 4 ? gs + Ly::S + wq * 2 * E : nullptr;
     T *s2 = sizeof(T) == 4 ? s1 + E : nullptr;
     T *cb = gs + Ly::CB;
@@ -212,11 +327,11 @@ __global__ void __launch_bounds__(2 * GT) chain_mid_kernel(ChainArgs<T> p)
     const int64_t nh = bottom ? L - 1 - m : m;        // blocks this group eliminates before m
     const T *Dg = p.diag + e * L * bb;
     const T *Bg = p.lower + e * (L - 1) * bb;
-    T *ws = p.ws + e * (L > 1 ? L - 1 : 0) * SLOT;    // slots of top block j at j, bottom block L-1-j at L-2-j
+    T *ws = WANT_G ? p.ws + e * (L > 1 ? L - 1 : 0) * SLOT : nullptr;
     // j-th block of this half (global index) and the lower block that couples it to the next one
     auto node = [&](int64_t j) { return bottom ? L - 1 - j : j; };
     auto cpl = [&](int64_t j) { return bottom ? L - 2 - j : j; };
-    auto slot = [&](int64_t j) { return ws + (bottom ? L - 2 - j : j) * SLOT; };
+    auto slot = [&](int64_t j) { return ws + (bottom ? L - 2 - j : j) * SLOT; };   // top j at j, bottom at L-2-j
 
     LogAcc det;
     det.init();
@@ -243,23 +358,20 @@ __global__ void __launch_bounds__(2 * GT) chain_mid_kernel(ChainArgs<T> p)
         bool bad = false;
         qinverse<T>(a, cb, I, J, g, t, bar, det, bad);              // a = S_j^-1
         if (bad && fail < 0) fail = (int)node(j);
-        if (WANT_G && !(I == 0 && J == 1)) {                         // keep the lower quadrants
-            const int qs = I == 0 ? 0 : (J == 0 ? 1 : 2);
-            T *dst = slot(j) + qs * 256 + lane * 8;
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) dst[4 * h + q] = a.v[h][q];
-        }
         to_smem<T>(quad(sX, I, J), a, g, t);
         cp_async_wait_all();
         group_bar(bar);
+        if (WANT_G) {                                                 // keep the lower quadrant images
+            copy_out<T>(slot(j), sX, E, gtid);
+            copy_out<T>(slot(j) + E, quad(sX, 1, 0), 2 * E, gtid);
+        }
         Tile<T> w;
         zero(w);
         if (bottom) qgemm<false, true, false, false>(w, sC, sX, I, J, s1, s2, g, t);   // W_j = C_j S_j^-1
         else qgemm<false, false, false, false>(w, sC, sX, I, J, s1, s2, g, t);
         to_smem<T>(quad(sY, I, J), w, g, t);
         group_bar(bar);
+        if (WANT_G) copy_out<T>(slot(j) + 3 * E, sY, 4 * E, gtid);     // and W_j for the distribute sweep
         const bool last = j == nh - 1;
         if (last && bottom) zero(a);                                  // bottom: only the contribution
         else sym_quad<T>(a, sD, I, J, g, t);                          // D of the next block (m for the top)
@@ -293,20 +405,27 @@ __global__ void __launch_bounds__(2 * GT) chain_mid_kernel(ChainArgs<T> p)
     if (!bottom) to_smem<T>(quad(ex, I, J), a, g, t);
     __syncthreads();
     sym_quad<T>(G, ex, I, J, g, t);                                   // exactly symmetric G_mm, both groups
-    // log det and info: the top group's thread 0 combines both halves
+    // log det and info.  float64: the pivots live in the diagonal warps (0,0)
+    // and (1,1) of each group; float32: every warp saw all of them, so the
+    // (1,1) warps add nothing to the log-determinant.
     double *shd = reinterpret_cast<double *>(base + Ly::D);          // group 0's diagonal images are free here
     __syncthreads();
-    if (gtid == 0) {
-        shd[2 * grp] = det.log_value();
-        reinterpret_cast<int *>(shd + 4)[grp] = fail;
+    if ((wq == 0 || wq == GW - 1) && lane == 0) {
+        const int d = wq == GW - 1;
+        shd[2 * grp + d] = (sizeof(T) == 8 || d == 0) ? det.log_value() : 0.0;
+        reinterpret_cast<int *>(shd + 4)[2 * grp + d] = fail;
     }
     __syncthreads();
     if (tid == 0) {
-        if (p.logdet) p.logdet[e] = shd[0] + shd[2];
-        const int f0 = reinterpret_cast<int *>(shd + 4)[0], f1 = reinterpret_cast<int *>(shd + 4)[1];
-        int f = -1;                                                  // first failing block in chain order
-        if (f0 >= 0) f = f0;
-        if (f1 >= 0 && (f < 0 || f1 < f)) f = f1;
+        if (p.logdet) p.logdet[e] = (shd[0] + shd[1]) + (shd[2] + shd[3]);
+        const int *fs = reinterpret_cast<const int *>(shd + 4);
+        // first failure of each half in its own elimination order (top: lowest
+        // index, bottom: highest), then the smaller index of the two halves
+        int ft = fs[0], fb = fs[2];
+        if (fs[1] >= 0 && (ft < 0 || fs[1] < ft)) ft = fs[1];
+        if (fs[3] >= 0 && (fb < 0 || fs[3] > fb)) fb = fs[3];
+        int f = ft;
+        if (fb >= 0 && (f < 0 || fb < f)) f = fb;
         p.info[e] = f;
     }
     __syncthreads();
@@ -314,54 +433,50 @@ __global__ void __launch_bounds__(2 * GT) chain_mid_kernel(ChainArgs<T> p)
     if (!bottom) store_quad<T, false>(p.G_diag + e * L * bb + m * bb, G, b, I, J, g, t);
 
     // ---------------- distribute sweeps, outward from m ----------------
+    // G_{next} is kept as an image whose lower quadrants are read symmetrically
+    // (sZa); S_j^-1 and W_j are staged from the workspace one block ahead into
+    // alternating buffers.
+    T *sZa = sZ, *sZb = sZ2;
+    to_smem<T>(quad(sZa, I, J), G, g, t);
     if (nh > 0) {
-        load_full<T, FULL>(sC, Bg + cpl(nh - 1) * bb, b, gtid);
+        stage_in<T>(sX, slot(nh - 1), E, gtid);
+        stage_in<T>(quad(sX, 1, 0), slot(nh - 1) + E, 2 * E, gtid);
+        stage_in<T>(sY, slot(nh - 1) + 3 * E, 4 * E, gtid);
         cp_async_commit();
     }
+    int cur = 0;
     for (int64_t j = nh - 1; j >= 0; --j) {
-        Tile<T> s;                                                    // S_j^-1
-        if (!(I == 0 && J == 1)) {
-            const int qs = I == 0 ? 0 : (J == 0 ? 1 : 2);
-            const T *src = slot(j) + qs * 256 + lane * 8;
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) s.v[h][q] = src[4 * h + q];
-            to_smem<T>(quad(sX, I, J), s, g, t);
-        }
+        T *bS = cur ? sD : sX, *bW = cur ? sC : sY;
         cp_async_wait_all();
-        group_bar(bar);
-        if (I == 0 && J == 1) {
-            from_smem_T<T>(s, quad(sX, 1, 0), g, t);
-            to_smem<T>(quad(sX, 0, 1), s, g, t);
-        }
-        to_smem<T>(quad(sZ, I, J), G, g, t);
-        group_bar(bar);
-        Tile<T> w, gl;
-        zero(w);
-        if (bottom) qgemm<false, true, false, false>(w, sC, sX, I, J, s1, s2, g, t);   // W_j = C_j S_j^-1
-        else qgemm<false, false, false, false>(w, sC, sX, I, J, s1, s2, g, t);
-        to_smem<T>(quad(sY, I, J), w, g, t);
-        group_bar(bar);
-        if (j > 0) {                                                  // next coupling block, early
-            load_full<T, FULL>(sC, Bg + cpl(j - 1) * bb, b, gtid);
+        group_bar(bar);                                               // S_j^-1, W_j staged; G_next image written
+        if (j > 0) {                                                  // next block's operands into the other buffers
+            T *nS = cur ? sX : sD, *nW = cur ? sY : sC;
+            stage_in<T>(nS, slot(j - 1), E, gtid);
+            stage_in<T>(quad(nS, 1, 0), slot(j - 1) + E, 2 * E, gtid);
+            stage_in<T>(nW, slot(j - 1) + 3 * E, 4 * E, gtid);
             cp_async_commit();
         }
+        Tile<T> s, gl;
+        sym_quad<T>(s, bS, I, J, g, t);                               // S_j^-1
         zero(gl);
-        qgemm<true, false, true, false>(gl, sZ, sY, I, J, s1, s2, g, t);   // G_{next,j} = -G_next W_j
+#pragma unroll
+        for (int K = 0; K < 2; ++K) {                                 // G_{next,j} = -G_next W_j
+            Tile<T> x, y;
+            sym_quad<T>(x, sZa, I, K, g, t);
+            from_smem_T<T>(y, quad(bW, K, J), g, t);
+            gemm_nt<true>(gl, x, y, s1, s2, g, t);
+        }
         T *Gl = p.G_lower + e * (L - 1) * bb + cpl(j) * bb;
         if (bottom) store_quad<T, true>(Gl, gl, b, I, J, g, t);       // G_lower = G_{next,j}^T below m
         else store_quad<T, false>(Gl, gl, b, I, J, g, t);
+        to_smem<T>(quad(sZb, I, J), gl, g, t);
         group_bar(bar);
-        to_smem<T>(quad(sZ, I, J), gl, g, t);
+        qgemm<true, true, true, false>(s, bW, sZb, I, J, s1, s2, g, t);   // G_jj = S_j^-1 - W_j^T G_{next,j}
+        to_smem<T>(quad(sZa, I, J), s, g, t);                         // sZa is free: all read it before the barrier
         group_bar(bar);
-        qgemm<true, true, true, false>(s, sY, sZ, I, J, s1, s2, g, t);     // G_jj = S_j^-1 - W_j^T G_{next,j}
-        group_bar(bar);
-        to_smem<T>(quad(sZ, I, J), s, g, t);
-        group_bar(bar);
-        sym_quad<T>(G, sZ, I, J, g, t);                               // exactly symmetric G_jj
+        sym_quad<T>(G, sZa, I, J, g, t);                              // exactly symmetric G_jj
         store_quad<T, false>(p.G_diag + e * L * bb + node(j) * bb, G, b, I, J, g, t);
-        group_bar(bar);
+        cur ^= 1;
     }
 }
 
@@ -382,7 +497,8 @@ bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 size_t chain_mid_workspace(size_t elem, int64_t batch, int64_t L)
 {
-    return (size_t)batch * (size_t)(L > 1 ? L - 1 : 0) * 3 * 256 * elem;
+    const size_t E = elem == 8 ? w16::SL<double>::ELEMS : w16::SL<float>::ELEMS;
+    return (size_t)batch * (size_t)(L > 1 ? L - 1 : 0) * 7 * E * elem;
 }
 
 template <class T> cudaError_t chain_mid_launch(const ChainArgs<T> &a, cudaStream_t s)
