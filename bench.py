@@ -40,7 +40,9 @@ from sparse_spd_selected_b200 import inputs  # noqa: E402
 PROFILES = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = {
     "chain_small_kernel": ["chain_small.cu", "warp16.cuh", "common.cuh"],
-    "chain_mid_kernel": ["chain_mid.cu", "warp16.cuh", "common.cuh"],
+    "chain_mid_kernel": ["chain_mid.cu", "quad32.cuh", "warp16.cuh", "common.cuh"],
+    "seg_collect_kernel": ["chain_seg.cu", "quad32.cuh", "warp16.cuh", "common.cuh"],
+    "seg_distribute_kernel": ["chain_seg.cu", "quad32.cuh", "warp16.cuh", "common.cuh"],
     "chain_large_kernel": ["chain_large.cu", "common.cuh"],
     "tree_collect_kernel": ["tree.cu", "warp16.cuh", "common.cuh"],
 }
@@ -345,8 +347,13 @@ def run_ours(args):
         ws = torch.empty(max(selinv.chain_workspace_size(tdt, batch, L, b, True, "rhs" in dev_in), 1),
                          dtype=torch.uint8, device="cuda")
         launches_per_step = 1
+        segments = selinv.chain_segments(batch, L, b, True, "rhs" in dev_in)
         if b <= 16:
             kernel = "chain_small_kernel"
+        elif segments > 0:
+            # segments' collect, separators' D', their two-ended chain, segments' distribute, log det
+            kernel = "seg_distribute_kernel"
+            launches_per_step = 5
         elif b <= 32 and "rhs" not in dev_in:
             kernel = "chain_mid_kernel"
         else:

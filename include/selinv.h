@@ -87,6 +87,21 @@ size_t selinv_chain_workspace_size(selinv_dtype dtype, int64_t batch, int64_t L,
                                    int32_t want_g, int32_t want_x);
 
 /*
+ * How many segments selinv_chain cuts each chain into for these sizes on the
+ * current device (0: it does not).  Only 16 < b <= 32 with G requested and no
+ * right-hand side is cut, and only when the batch is too small to fill the
+ * GPU (fewer than three chains per SM's worth of segments) and L >= 96.  The
+ * P - 1 separator blocks are eliminated last, so the blocks reach the same
+ * factorisation in another order (gabp-sparse-inv, "Implemented and tested
+ * kernels" -> Chain and Tree: a chain may be rooted at any node).  The
+ * workspace size depends on the answer, hence on the current device's SM
+ * count.  With segments, info reports the smallest block index at which any
+ * segment (in its own elimination order) or the separators' chain met a
+ * pivot that is not > 0.
+ */
+int32_t selinv_chain_segments(int64_t batch, int64_t L, int32_t b, int32_t want_g, int32_t want_x);
+
+/*
  * Selected inverse, log-determinant and (optionally) solve of `batch`
  * independent block-tridiagonal SPD chains of L blocks of size b.
  * (gabp-sparse-inv, "Implemented and tested kernels" -> Chain, and the

@@ -56,7 +56,11 @@ selinv_status run_chain(int64_t batch, int64_t L, int32_t b, const void *diag, c
                         aligned(G_lower, 16) && aligned(ws, 16);
         return from_cuda(chain_small_launch<T>(a, al, s));
     }
-    if (b <= 32 && rhs == nullptr) return from_cuda(chain_mid_launch<T>(a, s));
+    if (b <= 32 && rhs == nullptr) {
+        const int P = chain_seg_parts(batch, L, b, G_diag != nullptr, false);
+        if (P > 0) return from_cuda(chain_seg_launch<T>(a, P, s));
+        return from_cuda(chain_mid_launch<T>(a, s));
+    }
     return from_cuda(chain_large_launch<T>(a, s));
 }
 
@@ -65,7 +69,11 @@ size_t chain_ws(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b, bool wa
     if (!want_g && !want_x) return 0;
     const size_t es = elem_size(dtype);
     if (b <= 16) return round_up(chain_small_workspace(es, batch, L));
-    if (b <= 32 && !want_x) return round_up(chain_mid_workspace(es, batch, L));
+    if (b <= 32 && !want_x) {
+        const int P = chain_seg_parts(batch, L, b, want_g, want_x);
+        if (P > 0) return round_up(chain_seg_workspace(es, batch, L, b, P, want_g));
+        return round_up(chain_mid_workspace(es, batch, L));
+    }
     return round_up(chain_large_workspace(es, batch, L, b));
 }
 
@@ -90,6 +98,12 @@ const char *selinv_status_string(selinv_status s)
 int32_t selinv_version(void) { return 100; }
 
 int32_t selinv_max_block(void) { return MAX_BLOCK; }
+
+int32_t selinv_chain_segments(int64_t batch, int64_t L, int32_t b, int32_t want_g, int32_t want_x)
+{
+    if (batch < 0 || L < 1 || b < 1 || b > MAX_BLOCK) return 0;
+    return chain_seg_parts(batch, L, b, want_g != 0, want_x != 0);
+}
 
 size_t selinv_chain_workspace_size(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b,
                                    int32_t want_g, int32_t want_x)

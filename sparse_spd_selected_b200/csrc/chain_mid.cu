@@ -23,274 +23,13 @@
 // barrier per block, the block updates on the tensor cores), float32 one
 // pivot per barrier.
 #include "kernels.h"
-#include "warp16.cuh"
+#include "quad32.cuh"
 
 namespace selinv {
 
 namespace {
 
-constexpr int GW = 4;                  // warps per group
-constexpr int GT = GW * 32;            // threads per group
-
-template <class T> struct Lay {        // per-group shared memory (elements)
-    static constexpr int E = w16::SL<T>::ELEMS;
-    static constexpr int IMG = 4 * E;  // one 32 x 32 block = four quadrant images
-    static constexpr int SCR = sizeof(T) == 4 ? 2 * E * GW : 0;   // float products: per-warp scratch
-    static constexpr int C = 0, D = IMG, X = 2 * IMG, Y = 3 * IMG, Z = 4 * IMG, Z2 = 5 * IMG, S = 6 * IMG;
-    static constexpr int CB = S + SCR;
-    static constexpr int CBN = sizeof(T) == 8 ? 2 * (32 * 8 + 8 * 8) : 64;   // inverse broadcast buffers
-    static constexpr int GROUP = CB + CBN;
-    static constexpr int EXCH = 2 * GROUP;        // exchange image after both groups
-    static constexpr int TOTAL = EXCH + IMG;
-};
-
-SELINV_DEVINL void group_bar(int id) { asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(GT) : "memory"); }
-
-template <class T> SELINV_DEVINL T *quad(T *img, int r, int c) { return img + (2 * r + c) * w16::SL<T>::ELEMS; }
-
-// Quadrant (i, k) of an operand held as four images: TR = false gives
-// M[i][k]; TR = true gives (M^T)[i][k] = M[k][i]^T.
-template <bool TR, class T> SELINV_DEVINL void qget(w16::Tile<T> &o, T *img, int i, int k, int g, int t)
-{
-    if (TR) w16::from_smem_T<T>(o, quad(img, k, i), g, t);
-    else w16::from_smem<T>(o, quad(img, i, k), g, t);
-}
-
-// acc += (NEG ? -1 : 1) (X Y^T)_{IJ} = sum_K X_IK Y_JK^T, operands from images.
-template <bool NEG, bool TX, bool TY, bool LOWER, class T>
-SELINV_DEVINL void qgemm(w16::Tile<T> &acc, T *imgX, T *imgY, int I, int J, T *s1, T *s2, int g, int t)
-{
-#pragma unroll
-    for (int K = 0; K < 2; ++K) {
-        w16::Tile<T> x, y;
-        qget<TX>(x, imgX, I, K, g, t);
-        qget<TY>(y, imgY, J, K, g, t);
-        w16::gemm_nt<NEG, LOWER>(acc, x, y, s1, s2, g, t);
-    }
-}
-
-// Lower triangle of a diagonal block (row-major b x b, identity pad beyond b)
-// into the quadrant images (0,0), (1,0), (1,1); FULL: cp.async chunks.
-template <class T, bool FULL> SELINV_DEVINL void load_diag(T *img, const T *D, int b, int tid)
-{
-    constexpr int CH = 16 / sizeof(T);
-    if (FULL) {
-        for (int j = tid; j < 32 * (32 / CH); j += GT) {
-            const int r = j / (32 / CH), c = (j % (32 / CH)) * CH;
-            if (c <= r) cp_async16(quad(img, r >> 4, c >> 4) + w16::SL<T>::idx(r & 15, c & 15), D + r * 32 + c);
-        }
-    } else {
-        for (int j = tid; j < 1024; j += GT) {
-            const int r = j >> 5, c = j & 31;
-            if (c <= r)
-                quad(img, r >> 4, c >> 4)[w16::SL<T>::idx(r & 15, c & 15)] =
-                    (r < b && c < b) ? __ldg(D + r * b + c) : (r == c ? T(1) : T(0));
-        }
-    }
-}
-
-// A full off-diagonal block (row-major b x b, zero pad) into four images.
-template <class T, bool FULL> SELINV_DEVINL void load_full(T *img, const T *B, int b, int tid)
-{
-    constexpr int CH = 16 / sizeof(T);
-    if (FULL) {
-        for (int j = tid; j < 32 * (32 / CH); j += GT) {
-            const int r = j / (32 / CH), c = (j % (32 / CH)) * CH;
-            cp_async16(quad(img, r >> 4, c >> 4) + w16::SL<T>::idx(r & 15, c & 15), B + r * 32 + c);
-        }
-    } else {
-        for (int j = tid; j < 1024; j += GT) {
-            const int r = j >> 5, c = j & 31;
-            quad(img, r >> 4, c >> 4)[w16::SL<T>::idx(r & 15, c & 15)] = (r < b && c < b) ? __ldg(B + r * b + c) : T(0);
-        }
-    }
-}
-
-// The warp's quadrant of the symmetric block whose lower quadrants are in img.
-template <class T> SELINV_DEVINL void sym_quad(w16::Tile<T> &o, T *img, int I, int J, int g, int t)
-{
-    if (I == J) w16::from_smem_lower<T>(o, quad(img, I, J), g, t);
-    else if (I > J) w16::from_smem<T>(o, quad(img, I, J), g, t);
-    else w16::from_smem_T<T>(o, quad(img, J, I), g, t);
-}
-
-// Store a quadrant tile into a row-major b x b block (TR: transposed position).
-template <class T, bool TR> SELINV_DEVINL void store_quad(T *G, const w16::Tile<T> &a, int b, int I, int J, int g, int t)
-{
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            int r = 16 * I + g + 8 * h, c = 16 * J + w16::tcol(t, q);
-            if (TR) {
-                const int tmp = r;
-                r = c;
-                c = tmp;
-            }
-            if (r < b && c < b) G[r * b + c] = a.v[h][q];
-        }
-}
-
-// CTA-group inverse of a symmetric positive definite 32 x 32 block held as
-// quadrant tiles: the symmetric Gauss-Jordan sweep (A_ij -= A_ik A_kj / d,
-// A_ik /= d, A_kj /= d, A_kk = -1/d, then negate); pivots -> det, bad.
-template <class T>
-SELINV_DEVINL void qinverse_scalar(w16::Tile<T> &a, T *cbuf, int I, int J, int g, int t, int bar, LogAcc &det,
-                                   bool &bad)
-{
-    using V = typename w16::Vec2<T>::type;
-    for (int kb = 0; kb < 2; ++kb) {
-#pragma unroll
-        for (int kk = 0; kk < 16; ++kk) {
-            const int k = 16 * kb + kk;
-            const int kh = kk >> 3, kt = (kk & 7) >> 1, kq = (kk & 1) | ((kk >> 3) << 1);
-            T *cb = cbuf + 32 * (kk & 1);
-            const bool col_owner = (J == kb) && (t == kt);
-            if (col_owner) {
-                cb[16 * I + g] = a.v[0][kq];
-                cb[16 * I + g + 8] = a.v[1][kq];
-            }
-            group_bar(bar);
-            const T d = cb[k];
-            const T c0 = cb[16 * I + g], c1 = cb[16 * I + g + 8];
-            const V r01 = *reinterpret_cast<const V *>(cb + 16 * J + 2 * t);
-            const V r23 = *reinterpret_cast<const V *>(cb + 16 * J + 2 * t + 8);
-            const T row[4] = {r01.x, r01.y, r23.x, r23.y};
-            bad |= !(d > T(0));
-            det.mul((double)d);
-            const T p = recip(d);
-            const T tc[2] = {c0 * p, c1 * p};
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) a.v[h][q] = fma(-tc[h], row[q], a.v[h][q]);
-            if (col_owner) {
-                a.v[0][kq] = tc[0];
-                a.v[1][kq] = tc[1];
-            }
-            if (I == kb && g == (kk & 7)) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) a.v[kh][q] = row[q] * p;
-                if (col_owner) a.v[kh][kq] = -p;
-            }
-        }
-        det.renorm();
-    }
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) a.v[h][q] = -a.v[h][q];
-}
-
-// float64: four block steps of eight pivots.  Block K (rows and columns
-// 8K..8K+7) lies in quadrant kq = K >> 1, half kh = K & 1.  The diagonal warp
-// (kq, kq) inverts the pivot block P = A_KK in registers (shuffle-only sweep;
-// pivots -> det, bad) and publishes P^-1; the warps of quadrant column kq
-// publish block column K.  After one group barrier each warp updates its four
-// 8 x 8 subtiles (r, c) on the FP64 tensor cores:
-//   r, c != K:  A_rc -= T_r A_cK^T,  T_r = A_rK P^-1
-//   c == K:     A_rK = T_r;    r == K:  A_Kc = P^-1 A_cK^T;    A_KK = -P^-1
-// (the m8n8k4 k index runs over 2t, 2t + 1 of the block, the accumulator
-// layout itself).  The two broadcast buffers alternate between block steps,
-// so one barrier per step suffices.  Only the diagonal warps see the pivots.
-constexpr int QBUF = 32 * 8 + 8 * 8;
-
-SELINV_DEVINL void qinverse_blocked(w16::Tile<double> &a, double *buf, int I, int J, int g, int t, int bar,
-                                    LogAcc &det, bool &bad)
-{
-    const int lane = 4 * g + t;
-#pragma unroll
-    for (int K = 0; K < 4; ++K) {
-        const int kq = K >> 1, kh = K & 1;
-        double *col = buf + (K & 1) * QBUF;            // block column K, [32][8]
-        double *pin = col + 32 * 8;                     // P^-1, [8][8]
-        if (J == kq) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-                *reinterpret_cast<double2 *>(col + (16 * I + g + 8 * h) * 8 + 2 * t) =
-                    make_double2(a.v[h][2 * kh], a.v[h][2 * kh + 1]);
-            if (I == kq) {
-                double pv[2] = {a.v[kh][2 * kh], a.v[kh][2 * kh + 1]};
-                inv8_sweep(pv, lane, g, t, det, bad, true);
-                det.renorm();
-                *reinterpret_cast<double2 *>(pin + g * 8 + 2 * t) = make_double2(pv[0], pv[1]);
-            }
-        }
-        group_bar(bar);
-        const double2 pi = *reinterpret_cast<const double2 *>(pin + g * 8 + 2 * t);
-        double2 ar[2], ac[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            ar[h] = *reinterpret_cast<const double2 *>(col + (16 * I + g + 8 * h) * 8 + 2 * t);
-            ac[h] = *reinterpret_cast<const double2 *>(col + (16 * J + g + 8 * h) * 8 + 2 * t);
-        }
-        double tr[2][2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {                   // T_r = A_rK P^-1
-            tr[h][0] = tr[h][1] = 0.0;
-            dmma_8x8x4(tr[h][0], tr[h][1], ar[h].x, pi.x);
-            dmma_8x8x4(tr[h][0], tr[h][1], ar[h].y, pi.y);
-        }
-#pragma unroll
-        for (int h = 0; h < 2; ++h)                     // A_rc -= T_r A_cK^T
-#pragma unroll
-            for (int n = 0; n < 2; ++n) {
-                dmma_8x8x4(a.v[h][2 * n], a.v[h][2 * n + 1], -tr[h][0], ac[n].x);
-                dmma_8x8x4(a.v[h][2 * n], a.v[h][2 * n + 1], -tr[h][1], ac[n].y);
-            }
-        if (J == kq) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                a.v[h][2 * kh] = tr[h][0];
-                a.v[h][2 * kh + 1] = tr[h][1];
-            }
-        }
-        if (I == kq) {
-#pragma unroll
-            for (int n = 0; n < 2; ++n) {               // A_Kc = P^-1 A_cK^T
-                double u0 = 0.0, u1 = 0.0;
-                dmma_8x8x4(u0, u1, pi.x, ac[n].x);
-                dmma_8x8x4(u0, u1, pi.y, ac[n].y);
-                a.v[kh][2 * n] = u0;
-                a.v[kh][2 * n + 1] = u1;
-            }
-            if (J == kq) {
-                a.v[kh][2 * kh] = -pi.x;
-                a.v[kh][2 * kh + 1] = -pi.y;
-            }
-        }
-    }
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) a.v[h][q] = -a.v[h][q];
-}
-
-template <class T>
-SELINV_DEVINL void qinverse(w16::Tile<T> &a, T *cbuf, int I, int J, int g, int t, int bar, LogAcc &det, bool &bad)
-{
-    if constexpr (sizeof(T) == 8) qinverse_blocked(a, cbuf, I, J, g, t, bar, det, bad);
-    else qinverse_scalar(a, cbuf, I, J, g, t, bar, det, bad);
-}
-
-// Copy n elements (a multiple of 16 bytes) from shared to global memory, or
-// stage them from global to shared (cp.async; the caller commits / waits).
-template <class T> SELINV_DEVINL void copy_out(T *dst, const T *src, int n, int gtid)
-{
-    using V = typename w16::Vec2<T>::type;
-    constexpr int CH = 16 / sizeof(T);
-    for (int k = gtid; k < n / CH; k += GT) {
-        const V *s4 = reinterpret_cast<const V *>(src + k * CH);
-        V *d4 = reinterpret_cast<V *>(dst + k * CH);
-        d4[0] = s4[0];
-        if (CH == 4) d4[1] = s4[1];
-    }
-}
-template <class T> SELINV_DEVINL void stage_in(T *dst, const T *src, int n, int gtid)
-{
-    constexpr int CH = 16 / sizeof(T);
-    for (int k = gtid; k < n / CH; k += GT) cp_async16(dst + k * CH, src + k * CH);
-}
+using namespace q32;
 
 template <class T, bool FULL, bool WANT_G>
 __global__ void __launch_bounds__(2 * GT) chain_mid_kernel(ChainArgs<T> p)

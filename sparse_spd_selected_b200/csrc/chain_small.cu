@@ -114,7 +114,8 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
         from_smem_lower<T>(dn, sD, g, t);             // D_{i+1}
         zero(w);
         gemm_nt<false>(w, bt, a, sT, sT2, g, t);      // W_i = B_i S_i^-1  (S_i^-1 symmetric)
-        gemm_nt<true>(dn, w, bt, sT, sT2, g, t);      // S_{i+1} = D_{i+1} - W_i B_i^T
+        gemm_nt<true, true>(dn, w, bt, sT, sT2, g, t);   // S_{i+1} = D_{i+1} - W_i B_i^T (lower tiles)
+        mirror_upper(dn, g, t);                       // upper-right tile from the lower-left one
         a = dn;
 
         if (WANT_X) {                                 // y_{i+1} = r_{i+1} - W_i y_i

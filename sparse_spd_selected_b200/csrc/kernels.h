@@ -32,6 +32,13 @@ template <class T> cudaError_t chain_small_launch(const ChainArgs<T> &a, bool al
 size_t chain_mid_workspace(size_t elem, int64_t batch, int64_t L);
 template <class T> cudaError_t chain_mid_launch(const ChainArgs<T> &a, cudaStream_t s);
 
+// 16 < b <= 32 with G and no right-hand side, long chains and a batch too
+// small to fill the GPU: P segments per chain, one 4-warp CTA each (0 = not
+// used; depends on the current device's SM count).
+int chain_seg_parts(int64_t batch, int64_t L, int b, bool want_g, bool want_x);
+size_t chain_seg_workspace(size_t elem, int64_t batch, int64_t L, int b, int P, bool want_g);
+template <class T> cudaError_t chain_seg_launch(const ChainArgs<T> &a, int P, cudaStream_t s);
+
 // 16 < b <= 128: one CTA per chain.
 size_t chain_large_workspace(size_t elem, int64_t batch, int64_t L, int b);
 template <class T> cudaError_t chain_large_launch(const ChainArgs<T> &a, cudaStream_t s);

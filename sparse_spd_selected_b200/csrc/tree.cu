@@ -223,9 +223,11 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
     const int g = lane >> 2, t = lane & 3;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     T *base = reinterpret_cast<T *>(smem_raw) + wid * dist_smem_elems<T>();
-    T *sBuf[2] = {base, base + E};                    // E_v of the current / next node
+    // buffers of the current / next node (c = 0, 1), addressed arithmetically so
+    // that no pointer array ends up in local memory
+    auto sBuf = [&](int c) { return base + c * E; };                      // E_v
     T *sG = base + 2 * E, *sT = sG + E, *sT2 = sT + E;
-    T *stg[2] = {sT2 + E, sT2 + E + SLOT_ELEMS};     // S_v^-1 slots, current / next
+    auto stg = [&](int c) { return sT2 + E + c * SLOT_ELEMS; };          // S_v^-1 slots
     const int b = p.b;
     const int64_t bb = (int64_t)b * b;
     const unsigned long long cnt = (unsigned long long)count;
@@ -238,8 +240,8 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
     int cur = 0;
     if (k < cnt) {
         const int32_t v0 = nodes[k];
-        load_block_async<T, FULL>(sBuf[0], p.edge + v0 * bb, b, lane);
-        stage_lower_slot<T>(stg[0], p.ws_sinv + (int64_t)v0 * SLOT_ELEMS, lane, g, t);
+        load_block_async<T, FULL>(sBuf(0), p.edge + v0 * bb, b, lane);
+        stage_lower_slot<T>(stg(0), p.ws_sinv + (int64_t)v0 * SLOT_ELEMS, lane, g, t);
         cp_async_commit();
     }
     while (k < cnt) {
@@ -260,8 +262,8 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
         cp_async_commit();
         if (kn < cnt) {
             const int32_t vn = nodes[kn];
-            load_block_async<T, FULL>(sBuf[cur ^ 1], p.edge + vn * bb, b, lane);
-            stage_lower_slot<T>(stg[cur ^ 1], p.ws_sinv + (int64_t)vn * SLOT_ELEMS, lane, g, t);
+            load_block_async<T, FULL>(sBuf(cur ^ 1), p.edge + vn * bb, b, lane);
+            stage_lower_slot<T>(stg(cur ^ 1), p.ws_sinv + (int64_t)vn * SLOT_ELEMS, lane, g, t);
             cp_async_commit();
             cp_async_wait_one();
         } else {
@@ -275,26 +277,20 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
             continue;
         }
         Tile<T> a;
-        unstage_lower_slot<T>(a, stg[cur], lane, g, t);
+        unstage_lower_slot<T>(a, stg(cur), lane, g, t);
         to_smem<T>(sT, a, g, t);                      // lower entries of S_v^-1 valid
         __syncwarp();
         from_smem_lower<T>(a, sT, g, t);              // S_v^-1, full
-        Tile<T> gp, et, w, wt, ge, get;
+        Tile<T> gp, et, wt, get;
         from_smem_lower<T>(gp, sG, g, t);             // G_pp, full
-        from_smem<T>(et, sBuf[cur], g, t);            // E_v
-        zero(w);
-        gemm_nt<false>(w, et, a, sT, sT2, g, t);      // W_v = E_v S_v^-1
-        __syncwarp();
-        to_smem<T>(sT, w, g, t);
-        __syncwarp();
-        from_smem_T<T>(wt, sT, g, t);                 // W_v^T
-        zero(ge);
-        gemm_nt<true>(ge, gp, wt, sT, sT2, g, t);     // G_edge[v] = -G_pp W_v
-        store_block<T, FULL>(p.G_edge + v * bb, ge, b, g, t);
-        __syncwarp();
-        to_smem<T>(sT2, ge, g, t);
-        __syncwarp();
-        from_smem_T<T>(get, sT2, g, t);               // G_edge[v]^T
+        from_smem<T>(et, sBuf(cur), g, t);            // E_v
+        // W_v^T = S_v^-1 E_v^T and G_edge[v]^T = -W_v^T G_pp are X Y^T products of
+        // register tiles (S_v^-1, G_pp symmetric): nothing is transposed.
+        zero(wt);
+        gemm_nt<false>(wt, a, et, sT, sT2, g, t);     // W_v^T = S_v^-1 E_v^T
+        zero(get);
+        gemm_nt<true>(get, wt, gp, sT, sT2, g, t);    // G_edge[v]^T = -W_v^T G_pp
+        store_block_T<T, FULL>(p.G_edge + v * bb, get, b, g, t);
         gemm_nt<true, true>(a, wt, get, sT, sT2, g, t);   // G_vv = S_v^-1 - W_v^T G_edge[v] (lower tiles)
         __syncwarp();
         to_smem<T>(sT, a, g, t);

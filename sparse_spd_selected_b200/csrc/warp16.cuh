@@ -452,6 +452,19 @@ template <class T> SELINV_DEVINL void spd_inverse(Tile<T> &a, T *cbuf, int g, in
     else spd_inverse_scalar(a, cbuf, g, t, det, bad);
 }
 
+// Upper-right 8 x 8 tile of a symmetric tile set to the transpose of the
+// lower-left one, by shuffles: lane (g, t) takes A[8 + 2t + j][g] from lane
+// 4 (2t + j) + g / 2, register g & 1.
+template <class T> SELINV_DEVINL void mirror_upper(Tile<T> &a, int g, int t)
+{
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int src = ((2 * t + j) << 2) | (g >> 1);
+        const T u0 = shfl(a.v[1][0], src), u1 = shfl(a.v[1][1], src);
+        a.v[0][2 + j] = (g & 1) ? u1 : u0;
+    }
+}
+
 // y_r = sum_c A[r][c] x[c] for the lane's rows g, g + 8 (x in shared memory);
 // every lane of a row group ends with the full sums.
 template <class T> SELINV_DEVINL void row_matvec(T out[2], const Tile<T> &a, const T *x, int t)

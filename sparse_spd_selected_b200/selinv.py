@@ -55,6 +55,8 @@ def lib():
         L.selinv_max_block.restype = I32
         L.selinv_chain_workspace_size.argtypes = [ctypes.c_int, I64, I64, I32, I32, I32]
         L.selinv_chain_workspace_size.restype = SZ
+        L.selinv_chain_segments.argtypes = [I64, I64, I32, I32, I32]
+        L.selinv_chain_segments.restype = I32
         L.selinv_chain.argtypes = [ctypes.c_int, I64, I64, I32, P, P, P, P, P, P, P, P, P, SZ, P]
         L.selinv_chain.restype = ctypes.c_int
         L.chain_solve.argtypes = [ctypes.c_int, I64, I64, I32, P, P, P, P, P, P, P, SZ, P]
@@ -115,6 +117,11 @@ def _check(status, what):
 
 def chain_workspace_size(dtype, batch, L, b, want_g=True, want_x=False) -> int:
     return int(lib().selinv_chain_workspace_size(_code(dtype), batch, L, b, int(want_g), int(want_x)))
+
+
+def chain_segments(batch, L, b, want_g=True, want_x=False) -> int:
+    """Segments per chain selinv_chain uses for these sizes on the current device (0: none)."""
+    return int(lib().selinv_chain_segments(batch, L, b, int(want_g), int(want_x)))
 
 
 def _workspace(nbytes, device, workspace):

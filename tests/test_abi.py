@@ -86,3 +86,18 @@ def test_tree_plan_rejects_malformed_parents(lib):
     assert plan([-1, 5, 0]) == selinv.ERR_BAD_TREE           # out of range
     assert plan([[-1, 0, 1], [-1, -1, 0]]) == selinv.ERR_BAD_TREE   # second tree has two roots
     assert lib.selinv_tree_plan(None, 1, 3, ctypes.byref(ctypes.c_void_p())) == selinv.ERR_INVALID_ARG
+
+
+def test_segment_rules(lib):
+    """Only 16 < b <= 32 chains with G, no solve, L >= 96 and a small batch are cut."""
+    f = lib.selinv_chain_segments
+    f.restype = ctypes.c_int32
+    f.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
+    assert f(2, 600, 32, 1, 0) >= 3
+    assert f(2, 600, 16, 1, 0) == 0          # warp kernel
+    assert f(2, 600, 33, 1, 0) == 0          # CTA kernel
+    assert f(2, 600, 32, 0, 0) == 0          # log det only: two-ended kernel
+    assert f(2, 600, 32, 1, 1) == 0          # with a solve
+    assert f(2, 95, 32, 1, 0) == 0           # too short
+    assert f(100000, 4096, 32, 1, 0) == 0    # batch fills the GPU
+    assert f(1, 10 ** 6, 32, 1, 0) == 16     # at most 16 segments

@@ -252,3 +252,41 @@ def test_two_ended_logdet_only_and_not_spd(cuda_ok):
     out = selinv.selinv_chain(to_dev(bad, torch.float64), l, check=False)
     info = host(out["info"]).tolist()
     assert info[0] == -1 and info[3] == -1 and info[1] >= 0 and info[2] >= 0
+
+
+@pytest.mark.parametrize("batch,L,b", [(2, 600, 32), (3, 200, 20), (1, 96, 32), (5, 401, 17)])
+def test_segmented_chains_f64(cuda_ok, batch, L, b):
+    """Chains cut into segments (separators eliminated last) against the oracle's
+    sequential elimination: every block of G, log det."""
+    assert selinv.chain_segments(batch, L, b) >= 3
+    diag, lower, _ = inputs.chain_inputs(batch, L, b, seed=7000 + L + b, load=0.5, with_rhs=False)
+    errs, out = run_both(diag, lower, None, torch.float64)
+    assert max(errs.values()) <= TOL[torch.float64], errs
+    Gd = out["G_diag"]
+    assert torch.equal(Gd, Gd.transpose(-1, -2))
+
+
+def test_segmented_chains_f32(cuda_ok):
+    assert selinv.chain_segments(2, 300, 32) >= 3
+    diag, lower, _ = inputs.chain_inputs(2, 300, 32, seed=7100, load=1.0, with_rhs=False)
+    errs, _ = run_both(diag, lower, None, torch.float32)
+    assert max(errs.values()) <= TOL[torch.float32], errs
+
+
+def test_segmented_logdet_only_and_not_spd(cuda_ok):
+    """Log det without G (two-ended kernel) agrees with the segmented call; a
+    chain that is not positive definite is reported, its neighbours are not."""
+    diag, lower, _ = inputs.chain_inputs(3, 300, 32, seed=7200, load=1.0, with_rhs=False)
+    d, l = to_dev(diag, torch.float64), to_dev(lower, torch.float64)
+    assert selinv.chain_segments(3, 300, 32) >= 3 and selinv.chain_segments(3, 300, 32, want_g=False) == 0
+    full = selinv.selinv_chain(d, l)
+    only = selinv.selinv_chain(d, l, want_g=False)
+    assert logdet_err(host(only["logdet"]), host(full["logdet"])) <= 1e-12
+    bad = diag.copy()
+    bad[1, 150] = -np.eye(32)
+    bad[2, [7, 100, 299]] = -np.eye(32)
+    out = selinv.selinv_chain(to_dev(bad, torch.float64), l, check=False)
+    info = host(out["info"]).tolist()
+    assert info[0] == -1 and info[1] >= 0 and info[2] >= 0
+    with pytest.raises(selinv.NotSPDError):
+        selinv.selinv_chain(to_dev(bad, torch.float64), l)
