@@ -598,6 +598,10 @@ __global__ void __launch_bounds__(Geo<BP>::NT) chain_large_kernel(ChainArgs<T> p
     // ---------------- collect sweep ----------------
     for (int64_t i = 0; i < L; ++i) {
         bool bad = false;
+        if (i + 1 < L) {                           // next blocks into L2 while this one is inverted
+            prefetch_range_l2(D + (i + 1) * bb, bb, x.tid, Geo<BP>::NT);
+            if (i + 1 < L - 1) prefetch_range_l2(Bl + (i + 1) * bb, bb, x.tid, Geo<BP>::NT);
+        }
         if constexpr (sizeof(T) == 8) spd_inverse_blocked<BP>(a, pbuf, pbuf + 2 * BP * 8, x, det, bad);
         else spd_inverse<T, BP>(a, colbuf, x, det, bad);
         if (bad && fail < 0) fail = (int)i;
@@ -666,6 +670,7 @@ __global__ void __launch_bounds__(Geo<BP>::NT) chain_large_kernel(ChainArgs<T> p
     for (int64_t i = L - 2; i >= 0; --i) {
         const T *Sinv = ws + (2 * i) * BB;
         const T *W = ws + (2 * i + 1) * BB;
+        if (i > 0) prefetch_range_l2(ws + (2 * i - 2) * BB, 2 * BB, x.tid, Geo<BP>::NT);   // S_{i-1}^-1, W_{i-1}
         if (WANT_G) {
             zero(a);
             gemm<T, BP, OP_BIG, OP_ROWPANEL, true, FULL>(a, big, pbuf, W, b, x);          // G_{i+1,i} = -G_{i+1,i+1} W_i

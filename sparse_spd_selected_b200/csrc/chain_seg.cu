@@ -394,7 +394,10 @@ template <class T> __global__ void seg_finalize_kernel(ChainArgs<T> p, SegArgs<T
 
 // Segment boundaries: end segments RHO times as long as interior ones (the
 // interior blocks carry the fill products).
-constexpr double RHO = 1.4;
+#ifndef SELINV_SEG_RHO
+#define SELINV_SEG_RHO 1.7
+#endif
+constexpr double RHO = SELINV_SEG_RHO;
 
 SegGeo seg_geometry(int64_t L, int P)
 {
@@ -500,7 +503,10 @@ int chain_seg_parts(int64_t batch, int64_t L, int b, bool want_g, bool want_x)
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     // three distribute CTAs fit on an SM; the two-ended kernel already covers
     // two groups per chain
-    const int64_t slots = 3 * (int64_t)sms;
+#ifndef SELINV_SEG_SLOTS
+#define SELINV_SEG_SLOTS 3
+#endif
+    const int64_t slots = SELINV_SEG_SLOTS * (int64_t)sms;
     int64_t P = std::min<int64_t>(SEG_MAX, slots / batch);
     P = std::min<int64_t>(P, L / 32);
     return P >= 3 ? (int)P : 0;

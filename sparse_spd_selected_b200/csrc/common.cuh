@@ -23,6 +23,16 @@ SELINV_DEVINL void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" :::
 // Wait until at most one committed group (the most recent) is still in flight.
 SELINV_DEVINL void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 
+// Prefetch into L2 every 128-byte line of n elements at p (lines split over
+// nthreads threads; every address issued lies inside the range).
+SELINV_DEVINL void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];\n" ::"l"(p)); }
+template <class T> SELINV_DEVINL void prefetch_range_l2(const T *p, int64_t n, int tid, int nthreads)
+{
+    const char *c = reinterpret_cast<const char *>(p);
+    const int64_t bytes = n * (int64_t)sizeof(T);
+    for (int64_t off = (int64_t)tid * 128; off < bytes; off += (int64_t)nthreads * 128) prefetch_l2(c + off);
+}
+
 // Read-only global loads that should not linger in L1.
 template <class T> SELINV_DEVINL T ldg_stream(const T *p) { return __ldcs(p); }
 
