@@ -20,6 +20,7 @@ tests check against) on a bounded sample of the same workload instead.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -56,6 +57,8 @@ def parse():
     ap.add_argument("--workload", default="chain_4096x64_b16", choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--dtype", default="f64", choices=["f64", "f32"])
     ap.add_argument("--batch", type=int, default=None, help="override the per-GPU batch (profiling runs)")
+    ap.add_argument("--length", type=int, default=None,
+                    help="override the chain length / tree size (profiling runs of a smaller case)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -298,6 +301,9 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
 
     w = inputs.WORKLOADS[args.workload]
+    full_size = args.length is None and (args.batch is None or args.batch == w.batch)
+    if args.length is not None:
+        w = dataclasses.replace(w, L=args.length)
     batch = args.batch or w.batch
     tdt = torch.float64 if args.dtype == "f64" else torch.float32
     es = 8 if args.dtype == "f64" else 4
@@ -428,7 +434,7 @@ def run_ours(args):
     hbm_achieved = byt / (kernel_ms / 1e3) / 1e9
     flops = algorithmic_flops(w, batch)
     flop_rate = flops / (kernel_ms / 1e3) / 1e12
-    traffic = profiled_traffic(kernel, w.name) if batch == w.batch else None
+    traffic = profiled_traffic(kernel, w.name) if full_size else None
     hbm_src = f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback 6650 GB/s"
     if w.b >= 32 and args.dtype == "f64":
         # arithmetic intensity 7 b^3 / (32 b^2) flop/byte: past the FP64 ridge from b = 32 on
@@ -460,7 +466,7 @@ def run_ours(args):
         "value": value, "unit": "blocks/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": args.dtype, "data": "synthetic",
-        "config": {"workload": w.name if batch == w.batch else f"{w.name} (batch {batch} per GPU)",
+        "config": {"workload": w.name if full_size else f"{w.name} (batch {batch}, length {w.L} per GPU)",
                    "global_batch": batch * world, "block": w.b, "L_or_n": w.L,
                    "solve": bool(w.solve), "parallelism": f"dp{world} (independent chains per GPU)",
                    "l2": "inputs larger than L2 (no flush)"},

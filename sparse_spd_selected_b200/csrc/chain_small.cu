@@ -31,9 +31,6 @@ constexpr int WARPS = 4;
 #ifndef SELINV_CHAIN_MINB
 #define SELINV_CHAIN_MINB 4
 #endif
-#ifndef SELINV_COLLECT_MINB
-#define SELINV_COLLECT_MINB 4
-#endif
 
 template <class T> __host__ __device__ constexpr int warp_smem_elems()
 {
@@ -41,8 +38,7 @@ template <class T> __host__ __device__ constexpr int warp_smem_elems()
 }
 
 template <class T, bool FULL, bool WANT_G, bool WANT_X>
-__global__ void __launch_bounds__(WARPS * 32, (WANT_G || WANT_X) ? SELINV_CHAIN_MINB : SELINV_COLLECT_MINB)
-    chain_small_kernel(ChainArgs<T> p)
+__global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_kernel(ChainArgs<T> p)
 {
     using namespace w16;
     constexpr int E = SL<T>::ELEMS;
