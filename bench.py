@@ -358,7 +358,7 @@ def run_ours(args):
             kernel = "chain_small_kernel"
         elif segments > 0:
             # segments' collect, separators' D', their two-ended chain, segments' distribute, log det
-            kernel = "seg_distribute_kernel"
+            kernel = "seg_collect_kernel"
             launches_per_step = 5
         elif b <= 32 and "rhs" not in dev_in:
             kernel = "chain_mid_kernel"
