@@ -18,10 +18,10 @@
 // quadrant (I, J) = (w >> 1, w & 1) of every 32 x 32 block as a 16 x 16
 // register tile; products X Y^T are sums of two tile products whose operand
 // quadrants come from shared images, each a register-register FP64
-// tensor-core product; the 32 x 32 inverse is the symmetric Gauss-Jordan
-// sweep over the group: float64 in four blocks of eight pivots (one named
-// barrier per block, the block updates on the tensor cores), float32 one
-// pivot per barrier.
+// tensor-core product.  The 32 x 32 inverse: float64 through the quadrant
+// Schur complement (the diagonal warps invert A and S = C - B A^-1 B^T in
+// their own registers, three group barriers), float32 the symmetric
+// Gauss-Jordan sweep over the group, one pivot per barrier.
 #include "kernels.h"
 #include "quad32.cuh"
 

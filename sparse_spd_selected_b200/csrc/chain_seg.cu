@@ -86,7 +86,7 @@ template <class T> struct SegLay {
     static constexpr int E = w16::SL<T>::ELEMS;
     static constexpr int IMG = 4 * E;
     static constexpr int SCR = sizeof(T) == 4 ? 2 * E * GW : 0;
-    static constexpr int CBN = sizeof(T) == 8 ? 2 * QBUF : 64;
+    static constexpr int CBN = sizeof(T) == 8 ? QSCHUR : 64;
     // collect: C, D, X (S^-1), Y (W), V, F
     static constexpr int C = 0, D = IMG, X = 2 * IMG, Y = 3 * IMG, V = 4 * IMG, F = 5 * IMG;
     static constexpr int CS = 6 * IMG, CCB = CS + SCR, CTOTAL = CCB + CBN;

@@ -23,7 +23,7 @@ template <class T> struct Lay {        // per-group shared memory of the two-end
     static constexpr int SCR = sizeof(T) == 4 ? 2 * E * GW : 0;   // float products: per-warp scratch
     static constexpr int C = 0, D = IMG, X = 2 * IMG, Y = 3 * IMG, Z = 4 * IMG, Z2 = 5 * IMG, S = 6 * IMG;
     static constexpr int CB = S + SCR;
-    static constexpr int CBN = sizeof(T) == 8 ? 2 * (32 * 8 + 8 * 8) : 64;   // inverse broadcast buffers
+    static constexpr int CBN = sizeof(T) == 8 ? 4 * 256 : 64;     // inverse scratch (four 16 x 16 images / pivot column)
     static constexpr int GROUP = CB + CBN;
     static constexpr int EXCH = 2 * GROUP;        // exchange image after both groups
     static constexpr int TOTAL = EXCH + IMG;
@@ -167,94 +167,72 @@ SELINV_DEVINL void qinverse_scalar(w16::Tile<T> &a, T *cbuf, int I, int J, int g
         for (int q = 0; q < 4; ++q) a.v[h][q] = -a.v[h][q];
 }
 
-// float64: four block steps of eight pivots.  Block K (rows and columns
-// 8K..8K+7) lies in quadrant kq = K >> 1, half kh = K & 1.  The diagonal warp
-// (kq, kq) inverts the pivot block P = A_KK in registers (shuffle-only sweep;
-// pivots -> det, bad) and publishes P^-1; the warps of quadrant column kq
-// publish block column K.  After one group barrier each warp updates its four
-// 8 x 8 subtiles (r, c) on the FP64 tensor cores:
-//   r, c != K:  A_rc -= T_r A_cK^T,  T_r = A_rK P^-1
-//   c == K:     A_rK = T_r;    r == K:  A_Kc = P^-1 A_cK^T;    A_KK = -P^-1
-// (the m8n8k4 k index runs over 2t, 2t + 1 of the block, the accumulator
-// layout itself).  The two broadcast buffers alternate between block steps,
-// so one barrier per step suffices.  Only the diagonal warps see the pivots.
-constexpr int QBUF = 32 * 8 + 8 * 8;
+// float64 through the 2 x 2 quadrant structure M = [[A, B^T], [B, C]]
+// (B = the (1,0) quadrant; M symmetric):
+//   T = B A^-1,  S = C - T B^T,
+//   M^-1 = [[A^-1 + T^T S^-1 T, -T^T S^-1], [-S^-1 T, S^-1]].
+// Warp (0,0) inverts A and warp (1,1) inverts S, each in its own registers
+// (two 8-pivot block steps, warp16.cuh; pivots -> det, bad), so the group
+// meets at three barriers only; every product is a register-register FP64
+// tensor-core product with operands from four 16 x 16 images in buf.
+constexpr int QSCHUR = 4 * w16::SL<double>::ELEMS;
 
-SELINV_DEVINL void qinverse_blocked(w16::Tile<double> &a, double *buf, int I, int J, int g, int t, int bar,
-                                    LogAcc &det, bool &bad)
+SELINV_DEVINL void qinverse_schur(w16::Tile<double> &a, double *buf, int I, int J, int g, int t, int bar,
+                                  LogAcc &det, bool &bad)
 {
-    const int lane = 4 * g + t;
-#pragma unroll
-    for (int K = 0; K < 4; ++K) {
-        const int kq = K >> 1, kh = K & 1;
-        double *col = buf + (K & 1) * QBUF;            // block column K, [32][8]
-        double *pin = col + 32 * 8;                     // P^-1, [8][8]
-        if (J == kq) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-                *reinterpret_cast<double2 *>(col + (16 * I + g + 8 * h) * 8 + 2 * t) =
-                    make_double2(a.v[h][2 * kh], a.v[h][2 * kh + 1]);
-            if (I == kq) {
-                double pv[2] = {a.v[kh][2 * kh], a.v[kh][2 * kh + 1]};
-                inv8_sweep(pv, lane, g, t, det, bad, true);
-                det.renorm();
-                *reinterpret_cast<double2 *>(pin + g * 8 + 2 * t) = make_double2(pv[0], pv[1]);
-            }
-        }
-        group_bar(bar);
-        const double2 pi = *reinterpret_cast<const double2 *>(pin + g * 8 + 2 * t);
-        double2 ar[2], ac[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            ar[h] = *reinterpret_cast<const double2 *>(col + (16 * I + g + 8 * h) * 8 + 2 * t);
-            ac[h] = *reinterpret_cast<const double2 *>(col + (16 * J + g + 8 * h) * 8 + 2 * t);
-        }
-        double tr[2][2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {                   // T_r = A_rK P^-1
-            tr[h][0] = tr[h][1] = 0.0;
-            dmma_8x8x4(tr[h][0], tr[h][1], ar[h].x, pi.x);
-            dmma_8x8x4(tr[h][0], tr[h][1], ar[h].y, pi.y);
-        }
-#pragma unroll
-        for (int h = 0; h < 2; ++h)                     // A_rc -= T_r A_cK^T
-#pragma unroll
-            for (int n = 0; n < 2; ++n) {
-                dmma_8x8x4(a.v[h][2 * n], a.v[h][2 * n + 1], -tr[h][0], ac[n].x);
-                dmma_8x8x4(a.v[h][2 * n], a.v[h][2 * n + 1], -tr[h][1], ac[n].y);
-            }
-        if (J == kq) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                a.v[h][2 * kh] = tr[h][0];
-                a.v[h][2 * kh + 1] = tr[h][1];
-            }
-        }
-        if (I == kq) {
-#pragma unroll
-            for (int n = 0; n < 2; ++n) {               // A_Kc = P^-1 A_cK^T
-                double u0 = 0.0, u1 = 0.0;
-                dmma_8x8x4(u0, u1, pi.x, ac[n].x);
-                dmma_8x8x4(u0, u1, pi.y, ac[n].y);
-                a.v[kh][2 * n] = u0;
-                a.v[kh][2 * n + 1] = u1;
-            }
-            if (J == kq) {
-                a.v[kh][2 * kh] = -pi.x;
-                a.v[kh][2 * kh + 1] = -pi.y;
-            }
+    using namespace w16;
+    constexpr int E = SL<double>::ELEMS;
+    double *sAi = buf, *sB = buf + E, *sT = buf + 2 * E, *sSi = buf + 3 * E;
+    if (I == 0 && J == 0) {                                          // A^-1
+        spd_inverse_blocked(a, g, t, det, bad);
+        det.renorm();
+        to_smem<double>(sAi, a, g, t);
+    } else if (I == 1 && J == 0) {
+        to_smem<double>(sB, a, g, t);
+    }
+    group_bar(bar);
+    if (I == 1 && J == 0) {                                          // T = B A^-1
+        Tile<double> ai, tt;
+        from_smem<double>(ai, sAi, g, t);
+        zero(tt);
+        gemm_nt<false>(tt, a, ai, nullptr, nullptr, g, t);
+        to_smem<double>(sT, tt, g, t);
+        a = tt;
+    }
+    group_bar(bar);
+    if (I == 1 && J == 1) {                                          // S = C - T B^T, S^-1
+        Tile<double> tt, bq;
+        from_smem<double>(tt, sT, g, t);
+        from_smem<double>(bq, sB, g, t);
+        gemm_nt<true>(a, tt, bq, nullptr, nullptr, g, t);
+        spd_inverse_blocked(a, g, t, det, bad);
+        det.renorm();
+        to_smem<double>(sSi, a, g, t);
+    }
+    group_bar(bar);
+    if (!(I == 1 && J == 1)) {
+        Tile<double> si, tT;
+        from_smem<double>(si, sSi, g, t);
+        from_smem_T<double>(tT, sT, g, t);                         // T^T
+        if (I == 0 && J == 0) {                                      // A^-1 + T^T (S^-1 T)
+            Tile<double> ut;
+            zero(ut);
+            gemm_nt<false>(ut, tT, si, nullptr, nullptr, g, t);      // T^T S^-1
+            gemm_nt<false>(a, tT, ut, nullptr, nullptr, g, t);
+        } else if (I == 0) {                                         // -T^T S^-1
+            zero(a);
+            gemm_nt<true>(a, tT, si, nullptr, nullptr, g, t);
+        } else {                                                     // -S^-1 T
+            zero(a);
+            gemm_nt<true>(a, si, tT, nullptr, nullptr, g, t);
         }
     }
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) a.v[h][q] = -a.v[h][q];
 }
 
 template <class T>
 SELINV_DEVINL void qinverse(w16::Tile<T> &a, T *cbuf, int I, int J, int g, int t, int bar, LogAcc &det, bool &bad)
 {
-    if constexpr (sizeof(T) == 8) qinverse_blocked(a, cbuf, I, J, g, t, bar, det, bad);
+    if constexpr (sizeof(T) == 8) qinverse_schur(a, cbuf, I, J, g, t, bar, det, bad);
     else qinverse_scalar(a, cbuf, I, J, g, t, bar, det, bad);
 }
 
