@@ -95,6 +95,16 @@ SELINV_DEVINL int ld_acquire(const int32_t *p)
     return v;
 }
 
+// Atomic add with acquire-release semantics at GPU scope: releases the
+// caller's earlier writes (and, through a preceding warp barrier, its warp's)
+// and acquires every write released by earlier adds to the same counter.
+SELINV_DEVINL int atom_add_acq_rel(int32_t *p, int v)
+{
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
 SELINV_DEVINL void st_release(int32_t *p, int v)
 {
     asm volatile("st.release.gpu.global.s32 [%0], %1;\n" ::"l"(p), "r"(v) : "memory");
@@ -183,11 +193,8 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leave
                 Tile<T> z;
                 zero(z);
                 store_block<T, FULL>(p.G_edge + v * bb, z, b, g, t);
-                __syncwarp();
-                if (lane == 0) {
-                    __threadfence();
-                    st_release(sy.done + v, 1);
-                }
+                __syncwarp();                         // the warp's stores are ordered before lane 0's release
+                if (lane == 0) st_release(sy.done + v, 1);
                 __syncwarp();
                 break;
             }
@@ -199,14 +206,11 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leave
             zero(u);
             gemm_nt<false, true>(u, w, et, sT, sT2, g, t);   // U_v = W_v E_v^T (lower tiles)
             store_lower_slot<T>(p.ws_u + (int64_t)v * SLOT_ELEMS, u, lane, g, t);
-            __syncwarp();                             // the warp's stores are ordered before lane 0's fence
+            __syncwarp();                             // the warp's stores are ordered before lane 0's release
             int old = 0;
-            if (lane == 0) {
-                __threadfence();                      // release U_v before the count drops
-                old = atomicSub(sy.pending + par, 1);
-                if (old == 1) __threadfence();        // acquire every sibling's U
-            }
+            if (lane == 0) old = atom_add_acq_rel(sy.pending + par, -1);   // release U_v; the last child acquires all siblings'
             old = __shfl_sync(FULL_MASK, old, 0);
+            __syncwarp();                             // every lane's reads of the siblings' U follow lane 0's acquire
             if (old != 1) break;                      // a sibling is still running: it will go on
             v = par;
         }
@@ -297,11 +301,8 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
         __syncwarp();
         from_smem_lower<T>(a, sT, g, t);              // exactly symmetric
         store_block<T, FULL>(p.G_diag + v * bb, a, b, g, t);
-        __syncwarp();
-        if (lane == 0 && td.child_ptr[v + 1] > td.child_ptr[v]) {   // only parents are waited for
-            __threadfence();
-            st_release(sy.done + v, 1);
-        }
+        __syncwarp();                                 // the warp's stores are ordered before lane 0's release
+        if (lane == 0 && td.child_ptr[v + 1] > td.child_ptr[v]) st_release(sy.done + v, 1);   // only parents are waited for
         __syncwarp();
         k = kn;
         cur ^= 1;
