@@ -46,6 +46,8 @@ def _bind(path):
     lib.oracle_chain.restype = ctypes.c_int
     lib.oracle_tree.argtypes = [P, I64, I64, ctypes.c_int, P, P, P, P, P, P]
     lib.oracle_tree.restype = ctypes.c_int
+    lib.oracle_chain_sample.argtypes = [P, P, I64, I64, ctypes.c_int, P, P, P, P, P]
+    lib.oracle_chain_sample.restype = ctypes.c_int
     lib.oracle_threads.argtypes = []
     lib.oracle_threads.restype = ctypes.c_int
     return lib
@@ -108,6 +110,36 @@ def chain(diag, lower, rhs=None, want_g=True, lib=None):
         raise ValueError("oracle_chain: invalid arguments")
     return {"G_diag": G_diag, "G_lower": G_lower, "logdet": logdet, "x": x,
             "info": info, "asym": asym}
+
+
+def chain_sample(diag, lower, z, rhs=None, lib=None):
+    """Gaussian draw from the chain's own Cholesky factor A = L L^T:
+    eta = L^-T z (+ A^-1 rhs when rhs is given).
+
+    z [..., L, b] are the caller's standard normals.  Returns dict with eta
+    [..., L, b], logdet [...] and info [...] (-1 ok, else the first block
+    whose Schur complement is not positive definite).
+    """
+    diag = _f64(diag)
+    lead = diag.shape[:-3]
+    L, b = diag.shape[-3], diag.shape[-1]
+    batch = int(np.prod(lead)) if lead else 1
+    if lower is None or L == 1:
+        lower = np.zeros(lead + (max(L - 1, 0), b, b))
+    lower = _f64(lower)
+    z = _f64(z)
+    assert z.shape == lead + (L, b)
+    if rhs is not None:
+        rhs = _f64(rhs)
+        assert rhs.shape == lead + (L, b)
+    eta = np.empty(lead + (L, b))
+    logdet = np.empty(lead)
+    info = np.empty(lead, dtype=np.int32)
+    rc = _load(lib).oracle_chain_sample(_ptr(diag), _ptr(lower) if L > 1 else None, batch, L, b,
+                                        _ptr(rhs), _ptr(z), _ptr(eta), _ptr(logdet), _ptr(info))
+    if rc != 0:
+        raise ValueError("oracle_chain_sample: invalid arguments")
+    return {"eta": eta, "logdet": logdet, "info": info}
 
 
 def tree(parent, diag, edge, lib=None):

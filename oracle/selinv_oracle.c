@@ -248,6 +248,89 @@ int oracle_chain(const double *diag, const double *lower, int64_t batch, int64_t
     return 0;
 }
 
+/* ------------------------------ sampling --------------------------------- */
+
+/*
+ * Gaussian draw with the same factor (sparsax, PyPI page, "Factor once, do
+ * everything": sample_gaussian returns eta = A^-1 b + P^T L^-T z for the
+ * Cholesky factor A = P^T L L^T P; gabp-sparse-inv, "Gaussian sampling":
+ * x ~ N(0, A^-1) reusing the factorisation).  A chain is factorised in its
+ * own block order, so P = I and L is the block lower-bidiagonal Cholesky
+ * factor of A:
+ *   L_ii = R_i  (S_i = R_i R_i^T, R_i lower),   L_{i+1,i} = B_i R_i^-T.
+ * The draw w = L^-T z solves L^T w = z by block back substitution:
+ *   w_{L-1} = R_{L-1}^-T z_{L-1},
+ *   w_i     = R_i^-T (z_i - R_i^-1 B_i^T w_{i+1}).
+ * eta = x + w with x = A^-1 r (the solve above), or eta = w without r.
+ */
+static int chain_sample_one(int64_t L, int b, const double *diag, const double *lower,
+                            const double *rhs, const double *z, double *eta, double *logdet_out)
+{
+    const size_t bb = (size_t)b * b;
+    double *Rinv = malloc(sizeof(double) * bb * (size_t)L);   /* R_i^-1, all i */
+    double *S = malloc(sizeof(double) * bb);
+    double *R = malloc(sizeof(double) * bb);
+    double *Sinv = malloc(sizeof(double) * bb);
+    double *BS = malloc(sizeof(double) * bb);
+    double *BSB = malloc(sizeof(double) * bb);
+    double *v1 = malloc(sizeof(double) * (size_t)b);
+    double *v2 = malloc(sizeof(double) * (size_t)b);
+    int info = -1;
+    double logdet = 0.0;
+
+    /* the Cholesky factors R_i of the Schur complements, in block order */
+    sym_from_lower(b, diag, S);
+    for (int64_t i = 0; i < L; ++i) {
+        if (cholesky_lower(b, S, R) != 0) { info = (int)i; goto done; }
+        for (int k = 0; k < b; ++k) logdet += 2.0 * log(R[k * (b + 1)]);
+        lower_inverse(b, R, Rinv + bb * i);
+        if (i + 1 < L) {
+            const double *Bi = lower + bb * i;
+            matmul(b, Rinv + bb * i, 1, Rinv + bb * i, 0, Sinv);    /* S_i^-1 = R^-T R^-1 */
+            matmul(b, Bi, 0, Sinv, 0, BS);                           /* B_i S_i^-1 */
+            matmul(b, BS, 0, Bi, 1, BSB);                            /* B_i S_i^-1 B_i^T */
+            sym_from_lower(b, diag + bb * (i + 1), S);
+            for (size_t k = 0; k < bb; ++k) S[k] = S[k] - BSB[k];
+        }
+    }
+    if (logdet_out) *logdet_out = logdet;
+
+    /* w = L^-T z, back substitution; R_i^-T v = (R_i^-1)^T v */
+    matvec(b, Rinv + bb * (L - 1), 1, z + (size_t)b * (L - 1), eta + (size_t)b * (L - 1));
+    for (int64_t i = L - 2; i >= 0; --i) {
+        matvec(b, lower + bb * i, 1, eta + (size_t)b * (i + 1), v1);        /* B_i^T w_{i+1} */
+        matvec(b, Rinv + bb * i, 0, v1, v2);                                /* R_i^-1 B_i^T w_{i+1} */
+        for (int k = 0; k < b; ++k) v1[k] = z[(size_t)b * i + k] - v2[k];
+        matvec(b, Rinv + bb * i, 1, v1, eta + (size_t)b * i);              /* R_i^-T (...) */
+    }
+done:
+    free(Rinv); free(S); free(R); free(Sinv); free(BS); free(BSB); free(v1); free(v2);
+    if (info == -1 && rhs) {                                               /* + A^-1 r */
+        double *x = malloc(sizeof(double) * (size_t)b * (size_t)L);
+        info = chain_one(L, b, diag, lower, NULL, NULL, NULL, rhs, x, NULL);
+        for (size_t k = 0; k < (size_t)b * (size_t)L; ++k) eta[k] += x[k];
+        free(x);
+    }
+    return info;
+}
+
+/* Batched draws: z [batch,L,b] (standard normals, supplied by the caller),
+ * rhs [batch,L,b] or NULL, eta [batch,L,b] out, logdet [batch] or NULL. */
+int oracle_chain_sample(const double *diag, const double *lower, int64_t batch, int64_t L, int b,
+                        const double *rhs, const double *z, double *eta, double *logdet, int32_t *info)
+{
+    if (batch < 0 || L < 1 || b < 1 || !diag || !z || !eta || !info || (L > 1 && !lower)) return 1;
+    const size_t bb = (size_t)b * b;
+    int64_t e;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (e = 0; e < batch; ++e) {
+        info[e] = chain_sample_one(L, b, diag + bb * L * e, lower ? lower + bb * (L - 1) * e : NULL,
+                                   rhs ? rhs + (size_t)b * L * e : NULL, z + (size_t)b * L * e,
+                                   eta + (size_t)b * L * e, logdet ? logdet + e : NULL);
+    }
+    return 0;
+}
+
 /* -------------------------------- tree ---------------------------------- */
 
 /* One rooted tree (parent[root] = -1).  Collect in reverse breadth-first

@@ -15,7 +15,10 @@ Sources:
       ones.
     "Tests": every kernel against a dense fp64 oracle, symmetry / SPD
       properties, independent residuals, leading batch dimensions.
-  sparsax (PyPI page) "Quick start": the 3 x 3 SPD example.
+  sparsax (PyPI page) "Quick start": the 3 x 3 SPD example; "Factor once, do
+    everything": sample_gaussian draws eta = A^-1 b + P^T L^-T z from the
+    Cholesky factor (gabp-sparse-inv "Gaussian sampling": the covariance is
+    exactly A^-1, checked on the standard basis).
 """
 import json
 import math
@@ -326,6 +329,44 @@ def pin_not_spd(lib=None):
     return 0.0 if ok else 1.0
 
 
+def pin_sample_standard_basis(lib=None):
+    """Draws for z = e_k, k = 1..N, are the columns of L^-T with L = numpy's
+    Cholesky factor of the dense A (so W is upper triangular), and W W^T = A^-1:
+    the check the pages name for their sampler (the covariance is exactly A^-1
+    on the standard basis).  Log det against slogdet."""
+    worst = 0.0
+    for L, b, seed in [(3, 2, 61), (4, 3, 62), (1, 4, 63), (5, 1, 64)]:
+        d, l, _ = inputs.chain_inputs(1, L, b, seed=seed, load=1.0, with_rhs=False)
+        A = chain_dense(d[0], l[0])
+        N = L * b
+        Z = np.eye(N).reshape(N, L, b)
+        out = oracle.chain_sample(np.repeat(d, N, 0), np.repeat(l, N, 0), Z, lib=lib)
+        W = out["eta"].reshape(N, N).T
+        worst = max(worst, rel(W, np.linalg.inv(np.linalg.cholesky(A)).T))
+        worst = max(worst, rel(W @ W.T, np.linalg.inv(A)))
+        worst = max(worst, abs(out["logdet"][0] - np.linalg.slogdet(A)[1]) / max(1.0, abs(np.linalg.slogdet(A)[1])))
+        if (out["info"] != -1).any():
+            return float("inf")
+    return worst
+
+
+def pin_sample_mean(lib=None):
+    """z = 0 gives the solve A^-1 r; with both, eta = A^-1 r + L^-T z (numpy's
+    solve and Cholesky on the dense A)."""
+    d, l, r = inputs.chain_inputs(2, 5, 3, seed=65, load=0.8, with_rhs=True)
+    z = np.random.default_rng(66).standard_normal(r.shape)
+    zero = oracle.chain_sample(d, l, np.zeros_like(r), rhs=r, lib=lib)
+    both = oracle.chain_sample(d, l, z, rhs=r, lib=lib)
+    worst = 0.0
+    for e in range(2):
+        A = chain_dense(d[e], l[e])
+        mean = np.linalg.solve(A, r[e].ravel())
+        draw = np.linalg.inv(np.linalg.cholesky(A)).T @ z[e].ravel()
+        worst = max(worst, rel(zero["eta"][e].ravel(), mean))
+        worst = max(worst, rel(both["eta"][e].ravel(), mean + draw))
+    return worst
+
+
 # name -> (function, tolerance)
 PINS = {
     "tiny_chains_dense": (pin_tiny_chains_dense, 1e-12),
@@ -338,5 +379,7 @@ PINS = {
     "tiny_trees_dense": (pin_tiny_trees_dense, 1e-12),
     "tree_quickstart": (pin_tree_quickstart, 1e-10),
     "root_invariance": (pin_root_invariance, 1e-11),
+    "sample_standard_basis": (pin_sample_standard_basis, 1e-12),
+    "sample_mean": (pin_sample_mean, 1e-12),
     "not_spd": (pin_not_spd, 0.5),
 }

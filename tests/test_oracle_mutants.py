@@ -40,6 +40,14 @@ MUTANTS = {
                            "for (int64_t k = count[v] + 1; k < count[v + 1]; ++k) {"),
     "tree_edge_transposed": ("matmul(b, G_diag + bb * p, 0, edge + bb * v, 0, T1);",
                              "matmul(b, G_diag + bb * p, 0, edge + bb * v, 1, T1);"),
+    "sample_last_untransposed": ("matvec(b, Rinv + bb * (L - 1), 1, z + (size_t)b * (L - 1), eta + (size_t)b * (L - 1));",
+                                 "matvec(b, Rinv + bb * (L - 1), 0, z + (size_t)b * (L - 1), eta + (size_t)b * (L - 1));"),
+    "sample_coupling_transposed": ("matvec(b, lower + bb * i, 1, eta + (size_t)b * (i + 1), v1);",
+                                   "matvec(b, lower + bb * i, 0, eta + (size_t)b * (i + 1), v1);"),
+    "sample_sign": ("for (int k = 0; k < b; ++k) v1[k] = z[(size_t)b * i + k] - v2[k];",
+                    "for (int k = 0; k < b; ++k) v1[k] = z[(size_t)b * i + k] + v2[k];"),
+    "sample_schur_sign": ("for (size_t k = 0; k < bb; ++k) S[k] = S[k] - BSB[k];",
+                          "for (size_t k = 0; k < bb; ++k) S[k] = S[k] + BSB[k];"),
     "tree_g_diag_transposed": ("matmul(b, Sinv + bb * v, 0, edge + bb * v, 1, T1);",
                                "matmul(b, Sinv + bb * v, 0, edge + bb * v, 0, T1);"),
 }
