@@ -135,6 +135,34 @@ selinv_status chain_solve(selinv_dtype dtype, int64_t batch, int64_t L, int32_t 
                           void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Gaussian draw from the same factorisation (sparsax, "Factor once, do
+ * everything": sample_gaussian returns eta = A^-1 b + P^T L^-T z with
+ * A = P^T L L^T P its Cholesky factorisation; gabp-sparse-inv, "Gaussian
+ * sampling": x ~ N(0, A^-1) reusing the factor).  A chain is factorised in
+ * its own block order, so P = I and L is its block lower-bidiagonal Cholesky
+ * factor (diagonal blocks R_i with S_i = R_i R_i^T, R_i lower; sub-diagonal
+ * blocks B_i R_i^-T).  For each chain:
+ *
+ *   eta = A^-1 rhs + L^-T z        (eta = L^-T z when rhs is NULL)
+ *
+ * so that eta ~ N(A^-1 rhs, A^-1) when z ~ N(0, I).  The standard normals z
+ * are the caller's (the library draws no random numbers).
+ *
+ *   diag, lower   as in selinv_chain; b <= 16 (larger b: SELINV_ERR_UNSUPPORTED)
+ *   rhs     [batch, L, b]   mean's right-hand side, or NULL
+ *   z       [batch, L, b]   required
+ *   eta     [batch, L, b]   out, required
+ *   logdet  [batch] float64 out: log det A; may be NULL
+ *   info    [batch] int32   out: -1, or the first block whose Schur complement
+ *                           is not positive definite (eta then unspecified)
+ * Workspace: selinv_chain_workspace_size(dtype, batch, L, b, 0, 1) bytes.
+ */
+selinv_status selinv_chain_sample(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b,
+                                  const void *diag, const void *lower, const void *rhs,
+                                  const void *z, void *eta, double *logdet, int32_t *info,
+                                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Same computation as selinv_chain for b <= 16, with no workspace argument
  * and no allocation of any kind.  The pages have no counterpart: this entry
  * point exists for callers that cannot allocate device memory -- code running

@@ -139,6 +139,55 @@ selinv_status selinv_chain(selinv_dtype dtype, int64_t batch, int64_t L, int32_t
                             workspace, s);
 }
 
+selinv_status selinv_chain_sample(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b, const void *diag,
+                                  const void *lower, const void *rhs, const void *z, void *eta, double *logdet,
+                                  int32_t *info, void *workspace, size_t workspace_bytes, void *stream)
+{
+    selinv_status st = chain_check(dtype, batch, L, b, diag, lower, info);
+    if (st != SELINV_OK) return st;
+    if (b > 16) return SELINV_ERR_UNSUPPORTED;
+    const size_t es = elem_size(dtype);
+    if (batch > 0 && (z == nullptr || eta == nullptr)) return SELINV_ERR_INVALID_ARG;
+    if (!aligned(rhs, es) || !aligned(z, es) || !aligned(eta, es) || !aligned(logdet, 8) ||
+        !aligned(workspace, 16))
+        return SELINV_ERR_INVALID_ARG;
+    const size_t need = chain_ws(dtype, batch, L, b, false, true);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return SELINV_ERR_WORKSPACE;
+    if (batch == 0) return SELINV_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool al = aligned(diag, 16) && aligned(lower, 16) && aligned(workspace, 16);
+    if (dtype == SELINV_F64) {
+        ChainArgs<double> a;
+        a.diag = static_cast<const double *>(diag);
+        a.lower = static_cast<const double *>(lower);
+        a.G_diag = a.G_lower = nullptr;
+        a.logdet = logdet;
+        a.rhs = static_cast<const double *>(rhs);
+        a.x = static_cast<double *>(eta);
+        a.z = static_cast<const double *>(z);
+        a.info = info;
+        a.ws = static_cast<double *>(workspace);
+        a.batch = batch;
+        a.L = L;
+        a.b = b;
+        return from_cuda(chain_small_sample_launch<double>(a, al, s));
+    }
+    ChainArgs<float> a;
+    a.diag = static_cast<const float *>(diag);
+    a.lower = static_cast<const float *>(lower);
+    a.G_diag = a.G_lower = nullptr;
+    a.logdet = logdet;
+    a.rhs = static_cast<const float *>(rhs);
+    a.x = static_cast<float *>(eta);
+    a.z = static_cast<const float *>(z);
+    a.info = info;
+    a.ws = static_cast<float *>(workspace);
+    a.batch = batch;
+    a.L = L;
+    a.b = b;
+    return from_cuda(chain_small_sample_launch<float>(a, al, s));
+}
+
 selinv_status chain_solve(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b, const void *diag,
                           const void *lower, const void *rhs, void *x, double *logdet, int32_t *info,
                           void *workspace, size_t workspace_bytes, void *stream)

@@ -37,7 +37,7 @@ template <class T> __host__ __device__ constexpr int warp_smem_elems()
     return 4 * w16::SL<T>::ELEMS + w16::SLOT_ELEMS + 96;
 }
 
-template <class T, bool FULL, bool WANT_G, bool WANT_X>
+template <class T, bool FULL, bool WANT_G, bool WANT_X, bool SAMPLE = false>
 __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_kernel(ChainArgs<T> p)
 {
     using namespace w16;
@@ -65,8 +65,9 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
     const T *D = p.diag + e * L * bb;
     const T *Bl = p.lower + e * (L - 1) * bb;
     T *ws = (WANT_G || WANT_X) ? p.ws + e * (L - 1) * SLOT_ELEMS : nullptr;
-    const T *R = WANT_X ? p.rhs + e * L * b : nullptr;
+    const T *R = (WANT_X && p.rhs) ? p.rhs + e * L * b : nullptr;   // a draw may come without a mean
     T *X = WANT_X ? p.x + e * L * b : nullptr;
+    const T *Zv = SAMPLE ? p.z + e * L * b : nullptr;
 
     LogAcc det;
     det.init();
@@ -85,22 +86,51 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
         cp_async_commit();
     }
     T rn[2] = {T(0), T(0)};    // r_{i+1} at rows g, g+8 (lanes with t == 0)
+    T zc[4] = {T(0), T(0), T(0), T(0)};   // z_i at the lane's columns (draws)
     if (WANT_X) {
         if (lane < 16) {
-            const T r0 = lane < b ? R[lane] : T(0);
+            const T r0 = (R && lane < b) ? R[lane] : T(0);
             sy[lane] = r0;
             if (lane < b) X[lane] = r0;        // y_0 kept in x until the distribute sweep
         }
-        if (L > 1 && t == 0) {
+        if (R && L > 1 && t == 0) {
             rn[0] = g < b ? R[b + g] : T(0);
             rn[1] = g + 8 < b ? R[b + g + 8] : T(0);
         }
+    }
+    if (SAMPLE) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) zc[q] = tcol(t, q) < b ? Zv[tcol(t, q)] : T(0);
     }
     __syncwarp();
 
     // ---------------- collect sweep ----------------
     for (int64_t i = 0; i < L; ++i) {
         bool bad = false;
+        if (SAMPLE) {
+            // Draw: with S_i = R_i R_i^T, S_i^-1 (y_i + R_i z_i) = S_i^-1 y_i + R_i^-T z_i, so
+            // storing y_i + R_i z_i for the backward sweep turns its x = A^-1 r into
+            // eta = A^-1 r + L^-T z (L^-T z_i = R_i^-T z_i - W_i^T (L^-T z)_{i+1}).
+            Tile<T> rf = a;
+            chol_lower(rf, g, t);
+            T v[2];
+            lower_matvec(v, rf, zc, g, t);
+            T *ycur = sy + 16 * (i & 1);
+            if (t == 0) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int r = g + 8 * h;
+                    const T yv = ycur[r] + v[h];
+                    if (r < b) X[i * b + r] = yv;
+                    if (i == L - 1) ycur[r] = yv;     // the backward sweep starts from S^-1 (y + R z)
+                }
+            }
+            if (i + 1 < L) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) zc[q] = tcol(t, q) < b ? Zv[(i + 1) * b + tcol(t, q)] : T(0);
+            }
+            __syncwarp();
+        }
         spd_inverse<T>(a, cb, g, t, det, bad);        // a = S_i^-1
         det.renorm();
         if (bad && fail < 0) fail = (int)i;
@@ -137,7 +167,7 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
             load_block_async<T, FULL>(sB, Bl + (i + 1) * bb, b, lane);
             load_lower_async<T, FULL>(sD, D + (i + 2) * bb, b, lane);
             cp_async_commit();
-            if (WANT_X && t == 0) {
+            if (R && t == 0) {
                 rn[0] = g < b ? R[(i + 2) * b + g] : T(0);
                 rn[1] = g + 8 < b ? R[(i + 2) * b + g + 8] : T(0);
             }
@@ -253,11 +283,11 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
     }
 }
 
-template <class T, bool FULL, bool G, bool X>
+template <class T, bool FULL, bool G, bool X, bool SAMPLE = false>
 cudaError_t launch_t(const ChainArgs<T> &a, cudaStream_t s)
 {
     const size_t smem = sizeof(T) * warp_smem_elems<T>() * WARPS;
-    auto k = chain_small_kernel<T, FULL, G, X>;
+    auto k = chain_small_kernel<T, FULL, G, X, SAMPLE>;
     cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     const int64_t blocks = ceil_div(a.batch, WARPS);
@@ -289,7 +319,16 @@ template <class T> cudaError_t chain_small_launch(const ChainArgs<T> &a, bool al
     return launch_full<T, false>(a, s);
 }
 
+template <class T> cudaError_t chain_small_sample_launch(const ChainArgs<T> &a, bool aligned16, cudaStream_t s)
+{
+    if (a.batch == 0) return cudaSuccess;
+    if (a.b == 16 && aligned16) return launch_t<T, true, false, true, true>(a, s);
+    return launch_t<T, false, false, true, true>(a, s);
+}
+
 template cudaError_t chain_small_launch<double>(const ChainArgs<double> &, bool, cudaStream_t);
+template cudaError_t chain_small_sample_launch<double>(const ChainArgs<double> &, bool, cudaStream_t);
+template cudaError_t chain_small_sample_launch<float>(const ChainArgs<float> &, bool, cudaStream_t);
 template cudaError_t chain_small_launch<float>(const ChainArgs<float> &, bool, cudaStream_t);
 
 }  // namespace selinv

@@ -16,6 +16,7 @@ template <class T> struct ChainArgs {
     double *logdet;     // [batch] or null
     const T *rhs;       // [batch, L, b] or null
     T *x;               // [batch, L, b] or null (with rhs)
+    const T *z = nullptr;   // [batch, L, b] standard normals of a Gaussian draw, or null
     int32_t *info;      // [batch]
     T *ws;              // workspace
     int64_t batch;
@@ -26,6 +27,8 @@ template <class T> struct ChainArgs {
 // b <= 16: one warp per chain.
 size_t chain_small_workspace(size_t elem, int64_t batch, int64_t L);
 template <class T> cudaError_t chain_small_launch(const ChainArgs<T> &a, bool aligned16, cudaStream_t s);
+// The same kernel drawing eta = A^-1 rhs + L^-T z into a.x (rhs may be null; no G).
+template <class T> cudaError_t chain_small_sample_launch(const ChainArgs<T> &a, bool aligned16, cudaStream_t s);
 
 // 16 < b <= 32, no right-hand side: one CTA of two 4-warp groups per chain,
 // eliminating from both ends toward the middle block.

@@ -465,6 +465,60 @@ template <class T> SELINV_DEVINL void mirror_upper(Tile<T> &a, int g, int t)
     }
 }
 
+// In-register Cholesky factor of a symmetric positive definite tile,
+// A = R R^T with R lower triangular (entries above the diagonal are left
+// unspecified; lower_matvec ignores them).  Column k, for k = 0..15:
+// R_kk = sqrt(A_kk), R_ik = A_ik / R_kk (i > k), A_ij -= R_ik R_jk (i, j > k);
+// the column travels by shuffles (the lane's rows from lane (g, k_t), its
+// columns j from lane (j, k_t), A being symmetric).
+template <class T> SELINV_DEVINL void chol_lower(Tile<T> &a, int g, int t)
+{
+    const int lane = 4 * g + t;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const int kh = k >> 3, kt = (k & 7) >> 1, kq = (k & 1) | ((k >> 3) << 1);
+        const T d = shfl(a.v[kh][kq], ((k & 7) << 2) | kt);         // A_kk
+        const T inv = recip(sqrt(d));
+        T li[2], lj[4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {                               // R_ik at the lane's rows
+            const int r = g + 8 * h;
+            const T c = shfl(a.v[h][kq], (lane & ~3) | kt);
+            li[h] = r >= k ? c * inv : T(0);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {                               // R_jk at the lane's columns
+            const int j = tcol(t, q);
+            const T c = shfl(a.v[q >> 1][kq], ((2 * t + (q & 1)) << 2) | kt);
+            lj[q] = j > k ? c * inv : T(0);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (g + 8 * h > k) a.v[h][q] = fma(-li[h], lj[q], a.v[h][q]);
+                if (tcol(t, q) == k) a.v[h][q] = li[h];
+            }
+    }
+}
+
+// y_r = sum_{c <= r} R[r][c] x[c] for a lower-triangular tile and x given at the
+// lane's columns (xc[q] = x[tcol(t, q)]); every lane of a row group ends with
+// the sums for rows g, g + 8.
+template <class T> SELINV_DEVINL void lower_matvec(T out[2], const Tile<T> &a, const T xc[4], int g, int t)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        T s = T(0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            if (tcol(t, q) <= g + 8 * h) s = fma(a.v[h][q], xc[q], s);
+        s += shfl_xor(s, 1);
+        s += shfl_xor(s, 2);
+        out[h] = s;
+    }
+}
+
 // y_r = sum_c A[r][c] x[c] for the lane's rows g, g + 8 (x in shared memory);
 // every lane of a row group ends with the full sums.
 template <class T> SELINV_DEVINL void row_matvec(T out[2], const Tile<T> &a, const T *x, int t)
