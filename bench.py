@@ -60,6 +60,9 @@ def parse():
     ap.add_argument("--length", type=int, default=None,
                     help="override the chain length / tree size (profiling runs of a smaller case)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--op", default="selinv", choices=["selinv", "sample"],
+                    help="selinv: selected inverse + log det (+ solve); sample: Gaussian draw "
+                         "eta = A^-1 r + L^-T z + log det (chain workloads with b <= 16)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -150,19 +153,32 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def cpu_baseline(w, dtype_name, budget_s=10.0):
+def oracle_inputs(w, elems, op):
+    g = inputs.generate(w, elements=elems)
+    if op == "sample":
+        g["z"] = inputs.standard_normals(w.batch, w.L, w.b, w.seed, elems)
+    return g
+
+
+def oracle_run(oracle, w, g, op):
+    if w.kind == "tree":
+        oracle.tree(g["parent"], g["diag"], g["edge"])
+    elif op == "sample":
+        oracle.chain_sample(g["diag"], g["lower"], g["z"], rhs=g.get("rhs"))
+    else:
+        oracle.chain(g["diag"], g["lower"], g.get("rhs"))
+
+
+def cpu_baseline(w, dtype_name, op="selinv", budget_s=10.0):
     """The oracle, as it stands, on a bounded sample of the same workload (host cores)."""
     import oracle
     oracle.build()
     n_probe = 32 if w.kind != "grid" else 1
     elems = list(range(min(n_probe, w.batch)))
-    g = inputs.generate(w, elements=elems)
+    g = oracle_inputs(w, elems, op)
 
     def run(gg):
-        if w.kind == "tree":
-            oracle.tree(gg["parent"], gg["diag"], gg["edge"])
-        else:
-            oracle.chain(gg["diag"], gg["lower"], gg.get("rhs"))
+        oracle_run(oracle, w, gg, op)
 
     t0 = time.perf_counter()
     run(g)
@@ -170,7 +186,7 @@ def cpu_baseline(w, dtype_name, budget_s=10.0):
     n = int(min(w.batch, max(len(elems), len(elems) * budget_s / max(dt, 1e-6))))
     if n > len(elems):
         elems = list(range(n))
-        g = inputs.generate(w, elements=elems)
+        g = oracle_inputs(w, elems, op)
         t0 = time.perf_counter()
         run(g)
         dt = time.perf_counter() - t0
@@ -180,10 +196,14 @@ def cpu_baseline(w, dtype_name, budget_s=10.0):
             "sample": f"{len(elems)} of {w.batch} {unit_name} ({w.name}, float64), {dt:.2f} s"}
 
 
-def algorithmic_bytes(w, es, batch):
+def algorithmic_bytes(w, es, batch, op="selinv"):
     """Bytes the method must move: read D and B (or edge) blocks, write G_diag and G_lower
-    (or G_edge) blocks, plus the right-hand side and solution when solving."""
+    (or G_edge) blocks, plus the right-hand side and solution when solving.  A draw reads
+    D, B, r and z and writes eta."""
     b2 = w.b * w.b
+    if op == "sample":
+        nodes, edges = batch * w.L, batch * (w.L - 1)
+        return es * (b2 * nodes + b2 * edges + 3 * w.b * nodes)
     if w.kind == "tree":
         n = batch * w.L
         return es * (b2 * n + b2 * (n - batch) + b2 * n + b2 * (n - batch))
@@ -258,21 +278,18 @@ def run_reference(args):
     if w.kind == "chain" and w.L * w.b ** 3 > 64 * 16 ** 3 * 64:
         n_per_step = 2
     elems = list(range(min(n_per_step, w.batch)))
-    g = inputs.generate(w, elements=elems)
+    g = oracle_inputs(w, elems, args.op)
     times = []
     for it in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        if w.kind == "tree":
-            oracle.tree(g["parent"], g["diag"], g["edge"])
-        else:
-            oracle.chain(g["diag"], g["lower"], g.get("rhs"))
+        oracle_run(oracle, w, g, args.op)
         if it >= args.warmup:
             times.append(time.perf_counter() - t0)
     blocks = len(elems) * w.L
     value = blocks * len(times) / sum(times)
     sample = f"{len(elems)} of {w.batch} {'trees' if w.kind == 'tree' else 'chains'} per step"
     line = {
-        "impl": "reference", "metric": "selinv blocks/s (fp64)", "value": value, "unit": "blocks/s",
+        "impl": "reference", "metric": metric_name(args.op, "f64"), "value": value, "unit": "blocks/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -283,6 +300,11 @@ def run_reference(args):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def metric_name(op, dtype):
+    what = "draw" if op == "sample" else "selinv"
+    return f"{what} blocks/s ({'fp64' if dtype == 'f64' else 'fp32'})"
 
 
 def run_ours(args):
@@ -310,7 +332,7 @@ def run_ours(args):
     # cpu baseline first (host only), so nothing forks after CUDA work starts
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, args.dtype)
+        cpu = cpu_baseline(w, args.dtype, args.op)
 
     elems = shard_elements(rank, batch)
     stream = torch.cuda.current_stream()
@@ -321,6 +343,10 @@ def run_ours(args):
             host_in["rhs"] = rhs.cpu().pin_memory()
     else:
         g = inputs.generate(w, elements=elems)   # per-element seeds: rank r owns its own slice
+        if args.op == "sample":
+            if w.kind != "chain" or w.b > 16:
+                raise SystemExit("--op sample runs on chain workloads with b <= 16")
+            g["z"] = inputs.standard_normals(w.batch, w.L, w.b, w.seed, elems)
         host_in = {k: torch.from_numpy(v).to(tdt).pin_memory() for k, v in g.items()
                    if v is not None and k != "parent"}
         dev_in = {k: v.to("cuda", non_blocking=True) for k, v in host_in.items()}
@@ -354,7 +380,14 @@ def run_ours(args):
                          dtype=torch.uint8, device="cuda")
         launches_per_step = 1
         segments = selinv.chain_segments(batch, L, b, True, "rhs" in dev_in)
-        if b <= 16:
+        if args.op == "sample":
+            kernel = "chain_small_kernel (draw mode)"
+            out = {"eta": torch.empty((batch, L, b), dtype=tdt, device="cuda"),
+                   "logdet": torch.empty(batch, dtype=torch.float64, device="cuda"),
+                   "info": torch.empty(batch, dtype=torch.int32, device="cuda")}
+            ws = torch.empty(max(selinv.chain_workspace_size(tdt, batch, L, b, False, True), 1),
+                             dtype=torch.uint8, device="cuda")
+        elif b <= 16:
             kernel = "chain_small_kernel"
         elif segments > 0:
             # segments' collect, separators' D', their two-ended chain, segments' distribute, log det
@@ -365,9 +398,14 @@ def run_ours(args):
         else:
             kernel = "chain_large_kernel"
 
-        def step():
-            selinv.selinv_chain(dev_in["diag"], dev_in["lower"], dev_in.get("rhs"), check=False, out=out,
-                                workspace=ws)
+        if args.op == "sample":
+            def step():
+                selinv.chain_sample(dev_in["diag"], dev_in["lower"], dev_in["z"], dev_in.get("rhs"), check=False,
+                                    out=out, workspace=ws)
+        else:
+            def step():
+                selinv.selinv_chain(dev_in["diag"], dev_in["lower"], dev_in.get("rhs"), check=False, out=out,
+                                    workspace=ws)
 
     # correctness guard: the last warm-up step must report every element SPD
     for _ in range(max(args.warmup, 3)):
@@ -430,7 +468,7 @@ def run_ours(args):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     hbm, src = hbm_peak()
-    byt = algorithmic_bytes(w, es, batch)
+    byt = algorithmic_bytes(w, es, batch, args.op)
     hbm_achieved = byt / (kernel_ms / 1e3) / 1e9
     flops = algorithmic_flops(w, batch)
     flop_rate = flops / (kernel_ms / 1e3) / 1e12
@@ -462,13 +500,13 @@ def run_ours(args):
     if rank != 0:
         return 0
     line = {
-        "metric": "selinv blocks/s (fp64)" if args.dtype == "f64" else "selinv blocks/s (fp32)",
+        "metric": metric_name(args.op, args.dtype),
         "value": value, "unit": "blocks/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": args.dtype, "data": "synthetic",
         "config": {"workload": w.name if full_size else f"{w.name} (batch {batch}, length {w.L} per GPU)",
                    "global_batch": batch * world, "block": w.b, "L_or_n": w.L,
-                   "solve": bool(w.solve), "parallelism": f"dp{world} (independent chains per GPU)",
+                   "solve": bool(w.solve), "op": args.op, "parallelism": f"dp{world} (independent chains per GPU)",
                    "l2": "inputs larger than L2 (no flush)"},
         "roofline": roof,
         "cpu_baseline": cpu,

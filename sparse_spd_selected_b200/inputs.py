@@ -224,6 +224,13 @@ WORKLOADS = {
 }
 
 
+def standard_normals(batch: int, L: int, b: int, seed: int, elements: Optional[Sequence[int]] = None):
+    """Standard normals z [n, L, b] for Gaussian draws: batch element e uses its
+    own generator default_rng([seed, e, 1]), a stream apart from its matrix."""
+    elements = range(batch) if elements is None else elements
+    return np.stack([np.random.default_rng([int(seed), int(e), 1]).standard_normal((L, b)) for e in elements])
+
+
 def generate(w: Workload, elements: Optional[Sequence[int]] = None):
     """Host (NumPy) inputs of a workload, or of a subset of its batch elements."""
     if w.kind == "chain":
