@@ -135,6 +135,21 @@ selinv_status chain_solve(selinv_dtype dtype, int64_t batch, int64_t L, int32_t 
                           void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Solve with several right-hand sides from the same factorisation: X = A^-1 R
+ * for each chain, R and X [batch, L, b, nrhs] (row-major: block i of a chain
+ * is b x nrhs).  (sparsax, "Features": multiple right-hand sides, b may be
+ * (n,) or (n, n_rhs); "Factor once, do everything".)  b <= 16 (larger b:
+ * SELINV_ERR_UNSUPPORTED); nrhs >= 1.  Up to 16 right-hand sides share one
+ * pass over the factorisation; larger nrhs is taken 16 columns per pass.
+ * logdet may be NULL; info as in selinv_chain.  Workspace:
+ * selinv_chain_workspace_size(dtype, batch, L, b, 0, 1) bytes.
+ */
+selinv_status chain_solve_multi(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b, int32_t nrhs,
+                                const void *diag, const void *lower, const void *rhs, void *x,
+                                double *logdet, int32_t *info,
+                                void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Gaussian draw from the same factorisation (sparsax, "Factor once, do
  * everything": sample_gaussian returns eta = A^-1 b + P^T L^-T z with
  * A = P^T L L^T P its Cholesky factorisation; gabp-sparse-inv, "Gaussian

@@ -188,6 +188,63 @@ selinv_status selinv_chain_sample(selinv_dtype dtype, int64_t batch, int64_t L, 
     return from_cuda(chain_small_sample_launch<float>(a, al, s));
 }
 
+selinv_status chain_solve_multi(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b, int32_t nrhs,
+                                const void *diag, const void *lower, const void *rhs, void *x, double *logdet,
+                                int32_t *info, void *workspace, size_t workspace_bytes, void *stream)
+{
+    selinv_status st = chain_check(dtype, batch, L, b, diag, lower, info);
+    if (st != SELINV_OK) return st;
+    if (nrhs < 1) return SELINV_ERR_INVALID_ARG;
+    if (b > 16) return SELINV_ERR_UNSUPPORTED;
+    const size_t es = elem_size(dtype);
+    if (batch > 0 && (rhs == nullptr || x == nullptr)) return SELINV_ERR_INVALID_ARG;
+    if (!aligned(rhs, es) || !aligned(x, es) || !aligned(logdet, 8) || !aligned(workspace, 16))
+        return SELINV_ERR_INVALID_ARG;
+    const size_t need = chain_ws(dtype, batch, L, b, false, true);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return SELINV_ERR_WORKSPACE;
+    if (batch == 0) return SELINV_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool al = aligned(diag, 16) && aligned(lower, 16) && aligned(workspace, 16);
+    for (int32_t c0 = 0; c0 < nrhs; c0 += 16) {
+        cudaError_t err;
+        if (dtype == SELINV_F64) {
+            ChainArgs<double> a;
+            a.diag = static_cast<const double *>(diag);
+            a.lower = static_cast<const double *>(lower);
+            a.G_diag = a.G_lower = nullptr;
+            a.logdet = logdet;
+            a.rhs = static_cast<const double *>(rhs);
+            a.x = static_cast<double *>(x);
+            a.info = info;
+            a.ws = static_cast<double *>(workspace);
+            a.batch = batch;
+            a.L = L;
+            a.b = b;
+            a.nrhs = nrhs;
+            a.c0 = c0;
+            err = chain_small_multi_launch<double>(a, al, s);
+        } else {
+            ChainArgs<float> a;
+            a.diag = static_cast<const float *>(diag);
+            a.lower = static_cast<const float *>(lower);
+            a.G_diag = a.G_lower = nullptr;
+            a.logdet = logdet;
+            a.rhs = static_cast<const float *>(rhs);
+            a.x = static_cast<float *>(x);
+            a.info = info;
+            a.ws = static_cast<float *>(workspace);
+            a.batch = batch;
+            a.L = L;
+            a.b = b;
+            a.nrhs = nrhs;
+            a.c0 = c0;
+            err = chain_small_multi_launch<float>(a, al, s);
+        }
+        if (err != cudaSuccess) return SELINV_ERR_CUDA;
+    }
+    return SELINV_OK;
+}
+
 selinv_status chain_solve(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b, const void *diag,
                           const void *lower, const void *rhs, void *x, double *logdet, int32_t *info,
                           void *workspace, size_t workspace_bytes, void *stream)

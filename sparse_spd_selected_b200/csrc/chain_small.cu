@@ -283,6 +283,155 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
     }
 }
 
+// Several right-hand sides: X = A^-1 R for R [L, b, nrhs], 16 columns per
+// launch.  The solve recursions act on b x k blocks, so they run transposed,
+// as products X Y^T of register tiles on the tensor cores (rows = right-hand
+// sides, columns = block rows; no operand transposed):
+//   Y_0^T = R_0^T,  Y_{i+1}^T = R_{i+1}^T - Y_i^T W_i^T                 (collect)
+//   X_{L-1}^T = Y_{L-1}^T S_{L-1}^-1,  X_i^T = Y_i^T S_i^-1 - X_{i+1}^T W_i  (distribute)
+// with W_i^T = S_i^-1 B_i^T formed as in the G sweep.  Y_i is kept in x.
+template <class T, bool FULL>
+__global__ void __launch_bounds__(WARPS * 32, 3) chain_multi_kernel(ChainArgs<T> p)
+{
+    using namespace w16;
+    constexpr int E = SL<T>::ELEMS;
+    const int lane = threadIdx.x & 31;
+    const int wid = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int64_t e = (int64_t)blockIdx.x * WARPS + wid;
+    if (e >= p.batch) return;
+
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    T *sbase = reinterpret_cast<T *>(smem_raw) + wid * warp_smem_elems<T>();
+    T *sB = sbase, *sD = sB + E, *sT = sD + E, *sT2 = sT + E, *stg = sT2 + E;
+    T *cb = stg + SLOT_ELEMS + 64;
+
+    const int b = p.b;
+    const int64_t L = p.L;
+    const int64_t bb = (int64_t)b * b;
+    const int K = p.nrhs, c0 = p.c0;
+    const int kc = K - c0 < 16 ? K - c0 : 16;
+    const int64_t bk = (int64_t)b * K;
+    const T *D = p.diag + e * L * bb;
+    const T *Bl = p.lower + e * (L - 1) * bb;
+    T *ws = p.ws + e * (L - 1) * SLOT_ELEMS;
+    const T *R = p.rhs + e * L * bk;
+    T *X = p.x + e * L * bk;
+    // block i of R or X as a transposed tile: element (c, r) = M[r][c0 + c]
+    auto load_t = [&](Tile<T> &o, const T *M) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int c = g + 8 * h, r = tcol(t, q);
+                o.v[h][q] = (c < kc && r < b) ? M[(int64_t)r * K + c0 + c] : T(0);
+            }
+    };
+    auto store_t = [&](T *M, const Tile<T> &o) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int c = g + 8 * h, r = tcol(t, q);
+                if (c < kc && r < b) M[(int64_t)r * K + c0 + c] = o.v[h][q];
+            }
+    };
+
+    LogAcc det;
+    det.init();
+    int fail = -1;
+
+    Tile<T> a, w, bt, yt;
+    load_lower_async<T, FULL>(sD, D, b, lane);
+    cp_async_commit();
+    cp_async_wait_all();
+    __syncwarp();
+    from_smem_lower<T>(a, sD, g, t);
+    __syncwarp();
+    if (L > 1) {
+        load_block_async<T, FULL>(sB, Bl, b, lane);
+        load_lower_async<T, FULL>(sD, D + bb, b, lane);
+        cp_async_commit();
+    }
+    load_t(yt, R);                                    // Y_0^T = R_0^T
+    store_t(X, yt);
+
+    // ---------------- collect sweep ----------------
+    for (int64_t i = 0; i < L; ++i) {
+        bool bad = false;
+        spd_inverse<T>(a, cb, g, t, det, bad);        // a = S_i^-1
+        det.renorm();
+        if (bad && fail < 0) fail = (int)i;
+        if (i == L - 1) break;
+        store_lower_slot<T>(ws + i * SLOT_ELEMS, a, lane, g, t);
+        cp_async_wait_all();
+        __syncwarp();
+        from_smem<T>(bt, sB, g, t);                   // B_i
+        Tile<T> dn, rt;
+        from_smem_lower<T>(dn, sD, g, t);             // D_{i+1}
+        load_t(rt, R + (i + 1) * bk);                 // R_{i+1}^T
+        zero(w);
+        gemm_nt<false>(w, bt, a, sT, sT2, g, t);      // W_i = B_i S_i^-1
+        gemm_nt<true, true>(dn, w, bt, sT, sT2, g, t);   // S_{i+1} = D_{i+1} - W_i B_i^T (lower tiles)
+        mirror_upper(dn, g, t);
+        a = dn;
+        gemm_nt<true>(rt, yt, w, sT, sT2, g, t);      // Y_{i+1}^T = R_{i+1}^T - Y_i^T W_i^T
+        yt = rt;
+        store_t(X + (i + 1) * bk, yt);
+        __syncwarp();
+        if (i + 1 < L - 1) {
+            load_block_async<T, FULL>(sB, Bl + (i + 1) * bb, b, lane);
+            load_lower_async<T, FULL>(sD, D + (i + 2) * bb, b, lane);
+            cp_async_commit();
+        }
+    }
+    if (lane == 0) {
+        if (p.logdet && c0 == 0) p.logdet[e] = det.log_value();
+        if (c0 == 0) p.info[e] = fail;
+    }
+
+    // ---------------- distribute sweep ----------------
+    Tile<T> G, xt;
+    __syncwarp();
+    to_smem<T>(sT, a, g, t);
+    __syncwarp();
+    from_smem_lower<T>(G, sT, g, t);                  // S_{L-1}^-1, exactly symmetric
+    zero(xt);
+    gemm_nt<false>(xt, yt, G, sT, sT2, g, t);         // X_{L-1}^T = Y_{L-1}^T S_{L-1}^-1
+    store_t(X + (L - 1) * bk, xt);
+    __syncwarp();
+    if (L > 1) {
+        load_block_async<T, FULL>(sB, Bl + (L - 2) * bb, b, lane);
+        stage_lower_slot<T>(stg, ws + (L - 2) * SLOT_ELEMS, lane, g, t);
+        cp_async_commit();
+        load_t(yt, X + (L - 2) * bk);                 // Y_{L-2}^T
+    }
+    for (int64_t i = L - 2; i >= 0; --i) {
+        cp_async_wait_all();
+        unstage_lower_slot<T>(a, stg, lane, g, t);
+        to_smem<T>(sT, a, g, t);
+        __syncwarp();
+        from_smem_lower<T>(a, sT, g, t);              // S_i^-1, full and symmetric
+        from_smem<T>(bt, sB, g, t);                   // B_i
+        __syncwarp();
+        if (i > 0) {
+            load_block_async<T, FULL>(sB, Bl + (i - 1) * bb, b, lane);
+            stage_lower_slot<T>(stg, ws + (i - 1) * SLOT_ELEMS, lane, g, t);
+            cp_async_commit();
+        }
+        Tile<T> wt, xn;
+        zero(wt);
+        gemm_nt<false>(wt, a, bt, sT, sT2, g, t);     // W_i^T = S_i^-1 B_i^T
+        zero(xn);
+        gemm_nt<false>(xn, yt, a, sT, sT2, g, t);     // Y_i^T S_i^-1
+        gemm_nt<true>(xn, xt, wt, sT, sT2, g, t);     // - X_{i+1}^T W_i
+        xt = xn;
+        if (i > 0) load_t(yt, X + (i - 1) * bk);      // Y_{i-1}^T, before X_i overwrites nothing of it
+        store_t(X + i * bk, xt);
+        __syncwarp();
+    }
+}
+
 template <class T, bool FULL, bool G, bool X, bool SAMPLE = false>
 cudaError_t launch_t(const ChainArgs<T> &a, cudaStream_t s)
 {
@@ -318,6 +467,26 @@ template <class T> cudaError_t chain_small_launch(const ChainArgs<T> &a, bool al
     if (a.b == 16 && aligned16) return launch_full<T, true>(a, s);
     return launch_full<T, false>(a, s);
 }
+
+template <class T, bool FULL> cudaError_t launch_multi(const ChainArgs<T> &a, cudaStream_t s)
+{
+    const size_t smem = sizeof(T) * warp_smem_elems<T>() * WARPS;
+    auto k = chain_multi_kernel<T, FULL>;
+    cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    k<<<(unsigned)ceil_div(a.batch, WARPS), WARPS * 32, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <class T> cudaError_t chain_small_multi_launch(const ChainArgs<T> &a, bool aligned16, cudaStream_t s)
+{
+    if (a.batch == 0) return cudaSuccess;
+    if (a.b == 16 && aligned16) return launch_multi<T, true>(a, s);
+    return launch_multi<T, false>(a, s);
+}
+
+template cudaError_t chain_small_multi_launch<double>(const ChainArgs<double> &, bool, cudaStream_t);
+template cudaError_t chain_small_multi_launch<float>(const ChainArgs<float> &, bool, cudaStream_t);
 
 template <class T> cudaError_t chain_small_sample_launch(const ChainArgs<T> &a, bool aligned16, cudaStream_t s)
 {

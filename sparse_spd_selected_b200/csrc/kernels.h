@@ -17,6 +17,8 @@ template <class T> struct ChainArgs {
     const T *rhs;       // [batch, L, b] or null
     T *x;               // [batch, L, b] or null (with rhs)
     const T *z = nullptr;   // [batch, L, b] standard normals of a Gaussian draw, or null
+    int nrhs = 0;           // > 0: rhs / x are [batch, L, b, nrhs]; this launch takes columns
+    int c0 = 0;             //      c0 .. c0 + 15 (fewer at the end)
     int32_t *info;      // [batch]
     T *ws;              // workspace
     int64_t batch;
@@ -27,6 +29,8 @@ template <class T> struct ChainArgs {
 // b <= 16: one warp per chain.
 size_t chain_small_workspace(size_t elem, int64_t batch, int64_t L);
 template <class T> cudaError_t chain_small_launch(const ChainArgs<T> &a, bool aligned16, cudaStream_t s);
+// x = A^-1 rhs for nrhs right-hand sides (columns c0 .. c0 + 15 of them per launch; no G).
+template <class T> cudaError_t chain_small_multi_launch(const ChainArgs<T> &a, bool aligned16, cudaStream_t s);
 // The same kernel drawing eta = A^-1 rhs + L^-T z into a.x (rhs may be null; no G).
 template <class T> cudaError_t chain_small_sample_launch(const ChainArgs<T> &a, bool aligned16, cudaStream_t s);
 

@@ -59,6 +59,8 @@ def lib():
         L.selinv_chain_segments.restype = I32
         L.selinv_chain.argtypes = [ctypes.c_int, I64, I64, I32, P, P, P, P, P, P, P, P, P, SZ, P]
         L.selinv_chain.restype = ctypes.c_int
+        L.chain_solve_multi.argtypes = [ctypes.c_int, I64, I64, I32, I32, P, P, P, P, P, P, P, SZ, P]
+        L.chain_solve_multi.restype = ctypes.c_int
         L.selinv_chain_sample.argtypes = [ctypes.c_int, I64, I64, I32, P, P, P, P, P, P, P, P, SZ, P]
         L.selinv_chain_sample.restype = ctypes.c_int
         L.chain_solve.argtypes = [ctypes.c_int, I64, I64, I32, P, P, P, P, P, P, P, SZ, P]
@@ -212,6 +214,51 @@ def chain_solve(diag, lower, rhs, *, check=True, workspace=None, stream=None):
     r = selinv_chain(diag, lower, rhs, want_g=False, check=False, workspace=workspace, stream=stream)
     _raise_on_info(r["info"], check)
     return r["x"], r["logdet"], r["info"]
+
+
+def chain_solve_multi(diag, lower, rhs, *, check=True, out=None, workspace=None, stream=None):
+    """X = A^-1 R for block-tridiagonal SPD chains with several right-hand sides
+    (b <= 16): rhs [..., L, b, k].  Returns (x [..., L, b, k], logdet, info)."""
+    _cuda_contig("diag", diag)
+    dt = diag.dtype
+    if diag.dim() < 3 or diag.shape[-1] != diag.shape[-2]:
+        raise ValueError("diag must be [..., L, b, b]")
+    lead = tuple(diag.shape[:-3])
+    L, b = int(diag.shape[-3]), int(diag.shape[-1])
+    batch = 1
+    for d in lead:
+        batch *= int(d)
+    if L > 1:
+        if lower is None:
+            raise ValueError("lower is required when L > 1")
+        _cuda_contig("lower", lower, dt)
+        if tuple(lower.shape) != lead + (L - 1, b, b):
+            raise ValueError(f"lower must be {lead + (L - 1, b, b)}, got {tuple(lower.shape)}")
+    else:
+        lower = None
+    _cuda_contig("rhs", rhs, dt)
+    if rhs.dim() != len(lead) + 3 or tuple(rhs.shape[:-1]) != lead + (L, b):
+        raise ValueError(f"rhs must be {lead + (L, b)} + (k,)")
+    k = int(rhs.shape[-1])
+    dev = diag.device
+    out = dict(out or {})
+    x = out.get("x")
+    if x is None:
+        x = torch.empty(lead + (L, b, k), dtype=dt, device=dev)
+    logdet = out.get("logdet")
+    if logdet is None:
+        logdet = torch.empty(lead, dtype=torch.float64, device=dev)
+    info = out.get("info")
+    if info is None:
+        info = torch.empty(lead, dtype=torch.int32, device=dev)
+    nbytes = chain_workspace_size(dt, batch, L, b, False, True)
+    ws = _workspace(nbytes, dev, workspace)
+    with torch.cuda.device(dev):
+        st = lib().chain_solve_multi(_code(dt), batch, L, b, k, _ptr(diag), _ptr(lower), _ptr(rhs), _ptr(x),
+                                     _ptr(logdet), _ptr(info), _ptr(ws), nbytes, _stream_handle(stream))
+    _check(st, "chain_solve_multi")
+    _raise_on_info(info, check)
+    return x, logdet, info
 
 
 def chain_sample(diag, lower, z, rhs=None, *, check=True, out=None, workspace=None, stream=None):
