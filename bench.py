@@ -214,10 +214,12 @@ def algorithmic_bytes(w, es, batch, op="selinv"):
     return byt
 
 
-def algorithmic_flops(w, batch):
+def algorithmic_flops(w, batch, op="selinv"):
     """Nominal 7 b^3 flops per block: collect (Cholesky b^3/3 + trsm b^3 + syrk b^3) and
-    distribute (inverse 2b^3/3 + trmm b^3 + gemm 2b^3 + symmetric half-gemm b^3)."""
-    return 7.0 * w.b ** 3 * batch * w.L
+    distribute (inverse 2b^3/3 + trmm b^3 + gemm 2b^3 + symmetric half-gemm b^3).  A draw
+    needs the collect only (7 b^3 / 3; its triangular solves are O(b^2))."""
+    per = 7.0 / 3.0 if op == "sample" else 7.0
+    return per * w.b ** 3 * batch * w.L
 
 
 def fp64_peak_tflops(torch):
@@ -341,11 +343,14 @@ def run_ours(args):
         host_in = {"diag": diag.cpu().pin_memory(), "lower": lower.cpu().pin_memory()}
         if rhs is not None:
             host_in["rhs"] = rhs.cpu().pin_memory()
+        if args.op == "sample":
+            host_in["z"] = torch.from_numpy(inputs.standard_normals(batch, w.L, w.b, w.seed, elems)).to(
+                tdt).pin_memory()
     else:
         g = inputs.generate(w, elements=elems)   # per-element seeds: rank r owns its own slice
         if args.op == "sample":
-            if w.kind != "chain" or w.b > 16:
-                raise SystemExit("--op sample runs on chain workloads with b <= 16")
+            if w.kind != "chain" or (w.b > 16 and args.dtype != "f64"):
+                raise SystemExit("--op sample runs on chain workloads (b > 16 in float64 only)")
             g["z"] = inputs.standard_normals(w.batch, w.L, w.b, w.seed, elems)
         host_in = {k: torch.from_numpy(v).to(tdt).pin_memory() for k, v in g.items()
                    if v is not None and k != "parent"}
@@ -369,6 +374,8 @@ def run_ours(args):
             dev_in = {"diag": diag, "lower": lower}
             if rhs is not None:
                 dev_in["rhs"] = rhs
+            if args.op == "sample":
+                dev_in["z"] = host_in["z"].to("cuda")
         L, b = w.L, w.b
         out = {"G_diag": torch.empty((batch, L, b, b), dtype=tdt, device="cuda"),
                "G_lower": torch.empty((batch, L - 1, b, b), dtype=tdt, device="cuda"),
@@ -381,7 +388,7 @@ def run_ours(args):
         launches_per_step = 1
         segments = selinv.chain_segments(batch, L, b, True, "rhs" in dev_in)
         if args.op == "sample":
-            kernel = "chain_small_kernel (draw mode)"
+            kernel = "chain_small_kernel (draw mode)" if b <= 16 else "chain_large_kernel (draw mode)"
             out = {"eta": torch.empty((batch, L, b), dtype=tdt, device="cuda"),
                    "logdet": torch.empty(batch, dtype=torch.float64, device="cuda"),
                    "info": torch.empty(batch, dtype=torch.int32, device="cuda")}
@@ -470,7 +477,7 @@ def run_ours(args):
     hbm, src = hbm_peak()
     byt = algorithmic_bytes(w, es, batch, args.op)
     hbm_achieved = byt / (kernel_ms / 1e3) / 1e9
-    flops = algorithmic_flops(w, batch)
+    flops = algorithmic_flops(w, batch, args.op)
     flop_rate = flops / (kernel_ms / 1e3) / 1e12
     traffic = profiled_traffic(kernel, w.name) if full_size else None
     hbm_src = f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback 6650 GB/s"

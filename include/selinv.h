@@ -163,7 +163,8 @@ selinv_status chain_solve_multi(selinv_dtype dtype, int64_t batch, int64_t L, in
  * so that eta ~ N(A^-1 rhs, A^-1) when z ~ N(0, I).  The standard normals z
  * are the caller's (the library draws no random numbers).
  *
- *   diag, lower   as in selinv_chain; b <= 16 (larger b: SELINV_ERR_UNSUPPORTED)
+ *   diag, lower   as in selinv_chain; b <= 16, or 16 < b <= 128 in float64
+ *                 (float32 with b > 16: SELINV_ERR_UNSUPPORTED)
  *   rhs     [batch, L, b]   mean's right-hand side, or NULL
  *   z       [batch, L, b]   required
  *   eta     [batch, L, b]   out, required

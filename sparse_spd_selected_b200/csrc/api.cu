@@ -145,7 +145,7 @@ selinv_status selinv_chain_sample(selinv_dtype dtype, int64_t batch, int64_t L, 
 {
     selinv_status st = chain_check(dtype, batch, L, b, diag, lower, info);
     if (st != SELINV_OK) return st;
-    if (b > 16) return SELINV_ERR_UNSUPPORTED;
+    if (b > 16 && dtype != SELINV_F64) return SELINV_ERR_UNSUPPORTED;
     const size_t es = elem_size(dtype);
     if (batch > 0 && (z == nullptr || eta == nullptr)) return SELINV_ERR_INVALID_ARG;
     if (!aligned(rhs, es) || !aligned(z, es) || !aligned(eta, es) || !aligned(logdet, 8) ||
@@ -170,6 +170,7 @@ selinv_status selinv_chain_sample(selinv_dtype dtype, int64_t batch, int64_t L, 
         a.batch = batch;
         a.L = L;
         a.b = b;
+        if (b > 16) return from_cuda(chain_large_sample_launch(a, s));
         return from_cuda(chain_small_sample_launch<double>(a, al, s));
     }
     ChainArgs<float> a;

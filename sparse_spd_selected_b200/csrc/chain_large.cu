@@ -94,7 +94,8 @@ template <class T, int BP> struct Ctx {
 template <class T, int BP> constexpr size_t smem_elems()
 {
     using X = Ctx<T, BP>;
-    return (size_t)X::BIG + 2 * X::PANEL + 2 * BP /*colbuf*/ + 4 * BP /*y, x*/ + 2 * X::RW * BP /*red*/;
+    return (size_t)X::BIG + 2 * X::PANEL + 2 * BP /*colbuf*/ + 4 * BP /*y, x*/ + 2 * X::RW * BP /*red*/ +
+           BP /*z of a draw*/;
 }
 
 template <class T> SELINV_DEVINL void zero(Big<T> &a)
@@ -416,11 +417,17 @@ SELINV_DEVINL void spd_inverse(Big<T> &a, T *colbuf, const Ctx<T, BP> &x, LogAcc
 // cores (k permuted to the accumulator layout, as in the 16 x 16 products);
 // T is published for the owners of row block K.  Two barriers per eight
 // pivots instead of eight.
-template <int BP>
+// DRAW: also v = R z for the Cholesky factor S = R R^T of the input block
+// (z in shared memory, zs[r]; vacc[mi] = (R z) at row R(mi), formed by the
+// warps of quadrant column 0).  Block step K meets R's block column K:
+// R_KK = chol(P), P being the Schur complement the step pivots on, and
+// R_iK = T_i R_KK for the rows below, so v_K += R_KK z_K and v_i += T_i (R_KK z_K).
+template <int BP, bool DRAW = false>
 SELINV_DEVINL void spd_inverse_blocked(Big<double> &a, double *cbuf, double *tbuf, const Ctx<double, BP> &x,
-                                       LogAcc &det, bool &bad)
+                                       LogAcc &det, bool &bad, const double *zs = nullptr, double *vacc = nullptr)
 {
     constexpr int NB = BP / 8;
+    if (DRAW) vacc[0] = vacc[1] = vacc[2] = vacc[3] = 0.0;
     for (int K = 0; K < NB; ++K) {
         double *cb = cbuf + (K & 1) * BP * 8;                     // cb[r * 8 + c] = A[r][8K + c]
         double *tb = tbuf + (K & 1) * BP * 8;                     // tb[r * 8 + c] = T[r][c]
@@ -446,6 +453,12 @@ SELINV_DEVINL void spd_inverse_blocked(Big<double> &a, double *cbuf, double *tbu
             pv[0] = u.x;
             pv[1] = u.y;
         }
+        double wk = 0.0;                                          // (R_KK z_K) at row 8K + g
+        if (DRAW) {
+            double rc[2] = {pv[0], pv[1]};
+            chol8(rc, x.lane, x.g, x.t);
+            wk = lower8_rowdot(rc, zs[8 * K + 2 * x.t], zs[8 * K + 2 * x.t + 1], x.g, x.t);
+        }
         inv8_sweep(pv, x.lane, x.g, x.t, det, bad, x.tid == 0);
         // T = A_{rows,K} P^-1 for this warp's rows: 4 m-tiles x 2 k-steps
         double T[4][2];
@@ -455,6 +468,21 @@ SELINV_DEVINL void spd_inverse_blocked(Big<double> &a, double *cbuf, double *tbu
             T[mi][0] = T[mi][1] = 0.0;
             dmma_8x8x4(T[mi][0], T[mi][1], arow.x, pv[0]);
             dmma_8x8x4(T[mi][0], T[mi][1], arow.y, pv[1]);
+        }
+        if (DRAW && x.cw == 0) {                                  // v at this warp's rows
+            const double w0 = shfl(wk, (2 * x.t) << 2), w1 = shfl(wk, (2 * x.t + 1) << 2);
+#pragma unroll
+            for (int mi = 0; mi < 4; ++mi) {
+                const int rb = 4 * x.rw + mi;                         // 8-row block of m-tile mi
+                if (rb == K) {
+                    vacc[mi] += wk;
+                } else if (rb > K) {
+                    double s2 = fma(T[mi][0], w0, T[mi][1] * w1);
+                    s2 += shfl_xor(s2, 1);
+                    s2 += shfl_xor(s2, 2);
+                    vacc[mi] += s2;
+                }
+            }
         }
         if (x.cw == 0) {                                          // publish T (one copy per row)
 #pragma unroll
@@ -554,7 +582,7 @@ SELINV_DEVINL void col_partial(T s[4][2], const Big<T> &a, const T *v, const Ctx
         }
 }
 
-template <class T, int BP, bool FULL, bool WANT_G, bool WANT_X>
+template <class T, int BP, bool FULL, bool WANT_G, bool WANT_X, bool SAMPLE = false>
 __global__ void __launch_bounds__(Geo<BP>::NT) chain_large_kernel(ChainArgs<T> p)
 {
     using X = Ctx<T, BP>;
@@ -571,6 +599,7 @@ __global__ void __launch_bounds__(Geo<BP>::NT) chain_large_kernel(ChainArgs<T> p
     T *xbuf = ybuf + 2 * BP;       // two buffers
     T *red1 = xbuf + 2 * BP;       // [RW][BP]
     T *red2 = red1 + RW * BP;      // [RW][BP]
+    T *zs = red2 + RW * BP;        // z_i of a draw
 
     const int b = p.b;
     const int64_t L = p.L;
@@ -578,8 +607,9 @@ __global__ void __launch_bounds__(Geo<BP>::NT) chain_large_kernel(ChainArgs<T> p
     const T *D = p.diag + e * L * bb;
     const T *Bl = p.lower + e * (L - 1) * bb;
     T *ws = p.ws + e * (L - 1) * 2 * BB;
-    const T *Rv = WANT_X ? p.rhs + e * L * b : nullptr;
+    const T *Rv = (WANT_X && p.rhs) ? p.rhs + e * L * b : nullptr;   // a draw may come without a mean
     T *Xv = WANT_X ? p.x + e * L * b : nullptr;
+    const T *Zv = SAMPLE ? p.z + e * L * b : nullptr;
     constexpr bool KEEP = WANT_G || WANT_X;
 
     LogAcc det;
@@ -587,7 +617,7 @@ __global__ void __launch_bounds__(Geo<BP>::NT) chain_large_kernel(ChainArgs<T> p
     int fail = -1;
 
     if (WANT_X && x.tid < BP) {
-        const T r0 = x.tid < b ? Rv[x.tid] : T(0);
+        const T r0 = (Rv && x.tid < b) ? Rv[x.tid] : T(0);
         ybuf[x.tid] = r0;
         if (x.tid < b) Xv[x.tid] = r0;            // y_0 kept in x until the distribute sweep
     }
@@ -602,8 +632,27 @@ __global__ void __launch_bounds__(Geo<BP>::NT) chain_large_kernel(ChainArgs<T> p
             prefetch_range_l2(D + (i + 1) * bb, bb, x.tid, Geo<BP>::NT);
             if (i + 1 < L - 1) prefetch_range_l2(Bl + (i + 1) * bb, bb, x.tid, Geo<BP>::NT);
         }
-        if constexpr (sizeof(T) == 8) spd_inverse_blocked<BP>(a, pbuf, pbuf + 2 * BP * 8, x, det, bad);
-        else spd_inverse<T, BP>(a, colbuf, x, det, bad);
+        if constexpr (SAMPLE) {
+            // Draw: store y_i + R_i z_i for the backward sweep (S_i = R_i R_i^T), so that
+            // S_i^-1 (y_i + R_i z_i) = S_i^-1 y_i + R_i^-T z_i turns x = A^-1 r into
+            // eta = A^-1 r + L^-T z.  R_i z_i comes out of the blocked inverse.
+            if (x.tid < BP) zs[x.tid] = x.tid < b ? Zv[i * b + x.tid] : T(0);   // visible after its first barrier
+            double vacc[4];
+            spd_inverse_blocked<BP, true>(a, pbuf, pbuf + 2 * BP * 8, x, det, bad, zs, vacc);
+            if (x.cw == 0 && x.t == 0) {
+#pragma unroll
+                for (int mi = 0; mi < 4; ++mi) {
+                    const int r = x.R(mi);
+                    const T yv = ybuf[BP * (i & 1) + r] + vacc[mi];
+                    if (r < b) Xv[i * b + r] = yv;
+                    if (i == L - 1) ybuf[BP * (i & 1) + r] = yv;   // the backward sweep starts from S^-1 (y + R z)
+                }
+            }
+        } else if constexpr (sizeof(T) == 8) {
+            spd_inverse_blocked<BP>(a, pbuf, pbuf + 2 * BP * 8, x, det, bad);
+        } else {
+            spd_inverse<T, BP>(a, colbuf, x, det, bad);
+        }
         if (bad && fail < 0) fail = (int)i;
         if (i == L - 1) break;
         if (KEEP) store_ws<T, BP>(ws + (2 * i) * BB, a, x);
@@ -626,7 +675,7 @@ __global__ void __launch_bounds__(Geo<BP>::NT) chain_large_kernel(ChainArgs<T> p
         if (WANT_X && x.tid < BP) {
             T s = T(0);
             for (int c = 0; c < RW; ++c) s += red1[c * BP + x.tid];
-            const T r = x.tid < b ? Rv[(i + 1) * b + x.tid] : T(0);
+            const T r = (Rv && x.tid < b) ? Rv[(i + 1) * b + x.tid] : T(0);
             const T yv = r - s;
             ybuf[BP * ((i + 1) & 1) + x.tid] = yv;
             if (x.tid < b) Xv[(i + 1) * b + x.tid] = yv;
@@ -718,11 +767,11 @@ __global__ void __launch_bounds__(Geo<BP>::NT) chain_large_kernel(ChainArgs<T> p
     }
 }
 
-template <class T, int BP, bool FULL, bool G, bool Xs>
+template <class T, int BP, bool FULL, bool G, bool Xs, bool SAMPLE = false>
 cudaError_t launch_t(const ChainArgs<T> &a, cudaStream_t s)
 {
     const size_t smem = sizeof(T) * smem_elems<T, BP>();
-    auto k = chain_large_kernel<T, BP, FULL, G, Xs>;
+    auto k = chain_large_kernel<T, BP, FULL, G, Xs, SAMPLE>;
     cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     k<<<(unsigned)a.batch, Geo<BP>::NT, smem, s>>>(a);
@@ -765,6 +814,19 @@ template <class T> cudaError_t chain_large_launch(const ChainArgs<T> &a, cudaStr
     if (bp == 32) return launch_bp<T, 32>(a, full, s);
     if (bp == 64) return launch_bp<T, 64>(a, full, s);
     return launch_bp<T, 128>(a, full, s);
+}
+
+cudaError_t chain_large_sample_launch(const ChainArgs<double> &a, cudaStream_t s)
+{
+    if (a.batch == 0) return cudaSuccess;
+    const int bp = padded(a.b);
+    const bool full = a.b == bp && al16(a.diag) && al16(a.lower);
+    if (bp == 32) return full ? launch_t<double, 32, true, false, true, true>(a, s)
+                              : launch_t<double, 32, false, false, true, true>(a, s);
+    if (bp == 64) return full ? launch_t<double, 64, true, false, true, true>(a, s)
+                              : launch_t<double, 64, false, false, true, true>(a, s);
+    return full ? launch_t<double, 128, true, false, true, true>(a, s)
+                : launch_t<double, 128, false, false, true, true>(a, s);
 }
 
 template cudaError_t chain_large_launch<double>(const ChainArgs<double> &, cudaStream_t);

@@ -112,6 +112,43 @@ SELINV_DEVINL void inv8_sweep(double v[2], int lane, int g, int t, LogAcc &det, 
     v[1] = -v[1];
 }
 
+// Cholesky factor of a symmetric positive definite 8 x 8 matrix in the same
+// layout, P = R R^T with R lower triangular (entries above the diagonal left
+// unspecified): for each column k, R_kk = sqrt(P_kk), R_ik = P_ik / R_kk,
+// P_ij -= R_ik R_jk (i, j > k); the column travels by shuffles.
+SELINV_DEVINL void chol8(double v[2], int lane, int g, int t)
+{
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int kt = k >> 1, kj = k & 1;
+        const double inv = recip(sqrt(shfl(v[kj], (k << 2) | kt)));
+        const double c = shfl(v[kj], (lane & ~3) | kt);             // P[g][k]
+        const double li = g >= k ? c * inv : 0.0;
+        double lj[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {                                // P[2t+j][k]
+            const double u = shfl(v[kj], ((2 * t + j) << 2) | kt);
+            lj[j] = 2 * t + j > k ? u * inv : 0.0;
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            if (g > k) v[j] = fma(-li, lj[j], v[j]);
+            if (2 * t + j == k) v[j] = li;
+        }
+    }
+}
+
+// sum_c R[g][c] x[c] over an 8 x 8 lower-triangular R in that layout, x at the
+// lane's columns 2t, 2t+1; every lane of row g ends with the sum.
+SELINV_DEVINL double lower8_rowdot(const double r[2], double x0, double x1, int g, int t)
+{
+    double s = (2 * t <= g ? r[0] * x0 : 0.0);
+    if (2 * t + 1 <= g) s = fma(r[1], x1, s);
+    s += shfl_xor(s, 1);
+    s += shfl_xor(s, 2);
+    return s;
+}
+
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 }  // namespace selinv

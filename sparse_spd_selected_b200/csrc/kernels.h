@@ -49,5 +49,7 @@ template <class T> cudaError_t chain_seg_launch(const ChainArgs<T> &a, int P, cu
 // 16 < b <= 128: one CTA per chain.
 size_t chain_large_workspace(size_t elem, int64_t batch, int64_t L, int b);
 template <class T> cudaError_t chain_large_launch(const ChainArgs<T> &a, cudaStream_t s);
+// The same kernel drawing eta = A^-1 rhs + L^-T z into a.x (float64; rhs may be null; no G).
+cudaError_t chain_large_sample_launch(const ChainArgs<double> &a, cudaStream_t s);
 
 }  // namespace selinv

@@ -369,17 +369,39 @@ SELINV_DEVINL void gemm_nt(Tile<float> &acc, const Tile<float> &X, const Tile<fl
 // k index follows the accumulator layout (P^-1 and A_HK symmetric partners
 // supply the B fragments from the lane's own registers), and T^T is formed
 // by shuffles.  No shared memory, no barrier.
-SELINV_DEVINL void spd_inverse_blocked(Tile<double> &a, int g, int t, LogAcc &det, bool &bad)
+// DRAW: also v = R z for the Cholesky factor S = R R^T of the input tile
+// (zc[q] = z at the lane's column tcol(t, q); v[h] = (R z) at row g + 8h).
+// The block steps meet R block by block: R_KK = chol(P) of the pivot block as
+// the step finds it (a Schur complement), and below it R_HK = T R_KK, so
+//   v_K += R_KK z_K,  v_H += T (R_KK z_K)   (the second only for K = 0).
+template <bool DRAW = false>
+SELINV_DEVINL void spd_inverse_blocked(Tile<double> &a, int g, int t, LogAcc &det, bool &bad,
+                                       const double *zc = nullptr, double *v = nullptr)
 {
     const int lane = 4 * g + t;
+    if (DRAW) v[0] = v[1] = 0.0;
 #pragma unroll
     for (int K = 0; K < 2; ++K) {
         const int H = 1 - K;
         double pv[2] = {a.v[K][2 * K], a.v[K][2 * K + 1]};
+        double wk = 0.0;                                  // (R_KK z_K) at row 8K + g
+        if (DRAW) {
+            double rc[2] = {pv[0], pv[1]};
+            chol8(rc, lane, g, t);
+            wk = lower8_rowdot(rc, zc[2 * K], zc[2 * K + 1], g, t);
+            v[K] += wk;
+        }
         inv8_sweep(pv, lane, g, t, det, bad, true);
         double t0 = 0.0, t1 = 0.0;                        // T = A_HK P^-1
         dmma_8x8x4(t0, t1, a.v[H][2 * K], pv[0]);
         dmma_8x8x4(t0, t1, a.v[H][2 * K + 1], pv[1]);
+        if (DRAW && K == 0) {                             // v_H += T (R_00 z_0); T at rows 8 + g
+            const double w0 = shfl(wk, (2 * t) << 2), w1 = shfl(wk, (2 * t + 1) << 2);
+            double s2 = fma(t0, w0, t1 * w1);
+            s2 += shfl_xor(s2, 1);
+            s2 += shfl_xor(s2, 2);
+            v[H] += s2;
+        }
         // A_HH -= T A_KH, with A_KH[k][c] = A_HK[c][k]
         dmma_8x8x4(a.v[H][2 * H], a.v[H][2 * H + 1], -t0, a.v[H][2 * K]);
         dmma_8x8x4(a.v[H][2 * H], a.v[H][2 * H + 1], -t1, a.v[H][2 * K + 1]);

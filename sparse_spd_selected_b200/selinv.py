@@ -262,7 +262,7 @@ def chain_solve_multi(diag, lower, rhs, *, check=True, out=None, workspace=None,
 
 
 def chain_sample(diag, lower, z, rhs=None, *, check=True, out=None, workspace=None, stream=None):
-    """Gaussian draw from the chain's own Cholesky factor A = L L^T (b <= 16):
+    """Gaussian draw from the chain's own Cholesky factor A = L L^T (b <= 16; float64 up to b = 128):
     eta = L^-T z, plus A^-1 rhs when rhs is given, so eta ~ N(A^-1 rhs, A^-1)
     for standard normal z [..., L, b] supplied by the caller.  Returns a dict
     with eta, logdet (float64) and info (int32, -1 = ok)."""

@@ -86,5 +86,26 @@ def test_sample_not_spd_and_unsupported(cuda_ok):
     with pytest.raises(selinv.NotSPDError):
         selinv.chain_sample(to_dev(d, torch.float64), to_dev(l, torch.float64), to_dev(z, torch.float64))
     d2, l2, r2 = inputs.chain_inputs(1, 3, 20, seed=8401, load=1.0, with_rhs=True)
-    with pytest.raises(selinv.SelinvError):
-        selinv.chain_sample(to_dev(d2, torch.float64), to_dev(l2, torch.float64), to_dev(r2, torch.float64))
+    with pytest.raises(selinv.SelinvError):          # float32 draws stop at b = 16
+        selinv.chain_sample(to_dev(d2, torch.float32), to_dev(l2, torch.float32), to_dev(r2, torch.float32))
+
+
+@pytest.mark.parametrize("b", [17, 32, 40, 64, 100, 128])
+@pytest.mark.parametrize("L", [1, 3, 6])
+def test_sample_large_blocks_f64(cuda_ok, b, L):
+    """Draws through the CTA kernel (R_i z_i met inside its blocked inverse)."""
+    out, ref = draw(2, L, b, 8500 + b + L, L != 3, torch.float64)
+    assert worst(host(out["eta"]), ref["eta"]) <= TOL[torch.float64]
+    assert logdet_err(host(out["logdet"]), ref["logdet"]) <= TOL[torch.float64]
+
+
+def test_sample_grid_sampled(cuda_ok):
+    """The grid workload's shape (256 chains of 128 blocks of 128): a Gibbs step
+    eta = A^-1 r + L^-T z on all chains, two of them against the oracle."""
+    d, l, r, _ = inputs.grid_inputs_torch(256, 128, 4, "cuda", torch.float64, True)
+    z = torch.from_numpy(inputs.standard_normals(256, 128, 128, 4)).cuda()
+    out = selinv.chain_sample(d, l, z, r)
+    pick = [0, 255]
+    ref = oracle.chain_sample(host(d[pick]), host(l[pick]), host(z[pick]), rhs=host(r[pick]))
+    assert worst(host(out["eta"][pick]), ref["eta"]) <= TOL[torch.float64]
+    assert logdet_err(host(out["logdet"][pick]), ref["logdet"]) <= TOL[torch.float64]
