@@ -101,3 +101,22 @@ def test_segment_rules(lib):
     assert f(2, 95, 32, 1, 0) == 0           # too short
     assert f(100000, 4096, 32, 1, 0) == 0    # batch fills the GPU
     assert f(1, 10 ** 6, 32, 1, 0) == 16     # at most 16 segments
+
+
+def test_sample_and_multi_argument_errors(lib):
+    """The draw and the several-right-hand-side solve reject bad arguments before any launch."""
+    s = lib.selinv_chain_sample
+    # dtype, batch, L, b, diag, lower, rhs, z, eta, logdet, info, ws, ws_bytes, stream
+    assert s(0, 1, 4, 4, FAKE, FAKE, None, None, FAKE, None, FAKE, FAKE, 1 << 30, None) == selinv.ERR_INVALID_ARG
+    assert s(0, 1, 4, 4, FAKE, FAKE, None, FAKE, None, None, FAKE, FAKE, 1 << 30, None) == selinv.ERR_INVALID_ARG
+    assert s(1, 1, 4, 20, FAKE, FAKE, None, FAKE, FAKE, None, FAKE, FAKE, 1 << 30, None) == selinv.ERR_UNSUPPORTED
+    assert s(0, 1, 4, 129, FAKE, FAKE, None, FAKE, FAKE, None, FAKE, FAKE, 1 << 30, None) == selinv.ERR_UNSUPPORTED
+    assert s(0, 1, 4, 4, FAKE, FAKE, None, FAKE, FAKE, None, FAKE, FAKE, 16, None) == selinv.ERR_WORKSPACE
+    assert s(0, 0, 4, 4, FAKE, FAKE, None, FAKE, FAKE, None, FAKE, FAKE, 1 << 30, None) == selinv.OK
+    m = lib.chain_solve_multi
+    # dtype, batch, L, b, nrhs, diag, lower, rhs, x, logdet, info, ws, ws_bytes, stream
+    assert m(0, 1, 4, 4, 0, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 1 << 30, None) == selinv.ERR_INVALID_ARG
+    assert m(0, 1, 4, 4, 3, FAKE, FAKE, None, FAKE, None, FAKE, FAKE, 1 << 30, None) == selinv.ERR_INVALID_ARG
+    assert m(0, 1, 4, 20, 3, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 1 << 30, None) == selinv.ERR_UNSUPPORTED
+    assert m(0, 1, 4, 4, 3, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 16, None) == selinv.ERR_WORKSPACE
+    assert m(0, 0, 4, 4, 3, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 1 << 30, None) == selinv.OK
