@@ -48,6 +48,8 @@ def _bind(path):
     lib.oracle_tree.restype = ctypes.c_int
     lib.oracle_chain_sample.argtypes = [P, P, I64, I64, ctypes.c_int, P, P, P, P, P]
     lib.oracle_chain_sample.restype = ctypes.c_int
+    lib.oracle_tree_sample.argtypes = [P, I64, I64, ctypes.c_int, P, P, P, P, P, P]
+    lib.oracle_tree_sample.restype = ctypes.c_int
     lib.oracle_threads.argtypes = []
     lib.oracle_threads.restype = ctypes.c_int
     return lib
@@ -166,3 +168,23 @@ def tree(parent, diag, edge, lib=None):
     if rc != 0:
         raise ValueError("oracle_tree: invalid arguments")
     return {"G_diag": G_diag, "G_edge": G_edge, "logdet": logdet, "info": info}
+
+
+def tree_sample(parent, diag, edge, z, lib=None):
+    """Gaussian draw w = L^-T z on block trees (A = L L^T in the tree's own
+    elimination order, children before parents).  parent [trees, n], diag /
+    edge [trees, n, b, b], z [trees, n, b].  Returns dict with eta [trees, n, b],
+    logdet [trees], info [trees] (-1 ok, a failing node, or -2 for a malformed tree)."""
+    parent = np.ascontiguousarray(parent, dtype=np.int32)
+    diag, edge, z = _f64(diag), _f64(edge), _f64(z)
+    trees, n = parent.shape
+    b = diag.shape[-1]
+    assert diag.shape == (trees, n, b, b) and edge.shape == (trees, n, b, b) and z.shape == (trees, n, b)
+    w = np.empty((trees, n, b))
+    logdet = np.empty(trees)
+    info = np.empty(trees, dtype=np.int32)
+    rc = _load(lib).oracle_tree_sample(_ptr(parent), trees, n, b, _ptr(diag), _ptr(edge), _ptr(z), _ptr(w),
+                                       _ptr(logdet), _ptr(info))
+    if rc != 0:
+        raise ValueError("oracle_tree_sample: invalid arguments")
+    return {"eta": w, "logdet": logdet, "info": info}

@@ -416,6 +416,99 @@ done:
 }
 
 /*
+ * Gaussian draw on a tree (gabp-sparse-inv, "Gaussian sampling":
+ * sample_gaussian_tree draws x ~ N(0, A^-1) reusing the factorisation; the
+ * factor is the one sparsax's sample_gaussian names, A = P^T L L^T P, here
+ * with the tree's own elimination order, children before parents).  The
+ * Cholesky factor's blocks are L_vv = R_v (S_v = R_v R_v^T) and
+ * L_{p(v),v} = E_v R_v^-T (E_v = edge[v] = A_{p(v),v}); w = L^-T z by back
+ * substitution from the root:
+ *   w_root = R_root^-T z_root,   w_v = R_v^-T (z_v - R_v^-1 E_v^T w_{p(v)}).
+ * The sibling order does not change L (each S_v depends on v's subtree only).
+ */
+static int tree_sample_one(int64_t n, int b, const int32_t *parent, const double *diag,
+                           const double *edge, const double *z, double *w, double *logdet_out)
+{
+    const size_t bb = (size_t)b * b;
+    int64_t root = -1;
+    for (int64_t u = 0; u < n; ++u) {
+        if (parent[u] == -1) { if (root >= 0) return -2; root = u; }
+        else if (parent[u] < 0 || parent[u] >= n || parent[u] == u) return -2;
+    }
+    if (root < 0) return -2;
+    int64_t *first = calloc((size_t)n + 1, sizeof(int64_t));    /* children CSR */
+    int64_t *kids = malloc(sizeof(int64_t) * (size_t)(n > 0 ? n : 1));
+    int64_t *next = malloc(sizeof(int64_t) * (size_t)n);
+    int64_t *bfs = malloc(sizeof(int64_t) * (size_t)n);
+    for (int64_t u = 0; u < n; ++u) if (parent[u] >= 0) first[parent[u] + 1]++;
+    for (int64_t u = 0; u < n; ++u) first[u + 1] += first[u];
+    for (int64_t u = 0; u < n; ++u) next[u] = first[u];
+    for (int64_t u = 0; u < n; ++u) if (parent[u] >= 0) kids[next[parent[u]]++] = u;
+    int64_t qh = 0, qt = 0;
+    bfs[qt++] = root;
+    while (qh < qt) {
+        int64_t u = bfs[qh++];
+        for (int64_t k = first[u]; k < first[u + 1]; ++k) bfs[qt++] = kids[k];
+    }
+    int info = -1;
+    double *Rinv = NULL, *Sc = NULL, *Rf = NULL, *Si = NULL, *ES = NULL, *ESE = NULL, *t1 = NULL, *t2 = NULL;
+    if (qt != n) { info = -2; goto out; }
+    Rinv = malloc(sizeof(double) * bb * (size_t)n);              /* R_v^-1, all v */
+    Sc = malloc(sizeof(double) * bb);
+    Rf = malloc(sizeof(double) * bb);
+    Si = malloc(sizeof(double) * bb);
+    ES = malloc(sizeof(double) * bb);
+    ESE = malloc(sizeof(double) * bb);
+    t1 = malloc(sizeof(double) * (size_t)b);
+    t2 = malloc(sizeof(double) * (size_t)b);
+    double logdet = 0.0;
+    /* the factors R_v, leaves first: S_v = D_v - sum_c E_c S_c^-1 E_c^T */
+    for (int64_t q = n - 1; q >= 0; --q) {
+        int64_t u = bfs[q];
+        sym_from_lower(b, diag + bb * u, Sc);
+        for (int64_t k = first[u]; k < first[u + 1]; ++k) {
+            const double *Ec = edge + bb * kids[k];
+            matmul(b, Rinv + bb * kids[k], 1, Rinv + bb * kids[k], 0, Si);   /* S_c^-1 */
+            matmul(b, Ec, 0, Si, 0, ES);
+            matmul(b, ES, 0, Ec, 1, ESE);
+            for (size_t e2 = 0; e2 < bb; ++e2) Sc[e2] = Sc[e2] - ESE[e2];
+        }
+        if (cholesky_lower(b, Sc, Rf) != 0) { info = (int)u; goto out; }
+        for (int k = 0; k < b; ++k) logdet += 2.0 * log(Rf[k * (b + 1)]);
+        lower_inverse(b, Rf, Rinv + bb * u);
+    }
+    if (logdet_out) *logdet_out = logdet;
+    /* w = L^-T z, root first */
+    matvec(b, Rinv + bb * root, 1, z + (size_t)b * root, w + (size_t)b * root);
+    for (int64_t q = 1; q < n; ++q) {
+        int64_t u = bfs[q], pu = parent[u];
+        matvec(b, edge + bb * u, 1, w + (size_t)b * pu, t1);                 /* E_v^T w_p */
+        matvec(b, Rinv + bb * u, 0, t1, t2);                                 /* R_v^-1 E_v^T w_p */
+        for (int k = 0; k < b; ++k) t1[k] = z[(size_t)b * u + k] - t2[k];
+        matvec(b, Rinv + bb * u, 1, t1, w + (size_t)b * u);                  /* R_v^-T (...) */
+    }
+out:
+    free(first); free(kids); free(next); free(bfs);
+    free(Rinv); free(Sc); free(Rf); free(Si); free(ES); free(ESE); free(t1); free(t2);
+    return info;
+}
+
+/* Batched tree draws: z, w [trees,n,b]; logdet [trees] or NULL; info [trees]. */
+int oracle_tree_sample(const int32_t *parent, int64_t trees, int64_t n, int b, const double *diag,
+                       const double *edge, const double *z, double *w, double *logdet, int32_t *info)
+{
+    if (trees < 0 || n < 1 || b < 1 || !parent || !diag || !edge || !z || !w || !info) return 1;
+    const size_t bb = (size_t)b * b;
+    int64_t e;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (e = 0; e < trees; ++e) {
+        info[e] = tree_sample_one(n, b, parent + n * e, diag + bb * n * e, edge + bb * n * e,
+                                  z + (size_t)b * n * e, w + (size_t)b * n * e, logdet ? logdet + e : NULL);
+    }
+    return 0;
+}
+
+/*
  * Batched trees: parent [trees,n] (int32, root = -1), diag/edge
  * [trees,n,b,b] (edge root slot ignored), outputs G_diag/G_edge
  * [trees,n,b,b] (G_edge root slot set to 0), logdet [trees], info [trees]

@@ -367,6 +367,50 @@ def pin_sample_mean(lib=None):
     return worst
 
 
+def _children_first(parent):
+    """Reverse breadth-first order of a rooted tree (every child before its parent)."""
+    n = len(parent)
+    kids = [[] for _ in range(n)]
+    root = int(np.where(parent < 0)[0][0])
+    for v in range(n):
+        if parent[v] >= 0:
+            kids[parent[v]].append(v)
+    order, head = [root], 0
+    while head < len(order):
+        order.extend(kids[order[head]])
+        head += 1
+    return order[::-1]
+
+
+def pin_tree_sample_standard_basis(lib=None):
+    """Tree draws for z = e_k against numpy's dense Cholesky of A in a
+    children-first order (mapped back to node order), and W W^T = A^-1;
+    log det against slogdet.  Path, star, balanced and random trees."""
+    worst = 0.0
+    rng = np.random.default_rng(67)
+    cases = [path_parent(5), star_parent(5), balanced_parent(7), inputs.random_parent(rng, 9)]
+    for k, parent in enumerate(cases):
+        b = 2 if k % 2 else 3
+        n = len(parent)
+        P = parent[None]
+        d, e = inputs.tree_inputs_from_parent(P, b, seed=68 + k, load=1.0)
+        A = tree_dense(parent, d[0], e[0])
+        N = n * b
+        z = np.eye(N).reshape(N, n, b)
+        out = oracle.tree_sample(np.repeat(P, N, 0), np.repeat(d, N, 0), np.repeat(e, N, 0), z, lib=lib)
+        if (out["info"] != -1).any():
+            return float("inf")
+        W = out["eta"].reshape(N, N).T
+        idx = np.concatenate([np.arange(v * b, (v + 1) * b) for v in _children_first(parent)])
+        Mp = np.linalg.inv(np.linalg.cholesky(A[np.ix_(idx, idx)])).T
+        ref = np.empty_like(Mp)
+        ref[np.ix_(idx, idx)] = Mp
+        worst = max(worst, rel(W, ref), rel(W @ W.T, np.linalg.inv(A)))
+        sl = np.linalg.slogdet(A)[1]
+        worst = max(worst, abs(out["logdet"][0] - sl) / max(1.0, abs(sl)))
+    return worst
+
+
 # name -> (function, tolerance)
 PINS = {
     "tiny_chains_dense": (pin_tiny_chains_dense, 1e-12),
@@ -381,5 +425,6 @@ PINS = {
     "root_invariance": (pin_root_invariance, 1e-11),
     "sample_standard_basis": (pin_sample_standard_basis, 1e-12),
     "sample_mean": (pin_sample_mean, 1e-12),
+    "tree_sample_standard_basis": (pin_tree_sample_standard_basis, 1e-12),
     "not_spd": (pin_not_spd, 0.5),
 }

@@ -48,6 +48,12 @@ MUTANTS = {
                     "for (int k = 0; k < b; ++k) v1[k] = z[(size_t)b * i + k] + v2[k];"),
     "sample_schur_sign": ("for (size_t k = 0; k < bb; ++k) S[k] = S[k] - BSB[k];",
                           "for (size_t k = 0; k < bb; ++k) S[k] = S[k] + BSB[k];"),
+    "tree_sample_root_untransposed": ("matvec(b, Rinv + bb * root, 1, z + (size_t)b * root, w + (size_t)b * root);",
+                                      "matvec(b, Rinv + bb * root, 0, z + (size_t)b * root, w + (size_t)b * root);"),
+    "tree_sample_edge_transposed": ("matvec(b, edge + bb * u, 1, w + (size_t)b * pu, t1);",
+                                    "matvec(b, edge + bb * u, 0, w + (size_t)b * pu, t1);"),
+    "tree_sample_sign": ("for (int k = 0; k < b; ++k) t1[k] = z[(size_t)b * u + k] - t2[k];",
+                         "for (int k = 0; k < b; ++k) t1[k] = z[(size_t)b * u + k] + t2[k];"),
     "tree_g_diag_transposed": ("matmul(b, Sinv + bb * v, 0, edge + bb * v, 1, T1);",
                                "matmul(b, Sinv + bb * v, 0, edge + bb * v, 0, T1);"),
 }
