@@ -245,6 +245,21 @@ selinv_status selinv_tree(const selinv_tree_plan_t *plan, selinv_dtype dtype, in
                           void *G_diag, void *G_edge, double *logdet, int32_t *info,
                           void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Gaussian draw on block trees (gabp-sparse-inv, "Gaussian sampling":
+ * sample_gaussian_tree draws x ~ N(0, A^-1) reusing the factorisation):
+ *   eta = P^T L^-T z,  A = P^T L L^T P
+ * with P the tree's own elimination order (children before parents; the
+ * factor's blocks do not depend on the order among siblings): L_vv = R_v,
+ * S_v = R_v R_v^T, and L_{parent(v), v} = edge[v] R_v^-T.  z [trees, n, b]
+ * are the caller's standard normals, eta [trees, n, b] the draw; diag, edge,
+ * logdet, info, workspace and errors as in selinv_tree (b <= 16).
+ */
+selinv_status selinv_tree_sample(const selinv_tree_plan_t *plan, selinv_dtype dtype, int32_t b,
+                                 const void *diag, const void *edge, const void *z, void *eta,
+                                 double *logdet, int32_t *info,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -67,6 +67,8 @@ struct TreeDev {
 template <class T> struct TreeBufs {
     const T *diag, *edge;
     T *G_diag, *G_edge;
+    const T *z;              // draws: standard normals [N, b]
+    T *eta;                  // draws: R_v z_v after the collect sweep, the draw after the distribute sweep
     T *ws_sinv, *ws_u;       // per node lower slots
     double *ws_ld;           // per node log det S_v
     int32_t *info;           // per tree, INT_MAX = ok until finalised
@@ -129,7 +131,7 @@ template <class T> SELINV_DEVINL void load_lower_slot_l2(w16::Tile<T> &a, const 
     }
 }
 
-template <class T, bool FULL>
+template <class T, bool FULL, bool DRAW = false>
 __global__ void __launch_bounds__(TWARPS * 32)
 tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leaves, int64_t nleaves)
 {
@@ -179,10 +181,49 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leave
             LogAcc det;
             det.init();
             bool bad = false;
-            spd_inverse<T>(a, cb, g, t, det, bad);
+            T vv[2] = {T(0), T(0)};                  // draws: R_v z_v at rows g, g + 8 (S_v = R_v R_v^T)
+            if constexpr (DRAW) {
+                T zc[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) zc[q] = tcol(t, q) < b ? p.z[(int64_t)v * b + tcol(t, q)] : T(0);
+                if constexpr (sizeof(T) == 8) {
+                    spd_inverse_blocked<true>(a, g, t, det, bad, zc, vv);
+                } else {
+                    Tile<T> rf = a;
+                    chol_lower(rf, g, t);
+                    lower_matvec(vv, rf, zc, g, t);
+                    spd_inverse<T>(a, cb, g, t, det, bad);
+                }
+            } else {
+                spd_inverse<T>(a, cb, g, t, det, bad);
+            }
             if (lane == 0) {
                 p.ws_ld[v] = det.log_value();
                 if (bad) atomicMin(p.info + v / td.n, (int32_t)(v % td.n));
+            }
+            if (DRAW && par < 0) {                   // root: w = S^-1 R z = R^-T z, published
+                if (t == 0) {
+                    cb[g] = vv[0];
+                    cb[g + 8] = vv[1];
+                }
+                __syncwarp();
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    T s2 = T(0);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) s2 = fma(a.v[h][q], cb[tcol(t, q)], s2);
+                    s2 += shfl_xor(s2, 1);
+                    s2 += shfl_xor(s2, 2);
+                    if (t == 0 && g + 8 * h < b) p.eta[(int64_t)v * b + g + 8 * h] = s2;
+                }
+                __syncwarp();                         // the warp's stores are ordered before lane 0's release
+                if (lane == 0) st_release(sy.done + v, 1);
+                __syncwarp();
+                break;
+            }
+            if (DRAW && t == 0) {                     // R_v z_v, for the distribute sweep
+                if (g < b) p.eta[(int64_t)v * b + g] = vv[0];
+                if (g + 8 < b) p.eta[(int64_t)v * b + g + 8] = vv[1];
             }
             if (par < 0) {                            // root: G = S^-1, G_edge = 0, published
                 __syncwarp();
@@ -217,7 +258,7 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leave
     }
 }
 
-template <class T, bool FULL>
+template <class T, bool FULL, bool DRAW = false>
 __global__ void __launch_bounds__(TWARPS * 32)
 tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *nodes, int64_t count)
 {
@@ -262,7 +303,7 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
         }
         ok = __shfl_sync(FULL_MASK, ok, 0);
         __syncwarp();                                 // every lane's reads below are ordered after lane 0's acquire
-        if (ok) load_lower_async<T, FULL>(sG, p.G_diag + (int64_t)par * bb, b, lane);   // G_pp (lower), from L2
+        if (ok && !DRAW) load_lower_async<T, FULL>(sG, p.G_diag + (int64_t)par * bb, b, lane);   // G_pp, from L2
         cp_async_commit();
         if (kn < cnt) {
             const int32_t vn = nodes[kn];
@@ -285,6 +326,36 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
         to_smem<T>(sT, a, g, t);                      // lower entries of S_v^-1 valid
         __syncwarp();
         from_smem_lower<T>(a, sT, g, t);              // S_v^-1, full
+        if constexpr (DRAW) {
+            // w_v = R_v^-T z_v - S_v^-1 E_v^T w_p = S_v^-1 (R_v z_v) - W_v^T w_p, with
+            // R_v z_v left in eta by the collect sweep and w_p published by the parent
+            Tile<T> et, wt;
+            from_smem<T>(et, sBuf(cur), g, t);        // E_v
+            zero(wt);
+            gemm_nt<false>(wt, a, et, sT, sT2, g, t); // W_v^T = S_v^-1 E_v^T
+            T uc[4], wc[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int c = tcol(t, q);
+                uc[q] = c < b ? __ldcg(p.eta + (int64_t)v * b + c) : T(0);
+                wc[q] = c < b ? __ldcg(p.eta + (int64_t)par * b + c) : T(0);
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                T s2 = T(0);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) s2 = fma(a.v[h][q], uc[q], fma(-wt.v[h][q], wc[q], s2));
+                s2 += shfl_xor(s2, 1);
+                s2 += shfl_xor(s2, 2);
+                if (t == 0 && g + 8 * h < b) p.eta[(int64_t)v * b + g + 8 * h] = s2;
+            }
+            __syncwarp();                             // the warp's stores are ordered before lane 0's release
+            if (lane == 0 && td.child_ptr[v + 1] > td.child_ptr[v]) st_release(sy.done + v, 1);
+            __syncwarp();
+            k = kn;
+            cur ^= 1;
+            continue;
+        }
         Tile<T> gp, et, wt, get;
         from_smem_lower<T>(gp, sG, g, t);             // G_pp, full
         from_smem<T>(et, sBuf(cur), g, t);            // E_v
@@ -360,7 +431,8 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 template <class T>
 cudaError_t run_tree(const selinv_tree_plan_s *pl, int b, const T *diag, const T *edge, T *G_diag, T *G_edge,
-                     double *logdet, int32_t *info, void *ws, bool full, cudaStream_t s)
+                     double *logdet, int32_t *info, void *ws, bool full, cudaStream_t s, const T *z = nullptr,
+                     T *eta = nullptr)
 {
     const int64_t N = pl->trees * pl->n;
     char *w = static_cast<char *>(ws);
@@ -369,6 +441,9 @@ cudaError_t run_tree(const selinv_tree_plan_s *pl, int b, const T *diag, const T
     p.edge = edge;
     p.G_diag = G_diag;
     p.G_edge = G_edge;
+    p.z = z;
+    p.eta = eta;
+    const bool draw = z != nullptr;
     p.ws_sinv = reinterpret_cast<T *>(w);
     w += align256(N * slot_bytes<T>());
     p.ws_u = reinterpret_cast<T *>(w);
@@ -390,8 +465,10 @@ cudaError_t run_tree(const selinv_tree_plan_s *pl, int b, const T *diag, const T
                                                                info, pl->trees);
     const size_t smem = sizeof(T) * tree_smem_elems<T>() * TWARPS;
     const size_t smem_d = sizeof(T) * dist_smem_elems<T>() * TWARPS;
-    auto kc = full ? tree_collect_kernel<T, true> : tree_collect_kernel<T, false>;
-    auto kd = full ? tree_distribute_kernel<T, true> : tree_distribute_kernel<T, false>;
+    auto kc = draw ? (full ? tree_collect_kernel<T, true, true> : tree_collect_kernel<T, false, true>)
+                   : (full ? tree_collect_kernel<T, true> : tree_collect_kernel<T, false>);
+    auto kd = draw ? (full ? tree_distribute_kernel<T, true, true> : tree_distribute_kernel<T, false, true>)
+                   : (full ? tree_distribute_kernel<T, true> : tree_distribute_kernel<T, false>);
     cudaError_t err = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err == cudaSuccess) err = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_d);
     if (err != cudaSuccess) return err;
@@ -576,6 +653,36 @@ selinv_status selinv_tree(const selinv_tree_plan_t *pl, selinv_dtype dtype, int3
         err = run_tree<float>(pl, b, static_cast<const float *>(diag), static_cast<const float *>(edge),
                               static_cast<float *>(G_diag), static_cast<float *>(G_edge), logdet, info,
                               workspace, full, s);
+    return err == cudaSuccess ? SELINV_OK : SELINV_ERR_CUDA;
+}
+
+selinv_status selinv_tree_sample(const selinv_tree_plan_t *pl, selinv_dtype dtype, int32_t b, const void *diag,
+                                 const void *edge, const void *z, void *eta, double *logdet, int32_t *info,
+                                 void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!pl || (dtype != SELINV_F64 && dtype != SELINV_F32) || b < 1) return SELINV_ERR_INVALID_ARG;
+    if (b > 16) return SELINV_ERR_UNSUPPORTED;
+    if (!diag || !edge || !z || !eta || !info) return SELINV_ERR_INVALID_ARG;
+    const size_t es = dtype == SELINV_F64 ? 8 : 4;
+    if (!is_aligned(diag, es) || !is_aligned(edge, es) || !is_aligned(z, es) || !is_aligned(eta, es) ||
+        !is_aligned(logdet, 8) || !is_aligned(info, 4) || !is_aligned(workspace, 256))
+        return SELINV_ERR_INVALID_ARG;
+    const size_t need = tree_workspace(pl, es);
+    if (!workspace || workspace_bytes < need) return SELINV_ERR_WORKSPACE;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev != pl->device) return SELINV_ERR_INVALID_ARG;
+    const bool full = b == 16 && is_aligned(diag, 16) && is_aligned(edge, 16);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t err;
+    if (dtype == SELINV_F64)
+        err = run_tree<double>(pl, b, static_cast<const double *>(diag), static_cast<const double *>(edge), nullptr,
+                               nullptr, logdet, info, workspace, full, s, static_cast<const double *>(z),
+                               static_cast<double *>(eta));
+    else
+        err = run_tree<float>(pl, b, static_cast<const float *>(diag), static_cast<const float *>(edge), nullptr,
+                              nullptr, logdet, info, workspace, full, s, static_cast<const float *>(z),
+                              static_cast<float *>(eta));
     return err == cudaSuccess ? SELINV_OK : SELINV_ERR_CUDA;
 }
 

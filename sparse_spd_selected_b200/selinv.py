@@ -74,6 +74,8 @@ def lib():
         L.selinv_tree_workspace_size.argtypes = [P, ctypes.c_int, I32]
         L.selinv_tree_workspace_size.restype = SZ
         L.selinv_tree.argtypes = [P, ctypes.c_int, I32, P, P, P, P, P, P, P, SZ, P]
+        L.selinv_tree_sample.argtypes = [P, ctypes.c_int, I32, P, P, P, P, P, P, P, SZ, P]
+        L.selinv_tree_sample.restype = ctypes.c_int
         L.selinv_tree.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -396,3 +398,44 @@ def selinv_tree(plan: TreePlan, diag: torch.Tensor, edge: torch.Tensor, *, check
     if single:
         G_diag, G_edge = G_diag[0], G_edge[0]
     return {"G_diag": G_diag, "G_edge": G_edge, "logdet": logdet, "info": info}
+
+
+def tree_sample(plan: TreePlan, diag: torch.Tensor, edge: torch.Tensor, z: torch.Tensor, *, check=True, out=None,
+                workspace=None, stream=None):
+    """Gaussian draw on block trees: eta = L^-T z for A = L L^T in the tree's own
+    elimination order (children before parents), z [trees, n, b] the caller's
+    standard normals (b <= 16).  Returns dict with eta, logdet and info."""
+    _cuda_contig("diag", diag)
+    dt = diag.dtype
+    _cuda_contig("edge", edge, dt)
+    _cuda_contig("z", z, dt)
+    single = diag.dim() == 3
+    d4 = diag[None] if single else diag
+    e4 = edge[None] if single else edge
+    z3 = z[None] if single else z
+    if d4.dim() != 4 or tuple(d4.shape[:2]) != (plan.trees, plan.n) or d4.shape[-1] != d4.shape[-2]:
+        raise ValueError(f"diag must be [{plan.trees}, {plan.n}, b, b]")
+    if e4.shape != d4.shape:
+        raise ValueError("edge must have diag's shape")
+    b = int(d4.shape[-1])
+    if tuple(z3.shape) != (plan.trees, plan.n, b):
+        raise ValueError(f"z must be [{plan.trees}, {plan.n}, {b}]")
+    dev = diag.device
+    out = dict(out or {})
+    eta = out.get("eta")
+    if eta is None:
+        eta = torch.empty_like(z3)
+    logdet = out.get("logdet")
+    if logdet is None:
+        logdet = torch.empty(plan.trees, dtype=torch.float64, device=dev)
+    info = out.get("info")
+    if info is None:
+        info = torch.empty(plan.trees, dtype=torch.int32, device=dev)
+    nbytes = plan.workspace_size(dt, b)
+    ws = _workspace(nbytes, dev, workspace)
+    with torch.cuda.device(dev):
+        st = lib().selinv_tree_sample(plan.handle, _code(dt), b, _ptr(d4), _ptr(e4), _ptr(z3), _ptr(eta),
+                                      _ptr(logdet), _ptr(info), _ptr(ws), nbytes, _stream_handle(stream))
+    _check(st, "selinv_tree_sample")
+    _raise_on_info(info, check)
+    return {"eta": eta[0] if single else eta, "logdet": logdet, "info": info}
