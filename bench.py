@@ -62,7 +62,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--op", default="selinv", choices=["selinv", "sample"],
                     help="selinv: selected inverse + log det (+ solve); sample: Gaussian draw "
-                         "eta = A^-1 r + L^-T z + log det (chain workloads with b <= 16)")
+                         "eta = A^-1 r + L^-T z + log det (chains; on trees eta = L^-T z)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -161,7 +161,9 @@ def oracle_inputs(w, elems, op):
 
 
 def oracle_run(oracle, w, g, op):
-    if w.kind == "tree":
+    if w.kind == "tree" and op == "sample":
+        oracle.tree_sample(g["parent"], g["diag"], g["edge"], g["z"])
+    elif w.kind == "tree":
         oracle.tree(g["parent"], g["diag"], g["edge"])
     elif op == "sample":
         oracle.chain_sample(g["diag"], g["lower"], g["z"], rhs=g.get("rhs"))
@@ -199,8 +201,11 @@ def cpu_baseline(w, dtype_name, op="selinv", budget_s=10.0):
 def algorithmic_bytes(w, es, batch, op="selinv"):
     """Bytes the method must move: read D and B (or edge) blocks, write G_diag and G_lower
     (or G_edge) blocks, plus the right-hand side and solution when solving.  A draw reads
-    D, B, r and z and writes eta."""
+    D, B, r and z and writes eta (a tree draw has no r)."""
     b2 = w.b * w.b
+    if op == "sample" and w.kind == "tree":
+        n = batch * w.L
+        return es * (b2 * n + b2 * (n - batch) + 2 * w.b * n)
     if op == "sample":
         nodes, edges = batch * w.L, batch * (w.L - 1)
         return es * (b2 * nodes + b2 * edges + 3 * w.b * nodes)
@@ -349,8 +354,8 @@ def run_ours(args):
     else:
         g = inputs.generate(w, elements=elems)   # per-element seeds: rank r owns its own slice
         if args.op == "sample":
-            if w.kind != "chain" or (w.b > 16 and args.dtype != "f64"):
-                raise SystemExit("--op sample runs on chain workloads (b > 16 in float64 only)")
+            if w.b > 16 and args.dtype != "f64":
+                raise SystemExit("--op sample with b > 16 runs in float64 only")
             g["z"] = inputs.standard_normals(w.batch, w.L, w.b, w.seed, elems)
         host_in = {k: torch.from_numpy(v).to(tdt).pin_memory() for k, v in g.items()
                    if v is not None and k != "parent"}
@@ -365,10 +370,18 @@ def run_ours(args):
                "logdet": torch.empty(batch, dtype=torch.float64, device="cuda"),
                "info": torch.empty(batch, dtype=torch.int32, device="cuda")}
         ws = torch.empty(plan.workspace_size(tdt, w.b), dtype=torch.uint8, device="cuda")
-        kernel = "tree_collect_kernel"
+        if args.op == "sample":
+            kernel = "tree_collect_kernel (draw mode)"
+            out = {"eta": torch.empty_like(dev_in["z"]), "logdet": out["logdet"], "info": out["info"]}
 
-        def step():
-            selinv.selinv_tree(plan, dev_in["diag"], dev_in["edge"], check=False, out=out, workspace=ws)
+            def step():
+                selinv.tree_sample(plan, dev_in["diag"], dev_in["edge"], dev_in["z"], check=False, out=out,
+                                   workspace=ws)
+        else:
+            kernel = "tree_collect_kernel"
+
+            def step():
+                selinv.selinv_tree(plan, dev_in["diag"], dev_in["edge"], check=False, out=out, workspace=ws)
     else:
         if w.kind == "grid":
             dev_in = {"diag": diag, "lower": lower}

@@ -454,12 +454,11 @@ SELINV_DEVINL void spd_inverse_blocked(Big<double> &a, double *cbuf, double *tbu
             pv[1] = u.y;
         }
         double wk = 0.0;                                          // (R_KK z_K) at row 8K + g
-        if (DRAW) {
-            double rc[2] = {pv[0], pv[1]};
-            chol8(rc, x.lane, x.g, x.t);
-            wk = lower8_rowdot(rc, zs[8 * K + 2 * x.t], zs[8 * K + 2 * x.t + 1], x.g, x.t);
-        }
-        inv8_sweep(pv, x.lane, x.g, x.t, det, bad, x.tid == 0);
+        if (DRAW && x.cw == 0)
+            inv8_sweep<true>(pv, x.lane, x.g, x.t, det, bad, x.tid == 0, zs[8 * K + 2 * x.t],
+                             zs[8 * K + 2 * x.t + 1], &wk);
+        else
+            inv8_sweep(pv, x.lane, x.g, x.t, det, bad, x.tid == 0);
         // T = A_{rows,K} P^-1 for this warp's rows: 4 m-tiles x 2 k-steps
         double T[4][2];
 #pragma unroll

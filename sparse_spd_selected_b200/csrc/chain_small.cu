@@ -110,16 +110,13 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
         // Draw: with S_i = R_i R_i^T, S_i^-1 (y_i + R_i z_i) = S_i^-1 y_i + R_i^-T z_i, so
         // storing y_i + R_i z_i for the backward sweep turns its x = A^-1 r into
         // eta = A^-1 r + L^-T z (L^-T z_i = R_i^-T z_i - W_i^T (L^-T z)_{i+1}).
-        // float64 meets R_i z_i inside the blocked inverse; float32 factors a copy.
+        // The inverse's own pivot sweep meets R_i z_i on the way.
         T v[2] = {T(0), T(0)};
         if constexpr (SAMPLE && sizeof(T) == 8) {
             spd_inverse_blocked<true>(a, g, t, det, bad, zc, v);   // a = S_i^-1, v = R_i z_i
+        } else if constexpr (SAMPLE) {
+            spd_inverse_scalar<T, true>(a, cb, g, t, det, bad, zc, v);
         } else {
-            if (SAMPLE) {
-                Tile<T> rf = a;
-                chol_lower(rf, g, t);
-                lower_matvec(v, rf, zc, g, t);
-            }
             spd_inverse<T>(a, cb, g, t, det, bad);    // a = S_i^-1
         }
         if (SAMPLE) {

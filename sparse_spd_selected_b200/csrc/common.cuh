@@ -58,6 +58,8 @@ SELINV_DEVINL double recip(double d)
     return fma(r, fma(e, e, e), r);
 }
 SELINV_DEVINL float recip(float d) { return __frcp_rn(d); }
+SELINV_DEVINL double rsqrt_t(double d) { return rsqrt(d); }
+SELINV_DEVINL float rsqrt_t(float d) { return rsqrtf(d); }
 
 template <class T> SELINV_DEVINL T shfl(T v, int src) { return __shfl_sync(FULL_MASK, v, src); }
 template <class T> SELINV_DEVINL T shfl_xor(T v, int m) { return __shfl_xor_sync(FULL_MASK, v, m); }
@@ -84,7 +86,14 @@ struct LogAcc {
 // P_ij -= P_ik P_kj / d, P_ik /= d, P_kj /= d, P_kk = -1/d, then negated.
 // Row and column k travel by shuffles.  The pivots are multiplied into det
 // (when `count`), a pivot that is not > 0 sets bad.
-SELINV_DEVINL void inv8_sweep(double v[2], int lane, int g, int t, LogAcc &det, bool &bad, bool count)
+// DRAW: also rz = (R z)[g] for the Cholesky factor P = R R^T and z at the
+// lane's columns 2t, 2t+1 (z0, z1).  At step k the entries P[i][k], i >= k,
+// not yet swept are the Schur-complement column that Cholesky scales:
+// R[i][k] = P[i][k] / sqrt(d), so rz += P[g][k] z_k / sqrt(d) for g >= k.
+// The sweep's own chain does not wait for this sum.
+template <bool DRAW = false>
+SELINV_DEVINL void inv8_sweep(double v[2], int lane, int g, int t, LogAcc &det, bool &bad, bool count,
+                              double z0 = 0.0, double z1 = 0.0, double *rz = nullptr)
 {
     // v = P[g][2t], P[g][2t+1] of a symmetric positive definite 8 x 8 P
 #pragma unroll
@@ -98,6 +107,10 @@ SELINV_DEVINL void inv8_sweep(double v[2], int lane, int g, int t, LogAcc &det, 
         bad |= !(d > 0.0);
         if (count) det.mul(d);
         const double p = recip(d);
+        if (DRAW) {
+            const double zk = shfl(kj ? z1 : z0, (lane & ~3) | kt);
+            if (g >= k) *rz = fma(c, zk * rsqrt(d), *rz);
+        }
         const double tc = c * p;
         v[0] = fma(-tc, row[0], v[0]);
         v[1] = fma(-tc, row[1], v[1]);
@@ -110,43 +123,6 @@ SELINV_DEVINL void inv8_sweep(double v[2], int lane, int g, int t, LogAcc &det, 
     }
     v[0] = -v[0];
     v[1] = -v[1];
-}
-
-// Cholesky factor of a symmetric positive definite 8 x 8 matrix in the same
-// layout, P = R R^T with R lower triangular (entries above the diagonal left
-// unspecified): for each column k, R_kk = sqrt(P_kk), R_ik = P_ik / R_kk,
-// P_ij -= R_ik R_jk (i, j > k); the column travels by shuffles.
-SELINV_DEVINL void chol8(double v[2], int lane, int g, int t)
-{
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const int kt = k >> 1, kj = k & 1;
-        const double inv = recip(sqrt(shfl(v[kj], (k << 2) | kt)));
-        const double c = shfl(v[kj], (lane & ~3) | kt);             // P[g][k]
-        const double li = g >= k ? c * inv : 0.0;
-        double lj[2];
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {                                // P[2t+j][k]
-            const double u = shfl(v[kj], ((2 * t + j) << 2) | kt);
-            lj[j] = 2 * t + j > k ? u * inv : 0.0;
-        }
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            if (g > k) v[j] = fma(-li, lj[j], v[j]);
-            if (2 * t + j == k) v[j] = li;
-        }
-    }
-}
-
-// sum_c R[g][c] x[c] over an 8 x 8 lower-triangular R in that layout, x at the
-// lane's columns 2t, 2t+1; every lane of row g ends with the sum.
-SELINV_DEVINL double lower8_rowdot(const double r[2], double x0, double x1, int g, int t)
-{
-    double s = (2 * t <= g ? r[0] * x0 : 0.0);
-    if (2 * t + 1 <= g) s = fma(r[1], x1, s);
-    s += shfl_xor(s, 1);
-    s += shfl_xor(s, 2);
-    return s;
 }
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }

@@ -48,6 +48,7 @@ namespace selinv {
 namespace {
 
 constexpr int TWARPS = 4;
+constexpr int DRAW_SLOT = 256;      // draws: W_v^T per node, 16 x 16 row-major (>= SLOT_ELEMS)
 
 template <class T> __host__ __device__ constexpr int tree_smem_elems() { return 4 * w16::SL<T>::ELEMS + 64; }
 // distribute: two (edge, S^-1 slot) buffer sets for the node being processed
@@ -154,16 +155,23 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leave
             if (par >= 0) load_block_async<T, FULL>(sB, p.edge + v * bb, b, lane);   // E_v
             load_lower_async<T, FULL>(sD, p.diag + v * bb, b, lane);                 // D_v
             cp_async_commit();
-            Tile<T> acc;                              // sum of the children's U_c (lower slots)
-            zero(acc);
+            T zc[4];                                  // draws: z_v at the lane's columns
+            if constexpr (DRAW) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) zc[q] = tcol(t, q) < b ? p.z[(int64_t)v * b + tcol(t, q)] : T(0);
+            }
+            Tile<T> acc;                              // sum of the children's U_c (lower slots), two
+            zero(acc);                                // children's loads in flight at a time
             const int32_t c0 = td.child_ptr[v], c1 = td.child_ptr[v + 1];
-            for (int32_t c = c0; c < c1; ++c) {
-                Tile<T> u;
+            for (int32_t c = c0; c < c1; c += 2) {
+                Tile<T> u, u2;
                 load_lower_slot_l2<T>(u, p.ws_u + (int64_t)td.child_idx[c] * SLOT_ELEMS, lane, g, t);
+                if (c + 1 < c1) load_lower_slot_l2<T>(u2, p.ws_u + (int64_t)td.child_idx[c + 1] * SLOT_ELEMS, lane, g, t);
+                else zero(u2);
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) acc.v[h][q] += u.v[h][q];
+                    for (int q = 0; q < 4; ++q) acc.v[h][q] += u.v[h][q] + u2.v[h][q];
             }
             cp_async_wait_all();
             __syncwarp();
@@ -183,17 +191,8 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leave
             bool bad = false;
             T vv[2] = {T(0), T(0)};                  // draws: R_v z_v at rows g, g + 8 (S_v = R_v R_v^T)
             if constexpr (DRAW) {
-                T zc[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) zc[q] = tcol(t, q) < b ? p.z[(int64_t)v * b + tcol(t, q)] : T(0);
-                if constexpr (sizeof(T) == 8) {
-                    spd_inverse_blocked<true>(a, g, t, det, bad, zc, vv);
-                } else {
-                    Tile<T> rf = a;
-                    chol_lower(rf, g, t);
-                    lower_matvec(vv, rf, zc, g, t);
-                    spd_inverse<T>(a, cb, g, t, det, bad);
-                }
+                if constexpr (sizeof(T) == 8) spd_inverse_blocked<true>(a, g, t, det, bad, zc, vv);
+                else spd_inverse_scalar<T, true>(a, cb, g, t, det, bad, zc, vv);
             } else {
                 spd_inverse<T>(a, cb, g, t, det, bad);
             }
@@ -201,7 +200,7 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leave
                 p.ws_ld[v] = det.log_value();
                 if (bad) atomicMin(p.info + v / td.n, (int32_t)(v % td.n));
             }
-            if (DRAW && par < 0) {                   // root: w = S^-1 R z = R^-T z, published
+            if constexpr (DRAW) {                     // u_v = S_v^-1 R_v z_v = R_v^-T z_v
                 if (t == 0) {
                     cb[g] = vv[0];
                     cb[g + 8] = vv[1];
@@ -216,14 +215,12 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leave
                     s2 += shfl_xor(s2, 2);
                     if (t == 0 && g + 8 * h < b) p.eta[(int64_t)v * b + g + 8 * h] = s2;
                 }
-                __syncwarp();                         // the warp's stores are ordered before lane 0's release
-                if (lane == 0) st_release(sy.done + v, 1);
-                __syncwarp();
-                break;
-            }
-            if (DRAW && t == 0) {                     // R_v z_v, for the distribute sweep
-                if (g < b) p.eta[(int64_t)v * b + g] = vv[0];
-                if (g + 8 < b) p.eta[(int64_t)v * b + g + 8] = vv[1];
+                if (par < 0) {                        // root: its draw is u_v, published
+                    __syncwarp();                     // the warp's stores are ordered before lane 0's release
+                    if (lane == 0) st_release(sy.done + v, 1);
+                    __syncwarp();
+                    break;
+                }
             }
             if (par < 0) {                            // root: G = S^-1, G_edge = 0, published
                 __syncwarp();
@@ -239,11 +236,12 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leave
                 __syncwarp();
                 break;
             }
-            store_lower_slot<T>(p.ws_sinv + (int64_t)v * SLOT_ELEMS, a, lane, g, t);
+            if (!DRAW) store_lower_slot<T>(p.ws_sinv + (int64_t)v * SLOT_ELEMS, a, lane, g, t);
             Tile<T> et, w, u;
             from_smem<T>(et, sB, g, t);               // E_v
             zero(w);
             gemm_nt<false>(w, et, a, sT, sT2, g, t);  // W_v = E_v S_v^-1
+            if (DRAW) store_block_T<T, true>(p.ws_sinv + (int64_t)v * DRAW_SLOT, w, 16, g, t);   // W_v^T, 16 x 16
             zero(u);
             gemm_nt<false, true>(u, w, et, sT, sT2, g, t);   // U_v = W_v E_v^T (lower tiles)
             store_lower_slot<T>(p.ws_u + (int64_t)v * SLOT_ELEMS, u, lane, g, t);
@@ -258,7 +256,7 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leave
     }
 }
 
-template <class T, bool FULL, bool DRAW = false>
+template <class T, bool FULL>
 __global__ void __launch_bounds__(TWARPS * 32)
 tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *nodes, int64_t count)
 {
@@ -303,7 +301,7 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
         }
         ok = __shfl_sync(FULL_MASK, ok, 0);
         __syncwarp();                                 // every lane's reads below are ordered after lane 0's acquire
-        if (ok && !DRAW) load_lower_async<T, FULL>(sG, p.G_diag + (int64_t)par * bb, b, lane);   // G_pp, from L2
+        if (ok) load_lower_async<T, FULL>(sG, p.G_diag + (int64_t)par * bb, b, lane);   // G_pp, from L2
         cp_async_commit();
         if (kn < cnt) {
             const int32_t vn = nodes[kn];
@@ -326,36 +324,6 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
         to_smem<T>(sT, a, g, t);                      // lower entries of S_v^-1 valid
         __syncwarp();
         from_smem_lower<T>(a, sT, g, t);              // S_v^-1, full
-        if constexpr (DRAW) {
-            // w_v = R_v^-T z_v - S_v^-1 E_v^T w_p = S_v^-1 (R_v z_v) - W_v^T w_p, with
-            // R_v z_v left in eta by the collect sweep and w_p published by the parent
-            Tile<T> et, wt;
-            from_smem<T>(et, sBuf(cur), g, t);        // E_v
-            zero(wt);
-            gemm_nt<false>(wt, a, et, sT, sT2, g, t); // W_v^T = S_v^-1 E_v^T
-            T uc[4], wc[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int c = tcol(t, q);
-                uc[q] = c < b ? __ldcg(p.eta + (int64_t)v * b + c) : T(0);
-                wc[q] = c < b ? __ldcg(p.eta + (int64_t)par * b + c) : T(0);
-            }
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                T s2 = T(0);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) s2 = fma(a.v[h][q], uc[q], fma(-wt.v[h][q], wc[q], s2));
-                s2 += shfl_xor(s2, 1);
-                s2 += shfl_xor(s2, 2);
-                if (t == 0 && g + 8 * h < b) p.eta[(int64_t)v * b + g + 8 * h] = s2;
-            }
-            __syncwarp();                             // the warp's stores are ordered before lane 0's release
-            if (lane == 0 && td.child_ptr[v + 1] > td.child_ptr[v]) st_release(sy.done + v, 1);
-            __syncwarp();
-            k = kn;
-            cur ^= 1;
-            continue;
-        }
         Tile<T> gp, et, wt, get;
         from_smem_lower<T>(gp, sG, g, t);             // G_pp, full
         from_smem<T>(et, sBuf(cur), g, t);            // E_v
@@ -377,6 +345,92 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
         __syncwarp();
         k = kn;
         cur ^= 1;
+    }
+}
+
+// Draws, top-down: w_v = u_v - W_v^T w_p with u_v = R_v^-T z_v and W_v^T
+// left by the collect sweep (W_v^T as a 16 x 16 row-major slot, zero outside
+// b x b) and w_p published by the parent.  A warp takes DCHUNK consecutive
+// nodes of the depth order per atomic and loads all their W_v^T rows and u_v
+// before it waits for the first parent.  Lane (r, hf) = (lane / 2, lane % 2)
+// holds row r, columns 8 hf .. 8 hf + 7.  Every wait ends: a node's parent
+// comes earlier in the order, in an earlier chunk (taken by a running warp) or
+// earlier in the same chunk.
+constexpr int DCHUNK = 4;
+constexpr int DRAW_THREADS = 256;
+
+template <class T, bool FULL>
+__global__ void __launch_bounds__(DRAW_THREADS)
+tree_draw_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *nodes, int64_t count)
+{
+    const int lane = threadIdx.x & 31;
+    const int r = lane >> 1, hf = lane & 1;
+    const int b = p.b;
+    for (;;) {
+        const int64_t k0 = (int64_t)warp_take(sy.counters + 1, lane) * DCHUNK;
+        if (k0 >= count) break;
+        const int m = (int)(count - k0 < DCHUNK ? count - k0 : DCHUNK);
+        T wr[DCHUNK][8], uv[DCHUNK];
+        int32_t vs[DCHUNK], ps[DCHUNK];
+#pragma unroll
+        for (int j = 0; j < DCHUNK; ++j) {
+            vs[j] = j < m ? nodes[k0 + j] : 0;
+            ps[j] = j < m ? td.parent[vs[j]] : 0;
+            const T *row = p.ws_sinv + (int64_t)vs[j] * DRAW_SLOT + r * 16 + 8 * hf;
+            if (j < m) {
+                if constexpr (sizeof(T) == 8) {
+#pragma unroll
+                    for (int c = 0; c < 8; c += 2) {
+                        const double2 x = __ldcs(reinterpret_cast<const double2 *>(row + c));
+                        wr[j][c] = x.x;
+                        wr[j][c + 1] = x.y;
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 8; c += 4) {
+                        const float4 x = __ldcs(reinterpret_cast<const float4 *>(row + c));
+                        wr[j][c] = x.x;
+                        wr[j][c + 1] = x.y;
+                        wr[j][c + 2] = x.z;
+                        wr[j][c + 3] = x.w;
+                    }
+                }
+                uv[j] = r < b ? p.eta[(int64_t)vs[j] * b + r] : T(0);
+            } else {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) wr[j][c] = T(0);
+                uv[j] = T(0);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < DCHUNK; ++j) {
+            if (j >= m) break;
+            const int32_t v = vs[j], par = ps[j];
+            int ok = 1;                               // wait for w_p (bounded)
+            if (lane == 0) {
+                int n = 0;
+                while (ld_acquire(sy.done + par) == 0) {
+                    if (++n > SPIN_LIMIT) { ok = 0; break; }
+                    __nanosleep(32);
+                }
+            }
+            ok = __shfl_sync(FULL_MASK, ok, 0);
+            __syncwarp();                             // every lane's reads below follow lane 0's acquire
+            if (!ok) {                                // cannot happen for a valid plan: report, move on
+                if (lane == 0) atomicMin(p.info + v / td.n, -2);
+                continue;
+            }
+            const T *wp = p.eta + (int64_t)par * b + 8 * hf;
+            T s2 = T(0);
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                if (FULL || 8 * hf + c < b) s2 = fma(wr[j][c], __ldcg(wp + c), s2);
+            s2 += shfl_xor(s2, 1);
+            if (hf == 0 && r < b) p.eta[(int64_t)v * b + r] = uv[j] - s2;
+            __syncwarp();                             // the warp's stores are ordered before lane 0's release
+            if (lane == 0 && td.child_ptr[v + 1] > td.child_ptr[v]) st_release(sy.done + v, 1);
+            __syncwarp();
+        }
     }
 }
 
@@ -445,7 +499,7 @@ cudaError_t run_tree(const selinv_tree_plan_s *pl, int b, const T *diag, const T
     p.eta = eta;
     const bool draw = z != nullptr;
     p.ws_sinv = reinterpret_cast<T *>(w);
-    w += align256(N * slot_bytes<T>());
+    w += align256(N * sizeof(T) * DRAW_SLOT);
     p.ws_u = reinterpret_cast<T *>(w);
     w += align256(N * slot_bytes<T>());
     p.ws_ld = reinterpret_cast<double *>(w);
@@ -467,21 +521,32 @@ cudaError_t run_tree(const selinv_tree_plan_s *pl, int b, const T *diag, const T
     const size_t smem_d = sizeof(T) * dist_smem_elems<T>() * TWARPS;
     auto kc = draw ? (full ? tree_collect_kernel<T, true, true> : tree_collect_kernel<T, false, true>)
                    : (full ? tree_collect_kernel<T, true> : tree_collect_kernel<T, false>);
-    auto kd = draw ? (full ? tree_distribute_kernel<T, true, true> : tree_distribute_kernel<T, false, true>)
-                   : (full ? tree_distribute_kernel<T, true> : tree_distribute_kernel<T, false>);
+    auto kd = full ? tree_distribute_kernel<T, true> : tree_distribute_kernel<T, false>;
+    auto kw = full ? tree_draw_kernel<T, true> : tree_draw_kernel<T, false>;
     cudaError_t err = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err == cudaSuccess) err = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_d);
+    if (err == cudaSuccess && !draw)
+        err = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_d);
     if (err != cudaSuccess) return err;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t max_blocks = (int64_t)sms * 4;      // about one resident wave of warps
+    // one resident wave of CTAs per kernel (warps take their work from counters)
+    int occ_c = 0, occ_d = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_c, kc, TWARPS * 32, smem) != cudaSuccess || occ_c < 1)
+        occ_c = 4;
+    if (draw || cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_d, kd, TWARPS * 32, smem_d) != cudaSuccess ||
+        occ_d < 1)
+        occ_d = 4;
     const int64_t nleaves = pl->collect_off.size() > 1 ? pl->collect_off[1] - pl->collect_off[0] : 0;
     const int64_t ndist = pl->dist_off.empty() ? 0 : pl->dist_off.back();
-    const int64_t bc = std::min<int64_t>(max_blocks, std::max<int64_t>(1, ceil_div(nleaves, TWARPS)));
+    const int64_t bc = std::min<int64_t>((int64_t)sms * occ_c, std::max<int64_t>(1, ceil_div(nleaves, TWARPS)));
     kc<<<(unsigned)bc, TWARPS * 32, smem, s>>>(p, td, sy, pl->d_collect_nodes, nleaves);
-    if (ndist > 0) {
-        const int64_t bd = std::min<int64_t>(max_blocks, ceil_div(ndist, TWARPS));
+    if (ndist > 0 && draw) {
+        const int64_t wpb = DRAW_THREADS / 32;
+        const int64_t bw = std::min<int64_t>((int64_t)sms * 4, ceil_div(ceil_div(ndist, DCHUNK), wpb));
+        kw<<<(unsigned)bw, DRAW_THREADS, 0, s>>>(p, td, sy, pl->d_dist_nodes, ndist);
+    } else if (ndist > 0) {
+        const int64_t bd = std::min<int64_t>((int64_t)sms * occ_d, ceil_div(ndist, TWARPS));
         kd<<<(unsigned)bd, TWARPS * 32, smem_d, s>>>(p, td, sy, pl->d_dist_nodes, ndist);
     }
     tree_finalize<<<(unsigned)pl->trees, FIN_THREADS, 0, s>>>(p.ws_ld, pl->n, logdet, info);
@@ -495,7 +560,8 @@ bool is_aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p
 size_t tree_workspace(const selinv_tree_plan_s *pl, size_t elem)
 {
     const int64_t N = pl->trees * pl->n;
-    return 2 * align256((size_t)N * elem * w16::SLOT_ELEMS) + align256((size_t)N * sizeof(double)) +
+    return align256((size_t)N * elem * DRAW_SLOT) + align256((size_t)N * elem * w16::SLOT_ELEMS) +
+           align256((size_t)N * sizeof(double)) +
            2 * align256((size_t)N * sizeof(int32_t)) + 256;
 }
 

@@ -373,7 +373,8 @@ SELINV_DEVINL void gemm_nt(Tile<float> &acc, const Tile<float> &X, const Tile<fl
 // (zc[q] = z at the lane's column tcol(t, q); v[h] = (R z) at row g + 8h).
 // The block steps meet R block by block: R_KK = chol(P) of the pivot block as
 // the step finds it (a Schur complement), and below it R_HK = T R_KK, so
-//   v_K += R_KK z_K,  v_H += T (R_KK z_K)   (the second only for K = 0).
+//   v_K += R_KK z_K,  v_H += T (R_KK z_K)   (the second only for K = 0);
+// R_KK z_K comes out of the pivot block's own sweep.
 template <bool DRAW = false>
 SELINV_DEVINL void spd_inverse_blocked(Tile<double> &a, int g, int t, LogAcc &det, bool &bad,
                                        const double *zc = nullptr, double *v = nullptr)
@@ -385,13 +386,8 @@ SELINV_DEVINL void spd_inverse_blocked(Tile<double> &a, int g, int t, LogAcc &de
         const int H = 1 - K;
         double pv[2] = {a.v[K][2 * K], a.v[K][2 * K + 1]};
         double wk = 0.0;                                  // (R_KK z_K) at row 8K + g
-        if (DRAW) {
-            double rc[2] = {pv[0], pv[1]};
-            chol8(rc, lane, g, t);
-            wk = lower8_rowdot(rc, zc[2 * K], zc[2 * K + 1], g, t);
-            v[K] += wk;
-        }
-        inv8_sweep(pv, lane, g, t, det, bad, true);
+        inv8_sweep<DRAW>(pv, lane, g, t, det, bad, true, DRAW ? zc[2 * K] : 0.0, DRAW ? zc[2 * K + 1] : 0.0, &wk);
+        if (DRAW) v[K] += wk;
         double t0 = 0.0, t1 = 0.0;                        // T = A_HK P^-1
         dmma_8x8x4(t0, t1, a.v[H][2 * K], pv[0]);
         dmma_8x8x4(t0, t1, a.v[H][2 * K + 1], pv[1]);
@@ -425,10 +421,16 @@ SELINV_DEVINL void spd_inverse_blocked(Tile<double> &a, int g, int t, LogAcc &de
         for (int q = 0; q < 4; ++q) a.v[h][q] = -a.v[h][q];
 }
 
-template <class T>
-SELINV_DEVINL void spd_inverse_scalar(Tile<T> &a, T *cbuf, int g, int t, LogAcc &det, bool &bad)
+// DRAW: also v[h] = (R z)[g + 8h] for the Cholesky factor A = R R^T, z at the
+// lane's columns tcol(t, q) (zc[q]): the column k published at step k holds,
+// in the rows not yet swept (i >= k), the Schur-complement column that
+// Cholesky scales, R_ik = A_ik / sqrt(d), so v_i += A_ik z_k / sqrt(d).
+template <class T, bool DRAW = false>
+SELINV_DEVINL void spd_inverse_scalar(Tile<T> &a, T *cbuf, int g, int t, LogAcc &det, bool &bad,
+                                      const T *zc = nullptr, T *v = nullptr)
 {
     using V = typename Vec2<T>::type;
+    if (DRAW) v[0] = v[1] = T(0);
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
         const int kh = k >> 3, kt = (k & 7) >> 1, kq = (k & 1) | ((k >> 3) << 1);
@@ -446,6 +448,11 @@ SELINV_DEVINL void spd_inverse_scalar(Tile<T> &a, T *cbuf, int g, int t, LogAcc 
         bad |= !(d > T(0));
         det.mul((double)d);
         const T p = recip(d);
+        if (DRAW) {
+            const T s = shfl(zc[kq], kt) * rsqrt_t(d);
+            if (g >= k) v[0] = fma(c0, s, v[0]);
+            if (g + 8 >= k) v[1] = fma(c1, s, v[1]);
+        }
         const T tc[2] = {c0 * p, c1 * p};
 #pragma unroll
         for (int h = 0; h < 2; ++h)
@@ -484,60 +491,6 @@ template <class T> SELINV_DEVINL void mirror_upper(Tile<T> &a, int g, int t)
         const int src = ((2 * t + j) << 2) | (g >> 1);
         const T u0 = shfl(a.v[1][0], src), u1 = shfl(a.v[1][1], src);
         a.v[0][2 + j] = (g & 1) ? u1 : u0;
-    }
-}
-
-// In-register Cholesky factor of a symmetric positive definite tile,
-// A = R R^T with R lower triangular (entries above the diagonal are left
-// unspecified; lower_matvec ignores them).  Column k, for k = 0..15:
-// R_kk = sqrt(A_kk), R_ik = A_ik / R_kk (i > k), A_ij -= R_ik R_jk (i, j > k);
-// the column travels by shuffles (the lane's rows from lane (g, k_t), its
-// columns j from lane (j, k_t), A being symmetric).
-template <class T> SELINV_DEVINL void chol_lower(Tile<T> &a, int g, int t)
-{
-    const int lane = 4 * g + t;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        const int kh = k >> 3, kt = (k & 7) >> 1, kq = (k & 1) | ((k >> 3) << 1);
-        const T d = shfl(a.v[kh][kq], ((k & 7) << 2) | kt);         // A_kk
-        const T inv = recip(sqrt(d));
-        T li[2], lj[4];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {                               // R_ik at the lane's rows
-            const int r = g + 8 * h;
-            const T c = shfl(a.v[h][kq], (lane & ~3) | kt);
-            li[h] = r >= k ? c * inv : T(0);
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {                               // R_jk at the lane's columns
-            const int j = tcol(t, q);
-            const T c = shfl(a.v[q >> 1][kq], ((2 * t + (q & 1)) << 2) | kt);
-            lj[q] = j > k ? c * inv : T(0);
-        }
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                if (g + 8 * h > k) a.v[h][q] = fma(-li[h], lj[q], a.v[h][q]);
-                if (tcol(t, q) == k) a.v[h][q] = li[h];
-            }
-    }
-}
-
-// y_r = sum_{c <= r} R[r][c] x[c] for a lower-triangular tile and x given at the
-// lane's columns (xc[q] = x[tcol(t, q)]); every lane of a row group ends with
-// the sums for rows g, g + 8.
-template <class T> SELINV_DEVINL void lower_matvec(T out[2], const Tile<T> &a, const T xc[4], int g, int t)
-{
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        T s = T(0);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            if (tcol(t, q) <= g + 8 * h) s = fma(a.v[h][q], xc[q], s);
-        s += shfl_xor(s, 1);
-        s += shfl_xor(s, 2);
-        out[h] = s;
     }
 }
 
