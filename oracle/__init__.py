@@ -50,6 +50,8 @@ def _bind(path):
     lib.oracle_chain_sample.restype = ctypes.c_int
     lib.oracle_tree_sample.argtypes = [P, I64, I64, ctypes.c_int, P, P, P, P, P, P]
     lib.oracle_tree_sample.restype = ctypes.c_int
+    lib.oracle_chain_backward.argtypes = [P, P, I64, I64, ctypes.c_int, P, P, P, P, P]
+    lib.oracle_chain_backward.restype = ctypes.c_int
     lib.oracle_threads.argtypes = []
     lib.oracle_threads.restype = ctypes.c_int
     return lib
@@ -142,6 +144,35 @@ def chain_sample(diag, lower, z, rhs=None, lib=None):
     if rc != 0:
         raise ValueError("oracle_chain_sample: invalid arguments")
     return {"eta": eta, "logdet": logdet, "info": info}
+
+
+def chain_backward(diag, lower, Gb_diag, Gb_lower, lib=None):
+    """Cotangents of the chain's selected inverse: given the cotangents Gb_diag
+    [..., L, b, b] on G_diag and Gb_lower [..., L-1, b, b] on G_lower, returns
+    dict with Db [..., L, b, b] (lower-triangular: the forward reads only D's
+    lower triangle), Bb [..., L-1, b, b] and info [...].  Dense definition,
+    Ab = -A^-1 Gbar A^-1 (gabp-sparse-inv, "Differentiable selected inverse")."""
+    diag = _f64(diag)
+    lead = diag.shape[:-3]
+    L, b = diag.shape[-3], diag.shape[-1]
+    batch = int(np.prod(lead)) if lead else 1
+    Gb_diag = _f64(Gb_diag)
+    assert Gb_diag.shape == diag.shape
+    Db = np.empty(lead + (L, b, b))
+    info = np.empty(lead, dtype=np.int32)
+    Bb = lower_ = None
+    if L == 1:
+        Gb_lower = None
+    else:
+        lower_ = _f64(lower)
+        Gb_lower = _f64(Gb_lower)
+        assert lower_.shape == lead + (L - 1, b, b) and Gb_lower.shape == lower_.shape
+        Bb = np.empty(lead + (L - 1, b, b))
+    rc = _load(lib).oracle_chain_backward(_ptr(diag), _ptr(lower_), batch, L, b, _ptr(Gb_diag),
+                                          _ptr(Gb_lower), _ptr(Db), _ptr(Bb), _ptr(info))
+    if rc != 0:
+        raise ValueError("oracle_chain_backward: invalid arguments")
+    return {"Db": Db, "Bb": Bb if Bb is not None else np.empty(lead + (0, b, b)), "info": info}
 
 
 def tree(parent, diag, edge, lib=None):

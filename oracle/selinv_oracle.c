@@ -331,6 +331,97 @@ int oracle_chain_sample(const double *diag, const double *lower, int64_t batch, 
     return 0;
 }
 
+/* ------------------------------- backward -------------------------------- */
+
+/*
+ * Cotangents of the chain's selected inverse (gabp-sparse-inv, "Differentiable
+ * selected inverse": gradients of a loss over the selected blocks flow back to
+ * the input blocks as on-pattern cotangents).  Written from the definition:
+ * G = A^-1 gives dG = -G dA G, so for a loss with cotangents Gb_ii on G_ii and
+ * Gb_{i+1,i} on G_{i+1,i} (and nothing on the blocks above the diagonal, which
+ * are not outputs),
+ *     Ab = -G^T Gbar G^T = -G Gbar G         (dense, N = L b),
+ * and the inputs receive what the forward map reads:
+ *     D_i: only its lower triangle, the upper one being its mirror, so
+ *          Db_i[r][c] = Ab_ii[r][c] + Ab_ii[c][r] (r > c), Ab_ii[r][r] (r = c),
+ *          0 (r < c);
+ *     B_i: at block (i+1, i) and, transposed, at (i, i+1), so
+ *          Bb_i = Ab_{i+1,i} + (Ab_{i,i+1})^T.
+ * The dense inverse comes from the textbook Cholesky factor of A.  Returns
+ * info (-1 ok, else the block holding the first failing pivot).
+ */
+static int chain_backward_one(int64_t L, int b, const double *diag, const double *lower,
+                              const double *Gb_diag, const double *Gb_lower, double *Db, double *Bb)
+{
+    const size_t bb = (size_t)b * b;
+    const int N = (int)(L * b);
+    const size_t NN = (size_t)N * N;
+    double *A = calloc(NN, sizeof(double)), *R = malloc(NN * sizeof(double));
+    double *Ri = malloc(NN * sizeof(double)), *G = malloc(NN * sizeof(double));
+    double *Gbar = calloc(NN, sizeof(double)), *T = malloc(NN * sizeof(double));
+    double *Ab = malloc(NN * sizeof(double));
+    int info = -1;
+    for (int64_t i = 0; i < L; ++i)
+        for (int r = 0; r < b; ++r)
+            for (int c = 0; c < b; ++c) {
+                const size_t row = (size_t)(i * b + r), col = (size_t)(i * b + c);
+                A[row * N + col] = (c <= r) ? diag[bb * i + r * b + c] : diag[bb * i + c * b + r];
+                Gbar[row * N + col] = Gb_diag[bb * i + r * b + c];
+                if (i + 1 < L) {
+                    const size_t lrow = (size_t)((i + 1) * b + r);
+                    A[lrow * N + col] = lower[bb * i + r * b + c];              /* A_{i+1,i} = B_i */
+                    A[col * N + lrow] = lower[bb * i + r * b + c];              /* A_{i,i+1} = B_i^T */
+                    Gbar[lrow * N + col] = Gb_lower[bb * i + r * b + c];
+                }
+            }
+    if (cholesky_lower(N, A, R) != 0) {
+        for (int j = 0; j < N; ++j) {                /* the failing pivot's block */
+            double d = A[(size_t)j * N + j];
+            for (int k = 0; k < j; ++k) d -= R[(size_t)j * N + k] * R[(size_t)j * N + k];
+            if (!(d > 0.0)) { info = j / b; break; }
+        }
+        goto done;
+    }
+    lower_inverse(N, R, Ri);
+    matmul(N, Ri, 1, Ri, 0, G);                      /* A^-1 = R^-T R^-1 */
+    matmul(N, G, 0, Gbar, 0, T);                     /* G Gbar */
+    matmul(N, T, 0, G, 0, Ab);                       /* G Gbar G */
+    for (size_t k = 0; k < NN; ++k) Ab[k] = -Ab[k];
+    for (int64_t i = 0; i < L; ++i)
+        for (int r = 0; r < b; ++r)
+            for (int c = 0; c < b; ++c) {
+                const size_t row = (size_t)(i * b + r), col = (size_t)(i * b + c);
+                double v = 0.0;
+                if (c < r) v = Ab[row * N + col] + Ab[col * N + row];
+                else if (c == r) v = Ab[row * N + col];
+                Db[bb * i + r * b + c] = v;
+                if (i + 1 < L) {
+                    const size_t lrow = (size_t)((i + 1) * b + r);
+                    Bb[bb * i + r * b + c] = Ab[lrow * N + col] + Ab[col * N + lrow];
+                }
+            }
+done:
+    free(A); free(R); free(Ri); free(G); free(Gbar); free(T); free(Ab);
+    return info;
+}
+
+/* Batched backward: Gb_diag [batch,L,b,b], Gb_lower [batch,L-1,b,b] (NULL when
+ * L = 1) -> Db [batch,L,b,b], Bb [batch,L-1,b,b]; info [batch]. */
+int oracle_chain_backward(const double *diag, const double *lower, int64_t batch, int64_t L, int b,
+                          const double *Gb_diag, const double *Gb_lower, double *Db, double *Bb,
+                          int32_t *info)
+{
+    if (batch < 0 || L < 1 || b < 1 || !diag || !Gb_diag || !Db || !info) return 1;
+    if (L > 1 && (!lower || !Gb_lower || !Bb)) return 1;
+    const size_t bb = (size_t)b * b;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t e = 0; e < batch; ++e)
+        info[e] = chain_backward_one(L, b, diag + bb * L * e, L > 1 ? lower + bb * (L - 1) * e : NULL,
+                                     Gb_diag + bb * L * e, L > 1 ? Gb_lower + bb * (L - 1) * e : NULL,
+                                     Db + bb * L * e, L > 1 ? Bb + bb * (L - 1) * e : NULL);
+    return 0;
+}
+
 /* -------------------------------- tree ---------------------------------- */
 
 /* One rooted tree (parent[root] = -1).  Collect in reverse breadth-first

@@ -30,7 +30,7 @@ import numpy as np
 import oracle
 from sparse_spd_selected_b200 import inputs
 from tests.dense import (balanced_parent, blk, chain_dense, path_parent, rel,
-                         star_parent, tree_dense)
+                         star_parent, sym_lower, tree_dense)
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
@@ -411,6 +411,81 @@ def pin_tree_sample_standard_basis(lib=None):
     return worst
 
 
+def _proj_lower(M):
+    """What the forward's lower-triangle read makes of a cotangent on a full
+    diagonal block: M + M^T below the diagonal, M on it, zero above."""
+    return np.tril(M + M.T, -1) + np.diag(np.diag(M))
+
+
+def pin_backward_finite_differences(lib=None):
+    """Cotangents against central differences of the (pinned) forward oracle,
+    entry by entry, upper entries of D included (they must get zero)."""
+    worst = 0.0
+    for L, b, seed in [(3, 2, 31), (2, 3, 32), (1, 2, 33)]:
+        d, l, _ = inputs.chain_inputs(1, L, b, seed=seed, load=1.0, with_rhs=False)
+        rng = np.random.default_rng(seed)
+        gd, gl = rng.standard_normal(d.shape), rng.standard_normal(l.shape)
+        out = oracle.chain_backward(d, l, gd, gl, lib=lib)
+        if (out["info"] != -1).any():
+            return float("inf")
+
+        def loss(dd, ll):
+            o = oracle.chain(dd, ll, lib=lib)
+            return float((o["G_diag"] * gd).sum() + (o["G_lower"] * gl).sum())
+
+        h = 1e-5
+        scale = max(1.0, float(np.abs(out["Db"]).max()), float(np.abs(out["Bb"]).max()) if L > 1 else 0.0)
+        for idx in np.ndindex(*d.shape):
+            dp, dm = d.copy(), d.copy()
+            dp[idx] += h
+            dm[idx] -= h
+            worst = max(worst, abs((loss(dp, l) - loss(dm, l)) / (2 * h) - out["Db"][idx]) / scale)
+        for idx in np.ndindex(*l.shape):
+            lp, lm = l.copy(), l.copy()
+            lp[idx] += h
+            lm[idx] -= h
+            worst = max(worst, abs((loss(d, lp) - loss(d, lm)) / (2 * h) - out["Bb"][idx]) / scale)
+    return worst
+
+
+def pin_backward_decoupled(lib=None):
+    """B = 0: A^-1 is block diagonal (blocks D_i^-1), so -A^-1 Gbar A^-1 has
+    diagonal blocks -D_i^-1 Gb_ii D_i^-1 and blocks -D_{i+1}^-1 Gb_{i+1,i} D_i^-1
+    below them (none above: Gbar has nothing there), hence Db_i =
+    proj(-D_i^-1 Gb_ii D_i^-1) and Bb_i = -D_{i+1}^-1 Gb_{i+1,i} D_i^-1."""
+    L, b = 5, 4
+    d, _, _ = inputs.chain_inputs(2, L, b, seed=34, load=0.5, with_rhs=False)
+    lower = np.zeros((2, L - 1, b, b))
+    rng = np.random.default_rng(34)
+    gd, gl = rng.standard_normal(d.shape), rng.standard_normal(lower.shape)
+    out = oracle.chain_backward(d, lower, gd, gl, lib=lib)
+    worst = 0.0
+    for e in range(2):
+        inv = [np.linalg.inv(sym_lower(d[e, i])) for i in range(L)]
+        for i in range(L):
+            worst = max(worst, rel(out["Db"][e, i], _proj_lower(-inv[i] @ gd[e, i] @ inv[i])))
+        for i in range(L - 1):
+            worst = max(worst, rel(out["Bb"][e, i], -inv[i + 1] @ gl[e, i] @ inv[i]))
+    return worst
+
+
+def pin_backward_trace(lib=None):
+    """Loss = tr A^-1 (Gb_ii = I, Gb_lower = 0): dL/dA = -A^-2, so Db_i =
+    proj(-(A^-2)_ii) and Bb_i = -2 (A^-2)_{i+1,i}."""
+    L, b = 6, 3
+    d, l, _ = inputs.chain_inputs(2, L, b, seed=35, load=1.0, with_rhs=False)
+    gd = np.broadcast_to(np.eye(b), d.shape).copy()
+    out = oracle.chain_backward(d, l, gd, np.zeros(l.shape), lib=lib)
+    worst = 0.0
+    for e in range(2):
+        A2 = np.linalg.matrix_power(np.linalg.inv(chain_dense(d[e], l[e])), 2)
+        for i in range(L):
+            worst = max(worst, rel(out["Db"][e, i], _proj_lower(-blk(A2, i, i, b))))
+        for i in range(L - 1):
+            worst = max(worst, rel(out["Bb"][e, i], -2.0 * blk(A2, i + 1, i, b)))
+    return worst
+
+
 # name -> (function, tolerance)
 PINS = {
     "tiny_chains_dense": (pin_tiny_chains_dense, 1e-12),
@@ -427,4 +502,7 @@ PINS = {
     "sample_mean": (pin_sample_mean, 1e-12),
     "tree_sample_standard_basis": (pin_tree_sample_standard_basis, 1e-12),
     "not_spd": (pin_not_spd, 0.5),
+    "backward_finite_differences": (pin_backward_finite_differences, 1e-7),
+    "backward_decoupled": (pin_backward_decoupled, 1e-12),
+    "backward_trace": (pin_backward_trace, 1e-11),
 }

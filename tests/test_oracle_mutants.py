@@ -54,6 +54,16 @@ MUTANTS = {
                                     "matvec(b, edge + bb * u, 0, w + (size_t)b * pu, t1);"),
     "tree_sample_sign": ("for (int k = 0; k < b; ++k) t1[k] = z[(size_t)b * u + k] - t2[k];",
                          "for (int k = 0; k < b; ++k) t1[k] = z[(size_t)b * u + k] + t2[k];"),
+    "backward_sign": ("for (size_t k = 0; k < NN; ++k) Ab[k] = -Ab[k];",
+                      "for (size_t k = 0; k < NN; ++k) Ab[k] = Ab[k];"),
+    "backward_bbar_untransposed": ("Bb[bb * i + r * b + c] = Ab[lrow * N + col] + Ab[col * N + lrow];",
+                                   "Bb[bb * i + r * b + c] = Ab[lrow * N + col] + Ab[lrow * N + col];"),
+    "backward_dbar_mirror_dropped": ("if (c < r) v = Ab[row * N + col] + Ab[col * N + row];",
+                                     "if (c < r) v = Ab[row * N + col];"),
+    "backward_gbar_lower_above_untransposed": ("Gbar[lrow * N + col] = Gb_lower[bb * i + r * b + c];",
+                                               "Gbar[row * N + col + b] = Gb_lower[bb * i + r * b + c];"),
+    "backward_gbar_diag_dropped": ("Gbar[row * N + col] = Gb_diag[bb * i + r * b + c];",
+                                   "Gbar[row * N + col] = 0.0 * Gb_diag[bb * i + r * b + c];"),
     "tree_g_diag_transposed": ("matmul(b, Sinv + bb * v, 0, edge + bb * v, 1, T1);",
                                "matmul(b, Sinv + bb * v, 0, edge + bb * v, 0, T1);"),
 }
