@@ -46,6 +46,7 @@ KERNEL_SOURCES = {
     "seg_distribute_kernel": ["chain_seg.cu", "quad32.cuh", "warp16.cuh", "common.cuh"],
     "chain_large_kernel": ["chain_large.cu", "common.cuh"],
     "tree_collect_kernel": ["tree.cu", "warp16.cuh", "common.cuh"],
+    "chain_backward_kernel": ["chain_backward.cu", "warp16.cuh", "common.cuh"],
 }
 
 
@@ -60,9 +61,10 @@ def parse():
     ap.add_argument("--length", type=int, default=None,
                     help="override the chain length / tree size (profiling runs of a smaller case)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--op", default="selinv", choices=["selinv", "sample"],
+    ap.add_argument("--op", default="selinv", choices=["selinv", "sample", "backward"],
                     help="selinv: selected inverse + log det (+ solve); sample: Gaussian draw "
-                         "eta = A^-1 r + L^-T z + log det (chains; on trees eta = L^-T z)")
+                         "eta = A^-1 r + L^-T z + log det (chains; on trees eta = L^-T z); backward: "
+                         "cotangents of diag and lower from those of G_diag and G_lower (chains, b <= 16)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -157,6 +159,8 @@ def oracle_inputs(w, elems, op):
     g = inputs.generate(w, elements=elems)
     if op == "sample":
         g["z"] = inputs.standard_normals(w.batch, w.L, w.b, w.seed, elems)
+    if op == "backward":
+        g["Gb_diag"], g["Gb_lower"] = inputs.cotangents(w.batch, w.L, w.b, w.seed, elems)
     return g
 
 
@@ -167,6 +171,8 @@ def oracle_run(oracle, w, g, op):
         oracle.tree(g["parent"], g["diag"], g["edge"])
     elif op == "sample":
         oracle.chain_sample(g["diag"], g["lower"], g["z"], rhs=g.get("rhs"))
+    elif op == "backward":
+        oracle.chain_backward(g["diag"], g["lower"], g["Gb_diag"], g["Gb_lower"])
     else:
         oracle.chain(g["diag"], g["lower"], g.get("rhs"))
 
@@ -203,6 +209,10 @@ def algorithmic_bytes(w, es, batch, op="selinv"):
     (or G_edge) blocks, plus the right-hand side and solution when solving.  A draw reads
     D, B, r and z and writes eta (a tree draw has no r)."""
     b2 = w.b * w.b
+    if op == "backward":
+        # read D, G_diag, Gb_diag and B, G_lower, Gb_lower; write Db and Bb
+        nodes, edges = batch * w.L, batch * (w.L - 1)
+        return es * 4 * b2 * (nodes + edges)
     if op == "sample" and w.kind == "tree":
         n = batch * w.L
         return es * (b2 * n + b2 * (n - batch) + 2 * w.b * n)
@@ -310,7 +320,7 @@ def run_reference(args):
 
 
 def metric_name(op, dtype):
-    what = "draw" if op == "sample" else "selinv"
+    what = {"sample": "draw", "backward": "selinv backward"}.get(op, "selinv")
     return f"{what} blocks/s ({'fp64' if dtype == 'f64' else 'fp32'})"
 
 
@@ -357,6 +367,11 @@ def run_ours(args):
             if w.b > 16 and args.dtype != "f64":
                 raise SystemExit("--op sample with b > 16 runs in float64 only")
             g["z"] = inputs.standard_normals(w.batch, w.L, w.b, w.seed, elems)
+        if args.op == "backward":
+            if w.kind != "chain" or w.b > 16:
+                raise SystemExit("--op backward runs on chain workloads with b <= 16")
+            g.pop("rhs", None)
+            g["Gb_diag"], g["Gb_lower"] = inputs.cotangents(w.batch, w.L, w.b, w.seed, elems)
         host_in = {k: torch.from_numpy(v).to(tdt).pin_memory() for k, v in g.items()
                    if v is not None and k != "parent"}
         dev_in = {k: v.to("cuda", non_blocking=True) for k, v in host_in.items()}
@@ -400,7 +415,18 @@ def run_ours(args):
                          dtype=torch.uint8, device="cuda")
         launches_per_step = 1
         segments = selinv.chain_segments(batch, L, b, True, "rhs" in dev_in)
-        if args.op == "sample":
+        if args.op == "backward":
+            # the forward's outputs are the backward's inputs (computed once, outside the timing)
+            fwd = selinv.selinv_chain(dev_in["diag"], dev_in["lower"])
+            for k in ("G_diag", "G_lower"):
+                dev_in[k] = fwd[k]
+                host_in[k] = fwd[k].cpu().pin_memory()
+            kernel = "chain_backward_kernel"
+            out = {"Db": torch.empty_like(dev_in["diag"]), "Bb": torch.empty_like(dev_in["lower"]),
+                   "info": torch.empty(batch, dtype=torch.int32, device="cuda")}
+            ws = torch.empty(max(selinv.chain_backward_workspace_size(tdt, batch, L, b), 1), dtype=torch.uint8,
+                             device="cuda")
+        elif args.op == "sample":
             kernel = "chain_small_kernel (draw mode)" if b <= 16 else "chain_large_kernel (draw mode)"
             out = {"eta": torch.empty((batch, L, b), dtype=tdt, device="cuda"),
                    "logdet": torch.empty(batch, dtype=torch.float64, device="cuda"),
@@ -418,7 +444,11 @@ def run_ours(args):
         else:
             kernel = "chain_large_kernel"
 
-        if args.op == "sample":
+        if args.op == "backward":
+            def step():
+                selinv.chain_backward(dev_in["diag"], dev_in["lower"], dev_in["G_diag"], dev_in["G_lower"],
+                                      dev_in["Gb_diag"], dev_in["Gb_lower"], check=False, out=out, workspace=ws)
+        elif args.op == "sample":
             def step():
                 selinv.chain_sample(dev_in["diag"], dev_in["lower"], dev_in["z"], dev_in.get("rhs"), check=False,
                                     out=out, workspace=ws)

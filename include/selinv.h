@@ -179,6 +179,40 @@ selinv_status selinv_chain_sample(selinv_dtype dtype, int64_t batch, int64_t L, 
                                   void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Cotangents of the chain selected inverse (b <= 16): given the cotangents
+ * Gb_diag [batch, L, b, b] and Gb_lower [batch, L-1, b, b] of a loss with
+ * respect to selinv_chain's outputs G_diag and G_lower, writes the
+ * cotangents with respect to its inputs:
+ *   Db [batch, L, b, b]    of diag; lower-triangular, because selinv_chain
+ *                          reads only the lower triangle of each D_i (an entry
+ *                          below the diagonal stands for both mirror places,
+ *                          so it receives Ab[r][c] + Ab[c][r]; upper entries
+ *                          receive 0);
+ *   Bb [batch, L-1, b, b]  of lower (B_i sits at (i+1, i) and, transposed, at
+ *                          (i, i+1)),
+ * where Ab = -A^-1 Gbar A^-1 is the cotangent of A as a whole matrix (dG =
+ * -G dA G).  (gabp-sparse-inv 0.3.2, "Differentiable selected inverse":
+ * gradients over the selected blocks flow back to the input blocks through
+ * an analytic two-pass backward.)  The two passes are the reverse-mode forms
+ * of the forward's collect and distribute sweeps; nothing dense is formed.
+ *   diag, lower, G_diag, G_lower  the forward's inputs and outputs (device);
+ *                                 lower, G_lower, Gb_lower and Bb may be NULL
+ *                                 when L = 1
+ *   Gb_diag, Gb_lower   NULL stands for a zero cotangent
+ *   info [batch]    -1, or the first block whose Schur complement is not
+ *                   positive definite (the outputs are then unspecified)
+ * Workspace: selinv_chain_backward_workspace_size(dtype, batch, L, b) bytes
+ * (two 16 x 16 tiles per block).  b > 16 returns SELINV_ERR_UNSUPPORTED.
+ */
+size_t selinv_chain_backward_workspace_size(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b);
+
+selinv_status selinv_chain_backward(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b,
+                                    const void *diag, const void *lower, const void *G_diag,
+                                    const void *G_lower, const void *Gb_diag, const void *Gb_lower,
+                                    void *Db, void *Bb, int32_t *info, void *workspace,
+                                    size_t workspace_bytes, void *stream);
+
+/*
  * Same computation as selinv_chain for b <= 16, with no workspace argument
  * and no allocation of any kind.  The pages have no counterpart: this entry
  * point exists for callers that cannot allocate device memory -- code running

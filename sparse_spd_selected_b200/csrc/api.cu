@@ -2,6 +2,8 @@
 // dispatch.  Declarations and the full contract are in include/selinv.h.
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -187,6 +189,58 @@ selinv_status selinv_chain_sample(selinv_dtype dtype, int64_t batch, int64_t L, 
     a.L = L;
     a.b = b;
     return from_cuda(chain_small_sample_launch<float>(a, al, s));
+}
+
+size_t selinv_chain_backward_workspace_size(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b)
+{
+    if (!valid_dtype(dtype) || batch < 0 || L < 1 || b < 1 || b > 16) return 0;
+    return round_up(chain_backward_workspace(elem_size(dtype), batch, L));
+}
+
+selinv_status selinv_chain_backward(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b, const void *diag,
+                                    const void *lower, const void *G_diag, const void *G_lower, const void *Gb_diag,
+                                    const void *Gb_lower, void *Db, void *Bb, int32_t *info, void *workspace,
+                                    size_t workspace_bytes, void *stream)
+{
+    selinv_status st = chain_check(dtype, batch, L, b, diag, lower, info);
+    if (st != SELINV_OK) return st;
+    if (b > 16) return SELINV_ERR_UNSUPPORTED;
+    const size_t es = elem_size(dtype);
+    if (batch > 0 && (!G_diag || !Db || (L > 1 && (!G_lower || !Bb))))
+        return SELINV_ERR_INVALID_ARG;
+    if (!aligned(G_diag, es) || !aligned(G_lower, es) || !aligned(Gb_diag, es) || !aligned(Gb_lower, es) ||
+        !aligned(Db, es) || !aligned(Bb, es) || !aligned(workspace, 16))
+        return SELINV_ERR_INVALID_ARG;
+    const size_t need = selinv_chain_backward_workspace_size(dtype, batch, L, b);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return SELINV_ERR_WORKSPACE;
+    if (batch == 0) return SELINV_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool al = aligned(diag, 16) && aligned(lower, 16) && aligned(G_diag, 16) && aligned(G_lower, 16) &&
+                    aligned(Gb_diag, 16) && aligned(Gb_lower, 16) && aligned(Db, 16) && aligned(Bb, 16);
+    auto fill = [&](auto &a, auto *tag) {
+        using T = std::remove_pointer_t<decltype(tag)>;
+        a.diag = static_cast<const T *>(diag);
+        a.lower = static_cast<const T *>(lower);
+        a.G_diag = static_cast<const T *>(G_diag);
+        a.G_lower = static_cast<const T *>(G_lower);
+        a.Gb_diag = static_cast<const T *>(Gb_diag);
+        a.Gb_lower = static_cast<const T *>(Gb_lower);
+        a.Db = static_cast<T *>(Db);
+        a.Bb = static_cast<T *>(Bb);
+        a.info = info;
+        a.ws = static_cast<T *>(workspace);
+        a.batch = batch;
+        a.L = L;
+        a.b = b;
+    };
+    if (dtype == SELINV_F64) {
+        ChainBwdArgs<double> a;
+        fill(a, (double *)nullptr);
+        return from_cuda(chain_backward_launch<double>(a, al, s));
+    }
+    ChainBwdArgs<float> a;
+    fill(a, (float *)nullptr);
+    return from_cuda(chain_backward_launch<float>(a, al, s));
 }
 
 selinv_status chain_solve_multi(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b, int32_t nrhs,

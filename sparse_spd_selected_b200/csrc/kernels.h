@@ -52,4 +52,19 @@ template <class T> cudaError_t chain_large_launch(const ChainArgs<T> &a, cudaStr
 // The same kernel drawing eta = A^-1 rhs + L^-T z into a.x (float64; rhs may be null; no G).
 cudaError_t chain_large_sample_launch(const ChainArgs<double> &a, cudaStream_t s);
 
+// Cotangents of the chain selected inverse (b <= 16: one warp per chain).
+template <class T> struct ChainBwdArgs {
+    const T *diag, *lower;          // forward inputs
+    const T *G_diag, *G_lower;      // forward outputs
+    const T *Gb_diag, *Gb_lower;    // their cotangents
+    T *Db, *Bb;                     // cotangents of diag (lower-triangular) and lower
+    int32_t *info;                  // [batch]
+    T *ws;
+    int64_t batch;
+    int64_t L;
+    int b;
+};
+size_t chain_backward_workspace(size_t elem, int64_t batch, int64_t L);
+template <class T> cudaError_t chain_backward_launch(const ChainBwdArgs<T> &a, bool aligned16, cudaStream_t s);
+
 }  // namespace selinv

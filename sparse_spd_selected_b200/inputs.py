@@ -231,6 +231,19 @@ def standard_normals(batch: int, L: int, b: int, seed: int, elements: Optional[S
     return np.stack([np.random.default_rng([int(seed), int(e), 1]).standard_normal((L, b)) for e in elements])
 
 
+def cotangents(batch: int, L: int, b: int, seed: int, elements: Optional[Sequence[int]] = None):
+    """Standard-normal cotangents (Gb_diag [n, L, b, b], Gb_lower [n, L-1, b, b])
+    of a loss on a chain's selected inverse: element e draws from
+    default_rng([seed, e, 2]), a stream apart from its matrix and draws."""
+    elements = range(batch) if elements is None else elements
+    gd, gl = [], []
+    for e in elements:
+        rng = np.random.default_rng([int(seed), int(e), 2])
+        gd.append(rng.standard_normal((L, b, b)))
+        gl.append(rng.standard_normal((L - 1, b, b)))
+    return np.stack(gd), np.stack(gl)
+
+
 def generate(w: Workload, elements: Optional[Sequence[int]] = None):
     """Host (NumPy) inputs of a workload, or of a subset of its batch elements."""
     if w.kind == "chain":

@@ -65,6 +65,10 @@ def lib():
         L.selinv_chain_sample.restype = ctypes.c_int
         L.chain_solve.argtypes = [ctypes.c_int, I64, I64, I32, P, P, P, P, P, P, P, SZ, P]
         L.chain_solve.restype = ctypes.c_int
+        L.selinv_chain_backward_workspace_size.argtypes = [ctypes.c_int, I64, I64, I32]
+        L.selinv_chain_backward_workspace_size.restype = SZ
+        L.selinv_chain_backward.argtypes = [ctypes.c_int, I64, I64, I32, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.selinv_chain_backward.restype = ctypes.c_int
         L.selinv_tree_plan.argtypes = [P, I64, I64, ctypes.POINTER(P)]
         L.selinv_tree_plan.restype = ctypes.c_int
         L.selinv_tree_plan_free.argtypes = [P]
@@ -312,6 +316,93 @@ def chain_sample(diag, lower, z, rhs=None, *, check=True, out=None, workspace=No
     _check(st, "selinv_chain_sample")
     _raise_on_info(info, check)
     return {"eta": eta, "logdet": logdet, "info": info}
+
+
+def chain_backward_workspace_size(dtype, batch, L, b) -> int:
+    return int(lib().selinv_chain_backward_workspace_size(_code(dtype), batch, L, b))
+
+
+def chain_backward(diag, lower, G_diag, G_lower, Gb_diag=None, Gb_lower=None, *, check=True, out=None,
+                   workspace=None, stream=None):
+    """Cotangents of selinv_chain (b <= 16): from the cotangents Gb_diag, Gb_lower
+    of its outputs G_diag, G_lower (None = zero), the cotangents Db of diag
+    (lower-triangular: only D's lower triangle is read) and Bb of lower.
+    Returns a dict with Db, Bb and info (int32, -1 = ok)."""
+    _cuda_contig("diag", diag)
+    dt = diag.dtype
+    if diag.dim() < 3 or diag.shape[-1] != diag.shape[-2]:
+        raise ValueError("diag must be [..., L, b, b]")
+    lead = tuple(diag.shape[:-3])
+    L, b = int(diag.shape[-3]), int(diag.shape[-1])
+    batch = 1
+    for d in lead:
+        batch *= int(d)
+    _cuda_contig("G_diag", G_diag, dt)
+    if Gb_diag is not None:
+        _cuda_contig("Gb_diag", Gb_diag, dt)
+    for name, t in (("G_diag", G_diag), ("Gb_diag", Gb_diag)):
+        if t is not None and tuple(t.shape) != tuple(diag.shape):
+            raise ValueError(f"{name} must have diag's shape")
+    shape_l = lead + (L - 1, b, b)
+    if L > 1:
+        for name, t in (("lower", lower), ("G_lower", G_lower)):
+            if t is None:
+                raise ValueError(f"{name} is required when L > 1")
+            _cuda_contig(name, t, dt)
+            if tuple(t.shape) != shape_l:
+                raise ValueError(f"{name} must be {shape_l}")
+        if Gb_lower is not None:
+            _cuda_contig("Gb_lower", Gb_lower, dt)
+            if tuple(Gb_lower.shape) != shape_l:
+                raise ValueError(f"Gb_lower must be {shape_l}")
+    else:
+        lower = G_lower = Gb_lower = None
+    dev = diag.device
+    out = dict(out or {})
+    Db = out.get("Db")
+    if Db is None:
+        Db = torch.empty_like(diag)
+    Bb = out.get("Bb")
+    if Bb is None:
+        Bb = torch.empty(shape_l, dtype=dt, device=dev)
+    info = out.get("info")
+    if info is None:
+        info = torch.empty(lead, dtype=torch.int32, device=dev)
+    nbytes = chain_backward_workspace_size(dt, batch, L, b)
+    ws = _workspace(nbytes, dev, workspace)
+    with torch.cuda.device(dev):
+        st = lib().selinv_chain_backward(_code(dt), batch, L, b, _ptr(diag), _ptr(lower), _ptr(G_diag),
+                                         _ptr(G_lower), _ptr(Gb_diag), _ptr(Gb_lower), _ptr(Db),
+                                         _ptr(Bb if L > 1 else None), _ptr(info), _ptr(ws), nbytes,
+                                         _stream_handle(stream))
+    _check(st, "selinv_chain_backward")
+    _raise_on_info(info, check)
+    return {"Db": Db, "Bb": Bb, "info": info}
+
+
+class _SelinvChainFn(torch.autograd.Function):
+    """G_diag, G_lower = selinv_chain(diag, lower) with its analytic backward."""
+
+    @staticmethod
+    def forward(ctx, diag, lower):
+        out = selinv_chain(diag, lower)
+        ctx.save_for_backward(diag, lower, out["G_diag"], out["G_lower"])
+        return out["G_diag"], out["G_lower"]
+
+    @staticmethod
+    def backward(ctx, gb_diag, gb_lower):
+        diag, lower, G_diag, G_lower = ctx.saved_tensors
+        r = chain_backward(diag, lower, G_diag, G_lower,
+                           None if gb_diag is None else gb_diag.contiguous(),
+                           None if gb_lower is None else gb_lower.contiguous())
+        return r["Db"], r["Bb"]
+
+
+def selinv_chain_ad(diag, lower):
+    """Differentiable selected inverse of chains (b <= 16): returns (G_diag,
+    G_lower); gradients reach diag (its lower triangle: the forward reads no
+    other entry) and lower through chain_backward."""
+    return _SelinvChainFn.apply(diag, lower)
 
 
 class TreePlan:

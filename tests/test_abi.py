@@ -120,3 +120,30 @@ def test_sample_and_multi_argument_errors(lib):
     assert m(0, 1, 4, 20, 3, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 1 << 30, None) == selinv.ERR_UNSUPPORTED
     assert m(0, 1, 4, 4, 3, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 16, None) == selinv.ERR_WORKSPACE
     assert m(0, 0, 4, 4, 3, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 1 << 30, None) == selinv.OK
+
+
+def test_backward_argument_errors(lib):
+    """The backward rejects bad arguments before any launch."""
+    f = lib.selinv_chain_backward
+    ws = lib.selinv_chain_backward_workspace_size
+    ws.restype = ctypes.c_size_t
+    ws.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32]
+    assert ws(0, 3, 5, 16) >= 3 * 5 * 2 * 256 * 8 and ws(0, 3, 5, 16) % 256 == 0
+    assert ws(0, 3, 5, 17) == 0
+
+    # dtype, batch, L, b, diag, lower, G_diag, G_lower, Gb_diag, Gb_lower, Db, Bb, info, ws, ws_bytes, stream
+    def call(**kw):
+        args = dict(dtype=0, batch=1, L=4, b=4, diag=FAKE, lower=FAKE, Gd=FAKE, Gl=FAKE, Gbd=FAKE, Gbl=FAKE,
+                    Db=FAKE, Bb=FAKE, info=FAKE, ws=FAKE, nbytes=1 << 30)
+        args.update(kw)
+        return f(args["dtype"], args["batch"], args["L"], args["b"], args["diag"], args["lower"], args["Gd"],
+                 args["Gl"], args["Gbd"], args["Gbl"], args["Db"], args["Bb"], args["info"], args["ws"],
+                 args["nbytes"], None)
+    assert call(b=17) == selinv.ERR_UNSUPPORTED
+    assert call(Gd=None) == selinv.ERR_INVALID_ARG
+    assert call(Db=None) == selinv.ERR_INVALID_ARG
+    assert call(Bb=None) == selinv.ERR_INVALID_ARG
+    assert call(Gl=None) == selinv.ERR_INVALID_ARG
+    assert call(nbytes=16) == selinv.ERR_WORKSPACE
+    assert call(ws=None) == selinv.ERR_WORKSPACE
+    assert call(batch=0) == selinv.OK
