@@ -52,6 +52,8 @@ def _bind(path):
     lib.oracle_tree_sample.restype = ctypes.c_int
     lib.oracle_chain_backward.argtypes = [P, P, I64, I64, ctypes.c_int, P, P, P, P, P]
     lib.oracle_chain_backward.restype = ctypes.c_int
+    lib.oracle_tree_backward.argtypes = [P, I64, I64, ctypes.c_int, P, P, P, P, P, P, P]
+    lib.oracle_tree_backward.restype = ctypes.c_int
     lib.oracle_threads.argtypes = []
     lib.oracle_threads.restype = ctypes.c_int
     return lib
@@ -173,6 +175,31 @@ def chain_backward(diag, lower, Gb_diag, Gb_lower, lib=None):
     if rc != 0:
         raise ValueError("oracle_chain_backward: invalid arguments")
     return {"Db": Db, "Bb": Bb if Bb is not None else np.empty(lead + (0, b, b)), "info": info}
+
+
+def tree_backward(parent, diag, edge, Gb_diag, Gb_edge, lib=None):
+    """Cotangents of the tree selected inverse: from Gb_diag, Gb_edge [..., n, b, b]
+    (cotangents of G_diag, G_edge; the root's edge slot is ignored), returns dict
+    with Db (lower-triangular), Eb (root slot 0) and info [...].  Dense
+    definition Ab = -A^-1 Gbar A^-1 (gabp-sparse-inv, "Differentiable selected
+    inverse")."""
+    parent = np.ascontiguousarray(parent, dtype=np.int32)
+    diag, edge = _f64(diag), _f64(edge)
+    Gb_diag, Gb_edge = _f64(Gb_diag), _f64(Gb_edge)
+    lead = parent.shape[:-1]
+    n = parent.shape[-1]
+    b = diag.shape[-1]
+    trees = int(np.prod(lead)) if lead else 1
+    for a in (diag, edge, Gb_diag, Gb_edge):
+        assert a.shape == lead + (n, b, b)
+    Db = np.empty(lead + (n, b, b))
+    Eb = np.empty(lead + (n, b, b))
+    info = np.empty(lead, dtype=np.int32)
+    rc = _load(lib).oracle_tree_backward(_ptr(parent), trees, n, b, _ptr(diag), _ptr(edge), _ptr(Gb_diag),
+                                         _ptr(Gb_edge), _ptr(Db), _ptr(Eb), _ptr(info))
+    if rc != 0:
+        raise ValueError("oracle_tree_backward: invalid arguments")
+    return {"Db": Db, "Eb": Eb, "info": info}
 
 
 def tree(parent, diag, edge, lib=None):

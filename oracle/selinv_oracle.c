@@ -350,15 +350,41 @@ int oracle_chain_sample(const double *diag, const double *lower, int64_t batch, 
  * The dense inverse comes from the textbook Cholesky factor of A.  Returns
  * info (-1 ok, else the block holding the first failing pivot).
  */
+/* Ab := -A^-1 Gbar A^-1 for a dense SPD A (N x N, lower triangle read) from
+ * its textbook Cholesky factor.  Returns -1, or the row of the first pivot
+ * that is not > 0 (A is then not positive definite). */
+static int dense_cotangent(int N, const double *A, const double *Gbar, double *Ab)
+{
+    const size_t NN = (size_t)N * N;
+    double *R = malloc(NN * sizeof(double)), *Ri = malloc(NN * sizeof(double));
+    double *G = malloc(NN * sizeof(double)), *T = malloc(NN * sizeof(double));
+    int fail = -1;
+    if (cholesky_lower(N, A, R) != 0) {
+        for (int j = 0; j < N && fail < 0; ++j) {    /* the failing pivot's row */
+            double d = A[(size_t)j * N + j];
+            for (int k = 0; k < j; ++k) d -= R[(size_t)j * N + k] * R[(size_t)j * N + k];
+            if (!(d > 0.0)) fail = j;
+        }
+        if (fail < 0) fail = 0;
+        goto done;
+    }
+    lower_inverse(N, R, Ri);
+    matmul(N, Ri, 1, Ri, 0, G);                      /* A^-1 = R^-T R^-1 */
+    matmul(N, G, 0, Gbar, 0, T);                     /* G Gbar */
+    matmul(N, T, 0, G, 0, Ab);                       /* G Gbar G */
+    for (size_t k = 0; k < NN; ++k) Ab[k] = -Ab[k];
+done:
+    free(R); free(Ri); free(G); free(T);
+    return fail;
+}
+
 static int chain_backward_one(int64_t L, int b, const double *diag, const double *lower,
                               const double *Gb_diag, const double *Gb_lower, double *Db, double *Bb)
 {
     const size_t bb = (size_t)b * b;
     const int N = (int)(L * b);
     const size_t NN = (size_t)N * N;
-    double *A = calloc(NN, sizeof(double)), *R = malloc(NN * sizeof(double));
-    double *Ri = malloc(NN * sizeof(double)), *G = malloc(NN * sizeof(double));
-    double *Gbar = calloc(NN, sizeof(double)), *T = malloc(NN * sizeof(double));
+    double *A = calloc(NN, sizeof(double)), *Gbar = calloc(NN, sizeof(double));
     double *Ab = malloc(NN * sizeof(double));
     int info = -1;
     for (int64_t i = 0; i < L; ++i)
@@ -374,19 +400,8 @@ static int chain_backward_one(int64_t L, int b, const double *diag, const double
                     Gbar[lrow * N + col] = Gb_lower[bb * i + r * b + c];
                 }
             }
-    if (cholesky_lower(N, A, R) != 0) {
-        for (int j = 0; j < N; ++j) {                /* the failing pivot's block */
-            double d = A[(size_t)j * N + j];
-            for (int k = 0; k < j; ++k) d -= R[(size_t)j * N + k] * R[(size_t)j * N + k];
-            if (!(d > 0.0)) { info = j / b; break; }
-        }
-        goto done;
-    }
-    lower_inverse(N, R, Ri);
-    matmul(N, Ri, 1, Ri, 0, G);                      /* A^-1 = R^-T R^-1 */
-    matmul(N, G, 0, Gbar, 0, T);                     /* G Gbar */
-    matmul(N, T, 0, G, 0, Ab);                       /* G Gbar G */
-    for (size_t k = 0; k < NN; ++k) Ab[k] = -Ab[k];
+    const int fail = dense_cotangent(N, A, Gbar, Ab);
+    if (fail >= 0) { info = fail / b; goto done; }
     for (int64_t i = 0; i < L; ++i)
         for (int r = 0; r < b; ++r)
             for (int c = 0; c < b; ++c) {
@@ -401,7 +416,7 @@ static int chain_backward_one(int64_t L, int b, const double *diag, const double
                 }
             }
 done:
-    free(A); free(R); free(Ri); free(G); free(Gbar); free(T); free(Ab);
+    free(A); free(Gbar); free(Ab);
     return info;
 }
 
@@ -582,6 +597,93 @@ out:
     free(first); free(kids); free(next); free(bfs);
     free(Rinv); free(Sc); free(Rf); free(Si); free(ES); free(ESE); free(t1); free(t2);
     return info;
+}
+
+/*
+ * Cotangents of the tree selected inverse (gabp-sparse-inv, "Differentiable
+ * selected inverse": selinv_tree's gradients reach diag and edge).  The same
+ * dense definition as the chain's, Ab = -A^-1 Gbar A^-1, with Gbar holding
+ * Gb_diag[v] at (v, v) and Gb_edge[v] at (p(v), v) (the block G_edge[v]
+ * holds); D_v receives the lower-triangle projection of Ab_vv and edge[v],
+ * which sits at (p, v) and transposed at (v, p), receives
+ * Ab_{p,v} + (Ab_{v,p})^T; the root's edge slot receives 0.  Returns info:
+ * -1 ok, -2 malformed parent array, else the node of the first failing pivot
+ * in natural order (A is then not positive definite).
+ */
+static int tree_backward_one(int64_t n, int b, const int32_t *parent, const double *diag, const double *edge,
+                             const double *Gb_diag, const double *Gb_edge, double *Db, double *Eb)
+{
+    const size_t bb = (size_t)b * b;
+    int64_t root = -1;
+    for (int64_t v = 0; v < n; ++v) {
+        if (parent[v] == -1) { if (root >= 0) return -2; root = v; }
+        else if (parent[v] < 0 || parent[v] >= n || parent[v] == v) return -2;
+    }
+    if (root < 0) return -2;
+    for (int64_t v = 0; v < n; ++v) {                /* every node reaches the root */
+        int64_t u = v, steps = 0;
+        while (parent[u] >= 0 && steps <= n) { u = parent[u]; ++steps; }
+        if (u != root) return -2;
+    }
+    const int N = (int)(n * b);
+    const size_t NN = (size_t)N * N;
+    double *A = calloc(NN, sizeof(double)), *Gbar = calloc(NN, sizeof(double));
+    double *Ab = malloc(NN * sizeof(double));
+    int info = -1;
+    for (int64_t v = 0; v < n; ++v) {
+        const int64_t p = parent[v];
+        for (int r = 0; r < b; ++r)
+            for (int c = 0; c < b; ++c) {
+                const size_t vr = (size_t)(v * b + r), vc = (size_t)(v * b + c);
+                A[vr * N + vc] = (c <= r) ? diag[bb * v + r * b + c] : diag[bb * v + c * b + r];
+                Gbar[vr * N + vc] = Gb_diag[bb * v + r * b + c];
+                if (p >= 0) {
+                    const size_t pr = (size_t)(p * b + r);
+                    A[pr * N + vc] = edge[bb * v + r * b + c];                  /* A_{p,v} = E_v */
+                    A[vc * N + pr] = edge[bb * v + r * b + c];                  /* A_{v,p} = E_v^T */
+                    Gbar[pr * N + vc] = Gb_edge[bb * v + r * b + c];
+                }
+            }
+    }
+    const int fail = dense_cotangent(N, A, Gbar, Ab);
+    if (fail >= 0) { info = fail / b; goto done; }
+    for (int64_t v = 0; v < n; ++v) {
+        const int64_t p = parent[v];
+        for (int r = 0; r < b; ++r)
+            for (int c = 0; c < b; ++c) {
+                const size_t vr = (size_t)(v * b + r), vc = (size_t)(v * b + c);
+                const double lo = Ab[vr * N + vc], up = Ab[vc * N + vr];
+                Db[bb * v + r * b + c] = c < r ? lo + up : (c == r ? lo : 0.0);
+                if (p >= 0) {
+                    const size_t pr = (size_t)(p * b + r);
+                    Eb[bb * v + r * b + c] = Ab[pr * N + vc] + Ab[vc * N + pr];
+                } else {
+                    Eb[bb * v + r * b + c] = 0.0;
+                }
+            }
+    }
+done:
+    free(A); free(Gbar); free(Ab);
+    return info;
+}
+
+/* Batched tree backward: parent [trees,n]; diag, edge, Gb_diag, Gb_edge, Db,
+ * Eb [trees,n,b,b]; info [trees]. */
+int oracle_tree_backward(const int32_t *parent, int64_t trees, int64_t n, int b, const double *diag,
+                         const double *edge, const double *Gb_diag, const double *Gb_edge, double *Db,
+                         double *Eb, int32_t *info)
+{
+    if (trees < 0 || n < 1 || b < 1 || !parent || !diag || !edge || !Gb_diag || !Gb_edge || !Db || !Eb ||
+        !info)
+        return 1;
+    const size_t bb = (size_t)b * b;
+    int64_t t;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (t = 0; t < trees; ++t)
+        info[t] = tree_backward_one(n, b, parent + n * t, diag + bb * n * t, edge + bb * n * t,
+                                    Gb_diag + bb * n * t, Gb_edge + bb * n * t, Db + bb * n * t,
+                                    Eb + bb * n * t);
+    return 0;
 }
 
 /* Batched tree draws: z, w [trees,n,b]; logdet [trees] or NULL; info [trees]. */

@@ -486,6 +486,62 @@ def pin_backward_trace(lib=None):
     return worst
 
 
+def pin_tree_backward_finite_differences(lib=None):
+    """Tree cotangents against central differences of the (pinned) tree forward
+    oracle, every entry of diag and of the non-root edge slots."""
+    worst = 0.0
+    for parent, b, seed in [(np.array([-1, 0, 0, 0]), 2, 41), (np.array([2, 0, -1, 1, 1]), 2, 42)]:
+        P = parent[None].astype(np.int32)
+        d, e = inputs.tree_inputs_from_parent(P, b, seed=seed, load=1.0)
+        rng = np.random.default_rng(seed)
+        gd, ge = rng.standard_normal(d.shape), rng.standard_normal(e.shape)
+        out = oracle.tree_backward(P, d, e, gd, ge, lib=lib)
+        if (out["info"] != -1).any():
+            return float("inf")
+
+        def loss(dd, ee):
+            o = oracle.tree(P, dd, ee, lib=lib)
+            return float((o["G_diag"] * gd).sum() + (o["G_edge"] * ge).sum())
+
+        h = 1e-5
+        scale = max(1.0, float(np.abs(out["Db"]).max()), float(np.abs(out["Eb"]).max()))
+        for idx in np.ndindex(*d.shape):
+            dp, dm = d.copy(), d.copy()
+            dp[idx] += h
+            dm[idx] -= h
+            worst = max(worst, abs((loss(dp, e) - loss(dm, e)) / (2 * h) - out["Db"][idx]) / scale)
+        for idx in np.ndindex(*e.shape):
+            if parent[idx[1]] < 0:
+                worst = max(worst, abs(out["Eb"][idx]))      # the root slot gets nothing
+                continue
+            ep, em = e.copy(), e.copy()
+            ep[idx] += h
+            em[idx] -= h
+            worst = max(worst, abs((loss(d, ep) - loss(d, em)) / (2 * h) - out["Eb"][idx]) / scale)
+    return worst
+
+
+def pin_tree_backward_path_is_chain(lib=None):
+    """The path tree parent(i) = i + 1 is the chain (rooted at its last node):
+    its cotangents equal the chain backward's block for block."""
+    L, b = 7, 3
+    d, l, _ = inputs.chain_inputs(2, L, b, seed=43, load=1.0, with_rhs=False)
+    rng = np.random.default_rng(43)
+    gd, gl = rng.standard_normal(d.shape), rng.standard_normal(l.shape)
+    ref = oracle.chain_backward(d, l, gd, gl, lib=lib)
+    parent = np.repeat(np.array(list(range(1, L)) + [-1], dtype=np.int32)[None], 2, 0)
+    edge = np.zeros(d.shape)
+    edge[:, :L - 1] = l
+    ge = np.zeros(d.shape)
+    ge[:, :L - 1] = gl
+    ge[:, L - 1] = rng.standard_normal((2, b, b))        # the root slot's cotangent is ignored
+    out = oracle.tree_backward(parent, d, edge, gd, ge, lib=lib)
+    if (out["info"] != -1).any() or (ref["info"] != -1).any():
+        return float("inf")
+    return max(rel(out["Db"], ref["Db"]), rel(out["Eb"][:, :L - 1], ref["Bb"]),
+               float(np.abs(out["Eb"][:, L - 1]).max()))
+
+
 # name -> (function, tolerance)
 PINS = {
     "tiny_chains_dense": (pin_tiny_chains_dense, 1e-12),
@@ -505,4 +561,6 @@ PINS = {
     "backward_finite_differences": (pin_backward_finite_differences, 1e-7),
     "backward_decoupled": (pin_backward_decoupled, 1e-12),
     "backward_trace": (pin_backward_trace, 1e-11),
+    "tree_backward_finite_differences": (pin_tree_backward_finite_differences, 1e-7),
+    "tree_backward_path_is_chain": (pin_tree_backward_path_is_chain, 1e-12),
 }

@@ -64,6 +64,12 @@ MUTANTS = {
                                                "Gbar[row * N + col + b] = Gb_lower[bb * i + r * b + c];"),
     "backward_gbar_diag_dropped": ("Gbar[row * N + col] = Gb_diag[bb * i + r * b + c];",
                                    "Gbar[row * N + col] = 0.0 * Gb_diag[bb * i + r * b + c];"),
+    "tree_backward_eb_untransposed": ("Eb[bb * v + r * b + c] = Ab[pr * N + vc] + Ab[vc * N + pr];",
+                                      "Eb[bb * v + r * b + c] = Ab[pr * N + vc] + Ab[pr * N + vc];"),
+    "tree_backward_gbar_edge_untransposed_above": ("Gbar[pr * N + vc] = Gb_edge[bb * v + r * b + c];",
+                                                   "Gbar[vr * N + (size_t)(p * b + c)] = Gb_edge[bb * v + r * b + c];"),
+    "tree_backward_db_mirror_dropped": ("Db[bb * v + r * b + c] = c < r ? lo + up : (c == r ? lo : 0.0);",
+                                        "Db[bb * v + r * b + c] = c < r ? lo : (c == r ? lo : 0.0);"),
     "tree_g_diag_transposed": ("matmul(b, Sinv + bb * v, 0, edge + bb * v, 1, T1);",
                                "matmul(b, Sinv + bb * v, 0, edge + bb * v, 0, T1);"),
 }
