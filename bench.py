@@ -47,6 +47,7 @@ KERNEL_SOURCES = {
     "chain_large_kernel": ["chain_large.cu", "common.cuh"],
     "tree_collect_kernel": ["tree.cu", "warp16.cuh", "common.cuh"],
     "chain_backward_kernel": ["chain_backward.cu", "warp16.cuh", "common.cuh"],
+    "tree_bw_collect_kernel": ["tree.cu", "warp16.cuh", "common.cuh"],
 }
 
 
@@ -64,7 +65,8 @@ def parse():
     ap.add_argument("--op", default="selinv", choices=["selinv", "sample", "backward"],
                     help="selinv: selected inverse + log det (+ solve); sample: Gaussian draw "
                          "eta = A^-1 r + L^-T z + log det (chains; on trees eta = L^-T z); backward: "
-                         "cotangents of diag and lower from those of G_diag and G_lower (chains, b <= 16)")
+                         "cotangents of diag and lower (edge) from those of G_diag and G_lower (G_edge); "
+                         "chains and trees, b <= 16")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -159,7 +161,9 @@ def oracle_inputs(w, elems, op):
     g = inputs.generate(w, elements=elems)
     if op == "sample":
         g["z"] = inputs.standard_normals(w.batch, w.L, w.b, w.seed, elems)
-    if op == "backward":
+    if op == "backward" and w.kind == "tree":
+        g["Gb_diag"], g["Gb_edge"] = inputs.tree_cotangents(w.batch, w.L, w.b, w.seed, elems)
+    elif op == "backward":
         g["Gb_diag"], g["Gb_lower"] = inputs.cotangents(w.batch, w.L, w.b, w.seed, elems)
     return g
 
@@ -167,6 +171,8 @@ def oracle_inputs(w, elems, op):
 def oracle_run(oracle, w, g, op):
     if w.kind == "tree" and op == "sample":
         oracle.tree_sample(g["parent"], g["diag"], g["edge"], g["z"])
+    elif w.kind == "tree" and op == "backward":
+        oracle.tree_backward(g["parent"], g["diag"], g["edge"], g["Gb_diag"], g["Gb_edge"])
     elif w.kind == "tree":
         oracle.tree(g["parent"], g["diag"], g["edge"])
     elif op == "sample":
@@ -177,10 +183,22 @@ def oracle_run(oracle, w, g, op):
         oracle.chain(g["diag"], g["lower"], g.get("rhs"))
 
 
+def oracle_workload(w, op):
+    """The workload the oracle times: the same, except for the backward, whose
+    dense definition costs O((L b)^3) per chain or tree: there chains or trees
+    of 512 / b blocks drawn by the same recipe stand in (a few seconds each)."""
+    if op == "backward" and w.L * w.b > 512:
+        n = max(2, 512 // w.b)
+        what = "trees" if w.kind == "tree" else "chains"
+        return dataclasses.replace(w, L=n), f" ({what} of {n} blocks drawn like {w.name}'s)"
+    return w, ""
+
+
 def cpu_baseline(w, dtype_name, op="selinv", budget_s=10.0):
     """The oracle, as it stands, on a bounded sample of the same workload (host cores)."""
     import oracle
     oracle.build()
+    w, note = oracle_workload(w, op)
     n_probe = 32 if w.kind != "grid" else 1
     elems = list(range(min(n_probe, w.batch)))
     g = oracle_inputs(w, elems, op)
@@ -201,7 +219,7 @@ def cpu_baseline(w, dtype_name, op="selinv", budget_s=10.0):
     blocks = len(elems) * w.L
     unit_name = "trees" if w.kind == "tree" else "chains"
     return {"value": blocks / dt, "unit": "blocks/s", "cores": oracle.threads(), "kind": "oracle",
-            "sample": f"{len(elems)} of {w.batch} {unit_name} ({w.name}, float64), {dt:.2f} s"}
+            "sample": f"{len(elems)} of {w.batch} {unit_name} ({w.name}, float64){note}, {dt:.2f} s"}
 
 
 def algorithmic_bytes(w, es, batch, op="selinv"):
@@ -210,7 +228,7 @@ def algorithmic_bytes(w, es, batch, op="selinv"):
     D, B, r and z and writes eta (a tree draw has no r)."""
     b2 = w.b * w.b
     if op == "backward":
-        # read D, G_diag, Gb_diag and B, G_lower, Gb_lower; write Db and Bb
+        # read D, G_diag, Gb_diag and B (edge), G_lower (G_edge), Gb_lower (Gb_edge); write Db and Bb (Eb)
         nodes, edges = batch * w.L, batch * (w.L - 1)
         return es * 4 * b2 * (nodes + edges)
     if op == "sample" and w.kind == "tree":
@@ -233,7 +251,9 @@ def algorithmic_flops(w, batch, op="selinv"):
     """Nominal 7 b^3 flops per block: collect (Cholesky b^3/3 + trsm b^3 + syrk b^3) and
     distribute (inverse 2b^3/3 + trmm b^3 + gemm 2b^3 + symmetric half-gemm b^3).  A draw
     needs the collect only (7 b^3 / 3; its triangular solves are O(b^2))."""
-    per = 7.0 / 3.0 if op == "sample" else 7.0
+    # backward: the collect's 7/3 b^3, then six products in the reversed distribute
+    # step and five in the reversed collect step, 2 b^3 each
+    per = {"sample": 7.0 / 3.0, "backward": 73.0 / 3.0}.get(op, 7.0)
     return per * w.b ** 3 * batch * w.L
 
 
@@ -291,9 +311,12 @@ def run_reference(args):
     w = inputs.WORKLOADS[args.workload]
     import oracle
     oracle.build()
+    w, note = oracle_workload(w, args.op)
     n_per_step = {"chain": 64, "tree": 1, "grid": 1}[w.kind]
     if w.kind == "chain" and w.L * w.b ** 3 > 64 * 16 ** 3 * 64:
         n_per_step = 2
+    if args.op == "backward" and w.kind == "chain":
+        n_per_step = 16
     elems = list(range(min(n_per_step, w.batch)))
     g = oracle_inputs(w, elems, args.op)
     times = []
@@ -304,7 +327,7 @@ def run_reference(args):
             times.append(time.perf_counter() - t0)
     blocks = len(elems) * w.L
     value = blocks * len(times) / sum(times)
-    sample = f"{len(elems)} of {w.batch} {'trees' if w.kind == 'tree' else 'chains'} per step"
+    sample = f"{len(elems)} of {w.batch} {'trees' if w.kind == 'tree' else 'chains'} per step{note}"
     line = {
         "impl": "reference", "metric": metric_name(args.op, "f64"), "value": value, "unit": "blocks/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -368,10 +391,13 @@ def run_ours(args):
                 raise SystemExit("--op sample with b > 16 runs in float64 only")
             g["z"] = inputs.standard_normals(w.batch, w.L, w.b, w.seed, elems)
         if args.op == "backward":
-            if w.kind != "chain" or w.b > 16:
-                raise SystemExit("--op backward runs on chain workloads with b <= 16")
+            if w.b > 16:
+                raise SystemExit("--op backward runs on workloads with b <= 16")
             g.pop("rhs", None)
-            g["Gb_diag"], g["Gb_lower"] = inputs.cotangents(w.batch, w.L, w.b, w.seed, elems)
+            if w.kind == "tree":
+                g["Gb_diag"], g["Gb_edge"] = inputs.tree_cotangents(w.batch, w.L, w.b, w.seed, elems)
+            else:
+                g["Gb_diag"], g["Gb_lower"] = inputs.cotangents(w.batch, w.L, w.b, w.seed, elems)
         host_in = {k: torch.from_numpy(v).to(tdt).pin_memory() for k, v in g.items()
                    if v is not None and k != "parent"}
         dev_in = {k: v.to("cuda", non_blocking=True) for k, v in host_in.items()}
@@ -385,7 +411,21 @@ def run_ours(args):
                "logdet": torch.empty(batch, dtype=torch.float64, device="cuda"),
                "info": torch.empty(batch, dtype=torch.int32, device="cuda")}
         ws = torch.empty(plan.workspace_size(tdt, w.b), dtype=torch.uint8, device="cuda")
-        if args.op == "sample":
+        if args.op == "backward":
+            fwd = selinv.selinv_tree(plan, dev_in["diag"], dev_in["edge"])
+            for k in ("G_diag", "G_edge"):
+                dev_in[k] = fwd[k]
+                host_in[k] = fwd[k].cpu().pin_memory()
+            kernel = "tree_bw_collect_kernel"
+            launches_per_step = 4 if w.L > 1 else 3
+            out = {"Db": torch.empty_like(dev_in["diag"]), "Eb": torch.empty_like(dev_in["diag"]),
+                   "info": out["info"]}
+            ws = torch.empty(plan.backward_workspace_size(tdt, w.b), dtype=torch.uint8, device="cuda")
+
+            def step():
+                selinv.tree_backward(plan, dev_in["diag"], dev_in["edge"], dev_in["G_diag"], dev_in["G_edge"],
+                                     dev_in["Gb_diag"], dev_in["Gb_edge"], check=False, out=out, workspace=ws)
+        elif args.op == "sample":
             kernel = "tree_collect_kernel (draw mode)"
             out = {"eta": torch.empty_like(dev_in["z"]), "logdet": out["logdet"], "info": out["info"]}
 
@@ -524,7 +564,7 @@ def run_ours(args):
     flop_rate = flops / (kernel_ms / 1e3) / 1e12
     traffic = profiled_traffic(kernel, w.name) if full_size else None
     hbm_src = f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback 6650 GB/s"
-    if w.b >= 32 and args.dtype == "f64":
+    if (w.b >= 32 or args.op == "backward") and args.dtype == "f64":
         # arithmetic intensity 7 b^3 / (32 b^2) flop/byte: past the FP64 ridge from b = 32 on
         peak = fp64_peak_tflops(torch)
         roof = {"bound": "tensor", "achieved": flop_rate, "peak": peak, "unit": "TFLOP/s",

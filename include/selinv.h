@@ -294,6 +294,30 @@ selinv_status selinv_tree_sample(const selinv_tree_plan_t *plan, selinv_dtype dt
                                  double *logdet, int32_t *info,
                                  void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Cotangents of the tree selected inverse (b <= 16): the tree form of
+ * selinv_chain_backward.  From the cotangents Gb_diag, Gb_edge [trees, n, b, b]
+ * of selinv_tree's outputs (NULL = zero; the root's Gb_edge slot is ignored)
+ * writes Db [trees, n, b, b] (lower-triangular: only D_v's lower triangle is
+ * read) and Eb [trees, n, b, b] (edge[v] sits at (p(v), v) and, transposed,
+ * at (v, p(v)); the root slot is written 0), Ab = -A^-1 Gbar A^-1 read back
+ * onto the inputs.  (gabp-sparse-inv 0.3.2, "Differentiable selected
+ * inverse": selinv_tree's gradients reach diag and edge through an analytic
+ * two-pass backward.)  Pass 1 runs children before parents, pass 2 parents
+ * before children, like the forward's sweeps.
+ *   diag, edge, G_diag, G_edge  the forward's inputs and outputs (device)
+ *   info [trees]   -1, or a node whose Schur complement is not positive
+ *                  definite (outputs then unspecified)
+ * Workspace: selinv_tree_backward_workspace_size(plan, dtype, b) bytes.
+ */
+size_t selinv_tree_backward_workspace_size(const selinv_tree_plan_t *plan, selinv_dtype dtype, int32_t b);
+
+selinv_status selinv_tree_backward(const selinv_tree_plan_t *plan, selinv_dtype dtype, int32_t b,
+                                   const void *diag, const void *edge, const void *G_diag,
+                                   const void *G_edge, const void *Gb_diag, const void *Gb_edge,
+                                   void *Db, void *Eb, int32_t *info, void *workspace,
+                                   size_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -434,6 +434,276 @@ tree_draw_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *nodes, i
     }
 }
 
+// ---------------------------------------------------------------------------
+// Cotangents (gabp-sparse-inv, "Differentiable selected inverse": selinv_tree's
+// gradients reach diag and edge through an analytic two-pass backward).  The
+// passes are the reverse-mode forms of the forward's sweeps, with P_v = S_v^-1,
+// W_v = E_v P_v, p = parent(v):
+// pass 1, children before parents (a fresh collect that rebuilds P_v, fused
+// with the reversed distribute, which ran parents first):
+//   Ga   = Gb_vv + sum_{c in ch(v)} C_c
+//   Xb   = Gb_edge[v] - W_v Ga,  Wb = -G_edge[v] Ga^T - G_pp Xb
+//   C_v  = -Xb W_v^T (to the parent),  Eb_v <- Wb P_v,
+//   Pd_v = (Ga + E_v^T Wb) + its transpose   (only symmetric parts matter below)
+//   root: Pd = Ga + Ga^T.
+// pass 2, parents before children (the reversed collect), Sg = Sb + Sb^T:
+//   Sg_v = -P_v (Pd_v - E_v^T Sg_p E_v) P_v   (root: -P Pd P)
+//   Db_v = Sg_v below the diagonal, half of it on the diagonal, 0 above
+//   Eb_v -= Sg_p W_v
+// The root's pass-2 step runs where pass 1 ends, in the warp that reaches it.
+template <class T> struct TreeBwdBufs {
+    const T *diag, *edge, *G_diag, *G_edge, *Gb_diag, *Gb_edge;
+    T *Db, *Eb;
+    T *ws_P, *ws_U, *ws_C, *ws_Pd;   // per node: P_v and U_v (later Sg_v) lower slots, C_v full, Pd_v lower
+    int32_t *info;
+    int b;
+};
+
+constexpr int BW_CSLOT = 256;
+
+// Symmetric tile from a lower slot written earlier in this launch (read
+// through L2), rebuilt through the shared image s.
+template <class T> SELINV_DEVINL void sym_from_slot(w16::Tile<T> &a, const T *slot, T *s, int lane, int g, int t)
+{
+    load_lower_slot_l2<T>(a, slot, lane, g, t);
+    w16::to_smem<T>(s, a, g, t);
+    __syncwarp();
+    w16::from_smem_lower<T>(a, s, g, t);
+    __syncwarp();
+}
+
+template <class T> SELINV_DEVINL void transpose_t(w16::Tile<T> &out, const w16::Tile<T> &in, T *s, int g, int t)
+{
+    w16::to_smem<T>(s, in, g, t);
+    __syncwarp();
+    w16::from_smem_T<T>(out, s, g, t);
+    __syncwarp();
+}
+
+template <class T, bool FULL> SELINV_DEVINL void load_gen(w16::Tile<T> &a, const T *M, int b, int g, int t, bool l2)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = g + 8 * h, c = w16::tcol(t, q);
+            const int ld = FULL ? 16 : b;
+            a.v[h][q] = (FULL || (r < b && c < b)) ? (l2 ? __ldcg(M + r * ld + c) : __ldg(M + r * ld + c)) : T(0);
+        }
+}
+
+// Db_v from Sg_v, stored; Sg symmetric.
+template <class T, bool FULL> SELINV_DEVINL void store_db(T *Db, const w16::Tile<T> &sg, int b, int g, int t)
+{
+    w16::Tile<T> d;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = g + 8 * h, c = w16::tcol(t, q);
+            d.v[h][q] = c < r ? sg.v[h][q] : (c == r ? T(0.5) * sg.v[h][q] : T(0));
+        }
+    w16::store_block<T, FULL>(Db, d, b, g, t);
+}
+
+template <class T, bool FULL>
+__global__ void __launch_bounds__(TWARPS * 32)
+tree_bw_collect_kernel(TreeBwdBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leaves, int64_t nleaves)
+{
+    using namespace w16;
+    constexpr int E = SL<T>::ELEMS;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    T *s0 = reinterpret_cast<T *>(smem_raw) + wid * (3 * E + 32);
+    T *s1 = s0 + E, *s2 = s1 + E, *cb = s2 + E;
+    const int b = p.b;
+    const int64_t bb = (int64_t)b * b;
+
+    for (;;) {
+        const unsigned long long k = warp_take(sy.counters, lane);
+        if (k >= (unsigned long long)nleaves) break;
+        int32_t v = leaves[k];
+        for (;;) {                                   // v, then each parent this warp completes last
+            const int32_t par = td.parent[v];
+            Tile<T> S, Ga;
+            load_sym<T, FULL>(S, p.diag + v * bb, b, g, t);
+            if (p.Gb_diag) load_gen<T, FULL>(Ga, p.Gb_diag + v * bb, b, g, t, false);
+            else zero(Ga);
+            const int32_t c0 = td.child_ptr[v], c1 = td.child_ptr[v + 1];
+            for (int32_t c = c0; c < c1; ++c) {        // S -= U_c, Ga += C_c
+                const int32_t ch = td.child_idx[c];
+                Tile<T> u, cc;
+                sym_from_slot<T>(u, p.ws_U + (int64_t)ch * SLOT_ELEMS, s0, lane, g, t);
+                load_gen<T, true>(cc, p.ws_C + (int64_t)ch * BW_CSLOT, 16, g, t, true);
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        S.v[h][q] -= u.v[h][q];
+                        Ga.v[h][q] += cc.v[h][q];
+                    }
+            }
+            LogAcc det;
+            det.init();
+            bool bad = false;
+            spd_inverse<T>(S, cb, g, t, det, bad);  // S = P_v
+            if (lane == 0 && bad) atomicMin(p.info + v / td.n, (int32_t)(v % td.n));
+            store_lower_slot<T>(p.ws_P + (int64_t)v * SLOT_ELEMS, S, lane, g, t);
+            Tile<T> GaT;
+            transpose_t<T>(GaT, Ga, s0, g, t);
+            if (par < 0) {                            // root: Pd = Ga + Ga^T, then its pass-2 step
+                Tile<T> pd = Ga, q, sg;
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) pd.v[h][r] += GaT.v[h][r];
+                zero(q);
+                gemm_nt<false>(q, S, pd, s1, s2, g, t);            // P Pd
+                zero(sg);
+                gemm_nt<true, true>(sg, q, S, s1, s2, g, t);        // Sg = -P Pd P (lower tiles)
+                mirror_upper(sg, g, t);
+                store_db<T, FULL>(p.Db + v * bb, sg, b, g, t);
+                Tile<T> z;
+                zero(z);
+                store_block<T, FULL>(p.Eb + v * bb, z, b, g, t);
+                store_lower_slot<T>(p.ws_U + (int64_t)v * SLOT_ELEMS, sg, lane, g, t);
+                __syncwarp();                         // the warp's stores are ordered before lane 0's release
+                if (lane == 0) st_release(sy.done + v, 1);
+                __syncwarp();
+                break;
+            }
+            Tile<T> Ev, W;
+            load_gen<T, FULL>(Ev, p.edge + v * bb, b, g, t, false);
+            zero(W);
+            gemm_nt<false>(W, Ev, S, s1, s2, g, t);               // W = E P
+            {
+                Tile<T> u;
+                zero(u);
+                gemm_nt<false, true>(u, W, Ev, s1, s2, g, t);      // U = W E^T (lower tiles)
+                store_lower_slot<T>(p.ws_U + (int64_t)v * SLOT_ELEMS, u, lane, g, t);
+            }
+            Tile<T> Xb, Wb;
+            if (p.Gb_edge) load_gen<T, FULL>(Xb, p.Gb_edge + v * bb, b, g, t, false);
+            else zero(Xb);
+            gemm_nt<true>(Xb, W, GaT, s1, s2, g, t);              // Xb = Gb_edge - W Ga
+            {
+                Tile<T> X;
+                load_gen<T, FULL>(X, p.G_edge + v * bb, b, g, t, false);
+                zero(Wb);
+                gemm_nt<true>(Wb, X, Ga, s1, s2, g, t);           // Wb = -G_edge Ga^T
+            }
+            {
+                Tile<T> XbT, Gp;
+                transpose_t<T>(XbT, Xb, s0, g, t);
+                load_gen<T, FULL>(Gp, p.G_diag + (int64_t)par * bb, b, g, t, false);
+                gemm_nt<true>(Wb, Gp, XbT, s1, s2, g, t);         // Wb -= G_pp Xb
+            }
+            {
+                Tile<T> cv;
+                zero(cv);
+                gemm_nt<true>(cv, Xb, W, s1, s2, g, t);           // C_v = -Xb W^T
+                store_block<T, true>(p.ws_C + (int64_t)v * BW_CSLOT, cv, 16, g, t);
+            }
+            {
+                Tile<T> ET, WbT;
+                transpose_t<T>(ET, Ev, s0, g, t);
+                transpose_t<T>(WbT, Wb, s0, g, t);
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) Ga.v[h][r] += GaT.v[h][r];
+                gemm_nt<false>(Ga, ET, WbT, s1, s2, g, t);        // + E^T Wb
+                gemm_nt<false>(Ga, WbT, ET, s1, s2, g, t);        // + Wb^T E
+                store_lower_slot<T>(p.ws_Pd + (int64_t)v * SLOT_ELEMS, Ga, lane, g, t);
+            }
+            {
+                Tile<T> ed;
+                zero(ed);
+                gemm_nt<false>(ed, Wb, S, s1, s2, g, t);          // Eb_v <- Wb P
+                store_block<T, FULL>(p.Eb + v * bb, ed, b, g, t);
+            }
+            __syncwarp();                             // the warp's stores are ordered before lane 0's release
+            int old = 0;
+            if (lane == 0) old = atom_add_acq_rel(sy.pending + par, -1);
+            old = __shfl_sync(FULL_MASK, old, 0);
+            __syncwarp();                             // every lane's reads of the siblings' slots follow the acquire
+            if (old != 1) break;
+            v = par;
+        }
+    }
+}
+
+template <class T, bool FULL>
+__global__ void __launch_bounds__(TWARPS * 32)
+tree_bw_distribute_kernel(TreeBwdBufs<T> p, TreeDev td, TreeSync sy, const int32_t *nodes, int64_t count)
+{
+    using namespace w16;
+    constexpr int E = SL<T>::ELEMS;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    T *s0 = reinterpret_cast<T *>(smem_raw) + wid * (3 * E + 32);
+    T *s1 = s0 + E, *s2 = s1 + E;
+    const int b = p.b;
+    const int64_t bb = (int64_t)b * b;
+    for (;;) {
+        const unsigned long long k = warp_take(sy.counters + 1, lane);
+        if (k >= (unsigned long long)count) break;
+        const int32_t v = nodes[k];
+        const int32_t par = td.parent[v];
+        // operands that do not depend on the parent first
+        Tile<T> P, Pt, Ev, ed;
+        sym_from_slot<T>(P, p.ws_P + (int64_t)v * SLOT_ELEMS, s0, lane, g, t);
+        sym_from_slot<T>(Pt, p.ws_Pd + (int64_t)v * SLOT_ELEMS, s0, lane, g, t);
+        load_gen<T, FULL>(Ev, p.edge + v * bb, b, g, t, false);
+        load_gen<T, FULL>(ed, p.Eb + v * bb, b, g, t, true);
+        int ok = 1;                                   // wait for Sg_p (bounded)
+        if (lane == 0) {
+            int n = 0;
+            while (ld_acquire(sy.done + par) == 0) {
+                if (++n > SPIN_LIMIT) { ok = 0; break; }
+                __nanosleep(64);
+            }
+        }
+        ok = __shfl_sync(FULL_MASK, ok, 0);
+        __syncwarp();                                 // every lane's reads below follow lane 0's acquire
+        if (!ok) {                                    // cannot happen for a valid plan: report, move on
+            if (lane == 0) atomicMin(p.info + v / td.n, -2);
+            continue;
+        }
+        Tile<T> Sp, ET;
+        sym_from_slot<T>(Sp, p.ws_U + (int64_t)par * SLOT_ELEMS, s0, lane, g, t);
+        transpose_t<T>(ET, Ev, s0, g, t);
+        {
+            Tile<T> zt;
+            zero(zt);
+            gemm_nt<false>(zt, ET, Sp, s1, s2, g, t);             // E^T Sg_p
+            gemm_nt<true>(Pt, zt, ET, s1, s2, g, t);              // Pt = Pd - E^T Sg_p E
+        }
+        {
+            Tile<T> wt;
+            zero(wt);
+            gemm_nt<false>(wt, P, Ev, s1, s2, g, t);              // W^T = P E^T
+            gemm_nt<true>(ed, Sp, wt, s1, s2, g, t);              // Eb_v = Eb_v - Sg_p W
+            store_block<T, FULL>(p.Eb + v * bb, ed, b, g, t);
+        }
+        Tile<T> q, sg;
+        zero(q);
+        gemm_nt<false>(q, P, Pt, s1, s2, g, t);                   // P Pt (Pt symmetric)
+        zero(sg);
+        gemm_nt<true, true>(sg, q, P, s1, s2, g, t);              // Sg_v = -P Pt P (lower tiles)
+        mirror_upper(sg, g, t);
+        store_db<T, FULL>(p.Db + v * bb, sg, b, g, t);
+        if (td.child_ptr[v + 1] > td.child_ptr[v]) {
+            store_lower_slot<T>(p.ws_U + (int64_t)v * SLOT_ELEMS, sg, lane, g, t);
+            __syncwarp();                             // the warp's stores are ordered before lane 0's release
+            if (lane == 0) st_release(sy.done + v, 1);
+            __syncwarp();
+        }
+    }
+}
+
 __global__ void tree_init(const int32_t *child_ptr, int64_t N, int32_t *pending, int32_t *done,
                           unsigned long long *counters, int32_t *info, int64_t trees)
 {
@@ -477,6 +747,12 @@ __global__ void __launch_bounds__(FIN_THREADS) tree_finalize(const double *ws_ld
         if (logdet) logdet[tr] = part[0];
         if (info[tr] == INT_MAX) info[tr] = -1;
     }
+}
+
+__global__ void tree_info_finalize(int32_t *info, int64_t trees)
+{
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < trees && info[i] == INT_MAX) info[i] = -1;
 }
 
 template <class T> size_t slot_bytes() { return sizeof(T) * w16::SLOT_ELEMS; }
@@ -550,6 +826,76 @@ cudaError_t run_tree(const selinv_tree_plan_s *pl, int b, const T *diag, const T
         kd<<<(unsigned)bd, TWARPS * 32, smem_d, s>>>(p, td, sy, pl->d_dist_nodes, ndist);
     }
     tree_finalize<<<(unsigned)pl->trees, FIN_THREADS, 0, s>>>(p.ws_ld, pl->n, logdet, info);
+    return cudaGetLastError();
+}
+
+size_t tree_bw_workspace(const selinv_tree_plan_s *pl, size_t elem)
+{
+    const int64_t N = pl->trees * pl->n;
+    return 3 * align256((size_t)N * elem * w16::SLOT_ELEMS) + align256((size_t)N * elem * BW_CSLOT) +
+           2 * align256((size_t)N * sizeof(int32_t)) + 256;
+}
+
+template <class T>
+cudaError_t run_tree_backward(const selinv_tree_plan_s *pl, int b, const T *diag, const T *edge, const T *G_diag,
+                              const T *G_edge, const T *Gb_diag, const T *Gb_edge, T *Db, T *Eb, int32_t *info,
+                              void *ws, bool full, cudaStream_t s)
+{
+    const int64_t N = pl->trees * pl->n;
+    char *w = static_cast<char *>(ws);
+    TreeBwdBufs<T> p;
+    p.diag = diag;
+    p.edge = edge;
+    p.G_diag = G_diag;
+    p.G_edge = G_edge;
+    p.Gb_diag = Gb_diag;
+    p.Gb_edge = Gb_edge;
+    p.Db = Db;
+    p.Eb = Eb;
+    p.ws_P = reinterpret_cast<T *>(w);
+    w += align256(N * slot_bytes<T>());
+    p.ws_U = reinterpret_cast<T *>(w);
+    w += align256(N * slot_bytes<T>());
+    p.ws_Pd = reinterpret_cast<T *>(w);
+    w += align256(N * slot_bytes<T>());
+    p.ws_C = reinterpret_cast<T *>(w);
+    w += align256(N * sizeof(T) * BW_CSLOT);
+    TreeSync sy;
+    sy.pending = reinterpret_cast<int32_t *>(w);
+    w += align256(N * sizeof(int32_t));
+    sy.done = reinterpret_cast<int32_t *>(w);
+    w += align256(N * sizeof(int32_t));
+    sy.counters = reinterpret_cast<unsigned long long *>(w);
+    p.info = info;
+    p.b = b;
+    TreeDev td{pl->d_child_ptr, pl->d_child_idx, pl->d_parent, pl->n};
+
+    const int64_t init_n = std::max<int64_t>(N, pl->trees);
+    tree_init<<<(unsigned)ceil_div(init_n, 256), 256, 0, s>>>(pl->d_child_ptr, N, sy.pending, sy.done, sy.counters,
+                                                               info, pl->trees);
+    const size_t smem = sizeof(T) * (3 * w16::SL<T>::ELEMS + 32) * TWARPS;
+    auto kc = full ? tree_bw_collect_kernel<T, true> : tree_bw_collect_kernel<T, false>;
+    auto kd = full ? tree_bw_distribute_kernel<T, true> : tree_bw_distribute_kernel<T, false>;
+    cudaError_t err = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err == cudaSuccess) err = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int occ_c = 0, occ_d = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_c, kc, TWARPS * 32, smem) != cudaSuccess || occ_c < 1)
+        occ_c = 2;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_d, kd, TWARPS * 32, smem) != cudaSuccess || occ_d < 1)
+        occ_d = 2;
+    const int64_t nleaves = pl->collect_off.size() > 1 ? pl->collect_off[1] - pl->collect_off[0] : 0;
+    const int64_t ndist = pl->dist_off.empty() ? 0 : pl->dist_off.back();
+    const int64_t bc = std::min<int64_t>((int64_t)sms * occ_c, std::max<int64_t>(1, ceil_div(nleaves, TWARPS)));
+    kc<<<(unsigned)bc, TWARPS * 32, smem, s>>>(p, td, sy, pl->d_collect_nodes, nleaves);
+    if (ndist > 0) {
+        const int64_t bd = std::min<int64_t>((int64_t)sms * occ_d, ceil_div(ndist, TWARPS));
+        kd<<<(unsigned)bd, TWARPS * 32, smem, s>>>(p, td, sy, pl->d_dist_nodes, ndist);
+    }
+    tree_info_finalize<<<(unsigned)ceil_div(pl->trees, 256), 256, 0, s>>>(info, pl->trees);
     return cudaGetLastError();
 }
 
@@ -749,6 +1095,50 @@ selinv_status selinv_tree_sample(const selinv_tree_plan_t *pl, selinv_dtype dtyp
         err = run_tree<float>(pl, b, static_cast<const float *>(diag), static_cast<const float *>(edge), nullptr,
                               nullptr, logdet, info, workspace, full, s, static_cast<const float *>(z),
                               static_cast<float *>(eta));
+    return err == cudaSuccess ? SELINV_OK : SELINV_ERR_CUDA;
+}
+
+size_t selinv_tree_backward_workspace_size(const selinv_tree_plan_t *pl, selinv_dtype dtype, int32_t b)
+{
+    if (!pl || (dtype != SELINV_F64 && dtype != SELINV_F32) || b < 1 || b > 16) return 0;
+    return tree_bw_workspace(pl, dtype == SELINV_F64 ? 8 : 4);
+}
+
+selinv_status selinv_tree_backward(const selinv_tree_plan_t *pl, selinv_dtype dtype, int32_t b, const void *diag,
+                                   const void *edge, const void *G_diag, const void *G_edge, const void *Gb_diag,
+                                   const void *Gb_edge, void *Db, void *Eb, int32_t *info, void *workspace,
+                                   size_t workspace_bytes, void *stream)
+{
+    if (!pl || (dtype != SELINV_F64 && dtype != SELINV_F32) || b < 1) return SELINV_ERR_INVALID_ARG;
+    if (b > 16) return SELINV_ERR_UNSUPPORTED;
+    if (!diag || !edge || !G_diag || !G_edge || !Db || !Eb || !info) return SELINV_ERR_INVALID_ARG;
+    const size_t es = dtype == SELINV_F64 ? 8 : 4;
+    const void *ptrs[8] = {diag, edge, G_diag, G_edge, Gb_diag, Gb_edge, Db, Eb};
+    bool al16 = b == 16;
+    for (const void *q : ptrs) {
+        if (!is_aligned(q, es)) return SELINV_ERR_INVALID_ARG;
+        al16 = al16 && is_aligned(q, 16);
+    }
+    if (!is_aligned(info, 4) || !is_aligned(workspace, 256)) return SELINV_ERR_INVALID_ARG;
+    const size_t need = tree_bw_workspace(pl, es);
+    if (!workspace || workspace_bytes < need) return SELINV_ERR_WORKSPACE;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev != pl->device) return SELINV_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t err;
+    if (dtype == SELINV_F64)
+        err = run_tree_backward<double>(pl, b, static_cast<const double *>(diag), static_cast<const double *>(edge),
+                                        static_cast<const double *>(G_diag), static_cast<const double *>(G_edge),
+                                        static_cast<const double *>(Gb_diag), static_cast<const double *>(Gb_edge),
+                                        static_cast<double *>(Db), static_cast<double *>(Eb), info, workspace,
+                                        al16, s);
+    else
+        err = run_tree_backward<float>(pl, b, static_cast<const float *>(diag), static_cast<const float *>(edge),
+                                       static_cast<const float *>(G_diag), static_cast<const float *>(G_edge),
+                                       static_cast<const float *>(Gb_diag), static_cast<const float *>(Gb_edge),
+                                       static_cast<float *>(Db), static_cast<float *>(Eb), info, workspace,
+                                       al16, s);
     return err == cudaSuccess ? SELINV_OK : SELINV_ERR_CUDA;
 }
 

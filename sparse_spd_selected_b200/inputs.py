@@ -244,6 +244,18 @@ def cotangents(batch: int, L: int, b: int, seed: int, elements: Optional[Sequenc
     return np.stack(gd), np.stack(gl)
 
 
+def tree_cotangents(trees: int, n: int, b: int, seed: int, elements: Optional[Sequence[int]] = None):
+    """Standard-normal cotangents (Gb_diag, Gb_edge [n_trees, n, b, b]) of a loss
+    on a tree's selected inverse, tree e drawing from default_rng([seed, e, 2])."""
+    elements = range(trees) if elements is None else elements
+    gd, ge = [], []
+    for e in elements:
+        rng = np.random.default_rng([int(seed), int(e), 2])
+        gd.append(rng.standard_normal((n, b, b)))
+        ge.append(rng.standard_normal((n, b, b)))
+    return np.stack(gd), np.stack(ge)
+
+
 def generate(w: Workload, elements: Optional[Sequence[int]] = None):
     """Host (NumPy) inputs of a workload, or of a subset of its batch elements."""
     if w.kind == "chain":

@@ -69,6 +69,10 @@ def lib():
         L.selinv_chain_backward_workspace_size.restype = SZ
         L.selinv_chain_backward.argtypes = [ctypes.c_int, I64, I64, I32, P, P, P, P, P, P, P, P, P, P, SZ, P]
         L.selinv_chain_backward.restype = ctypes.c_int
+        L.selinv_tree_backward_workspace_size.argtypes = [P, ctypes.c_int, I32]
+        L.selinv_tree_backward_workspace_size.restype = SZ
+        L.selinv_tree_backward.argtypes = [P, ctypes.c_int, I32, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.selinv_tree_backward.restype = ctypes.c_int
         L.selinv_tree_plan.argtypes = [P, I64, I64, ctypes.POINTER(P)]
         L.selinv_tree_plan.restype = ctypes.c_int
         L.selinv_tree_plan_free.argtypes = [P]
@@ -433,6 +437,9 @@ class TreePlan:
     def workspace_size(self, dtype, b) -> int:
         return int(lib().selinv_tree_workspace_size(self._h, _code(dtype), b))
 
+    def backward_workspace_size(self, dtype, b) -> int:
+        return int(lib().selinv_tree_backward_workspace_size(self._h, _code(dtype), b))
+
     def close(self):
         if getattr(self, "_h", None) and _lib is not None:
             _lib.selinv_tree_plan_free(self._h)
@@ -489,6 +496,80 @@ def selinv_tree(plan: TreePlan, diag: torch.Tensor, edge: torch.Tensor, *, check
     if single:
         G_diag, G_edge = G_diag[0], G_edge[0]
     return {"G_diag": G_diag, "G_edge": G_edge, "logdet": logdet, "info": info}
+
+
+def tree_backward(plan: TreePlan, diag, edge, G_diag, G_edge, Gb_diag=None, Gb_edge=None, *, check=True, out=None,
+                  workspace=None, stream=None):
+    """Cotangents of selinv_tree (b <= 16): from the cotangents Gb_diag, Gb_edge
+    of its outputs G_diag, G_edge (None = zero; the root's edge slot is
+    ignored), the cotangents Db of diag (lower-triangular: only D's lower
+    triangle is read) and Eb of edge (root slot 0).  Returns a dict with Db,
+    Eb and info."""
+    _cuda_contig("diag", diag)
+    dt = diag.dtype
+    single = diag.dim() == 3
+    lift = (lambda x: None if x is None else (x[None] if single else x))
+    d4, e4, gd4, ge4 = lift(diag), lift(edge), lift(G_diag), lift(G_edge)
+    gbd4, gbe4 = lift(Gb_diag), lift(Gb_edge)
+    if d4.dim() != 4 or tuple(d4.shape[:2]) != (plan.trees, plan.n) or d4.shape[-1] != d4.shape[-2]:
+        raise ValueError(f"diag must be [{plan.trees}, {plan.n}, b, b]")
+    for name, x in (("edge", e4), ("G_diag", gd4), ("G_edge", ge4), ("Gb_diag", gbd4), ("Gb_edge", gbe4)):
+        if x is None:
+            if name in ("edge", "G_diag", "G_edge"):
+                raise ValueError(f"{name} is required")
+            continue
+        _cuda_contig(name, x, dt)
+        if x.shape != d4.shape:
+            raise ValueError(f"{name} must have diag's shape")
+    b = int(d4.shape[-1])
+    dev = diag.device
+    out = dict(out or {})
+    Db = out.get("Db")
+    if Db is None:
+        Db = torch.empty_like(d4)
+    Eb = out.get("Eb")
+    if Eb is None:
+        Eb = torch.empty_like(d4)
+    info = out.get("info")
+    if info is None:
+        info = torch.empty(plan.trees, dtype=torch.int32, device=dev)
+    nbytes = plan.backward_workspace_size(dt, b)
+    ws = _workspace(nbytes, dev, workspace)
+    with torch.cuda.device(dev):
+        st = lib().selinv_tree_backward(plan.handle, _code(dt), b, _ptr(d4), _ptr(e4), _ptr(gd4), _ptr(ge4),
+                                        _ptr(gbd4), _ptr(gbe4), _ptr(Db), _ptr(Eb), _ptr(info), _ptr(ws), nbytes,
+                                        _stream_handle(stream))
+    _check(st, "selinv_tree_backward")
+    _raise_on_info(info, check)
+    if single:
+        Db, Eb = Db[0], Eb[0]
+    return {"Db": Db, "Eb": Eb, "info": info}
+
+
+class _SelinvTreeFn(torch.autograd.Function):
+    """G_diag, G_edge = selinv_tree(plan, diag, edge) with its analytic backward."""
+
+    @staticmethod
+    def forward(ctx, diag, edge, plan):
+        out = selinv_tree(plan, diag, edge)
+        ctx.plan = plan
+        ctx.save_for_backward(diag, edge, out["G_diag"], out["G_edge"])
+        return out["G_diag"], out["G_edge"]
+
+    @staticmethod
+    def backward(ctx, gb_diag, gb_edge):
+        diag, edge, G_diag, G_edge = ctx.saved_tensors
+        r = tree_backward(ctx.plan, diag, edge, G_diag, G_edge,
+                          None if gb_diag is None else gb_diag.contiguous(),
+                          None if gb_edge is None else gb_edge.contiguous())
+        return r["Db"], r["Eb"], None
+
+
+def selinv_tree_ad(plan: TreePlan, diag, edge):
+    """Differentiable selected inverse of block trees (b <= 16): returns
+    (G_diag, G_edge); gradients reach diag (its lower triangle) and edge
+    through tree_backward -- the pages' selinv_tree."""
+    return _SelinvTreeFn.apply(diag, edge, plan)
 
 
 def tree_sample(plan: TreePlan, diag: torch.Tensor, edge: torch.Tensor, z: torch.Tensor, *, check=True, out=None,

@@ -147,3 +147,15 @@ def test_backward_argument_errors(lib):
     assert call(nbytes=16) == selinv.ERR_WORKSPACE
     assert call(ws=None) == selinv.ERR_WORKSPACE
     assert call(batch=0) == selinv.OK
+
+
+def test_tree_backward_argument_errors(lib):
+    """Without a GPU no plan can be built; a null plan is rejected before any launch."""
+    ws = lib.selinv_tree_backward_workspace_size
+    ws.restype = ctypes.c_size_t
+    ws.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int32]
+    assert ws(None, 0, 16) == 0
+    f = lib.selinv_tree_backward
+    # plan, dtype, b, diag, edge, G_diag, G_edge, Gb_diag, Gb_edge, Db, Eb, info, ws, ws_bytes, stream
+    assert f(None, 0, 4, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == \
+        selinv.ERR_INVALID_ARG
