@@ -54,6 +54,8 @@ def _bind(path):
     lib.oracle_chain_backward.restype = ctypes.c_int
     lib.oracle_tree_backward.argtypes = [P, I64, I64, ctypes.c_int, P, P, P, P, P, P, P]
     lib.oracle_tree_backward.restype = ctypes.c_int
+    lib.oracle_bidiag.argtypes = [P, P, I64, I64, ctypes.c_int, P, P, P]
+    lib.oracle_bidiag.restype = ctypes.c_int
     lib.oracle_threads.argtypes = []
     lib.oracle_threads.restype = ctypes.c_int
     return lib
@@ -200,6 +202,29 @@ def tree_backward(parent, diag, edge, Gb_diag, Gb_edge, lib=None):
     if rc != 0:
         raise ValueError("oracle_tree_backward: invalid arguments")
     return {"Db": Db, "Eb": Eb, "info": info}
+
+
+def bidiag(diag, lower, lib=None):
+    """Selected inverse of block lower-bidiagonal matrices (general blocks):
+    diag [..., L, b, b] = M_ii, lower [..., L-1, b, b] = M_{i+1,i}.  Returns
+    dict with G_diag = (M^-1)_ii, G_lower = (M^-1)_{i+1,i} and info [...]
+    (-1 ok, else the block of the first zero pivot).  Dense definition with
+    partial pivoting (gabp-sparse-inv, "Non-symmetric selected inverse")."""
+    diag = _f64(diag)
+    lead = diag.shape[:-3]
+    L, b = diag.shape[-3], diag.shape[-1]
+    batch = int(np.prod(lead)) if lead else 1
+    G_diag = np.empty(lead + (L, b, b))
+    G_lower = np.empty(lead + (max(L - 1, 0), b, b))
+    info = np.empty(lead, dtype=np.int32)
+    lower = _f64(lower) if L > 1 else None
+    if L > 1:
+        assert lower.shape == lead + (L - 1, b, b)
+    rc = _load(lib).oracle_bidiag(_ptr(diag), _ptr(lower), batch, L, b, _ptr(G_diag),
+                                  _ptr(G_lower) if L > 1 else None, _ptr(info))
+    if rc != 0:
+        raise ValueError("oracle_bidiag: invalid arguments")
+    return {"G_diag": G_diag, "G_lower": G_lower, "info": info}
 
 
 def tree(parent, diag, edge, lib=None):

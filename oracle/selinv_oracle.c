@@ -437,6 +437,102 @@ int oracle_chain_backward(const double *diag, const double *lower, int64_t batch
     return 0;
 }
 
+/* ---------------------------- non-symmetric ------------------------------ */
+
+/* Ainv := A^-1 for a general N x N matrix by Gauss-Jordan elimination with
+ * partial pivoting (row exchanges on the augmented [A | I]).  Returns -1, or
+ * the first column whose pivot is zero or not finite (A singular). */
+static int general_inverse(int N, const double *A, double *Ainv)
+{
+    const size_t W = 2 * (size_t)N;
+    double *aug = malloc(sizeof(double) * (size_t)N * W);
+    int fail = -1;
+    for (int r = 0; r < N; ++r)
+        for (int c = 0; c < N; ++c) {
+            aug[r * W + c] = A[(size_t)r * N + c];
+            aug[r * W + N + c] = (r == c) ? 1.0 : 0.0;
+        }
+    for (int k = 0; k < N; ++k) {
+        int piv = k;
+        for (int r = k + 1; r < N; ++r)
+            if (fabs(aug[r * W + k]) > fabs(aug[piv * W + k])) piv = r;
+        const double d = aug[piv * W + k];
+        if (!(fabs(d) > 0.0) || !isfinite(d)) { fail = k; break; }
+        if (piv != k)
+            for (size_t c = 0; c < W; ++c) {
+                const double tmp = aug[k * W + c];
+                aug[k * W + c] = aug[piv * W + c];
+                aug[piv * W + c] = tmp;
+            }
+        for (size_t c = 0; c < W; ++c) aug[k * W + c] /= d;
+        for (int r = 0; r < N; ++r) {
+            if (r == k) continue;
+            const double f = aug[r * W + k];
+            if (f != 0.0)
+                for (size_t c = 0; c < W; ++c) aug[r * W + c] -= f * aug[k * W + c];
+        }
+    }
+    if (fail < 0)
+        for (int r = 0; r < N; ++r)
+            for (int c = 0; c < N; ++c) Ainv[(size_t)r * N + c] = aug[r * W + N + c];
+    free(aug);
+    return fail;
+}
+
+/*
+ * Selected inverse of a block lower-bidiagonal matrix M (general blocks, no
+ * symmetry): gabp-sparse-inv 0.3.2, "Implemented and tested kernels" ->
+ * Non-symmetric chain and "Non-symmetric selected inverse": G_ii and G_{i+1,i}
+ * on M's pattern.  Written from the definition: the dense M^-1 (Gauss-Jordan
+ * with partial pivoting) and its blocks (i, i) and (i+1, i).  M is block
+ * lower triangular, so det M = prod det M_ii: info = -1, or the first block
+ * i whose M_ii meets a zero pivot in its own pivoted elimination (M is then
+ * singular and nothing is written).
+ */
+static int bidiag_one(int64_t L, int b, const double *diag, const double *lower, double *G_diag,
+                      double *G_lower)
+{
+    const size_t bb = (size_t)b * b;
+    const int N = (int)(L * b);
+    const size_t NN = (size_t)N * N;
+    double *M = calloc(NN, sizeof(double)), *Mi = malloc(NN * sizeof(double));
+    int info = -1;
+    for (int64_t i = 0; i < L; ++i)
+        for (int r = 0; r < b; ++r)
+            for (int c = 0; c < b; ++c) {
+                const size_t row = (size_t)(i * b + r), col = (size_t)(i * b + c);
+                M[row * N + col] = diag[bb * i + r * b + c];
+                if (i + 1 < L) M[(row + b) * N + col] = lower[bb * i + r * b + c];   /* M_{i+1,i} */
+            }
+    for (int64_t i = 0; i < L; ++i)
+        if (general_inverse(b, diag + bb * i, Mi) >= 0) { info = (int)i; goto done; }
+    if (general_inverse(N, M, Mi) >= 0) { info = 0; goto done; }   /* not reached: det M != 0 */
+    for (int64_t i = 0; i < L; ++i)
+        for (int r = 0; r < b; ++r)
+            for (int c = 0; c < b; ++c) {
+                const size_t row = (size_t)(i * b + r), col = (size_t)(i * b + c);
+                G_diag[bb * i + r * b + c] = Mi[row * N + col];
+                if (i + 1 < L) G_lower[bb * i + r * b + c] = Mi[(row + b) * N + col];
+            }
+done:
+    free(M); free(Mi);
+    return info;
+}
+
+/* Batched: diag [batch,L,b,b], lower [batch,L-1,b,b] -> G_diag, G_lower; info [batch]. */
+int oracle_bidiag(const double *diag, const double *lower, int64_t batch, int64_t L, int b, double *G_diag,
+                  double *G_lower, int32_t *info)
+{
+    if (batch < 0 || L < 1 || b < 1 || !diag || !G_diag || !info) return 1;
+    if (L > 1 && (!lower || !G_lower)) return 1;
+    const size_t bb = (size_t)b * b;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t e = 0; e < batch; ++e)
+        info[e] = bidiag_one(L, b, diag + bb * L * e, L > 1 ? lower + bb * (L - 1) * e : NULL,
+                             G_diag + bb * L * e, L > 1 ? G_lower + bb * (L - 1) * e : NULL);
+    return 0;
+}
+
 /* -------------------------------- tree ---------------------------------- */
 
 /* One rooted tree (parent[root] = -1).  Collect in reverse breadth-first

@@ -231,6 +231,21 @@ def standard_normals(batch: int, L: int, b: int, seed: int, elements: Optional[S
     return np.stack([np.random.default_rng([int(seed), int(e), 1]).standard_normal((L, b)) for e in elements])
 
 
+def bidiag_inputs(batch: int, L: int, b: int, seed: int, load: float,
+                  elements: Optional[Sequence[int]] = None):
+    """Block lower-bidiagonal matrices with general blocks: M_ii = C_i / sqrt(b)
+    + load I and M_{i+1,i} = B_i / sqrt(b), C_i and B_i standard normal (the
+    pages' random_nonsym_bidiag shape with its diag_load); element e draws from
+    default_rng([seed, e, 3])."""
+    elements = range(batch) if elements is None else elements
+    diag, lower = [], []
+    for e in elements:
+        rng = np.random.default_rng([int(seed), int(e), 3])
+        lower.append(rng.standard_normal((L - 1, b, b)) / math.sqrt(b))
+        diag.append(rng.standard_normal((L, b, b)) / math.sqrt(b) + load * np.eye(b))
+    return np.stack(diag), np.stack(lower)
+
+
 def cotangents(batch: int, L: int, b: int, seed: int, elements: Optional[Sequence[int]] = None):
     """Standard-normal cotangents (Gb_diag [n, L, b, b], Gb_lower [n, L-1, b, b])
     of a loss on a chain's selected inverse: element e draws from

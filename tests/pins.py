@@ -542,6 +542,63 @@ def pin_tree_backward_path_is_chain(lib=None):
                float(np.abs(out["Eb"][:, L - 1]).max()))
 
 
+def _bidiag_dense(d, l):
+    L, b = d.shape[0], d.shape[-1]
+    M = np.zeros((L * b, L * b))
+    for i in range(L):
+        M[i * b:(i + 1) * b, i * b:(i + 1) * b] = d[i]
+    for i in range(L - 1):
+        M[(i + 1) * b:(i + 2) * b, i * b:(i + 1) * b] = l[i]
+    return M
+
+
+def pin_bidiag_dense(lib=None):
+    """Non-symmetric chain blocks against numpy's inverse of the dense M, and
+    against the pages' block formula G_{i+1,i} = -M_{i+1,i+1}^-1 M_{i+1,i} M_ii^-1;
+    blocks with a zero diagonal force row exchanges."""
+    worst = 0.0
+    cases = [inputs.bidiag_inputs(2, 6, 3, seed=51, load=2.0), inputs.bidiag_inputs(1, 1, 4, seed=52, load=2.0)]
+    d, l = inputs.bidiag_inputs(1, 4, 2, seed=53, load=0.0)
+    d[0, :] = np.array([[0.0, 1.5], [-2.0, 0.3]])           # zero pivot in column 0 without exchanges
+    cases.append((d, l))
+    for d, l in cases:
+        out = oracle.bidiag(d, l, lib=lib)
+        if (out["info"] != -1).any():
+            return float("inf")
+        L, b = d.shape[1], d.shape[-1]
+        for e in range(d.shape[0]):
+            inv = np.linalg.inv(_bidiag_dense(d[e], l[e]))
+            for i in range(L):
+                worst = max(worst, rel(out["G_diag"][e, i], blk(inv, i, i, b)))
+            for i in range(L - 1):
+                worst = max(worst, rel(out["G_lower"][e, i], blk(inv, i + 1, i, b)))
+                formula = -np.linalg.inv(d[e, i + 1]) @ l[e, i] @ np.linalg.inv(d[e, i])
+                worst = max(worst, rel(out["G_lower"][e, i], formula))
+    return worst
+
+
+def pin_bidiag_scalar_exact(lib=None):
+    """b = 1 in exact rationals: G_ii = 1/m_i, G_{i+1,i} = -l_i / (m_i m_{i+1})."""
+    m = [Fraction(3), Fraction(-2), Fraction(5, 2), Fraction(7)]
+    lo = [Fraction(1), Fraction(-4), Fraction(3, 2)]
+    out = oracle.bidiag(np.array([[[[float(x)]] for x in m]]), np.array([[[[float(x)]] for x in lo]]), lib=lib)
+    worst = 0.0
+    for i, x in enumerate(m):
+        worst = max(worst, abs(out["G_diag"][0, i, 0, 0] - float(1 / x)) / abs(float(1 / x)))
+    for i, x in enumerate(lo):
+        ref = float(-x / (m[i] * m[i + 1]))
+        worst = max(worst, abs(out["G_lower"][0, i, 0, 0] - ref) / abs(ref))
+    return worst
+
+
+def pin_bidiag_singular(lib=None):
+    """A singular diagonal block is reported as that block; others are fine."""
+    d, l = inputs.bidiag_inputs(2, 5, 3, seed=54, load=2.0)
+    d[1, 3] = np.array([[1.0, 2.0, 3.0], [2.0, 4.0, 6.0], [0.5, -1.0, 2.0]])   # rank 2
+    out = oracle.bidiag(d, l, lib=lib)
+    return 0.0 if (out["info"][0] == -1 and out["info"][1] == 3) else float("inf")
+
+
 # name -> (function, tolerance)
 PINS = {
     "tiny_chains_dense": (pin_tiny_chains_dense, 1e-12),
@@ -563,4 +620,7 @@ PINS = {
     "backward_trace": (pin_backward_trace, 1e-11),
     "tree_backward_finite_differences": (pin_tree_backward_finite_differences, 1e-7),
     "tree_backward_path_is_chain": (pin_tree_backward_path_is_chain, 1e-12),
+    "bidiag_dense": (pin_bidiag_dense, 1e-12),
+    "bidiag_scalar_exact": (pin_bidiag_scalar_exact, 1e-15),
+    "bidiag_singular": (pin_bidiag_singular, 0.5),
 }

@@ -70,6 +70,13 @@ MUTANTS = {
                                                    "Gbar[vr * N + (size_t)(p * b + c)] = Gb_edge[bb * v + r * b + c];"),
     "tree_backward_db_mirror_dropped": ("Db[bb * v + r * b + c] = c < r ? lo + up : (c == r ? lo : 0.0);",
                                         "Db[bb * v + r * b + c] = c < r ? lo : (c == r ? lo : 0.0);"),
+    "bidiag_pivot_smallest": ("if (fabs(aug[r * W + k]) > fabs(aug[piv * W + k])) piv = r;",
+                              "if (fabs(aug[r * W + k]) < fabs(aug[piv * W + k])) piv = r;"),
+    "bidiag_no_row_exchange": ("if (piv != k)\n", "if (piv != k && 0)\n"),
+    "bidiag_lower_transposed": ("if (i + 1 < L) M[(row + b) * N + col] = lower[bb * i + r * b + c];",
+                                "if (i + 1 < L) M[(row + b) * N + col] = lower[bb * i + c * b + r];"),
+    "bidiag_lower_above": ("if (i + 1 < L) G_lower[bb * i + r * b + c] = Mi[(row + b) * N + col];",
+                           "if (i + 1 < L) G_lower[bb * i + r * b + c] = Mi[row * N + col + b];"),
     "tree_g_diag_transposed": ("matmul(b, Sinv + bb * v, 0, edge + bb * v, 1, T1);",
                                "matmul(b, Sinv + bb * v, 0, edge + bb * v, 0, T1);"),
 }
