@@ -48,6 +48,7 @@ KERNEL_SOURCES = {
     "tree_collect_kernel": ["tree.cu", "warp16.cuh", "common.cuh"],
     "chain_backward_kernel": ["chain_backward.cu", "warp16.cuh", "common.cuh"],
     "tree_bw_collect_kernel": ["tree.cu", "warp16.cuh", "common.cuh"],
+    "bidiag_kernel": ["bidiag.cu", "common.cuh"],
 }
 
 
@@ -62,11 +63,12 @@ def parse():
     ap.add_argument("--length", type=int, default=None,
                     help="override the chain length / tree size (profiling runs of a smaller case)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--op", default="selinv", choices=["selinv", "sample", "backward"],
+    ap.add_argument("--op", default="selinv", choices=["selinv", "sample", "backward", "bidiag"],
                     help="selinv: selected inverse + log det (+ solve); sample: Gaussian draw "
                          "eta = A^-1 r + L^-T z + log det (chains; on trees eta = L^-T z); backward: "
                          "cotangents of diag and lower (edge) from those of G_diag and G_lower (G_edge); "
-                         "chains and trees, b <= 16")
+                         "chains and trees, b <= 16; bidiag: the selected inverse of a block "
+                         "lower-bidiagonal matrix with general blocks of the chain workload's shape (b <= 16)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -161,6 +163,8 @@ def oracle_inputs(w, elems, op):
     g = inputs.generate(w, elements=elems)
     if op == "sample":
         g["z"] = inputs.standard_normals(w.batch, w.L, w.b, w.seed, elems)
+    if op == "bidiag":
+        g = dict(zip(("diag", "lower"), inputs.bidiag_inputs(w.batch, w.L, w.b, w.seed, 2.0, elems)))
     if op == "backward" and w.kind == "tree":
         g["Gb_diag"], g["Gb_edge"] = inputs.tree_cotangents(w.batch, w.L, w.b, w.seed, elems)
     elif op == "backward":
@@ -179,6 +183,8 @@ def oracle_run(oracle, w, g, op):
         oracle.chain_sample(g["diag"], g["lower"], g["z"], rhs=g.get("rhs"))
     elif op == "backward":
         oracle.chain_backward(g["diag"], g["lower"], g["Gb_diag"], g["Gb_lower"])
+    elif op == "bidiag":
+        oracle.bidiag(g["diag"], g["lower"])
     else:
         oracle.chain(g["diag"], g["lower"], g.get("rhs"))
 
@@ -187,7 +193,7 @@ def oracle_workload(w, op):
     """The workload the oracle times: the same, except for the backward, whose
     dense definition costs O((L b)^3) per chain or tree: there chains or trees
     of 512 / b blocks drawn by the same recipe stand in (a few seconds each)."""
-    if op == "backward" and w.L * w.b > 512:
+    if op in ("backward", "bidiag") and w.L * w.b > 512:
         n = max(2, 512 // w.b)
         what = "trees" if w.kind == "tree" else "chains"
         return dataclasses.replace(w, L=n), f" ({what} of {n} blocks drawn like {w.name}'s)"
@@ -227,6 +233,10 @@ def algorithmic_bytes(w, es, batch, op="selinv"):
     (or G_edge) blocks, plus the right-hand side and solution when solving.  A draw reads
     D, B, r and z and writes eta (a tree draw has no r)."""
     b2 = w.b * w.b
+    if op == "bidiag":
+        # read M_ii and M_{i+1,i}, write G_ii and G_{i+1,i}
+        nodes, edges = batch * w.L, batch * (w.L - 1)
+        return es * 2 * b2 * (nodes + edges)
     if op == "backward":
         # read D, G_diag, Gb_diag and B (edge), G_lower (G_edge), Gb_lower (Gb_edge); write Db and Bb (Eb)
         nodes, edges = batch * w.L, batch * (w.L - 1)
@@ -315,7 +325,7 @@ def run_reference(args):
     n_per_step = {"chain": 64, "tree": 1, "grid": 1}[w.kind]
     if w.kind == "chain" and w.L * w.b ** 3 > 64 * 16 ** 3 * 64:
         n_per_step = 2
-    if args.op == "backward" and w.kind == "chain":
+    if args.op in ("backward", "bidiag") and w.kind == "chain":
         n_per_step = 16
     elems = list(range(min(n_per_step, w.batch)))
     g = oracle_inputs(w, elems, args.op)
@@ -343,7 +353,7 @@ def run_reference(args):
 
 
 def metric_name(op, dtype):
-    what = {"sample": "draw", "backward": "selinv backward"}.get(op, "selinv")
+    what = {"sample": "draw", "backward": "selinv backward", "bidiag": "bidiag selinv"}.get(op, "selinv")
     return f"{what} blocks/s ({'fp64' if dtype == 'f64' else 'fp32'})"
 
 
@@ -386,6 +396,10 @@ def run_ours(args):
                 tdt).pin_memory()
     else:
         g = inputs.generate(w, elements=elems)   # per-element seeds: rank r owns its own slice
+        if args.op == "bidiag":
+            if w.kind != "chain" or w.b > 16:
+                raise SystemExit("--op bidiag runs on chain workload shapes with b <= 16")
+            g = dict(zip(("diag", "lower"), inputs.bidiag_inputs(w.batch, w.L, w.b, w.seed, 2.0, elems)))
         if args.op == "sample":
             if w.b > 16 and args.dtype != "f64":
                 raise SystemExit("--op sample with b > 16 runs in float64 only")
@@ -455,7 +469,11 @@ def run_ours(args):
                          dtype=torch.uint8, device="cuda")
         launches_per_step = 1
         segments = selinv.chain_segments(batch, L, b, True, "rhs" in dev_in)
-        if args.op == "backward":
+        if args.op == "bidiag":
+            kernel = "bidiag_kernel"
+            out = {"G_diag": torch.empty_like(dev_in["diag"]), "G_lower": torch.empty_like(dev_in["lower"]),
+                   "info": torch.empty(batch, dtype=torch.int32, device="cuda")}
+        elif args.op == "backward":
             # the forward's outputs are the backward's inputs (computed once, outside the timing)
             fwd = selinv.selinv_chain(dev_in["diag"], dev_in["lower"])
             for k in ("G_diag", "G_lower"):
@@ -484,7 +502,10 @@ def run_ours(args):
         else:
             kernel = "chain_large_kernel"
 
-        if args.op == "backward":
+        if args.op == "bidiag":
+            def step():
+                selinv.bidiag(dev_in["diag"], dev_in["lower"], check=False, out=out)
+        elif args.op == "backward":
             def step():
                 selinv.chain_backward(dev_in["diag"], dev_in["lower"], dev_in["G_diag"], dev_in["G_lower"],
                                       dev_in["Gb_diag"], dev_in["Gb_lower"], check=False, out=out, workspace=ws)

@@ -179,6 +179,24 @@ selinv_status selinv_chain_sample(selinv_dtype dtype, int64_t batch, int64_t L, 
                                   void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Selected inverse of block lower-bidiagonal matrices with general
+ * (non-symmetric) blocks, b <= 16: gabp-sparse-inv 0.3.2, "Implemented and
+ * tested kernels" -> Non-symmetric chain:
+ *   G_ii = M_ii^-1,   G_{i+1,i} = -M_{i+1,i+1}^-1 M_{i+1,i} M_ii^-1,
+ * the blocks of M^-1 on M's pattern.
+ *   diag  [batch, L, b, b]    M_ii, read in full (no symmetry assumed)
+ *   lower [batch, L-1, b, b]  M_{i+1,i} (NULL when L = 1)
+ *   G_diag, G_lower           outputs, same shapes
+ *   info [batch]              -1, or the first block i whose M_ii is singular
+ *                             (a zero or non-finite pivot under partial
+ *                             pivoting; that chain's outputs are then
+ *                             unspecified)
+ * No workspace.  b > 16 returns SELINV_ERR_UNSUPPORTED.
+ */
+selinv_status selinv_bidiag(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b, const void *diag,
+                            const void *lower, void *G_diag, void *G_lower, int32_t *info, void *stream);
+
+/*
  * Cotangents of the chain selected inverse (b <= 16): given the cotangents
  * Gb_diag [batch, L, b, b] and Gb_lower [batch, L-1, b, b] of a loss with
  * respect to selinv_chain's outputs G_diag and G_lower, writes the

@@ -191,6 +191,28 @@ selinv_status selinv_chain_sample(selinv_dtype dtype, int64_t batch, int64_t L, 
     return from_cuda(chain_small_sample_launch<float>(a, al, s));
 }
 
+selinv_status selinv_bidiag(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b, const void *diag,
+                            const void *lower, void *G_diag, void *G_lower, int32_t *info, void *stream)
+{
+    selinv_status st = chain_check(dtype, batch, L, b, diag, lower, info);
+    if (st != SELINV_OK) return st;
+    if (b > 16) return SELINV_ERR_UNSUPPORTED;
+    const size_t es = elem_size(dtype);
+    if (batch > 0 && (!G_diag || (L > 1 && !G_lower))) return SELINV_ERR_INVALID_ARG;
+    if (!aligned(G_diag, es) || !aligned(G_lower, es)) return SELINV_ERR_INVALID_ARG;
+    if (batch == 0) return SELINV_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool al = aligned(diag, 16) && aligned(lower, 16) && aligned(G_diag, 16) && aligned(G_lower, 16);
+    if (dtype == SELINV_F64) {
+        BidiagArgs<double> p{static_cast<const double *>(diag), static_cast<const double *>(lower),
+                             static_cast<double *>(G_diag), static_cast<double *>(G_lower), info, batch, L, b};
+        return from_cuda(bidiag_launch<double>(p, al, s));
+    }
+    BidiagArgs<float> p{static_cast<const float *>(diag), static_cast<const float *>(lower),
+                        static_cast<float *>(G_diag), static_cast<float *>(G_lower), info, batch, L, b};
+    return from_cuda(bidiag_launch<float>(p, al, s));
+}
+
 size_t selinv_chain_backward_workspace_size(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b)
 {
     if (!valid_dtype(dtype) || batch < 0 || L < 1 || b < 1 || b > 16) return 0;

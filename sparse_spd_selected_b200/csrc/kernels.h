@@ -67,4 +67,15 @@ template <class T> struct ChainBwdArgs {
 size_t chain_backward_workspace(size_t elem, int64_t batch, int64_t L);
 template <class T> cudaError_t chain_backward_launch(const ChainBwdArgs<T> &a, bool aligned16, cudaStream_t s);
 
+// Block lower-bidiagonal matrices with general blocks (b <= 16).
+template <class T> struct BidiagArgs {
+    const T *diag, *lower;          // M_ii [batch, L, b, b], M_{i+1,i} [batch, L-1, b, b]
+    T *G_diag, *G_lower;            // (M^-1)_ii, (M^-1)_{i+1,i}
+    int32_t *info;                  // [batch]
+    int64_t batch;
+    int64_t L;
+    int b;
+};
+template <class T> cudaError_t bidiag_launch(const BidiagArgs<T> &p, bool aligned16, cudaStream_t s);
+
 }  // namespace selinv

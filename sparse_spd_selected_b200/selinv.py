@@ -40,6 +40,14 @@ class NotSPDError(SelinvError):
         super().__init__(ERR_NOT_SPD, f"first failing block per batch element: {info}")
 
 
+class SingularBlockError(SelinvError):
+    """A diagonal block of a non-symmetric chain is singular."""
+
+    def __init__(self, info):
+        self.info = info
+        super().__init__(ERR_NOT_SPD, f"first singular diagonal block per batch element: {info}")
+
+
 def lib():
     """The loaded libselinv.so (raises if it has not been built)."""
     global _lib
@@ -65,6 +73,8 @@ def lib():
         L.selinv_chain_sample.restype = ctypes.c_int
         L.chain_solve.argtypes = [ctypes.c_int, I64, I64, I32, P, P, P, P, P, P, P, SZ, P]
         L.chain_solve.restype = ctypes.c_int
+        L.selinv_bidiag.argtypes = [ctypes.c_int, I64, I64, I32, P, P, P, P, P, P]
+        L.selinv_bidiag.restype = ctypes.c_int
         L.selinv_chain_backward_workspace_size.argtypes = [ctypes.c_int, I64, I64, I32]
         L.selinv_chain_backward_workspace_size.restype = SZ
         L.selinv_chain_backward.argtypes = [ctypes.c_int, I64, I64, I32, P, P, P, P, P, P, P, P, P, P, SZ, P]
@@ -320,6 +330,50 @@ def chain_sample(diag, lower, z, rhs=None, *, check=True, out=None, workspace=No
     _check(st, "selinv_chain_sample")
     _raise_on_info(info, check)
     return {"eta": eta, "logdet": logdet, "info": info}
+
+
+def bidiag(diag, lower=None, *, check=True, out=None, stream=None):
+    """Selected inverse of block lower-bidiagonal matrices with general blocks
+    (b <= 16): diag [..., L, b, b] = M_ii, lower [..., L-1, b, b] = M_{i+1,i}.
+    Returns a dict with G_diag = (M^-1)_ii, G_lower = (M^-1)_{i+1,i} and info
+    (int32, -1 = ok, else the first singular diagonal block)."""
+    _cuda_contig("diag", diag)
+    dt = diag.dtype
+    if diag.dim() < 3 or diag.shape[-1] != diag.shape[-2]:
+        raise ValueError("diag must be [..., L, b, b]")
+    lead = tuple(diag.shape[:-3])
+    L, b = int(diag.shape[-3]), int(diag.shape[-1])
+    batch = 1
+    for d in lead:
+        batch *= int(d)
+    if L > 1:
+        if lower is None:
+            raise ValueError("lower is required when L > 1")
+        _cuda_contig("lower", lower, dt)
+        if tuple(lower.shape) != lead + (L - 1, b, b):
+            raise ValueError(f"lower must be {lead + (L - 1, b, b)}")
+    else:
+        lower = None
+    dev = diag.device
+    out = dict(out or {})
+    G_diag = out.get("G_diag")
+    if G_diag is None:
+        G_diag = torch.empty_like(diag)
+    G_lower = out.get("G_lower")
+    if G_lower is None:
+        G_lower = torch.empty(lead + (max(L - 1, 0), b, b), dtype=dt, device=dev)
+    info = out.get("info")
+    if info is None:
+        info = torch.empty(lead, dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        st = lib().selinv_bidiag(_code(dt), batch, L, b, _ptr(diag), _ptr(lower), _ptr(G_diag),
+                                 _ptr(G_lower if L > 1 else None), _ptr(info), _stream_handle(stream))
+    _check(st, "selinv_bidiag")
+    if check:
+        host = info.cpu()
+        if bool((host >= 0).any()):
+            raise SingularBlockError(host.tolist())
+    return {"G_diag": G_diag, "G_lower": G_lower, "info": info}
 
 
 def chain_backward_workspace_size(dtype, batch, L, b) -> int:

@@ -159,3 +159,13 @@ def test_tree_backward_argument_errors(lib):
     # plan, dtype, b, diag, edge, G_diag, G_edge, Gb_diag, Gb_edge, Db, Eb, info, ws, ws_bytes, stream
     assert f(None, 0, 4, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == \
         selinv.ERR_INVALID_ARG
+
+
+def test_bidiag_argument_errors(lib):
+    f = lib.selinv_bidiag
+    # dtype, batch, L, b, diag, lower, G_diag, G_lower, info, stream
+    assert f(0, 1, 4, 17, FAKE, FAKE, FAKE, FAKE, FAKE, None) == selinv.ERR_UNSUPPORTED
+    assert f(0, 1, 4, 4, FAKE, None, FAKE, FAKE, FAKE, None) == selinv.ERR_INVALID_ARG
+    assert f(0, 1, 4, 4, FAKE, FAKE, None, FAKE, FAKE, None) == selinv.ERR_INVALID_ARG
+    assert f(0, 1, 4, 4, FAKE, FAKE, FAKE, None, FAKE, None) == selinv.ERR_INVALID_ARG
+    assert f(0, 0, 4, 4, FAKE, FAKE, FAKE, FAKE, FAKE, None) == selinv.OK
