@@ -56,6 +56,8 @@ def _bind(path):
     lib.oracle_tree_backward.restype = ctypes.c_int
     lib.oracle_bidiag.argtypes = [P, P, I64, I64, ctypes.c_int, P, P, P]
     lib.oracle_bidiag.restype = ctypes.c_int
+    lib.oracle_bidiag_backward.argtypes = [P, P, I64, I64, ctypes.c_int, P, P, P, P, P]
+    lib.oracle_bidiag_backward.restype = ctypes.c_int
     lib.oracle_threads.argtypes = []
     lib.oracle_threads.restype = ctypes.c_int
     return lib
@@ -225,6 +227,30 @@ def bidiag(diag, lower, lib=None):
     if rc != 0:
         raise ValueError("oracle_bidiag: invalid arguments")
     return {"G_diag": G_diag, "G_lower": G_lower, "info": info}
+
+
+def bidiag_backward(diag, lower, Gb_diag, Gb_lower, lib=None):
+    """Cotangents of the non-symmetric chain: from Gb_diag, Gb_lower (cotangents
+    of G_diag, G_lower) returns dict with Mb_diag, Mb_lower and info.  Dense
+    definition Mb = -G^T Gbar G^T (gabp-sparse-inv, selinv_bidiag's backward)."""
+    diag = _f64(diag)
+    lead = diag.shape[:-3]
+    L, b = diag.shape[-3], diag.shape[-1]
+    batch = int(np.prod(lead)) if lead else 1
+    Gb_diag = _f64(Gb_diag)
+    assert Gb_diag.shape == diag.shape
+    Mb_diag = np.empty(lead + (L, b, b))
+    Mb_lower = np.empty(lead + (max(L - 1, 0), b, b))
+    info = np.empty(lead, dtype=np.int32)
+    lower_ = Gb_l = None
+    if L > 1:
+        lower_, Gb_l = _f64(lower), _f64(Gb_lower)
+        assert lower_.shape == lead + (L - 1, b, b) and Gb_l.shape == lower_.shape
+    rc = _load(lib).oracle_bidiag_backward(_ptr(diag), _ptr(lower_), batch, L, b, _ptr(Gb_diag), _ptr(Gb_l),
+                                           _ptr(Mb_diag), _ptr(Mb_lower) if L > 1 else None, _ptr(info))
+    if rc != 0:
+        raise ValueError("oracle_bidiag_backward: invalid arguments")
+    return {"Mb_diag": Mb_diag, "Mb_lower": Mb_lower, "info": info}
 
 
 def tree(parent, diag, edge, lib=None):

@@ -533,6 +533,69 @@ int oracle_bidiag(const double *diag, const double *lower, int64_t batch, int64_
     return 0;
 }
 
+/*
+ * Cotangents of the non-symmetric chain (gabp-sparse-inv: selinv_bidiag's
+ * hand-written analytic backward).  From the definition: G = M^-1 gives
+ * dG = -G dM G, so Mb = -G^T Gbar G^T (dense), with Gbar holding Gb_ii at
+ * (i, i) and Gb_{i+1,i} at (i+1, i); every entry of M_ii and M_{i+1,i} is
+ * an independent input, so Mb_ii and Mb_{i+1,i} are just those blocks of Mb.
+ * Returns info like bidiag_one.
+ */
+static int bidiag_backward_one(int64_t L, int b, const double *diag, const double *lower,
+                               const double *Gb_diag, const double *Gb_lower, double *Mb_diag,
+                               double *Mb_lower)
+{
+    const size_t bb = (size_t)b * b;
+    const int N = (int)(L * b);
+    const size_t NN = (size_t)N * N;
+    double *M = calloc(NN, sizeof(double)), *Mi = malloc(NN * sizeof(double));
+    double *Gbar = calloc(NN, sizeof(double)), *T = malloc(NN * sizeof(double));
+    double *Mb = malloc(NN * sizeof(double));
+    int info = -1;
+    for (int64_t i = 0; i < L; ++i)
+        for (int r = 0; r < b; ++r)
+            for (int c = 0; c < b; ++c) {
+                const size_t row = (size_t)(i * b + r), col = (size_t)(i * b + c);
+                const size_t k = bb * i + (size_t)r * b + c;       /* entry (r, c) of block i */
+                M[row * N + col] = diag[k];
+                Gbar[row * N + col] = Gb_diag[k];
+                if (i + 1 < L) {
+                    M[(row + b) * N + col] = lower[k];
+                    Gbar[(row + b) * N + col] = Gb_lower[k];
+                }
+            }
+    for (int64_t i = 0; i < L; ++i)
+        if (general_inverse(b, diag + bb * i, Mi) >= 0) { info = (int)i; goto done; }
+    if (general_inverse(N, M, Mi) >= 0) { info = 0; goto done; }
+    matmul(N, Mi, 1, Gbar, 0, T);                    /* G^T Gbar */
+    matmul(N, T, 0, Mi, 1, Mb);                      /* G^T Gbar G^T */
+    for (int64_t i = 0; i < L; ++i)
+        for (int r = 0; r < b; ++r)
+            for (int c = 0; c < b; ++c) {
+                const size_t row = (size_t)(i * b + r), col = (size_t)(i * b + c);
+                Mb_diag[bb * i + r * b + c] = -Mb[row * N + col];
+                if (i + 1 < L) Mb_lower[bb * i + r * b + c] = -Mb[(row + b) * N + col];
+            }
+done:
+    free(M); free(Mi); free(Gbar); free(T); free(Mb);
+    return info;
+}
+
+int oracle_bidiag_backward(const double *diag, const double *lower, int64_t batch, int64_t L, int b,
+                           const double *Gb_diag, const double *Gb_lower, double *Mb_diag, double *Mb_lower,
+                           int32_t *info)
+{
+    if (batch < 0 || L < 1 || b < 1 || !diag || !Gb_diag || !Mb_diag || !info) return 1;
+    if (L > 1 && (!lower || !Gb_lower || !Mb_lower)) return 1;
+    const size_t bb = (size_t)b * b;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t e = 0; e < batch; ++e)
+        info[e] = bidiag_backward_one(L, b, diag + bb * L * e, L > 1 ? lower + bb * (L - 1) * e : NULL,
+                                      Gb_diag + bb * L * e, L > 1 ? Gb_lower + bb * (L - 1) * e : NULL,
+                                      Mb_diag + bb * L * e, L > 1 ? Mb_lower + bb * (L - 1) * e : NULL);
+    return 0;
+}
+
 /* -------------------------------- tree ---------------------------------- */
 
 /* One rooted tree (parent[root] = -1).  Collect in reverse breadth-first

@@ -599,6 +599,61 @@ def pin_bidiag_singular(lib=None):
     return 0.0 if (out["info"][0] == -1 and out["info"][1] == 3) else float("inf")
 
 
+def pin_bidiag_backward_finite_differences(lib=None):
+    """Non-symmetric chain cotangents against central differences of the
+    (pinned) forward oracle, every entry of M_ii and M_{i+1,i}."""
+    worst = 0.0
+    for L, b, seed in [(3, 2, 61), (2, 3, 62), (1, 2, 63)]:
+        d, l = inputs.bidiag_inputs(1, L, b, seed=seed, load=2.0)
+        rng = np.random.default_rng(seed)
+        gd, gl = rng.standard_normal(d.shape), rng.standard_normal(l.shape)
+        out = oracle.bidiag_backward(d, l, gd, gl, lib=lib)
+        if (out["info"] != -1).any():
+            return float("inf")
+
+        def loss(dd, ll):
+            o = oracle.bidiag(dd, ll, lib=lib)
+            return float((o["G_diag"] * gd).sum() + (o["G_lower"] * gl).sum())
+
+        h = 1e-5
+        scale = max(1.0, float(np.abs(out["Mb_diag"]).max()))
+        for idx in np.ndindex(*d.shape):
+            dp, dm = d.copy(), d.copy()
+            dp[idx] += h
+            dm[idx] -= h
+            worst = max(worst, abs((loss(dp, l) - loss(dm, l)) / (2 * h) - out["Mb_diag"][idx]) / scale)
+        for idx in np.ndindex(*l.shape):
+            lp, lm = l.copy(), l.copy()
+            lp[idx] += h
+            lm[idx] -= h
+            worst = max(worst, abs((loss(d, lp) - loss(d, lm)) / (2 * h) - out["Mb_lower"][idx]) / scale)
+    return worst
+
+
+def pin_bidiag_backward_scalar_exact(lib=None):
+    """b = 1 in exact rationals: with g_i = 1/m_i and h_i = -l_i g_i g_{i+1},
+    Mb_ii = -(g_i^2 Gd_i + h_i Gl_i g_i + g_i Gl_{i-1} h_{i-1}) and
+    Mb_{i+1,i} = -g_{i+1} Gl_i g_i (dG = -G dM G, written out by hand)."""
+    m = [Fraction(3), Fraction(-2), Fraction(5, 2)]
+    lo = [Fraction(1), Fraction(-4)]
+    gd = [Fraction(1, 2), Fraction(-3), Fraction(2)]
+    gl = [Fraction(5), Fraction(1, 3)]
+    g = [1 / x for x in m]
+    h = [-lo[i] * g[i] * g[i + 1] for i in range(2)]
+    out = oracle.bidiag_backward(np.array([[[[float(x)]] for x in m]]), np.array([[[[float(x)]] for x in lo]]),
+                                 np.array([[[[float(x)]] for x in gd]]), np.array([[[[float(x)]] for x in gl]]),
+                                 lib=lib)
+    worst = 0.0
+    for i in range(3):
+        ref = -(g[i] * g[i] * gd[i] + (h[i] * gl[i] * g[i] if i < 2 else 0) +
+                (g[i] * gl[i - 1] * h[i - 1] if i > 0 else 0))
+        worst = max(worst, abs(out["Mb_diag"][0, i, 0, 0] - float(ref)) / abs(float(ref)))
+    for i in range(2):
+        ref = -g[i + 1] * gl[i] * g[i]
+        worst = max(worst, abs(out["Mb_lower"][0, i, 0, 0] - float(ref)) / abs(float(ref)))
+    return worst
+
+
 # name -> (function, tolerance)
 PINS = {
     "tiny_chains_dense": (pin_tiny_chains_dense, 1e-12),
@@ -623,4 +678,6 @@ PINS = {
     "bidiag_dense": (pin_bidiag_dense, 1e-12),
     "bidiag_scalar_exact": (pin_bidiag_scalar_exact, 1e-15),
     "bidiag_singular": (pin_bidiag_singular, 0.5),
+    "bidiag_backward_finite_differences": (pin_bidiag_backward_finite_differences, 1e-7),
+    "bidiag_backward_scalar_exact": (pin_bidiag_backward_scalar_exact, 1e-14),
 }

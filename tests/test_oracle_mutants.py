@@ -77,6 +77,9 @@ MUTANTS = {
                                 "if (i + 1 < L) M[(row + b) * N + col] = lower[bb * i + c * b + r];"),
     "bidiag_lower_above": ("if (i + 1 < L) G_lower[bb * i + r * b + c] = Mi[(row + b) * N + col];",
                            "if (i + 1 < L) G_lower[bb * i + r * b + c] = Mi[row * N + col + b];"),
+    "bidiag_backward_untransposed": ("matmul(N, Mi, 1, Gbar, 0, T);", "matmul(N, Mi, 0, Gbar, 0, T);"),
+    "bidiag_backward_lower_above": ("if (i + 1 < L) Mb_lower[bb * i + r * b + c] = -Mb[(row + b) * N + col];",
+                                    "if (i + 1 < L) Mb_lower[bb * i + r * b + c] = -Mb[row * N + col + b];"),
     "tree_g_diag_transposed": ("matmul(b, Sinv + bb * v, 0, edge + bb * v, 1, T1);",
                                "matmul(b, Sinv + bb * v, 0, edge + bb * v, 0, T1);"),
 }
