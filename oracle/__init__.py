@@ -58,6 +58,8 @@ def _bind(path):
     lib.oracle_bidiag.restype = ctypes.c_int
     lib.oracle_bidiag_backward.argtypes = [P, P, I64, I64, ctypes.c_int, P, P, P, P, P]
     lib.oracle_bidiag_backward.restype = ctypes.c_int
+    lib.oracle_spd_inverse.argtypes = [P, ctypes.c_int, P, P]
+    lib.oracle_spd_inverse.restype = ctypes.c_int
     lib.oracle_threads.argtypes = []
     lib.oracle_threads.restype = ctypes.c_int
     return lib
@@ -251,6 +253,95 @@ def bidiag_backward(diag, lower, Gb_diag, Gb_lower, lib=None):
     if rc != 0:
         raise ValueError("oracle_bidiag_backward: invalid arguments")
     return {"Mb_diag": Mb_diag, "Mb_lower": Mb_lower, "info": info}
+
+
+def junction_symbolic(n, edge_index, order=None):
+    """Elimination order and filled pattern of a block graph (gabp-sparse-inv,
+    "General sparse selected inverse (junction tree)": the pattern completed to
+    its chordal fill S = pattern(L + L^T) by a min-degree elimination order).
+
+    edge_index [2, m] holds the lower blocks (i, j), i > j.  Without `order`
+    the order is greedy minimum degree on the elimination graph, ties going
+    to the smaller node index.  Eliminating v joins its remaining neighbours
+    into a clique.  Returns (order [n], S_index [2, nnz_S]) with S_index the
+    pairs (i, j), i > j, of S sorted by j, then i."""
+    ei = [int(x) for x in edge_index[0]]
+    ej = [int(x) for x in edge_index[1]]
+    adj = [set() for _ in range(n)]
+    for i, j in zip(ei, ej):
+        adj[i].add(j)
+        adj[j].add(i)
+    remaining = set(range(n))
+    seq = []
+    S = set((max(i, j), min(i, j)) for i, j in zip(ei, ej))
+    given = None if order is None else [int(v) for v in order]
+    for step in range(n):
+        if given is None:
+            v = min(remaining, key=lambda u: (len(adj[u]), u))
+        else:
+            v = given[step]
+        nb = sorted(adj[v])
+        for a in nb:                           # clique of the remaining neighbours
+            for c in nb:
+                if a < c and c not in adj[a]:
+                    adj[a].add(c)
+                    adj[c].add(a)
+                    S.add((c, a))
+        for a in nb:
+            adj[a].discard(v)
+        adj[v] = set()
+        remaining.discard(v)
+        seq.append(v)
+    Sl = sorted(S, key=lambda p: (p[1], p[0]))
+    return np.array(seq, dtype=np.int32), np.array(Sl, dtype=np.int64).T.reshape(2, -1)
+
+
+def junction(diag, edge_index, edge_val, order=None, lib=None):
+    """Selected inverse of a general block-sparse SPD matrix on its filled
+    pattern S (gabp-sparse-inv, "General sparse selected inverse"): diag
+    [..., n, b, b] (lower triangle read), edge_val [..., m, b, b] = A_{i,j} for
+    the pairs (i, j), i > j, of edge_index.  Written from the definition: the
+    dense A^-1 (textbook Cholesky) read on S.  Returns dict with G_diag,
+    S_index, G_lower [..., nnz_S, b, b] (A^-1)_{i,j}, logdet, info (-1, or
+    the node holding the first failing pivot in natural order)."""
+    diag = _f64(diag)
+    edge_val = _f64(edge_val)
+    lead = diag.shape[:-3]
+    n, b = diag.shape[-3], diag.shape[-1]
+    ei = np.asarray(edge_index[0], dtype=np.int64)
+    ej = np.asarray(edge_index[1], dtype=np.int64)
+    _, S = junction_symbolic(n, np.stack([ei, ej]), order)
+    batch = int(np.prod(lead)) if lead else 1
+    d2 = diag.reshape(batch, n, b, b)
+    e2 = edge_val.reshape(batch, len(ei), b, b)
+    G_diag = np.zeros((batch, n, b, b))
+    G_lower = np.zeros((batch, S.shape[1], b, b))
+    logdet = np.zeros(batch)
+    info = np.full(batch, -1, dtype=np.int32)
+    N = n * b
+    for e in range(batch):
+        A = np.zeros((N, N))
+        for v in range(n):
+            A[v * b:(v + 1) * b, v * b:(v + 1) * b] = np.tril(d2[e, v]) + np.tril(d2[e, v], -1).T
+        for k, (i, j) in enumerate(zip(ei, ej)):
+            A[i * b:(i + 1) * b, j * b:(j + 1) * b] = e2[e, k]
+            A[j * b:(j + 1) * b, i * b:(i + 1) * b] = e2[e, k].T
+        A = np.ascontiguousarray(A)
+        inv = np.empty((N, N))
+        ld = np.zeros(1)
+        rc = _load(lib).oracle_spd_inverse(_ptr(A), N, _ptr(inv), _ptr(ld))
+        if rc != 0:
+            info[e] = (rc - 1) // b
+            continue
+        logdet[e] = ld[0]
+        for v in range(n):
+            G_diag[e, v] = inv[v * b:(v + 1) * b, v * b:(v + 1) * b]
+        for k in range(S.shape[1]):
+            i, j = int(S[0, k]), int(S[1, k])
+            G_lower[e, k] = inv[i * b:(i + 1) * b, j * b:(j + 1) * b]
+    return {"G_diag": G_diag.reshape(lead + (n, b, b)), "S_index": S,
+            "G_lower": G_lower.reshape(lead + (S.shape[1], b, b)), "logdet": logdet.reshape(lead),
+            "info": info.reshape(lead)}
 
 
 def tree(parent, diag, edge, lib=None):

@@ -437,6 +437,34 @@ int oracle_chain_backward(const double *diag, const double *lower, int64_t batch
     return 0;
 }
 
+/* ------------------------------ dense SPD -------------------------------- */
+
+/* A^-1 and log det A of a dense SPD matrix (lower triangle read) from its
+ * textbook Cholesky factor: the definition the general sparse case is read
+ * against.  Returns 0, or 1 + the row of the first pivot that is not > 0. */
+int oracle_spd_inverse(const double *A, int N, double *Ainv, double *logdet)
+{
+    const size_t NN = (size_t)N * N;
+    double *R = malloc(NN * sizeof(double)), *Ri = malloc(NN * sizeof(double));
+    int rc = 0;
+    if (cholesky_lower(N, A, R) != 0) {
+        for (int j = 0; j < N && rc == 0; ++j) {
+            double d = A[(size_t)j * N + j];
+            for (int k = 0; k < j; ++k) d -= R[(size_t)j * N + k] * R[(size_t)j * N + k];
+            if (!(d > 0.0)) rc = 1 + j;
+        }
+        if (rc == 0) rc = 1;
+    } else {
+        double ld = 0.0;
+        for (int k = 0; k < N; ++k) ld += 2.0 * log(R[(size_t)k * N + k]);
+        *logdet = ld;
+        lower_inverse(N, R, Ri);
+        matmul(N, Ri, 1, Ri, 0, Ainv);
+    }
+    free(R); free(Ri);
+    return rc;
+}
+
 /* ---------------------------- non-symmetric ------------------------------ */
 
 /* Ainv := A^-1 for a general N x N matrix by Gauss-Jordan elimination with

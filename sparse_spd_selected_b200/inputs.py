@@ -231,6 +231,43 @@ def standard_normals(batch: int, L: int, b: int, seed: int, elements: Optional[S
     return np.stack([np.random.default_rng([int(seed), int(e), 1]).standard_normal((L, b)) for e in elements])
 
 
+def grid_edges(rows: int, cols: int) -> np.ndarray:
+    """Lower pairs (i, j), i > j, of a rows x cols 4-neighbour lattice, node r*cols + c."""
+    E = []
+    for r in range(rows):
+        for c in range(cols):
+            v = r * cols + c
+            if c + 1 < cols:
+                E.append((v + 1, v))
+            if r + 1 < rows:
+                E.append((v + cols, v))
+    return np.array(E, dtype=np.int64).T.reshape(2, -1)
+
+
+def graph_inputs(batch: int, n: int, b: int, edge_index: np.ndarray, seed: int, load: float,
+                 elements: Optional[Sequence[int]] = None):
+    """Block-sparse SPD matrices on a given pattern (the pages' random_spd_graph
+    shape): edge blocks A_{i,j} = B / sqrt(b), diagonals C C^T / b + (load +
+    delta_v) I with delta_v the sum over v's incident blocks of their largest
+    absolute row sum as they sit in block row v (strict block-row dominance,
+    hence SPD).  Element e draws from default_rng([seed, e, 4])."""
+    elements = range(batch) if elements is None else elements
+    ei, ej = np.asarray(edge_index[0]), np.asarray(edge_index[1])
+    m = ei.size
+    diag, edge = [], []
+    for e in elements:
+        rng = np.random.default_rng([int(seed), int(e), 4])
+        E = rng.standard_normal((m, b, b)) / math.sqrt(b)
+        C = rng.standard_normal((n, b, b))
+        delta = np.zeros(n)
+        absE = np.abs(E)
+        np.add.at(delta, ei, absE.sum(axis=2).max(axis=1))      # A_{i,j} in block row i
+        np.add.at(delta, ej, absE.sum(axis=1).max(axis=1))      # A_{j,i} = A_{i,j}^T in block row j
+        diag.append(np.matmul(C, np.swapaxes(C, 1, 2)) / b + (load + delta)[:, None, None] * np.eye(b))
+        edge.append(E)
+    return np.stack(diag), np.stack(edge)
+
+
 def bidiag_inputs(batch: int, L: int, b: int, seed: int, load: float,
                   elements: Optional[Sequence[int]] = None):
     """Block lower-bidiagonal matrices with general blocks: M_ii = C_i / sqrt(b)

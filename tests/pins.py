@@ -654,6 +654,84 @@ def pin_bidiag_backward_scalar_exact(lib=None):
     return worst
 
 
+def _graph_dense(n, b, ei, ej, d, e):
+    A = np.zeros((n * b, n * b))
+    for v in range(n):
+        A[v * b:(v + 1) * b, v * b:(v + 1) * b] = sym_lower(d[v])
+    for k, (i, j) in enumerate(zip(ei, ej)):
+        A[i * b:(i + 1) * b, j * b:(j + 1) * b] = e[k]
+        A[j * b:(j + 1) * b, i * b:(i + 1) * b] = e[k].T
+    return A
+
+
+def pin_junction_dense(lib=None):
+    """General sparse SPD (the pages' 3 x 3 grid with blocks of 2, a random
+    graph): every block on S against numpy's inverse, log det against slogdet,
+    and S strictly larger than the input pattern (fill)."""
+    worst = 0.0
+    rng = np.random.default_rng(71)
+    cases = [(9, 2, inputs.grid_edges(3, 3))]
+    pairs = sorted({(max(a, c), min(a, c)) for a, c in rng.integers(0, 12, (20, 2)) if a != c})
+    cases.append((12, 3, np.array(pairs).T))
+    for n, b, E in cases:
+        d, e = inputs.graph_inputs(2, n, b, E, seed=72, load=1.0)
+        out = oracle.junction(d, E, e, lib=lib)
+        if (out["info"] != -1).any() or out["S_index"].shape[1] <= E.shape[1]:
+            return float("inf")
+        for k in range(2):
+            A = _graph_dense(n, b, E[0], E[1], d[k], e[k])
+            inv = np.linalg.inv(A)
+            for v in range(n):
+                worst = max(worst, rel(out["G_diag"][k, v], blk(inv, v, v, b)))
+            for s_, (i, j) in enumerate(out["S_index"].T):
+                worst = max(worst, rel(out["G_lower"][k, s_], blk(inv, int(i), int(j), b)))
+            sl = np.linalg.slogdet(A)[1]
+            worst = max(worst, abs(out["logdet"][k] - sl) / abs(sl))
+    return worst
+
+
+def pin_junction_symbolic(lib=None):
+    """Minimum-degree elimination and fill on graphs worked by hand: the 4-cycle
+    (all degrees 2: node 0 first, joining 1 and 3: one fill block (3, 1)); a
+    star (leaves first, no fill); a path (no fill)."""
+    o, S = oracle.junction_symbolic(4, np.array([[1, 2, 3, 3], [0, 1, 2, 0]]))
+    bad = o.tolist() != [0, 1, 2, 3] or S.T.tolist() != [[1, 0], [3, 0], [2, 1], [3, 1], [3, 2]]
+    o, S = oracle.junction_symbolic(6, np.array([[1, 2, 3, 4, 5], [0, 0, 0, 0, 0]]))
+    bad |= o.tolist() != [1, 2, 3, 4, 0, 5] or S.shape[1] != 5
+    o, S = oracle.junction_symbolic(5, np.array([[1, 2, 3, 4], [0, 1, 2, 3]]))
+    bad |= o.tolist() != [0, 1, 2, 3, 4] or S.shape[1] != 4
+    return float("inf") if bad else 0.0
+
+
+def pin_junction_tree_and_order(lib=None):
+    """Zero fill on a tree: S is the input pattern and the blocks equal the
+    (pinned) tree oracle's; another elimination order changes S but not the
+    blocks of A^-1 on the input pattern."""
+    parent = np.array([-1, 0, 0, 1, 1, 2, 5, 5])
+    n, b = parent.size, 3
+    P = parent[None].astype(np.int32)
+    d, edge = inputs.tree_inputs_from_parent(P, b, seed=73, load=1.0)
+    kids = [v for v in range(n) if parent[v] >= 0]
+    E = np.array([[max(v, parent[v]) for v in kids], [min(v, parent[v]) for v in kids]])
+    # edge[v] = A_{p(v), v}; the junction input holds A_{i,j} with i > j
+    vals = np.stack([edge[0, v] if parent[v] > v else edge[0, v].T for v in kids])[None]
+    out = oracle.junction(d, E, vals, lib=lib)
+    ref = oracle.tree(P, d, edge, lib=lib)
+    worst = rel(out["G_diag"], ref["G_diag"])
+    if out["S_index"].shape[1] != E.shape[1]:
+        return float("inf")
+    for s_, (i, j) in enumerate(out["S_index"].T):
+        v = int(i) if parent[int(i)] == int(j) else int(j)          # the child of the pair
+        g = ref["G_edge"][0, v]                                      # (A^-1)_{p(v), v}
+        worst = max(worst, rel(out["G_lower"][0, s_], g if parent[v] > v else g.T))
+    rev = oracle.junction(d, E, vals, order=np.arange(n)[::-1], lib=lib)
+    worst = max(worst, rel(rev["G_diag"], out["G_diag"]))
+    Sr = {(int(i), int(j)): s_ for s_, (i, j) in enumerate(rev["S_index"].T)}
+    for s_, (i, j) in enumerate(out["S_index"].T):
+        worst = max(worst, rel(rev["G_lower"][0, Sr[(int(i), int(j))]], out["G_lower"][0, s_]))
+    return worst
+
+
 # name -> (function, tolerance)
 PINS = {
     "tiny_chains_dense": (pin_tiny_chains_dense, 1e-12),
@@ -680,4 +758,7 @@ PINS = {
     "bidiag_singular": (pin_bidiag_singular, 0.5),
     "bidiag_backward_finite_differences": (pin_bidiag_backward_finite_differences, 1e-7),
     "bidiag_backward_scalar_exact": (pin_bidiag_backward_scalar_exact, 1e-14),
+    "junction_dense": (pin_junction_dense, 1e-11),
+    "junction_symbolic": (pin_junction_symbolic, 0.5),
+    "junction_tree_and_order": (pin_junction_tree_and_order, 1e-12),
 }
