@@ -197,6 +197,23 @@ selinv_status selinv_bidiag(selinv_dtype dtype, int64_t batch, int64_t L, int32_
                             const void *lower, void *G_diag, void *G_lower, int32_t *info, void *stream);
 
 /*
+ * Cotangents of selinv_bidiag (b <= 16): the pages' hand-written analytic
+ * backward of selinv_bidiag, one batched block op.  From its outputs G_diag,
+ * G_lower and their cotangents Gb_diag, Gb_lower (NULL = zero) writes the
+ * cotangents of M:
+ *   Mb_diag [batch, L, b, b]    Mb_ii = -G_ii^T Gb_ii G_ii^T
+ *                                     - G_{i+1,i}^T Gb_{i+1,i} G_ii^T
+ *                                     - G_ii^T Gb_{i,i-1} G_{i,i-1}^T
+ *   Mb_lower [batch, L-1, b, b] Mb_{i+1,i} = -G_{i+1,i+1}^T Gb_{i+1,i} G_ii^T
+ * (Mb = -G^T Gbar G^T on M's pattern, dG = -G dM G; M^-1 block lower
+ * triangular leaves only these terms).  M itself is not needed; G_lower,
+ * Gb_lower and Mb_lower may be NULL when L = 1.  No workspace.
+ */
+selinv_status selinv_bidiag_backward(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b,
+                                     const void *G_diag, const void *G_lower, const void *Gb_diag,
+                                     const void *Gb_lower, void *Mb_diag, void *Mb_lower, void *stream);
+
+/*
  * Cotangents of the chain selected inverse (b <= 16): given the cotangents
  * Gb_diag [batch, L, b, b] and Gb_lower [batch, L-1, b, b] of a loss with
  * respect to selinv_chain's outputs G_diag and G_lower, writes the
@@ -257,6 +274,49 @@ selinv_status selinv_chain_noalloc(selinv_dtype dtype, int64_t batch, int64_t L,
                                    const void *diag, const void *lower,
                                    void *G_diag, void *G_lower, double *logdet,
                                    const void *rhs, void *x, int32_t *info, void *stream);
+
+/*
+ * General block-sparse SPD matrices (b <= 16): gabp-sparse-inv 0.3.2,
+ * "General sparse selected inverse (junction tree)".  The block pattern is
+ * completed to its chordal fill S by an elimination order, then the
+ * multi-neighbour Takahashi recurrence returns A^-1 on S.
+ *
+ * selinv_junction_plan (host work, cached per pattern): n nodes, m lower
+ * blocks (ei[k], ej[k]) with 0 <= ej[k] < ei[k] < n, no repeats (HOST int32
+ * arrays); order = a permutation of 0..n-1 (HOST) or NULL for greedy minimum
+ * degree on the elimination graph, ties to the smaller node index.  Builds
+ * the fill, the elimination tree, its levels and the index lists, and copies
+ * them to the current device.  Bad input returns SELINV_ERR_INVALID_ARG.
+ * selinv_junction_plan_info: nnz_S (blocks of S below the diagonal) and the
+ * number of levels of each sweep.  selinv_junction_plan_pattern: S as
+ * (S_i[k], S_j[k]), S_i > S_j, sorted by S_j then S_i, and the elimination
+ * order (HOST outputs of nnz_S and n entries; any may be NULL).
+ *
+ * selinv_junction: for `batch` matrices on the plan's pattern:
+ *   diag     [batch, n, b, b]     D_v (lower triangle read)
+ *   edge_val [batch, m, b, b]     A_{ei[k], ej[k]}
+ *   G_diag   [batch, n, b, b]     (A^-1)_vv, exactly symmetric
+ *   G_lower  [batch, nnz_S, b, b] (A^-1)_{S_i[k], S_j[k]}
+ *   logdet [batch] (may be NULL), info [batch]: -1, or a node whose Schur
+ *   complement is not positive definite (outputs then unspecified)
+ * Workspace: selinv_junction_workspace_size(plan, dtype, b, batch) bytes.
+ * One launch per level of each sweep.
+ */
+typedef struct selinv_junction_plan_s selinv_junction_plan_t;
+
+selinv_status selinv_junction_plan(int64_t n, int64_t m, const int32_t *ei, const int32_t *ej,
+                                   const int32_t *order, selinv_junction_plan_t **out);
+void selinv_junction_plan_free(selinv_junction_plan_t *plan);
+selinv_status selinv_junction_plan_info(const selinv_junction_plan_t *plan, int64_t *nnz_S,
+                                        int32_t *collect_levels, int32_t *distribute_levels);
+selinv_status selinv_junction_plan_pattern(const selinv_junction_plan_t *plan, int32_t *S_i, int32_t *S_j,
+                                           int32_t *order);
+size_t selinv_junction_workspace_size(const selinv_junction_plan_t *plan, selinv_dtype dtype, int32_t b,
+                                      int64_t batch);
+selinv_status selinv_junction(const selinv_junction_plan_t *plan, selinv_dtype dtype, int32_t b, int64_t batch,
+                              const void *diag, const void *edge_val, void *G_diag, void *G_lower,
+                              double *logdet, int32_t *info, void *workspace, size_t workspace_bytes,
+                              void *stream);
 
 /*
  * Tree plan: validates `trees` parent arrays of n nodes each (HOST memory,

@@ -213,6 +213,33 @@ selinv_status selinv_bidiag(selinv_dtype dtype, int64_t batch, int64_t L, int32_
     return from_cuda(bidiag_launch<float>(p, al, s));
 }
 
+selinv_status selinv_bidiag_backward(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b, const void *G_diag,
+                                     const void *G_lower, const void *Gb_diag, const void *Gb_lower, void *Mb_diag,
+                                     void *Mb_lower, void *stream)
+{
+    if (!valid_dtype(dtype) || batch < 0 || L < 1 || b < 1) return SELINV_ERR_INVALID_ARG;
+    if (b > 16) return SELINV_ERR_UNSUPPORTED;
+    if (batch > 0 && (!G_diag || !Mb_diag || (L > 1 && (!G_lower || !Mb_lower)))) return SELINV_ERR_INVALID_ARG;
+    const size_t es = elem_size(dtype);
+    if (!aligned(G_diag, es) || !aligned(G_lower, es) || !aligned(Gb_diag, es) || !aligned(Gb_lower, es) ||
+        !aligned(Mb_diag, es) || !aligned(Mb_lower, es))
+        return SELINV_ERR_INVALID_ARG;
+    if (batch == 0) return SELINV_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool al = aligned(G_diag, 16) && aligned(G_lower, 16) && aligned(Gb_diag, 16) && aligned(Gb_lower, 16) &&
+                    aligned(Mb_diag, 16) && aligned(Mb_lower, 16);
+    if (dtype == SELINV_F64) {
+        BidiagBwdArgs<double> a{static_cast<const double *>(G_diag), static_cast<const double *>(G_lower),
+                                static_cast<const double *>(Gb_diag), static_cast<const double *>(Gb_lower),
+                                static_cast<double *>(Mb_diag), static_cast<double *>(Mb_lower), batch, L, b};
+        return from_cuda(bidiag_backward_launch<double>(a, al, s));
+    }
+    BidiagBwdArgs<float> a{static_cast<const float *>(G_diag), static_cast<const float *>(G_lower),
+                           static_cast<const float *>(Gb_diag), static_cast<const float *>(Gb_lower),
+                           static_cast<float *>(Mb_diag), static_cast<float *>(Mb_lower), batch, L, b};
+    return from_cuda(bidiag_backward_launch<float>(a, al, s));
+}
+
 size_t selinv_chain_backward_workspace_size(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b)
 {
     if (!valid_dtype(dtype) || batch < 0 || L < 1 || b < 1 || b > 16) return 0;

@@ -4,29 +4,31 @@
 //   G_ii = M_ii^-1,   G_{i+1,i} = -M_{i+1,i+1}^-1 M_{i+1,i} M_ii^-1
 // on M's pattern; no symmetry, no sweep (every block is local).
 //
-// One half-warp per chain walks i = 0 .. L-1 so that each diagonal block is
-// inverted once; lane r of the half holds row r of the block being inverted.
-// The inverse is Gauss-Jordan elimination on [M_ii | I] with partial
-// pivoting: at column k the unused row with the largest |entry| (a
-// half-warp arg-max) is the pivot; it is broadcast by shuffles, scaled, and
-// removed from every other row.  No row is moved: the lane that pivots
-// column k ends with row k of the inverse, which it writes to shared memory.
-// The two products of G_{i+1,i} then read their right-hand factor row by row
-// from shared memory (pitch 17: a column of a padded image spans distinct
-// banks).  A zero or non-finite pivot marks M_ii singular (info = first such
-// block; the chain's outputs are then unspecified).
+// Every block is local, so the work is spread over all blocks of all chains:
+//  * bidiag_inverse_kernel: one half-warp per diagonal block, lane r holding
+//    row r.  Gauss-Jordan elimination on [M_ii | I] with partial pivoting: at
+//    column k the unused row with the largest |entry| (a half-warp arg-max)
+//    is the pivot; it is broadcast by shuffles, scaled and removed from every
+//    other row.  No row is moved: the lane that pivots column k ends with row
+//    k of G_ii = M_ii^-1 and stores it.  A zero or non-finite pivot marks the
+//    block singular (info = the chain's first such block; its outputs are
+//    then unspecified).
+//  * bidiag_lower_kernel: one warp per sub-diagonal block, after the first
+//    kernel: G_{i+1,i} = -G_{i+1,i+1} (M_{i+1,i} G_ii) as two X Y^T products
+//    of register tiles on the FP64 tensor cores, G_ii loaded transposed.
 #include <type_traits>
 
-#include "common.cuh"
+#include <algorithm>
+#include <climits>
+
 #include "kernels.h"
+#include "warp16.cuh"
 
 namespace selinv {
 
 namespace {
 
 constexpr int BD_WARPS = 4;
-constexpr int BD_PITCH = 17;
-constexpr int BD_IMG = 16 * BD_PITCH;                 // one padded 16 x 16 image
 
 template <class T> SELINV_DEVINL T hshfl(T v, int src) { return __shfl_sync(FULL_MASK, v, src, 16); }
 template <class T> SELINV_DEVINL T hshfl_xor(T v, int m) { return __shfl_xor_sync(FULL_MASK, v, m, 16); }
@@ -72,16 +74,16 @@ template <class T, bool FULL> SELINV_DEVINL void store_row(T *M, const T x[16], 
     }
 }
 
-// Inverse of the b x b block whose row r the lane holds in a (zero beyond b);
-// row k(r) of the inverse is written to img[k(r) * BD_PITCH + .].  Returns
-// false (for every lane of the half) if a pivot is zero or not finite.
-template <class T> SELINV_DEVINL bool gj_inverse(T a[16], T *img, int b, int r)
+// Inverse of the b x b block whose row r the lane holds in a (zero beyond b):
+// on return the lane holds row krow of the inverse in e (krow = the column it
+// pivoted; lanes r >= b hold nothing).  Returns false (for every lane of the
+// half) if a pivot is zero or not finite.
+template <class T> SELINV_DEVINL bool gj_inverse(T a[16], T e[16], int &krow, int b, int r)
 {
-    T e[16];
 #pragma unroll
     for (int c = 0; c < 16; ++c) e[c] = (c == r) ? T(1) : T(0);
     bool used = r >= b;                               // pad rows never pivot
-    int krow = 0;
+    krow = 0;
     bool ok = true;
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
@@ -101,108 +103,139 @@ template <class T> SELINV_DEVINL bool gj_inverse(T a[16], T *img, int b, int r)
             const T d = hshfl(a[k], who);
             ok = ok && (fabs(d) > T(0)) && isfinite(d);
             const T inv = T(1) / d;
-            T pr[16], pe[16];
+            const bool piv = r == who;
+            const T f = a[k];
+            // columns left of k are already eliminated in every unused row
+            // (the pivot row included), so a changes only from column k on
+#pragma unroll
+            for (int c = k; c < 16; ++c) {
+                const T pc = hshfl(a[c], who) * inv;
+                a[c] = piv ? pc : fma(-f, pc, a[c]);
+            }
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
-                pr[c] = hshfl(a[c], who) * inv;
-                pe[c] = hshfl(e[c], who) * inv;
+                const T pc = hshfl(e[c], who) * inv;
+                e[c] = piv ? pc : fma(-f, pc, e[c]);
             }
-            if (r == who) {
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    a[c] = pr[c];
-                    e[c] = pe[c];
-                }
+            if (piv) {
                 used = true;
                 krow = k;
-            } else {
-                const T f = a[k];
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    a[c] = fma(-f, pr[c], a[c]);
-                    e[c] = fma(-f, pe[c], e[c]);
-                }
             }
         }
-    }
-    if (r < b) {
-#pragma unroll
-        for (int c = 0; c < 16; ++c) img[krow * BD_PITCH + c] = e[c];
     }
     return ok;
 }
 
+// One half-warp per diagonal block (grid-stride): G_ii = M_ii^-1.
 template <class T, bool FULL>
-__global__ void __launch_bounds__(BD_WARPS * 32) bidiag_kernel(BidiagArgs<T> p)
+__global__ void __launch_bounds__(BD_WARPS * 32) bidiag_inverse_kernel(BidiagArgs<T> p)
 {
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int half = lane >> 4, r = lane & 15;
-    const int64_t e = ((int64_t)blockIdx.x * BD_WARPS + wid) * 2 + half;
-    if (((int64_t)blockIdx.x * BD_WARPS + wid) * 2 >= p.batch) return;   // whole warp idle
-    const bool live = e < p.batch;                    // the second half of the last warp may have no chain
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    T *base = reinterpret_cast<T *>(smem_raw) + (wid * 2 + half) * 3 * BD_IMG;
-    T *timg = base + 2 * BD_IMG;                      // M_{i,i-1} M_{i-1,i-1}^-1 (two images before it
-                                                      // hold the inverses of blocks i-1 and i, by parity)
+    const int lane = threadIdx.x & 31, r = lane & 15;
+    const int64_t nblk = p.batch * p.L;
+    const int64_t halves = (int64_t)gridDim.x * BD_WARPS * 2;
     const int b = p.b;
-    const int64_t L = p.L, bb = (int64_t)b * b;
-    const int64_t ec = live ? e : 0;
-    const T *D = p.diag + ec * L * bb;
-    const T *Bl = p.lower + ec * (L - 1) * bb;
-    T *Gd = p.G_diag + ec * L * bb;
-    T *Gl = p.G_lower + ec * (L - 1) * bb;
-    int bad_at = -1;
-    for (int64_t i = 0; i < L; ++i) {
-        if (live && i + 1 < L) {                      // next step's blocks toward L2
-            prefetch_range_l2(D + (i + 1) * bb, bb, r, 16);
-            prefetch_range_l2(Bl + i * bb, bb, r, 16);
+    const int64_t bb = (int64_t)b * b;
+    const int64_t h0 = ((int64_t)blockIdx.x * BD_WARPS + (threadIdx.x >> 5)) * 2 + (lane >> 4);
+    // every half of a warp runs the same number of iterations (shuffles span the warp)
+    const int64_t w0 = h0 - (lane >> 4);
+    for (int64_t base = w0; base < nblk; base += halves) {
+        const int64_t blk = base + (lane >> 4);
+        const bool live = blk < nblk;
+        T a[16], e[16];
+        int krow;
+        load_row<T, FULL>(a, p.diag + (live ? blk : 0) * bb, b, r, live);
+        const bool ok = gj_inverse<T>(a, e, krow, b, r);
+        if (live) {
+            if (r < b) store_row<T, FULL>(p.G_diag + blk * bb, e, b, krow);
+            if (!ok && r == 0) atomicMin(p.info + blk / p.L, (int32_t)(blk % p.L));
         }
-        T a[16];
-        load_row<T, FULL>(a, D + i * bb, b, r, live);
-        T *cur = base + (i & 1) * BD_IMG, *prev = base + ((i & 1) ^ 1) * BD_IMG;
-        const bool ok = gj_inverse<T>(a, cur, b, r);
-        if (!ok && bad_at < 0) bad_at = (int)i;
-        __syncwarp();
-        T g[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) g[c] = cur[r * BD_PITCH + c];
-        if (live) store_row<T, FULL>(Gd + i * bb, g, b, r);     // G_ii = M_ii^-1
-        if (i > 0) {
-            // T = M_{i,i-1} M_{i-1,i-1}^-1 (row r), then G_{i,i-1} = -M_ii^-1 T
-            T m[16], t[16];
-            load_row<T, FULL>(m, Bl + (i - 1) * bb, b, r, live);
-#pragma unroll
-            for (int c = 0; c < 16; ++c) t[c] = T(0);
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-                if (k < b)
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) t[c] = fma(m[k], prev[k * BD_PITCH + c], t[c]);
-#pragma unroll
-            for (int c = 0; c < 16; ++c) timg[r * BD_PITCH + c] = t[c];
-            __syncwarp();
-#pragma unroll
-            for (int c = 0; c < 16; ++c) t[c] = T(0);
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-                if (k < b)
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) t[c] = fma(-g[k], timg[k * BD_PITCH + c], t[c]);
-            if (live) store_row<T, FULL>(Gl + (i - 1) * bb, t, b, r);
-        }
-        __syncwarp();                                 // cur becomes prev; timg is free again
     }
-    if (live && r == 0) p.info[e] = bad_at;
+}
+
+// Tile of a row-major b x b block, transposed on the way in (zero beyond b).
+template <class T> SELINV_DEVINL void load_tile_T(w16::Tile<T> &a, const T *M, int b, int g, int t)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = g + 8 * h, c = w16::tcol(t, q);
+            a.v[h][q] = (r < b && c < b) ? __ldcg(M + c * b + r) : T(0);
+        }
+}
+
+template <class T> SELINV_DEVINL void load_tile_l2(w16::Tile<T> &a, const T *M, int b, int g, int t)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = g + 8 * h, c = w16::tcol(t, q);
+            a.v[h][q] = (r < b && c < b) ? __ldcg(M + r * b + c) : T(0);
+        }
+}
+
+// One warp per sub-diagonal block (grid-stride): G_{i+1,i} = -G_{i+1,i+1} (M_{i+1,i} G_ii).
+template <class T>
+__global__ void __launch_bounds__(BD_WARPS * 32) bidiag_lower_kernel(BidiagArgs<T> p)
+{
+    using namespace w16;
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    T *sX = reinterpret_cast<T *>(smem_raw) + (threadIdx.x >> 5) * 2 * SL<T>::ELEMS, *sY = sX + SL<T>::ELEMS;
+    const int64_t L1 = p.L - 1, nblk = p.batch * L1;
+    const int b = p.b;
+    const int64_t bb = (int64_t)b * b;
+    for (int64_t k = (int64_t)blockIdx.x * BD_WARPS + (threadIdx.x >> 5); k < nblk;
+         k += (int64_t)gridDim.x * BD_WARPS) {
+        const int64_t e = k / L1, i = k % L1;
+        const T *Gii = p.G_diag + (e * p.L + i) * bb;
+        Tile<T> giT, ml, gn, xt, gl;
+        load_tile_T<T>(giT, Gii, b, g, t);
+        load_tile_l2<T>(ml, p.lower + k * bb, b, g, t);
+        load_tile_l2<T>(gn, Gii + bb, b, g, t);
+        zero(xt);
+        gemm_nt<false>(xt, giT, ml, sX, sY, g, t);     // (M_{i+1,i} G_ii)^T = G_ii^T M_{i+1,i}^T
+        zero(gl);
+        gemm_nt<true>(gl, gn, xt, sX, sY, g, t);       // -G_{i+1,i+1} (M_{i+1,i} G_ii)
+        store_block<T, false>(p.G_lower + k * bb, gl, b, g, t);
+    }
+}
+
+__global__ void bidiag_info(int32_t *info, int64_t batch, int final_pass)
+{
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= batch) return;
+    if (!final_pass) info[i] = INT_MAX;
+    else if (info[i] == INT_MAX) info[i] = -1;
 }
 
 template <class T> cudaError_t launch(const BidiagArgs<T> &p, bool full, cudaStream_t s)
 {
-    const size_t smem = sizeof(T) * 3 * BD_IMG * 2 * BD_WARPS;
-    auto k = full ? bidiag_kernel<T, true> : bidiag_kernel<T, false>;
-    cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    const int64_t warps = ceil_div(p.batch, 2);
-    k<<<(unsigned)ceil_div(warps, BD_WARPS), BD_WARPS * 32, smem, s>>>(p);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const unsigned ib = (unsigned)ceil_div(p.batch, 256);
+    bidiag_info<<<ib, 256, 0, s>>>(p.info, p.batch, 0);
+    auto ki = full ? bidiag_inverse_kernel<T, true> : bidiag_inverse_kernel<T, false>;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, ki, BD_WARPS * 32, 0) != cudaSuccess || occ < 1) occ = 2;
+    const int64_t halves = p.batch * p.L;
+    const int64_t gi = std::min<int64_t>((int64_t)sms * occ, ceil_div(halves, 2 * BD_WARPS));
+    ki<<<(unsigned)gi, BD_WARPS * 32, 0, s>>>(p);
+    if (p.L > 1) {
+        const size_t smem = sizeof(T) * 2 * w16::SL<T>::ELEMS * BD_WARPS;
+        auto kl = bidiag_lower_kernel<T>;
+        cudaError_t err = cudaFuncSetAttribute(kl, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess) return err;
+        int occ_l = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_l, kl, BD_WARPS * 32, smem) != cudaSuccess ||
+            occ_l < 1)
+            occ_l = 4;
+        const int64_t gl = std::min<int64_t>((int64_t)sms * occ_l, ceil_div(p.batch * (p.L - 1), BD_WARPS));
+        kl<<<(unsigned)gl, BD_WARPS * 32, smem, s>>>(p);
+    }
+    bidiag_info<<<ib, 256, 0, s>>>(p.info, p.batch, 1);
     return cudaGetLastError();
 }
 

@@ -235,6 +235,92 @@ __global__ void __launch_bounds__(BW_WARPS * 32) chain_backward_kernel(ChainBwdA
     }
 }
 
+// Cotangents of the non-symmetric chain (gabp-sparse-inv: selinv_bidiag's
+// analytic backward, one batched block op).  G = M^-1 is block lower
+// triangular, so Mb = -G^T Gbar G^T on M's pattern needs only the forward's
+// outputs:
+//   Mb_ii      = -G_ii^T Gb_ii G_ii^T - G_{i+1,i}^T Gb_{i+1,i} G_ii^T
+//                - G_ii^T Gb_{i,i-1} G_{i,i-1}^T
+//   Mb_{i+1,i} = -G_{i+1,i+1}^T Gb_{i+1,i} G_ii^T.
+// One warp per chain walks i = 0 .. L-1 and forms the transposes
+//   Mb_ii^T = -(G_ii Gb_ii^T + G_{i,i-1} Gb_{i,i-1}^T) G_ii - Y_i^T G_{i+1,i},
+//   Mb_{i,i-1}^T = -Y_{i-1}^T G_ii,   Y_i^T = G_ii Gb_{i+1,i}^T,
+// as X Y^T products of register tiles, written back transposed.
+template <class T, bool FULL>
+__global__ void __launch_bounds__(BW_WARPS * 32) bidiag_backward_kernel(BidiagBwdArgs<T> a)
+{
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int64_t e = (int64_t)blockIdx.x * BW_WARPS + wid;
+    if (e >= a.batch) return;                          // the whole warp leaves together
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    T *s0 = reinterpret_cast<T *>(smem_raw) + wid * bw_smem_elems<T>();
+    T *s1 = s0 + SL<T>::ELEMS, *s2 = s1 + SL<T>::ELEMS;
+    const int b = a.b;
+    const int64_t L = a.L, bb = (int64_t)b * b;
+    const T *G = a.G_diag + e * L * bb;
+    const T *Gl = a.G_lower + e * (L - 1) * bb;
+    const T *Gbd = a.Gb_diag + e * L * bb;
+    const T *Gbl = a.Gb_lower + e * (L - 1) * bb;
+    T *Mbd = a.Mb_diag + e * L * bb;
+    T *Mbl = a.Mb_lower + e * (L - 1) * bb;
+    Tile<T> Gp, Lp, Yp;                                // G_{i,i-1}, Gb_{i,i-1}, Y_{i-1}^T
+    zero(Gp);
+    zero(Lp);
+    zero(Yp);
+    for (int64_t i = 0; i < L; ++i) {
+        if (i + 1 < L) {                              // next step's blocks toward L2
+            prefetch_block(G + (i + 1) * bb, bb, lane);
+            if (a.Gb_diag) prefetch_block(Gbd + (i + 1) * bb, bb, lane);
+            if (i + 2 < L) {
+                prefetch_block(Gl + (i + 1) * bb, bb, lane);
+                if (a.Gb_lower) prefetch_block(Gbl + (i + 1) * bb, bb, lane);
+            }
+        }
+        Tile<T> Gii, GiiT, U, R;
+        load_tile<T, FULL, true>(Gii, G + i * bb, b, g, t);
+        transpose(GiiT, Gii, s0, g, t);
+        zero(U);
+        if (a.Gb_diag) {
+            Tile<T> gd;
+            load_tile<T, FULL, true>(gd, Gbd + i * bb, b, g, t);
+            gemm_nt<false>(U, Gii, gd, s1, s2, g, t);          // G_ii Gb_ii^T
+        }
+        if (i > 0) {
+            gemm_nt<false>(U, Gp, Lp, s1, s2, g, t);            // + G_{i,i-1} Gb_{i,i-1}^T
+            Tile<T> ml;
+            zero(ml);
+            gemm_nt<true>(ml, Yp, GiiT, s1, s2, g, t);          // Mb_{i,i-1}^T = -Y_{i-1}^T G_ii
+            store_block_T<T, FULL>(Mbl + (i - 1) * bb, ml, b, g, t);
+        }
+        zero(R);
+        gemm_nt<true>(R, U, GiiT, s1, s2, g, t);                // -U G_ii
+        if (i + 1 < L) {
+            Tile<T> gl, lb, glT;
+            load_tile<T, FULL, true>(gl, Gl + i * bb, b, g, t);
+            if (a.Gb_lower) load_tile<T, FULL, true>(lb, Gbl + i * bb, b, g, t);
+            else zero(lb);
+            zero(Yp);
+            gemm_nt<false>(Yp, Gii, lb, s1, s2, g, t);          // Y_i^T = G_ii Gb_{i+1,i}^T
+            transpose(glT, gl, s0, g, t);
+            gemm_nt<true>(R, Yp, glT, s1, s2, g, t);            // - Y_i^T G_{i+1,i}
+            Gp = gl;
+            Lp = lb;
+        }
+        store_block_T<T, FULL>(Mbd + i * bb, R, b, g, t);       // Mb_ii = R^T
+    }
+}
+
+template <class T> cudaError_t launch_bidiag_bwd(const BidiagBwdArgs<T> &a, bool full, cudaStream_t s)
+{
+    const size_t smem = sizeof(T) * bw_smem_elems<T>() * BW_WARPS;
+    auto k = full ? bidiag_backward_kernel<T, true> : bidiag_backward_kernel<T, false>;
+    cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    k<<<(unsigned)ceil_div(a.batch, BW_WARPS), BW_WARPS * 32, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
 template <class T> cudaError_t launch_bwd(const ChainBwdArgs<T> &a, bool full, cudaStream_t s)
 {
     const size_t smem = sizeof(T) * bw_smem_elems<T>() * BW_WARPS;
@@ -258,6 +344,13 @@ template <class T> cudaError_t chain_backward_launch(const ChainBwdArgs<T> &a, b
     return launch_bwd<T>(a, a.b == 16 && aligned16, s);
 }
 
+template <class T> cudaError_t bidiag_backward_launch(const BidiagBwdArgs<T> &a, bool aligned16, cudaStream_t s)
+{
+    return launch_bidiag_bwd<T>(a, a.b == 16 && aligned16, s);
+}
+
+template cudaError_t bidiag_backward_launch<double>(const BidiagBwdArgs<double> &, bool, cudaStream_t);
+template cudaError_t bidiag_backward_launch<float>(const BidiagBwdArgs<float> &, bool, cudaStream_t);
 template cudaError_t chain_backward_launch<double>(const ChainBwdArgs<double> &, bool, cudaStream_t);
 template cudaError_t chain_backward_launch<float>(const ChainBwdArgs<float> &, bool, cudaStream_t);
 

@@ -1,0 +1,599 @@
+// General block-sparse SPD matrices (b <= 16): gabp-sparse-inv 0.3.2 (PyPI
+// page), "General sparse selected inverse (junction tree)": the block pattern
+// is completed to its chordal fill S = pattern(L + L^T) by an elimination
+// order (greedy minimum degree unless the caller gives one), then the
+// multi-neighbour Takahashi recurrence runs over the elimination tree.
+//
+// With N(v) the neighbours of v still present when v is eliminated (a clique
+// after v's elimination), in elimination order:
+//  collect (children before parents; left-looking, so every block has one
+//  writer): for u in {v} + N(v)
+//     A'_{u,v} = A_{u,v} - sum_{k : u, v in N(k)} W_{u,k} A'_{v,k}^T
+//     (A_{u,v} = 0 for a fill block), S_v = A'_{v,v}, P_v = S_v^-1,
+//     W_{u,v} = A'_{u,v} P_v, log|A| += log det S_v;
+//  distribute (parents before children):
+//     G_{u,v} = -sum_{l in N(v)} G_{u,l} W_{l,v}   (u in N(v)),
+//     G_{v,v} = P_v - sum_{l in N(v)} W_{l,v}^T G_{l,v}.
+// All k above are descendants of v in the elimination tree and all u, l are
+// ancestors, so each sweep runs one launch per tree level (heights for the
+// collect, depths for the distribute), one warp per (node, matrix) item.
+// The host plan holds the symbolic work: order, fill, the tree and its
+// levels, the index lists of every contribution and of every G_{u,l} a
+// clique reads.  Off-diagonal blocks of S are stored as (i, j), i > j, in the
+// caller's numbering; a block met in the other orientation is read or
+// written transposed.
+#include <algorithm>
+#include <climits>
+#include <cmath>
+#include <map>
+#include <new>
+#include <set>
+#include <unordered_map>
+#include <vector>
+
+#include "kernels.h"
+#include "warp16.cuh"
+
+struct selinv_junction_plan_s {
+    int64_t n = 0, m = 0, nnz = 0, E = 0;       // nodes, input blocks, blocks of S, clique entries
+    int device = 0;
+    std::vector<int32_t> order, S_i, S_j;       // host copies for the caller
+    std::vector<int64_t> c_off, d_off;          // level offsets (collect by height, distribute by depth)
+    int32_t *d_c_nodes = nullptr, *d_d_nodes = nullptr;
+    int32_t *d_col_ptr = nullptr;               // [n+1] entries of node v: its N(v) in elimination order
+    int32_t *d_ent_slot = nullptr;              // [E] block of S holding (u, v)
+    int32_t *d_ent_trans = nullptr;             // [E] 1: S holds (v, u), read / write transposed
+    int32_t *d_ent_src = nullptr;               // [E] input block index of that slot, or -1 (fill)
+    int32_t *d_con_ptr = nullptr;               // [E + n + 1] contributions per target (v, t)
+    int32_t *d_con_w = nullptr, *d_con_a = nullptr;   // entries of W_{u,k} and A'_{v,k}
+    int32_t *d_pair_ptr = nullptr;              // [n+1] into pair codes (|N(v)|^2 per node)
+    int32_t *d_pair = nullptr;                  // -(w+1): diagonal of node w; else 2 * slot + transposed
+};
+
+namespace selinv {
+
+namespace {
+
+constexpr int JWARPS = 4;
+constexpr int JSLOT = 256;                       // one 16 x 16 tile per workspace block
+
+struct JDev {
+    const int32_t *col_ptr, *ent_slot, *ent_trans, *ent_src, *con_ptr, *con_w, *con_a, *pair_ptr, *pair;
+    int64_t n, m, nnz, E;
+};
+
+template <class T> struct JBufs {
+    const T *diag, *edge;
+    T *G_diag, *G_lower;
+    T *Sinv, *Ap, *W;                            // workspace tiles: [batch][n], [batch][E], [batch][E]
+    double *ld;                                  // [batch][n]
+    int32_t *info;
+    int b;
+};
+
+// Tile from a 16-pitch workspace tile (read through L2: written earlier in the call).
+template <class T> SELINV_DEVINL void ld_ws(w16::Tile<T> &a, const T *M, int g, int t, bool trans)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = g + 8 * h, c = w16::tcol(t, q);
+            a.v[h][q] = __ldcg(trans ? M + c * 16 + r : M + r * 16 + c);
+        }
+}
+
+template <class T> SELINV_DEVINL void st_ws(T *M, const w16::Tile<T> &a, int g, int t)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) M[(g + 8 * h) * 16 + w16::tcol(t, q)] = a.v[h][q];
+}
+
+// b x b block (row-major), possibly transposed, into a tile; zero pad.
+template <class T> SELINV_DEVINL void ld_blk(w16::Tile<T> &a, const T *M, int b, int g, int t, bool trans, bool l2)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = g + 8 * h, c = w16::tcol(t, q);
+            const T *p = trans ? M + c * b + r : M + r * b + c;
+            a.v[h][q] = (r < b && c < b) ? (l2 ? __ldcg(p) : __ldg(p)) : T(0);
+        }
+}
+
+template <class T> SELINV_DEVINL void st_blk(T *M, const w16::Tile<T> &a, int b, int g, int t, bool trans)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = g + 8 * h, c = w16::tcol(t, q);
+            if (r < b && c < b) {
+                if (trans) M[c * b + r] = a.v[h][q];
+                else M[r * b + c] = a.v[h][q];
+            }
+        }
+}
+
+template <class T>
+__global__ void __launch_bounds__(JWARPS * 32)
+junction_collect_kernel(JBufs<T> p, JDev jd, const int32_t *nodes, int64_t count, int64_t batch)
+{
+    using namespace w16;
+    constexpr int EL = SL<T>::ELEMS;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    T *s1 = reinterpret_cast<T *>(smem_raw) + wid * (2 * EL + 32), *s2 = s1 + EL, *cb = s2 + EL;
+    const int64_t item = (int64_t)blockIdx.x * JWARPS + wid;
+    if (item >= count * batch) return;                 // the whole warp leaves together
+    const int32_t v = nodes[item % count];
+    const int64_t e = item / count;
+    const int b = p.b;
+    const int64_t bb = (int64_t)b * b;
+    const int32_t c0 = jd.col_ptr[v], c1 = jd.col_ptr[v + 1];
+    const int64_t tb = (int64_t)c0 + v;               // first target of v
+    T *Ap = p.Ap + e * jd.E * JSLOT, *W = p.W + e * jd.E * JSLOT;
+    Tile<T> S;
+    for (int32_t tt = 0; tt <= c1 - c0; ++tt) {
+        Tile<T> acc;
+        if (tt == 0) {
+            load_sym<T, false>(acc, p.diag + (e * jd.n + v) * bb, b, g, t);
+        } else {
+            const int32_t ent = c0 + tt - 1, src = jd.ent_src[ent];
+            if (src >= 0) ld_blk<T>(acc, p.edge + (e * jd.m + src) * bb, b, g, t, jd.ent_trans[ent] != 0, false);
+            else zero(acc);
+        }
+        for (int32_t c = jd.con_ptr[tb + tt]; c < jd.con_ptr[tb + tt + 1]; ++c) {
+            Tile<T> w, a;
+            ld_ws<T>(w, W + (int64_t)jd.con_w[c] * JSLOT, g, t, false);
+            ld_ws<T>(a, Ap + (int64_t)jd.con_a[c] * JSLOT, g, t, false);
+            gemm_nt<true>(acc, w, a, s1, s2, g, t);          // -= W_{u,k} A'_{v,k}^T
+        }
+        if (tt == 0) S = acc;
+        else st_ws<T>(Ap + (int64_t)(c0 + tt - 1) * JSLOT, acc, g, t);
+    }
+    mirror_upper(S, g, t);
+    LogAcc det;
+    det.init();
+    bool bad = false;
+    spd_inverse<T>(S, cb, g, t, det, bad);              // S = P_v
+    if (lane == 0) {
+        p.ld[e * jd.n + v] = det.log_value();
+        if (bad) atomicMin(p.info + e, v);
+    }
+    st_ws<T>(p.Sinv + (e * jd.n + v) * JSLOT, S, g, t);
+    __syncwarp();
+    for (int32_t ent = c0; ent < c1; ++ent) {         // W_{u,v} = A'_{u,v} P_v
+        Tile<T> a, w;
+        ld_ws<T>(a, Ap + (int64_t)ent * JSLOT, g, t, false);
+        zero(w);
+        gemm_nt<false>(w, a, S, s1, s2, g, t);
+        st_ws<T>(W + (int64_t)ent * JSLOT, w, g, t);
+    }
+}
+
+template <class T>
+__global__ void __launch_bounds__(JWARPS * 32)
+junction_distribute_kernel(JBufs<T> p, JDev jd, const int32_t *nodes, int64_t count, int64_t batch)
+{
+    using namespace w16;
+    constexpr int EL = SL<T>::ELEMS;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    T *s0 = reinterpret_cast<T *>(smem_raw) + wid * (3 * EL + 32), *s1 = s0 + EL, *s2 = s1 + EL;
+    const int64_t item = (int64_t)blockIdx.x * JWARPS + wid;
+    if (item >= count * batch) return;
+    const int32_t v = nodes[item % count];
+    const int64_t e = item / count;
+    const int b = p.b;
+    const int64_t bb = (int64_t)b * b;
+    const int32_t c0 = jd.col_ptr[v], d = jd.col_ptr[v + 1] - c0;
+    const T *W = p.W + e * jd.E * JSLOT;
+    T *Gd = p.G_diag + e * jd.n * bb, *Gl = p.G_lower + e * jd.nnz * bb;
+    Tile<T> gvv;
+    ld_ws<T>(gvv, p.Sinv + (e * jd.n + v) * JSLOT, g, t, false);
+    const int32_t *pc = jd.pair + jd.pair_ptr[v];
+    for (int32_t a = 0; a < d; ++a) {                  // G_{u,v}, u = N(v)[a]
+        Tile<T> acc;
+        zero(acc);
+        for (int32_t c = 0; c < d; ++c) {
+            const int32_t code = pc[a * d + c];
+            Tile<T> gul, wt;
+            if (code < 0) ld_blk<T>(gul, Gd + (int64_t)(-code - 1) * bb, b, g, t, false, true);
+            else ld_blk<T>(gul, Gl + (int64_t)(code >> 1) * bb, b, g, t, (code & 1) != 0, true);
+            ld_ws<T>(wt, W + (int64_t)(c0 + c) * JSLOT, g, t, true);     // W_{l,v}^T
+            gemm_nt<true>(acc, gul, wt, s1, s2, g, t);                  // -= G_{u,l} W_{l,v}
+        }
+        const int32_t ent = c0 + a;
+        st_blk<T>(Gl + (int64_t)jd.ent_slot[ent] * bb, acc, b, g, t, jd.ent_trans[ent] != 0);
+        Tile<T> accT, wt;                              // G_vv -= W_{u,v}^T G_{u,v}
+        to_smem<T>(s0, acc, g, t);
+        __syncwarp();
+        from_smem_T<T>(accT, s0, g, t);
+        __syncwarp();
+        ld_ws<T>(wt, W + (int64_t)ent * JSLOT, g, t, true);
+        gemm_nt<true>(gvv, wt, accT, s1, s2, g, t);
+    }
+    to_smem<T>(s0, gvv, g, t);                         // exactly symmetric from the lower triangle
+    __syncwarp();
+    from_smem_lower<T>(gvv, s0, g, t);
+    __syncwarp();
+    st_blk<T>(Gd + (int64_t)v * bb, gvv, b, g, t, false);
+}
+
+__global__ void junction_init(int32_t *info, int64_t batch)
+{
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < batch) info[i] = INT_MAX;
+}
+
+// log det per matrix = sum of its nodes' log det S_v in node order (deterministic).
+__global__ void junction_finalize(const double *ld, int64_t n, int64_t batch, double *logdet, int32_t *info)
+{
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= batch) return;
+    double s = 0.0;
+    for (int64_t v = 0; v < n; ++v) s += ld[i * n + v];
+    if (logdet) logdet[i] = s;
+    if (info[i] == INT_MAX) info[i] = -1;
+}
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+template <class T> size_t ws_bytes(const selinv_junction_plan_s *pl, int64_t batch)
+{
+    return align256(sizeof(T) * JSLOT * (size_t)(batch * pl->n)) +
+           2 * align256(sizeof(T) * JSLOT * (size_t)(batch * pl->E)) + align256(sizeof(double) * (size_t)(batch * pl->n));
+}
+
+template <class T>
+cudaError_t run_junction(const selinv_junction_plan_s *pl, int b, int64_t batch, const T *diag, const T *edge,
+                         T *G_diag, T *G_lower, double *logdet, int32_t *info, void *ws, cudaStream_t s)
+{
+    char *w = static_cast<char *>(ws);
+    JBufs<T> p;
+    p.diag = diag;
+    p.edge = edge;
+    p.G_diag = G_diag;
+    p.G_lower = G_lower;
+    p.Sinv = reinterpret_cast<T *>(w);
+    w += align256(sizeof(T) * JSLOT * (size_t)(batch * pl->n));
+    p.Ap = reinterpret_cast<T *>(w);
+    w += align256(sizeof(T) * JSLOT * (size_t)(batch * pl->E));
+    p.W = reinterpret_cast<T *>(w);
+    w += align256(sizeof(T) * JSLOT * (size_t)(batch * pl->E));
+    p.ld = reinterpret_cast<double *>(w);
+    p.info = info;
+    p.b = b;
+    JDev jd{pl->d_col_ptr, pl->d_ent_slot, pl->d_ent_trans, pl->d_ent_src, pl->d_con_ptr, pl->d_con_w,
+            pl->d_con_a, pl->d_pair_ptr, pl->d_pair, pl->n, pl->m, pl->nnz, pl->E};
+    const unsigned ib = (unsigned)ceil_div(batch, 256);
+    junction_init<<<ib, 256, 0, s>>>(info, batch);
+    constexpr int EL = w16::SL<T>::ELEMS;
+    const size_t smem_c = sizeof(T) * (2 * EL + 32) * JWARPS, smem_d = sizeof(T) * (3 * EL + 32) * JWARPS;
+    cudaError_t err = cudaFuncSetAttribute(junction_collect_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)smem_c);
+    if (err == cudaSuccess)
+        err = cudaFuncSetAttribute(junction_distribute_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)smem_d);
+    if (err != cudaSuccess) return err;
+    for (size_t l = 0; l + 1 < pl->c_off.size(); ++l) {
+        const int64_t cnt = pl->c_off[l + 1] - pl->c_off[l];
+        junction_collect_kernel<T><<<(unsigned)ceil_div(cnt * batch, JWARPS), JWARPS * 32, smem_c, s>>>(
+            p, jd, pl->d_c_nodes + pl->c_off[l], cnt, batch);
+    }
+    for (size_t l = 0; l + 1 < pl->d_off.size(); ++l) {
+        const int64_t cnt = pl->d_off[l + 1] - pl->d_off[l];
+        junction_distribute_kernel<T><<<(unsigned)ceil_div(cnt * batch, JWARPS), JWARPS * 32, smem_d, s>>>(
+            p, jd, pl->d_d_nodes + pl->d_off[l], cnt, batch);
+    }
+    junction_finalize<<<ib, 256, 0, s>>>(p.ld, pl->n, batch, logdet, info);
+    return cudaGetLastError();
+}
+
+bool is_aligned(const void *q, size_t a) { return (reinterpret_cast<uintptr_t>(q) % a) == 0; }
+
+}  // namespace
+
+}  // namespace selinv
+
+using namespace selinv;
+
+extern "C" {
+
+void selinv_junction_plan_free(selinv_junction_plan_t *pl)
+{
+    if (!pl) return;
+    int32_t *arrs[] = {pl->d_c_nodes, pl->d_d_nodes, pl->d_col_ptr, pl->d_ent_slot, pl->d_ent_trans, pl->d_ent_src,
+                       pl->d_con_ptr, pl->d_con_w, pl->d_con_a, pl->d_pair_ptr, pl->d_pair};
+    for (int32_t *a : arrs) cudaFree(a);
+    delete pl;
+}
+
+selinv_status selinv_junction_plan(int64_t n, int64_t m, const int32_t *ei, const int32_t *ej, const int32_t *order,
+                                   selinv_junction_plan_t **out)
+{
+    if (!out) return SELINV_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (n < 1 || m < 0 || (m > 0 && (!ei || !ej)) || n >= (int64_t)INT32_MAX / 2) return SELINV_ERR_INVALID_ARG;
+    // pattern: (i, j), 0 <= j < i < n, no repeats
+    std::vector<std::set<int32_t>> adj(n);
+    std::unordered_map<int64_t, int32_t> input;     // key i * n + j -> input block index
+    for (int64_t k = 0; k < m; ++k) {
+        const int32_t i = ei[k], j = ej[k];
+        if (j < 0 || i <= j || i >= n) return SELINV_ERR_INVALID_ARG;
+        if (!input.emplace((int64_t)i * n + j, (int32_t)k).second) return SELINV_ERR_INVALID_ARG;
+        adj[i].insert(j);
+        adj[j].insert(i);
+    }
+    std::vector<int32_t> seq;
+    seq.reserve(n);
+    if (order) {
+        std::vector<char> seen(n, 0);
+        for (int64_t k = 0; k < n; ++k) {
+            const int32_t v = order[k];
+            if (v < 0 || v >= n || seen[v]) return SELINV_ERR_INVALID_ARG;
+            seen[v] = 1;
+        }
+    }
+    // eliminate: N(v) = the neighbours still present; they become a clique
+    std::vector<std::vector<int32_t>> nbr(n);
+    std::set<std::pair<int32_t, int32_t>> bydeg;     // (degree, node) of the remaining nodes
+    if (!order)
+        for (int32_t v = 0; v < n; ++v) bydeg.insert({(int32_t)adj[v].size(), v});
+    std::map<std::pair<int32_t, int32_t>, int32_t> Sset;   // (i, j), i > j -> slot (filled later)
+    for (const auto &kv : input) Sset.emplace(std::make_pair((int32_t)(kv.first / n), (int32_t)(kv.first % n)), -1);
+    for (int64_t step = 0; step < n; ++step) {
+        int32_t v;
+        if (order) {
+            v = order[step];
+        } else {
+            v = bydeg.begin()->second;
+            bydeg.erase(bydeg.begin());
+        }
+        std::vector<int32_t> nb(adj[v].begin(), adj[v].end());
+        for (size_t a = 0; a < nb.size(); ++a)
+            for (size_t c = a + 1; c < nb.size(); ++c) {
+                const int32_t x = nb[a], y = nb[c];
+                if (adj[x].count(y)) continue;
+                if (!order) {
+                    bydeg.erase({(int32_t)adj[x].size(), x});
+                    bydeg.erase({(int32_t)adj[y].size(), y});
+                }
+                adj[x].insert(y);
+                adj[y].insert(x);
+                if (!order) {
+                    bydeg.insert({(int32_t)adj[x].size(), x});
+                    bydeg.insert({(int32_t)adj[y].size(), y});
+                }
+                Sset.emplace(std::make_pair(std::max(x, y), std::min(x, y)), -1);
+            }
+        for (int32_t x : nb) {
+            if (!order) bydeg.erase({(int32_t)adj[x].size(), x});
+            adj[x].erase(v);
+            if (!order) bydeg.insert({(int32_t)adj[x].size(), x});
+        }
+        adj[v].clear();
+        nbr[v] = nb;
+        seq.push_back(v);
+    }
+    std::vector<int32_t> pos(n);
+    for (int64_t k = 0; k < n; ++k) pos[seq[k]] = (int32_t)k;
+    // S sorted by (j, i)
+    std::vector<std::pair<int32_t, int32_t>> S(Sset.size());
+    {
+        size_t k = 0;
+        for (const auto &kv : Sset) S[k++] = kv.first;
+        std::sort(S.begin(), S.end(), [](const std::pair<int32_t, int32_t> &x, const std::pair<int32_t, int32_t> &y) {
+            return x.second != y.second ? x.second < y.second : x.first < y.first;
+        });
+        for (size_t q = 0; q < S.size(); ++q) Sset[S[q]] = (int32_t)q;
+    }
+    auto slot_of = [&](int32_t x, int32_t y) { return Sset.at(std::make_pair(std::max(x, y), std::min(x, y))); };
+    // entries: N(v) in elimination order
+    std::vector<int32_t> col_ptr(n + 1, 0);
+    for (int32_t v = 0; v < n; ++v) {
+        std::sort(nbr[v].begin(), nbr[v].end(), [&](int32_t x, int32_t y) { return pos[x] < pos[y]; });
+        col_ptr[v + 1] = col_ptr[v] + (int32_t)nbr[v].size();
+    }
+    const int64_t E = col_ptr[n];
+    std::vector<int32_t> ent_slot(std::max<int64_t>(E, 1)), ent_trans(std::max<int64_t>(E, 1)),
+        ent_src(std::max<int64_t>(E, 1));
+    std::vector<int32_t> slot_src(S.size(), -1);
+    for (const auto &kv : input) slot_src[slot_of((int32_t)(kv.first / n), (int32_t)(kv.first % n))] = kv.second;
+    for (int32_t v = 0; v < n; ++v)
+        for (int32_t a = 0; a < (int32_t)nbr[v].size(); ++a) {
+            const int32_t u = nbr[v][a], ent = col_ptr[v] + a;
+            ent_slot[ent] = slot_of(u, v);
+            ent_trans[ent] = u < v ? 1 : 0;                 // S holds (v, u) = (u, v)^T
+            ent_src[ent] = slot_src[ent_slot[ent]];
+        }
+    // contributions: for k, pairs (v, u) of N(k) with pos[v] <= pos[u] feed target (v, t(u))
+    const int64_t T = E + n;
+    std::vector<int32_t> tcount(T + 1, 0);
+    auto tindex = [&](int32_t v, int32_t u) -> int64_t {
+        if (u == v) return (int64_t)col_ptr[v] + v;
+        const auto &nv = nbr[v];
+        const int32_t a = (int32_t)(std::find(nv.begin(), nv.end(), u) - nv.begin());
+        return (int64_t)col_ptr[v] + v + 1 + a;
+    };
+    std::vector<int32_t> cw, ca;                       // per contribution: W_{u,k} and A'_{v,k} entries
+    for (int pass = 0; pass < 2; ++pass) {             // count per target, then fill
+        std::vector<int32_t> fillp;
+        if (pass == 1) fillp.assign(tcount.begin(), tcount.end() - 1);
+        if (pass == 1) {
+            cw.assign(tcount[T], 0);
+            ca.assign(tcount[T], 0);
+        }
+        for (int64_t sk = 0; sk < n; ++sk) {
+            const int32_t k = seq[sk];
+            const auto &nk = nbr[k];
+            for (int32_t a = 0; a < (int32_t)nk.size(); ++a)
+                for (int32_t c = a; c < (int32_t)nk.size(); ++c) {
+                    const int32_t vv = nk[a], uu = nk[c];           // pos[vv] <= pos[uu]
+                    const int64_t tgt = tindex(vv, uu);
+                    if (pass == 0) {
+                        tcount[tgt + 1]++;
+                    } else {
+                        const int32_t at = fillp[tgt]++;
+                        cw[at] = col_ptr[k] + c;                    // W_{uu,k}
+                        ca[at] = col_ptr[k] + a;                    // A'_{vv,k}
+                    }
+                }
+        }
+        if (pass == 0)
+            for (int64_t q = 0; q < T; ++q) tcount[q + 1] += tcount[q];
+        if (pass == 1) {
+            // tree of the elimination: parent = first-eliminated later neighbour
+            std::vector<int32_t> parent(n, -1), height(n, 0), depth(n, 0);
+            for (int32_t v = 0; v < n; ++v)
+                if (!nbr[v].empty()) parent[v] = nbr[v][0];
+            for (int64_t sk = 0; sk < n; ++sk) {
+                const int32_t v = seq[sk];
+                if (parent[v] >= 0) height[parent[v]] = std::max(height[parent[v]], height[v] + 1);
+            }
+            for (int64_t sk = n - 1; sk >= 0; --sk) {
+                const int32_t v = seq[sk];
+                depth[v] = parent[v] < 0 ? 0 : depth[parent[v]] + 1;
+            }
+            int32_t H = 0, Dm = 0;
+            for (int32_t v = 0; v < n; ++v) {
+                H = std::max(H, height[v]);
+                Dm = std::max(Dm, depth[v]);
+            }
+            std::vector<int64_t> c_off(H + 2, 0), d_off(Dm + 2, 0);
+            for (int32_t v = 0; v < n; ++v) {
+                c_off[height[v] + 1]++;
+                d_off[depth[v] + 1]++;
+            }
+            for (int32_t h = 0; h <= H; ++h) c_off[h + 1] += c_off[h];
+            for (int32_t h = 0; h <= Dm; ++h) d_off[h + 1] += d_off[h];
+            std::vector<int32_t> cn(n), dn(n);
+            {
+                std::vector<int64_t> pc(c_off.begin(), c_off.end() - 1), pd(d_off.begin(), d_off.end() - 1);
+                for (int32_t v = 0; v < n; ++v) {
+                    cn[pc[height[v]]++] = v;
+                    dn[pd[depth[v]]++] = v;
+                }
+            }
+            // distribute pair codes
+            std::vector<int32_t> pair_ptr(n + 1, 0), pair;
+            for (int32_t v = 0; v < n; ++v) pair_ptr[v + 1] = pair_ptr[v] + (int32_t)(nbr[v].size() * nbr[v].size());
+            pair.resize(std::max<int32_t>(pair_ptr[n], 1));
+            for (int32_t v = 0; v < n; ++v) {
+                const auto &nv = nbr[v];
+                const int32_t d = (int32_t)nv.size();
+                for (int32_t a = 0; a < d; ++a)
+                    for (int32_t c = 0; c < d; ++c) {
+                        const int32_t x = nv[a], y = nv[c];
+                        pair[pair_ptr[v] + a * d + c] = x == y ? -(x + 1) : 2 * slot_of(x, y) + (x < y ? 1 : 0);
+                    }
+            }
+            auto *pl = new (std::nothrow) selinv_junction_plan_s();
+            if (!pl) return SELINV_ERR_INVALID_ARG;
+            pl->n = n;
+            pl->m = m;
+            pl->nnz = (int64_t)S.size();
+            pl->E = E;
+            cudaGetDevice(&pl->device);
+            pl->order = seq;
+            pl->S_i.resize(S.size());
+            pl->S_j.resize(S.size());
+            for (size_t q = 0; q < S.size(); ++q) {
+                pl->S_i[q] = S[q].first;
+                pl->S_j[q] = S[q].second;
+            }
+            pl->c_off = c_off;
+            pl->d_off = d_off;
+            bool ok = true;
+            auto up = [&](int32_t **dst, const std::vector<int32_t> &src) {
+                if (!ok) return;
+                const size_t nb = std::max<size_t>(src.size(), 1) * sizeof(int32_t);
+                ok = cudaMalloc(dst, nb) == cudaSuccess &&
+                     (src.empty() || cudaMemcpy(*dst, src.data(), src.size() * sizeof(int32_t),
+                                                cudaMemcpyHostToDevice) == cudaSuccess);
+            };
+            up(&pl->d_c_nodes, cn);
+            up(&pl->d_d_nodes, dn);
+            up(&pl->d_col_ptr, col_ptr);
+            up(&pl->d_ent_slot, ent_slot);
+            up(&pl->d_ent_trans, ent_trans);
+            up(&pl->d_ent_src, ent_src);
+            up(&pl->d_con_ptr, tcount);
+            up(&pl->d_con_w, cw);
+            up(&pl->d_con_a, ca);
+            up(&pl->d_pair_ptr, pair_ptr);
+            up(&pl->d_pair, pair);
+            if (!ok) {
+                selinv_junction_plan_free(pl);
+                return SELINV_ERR_CUDA;
+            }
+            *out = pl;
+        }
+    }
+    return SELINV_OK;
+}
+
+selinv_status selinv_junction_plan_info(const selinv_junction_plan_t *pl, int64_t *nnz_S, int32_t *collect_levels,
+                                        int32_t *distribute_levels)
+{
+    if (!pl) return SELINV_ERR_INVALID_ARG;
+    if (nnz_S) *nnz_S = pl->nnz;
+    if (collect_levels) *collect_levels = (int32_t)pl->c_off.size() - 1;
+    if (distribute_levels) *distribute_levels = (int32_t)pl->d_off.size() - 1;
+    return SELINV_OK;
+}
+
+selinv_status selinv_junction_plan_pattern(const selinv_junction_plan_t *pl, int32_t *S_i, int32_t *S_j,
+                                           int32_t *order)
+{
+    if (!pl) return SELINV_ERR_INVALID_ARG;
+    if (S_i) std::copy(pl->S_i.begin(), pl->S_i.end(), S_i);
+    if (S_j) std::copy(pl->S_j.begin(), pl->S_j.end(), S_j);
+    if (order) std::copy(pl->order.begin(), pl->order.end(), order);
+    return SELINV_OK;
+}
+
+size_t selinv_junction_workspace_size(const selinv_junction_plan_t *pl, selinv_dtype dtype, int32_t b, int64_t batch)
+{
+    if (!pl || (dtype != SELINV_F64 && dtype != SELINV_F32) || b < 1 || b > 16 || batch < 0) return 0;
+    return dtype == SELINV_F64 ? ws_bytes<double>(pl, batch) : ws_bytes<float>(pl, batch);
+}
+
+selinv_status selinv_junction(const selinv_junction_plan_t *pl, selinv_dtype dtype, int32_t b, int64_t batch,
+                              const void *diag, const void *edge_val, void *G_diag, void *G_lower, double *logdet,
+                              int32_t *info, void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!pl || (dtype != SELINV_F64 && dtype != SELINV_F32) || b < 1 || batch < 0) return SELINV_ERR_INVALID_ARG;
+    if (b > 16) return SELINV_ERR_UNSUPPORTED;
+    if (batch == 0) return SELINV_OK;
+    if (!diag || (pl->m > 0 && !edge_val) || !G_diag || (pl->nnz > 0 && !G_lower) || !info)
+        return SELINV_ERR_INVALID_ARG;
+    const size_t es = dtype == SELINV_F64 ? 8 : 4;
+    if (!is_aligned(diag, es) || !is_aligned(edge_val, es) || !is_aligned(G_diag, es) || !is_aligned(G_lower, es) ||
+        !is_aligned(logdet, 8) || !is_aligned(info, 4) || !is_aligned(workspace, 256))
+        return SELINV_ERR_INVALID_ARG;
+    const size_t need = selinv_junction_workspace_size(pl, dtype, b, batch);
+    if (!workspace || workspace_bytes < need) return SELINV_ERR_WORKSPACE;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev != pl->device) return SELINV_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t err;
+    if (dtype == SELINV_F64)
+        err = run_junction<double>(pl, b, batch, static_cast<const double *>(diag), static_cast<const double *>(edge_val),
+                                   static_cast<double *>(G_diag), static_cast<double *>(G_lower), logdet, info,
+                                   workspace, s);
+    else
+        err = run_junction<float>(pl, b, batch, static_cast<const float *>(diag), static_cast<const float *>(edge_val),
+                                  static_cast<float *>(G_diag), static_cast<float *>(G_lower), logdet, info, workspace,
+                                  s);
+    return err == cudaSuccess ? SELINV_OK : SELINV_ERR_CUDA;
+}
+
+}  // extern "C"

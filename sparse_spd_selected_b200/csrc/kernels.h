@@ -77,5 +77,15 @@ template <class T> struct BidiagArgs {
     int b;
 };
 template <class T> cudaError_t bidiag_launch(const BidiagArgs<T> &p, bool aligned16, cudaStream_t s);
+// Its cotangents from the forward's outputs (b <= 16).
+template <class T> struct BidiagBwdArgs {
+    const T *G_diag, *G_lower;      // forward outputs
+    const T *Gb_diag, *Gb_lower;    // their cotangents (null = zero)
+    T *Mb_diag, *Mb_lower;          // cotangents of M_ii and M_{i+1,i}
+    int64_t batch;
+    int64_t L;
+    int b;
+};
+template <class T> cudaError_t bidiag_backward_launch(const BidiagBwdArgs<T> &a, bool aligned16, cudaStream_t s);
 
 }  // namespace selinv

@@ -75,6 +75,8 @@ def lib():
         L.chain_solve.restype = ctypes.c_int
         L.selinv_bidiag.argtypes = [ctypes.c_int, I64, I64, I32, P, P, P, P, P, P]
         L.selinv_bidiag.restype = ctypes.c_int
+        L.selinv_bidiag_backward.argtypes = [ctypes.c_int, I64, I64, I32, P, P, P, P, P, P, P]
+        L.selinv_bidiag_backward.restype = ctypes.c_int
         L.selinv_chain_backward_workspace_size.argtypes = [ctypes.c_int, I64, I64, I32]
         L.selinv_chain_backward_workspace_size.restype = SZ
         L.selinv_chain_backward.argtypes = [ctypes.c_int, I64, I64, I32, P, P, P, P, P, P, P, P, P, P, SZ, P]
@@ -83,6 +85,18 @@ def lib():
         L.selinv_tree_backward_workspace_size.restype = SZ
         L.selinv_tree_backward.argtypes = [P, ctypes.c_int, I32, P, P, P, P, P, P, P, P, P, P, SZ, P]
         L.selinv_tree_backward.restype = ctypes.c_int
+        L.selinv_junction_plan.argtypes = [I64, I64, P, P, P, ctypes.POINTER(P)]
+        L.selinv_junction_plan.restype = ctypes.c_int
+        L.selinv_junction_plan_free.argtypes = [P]
+        L.selinv_junction_plan_free.restype = None
+        L.selinv_junction_plan_info.argtypes = [P, ctypes.POINTER(I64), ctypes.POINTER(I32), ctypes.POINTER(I32)]
+        L.selinv_junction_plan_info.restype = ctypes.c_int
+        L.selinv_junction_plan_pattern.argtypes = [P, P, P, P]
+        L.selinv_junction_plan_pattern.restype = ctypes.c_int
+        L.selinv_junction_workspace_size.argtypes = [P, ctypes.c_int, I32, I64]
+        L.selinv_junction_workspace_size.restype = SZ
+        L.selinv_junction.argtypes = [P, ctypes.c_int, I32, I64, P, P, P, P, P, P, P, SZ, P]
+        L.selinv_junction.restype = ctypes.c_int
         L.selinv_tree_plan.argtypes = [P, I64, I64, ctypes.POINTER(P)]
         L.selinv_tree_plan.restype = ctypes.c_int
         L.selinv_tree_plan_free.argtypes = [P]
@@ -376,6 +390,71 @@ def bidiag(diag, lower=None, *, check=True, out=None, stream=None):
     return {"G_diag": G_diag, "G_lower": G_lower, "info": info}
 
 
+def bidiag_backward(G_diag, G_lower, Gb_diag=None, Gb_lower=None, *, out=None, stream=None):
+    """Cotangents of bidiag (b <= 16) from its outputs G_diag, G_lower and their
+    cotangents (None = zero): returns a dict with Mb_diag and Mb_lower."""
+    _cuda_contig("G_diag", G_diag)
+    dt = G_diag.dtype
+    if G_diag.dim() < 3 or G_diag.shape[-1] != G_diag.shape[-2]:
+        raise ValueError("G_diag must be [..., L, b, b]")
+    lead = tuple(G_diag.shape[:-3])
+    L, b = int(G_diag.shape[-3]), int(G_diag.shape[-1])
+    batch = 1
+    for d in lead:
+        batch *= int(d)
+    shape_l = lead + (max(L - 1, 0), b, b)
+    if Gb_diag is not None:
+        _cuda_contig("Gb_diag", Gb_diag, dt)
+        if Gb_diag.shape != G_diag.shape:
+            raise ValueError("Gb_diag must have G_diag's shape")
+    if L > 1:
+        _cuda_contig("G_lower", G_lower, dt)
+        if tuple(G_lower.shape) != shape_l:
+            raise ValueError(f"G_lower must be {shape_l}")
+        if Gb_lower is not None:
+            _cuda_contig("Gb_lower", Gb_lower, dt)
+            if tuple(Gb_lower.shape) != shape_l:
+                raise ValueError(f"Gb_lower must be {shape_l}")
+    else:
+        G_lower = Gb_lower = None
+    out = dict(out or {})
+    Mb_diag = out.get("Mb_diag")
+    if Mb_diag is None:
+        Mb_diag = torch.empty_like(G_diag)
+    Mb_lower = out.get("Mb_lower")
+    if Mb_lower is None:
+        Mb_lower = torch.empty(shape_l, dtype=dt, device=G_diag.device)
+    with torch.cuda.device(G_diag.device):
+        st = lib().selinv_bidiag_backward(_code(dt), batch, L, b, _ptr(G_diag), _ptr(G_lower), _ptr(Gb_diag),
+                                          _ptr(Gb_lower), _ptr(Mb_diag), _ptr(Mb_lower if L > 1 else None),
+                                          _stream_handle(stream))
+    _check(st, "selinv_bidiag_backward")
+    return {"Mb_diag": Mb_diag, "Mb_lower": Mb_lower}
+
+
+class _BidiagFn(torch.autograd.Function):
+    """G_diag, G_lower = bidiag(diag, lower) with its analytic backward."""
+
+    @staticmethod
+    def forward(ctx, diag, lower):
+        out = bidiag(diag, lower)
+        ctx.save_for_backward(out["G_diag"], out["G_lower"])
+        return out["G_diag"], out["G_lower"]
+
+    @staticmethod
+    def backward(ctx, gb_diag, gb_lower):
+        G_diag, G_lower = ctx.saved_tensors
+        r = bidiag_backward(G_diag, G_lower, None if gb_diag is None else gb_diag.contiguous(),
+                            None if gb_lower is None else gb_lower.contiguous())
+        return r["Mb_diag"], r["Mb_lower"]
+
+
+def bidiag_ad(diag, lower):
+    """Differentiable selected inverse of block lower-bidiagonal matrices (the
+    pages' selinv_bidiag, b <= 16): returns (G_diag, G_lower)."""
+    return _BidiagFn.apply(diag, lower)
+
+
 def chain_backward_workspace_size(dtype, batch, L, b) -> int:
     return int(lib().selinv_chain_backward_workspace_size(_code(dtype), batch, L, b))
 
@@ -461,6 +540,101 @@ def selinv_chain_ad(diag, lower):
     G_lower); gradients reach diag (its lower triangle: the forward reads no
     other entry) and lower through chain_backward."""
     return _SelinvChainFn.apply(diag, lower)
+
+
+class JunctionPlan:
+    """Symbolic analysis of a block-sparse SPD pattern, cached on the device:
+    elimination order (greedy minimum degree unless given), filled pattern S,
+    elimination tree and its levels.  edge_index [2, m] holds the lower blocks
+    (i, j), i > j.  After construction: .order [n] and .S_index [2, nnz_S]
+    (pairs (i, j), i > j, sorted by j then i)."""
+
+    def __init__(self, n, edge_index, order=None):
+        import numpy as np
+        ei = np.ascontiguousarray(np.asarray(edge_index[0], dtype=np.int32))
+        ej = np.ascontiguousarray(np.asarray(edge_index[1], dtype=np.int32))
+        if ei.shape != ej.shape or ei.ndim != 1:
+            raise ValueError("edge_index must be [2, m]")
+        o = None if order is None else np.ascontiguousarray(np.asarray(order, dtype=np.int32))
+        h = ctypes.c_void_p()
+        st = lib().selinv_junction_plan(int(n), ei.size, ei.ctypes.data_as(ctypes.c_void_p),
+                                        ej.ctypes.data_as(ctypes.c_void_p),
+                                        None if o is None else o.ctypes.data_as(ctypes.c_void_p), ctypes.byref(h))
+        _check(st, "selinv_junction_plan")
+        self._h = h
+        self.n, self.m = int(n), int(ei.size)
+        nnz, lc, ld = ctypes.c_int64(), ctypes.c_int32(), ctypes.c_int32()
+        _check(lib().selinv_junction_plan_info(h, ctypes.byref(nnz), ctypes.byref(lc), ctypes.byref(ld)),
+               "selinv_junction_plan_info")
+        self.nnz = int(nnz.value)
+        self.levels = (int(lc.value), int(ld.value))
+        si = np.empty(max(self.nnz, 1), dtype=np.int32)
+        sj = np.empty(max(self.nnz, 1), dtype=np.int32)
+        od = np.empty(self.n, dtype=np.int32)
+        _check(lib().selinv_junction_plan_pattern(h, si.ctypes.data_as(ctypes.c_void_p),
+                                                  sj.ctypes.data_as(ctypes.c_void_p),
+                                                  od.ctypes.data_as(ctypes.c_void_p)), "selinv_junction_plan_pattern")
+        self.S_index = np.stack([si[:self.nnz], sj[:self.nnz]]).astype(np.int64)
+        self.order = od
+
+    @property
+    def handle(self):
+        return self._h
+
+    def workspace_size(self, dtype, b, batch) -> int:
+        return int(lib().selinv_junction_workspace_size(self._h, _code(dtype), b, batch))
+
+    def close(self):
+        if getattr(self, "_h", None) and _lib is not None:
+            _lib.selinv_junction_plan_free(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def junction(plan: JunctionPlan, diag, edge_val, *, check=True, out=None, workspace=None, stream=None):
+    """Selected inverse of general block-sparse SPD matrices on the plan's
+    filled pattern (b <= 16): diag [..., n, b, b], edge_val [..., m, b, b].
+    Returns dict with G_diag, G_lower [..., nnz_S, b, b] on plan.S_index,
+    logdet and info."""
+    _cuda_contig("diag", diag)
+    dt = diag.dtype
+    if diag.dim() < 3 or diag.shape[-1] != diag.shape[-2] or int(diag.shape[-3]) != plan.n:
+        raise ValueError(f"diag must be [..., {plan.n}, b, b]")
+    lead = tuple(diag.shape[:-3])
+    b = int(diag.shape[-1])
+    batch = 1
+    for d in lead:
+        batch *= int(d)
+    _cuda_contig("edge_val", edge_val, dt)
+    if tuple(edge_val.shape) != lead + (plan.m, b, b):
+        raise ValueError(f"edge_val must be {lead + (plan.m, b, b)}")
+    dev = diag.device
+    out = dict(out or {})
+    G_diag = out.get("G_diag")
+    if G_diag is None:
+        G_diag = torch.empty_like(diag)
+    G_lower = out.get("G_lower")
+    if G_lower is None:
+        G_lower = torch.empty(lead + (plan.nnz, b, b), dtype=dt, device=dev)
+    logdet = out.get("logdet")
+    if logdet is None:
+        logdet = torch.empty(lead, dtype=torch.float64, device=dev)
+    info = out.get("info")
+    if info is None:
+        info = torch.empty(lead, dtype=torch.int32, device=dev)
+    nbytes = plan.workspace_size(dt, b, batch)
+    ws = _workspace(nbytes, dev, workspace)
+    with torch.cuda.device(dev):
+        st = lib().selinv_junction(plan.handle, _code(dt), b, batch, _ptr(diag), _ptr(edge_val), _ptr(G_diag),
+                                   _ptr(G_lower), _ptr(logdet), _ptr(info), _ptr(ws), nbytes, _stream_handle(stream))
+    _check(st, "selinv_junction")
+    _raise_on_info(info, check)
+    return {"G_diag": G_diag, "G_lower": G_lower, "S_index": plan.S_index, "logdet": logdet, "info": info}
 
 
 class TreePlan:

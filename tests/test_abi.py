@@ -169,3 +169,30 @@ def test_bidiag_argument_errors(lib):
     assert f(0, 1, 4, 4, FAKE, FAKE, None, FAKE, FAKE, None) == selinv.ERR_INVALID_ARG
     assert f(0, 1, 4, 4, FAKE, FAKE, FAKE, None, FAKE, None) == selinv.ERR_INVALID_ARG
     assert f(0, 0, 4, 4, FAKE, FAKE, FAKE, FAKE, FAKE, None) == selinv.OK
+
+
+def test_bidiag_backward_argument_errors(lib):
+    f = lib.selinv_bidiag_backward
+    # dtype, batch, L, b, G_diag, G_lower, Gb_diag, Gb_lower, Mb_diag, Mb_lower, stream
+    assert f(0, 1, 4, 17, FAKE, FAKE, None, None, FAKE, FAKE, None) == selinv.ERR_UNSUPPORTED
+    assert f(0, 1, 4, 4, None, FAKE, None, None, FAKE, FAKE, None) == selinv.ERR_INVALID_ARG
+    assert f(0, 1, 4, 4, FAKE, FAKE, None, None, FAKE, None, None) == selinv.ERR_INVALID_ARG
+    assert f(0, 0, 4, 4, FAKE, FAKE, None, None, FAKE, FAKE, None) == selinv.OK
+
+
+def test_junction_plan_rejects_bad_patterns(lib):
+    """Pattern and order checks run on the host before anything touches a device."""
+    def plan(ei, ej, n, order=None):
+        a = np.ascontiguousarray(np.asarray(ei, dtype=np.int32))
+        c = np.ascontiguousarray(np.asarray(ej, dtype=np.int32))
+        o = None if order is None else np.ascontiguousarray(np.asarray(order, dtype=np.int32))
+        h = ctypes.c_void_p()
+        return lib.selinv_junction_plan(n, a.size, a.ctypes.data_as(ctypes.c_void_p), c.ctypes.data_as(ctypes.c_void_p),
+                                        None if o is None else o.ctypes.data_as(ctypes.c_void_p), ctypes.byref(h))
+    assert plan([0], [1], 3) == selinv.ERR_INVALID_ARG             # i < j
+    assert plan([1], [1], 3) == selinv.ERR_INVALID_ARG             # diagonal
+    assert plan([3], [0], 3) == selinv.ERR_INVALID_ARG             # out of range
+    assert plan([2, 2], [1, 1], 3) == selinv.ERR_INVALID_ARG       # repeated block
+    assert plan([1], [0], 3, order=[0, 0, 1]) == selinv.ERR_INVALID_ARG   # not a permutation
+    assert lib.selinv_junction(None, 0, 4, 1, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 1 << 30, None) == \
+        selinv.ERR_INVALID_ARG

@@ -1,0 +1,88 @@
+"""General block-sparse SPD matrices on the GPU (selinv_junction, b <= 16)
+against the oracle: the plan's elimination order and filled pattern S must
+equal the oracle's symbolic elimination exactly, and every block of A^-1 on
+S its dense inverse, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_spd_selected_b200 import inputs, selinv
+from tests.parity import TOL, host, logdet_err, to_dev, worst
+
+pytestmark = pytest.mark.gpu
+
+
+def random_pattern(n, m, seed):
+    rng = np.random.default_rng(seed)
+    pairs = sorted({(max(a, c), min(a, c)) for a, c in rng.integers(0, n, (m, 2)) if a != c})
+    return np.array(pairs, dtype=np.int64).T.reshape(2, -1)
+
+
+def run(n, E, b, seed, dtype, lead=(2,), order=None, load=1.0):
+    batch = int(np.prod(lead))
+    d, e = inputs.graph_inputs(batch, n, b, E, seed=seed, load=load)
+    d = d.reshape(lead + (n, b, b))
+    e = e.reshape(lead + (E.shape[1], b, b))
+    plan = selinv.JunctionPlan(n, E, order)
+    o_ref, S_ref = oracle.junction_symbolic(n, E, order)
+    assert plan.order.tolist() == o_ref.tolist()
+    assert np.array_equal(plan.S_index, S_ref)
+    dd, ee = to_dev(d, dtype), to_dev(e, dtype)
+    out = selinv.junction(plan, dd, ee)
+    ref = oracle.junction(host(dd), E, host(ee), order)
+    assert (ref["info"] == -1).all()
+    nl = len(lead)
+    assert worst(host(out["G_diag"]), ref["G_diag"], nl) <= TOL[dtype]
+    if plan.nnz:
+        assert worst(host(out["G_lower"]), ref["G_lower"], nl) <= TOL[dtype]
+    assert logdet_err(host(out["logdet"]), ref["logdet"]) <= TOL[dtype]
+    assert (host(out["info"]) == -1).all()
+    return plan
+
+
+@pytest.mark.parametrize("b", [1, 2, 5, 16])
+def test_junction_grid_3x3(cuda_ok, b):
+    """The pages' loopy 3 x 3 grid: S grows past the input pattern."""
+    E = inputs.grid_edges(3, 3)
+    plan = run(9, E, b, 11000 + b, torch.float64)
+    assert plan.nnz > E.shape[1]
+
+
+@pytest.mark.parametrize("b", [1, 3, 8, 16])
+@pytest.mark.parametrize("n,m", [(12, 20), (40, 90)])
+def test_junction_random_graphs(cuda_ok, b, n, m):
+    run(n, random_pattern(n, m, 11100 + n + b), b, 11200 + n + b, torch.float64)
+
+
+def test_junction_given_order_tree_and_single_node(cuda_ok):
+    E = inputs.grid_edges(4, 5)
+    run(20, E, 4, 11300, torch.float64, order=np.arange(20)[::-1].copy())
+    parent = inputs.random_parent(np.random.default_rng(5), 30)
+    T = np.array([[max(v, p) for v, p in enumerate(parent) if p >= 0],
+                  [min(v, p) for v, p in enumerate(parent) if p >= 0]])
+    plan = run(30, T, 6, 11301, torch.float64)
+    assert plan.nnz == T.shape[1]                       # a tree has no fill
+    run(1, np.zeros((2, 0), dtype=np.int64), 7, 11302, torch.float64)
+
+
+def test_junction_f32_and_leading_dims(cuda_ok):
+    run(16, inputs.grid_edges(4, 4), 16, 11400, torch.float32, lead=(3,), load=2.0)
+    run(12, random_pattern(12, 25, 3), 4, 11401, torch.float64, lead=(2, 3))
+
+
+def test_junction_grid_16x16(cuda_ok):
+    """A 16 x 16 lattice of blocks of 4 (N = 1024), three matrices."""
+    run(256, inputs.grid_edges(16, 16), 4, 11500, torch.float64, lead=(3,))
+
+
+def test_junction_not_spd(cuda_ok):
+    E = inputs.grid_edges(3, 4)
+    d, e = inputs.graph_inputs(2, 12, 3, E, seed=11600, load=1.0)
+    d[1, 5] = -np.eye(3)
+    plan = selinv.JunctionPlan(12, E)
+    out = selinv.junction(plan, to_dev(d, torch.float64), to_dev(e, torch.float64), check=False)
+    info = host(out["info"])
+    assert info[0] == -1 and info[1] >= 0
+    with pytest.raises(selinv.NotSPDError):
+        selinv.junction(plan, to_dev(d, torch.float64), to_dev(e, torch.float64))
