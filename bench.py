@@ -49,6 +49,7 @@ KERNEL_SOURCES = {
     "chain_backward_kernel": ["chain_backward.cu", "warp16.cuh", "common.cuh"],
     "tree_bw_collect_kernel": ["tree.cu", "warp16.cuh", "common.cuh"],
     "bidiag_kernel": ["bidiag.cu", "common.cuh"],
+    "junction_collect_kernel": ["junction.cu", "warp16.cuh", "common.cuh"],
 }
 
 
@@ -179,6 +180,8 @@ def oracle_run(oracle, w, g, op):
         oracle.tree_backward(g["parent"], g["diag"], g["edge"], g["Gb_diag"], g["Gb_edge"])
     elif w.kind == "tree":
         oracle.tree(g["parent"], g["diag"], g["edge"])
+    elif w.kind == "junction":
+        oracle.junction(g["diag"], g["edge_index"], g["edge_val"])
     elif op == "sample":
         oracle.chain_sample(g["diag"], g["lower"], g["z"], rhs=g.get("rhs"))
     elif op == "backward":
@@ -193,6 +196,10 @@ def oracle_workload(w, op):
     """The workload the oracle times: the same, except for the backward, whose
     dense definition costs O((L b)^3) per chain or tree: there chains or trees
     of 512 / b blocks drawn by the same recipe stand in (a few seconds each)."""
+    if w.kind == "junction" and w.L * w.b > 512:
+        side = max(2, int((512 // w.b) ** 0.5))
+        return (dataclasses.replace(w, L=side * side),
+                f" (lattices of {side} x {side} blocks drawn like {w.name}'s: the dense definition is O((n b)^3))")
     if op in ("backward", "bidiag") and w.L * w.b > 512:
         n = max(2, 512 // w.b)
         what = "trees" if w.kind == "tree" else "chains"
@@ -228,11 +235,51 @@ def cpu_baseline(w, dtype_name, op="selinv", budget_s=10.0):
             "sample": f"{len(elems)} of {w.batch} {unit_name} ({w.name}, float64){note}, {dt:.2f} s"}
 
 
+_JPLAN = {}
+
+
+def _lattice_plan(w):
+    """The junction plan of a lattice workload (cached; built on the current device)."""
+    if w.name not in _JPLAN:
+        from sparse_spd_selected_b200 import selinv
+        side = int(round(w.L ** 0.5))
+        _JPLAN[w.name] = selinv.JunctionPlan(w.L, inputs.grid_edges(side, w.L // side))
+    return _JPLAN[w.name]
+
+
+def _lattice_m(w):
+    side = int(round(w.L ** 0.5))
+    return inputs.grid_edges(side, w.L // side).shape[1]
+
+
+def _lattice_nnz(w):
+    return _lattice_plan(w).nnz
+
+
+def junction_flops(w, batch):
+    """Nominal flops of the general sparse path: 2 b^3 per block product it takes.
+    Per node v with clique N(v) (d = |N(v)|): d(d + 1)/2 updates it sends to
+    its ancestors' blocks, d products W = A' P, d^2 + d products in the
+    distribute; plus b^3 for the inverse of S_v."""
+    import numpy as np
+    pl = _lattice_plan(w)
+    pos = np.empty(w.L, dtype=np.int64)
+    pos[pl.order] = np.arange(w.L)
+    i, j = pl.S_index
+    later = np.where(pos[i] > pos[j], j, i)          # the earlier-eliminated end owns the pair
+    d = np.bincount(later, minlength=w.L).astype(np.float64)
+    prods = d * (d + 1) / 2 + d + d * d + d
+    return batch * (2.0 * w.b ** 3 * prods.sum() + w.L * float(w.b) ** 3)
+
+
 def algorithmic_bytes(w, es, batch, op="selinv"):
     """Bytes the method must move: read D and B (or edge) blocks, write G_diag and G_lower
     (or G_edge) blocks, plus the right-hand side and solution when solving.  A draw reads
     D, B, r and z and writes eta (a tree draw has no r)."""
     b2 = w.b * w.b
+    if w.kind == "junction":
+        # read D and the input blocks, write G_diag and G on the filled pattern S
+        return es * b2 * batch * (2 * w.L + _lattice_m(w) + _lattice_nnz(w))
     if op == "bidiag":
         # read M_ii and M_{i+1,i}, write G_ii and G_{i+1,i}
         nodes, edges = batch * w.L, batch * (w.L - 1)
@@ -260,7 +307,10 @@ def algorithmic_bytes(w, es, batch, op="selinv"):
 def algorithmic_flops(w, batch, op="selinv"):
     """Nominal 7 b^3 flops per block: collect (Cholesky b^3/3 + trsm b^3 + syrk b^3) and
     distribute (inverse 2b^3/3 + trmm b^3 + gemm 2b^3 + symmetric half-gemm b^3).  A draw
-    needs the collect only (7 b^3 / 3; its triangular solves are O(b^2))."""
+    needs the collect only (7 b^3 / 3; its triangular solves are O(b^2)).  The general
+    sparse path counts its own products (junction_flops)."""
+    if w.kind == "junction":
+        return junction_flops(w, batch)
     # backward: the collect's 7/3 b^3, then six products in the reversed distribute
     # step and five in the reversed collect step, 2 b^3 each
     per = {"sample": 7.0 / 3.0, "backward": 73.0 / 3.0}.get(op, 7.0)
@@ -322,7 +372,7 @@ def run_reference(args):
     import oracle
     oracle.build()
     w, note = oracle_workload(w, args.op)
-    n_per_step = {"chain": 64, "tree": 1, "grid": 1}[w.kind]
+    n_per_step = {"chain": 64, "tree": 1, "grid": 1, "junction": 4}[w.kind]
     if w.kind == "chain" and w.L * w.b ** 3 > 64 * 16 ** 3 * 64:
         n_per_step = 2
     if args.op in ("backward", "bidiag") and w.kind == "chain":
@@ -413,11 +463,23 @@ def run_ours(args):
             else:
                 g["Gb_diag"], g["Gb_lower"] = inputs.cotangents(w.batch, w.L, w.b, w.seed, elems)
         host_in = {k: torch.from_numpy(v).to(tdt).pin_memory() for k, v in g.items()
-                   if v is not None and k != "parent"}
+                   if v is not None and k not in ("parent", "edge_index")}
         dev_in = {k: v.to("cuda", non_blocking=True) for k, v in host_in.items()}
         torch.cuda.synchronize()
 
-    if w.kind == "tree":
+    if w.kind == "junction":
+        plan = _lattice_plan(w)
+        kernel = "junction_collect_kernel"
+        launches_per_step = plan.launches
+        out = {"G_diag": torch.empty_like(dev_in["diag"]),
+               "G_lower": torch.empty((batch, plan.nnz, w.b, w.b), dtype=tdt, device="cuda"),
+               "logdet": torch.empty(batch, dtype=torch.float64, device="cuda"),
+               "info": torch.empty(batch, dtype=torch.int32, device="cuda")}
+        ws = torch.empty(plan.workspace_size(tdt, w.b, batch), dtype=torch.uint8, device="cuda")
+
+        def step():
+            selinv.junction(plan, dev_in["diag"], dev_in["edge_val"], check=False, out=out, workspace=ws)
+    elif w.kind == "tree":
         plan = selinv.TreePlan(g["parent"])
         # init, collect sweep, distribute sweep (trees with more than one node), log-det finalize
         launches_per_step = 4 if w.L > 1 else 3
@@ -585,7 +647,9 @@ def run_ours(args):
     flop_rate = flops / (kernel_ms / 1e3) / 1e12
     traffic = profiled_traffic(kernel, w.name) if full_size else None
     hbm_src = f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback 6650 GB/s"
-    if (w.b >= 32 or args.op == "backward") and args.dtype == "f64":
+    ridge = 35.5e12 / (hbm * 1e9)                      # FP64 flop per byte where the two roofs meet
+    contraction = w.kind == "junction" and flops / byt > ridge
+    if (w.b >= 32 or args.op == "backward" or contraction) and args.dtype == "f64":
         # arithmetic intensity 7 b^3 / (32 b^2) flop/byte: past the FP64 ridge from b = 32 on
         peak = fp64_peak_tflops(torch)
         roof = {"bound": "tensor", "achieved": flop_rate, "peak": peak, "unit": "TFLOP/s",

@@ -300,7 +300,8 @@ selinv_status selinv_chain_noalloc(selinv_dtype dtype, int64_t batch, int64_t L,
  *   logdet [batch] (may be NULL), info [batch]: -1, or a node whose Schur
  *   complement is not positive definite (outputs then unspecified)
  * Workspace: selinv_junction_workspace_size(plan, dtype, b, batch) bytes.
- * One launch per level of each sweep.
+ * Each level of the collect is three launches (target blocks, inverses,
+ * W products), each level of the distribute two (clique columns, diagonals).
  */
 typedef struct selinv_junction_plan_s selinv_junction_plan_t;
 
@@ -311,6 +312,8 @@ selinv_status selinv_junction_plan_info(const selinv_junction_plan_t *plan, int6
                                         int32_t *collect_levels, int32_t *distribute_levels);
 selinv_status selinv_junction_plan_pattern(const selinv_junction_plan_t *plan, int32_t *S_i, int32_t *S_j,
                                            int32_t *order);
+/* Kernel launches one selinv_junction call makes with this plan (-1 for NULL). */
+int64_t selinv_junction_plan_launches(const selinv_junction_plan_t *plan);
 size_t selinv_junction_workspace_size(const selinv_junction_plan_t *plan, selinv_dtype dtype, int32_t b,
                                       int64_t batch);
 selinv_status selinv_junction(const selinv_junction_plan_t *plan, selinv_dtype dtype, int32_t b, int64_t batch,

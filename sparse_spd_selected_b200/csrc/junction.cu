@@ -15,8 +15,13 @@
 //     G_{u,v} = -sum_{l in N(v)} G_{u,l} W_{l,v}   (u in N(v)),
 //     G_{v,v} = P_v - sum_{l in N(v)} W_{l,v}^T G_{l,v}.
 // All k above are descendants of v in the elimination tree and all u, l are
-// ancestors, so each sweep runs one launch per tree level (heights for the
-// collect, depths for the distribute), one warp per (node, matrix) item.
+// ancestors, so each sweep goes level by level (heights for the collect,
+// depths for the distribute).  A level of the collect is three launches: one
+// 4-warp CTA per target block (the warps split its contributions and add
+// their partial sums in a fixed order), one warp per node for P_v, one warp
+// per clique entry for W; a level of the distribute is two: one CTA per
+// clique entry for G_{u,v}, one CTA per node for G_vv.  Wide cliques near the
+// root so spread over many CTAs instead of one warp.
 // The host plan holds the symbolic work: order, fill, the tree and its
 // levels, the index lists of every contribution and of every G_{u,l} a
 // clique reads.  Off-diagonal blocks of S are stored as (i, j), i > j, in the
@@ -48,6 +53,11 @@ struct selinv_junction_plan_s {
     int32_t *d_con_w = nullptr, *d_con_a = nullptr;   // entries of W_{u,k} and A'_{v,k}
     int32_t *d_pair_ptr = nullptr;              // [n+1] into pair codes (|N(v)|^2 per node)
     int32_t *d_pair = nullptr;                  // -(w+1): diagonal of node w; else 2 * slot + transposed
+    // per-level work lists: collect targets (node, t), collect entries (entry, node),
+    // distribute entries (entry, node, index in N(node))
+    std::vector<int64_t> ct_off, ce_off, de_off;
+    int32_t *d_ct_node = nullptr, *d_ct_t = nullptr, *d_ce_ent = nullptr, *d_ce_node = nullptr;
+    int32_t *d_de_ent = nullptr, *d_de_node = nullptr, *d_de_a = nullptr;
 };
 
 namespace selinv {
@@ -118,112 +128,210 @@ template <class T> SELINV_DEVINL void st_blk(T *M, const w16::Tile<T> &a, int b,
         }
 }
 
+// Four warps split one sum of tile products; warps 1..3 leave their partial
+// tiles in shared memory and warp 0 adds them in a fixed order, so the result
+// does not depend on timing.  Returns true in warp 0, which holds the total.
+template <class T> SELINV_DEVINL bool reduce4(w16::Tile<T> &acc, T *img, int wid, int g, int t)
+{
+    constexpr int EL = w16::SL<T>::ELEMS;
+    if (wid > 0) w16::to_smem<T>(img + (wid - 1) * EL, acc, g, t);
+    __syncthreads();
+    if (wid != 0) return false;
+#pragma unroll
+    for (int k = 0; k < JWARPS - 1; ++k) {
+        w16::Tile<T> u;
+        w16::from_smem<T>(u, img + k * EL, g, t);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc.v[h][q] += u.v[h][q];
+    }
+    return true;
+}
+
+template <class T> __host__ __device__ constexpr int j_smem_elems()
+{
+    return (JWARPS - 1) * w16::SL<T>::ELEMS + JWARPS * (2 * w16::SL<T>::ELEMS + 32);
+}
+
+// Collect, one CTA per target block (v, t) of a level: t = 0 is S_v, t >= 1
+// is A'_{u,v} for u = N(v)[t-1]; the warps split the contributions
+// -W_{u,k} A'_{v,k}^T listed by the plan.
 template <class T>
 __global__ void __launch_bounds__(JWARPS * 32)
-junction_collect_kernel(JBufs<T> p, JDev jd, const int32_t *nodes, int64_t count, int64_t batch)
+jn_target_kernel(JBufs<T> p, JDev jd, const int32_t *tnode, const int32_t *tt, int64_t count)
 {
     using namespace w16;
     constexpr int EL = SL<T>::ELEMS;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    T *s1 = reinterpret_cast<T *>(smem_raw) + wid * (2 * EL + 32), *s2 = s1 + EL, *cb = s2 + EL;
-    const int64_t item = (int64_t)blockIdx.x * JWARPS + wid;
-    if (item >= count * batch) return;                 // the whole warp leaves together
-    const int32_t v = nodes[item % count];
+    T *img = reinterpret_cast<T *>(smem_raw);
+    T *s1 = img + (JWARPS - 1) * EL + wid * (2 * EL + 32), *s2 = s1 + EL;
+    const int64_t item = blockIdx.x;
+    const int32_t v = tnode[item % count], tg = tt[item % count];
     const int64_t e = item / count;
     const int b = p.b;
     const int64_t bb = (int64_t)b * b;
-    const int32_t c0 = jd.col_ptr[v], c1 = jd.col_ptr[v + 1];
-    const int64_t tb = (int64_t)c0 + v;               // first target of v
-    T *Ap = p.Ap + e * jd.E * JSLOT, *W = p.W + e * jd.E * JSLOT;
-    Tile<T> S;
-    for (int32_t tt = 0; tt <= c1 - c0; ++tt) {
-        Tile<T> acc;
-        if (tt == 0) {
-            load_sym<T, false>(acc, p.diag + (e * jd.n + v) * bb, b, g, t);
-        } else {
-            const int32_t ent = c0 + tt - 1, src = jd.ent_src[ent];
-            if (src >= 0) ld_blk<T>(acc, p.edge + (e * jd.m + src) * bb, b, g, t, jd.ent_trans[ent] != 0, false);
-            else zero(acc);
-        }
-        for (int32_t c = jd.con_ptr[tb + tt]; c < jd.con_ptr[tb + tt + 1]; ++c) {
-            Tile<T> w, a;
-            ld_ws<T>(w, W + (int64_t)jd.con_w[c] * JSLOT, g, t, false);
-            ld_ws<T>(a, Ap + (int64_t)jd.con_a[c] * JSLOT, g, t, false);
-            gemm_nt<true>(acc, w, a, s1, s2, g, t);          // -= W_{u,k} A'_{v,k}^T
-        }
-        if (tt == 0) S = acc;
-        else st_ws<T>(Ap + (int64_t)(c0 + tt - 1) * JSLOT, acc, g, t);
+    const int32_t c0 = jd.col_ptr[v];
+    const int64_t tau = (int64_t)c0 + v + tg;
+    const T *Ap = p.Ap + e * jd.E * JSLOT, *W = p.W + e * jd.E * JSLOT;
+    Tile<T> acc;
+    zero(acc);
+    for (int32_t c = jd.con_ptr[tau] + wid; c < jd.con_ptr[tau + 1]; c += JWARPS) {
+        Tile<T> w, a;
+        ld_ws<T>(w, W + (int64_t)jd.con_w[c] * JSLOT, g, t, false);
+        ld_ws<T>(a, Ap + (int64_t)jd.con_a[c] * JSLOT, g, t, false);
+        gemm_nt<true>(acc, w, a, s1, s2, g, t);              // -= W_{u,k} A'_{v,k}^T
     }
+    if (!reduce4<T>(acc, img, wid, g, t)) return;
+    Tile<T> a0;
+    if (tg == 0) {
+        load_sym<T, false>(a0, p.diag + (e * jd.n + v) * bb, b, g, t);
+    } else {
+        const int32_t ent = c0 + tg - 1, src = jd.ent_src[ent];
+        if (src >= 0) ld_blk<T>(a0, p.edge + (e * jd.m + src) * bb, b, g, t, jd.ent_trans[ent] != 0, false);
+        else zero(a0);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc.v[h][q] += a0.v[h][q];
+    if (tg == 0) st_ws<T>(p.Sinv + (e * jd.n + v) * JSLOT, acc, g, t);      // S_v, inverted next
+    else st_ws<T>(p.Ap + (e * jd.E + c0 + tg - 1) * JSLOT, acc, g, t);
+}
+
+// One warp per node of a level: P_v = S_v^-1 in place, log det, info.
+template <class T>
+__global__ void __launch_bounds__(JWARPS * 32)
+jn_inverse_kernel(JBufs<T> p, JDev jd, const int32_t *nodes, int64_t count, int64_t batch)
+{
+    using namespace w16;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    T *cb = reinterpret_cast<T *>(smem_raw) + wid * 32;
+    const int64_t item = (int64_t)blockIdx.x * JWARPS + wid;
+    if (item >= count * batch) return;
+    const int32_t v = nodes[item % count];
+    const int64_t e = item / count;
+    T *slot = p.Sinv + (e * jd.n + v) * JSLOT;
+    Tile<T> S;
+    ld_ws<T>(S, slot, g, t, false);
     mirror_upper(S, g, t);
     LogAcc det;
     det.init();
     bool bad = false;
-    spd_inverse<T>(S, cb, g, t, det, bad);              // S = P_v
+    spd_inverse<T>(S, cb, g, t, det, bad);
     if (lane == 0) {
         p.ld[e * jd.n + v] = det.log_value();
         if (bad) atomicMin(p.info + e, v);
     }
-    st_ws<T>(p.Sinv + (e * jd.n + v) * JSLOT, S, g, t);
     __syncwarp();
-    for (int32_t ent = c0; ent < c1; ++ent) {         // W_{u,v} = A'_{u,v} P_v
-        Tile<T> a, w;
-        ld_ws<T>(a, Ap + (int64_t)ent * JSLOT, g, t, false);
-        zero(w);
-        gemm_nt<false>(w, a, S, s1, s2, g, t);
-        st_ws<T>(W + (int64_t)ent * JSLOT, w, g, t);
-    }
+    st_ws<T>(slot, S, g, t);
 }
 
+// One warp per clique entry (u, v) of a level: W_{u,v} = A'_{u,v} P_v.
 template <class T>
 __global__ void __launch_bounds__(JWARPS * 32)
-junction_distribute_kernel(JBufs<T> p, JDev jd, const int32_t *nodes, int64_t count, int64_t batch)
+jn_w_kernel(JBufs<T> p, JDev jd, const int32_t *ents, const int32_t *enodes, int64_t count, int64_t batch)
 {
     using namespace w16;
     constexpr int EL = SL<T>::ELEMS;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    T *s0 = reinterpret_cast<T *>(smem_raw) + wid * (3 * EL + 32), *s1 = s0 + EL, *s2 = s1 + EL;
+    T *s1 = reinterpret_cast<T *>(smem_raw) + wid * 2 * EL, *s2 = s1 + EL;
     const int64_t item = (int64_t)blockIdx.x * JWARPS + wid;
     if (item >= count * batch) return;
+    const int32_t ent = ents[item % count], v = enodes[item % count];
+    const int64_t e = item / count;
+    Tile<T> a, P, w;
+    ld_ws<T>(a, p.Ap + (e * jd.E + ent) * JSLOT, g, t, false);
+    ld_ws<T>(P, p.Sinv + (e * jd.n + v) * JSLOT, g, t, false);
+    zero(w);
+    gemm_nt<false>(w, a, P, s1, s2, g, t);                   // P symmetric
+    st_ws<T>(p.W + (e * jd.E + ent) * JSLOT, w, g, t);
+}
+
+// Distribute, one CTA per clique entry (u, v) of a level:
+// G_{u,v} = -sum_{l in N(v)} G_{u,l} W_{l,v}, the warps splitting l.
+template <class T>
+__global__ void __launch_bounds__(JWARPS * 32)
+jn_gcol_kernel(JBufs<T> p, JDev jd, const int32_t *ents, const int32_t *enodes, const int32_t *eidx, int64_t count)
+{
+    using namespace w16;
+    constexpr int EL = SL<T>::ELEMS;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    T *img = reinterpret_cast<T *>(smem_raw);
+    T *s1 = img + (JWARPS - 1) * EL + wid * (2 * EL + 32), *s2 = s1 + EL;
+    const int64_t item = blockIdx.x;
+    const int32_t ent = ents[item % count], v = enodes[item % count], a = eidx[item % count];
+    const int64_t e = item / count;
+    const int b = p.b;
+    const int64_t bb = (int64_t)b * b;
+    const int32_t c0 = jd.col_ptr[v], d = jd.col_ptr[v + 1] - c0;
+    const T *W = p.W + e * jd.E * JSLOT;
+    const T *Gd = p.G_diag + e * jd.n * bb, *Gl = p.G_lower + e * jd.nnz * bb;
+    const int32_t *pc = jd.pair + jd.pair_ptr[v] + (int64_t)a * d;
+    Tile<T> acc;
+    zero(acc);
+    for (int32_t c = wid; c < d; c += JWARPS) {
+        const int32_t code = pc[c];
+        Tile<T> gul, wt;
+        if (code < 0) ld_blk<T>(gul, Gd + (int64_t)(-code - 1) * bb, b, g, t, false, true);
+        else ld_blk<T>(gul, Gl + (int64_t)(code >> 1) * bb, b, g, t, (code & 1) != 0, true);
+        ld_ws<T>(wt, W + (int64_t)(c0 + c) * JSLOT, g, t, true);           // W_{l,v}^T
+        gemm_nt<true>(acc, gul, wt, s1, s2, g, t);                        // -= G_{u,l} W_{l,v}
+    }
+    if (!reduce4<T>(acc, img, wid, g, t)) return;
+    st_blk<T>(p.G_lower + (e * jd.nnz + jd.ent_slot[ent]) * bb, acc, b, g, t, jd.ent_trans[ent] != 0);
+}
+
+// One CTA per node of a level: G_vv = P_v - sum_{l in N(v)} W_{l,v}^T G_{l,v},
+// the warps splitting l; written exactly symmetric.
+template <class T>
+__global__ void __launch_bounds__(JWARPS * 32)
+jn_gdiag_kernel(JBufs<T> p, JDev jd, const int32_t *nodes, int64_t count)
+{
+    using namespace w16;
+    constexpr int EL = SL<T>::ELEMS;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    T *img = reinterpret_cast<T *>(smem_raw);
+    T *s1 = img + (JWARPS - 1) * EL + wid * (2 * EL + 32), *s2 = s1 + EL;
+    const int64_t item = blockIdx.x;
     const int32_t v = nodes[item % count];
     const int64_t e = item / count;
     const int b = p.b;
     const int64_t bb = (int64_t)b * b;
     const int32_t c0 = jd.col_ptr[v], d = jd.col_ptr[v + 1] - c0;
     const T *W = p.W + e * jd.E * JSLOT;
-    T *Gd = p.G_diag + e * jd.n * bb, *Gl = p.G_lower + e * jd.nnz * bb;
-    Tile<T> gvv;
-    ld_ws<T>(gvv, p.Sinv + (e * jd.n + v) * JSLOT, g, t, false);
-    const int32_t *pc = jd.pair + jd.pair_ptr[v];
-    for (int32_t a = 0; a < d; ++a) {                  // G_{u,v}, u = N(v)[a]
-        Tile<T> acc;
-        zero(acc);
-        for (int32_t c = 0; c < d; ++c) {
-            const int32_t code = pc[a * d + c];
-            Tile<T> gul, wt;
-            if (code < 0) ld_blk<T>(gul, Gd + (int64_t)(-code - 1) * bb, b, g, t, false, true);
-            else ld_blk<T>(gul, Gl + (int64_t)(code >> 1) * bb, b, g, t, (code & 1) != 0, true);
-            ld_ws<T>(wt, W + (int64_t)(c0 + c) * JSLOT, g, t, true);     // W_{l,v}^T
-            gemm_nt<true>(acc, gul, wt, s1, s2, g, t);                  // -= G_{u,l} W_{l,v}
-        }
-        const int32_t ent = c0 + a;
-        st_blk<T>(Gl + (int64_t)jd.ent_slot[ent] * bb, acc, b, g, t, jd.ent_trans[ent] != 0);
-        Tile<T> accT, wt;                              // G_vv -= W_{u,v}^T G_{u,v}
-        to_smem<T>(s0, acc, g, t);
-        __syncwarp();
-        from_smem_T<T>(accT, s0, g, t);
-        __syncwarp();
-        ld_ws<T>(wt, W + (int64_t)ent * JSLOT, g, t, true);
-        gemm_nt<true>(gvv, wt, accT, s1, s2, g, t);
+    const T *Gl = p.G_lower + e * jd.nnz * bb;
+    Tile<T> acc;
+    zero(acc);
+    for (int32_t c = wid; c < d; c += JWARPS) {
+        const int32_t ent = c0 + c;
+        Tile<T> wt, glT;
+        ld_ws<T>(wt, W + (int64_t)ent * JSLOT, g, t, true);                 // W_{l,v}^T
+        ld_blk<T>(glT, Gl + (int64_t)jd.ent_slot[ent] * bb, b, g, t, jd.ent_trans[ent] == 0, true);   // G_{l,v}^T
+        gemm_nt<true>(acc, wt, glT, s1, s2, g, t);                          // -= W^T G
     }
-    to_smem<T>(s0, gvv, g, t);                         // exactly symmetric from the lower triangle
+    if (!reduce4<T>(acc, img, wid, g, t)) return;
+    Tile<T> P;
+    ld_ws<T>(P, p.Sinv + (e * jd.n + v) * JSLOT, g, t, false);
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc.v[h][q] += P.v[h][q];
+    to_smem<T>(img, acc, g, t);                       // exactly symmetric from the lower triangle
     __syncwarp();
-    from_smem_lower<T>(gvv, s0, g, t);
+    from_smem_lower<T>(acc, img, g, t);
     __syncwarp();
-    st_blk<T>(Gd + (int64_t)v * bb, gvv, b, g, t, false);
+    st_blk<T>(p.G_diag + (e * jd.n + v) * bb, acc, b, g, t, false);
 }
 
 __global__ void junction_init(int32_t *info, int64_t batch)
@@ -275,22 +383,32 @@ cudaError_t run_junction(const selinv_junction_plan_s *pl, int b, int64_t batch,
     const unsigned ib = (unsigned)ceil_div(batch, 256);
     junction_init<<<ib, 256, 0, s>>>(info, batch);
     constexpr int EL = w16::SL<T>::ELEMS;
-    const size_t smem_c = sizeof(T) * (2 * EL + 32) * JWARPS, smem_d = sizeof(T) * (3 * EL + 32) * JWARPS;
-    cudaError_t err = cudaFuncSetAttribute(junction_collect_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)smem_c);
-    if (err == cudaSuccess)
-        err = cudaFuncSetAttribute(junction_distribute_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)smem_d);
+    const size_t smem_r = sizeof(T) * j_smem_elems<T>();           // CTA-per-item kernels
+    const size_t smem_w = sizeof(T) * JWARPS * 2 * EL, smem_i = sizeof(T) * JWARPS * 32;
+    cudaError_t err = cudaSuccess;
+    for (auto k : {(const void *)jn_target_kernel<T>, (const void *)jn_gcol_kernel<T>, (const void *)jn_gdiag_kernel<T>})
+        if (err == cudaSuccess) err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_r);
+    if (err == cudaSuccess) err = cudaFuncSetAttribute(jn_w_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_w);
     if (err != cudaSuccess) return err;
     for (size_t l = 0; l + 1 < pl->c_off.size(); ++l) {
-        const int64_t cnt = pl->c_off[l + 1] - pl->c_off[l];
-        junction_collect_kernel<T><<<(unsigned)ceil_div(cnt * batch, JWARPS), JWARPS * 32, smem_c, s>>>(
-            p, jd, pl->d_c_nodes + pl->c_off[l], cnt, batch);
+        const int64_t nt = pl->ct_off[l + 1] - pl->ct_off[l];
+        const int64_t nn = pl->c_off[l + 1] - pl->c_off[l];
+        const int64_t ne = pl->ce_off[l + 1] - pl->ce_off[l];
+        jn_target_kernel<T><<<(unsigned)(nt * batch), JWARPS * 32, smem_r, s>>>(
+            p, jd, pl->d_ct_node + pl->ct_off[l], pl->d_ct_t + pl->ct_off[l], nt);
+        jn_inverse_kernel<T><<<(unsigned)ceil_div(nn * batch, JWARPS), JWARPS * 32, smem_i, s>>>(
+            p, jd, pl->d_c_nodes + pl->c_off[l], nn, batch);
+        if (ne > 0)
+            jn_w_kernel<T><<<(unsigned)ceil_div(ne * batch, JWARPS), JWARPS * 32, smem_w, s>>>(
+                p, jd, pl->d_ce_ent + pl->ce_off[l], pl->d_ce_node + pl->ce_off[l], ne, batch);
     }
     for (size_t l = 0; l + 1 < pl->d_off.size(); ++l) {
-        const int64_t cnt = pl->d_off[l + 1] - pl->d_off[l];
-        junction_distribute_kernel<T><<<(unsigned)ceil_div(cnt * batch, JWARPS), JWARPS * 32, smem_d, s>>>(
-            p, jd, pl->d_d_nodes + pl->d_off[l], cnt, batch);
+        const int64_t nn = pl->d_off[l + 1] - pl->d_off[l];
+        const int64_t ne = pl->de_off[l + 1] - pl->de_off[l];
+        if (ne > 0)
+            jn_gcol_kernel<T><<<(unsigned)(ne * batch), JWARPS * 32, smem_r, s>>>(
+                p, jd, pl->d_de_ent + pl->de_off[l], pl->d_de_node + pl->de_off[l], pl->d_de_a + pl->de_off[l], ne);
+        jn_gdiag_kernel<T><<<(unsigned)(nn * batch), JWARPS * 32, smem_r, s>>>(p, jd, pl->d_d_nodes + pl->d_off[l], nn);
     }
     junction_finalize<<<ib, 256, 0, s>>>(p.ld, pl->n, batch, logdet, info);
     return cudaGetLastError();
@@ -310,7 +428,8 @@ void selinv_junction_plan_free(selinv_junction_plan_t *pl)
 {
     if (!pl) return;
     int32_t *arrs[] = {pl->d_c_nodes, pl->d_d_nodes, pl->d_col_ptr, pl->d_ent_slot, pl->d_ent_trans, pl->d_ent_src,
-                       pl->d_con_ptr, pl->d_con_w, pl->d_con_a, pl->d_pair_ptr, pl->d_pair};
+                       pl->d_con_ptr, pl->d_con_w, pl->d_con_a, pl->d_pair_ptr, pl->d_pair, pl->d_ct_node,
+                       pl->d_ct_t, pl->d_ce_ent, pl->d_ce_node, pl->d_de_ent, pl->d_de_node, pl->d_de_a};
     for (int32_t *a : arrs) cudaFree(a);
     delete pl;
 }
@@ -481,6 +600,35 @@ selinv_status selinv_junction_plan(int64_t n, int64_t m, const int32_t *ei, cons
                     dn[pd[depth[v]]++] = v;
                 }
             }
+            // per-level work lists
+            std::vector<int64_t> ct_off(1, 0), ce_off(1, 0), de_off(1, 0);
+            std::vector<int32_t> ct_node, ct_t, ce_ent, ce_node, de_ent, de_node, de_a;
+            for (size_t l = 0; l + 1 < c_off.size(); ++l) {
+                for (int64_t q = c_off[l]; q < c_off[l + 1]; ++q) {
+                    const int32_t v = cn[q];
+                    for (int32_t tt = 0; tt <= (int32_t)nbr[v].size(); ++tt) {
+                        ct_node.push_back(v);
+                        ct_t.push_back(tt);
+                    }
+                    for (int32_t a = 0; a < (int32_t)nbr[v].size(); ++a) {
+                        ce_ent.push_back(col_ptr[v] + a);
+                        ce_node.push_back(v);
+                    }
+                }
+                ct_off.push_back((int64_t)ct_node.size());
+                ce_off.push_back((int64_t)ce_ent.size());
+            }
+            for (size_t l = 0; l + 1 < d_off.size(); ++l) {
+                for (int64_t q = d_off[l]; q < d_off[l + 1]; ++q) {
+                    const int32_t v = dn[q];
+                    for (int32_t a = 0; a < (int32_t)nbr[v].size(); ++a) {
+                        de_ent.push_back(col_ptr[v] + a);
+                        de_node.push_back(v);
+                        de_a.push_back(a);
+                    }
+                }
+                de_off.push_back((int64_t)de_ent.size());
+            }
             // distribute pair codes
             std::vector<int32_t> pair_ptr(n + 1, 0), pair;
             for (int32_t v = 0; v < n; ++v) pair_ptr[v + 1] = pair_ptr[v] + (int32_t)(nbr[v].size() * nbr[v].size());
@@ -510,6 +658,9 @@ selinv_status selinv_junction_plan(int64_t n, int64_t m, const int32_t *ei, cons
             }
             pl->c_off = c_off;
             pl->d_off = d_off;
+            pl->ct_off = ct_off;
+            pl->ce_off = ce_off;
+            pl->de_off = de_off;
             bool ok = true;
             auto up = [&](int32_t **dst, const std::vector<int32_t> &src) {
                 if (!ok) return;
@@ -529,6 +680,13 @@ selinv_status selinv_junction_plan(int64_t n, int64_t m, const int32_t *ei, cons
             up(&pl->d_con_a, ca);
             up(&pl->d_pair_ptr, pair_ptr);
             up(&pl->d_pair, pair);
+            up(&pl->d_ct_node, ct_node);
+            up(&pl->d_ct_t, ct_t);
+            up(&pl->d_ce_ent, ce_ent);
+            up(&pl->d_ce_node, ce_node);
+            up(&pl->d_de_ent, de_ent);
+            up(&pl->d_de_node, de_node);
+            up(&pl->d_de_a, de_a);
             if (!ok) {
                 selinv_junction_plan_free(pl);
                 return SELINV_ERR_CUDA;
@@ -547,6 +705,15 @@ selinv_status selinv_junction_plan_info(const selinv_junction_plan_t *pl, int64_
     if (collect_levels) *collect_levels = (int32_t)pl->c_off.size() - 1;
     if (distribute_levels) *distribute_levels = (int32_t)pl->d_off.size() - 1;
     return SELINV_OK;
+}
+
+int64_t selinv_junction_plan_launches(const selinv_junction_plan_t *pl)
+{
+    if (!pl) return -1;
+    int64_t k = 2;                                     // init, finalize
+    for (size_t l = 0; l + 1 < pl->c_off.size(); ++l) k += 2 + (pl->ce_off[l + 1] > pl->ce_off[l] ? 1 : 0);
+    for (size_t l = 0; l + 1 < pl->d_off.size(); ++l) k += 1 + (pl->de_off[l + 1] > pl->de_off[l] ? 1 : 0);
+    return k;
 }
 
 selinv_status selinv_junction_plan_pattern(const selinv_junction_plan_t *pl, int32_t *S_i, int32_t *S_j,

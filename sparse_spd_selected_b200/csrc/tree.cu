@@ -647,11 +647,25 @@ tree_bw_distribute_kernel(TreeBwdBufs<T> p, TreeDev td, TreeSync sy, const int32
     T *s1 = s0 + E, *s2 = s1 + E;
     const int b = p.b;
     const int64_t bb = (int64_t)b * b;
-    for (;;) {
-        const unsigned long long k = warp_take(sy.counters + 1, lane);
-        if (k >= (unsigned long long)count) break;
+    const unsigned long long cnt = (unsigned long long)count;
+    // Nodes are taken one ahead and the next node's operands sent toward L2
+    // while the current one waits and computes.  Every wait still ends: the
+    // smallest unfinished node is always some warp's current node (a node
+    // held as "next" comes after its warp's current one), and its parent,
+    // earlier in the depth order, is finished.
+    unsigned long long k = warp_take(sy.counters + 1, lane);
+    while (k < cnt) {
+        const unsigned long long kn = warp_take(sy.counters + 1, lane);
+        if (kn < cnt) {
+            const int32_t vn = nodes[kn];
+            prefetch_range_l2(p.ws_P + (int64_t)vn * SLOT_ELEMS, SLOT_ELEMS, lane, 32);
+            prefetch_range_l2(p.ws_Pd + (int64_t)vn * SLOT_ELEMS, SLOT_ELEMS, lane, 32);
+            prefetch_range_l2(p.edge + vn * bb, bb, lane, 32);
+            prefetch_range_l2(p.Eb + vn * bb, bb, lane, 32);
+        }
         const int32_t v = nodes[k];
         const int32_t par = td.parent[v];
+        k = kn;
         // operands that do not depend on the parent first
         Tile<T> P, Pt, Ev, ed;
         sym_from_slot<T>(P, p.ws_P + (int64_t)v * SLOT_ELEMS, s0, lane, g, t);

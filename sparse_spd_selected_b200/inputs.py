@@ -211,7 +211,8 @@ class Workload:
         return self.batch * self.L
 
 
-# The five workloads of the problem statement, named by what they are.
+# The five workloads of the problem statement, named by what they are, and a
+# lattice for the general sparse case.
 WORKLOADS = {
     w.name: w for w in [
         Workload("chain_1x8_b4", "chain", 1, 8, 4, seed=0, load=2.0, solve=True),
@@ -220,6 +221,9 @@ WORKLOADS = {
                  dtypes=("f64", "f32")),
         Workload("forest_8x32768_b16", "tree", 8, 32768, 16, seed=3, load=1.0),
         Workload("grid_256x128_b128", "grid", 256, 128, 128, seed=4, solve=True),
+        # general sparse SPD on a loopy pattern (the pages' grid-graph example):
+        # 64 matrices on a 32 x 32 lattice of 8 x 8 blocks
+        Workload("lattice_64x1024_b8", "junction", 64, 1024, 8, seed=5, load=1.0),
     ]
 }
 
@@ -319,4 +323,9 @@ def generate(w: Workload, elements: Optional[Sequence[int]] = None):
     if w.kind == "grid":
         diag, lower, rhs, tau = grid_inputs(w.batch, w.b, w.seed, w.solve, elements)
         return {"diag": diag, "lower": lower, "rhs": rhs, "tau": tau}
+    if w.kind == "junction":
+        side = int(round(math.sqrt(w.L)))
+        E = grid_edges(side, w.L // side)
+        diag, edge = graph_inputs(w.batch, w.L, w.b, E, w.seed, w.load, elements)
+        return {"diag": diag, "edge_val": edge, "edge_index": E}
     raise ValueError(w.kind)

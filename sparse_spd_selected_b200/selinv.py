@@ -93,6 +93,8 @@ def lib():
         L.selinv_junction_plan_info.restype = ctypes.c_int
         L.selinv_junction_plan_pattern.argtypes = [P, P, P, P]
         L.selinv_junction_plan_pattern.restype = ctypes.c_int
+        L.selinv_junction_plan_launches.argtypes = [P]
+        L.selinv_junction_plan_launches.restype = I64
         L.selinv_junction_workspace_size.argtypes = [P, ctypes.c_int, I32, I64]
         L.selinv_junction_workspace_size.restype = SZ
         L.selinv_junction.argtypes = [P, ctypes.c_int, I32, I64, P, P, P, P, P, P, P, SZ, P]
@@ -576,6 +578,7 @@ class JunctionPlan:
                                                   od.ctypes.data_as(ctypes.c_void_p)), "selinv_junction_plan_pattern")
         self.S_index = np.stack([si[:self.nnz], sj[:self.nnz]]).astype(np.int64)
         self.order = od
+        self.launches = int(lib().selinv_junction_plan_launches(h))
 
     @property
     def handle(self):
