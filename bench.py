@@ -48,8 +48,8 @@ KERNEL_SOURCES = {
     "tree_collect_kernel": ["tree.cu", "warp16.cuh", "common.cuh"],
     "chain_backward_kernel": ["chain_backward.cu", "warp16.cuh", "common.cuh"],
     "tree_bw_collect_kernel": ["tree.cu", "warp16.cuh", "common.cuh"],
-    "bidiag_kernel": ["bidiag.cu", "common.cuh"],
-    "junction_collect_kernel": ["junction.cu", "warp16.cuh", "common.cuh"],
+    "bidiag_inverse_kernel": ["bidiag.cu", "warp16.cuh", "common.cuh"],
+    "jn_target_kernel": ["junction.cu", "warp16.cuh", "common.cuh"],
 }
 
 
@@ -469,7 +469,7 @@ def run_ours(args):
 
     if w.kind == "junction":
         plan = _lattice_plan(w)
-        kernel = "junction_collect_kernel"
+        kernel = "jn_target_kernel"
         launches_per_step = plan.launches
         out = {"G_diag": torch.empty_like(dev_in["diag"]),
                "G_lower": torch.empty((batch, plan.nnz, w.b, w.b), dtype=tdt, device="cuda"),
@@ -532,7 +532,7 @@ def run_ours(args):
         launches_per_step = 1
         segments = selinv.chain_segments(batch, L, b, True, "rhs" in dev_in)
         if args.op == "bidiag":
-            kernel = "bidiag_kernel"
+            kernel = "bidiag_inverse_kernel"
             out = {"G_diag": torch.empty_like(dev_in["diag"]), "G_lower": torch.empty_like(dev_in["lower"]),
                    "info": torch.empty(batch, dtype=torch.int32, device="cuda")}
         elif args.op == "backward":

@@ -91,27 +91,27 @@ struct LogAcc {
 // not yet swept are the Schur-complement column that Cholesky scales:
 // R[i][k] = P[i][k] / sqrt(d), so rz += P[g][k] z_k / sqrt(d) for g >= k.
 // The sweep's own chain does not wait for this sum.
-template <bool DRAW = false>
-SELINV_DEVINL void inv8_sweep(double v[2], int lane, int g, int t, LogAcc &det, bool &bad, bool count,
-                              double z0 = 0.0, double z1 = 0.0, double *rz = nullptr)
+template <bool DRAW = false, class T = double>
+SELINV_DEVINL void inv8_sweep(T v[2], int lane, int g, int t, LogAcc &det, bool &bad, bool count,
+                              T z0 = T(0), T z1 = T(0), T *rz = nullptr)
 {
     // v = P[g][2t], P[g][2t+1] of a symmetric positive definite 8 x 8 P
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
         const int kt = k >> 1, kj = k & 1;
-        const double c = shfl(v[kj], (lane & ~3) | kt);          // P[g][k]
-        double row[2];
+        const T c = shfl(v[kj], (lane & ~3) | kt);               // P[g][k]
+        T row[2];
         row[0] = shfl(v[0], (k << 2) | t);                         // P[k][2t]
         row[1] = shfl(v[1], (k << 2) | t);                         // P[k][2t+1]
-        const double d = shfl(v[kj], (k << 2) | kt);               // P[k][k]
-        bad |= !(d > 0.0);
-        if (count) det.mul(d);
-        const double p = recip(d);
+        const T d = shfl(v[kj], (k << 2) | kt);                    // P[k][k]
+        bad |= !(d > T(0));
+        if (count) det.mul((double)d);
+        const T p = recip(d);
         if (DRAW) {
-            const double zk = shfl(kj ? z1 : z0, (lane & ~3) | kt);
-            if (g >= k) *rz = fma(c, zk * rsqrt(d), *rz);
+            const T zk = shfl(kj ? z1 : z0, (lane & ~3) | kt);
+            if (g >= k) *rz = fma(c, zk * rsqrt_t(d), *rz);
         }
-        const double tc = c * p;
+        const T tc = c * p;
         v[0] = fma(-tc, row[0], v[0]);
         v[1] = fma(-tc, row[1], v[1]);
         if (t == kt) v[kj] = tc;

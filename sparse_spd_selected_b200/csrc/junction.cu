@@ -65,7 +65,6 @@ namespace selinv {
 namespace {
 
 constexpr int JWARPS = 4;
-constexpr int JSLOT = 256;                       // one 16 x 16 tile per workspace block
 
 struct JDev {
     const int32_t *col_ptr, *ent_slot, *ent_trans, *ent_src, *con_ptr, *con_w, *con_a, *pair_ptr, *pair;
@@ -81,93 +80,230 @@ template <class T> struct JBufs {
     int b;
 };
 
-// Tile from a 16-pitch workspace tile (read through L2: written earlier in the call).
-template <class T> SELINV_DEVINL void ld_ws(w16::Tile<T> &a, const T *M, int g, int t, bool trans)
-{
+// Tile policies.  Pol16: the 16 x 16 register tile of warp16.cuh (b <= 16).
+// Pol8: an 8 x 8 tile in the m8n8 accumulator layout (lane 4g + t holds row
+// g, columns 2t, 2t + 1) for b <= 8, where a 16 x 16 tile would be three
+// quarters padding: an 8 x 8 x 8 product is two FP64 tensor-core steps whose
+// k index follows the lane's own columns (k = 2t + s at step s, the same for
+// both operands), transposes and mirrors are shuffles, and the inverse is the
+// 8-pivot sweep.  Workspace blocks are SLOT-element tiles of pitch DIM.
+template <class T> struct Pol16 {
+    using Tile = w16::Tile<T>;
+    static constexpr int DIM = 16, SLOT = 256, IMG = w16::SL<T>::ELEMS;
+    static SELINV_DEVINL void zero(Tile &a) { w16::zero(a); }
+    static SELINV_DEVINL void add(Tile &a, const Tile &x)
+    {
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
+        for (int h = 0; h < 2; ++h)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int r = g + 8 * h, c = w16::tcol(t, q);
-            a.v[h][q] = __ldcg(trans ? M + c * 16 + r : M + r * 16 + c);
-        }
-}
+            for (int q = 0; q < 4; ++q) a.v[h][q] += x.v[h][q];
+    }
+    static SELINV_DEVINL void ld_ws(Tile &a, const T *M, int g, int t, bool trans)
+    {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int r = g + 8 * h, c = w16::tcol(t, q);
+                a.v[h][q] = __ldcg(trans ? M + c * 16 + r : M + r * 16 + c);
+            }
+    }
+    static SELINV_DEVINL void st_ws(T *M, const Tile &a, int g, int t)
+    {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) M[(g + 8 * h) * 16 + w16::tcol(t, q)] = a.v[h][q];
+    }
+    static SELINV_DEVINL void ld_blk(Tile &a, const T *M, int b, int g, int t, bool trans, bool l2)
+    {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int r = g + 8 * h, c = w16::tcol(t, q);
+                const T *p = trans ? M + c * b + r : M + r * b + c;
+                a.v[h][q] = (r < b && c < b) ? (l2 ? __ldcg(p) : __ldg(p)) : T(0);
+            }
+    }
+    static SELINV_DEVINL void st_blk(T *M, const Tile &a, int b, int g, int t, bool trans)
+    {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int r = g + 8 * h, c = w16::tcol(t, q);
+                if (r < b && c < b) {
+                    if (trans) M[c * b + r] = a.v[h][q];
+                    else M[r * b + c] = a.v[h][q];
+                }
+            }
+    }
+    static SELINV_DEVINL void load_sym(Tile &a, const T *D, int b, int g, int t) { w16::load_sym<T, false>(a, D, b, g, t); }
+    template <bool NEG> static SELINV_DEVINL void gemm(Tile &acc, const Tile &X, const Tile &Y, T *sX, T *sY, int g, int t)
+    {
+        w16::gemm_nt<NEG>(acc, X, Y, sX, sY, g, t);
+    }
+    static SELINV_DEVINL void make_sym(Tile &a, int g, int t) { w16::mirror_upper(a, g, t); }
+    static SELINV_DEVINL void sym_from_lower(Tile &a, T *img, int g, int t)
+    {
+        w16::to_smem<T>(img, a, g, t);
+        __syncwarp();
+        w16::from_smem_lower<T>(a, img, g, t);
+        __syncwarp();
+    }
+    static SELINV_DEVINL void inverse(Tile &a, T *cb, int g, int t, LogAcc &det, bool &bad)
+    {
+        w16::spd_inverse<T>(a, cb, g, t, det, bad);
+    }
+    static SELINV_DEVINL void to_img(T *img, const Tile &a, int g, int t) { w16::to_smem<T>(img, a, g, t); }
+    static SELINV_DEVINL void from_img(Tile &a, const T *img, int g, int t) { w16::from_smem<T>(a, img, g, t); }
+};
 
-template <class T> SELINV_DEVINL void st_ws(T *M, const w16::Tile<T> &a, int g, int t)
-{
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) M[(g + 8 * h) * 16 + w16::tcol(t, q)] = a.v[h][q];
-}
+template <class T> struct Tile8 {
+    T v[2];
+};
 
-// b x b block (row-major), possibly transposed, into a tile; zero pad.
-template <class T> SELINV_DEVINL void ld_blk(w16::Tile<T> &a, const T *M, int b, int g, int t, bool trans, bool l2)
-{
+template <class T> struct Pol8 {
+    using Tile = Tile8<T>;
+    static constexpr int DIM = 8, SLOT = 64, IMG = 8 * 9;
+    static SELINV_DEVINL void zero(Tile &a) { a.v[0] = a.v[1] = T(0); }
+    static SELINV_DEVINL void add(Tile &a, const Tile &x)
+    {
+        a.v[0] += x.v[0];
+        a.v[1] += x.v[1];
+    }
+    static SELINV_DEVINL void ld_ws(Tile &a, const T *M, int g, int t, bool trans)
+    {
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
+        for (int j = 0; j < 2; ++j) a.v[j] = __ldcg(trans ? M + (2 * t + j) * 8 + g : M + g * 8 + 2 * t + j);
+    }
+    static SELINV_DEVINL void st_ws(T *M, const Tile &a, int g, int t)
+    {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int r = g + 8 * h, c = w16::tcol(t, q);
+        for (int j = 0; j < 2; ++j) M[g * 8 + 2 * t + j] = a.v[j];
+    }
+    static SELINV_DEVINL void ld_blk(Tile &a, const T *M, int b, int g, int t, bool trans, bool l2)
+    {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int r = g, c = 2 * t + j;
             const T *p = trans ? M + c * b + r : M + r * b + c;
-            a.v[h][q] = (r < b && c < b) ? (l2 ? __ldcg(p) : __ldg(p)) : T(0);
+            a.v[j] = (r < b && c < b) ? (l2 ? __ldcg(p) : __ldg(p)) : T(0);
         }
-}
-
-template <class T> SELINV_DEVINL void st_blk(T *M, const w16::Tile<T> &a, int b, int g, int t, bool trans)
-{
+    }
+    static SELINV_DEVINL void st_blk(T *M, const Tile &a, int b, int g, int t, bool trans)
+    {
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int r = g + 8 * h, c = w16::tcol(t, q);
+        for (int j = 0; j < 2; ++j) {
+            const int r = g, c = 2 * t + j;
             if (r < b && c < b) {
-                if (trans) M[c * b + r] = a.v[h][q];
-                else M[r * b + c] = a.v[h][q];
+                if (trans) M[c * b + r] = a.v[j];
+                else M[r * b + c] = a.v[j];
             }
         }
-}
+    }
+    static SELINV_DEVINL void load_sym(Tile &a, const T *D, int b, int g, int t)
+    {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int r = g, c = 2 * t + j;
+            const int rr = c <= r ? r : c, cc = c <= r ? c : r;
+            a.v[j] = (r < b && c < b) ? __ldg(D + rr * b + cc) : (r == c ? T(1) : T(0));
+        }
+    }
+    // acc += (NEG ? -1 : 1) X Y^T
+    template <bool NEG> static SELINV_DEVINL void gemm(Tile &acc, const Tile &X, const Tile &Y, T *sX, T *sY, int g, int t)
+    {
+        if constexpr (sizeof(T) == 8) {
+#pragma unroll
+            for (int s2 = 0; s2 < 2; ++s2) dmma_8x8x4(acc.v[0], acc.v[1], NEG ? -X.v[s2] : X.v[s2], Y.v[s2]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                sX[g * 9 + 2 * t + j] = X.v[j];
+                sY[g * 9 + 2 * t + j] = Y.v[j];
+            }
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                T s = T(0);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) s = fma(sX[g * 9 + k], sY[(2 * t + j) * 9 + k], s);
+                acc.v[j] += NEG ? -s : s;
+            }
+            __syncwarp();
+        }
+    }
+    // entry (c, r) of a, for the lane's (r, c) = (g, 2t + j): held by lane 4c + r / 2, register r & 1
+    static SELINV_DEVINL T mirror_of(const Tile &a, int g, int t, int j)
+    {
+        const int src = ((2 * t + j) << 2) | (g >> 1);
+        const T u0 = shfl(a.v[0], src), u1 = shfl(a.v[1], src);
+        return (g & 1) ? u1 : u0;
+    }
+    static SELINV_DEVINL void sym_from_lower(Tile &a, T *, int g, int t)
+    {
+        const T m0 = mirror_of(a, g, t, 0), m1 = mirror_of(a, g, t, 1);
+        if (2 * t > g) a.v[0] = m0;
+        if (2 * t + 1 > g) a.v[1] = m1;
+    }
+    static SELINV_DEVINL void make_sym(Tile &a, int g, int t) { sym_from_lower(a, nullptr, g, t); }
+    static SELINV_DEVINL void inverse(Tile &a, T *, int g, int t, LogAcc &det, bool &bad)
+    {
+        inv8_sweep<false, T>(a.v, 4 * g + t, g, t, det, bad, true);
+    }
+    static SELINV_DEVINL void to_img(T *img, const Tile &a, int g, int t)
+    {
+        img[g * 9 + 2 * t] = a.v[0];
+        img[g * 9 + 2 * t + 1] = a.v[1];
+    }
+    static SELINV_DEVINL void from_img(Tile &a, const T *img, int g, int t)
+    {
+        a.v[0] = img[g * 9 + 2 * t];
+        a.v[1] = img[g * 9 + 2 * t + 1];
+    }
+};
 
 // Four warps split one sum of tile products; warps 1..3 leave their partial
 // tiles in shared memory and warp 0 adds them in a fixed order, so the result
 // does not depend on timing.  Returns true in warp 0, which holds the total.
-template <class T> SELINV_DEVINL bool reduce4(w16::Tile<T> &acc, T *img, int wid, int g, int t)
+template <class T, class Pol> SELINV_DEVINL bool reduce4(typename Pol::Tile &acc, T *img, int wid, int g, int t)
 {
-    constexpr int EL = w16::SL<T>::ELEMS;
-    if (wid > 0) w16::to_smem<T>(img + (wid - 1) * EL, acc, g, t);
+    if (wid > 0) Pol::to_img(img + (wid - 1) * Pol::IMG, acc, g, t);
     __syncthreads();
     if (wid != 0) return false;
 #pragma unroll
     for (int k = 0; k < JWARPS - 1; ++k) {
-        w16::Tile<T> u;
-        w16::from_smem<T>(u, img + k * EL, g, t);
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) acc.v[h][q] += u.v[h][q];
+        typename Pol::Tile u;
+        Pol::from_img(u, img + k * Pol::IMG, g, t);
+        Pol::add(acc, u);
     }
     return true;
 }
 
-template <class T> __host__ __device__ constexpr int j_smem_elems()
+// shared memory of the CTA-per-item kernels: three partial images, then per
+// warp two product scratch images (float products) and 32 elements
+template <class T, class Pol> __host__ __device__ constexpr int j_smem_elems()
 {
-    return (JWARPS - 1) * w16::SL<T>::ELEMS + JWARPS * (2 * w16::SL<T>::ELEMS + 32);
+    return (JWARPS - 1) * Pol::IMG + JWARPS * (2 * Pol::IMG + 32);
 }
 
 // Collect, one CTA per target block (v, t) of a level: t = 0 is S_v, t >= 1
 // is A'_{u,v} for u = N(v)[t-1]; the warps split the contributions
-// -W_{u,k} A'_{v,k}^T listed by the plan.
-template <class T>
+// -W_{u,k} A'_{v,k}^T listed by the plan, each loading its next pair of
+// tiles before the current product.
+template <class T, class Pol>
 __global__ void __launch_bounds__(JWARPS * 32)
 jn_target_kernel(JBufs<T> p, JDev jd, const int32_t *tnode, const int32_t *tt, int64_t count)
 {
-    using namespace w16;
-    constexpr int EL = SL<T>::ELEMS;
+    using Tile = typename Pol::Tile;
+    constexpr int S = Pol::SLOT;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     T *img = reinterpret_cast<T *>(smem_raw);
-    T *s1 = img + (JWARPS - 1) * EL + wid * (2 * EL + 32), *s2 = s1 + EL;
+    T *s1 = img + (JWARPS - 1) * Pol::IMG + wid * (2 * Pol::IMG + 32), *s2 = s1 + Pol::IMG;
     const int64_t item = blockIdx.x;
     const int32_t v = tnode[item % count], tg = tt[item % count];
     const int64_t e = item / count;
@@ -175,38 +311,50 @@ jn_target_kernel(JBufs<T> p, JDev jd, const int32_t *tnode, const int32_t *tt, i
     const int64_t bb = (int64_t)b * b;
     const int32_t c0 = jd.col_ptr[v];
     const int64_t tau = (int64_t)c0 + v + tg;
-    const T *Ap = p.Ap + e * jd.E * JSLOT, *W = p.W + e * jd.E * JSLOT;
-    Tile<T> acc;
-    zero(acc);
-    for (int32_t c = jd.con_ptr[tau] + wid; c < jd.con_ptr[tau + 1]; c += JWARPS) {
-        Tile<T> w, a;
-        ld_ws<T>(w, W + (int64_t)jd.con_w[c] * JSLOT, g, t, false);
-        ld_ws<T>(a, Ap + (int64_t)jd.con_a[c] * JSLOT, g, t, false);
-        gemm_nt<true>(acc, w, a, s1, s2, g, t);              // -= W_{u,k} A'_{v,k}^T
+    const T *Ap = p.Ap + e * jd.E * S, *W = p.W + e * jd.E * S;
+    Tile acc;
+    Pol::zero(acc);
+    {
+        const int32_t cend = jd.con_ptr[tau + 1];
+        int32_t c = jd.con_ptr[tau] + wid;
+        Tile w, a;
+        if (c < cend) {
+            Pol::ld_ws(w, W + (int64_t)jd.con_w[c] * S, g, t, false);
+            Pol::ld_ws(a, Ap + (int64_t)jd.con_a[c] * S, g, t, false);
+        }
+        while (c < cend) {
+            const int32_t cn = c + JWARPS;
+            Tile wn, an;
+            if (cn < cend) {
+                Pol::ld_ws(wn, W + (int64_t)jd.con_w[cn] * S, g, t, false);
+                Pol::ld_ws(an, Ap + (int64_t)jd.con_a[cn] * S, g, t, false);
+            }
+            Pol::template gemm<true>(acc, w, a, s1, s2, g, t);        // -= W_{u,k} A'_{v,k}^T
+            w = wn;
+            a = an;
+            c = cn;
+        }
     }
-    if (!reduce4<T>(acc, img, wid, g, t)) return;
-    Tile<T> a0;
+    if (!reduce4<T, Pol>(acc, img, wid, g, t)) return;
+    Tile a0;
     if (tg == 0) {
-        load_sym<T, false>(a0, p.diag + (e * jd.n + v) * bb, b, g, t);
+        Pol::load_sym(a0, p.diag + (e * jd.n + v) * bb, b, g, t);
     } else {
         const int32_t ent = c0 + tg - 1, src = jd.ent_src[ent];
-        if (src >= 0) ld_blk<T>(a0, p.edge + (e * jd.m + src) * bb, b, g, t, jd.ent_trans[ent] != 0, false);
-        else zero(a0);
+        if (src >= 0) Pol::ld_blk(a0, p.edge + (e * jd.m + src) * bb, b, g, t, jd.ent_trans[ent] != 0, false);
+        else Pol::zero(a0);
     }
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc.v[h][q] += a0.v[h][q];
-    if (tg == 0) st_ws<T>(p.Sinv + (e * jd.n + v) * JSLOT, acc, g, t);      // S_v, inverted next
-    else st_ws<T>(p.Ap + (e * jd.E + c0 + tg - 1) * JSLOT, acc, g, t);
+    Pol::add(acc, a0);
+    if (tg == 0) Pol::st_ws(p.Sinv + (e * jd.n + v) * S, acc, g, t);      // S_v, inverted next
+    else Pol::st_ws(p.Ap + (e * jd.E + c0 + tg - 1) * S, acc, g, t);
 }
 
 // One warp per node of a level: P_v = S_v^-1 in place, log det, info.
-template <class T>
+template <class T, class Pol>
 __global__ void __launch_bounds__(JWARPS * 32)
 jn_inverse_kernel(JBufs<T> p, JDev jd, const int32_t *nodes, int64_t count, int64_t batch)
 {
-    using namespace w16;
+    using Tile = typename Pol::Tile;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -215,123 +363,129 @@ jn_inverse_kernel(JBufs<T> p, JDev jd, const int32_t *nodes, int64_t count, int6
     if (item >= count * batch) return;
     const int32_t v = nodes[item % count];
     const int64_t e = item / count;
-    T *slot = p.Sinv + (e * jd.n + v) * JSLOT;
-    Tile<T> S;
-    ld_ws<T>(S, slot, g, t, false);
-    mirror_upper(S, g, t);
+    T *slot = p.Sinv + (e * jd.n + v) * Pol::SLOT;
+    Tile S;
+    Pol::ld_ws(S, slot, g, t, false);
+    Pol::make_sym(S, g, t);
     LogAcc det;
     det.init();
     bool bad = false;
-    spd_inverse<T>(S, cb, g, t, det, bad);
+    Pol::inverse(S, cb, g, t, det, bad);
     if (lane == 0) {
         p.ld[e * jd.n + v] = det.log_value();
         if (bad) atomicMin(p.info + e, v);
     }
     __syncwarp();
-    st_ws<T>(slot, S, g, t);
+    Pol::st_ws(slot, S, g, t);
 }
 
 // One warp per clique entry (u, v) of a level: W_{u,v} = A'_{u,v} P_v.
-template <class T>
+template <class T, class Pol>
 __global__ void __launch_bounds__(JWARPS * 32)
 jn_w_kernel(JBufs<T> p, JDev jd, const int32_t *ents, const int32_t *enodes, int64_t count, int64_t batch)
 {
-    using namespace w16;
-    constexpr int EL = SL<T>::ELEMS;
+    using Tile = typename Pol::Tile;
+    constexpr int S = Pol::SLOT;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    T *s1 = reinterpret_cast<T *>(smem_raw) + wid * 2 * EL, *s2 = s1 + EL;
+    T *s1 = reinterpret_cast<T *>(smem_raw) + wid * 2 * Pol::IMG, *s2 = s1 + Pol::IMG;
     const int64_t item = (int64_t)blockIdx.x * JWARPS + wid;
     if (item >= count * batch) return;
     const int32_t ent = ents[item % count], v = enodes[item % count];
     const int64_t e = item / count;
-    Tile<T> a, P, w;
-    ld_ws<T>(a, p.Ap + (e * jd.E + ent) * JSLOT, g, t, false);
-    ld_ws<T>(P, p.Sinv + (e * jd.n + v) * JSLOT, g, t, false);
-    zero(w);
-    gemm_nt<false>(w, a, P, s1, s2, g, t);                   // P symmetric
-    st_ws<T>(p.W + (e * jd.E + ent) * JSLOT, w, g, t);
+    Tile a, P, w;
+    Pol::ld_ws(a, p.Ap + (e * jd.E + ent) * S, g, t, false);
+    Pol::ld_ws(P, p.Sinv + (e * jd.n + v) * S, g, t, false);
+    Pol::zero(w);
+    Pol::template gemm<false>(w, a, P, s1, s2, g, t);            // P symmetric
+    Pol::st_ws(p.W + (e * jd.E + ent) * S, w, g, t);
 }
 
 // Distribute, one CTA per clique entry (u, v) of a level:
 // G_{u,v} = -sum_{l in N(v)} G_{u,l} W_{l,v}, the warps splitting l.
-template <class T>
+template <class T, class Pol>
 __global__ void __launch_bounds__(JWARPS * 32)
 jn_gcol_kernel(JBufs<T> p, JDev jd, const int32_t *ents, const int32_t *enodes, const int32_t *eidx, int64_t count)
 {
-    using namespace w16;
-    constexpr int EL = SL<T>::ELEMS;
+    using Tile = typename Pol::Tile;
+    constexpr int S = Pol::SLOT;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     T *img = reinterpret_cast<T *>(smem_raw);
-    T *s1 = img + (JWARPS - 1) * EL + wid * (2 * EL + 32), *s2 = s1 + EL;
+    T *s1 = img + (JWARPS - 1) * Pol::IMG + wid * (2 * Pol::IMG + 32), *s2 = s1 + Pol::IMG;
     const int64_t item = blockIdx.x;
     const int32_t ent = ents[item % count], v = enodes[item % count], a = eidx[item % count];
     const int64_t e = item / count;
     const int b = p.b;
     const int64_t bb = (int64_t)b * b;
     const int32_t c0 = jd.col_ptr[v], d = jd.col_ptr[v + 1] - c0;
-    const T *W = p.W + e * jd.E * JSLOT;
+    const T *W = p.W + e * jd.E * S;
     const T *Gd = p.G_diag + e * jd.n * bb, *Gl = p.G_lower + e * jd.nnz * bb;
     const int32_t *pc = jd.pair + jd.pair_ptr[v] + (int64_t)a * d;
-    Tile<T> acc;
-    zero(acc);
-    for (int32_t c = wid; c < d; c += JWARPS) {
+    Tile acc;
+    Pol::zero(acc);
+    auto load_pair = [&](int32_t c, Tile &gul, Tile &wt) {
         const int32_t code = pc[c];
-        Tile<T> gul, wt;
-        if (code < 0) ld_blk<T>(gul, Gd + (int64_t)(-code - 1) * bb, b, g, t, false, true);
-        else ld_blk<T>(gul, Gl + (int64_t)(code >> 1) * bb, b, g, t, (code & 1) != 0, true);
-        ld_ws<T>(wt, W + (int64_t)(c0 + c) * JSLOT, g, t, true);           // W_{l,v}^T
-        gemm_nt<true>(acc, gul, wt, s1, s2, g, t);                        // -= G_{u,l} W_{l,v}
+        if (code < 0) Pol::ld_blk(gul, Gd + (int64_t)(-code - 1) * bb, b, g, t, false, true);
+        else Pol::ld_blk(gul, Gl + (int64_t)(code >> 1) * bb, b, g, t, (code & 1) != 0, true);
+        Pol::ld_ws(wt, W + (int64_t)(c0 + c) * S, g, t, true);            // W_{l,v}^T
+    };
+    {
+        int32_t c = wid;
+        Tile gul, wt;
+        if (c < d) load_pair(c, gul, wt);
+        while (c < d) {
+            const int32_t cn = c + JWARPS;
+            Tile gn, wn;
+            if (cn < d) load_pair(cn, gn, wn);
+            Pol::template gemm<true>(acc, gul, wt, s1, s2, g, t);        // -= G_{u,l} W_{l,v}
+            gul = gn;
+            wt = wn;
+            c = cn;
+        }
     }
-    if (!reduce4<T>(acc, img, wid, g, t)) return;
-    st_blk<T>(p.G_lower + (e * jd.nnz + jd.ent_slot[ent]) * bb, acc, b, g, t, jd.ent_trans[ent] != 0);
+    if (!reduce4<T, Pol>(acc, img, wid, g, t)) return;
+    Pol::st_blk(p.G_lower + (e * jd.nnz + jd.ent_slot[ent]) * bb, acc, b, g, t, jd.ent_trans[ent] != 0);
 }
 
 // One CTA per node of a level: G_vv = P_v - sum_{l in N(v)} W_{l,v}^T G_{l,v},
 // the warps splitting l; written exactly symmetric.
-template <class T>
+template <class T, class Pol>
 __global__ void __launch_bounds__(JWARPS * 32)
 jn_gdiag_kernel(JBufs<T> p, JDev jd, const int32_t *nodes, int64_t count)
 {
-    using namespace w16;
-    constexpr int EL = SL<T>::ELEMS;
+    using Tile = typename Pol::Tile;
+    constexpr int S = Pol::SLOT;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     T *img = reinterpret_cast<T *>(smem_raw);
-    T *s1 = img + (JWARPS - 1) * EL + wid * (2 * EL + 32), *s2 = s1 + EL;
+    T *s1 = img + (JWARPS - 1) * Pol::IMG + wid * (2 * Pol::IMG + 32), *s2 = s1 + Pol::IMG;
     const int64_t item = blockIdx.x;
     const int32_t v = nodes[item % count];
     const int64_t e = item / count;
     const int b = p.b;
     const int64_t bb = (int64_t)b * b;
     const int32_t c0 = jd.col_ptr[v], d = jd.col_ptr[v + 1] - c0;
-    const T *W = p.W + e * jd.E * JSLOT;
+    const T *W = p.W + e * jd.E * S;
     const T *Gl = p.G_lower + e * jd.nnz * bb;
-    Tile<T> acc;
-    zero(acc);
+    Tile acc;
+    Pol::zero(acc);
     for (int32_t c = wid; c < d; c += JWARPS) {
         const int32_t ent = c0 + c;
-        Tile<T> wt, glT;
-        ld_ws<T>(wt, W + (int64_t)ent * JSLOT, g, t, true);                 // W_{l,v}^T
-        ld_blk<T>(glT, Gl + (int64_t)jd.ent_slot[ent] * bb, b, g, t, jd.ent_trans[ent] == 0, true);   // G_{l,v}^T
-        gemm_nt<true>(acc, wt, glT, s1, s2, g, t);                          // -= W^T G
+        Tile wt, glT;
+        Pol::ld_ws(wt, W + (int64_t)ent * S, g, t, true);                  // W_{l,v}^T
+        Pol::ld_blk(glT, Gl + (int64_t)jd.ent_slot[ent] * bb, b, g, t, jd.ent_trans[ent] == 0, true);   // G_{l,v}^T
+        Pol::template gemm<true>(acc, wt, glT, s1, s2, g, t);              // -= W^T G
     }
-    if (!reduce4<T>(acc, img, wid, g, t)) return;
-    Tile<T> P;
-    ld_ws<T>(P, p.Sinv + (e * jd.n + v) * JSLOT, g, t, false);
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc.v[h][q] += P.v[h][q];
-    to_smem<T>(img, acc, g, t);                       // exactly symmetric from the lower triangle
-    __syncwarp();
-    from_smem_lower<T>(acc, img, g, t);
-    __syncwarp();
-    st_blk<T>(p.G_diag + (e * jd.n + v) * bb, acc, b, g, t, false);
+    if (!reduce4<T, Pol>(acc, img, wid, g, t)) return;
+    Tile P;
+    Pol::ld_ws(P, p.Sinv + (e * jd.n + v) * S, g, t, false);
+    Pol::add(acc, P);
+    Pol::sym_from_lower(acc, img, g, t);             // exactly symmetric from the lower triangle
+    Pol::st_blk(p.G_diag + (e * jd.n + v) * bb, acc, b, g, t, false);
 }
 
 __global__ void junction_init(int32_t *info, int64_t batch)
@@ -353,16 +507,17 @@ __global__ void junction_finalize(const double *ld, int64_t n, int64_t batch, do
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-template <class T> size_t ws_bytes(const selinv_junction_plan_s *pl, int64_t batch)
+template <class T, int SLOT> size_t ws_bytes(const selinv_junction_plan_s *pl, int64_t batch)
 {
-    return align256(sizeof(T) * JSLOT * (size_t)(batch * pl->n)) +
-           2 * align256(sizeof(T) * JSLOT * (size_t)(batch * pl->E)) + align256(sizeof(double) * (size_t)(batch * pl->n));
+    return align256(sizeof(T) * SLOT * (size_t)(batch * pl->n)) +
+           2 * align256(sizeof(T) * SLOT * (size_t)(batch * pl->E)) + align256(sizeof(double) * (size_t)(batch * pl->n));
 }
 
-template <class T>
+template <class T, class Pol>
 cudaError_t run_junction(const selinv_junction_plan_s *pl, int b, int64_t batch, const T *diag, const T *edge,
                          T *G_diag, T *G_lower, double *logdet, int32_t *info, void *ws, cudaStream_t s)
 {
+    constexpr int S = Pol::SLOT;
     char *w = static_cast<char *>(ws);
     JBufs<T> p;
     p.diag = diag;
@@ -370,11 +525,11 @@ cudaError_t run_junction(const selinv_junction_plan_s *pl, int b, int64_t batch,
     p.G_diag = G_diag;
     p.G_lower = G_lower;
     p.Sinv = reinterpret_cast<T *>(w);
-    w += align256(sizeof(T) * JSLOT * (size_t)(batch * pl->n));
+    w += align256(sizeof(T) * S * (size_t)(batch * pl->n));
     p.Ap = reinterpret_cast<T *>(w);
-    w += align256(sizeof(T) * JSLOT * (size_t)(batch * pl->E));
+    w += align256(sizeof(T) * S * (size_t)(batch * pl->E));
     p.W = reinterpret_cast<T *>(w);
-    w += align256(sizeof(T) * JSLOT * (size_t)(batch * pl->E));
+    w += align256(sizeof(T) * S * (size_t)(batch * pl->E));
     p.ld = reinterpret_cast<double *>(w);
     p.info = info;
     p.b = b;
@@ -382,33 +537,35 @@ cudaError_t run_junction(const selinv_junction_plan_s *pl, int b, int64_t batch,
             pl->d_con_a, pl->d_pair_ptr, pl->d_pair, pl->n, pl->m, pl->nnz, pl->E};
     const unsigned ib = (unsigned)ceil_div(batch, 256);
     junction_init<<<ib, 256, 0, s>>>(info, batch);
-    constexpr int EL = w16::SL<T>::ELEMS;
-    const size_t smem_r = sizeof(T) * j_smem_elems<T>();           // CTA-per-item kernels
-    const size_t smem_w = sizeof(T) * JWARPS * 2 * EL, smem_i = sizeof(T) * JWARPS * 32;
+    const size_t smem_r = sizeof(T) * j_smem_elems<T, Pol>();      // CTA-per-item kernels
+    const size_t smem_w = sizeof(T) * JWARPS * 2 * Pol::IMG, smem_i = sizeof(T) * JWARPS * 32;
     cudaError_t err = cudaSuccess;
-    for (auto k : {(const void *)jn_target_kernel<T>, (const void *)jn_gcol_kernel<T>, (const void *)jn_gdiag_kernel<T>})
+    for (auto k : {(const void *)jn_target_kernel<T, Pol>, (const void *)jn_gcol_kernel<T, Pol>,
+                   (const void *)jn_gdiag_kernel<T, Pol>})
         if (err == cudaSuccess) err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_r);
-    if (err == cudaSuccess) err = cudaFuncSetAttribute(jn_w_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_w);
+    if (err == cudaSuccess)
+        err = cudaFuncSetAttribute(jn_w_kernel<T, Pol>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_w);
     if (err != cudaSuccess) return err;
     for (size_t l = 0; l + 1 < pl->c_off.size(); ++l) {
         const int64_t nt = pl->ct_off[l + 1] - pl->ct_off[l];
         const int64_t nn = pl->c_off[l + 1] - pl->c_off[l];
         const int64_t ne = pl->ce_off[l + 1] - pl->ce_off[l];
-        jn_target_kernel<T><<<(unsigned)(nt * batch), JWARPS * 32, smem_r, s>>>(
+        jn_target_kernel<T, Pol><<<(unsigned)(nt * batch), JWARPS * 32, smem_r, s>>>(
             p, jd, pl->d_ct_node + pl->ct_off[l], pl->d_ct_t + pl->ct_off[l], nt);
-        jn_inverse_kernel<T><<<(unsigned)ceil_div(nn * batch, JWARPS), JWARPS * 32, smem_i, s>>>(
+        jn_inverse_kernel<T, Pol><<<(unsigned)ceil_div(nn * batch, JWARPS), JWARPS * 32, smem_i, s>>>(
             p, jd, pl->d_c_nodes + pl->c_off[l], nn, batch);
         if (ne > 0)
-            jn_w_kernel<T><<<(unsigned)ceil_div(ne * batch, JWARPS), JWARPS * 32, smem_w, s>>>(
+            jn_w_kernel<T, Pol><<<(unsigned)ceil_div(ne * batch, JWARPS), JWARPS * 32, smem_w, s>>>(
                 p, jd, pl->d_ce_ent + pl->ce_off[l], pl->d_ce_node + pl->ce_off[l], ne, batch);
     }
     for (size_t l = 0; l + 1 < pl->d_off.size(); ++l) {
         const int64_t nn = pl->d_off[l + 1] - pl->d_off[l];
         const int64_t ne = pl->de_off[l + 1] - pl->de_off[l];
         if (ne > 0)
-            jn_gcol_kernel<T><<<(unsigned)(ne * batch), JWARPS * 32, smem_r, s>>>(
+            jn_gcol_kernel<T, Pol><<<(unsigned)(ne * batch), JWARPS * 32, smem_r, s>>>(
                 p, jd, pl->d_de_ent + pl->de_off[l], pl->d_de_node + pl->de_off[l], pl->d_de_a + pl->de_off[l], ne);
-        jn_gdiag_kernel<T><<<(unsigned)(nn * batch), JWARPS * 32, smem_r, s>>>(p, jd, pl->d_d_nodes + pl->d_off[l], nn);
+        jn_gdiag_kernel<T, Pol><<<(unsigned)(nn * batch), JWARPS * 32, smem_r, s>>>(p, jd, pl->d_d_nodes + pl->d_off[l],
+                                                                                     nn);
     }
     junction_finalize<<<ib, 256, 0, s>>>(p.ld, pl->n, batch, logdet, info);
     return cudaGetLastError();
@@ -729,7 +886,8 @@ selinv_status selinv_junction_plan_pattern(const selinv_junction_plan_t *pl, int
 size_t selinv_junction_workspace_size(const selinv_junction_plan_t *pl, selinv_dtype dtype, int32_t b, int64_t batch)
 {
     if (!pl || (dtype != SELINV_F64 && dtype != SELINV_F32) || b < 1 || b > 16 || batch < 0) return 0;
-    return dtype == SELINV_F64 ? ws_bytes<double>(pl, batch) : ws_bytes<float>(pl, batch);
+    if (b <= 8) return dtype == SELINV_F64 ? ws_bytes<double, 64>(pl, batch) : ws_bytes<float, 64>(pl, batch);
+    return dtype == SELINV_F64 ? ws_bytes<double, 256>(pl, batch) : ws_bytes<float, 256>(pl, batch);
 }
 
 selinv_status selinv_junction(const selinv_junction_plan_t *pl, selinv_dtype dtype, int32_t b, int64_t batch,
@@ -752,14 +910,16 @@ selinv_status selinv_junction(const selinv_junction_plan_t *pl, selinv_dtype dty
     if (dev != pl->device) return SELINV_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t err;
+    const double *dd = static_cast<const double *>(diag), *de = static_cast<const double *>(edge_val);
+    const float *fd = static_cast<const float *>(diag), *fe = static_cast<const float *>(edge_val);
+    double *dg = static_cast<double *>(G_diag), *dl = static_cast<double *>(G_lower);
+    float *fg = static_cast<float *>(G_diag), *fl = static_cast<float *>(G_lower);
     if (dtype == SELINV_F64)
-        err = run_junction<double>(pl, b, batch, static_cast<const double *>(diag), static_cast<const double *>(edge_val),
-                                   static_cast<double *>(G_diag), static_cast<double *>(G_lower), logdet, info,
-                                   workspace, s);
+        err = b <= 8 ? run_junction<double, Pol8<double>>(pl, b, batch, dd, de, dg, dl, logdet, info, workspace, s)
+                     : run_junction<double, Pol16<double>>(pl, b, batch, dd, de, dg, dl, logdet, info, workspace, s);
     else
-        err = run_junction<float>(pl, b, batch, static_cast<const float *>(diag), static_cast<const float *>(edge_val),
-                                  static_cast<float *>(G_diag), static_cast<float *>(G_lower), logdet, info, workspace,
-                                  s);
+        err = b <= 8 ? run_junction<float, Pol8<float>>(pl, b, batch, fd, fe, fg, fl, logdet, info, workspace, s)
+                     : run_junction<float, Pol16<float>>(pl, b, batch, fd, fe, fg, fl, logdet, info, workspace, s);
     return err == cudaSuccess ? SELINV_OK : SELINV_ERR_CUDA;
 }
 

@@ -68,6 +68,7 @@ def test_junction_given_order_tree_and_single_node(cuda_ok):
 
 def test_junction_f32_and_leading_dims(cuda_ok):
     run(16, inputs.grid_edges(4, 4), 16, 11400, torch.float32, lead=(3,), load=2.0)
+    run(16, inputs.grid_edges(4, 4), 8, 11402, torch.float32, lead=(3,), load=2.0)      # the 8 x 8 tile path
     run(12, random_pattern(12, 25, 3), 4, 11401, torch.float64, lead=(2, 3))
 
 
