@@ -8,8 +8,15 @@ the oracle shares no code with the CUDA library.
 What it computes follows gabp-sparse-inv 0.3.2 (PyPI page), "Implemented and
 tested kernels" -> Chain and Tree, and the "Quickstart" conventions: the
 on-pattern blocks of A^-1 (G_diag, G_lower / G_edge), log det A from the same
-factorisation, and the chain solve x = A^-1 r.  The C file's header states the
-recursion and every reading taken where the pages are silent.
+factorisation, and the chain solve x = A^-1 r; then the rows beyond them:
+Gaussian draws from the factor ("Gaussian sampling"), the cotangents of the
+selected inverse ("Differentiable selected inverse", written from the dense
+definition Ab = -A^-1 Gbar A^-1), the block lower-bidiagonal non-symmetric
+case and its cotangents ("Non-symmetric selected inverse"), and general
+block-sparse SPD patterns ("General sparse selected inverse": its own
+minimum-degree symbolic elimination, then the dense inverse read on the fill).
+The C file states each recursion or definition and every reading taken where
+the pages are silent.
 """
 from __future__ import annotations
 
