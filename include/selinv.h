@@ -65,7 +65,8 @@ typedef enum {
     SELINV_ERR_BAD_TREE = 3,      /* parent array is not one rooted tree per slot */
     SELINV_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
     SELINV_ERR_WORKSPACE = 5,     /* workspace smaller than *_workspace_size */
-    SELINV_ERR_UNSUPPORTED = 6    /* block size beyond selinv_max_block() */
+    SELINV_ERR_UNSUPPORTED = 6,   /* block size beyond selinv_max_block() */
+    SELINV_ERR_HOST_MEMORY = 7    /* a plan's host-side tables could not be allocated */
 } selinv_status;
 
 typedef enum { SELINV_F64 = 0, SELINV_F32 = 1 } selinv_dtype;

@@ -93,6 +93,7 @@ const char *selinv_status_string(selinv_status s)
     case SELINV_ERR_CUDA: return "CUDA error";
     case SELINV_ERR_WORKSPACE: return "workspace too small";
     case SELINV_ERR_UNSUPPORTED: return "block size not supported";
+    case SELINV_ERR_HOST_MEMORY: return "host memory exhausted";
     }
     return "unknown status";
 }

@@ -591,7 +591,7 @@ void selinv_junction_plan_free(selinv_junction_plan_t *pl)
     delete pl;
 }
 
-selinv_status selinv_junction_plan(int64_t n, int64_t m, const int32_t *ei, const int32_t *ej, const int32_t *order,
+static selinv_status junction_plan_impl(int64_t n, int64_t m, const int32_t *ei, const int32_t *ej, const int32_t *order,
                                    selinv_junction_plan_t **out)
 {
     if (!out) return SELINV_ERR_INVALID_ARG;
@@ -852,6 +852,21 @@ selinv_status selinv_junction_plan(int64_t n, int64_t m, const int32_t *ei, cons
         }
     }
     return SELINV_OK;
+}
+
+selinv_status selinv_junction_plan(int64_t n, int64_t m, const int32_t *ei, const int32_t *ej, const int32_t *order,
+                                   selinv_junction_plan_t **out)
+{
+    // host tables are C++ containers: no exception may leave the C ABI
+    try {
+        return junction_plan_impl(n, m, ei, ej, order, out);
+    } catch (const std::bad_alloc &) {
+        if (out) *out = nullptr;
+        return SELINV_ERR_HOST_MEMORY;
+    } catch (...) {
+        if (out) *out = nullptr;
+        return SELINV_ERR_INVALID_ARG;
+    }
 }
 
 selinv_status selinv_junction_plan_info(const selinv_junction_plan_t *pl, int64_t *nnz_S, int32_t *collect_levels,

@@ -22,7 +22,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.environ.get("SELINV_LIB") or os.path.join(_HERE, "libselinv.so")
 
-OK, ERR_INVALID_ARG, ERR_NOT_SPD, ERR_BAD_TREE, ERR_CUDA, ERR_WORKSPACE, ERR_UNSUPPORTED = range(7)
+OK, ERR_INVALID_ARG, ERR_NOT_SPD, ERR_BAD_TREE, ERR_CUDA, ERR_WORKSPACE, ERR_UNSUPPORTED, ERR_HOST_MEMORY = range(8)
 F64, F32 = 0, 1
 
 _lib = None
