@@ -313,6 +313,14 @@ selinv_status selinv_junction_plan_info(const selinv_junction_plan_t *plan, int6
                                         int32_t *collect_levels, int32_t *distribute_levels);
 selinv_status selinv_junction_plan_pattern(const selinv_junction_plan_t *plan, int32_t *S_i, int32_t *S_j,
                                            int32_t *order);
+/* The plan's symbolic phase alone, on the host (no device touched): the same
+ * validation, order and filled pattern as selinv_junction_plan.  Writes
+ * *nnz_S, the first min(nnz_S, capacity) pairs of S to S_i / S_j and the
+ * order to order_out [n] (any of them may be NULL). */
+selinv_status selinv_junction_symbolic(int64_t n, int64_t m, const int32_t *ei, const int32_t *ej,
+                                       const int32_t *order, int64_t *nnz_S, int32_t *S_i, int32_t *S_j,
+                                       int64_t capacity, int32_t *order_out);
+
 /* Kernel launches one selinv_junction call makes with this plan (-1 for NULL). */
 int64_t selinv_junction_plan_launches(const selinv_junction_plan_t *plan);
 size_t selinv_junction_workspace_size(const selinv_junction_plan_t *plan, selinv_dtype dtype, int32_t b,

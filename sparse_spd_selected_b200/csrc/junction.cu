@@ -591,15 +591,29 @@ void selinv_junction_plan_free(selinv_junction_plan_t *pl)
     delete pl;
 }
 
-static selinv_status junction_plan_impl(int64_t n, int64_t m, const int32_t *ei, const int32_t *ej, const int32_t *order,
-                                   selinv_junction_plan_t **out)
+// The symbolic phase: validation, elimination (minimum degree with ties to
+// the smaller node, or the given order), the cliques N(v) and the filled
+// pattern S with its slots (sorted by j, then i).  Host only.
+struct JSym {
+    std::vector<int32_t> seq, pos;
+    std::vector<std::vector<int32_t>> nbr;
+    std::vector<std::pair<int32_t, int32_t>> S;
+    std::map<std::pair<int32_t, int32_t>, int32_t> Sset;
+    std::unordered_map<int64_t, int32_t> input;       // key i * n + j -> input block index
+};
+
+static selinv_status junction_symbolic_impl(int64_t n, int64_t m, const int32_t *ei, const int32_t *ej,
+                                            const int32_t *order, JSym &sy)
 {
-    if (!out) return SELINV_ERR_INVALID_ARG;
-    *out = nullptr;
     if (n < 1 || m < 0 || (m > 0 && (!ei || !ej)) || n >= (int64_t)INT32_MAX / 2) return SELINV_ERR_INVALID_ARG;
+    auto &seq = sy.seq;
+    auto &nbr = sy.nbr;
+    auto &S = sy.S;
+    auto &Sset = sy.Sset;
+    auto &input = sy.input;
+    nbr.assign(n, {});
     // pattern: (i, j), 0 <= j < i < n, no repeats
     std::vector<std::set<int32_t>> adj(n);
-    std::unordered_map<int64_t, int32_t> input;     // key i * n + j -> input block index
     for (int64_t k = 0; k < m; ++k) {
         const int32_t i = ei[k], j = ej[k];
         if (j < 0 || i <= j || i >= n) return SELINV_ERR_INVALID_ARG;
@@ -607,7 +621,7 @@ static selinv_status junction_plan_impl(int64_t n, int64_t m, const int32_t *ei,
         adj[i].insert(j);
         adj[j].insert(i);
     }
-    std::vector<int32_t> seq;
+    seq.clear();
     seq.reserve(n);
     if (order) {
         std::vector<char> seen(n, 0);
@@ -618,11 +632,9 @@ static selinv_status junction_plan_impl(int64_t n, int64_t m, const int32_t *ei,
         }
     }
     // eliminate: N(v) = the neighbours still present; they become a clique
-    std::vector<std::vector<int32_t>> nbr(n);
     std::set<std::pair<int32_t, int32_t>> bydeg;     // (degree, node) of the remaining nodes
     if (!order)
         for (int32_t v = 0; v < n; ++v) bydeg.insert({(int32_t)adj[v].size(), v});
-    std::map<std::pair<int32_t, int32_t>, int32_t> Sset;   // (i, j), i > j -> slot (filled later)
     for (const auto &kv : input) Sset.emplace(std::make_pair((int32_t)(kv.first / n), (int32_t)(kv.first % n)), -1);
     for (int64_t step = 0; step < n; ++step) {
         int32_t v;
@@ -658,10 +670,10 @@ static selinv_status junction_plan_impl(int64_t n, int64_t m, const int32_t *ei,
         nbr[v] = nb;
         seq.push_back(v);
     }
-    std::vector<int32_t> pos(n);
-    for (int64_t k = 0; k < n; ++k) pos[seq[k]] = (int32_t)k;
+    sy.pos.assign(n, 0);
+    for (int64_t k = 0; k < n; ++k) sy.pos[seq[k]] = (int32_t)k;
     // S sorted by (j, i)
-    std::vector<std::pair<int32_t, int32_t>> S(Sset.size());
+    S.assign(Sset.size(), {});
     {
         size_t k = 0;
         for (const auto &kv : Sset) S[k++] = kv.first;
@@ -670,6 +682,23 @@ static selinv_status junction_plan_impl(int64_t n, int64_t m, const int32_t *ei,
         });
         for (size_t q = 0; q < S.size(); ++q) Sset[S[q]] = (int32_t)q;
     }
+    return SELINV_OK;
+}
+
+static selinv_status junction_plan_impl(int64_t n, int64_t m, const int32_t *ei, const int32_t *ej, const int32_t *order,
+                                   selinv_junction_plan_t **out)
+{
+    if (!out) return SELINV_ERR_INVALID_ARG;
+    *out = nullptr;
+    JSym sy;
+    const selinv_status st = junction_symbolic_impl(n, m, ei, ej, order, sy);
+    if (st != SELINV_OK) return st;
+    auto &seq = sy.seq;
+    auto &pos = sy.pos;
+    auto &nbr = sy.nbr;
+    auto &S = sy.S;
+    auto &Sset = sy.Sset;
+    auto &input = sy.input;
     auto slot_of = [&](int32_t x, int32_t y) { return Sset.at(std::make_pair(std::max(x, y), std::min(x, y))); };
     // entries: N(v) in elimination order
     std::vector<int32_t> col_ptr(n + 1, 0);
@@ -865,6 +894,28 @@ selinv_status selinv_junction_plan(int64_t n, int64_t m, const int32_t *ei, cons
         return SELINV_ERR_HOST_MEMORY;
     } catch (...) {
         if (out) *out = nullptr;
+        return SELINV_ERR_INVALID_ARG;
+    }
+}
+
+selinv_status selinv_junction_symbolic(int64_t n, int64_t m, const int32_t *ei, const int32_t *ej, const int32_t *order,
+                                       int64_t *nnz_S, int32_t *S_i, int32_t *S_j, int64_t capacity,
+                                       int32_t *order_out)
+{
+    try {
+        JSym sy;
+        const selinv_status st = junction_symbolic_impl(n, m, ei, ej, order, sy);
+        if (st != SELINV_OK) return st;
+        if (nnz_S) *nnz_S = (int64_t)sy.S.size();
+        for (int64_t q = 0; q < (int64_t)sy.S.size() && q < capacity; ++q) {
+            if (S_i) S_i[q] = sy.S[q].first;
+            if (S_j) S_j[q] = sy.S[q].second;
+        }
+        if (order_out) std::copy(sy.seq.begin(), sy.seq.end(), order_out);
+        return SELINV_OK;
+    } catch (const std::bad_alloc &) {
+        return SELINV_ERR_HOST_MEMORY;
+    } catch (...) {
         return SELINV_ERR_INVALID_ARG;
     }
 }

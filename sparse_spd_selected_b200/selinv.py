@@ -93,6 +93,8 @@ def lib():
         L.selinv_junction_plan_info.restype = ctypes.c_int
         L.selinv_junction_plan_pattern.argtypes = [P, P, P, P]
         L.selinv_junction_plan_pattern.restype = ctypes.c_int
+        L.selinv_junction_symbolic.argtypes = [I64, I64, P, P, P, ctypes.POINTER(I64), P, P, I64, P]
+        L.selinv_junction_symbolic.restype = ctypes.c_int
         L.selinv_junction_plan_launches.argtypes = [P]
         L.selinv_junction_plan_launches.restype = I64
         L.selinv_junction_workspace_size.argtypes = [P, ctypes.c_int, I32, I64]
@@ -542,6 +544,26 @@ def selinv_chain_ad(diag, lower):
     G_lower); gradients reach diag (its lower triangle: the forward reads no
     other entry) and lower through chain_backward."""
     return _SelinvChainFn.apply(diag, lower)
+
+
+def junction_symbolic(n, edge_index, order=None):
+    """The junction plan's symbolic phase on the host (no device): returns
+    (order [n], S_index [2, nnz_S]) exactly as JunctionPlan would."""
+    import numpy as np
+    ei = np.ascontiguousarray(np.asarray(edge_index[0], dtype=np.int32))
+    ej = np.ascontiguousarray(np.asarray(edge_index[1], dtype=np.int32))
+    o = None if order is None else np.ascontiguousarray(np.asarray(order, dtype=np.int32))
+    args = (int(n), ei.size, ei.ctypes.data_as(ctypes.c_void_p), ej.ctypes.data_as(ctypes.c_void_p),
+            None if o is None else o.ctypes.data_as(ctypes.c_void_p))
+    nnz = ctypes.c_int64()
+    _check(lib().selinv_junction_symbolic(*args, ctypes.byref(nnz), None, None, 0, None), "selinv_junction_symbolic")
+    si = np.empty(max(nnz.value, 1), dtype=np.int32)
+    sj = np.empty(max(nnz.value, 1), dtype=np.int32)
+    od = np.empty(int(n), dtype=np.int32)
+    _check(lib().selinv_junction_symbolic(*args, ctypes.byref(nnz), si.ctypes.data_as(ctypes.c_void_p),
+                                          sj.ctypes.data_as(ctypes.c_void_p), nnz.value,
+                                          od.ctypes.data_as(ctypes.c_void_p)), "selinv_junction_symbolic")
+    return od, np.stack([si[:nnz.value], sj[:nnz.value]]).astype(np.int64)
 
 
 class JunctionPlan:
