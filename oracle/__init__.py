@@ -351,6 +351,61 @@ def junction(diag, edge_index, edge_val, order=None, lib=None):
             "info": info.reshape(lead)}
 
 
+def junction_backward(diag, edge_index, edge_val, Gb_diag, Gb_lower, order=None, lib=None):
+    """Cotangents of the general sparse selected inverse (gabp-sparse-inv,
+    "General sparse selected inverse": selinv_junction's gradients reach diag
+    and edge_val).  Gb_diag [..., n, b, b] and Gb_lower [..., nnz_S, b, b] are
+    the cotangents of G_diag and of G_lower on S (junction_symbolic's S for the
+    same order).  The dense definition Ab = -A^-1 Gbar A^-1 (Gbar holding
+    Gb_lower[k] at (S_i[k], S_j[k])) is read back onto what the forward reads:
+    Db = the lower-triangle projection of Ab_vv, and for input block k at
+    (i, j), sitting at (i, j) and transposed at (j, i), Eb[k] = Ab_{i,j} +
+    (Ab_{j,i})^T.  Returns dict with Db, Eb, info."""
+    diag, edge_val = _f64(diag), _f64(edge_val)
+    Gb_diag, Gb_lower = _f64(Gb_diag), _f64(Gb_lower)
+    lead = diag.shape[:-3]
+    n, b = diag.shape[-3], diag.shape[-1]
+    ei = np.asarray(edge_index[0], dtype=np.int64)
+    ej = np.asarray(edge_index[1], dtype=np.int64)
+    _, S = junction_symbolic(n, np.stack([ei, ej]), order)
+    batch = int(np.prod(lead)) if lead else 1
+    d2 = diag.reshape(batch, n, b, b)
+    e2 = edge_val.reshape(batch, len(ei), b, b)
+    gd2 = Gb_diag.reshape(batch, n, b, b)
+    gl2 = Gb_lower.reshape(batch, S.shape[1], b, b)
+    Db = np.zeros((batch, n, b, b))
+    Eb = np.zeros((batch, len(ei), b, b))
+    info = np.full(batch, -1, dtype=np.int32)
+    N = n * b
+    for e in range(batch):
+        A = np.zeros((N, N))
+        Gbar = np.zeros((N, N))
+        for v in range(n):
+            A[v * b:(v + 1) * b, v * b:(v + 1) * b] = np.tril(d2[e, v]) + np.tril(d2[e, v], -1).T
+            Gbar[v * b:(v + 1) * b, v * b:(v + 1) * b] = gd2[e, v]
+        for k, (i, j) in enumerate(zip(ei, ej)):
+            A[i * b:(i + 1) * b, j * b:(j + 1) * b] = e2[e, k]
+            A[j * b:(j + 1) * b, i * b:(i + 1) * b] = e2[e, k].T
+        for k in range(S.shape[1]):
+            i, j = int(S[0, k]), int(S[1, k])
+            Gbar[i * b:(i + 1) * b, j * b:(j + 1) * b] = gl2[e, k]
+        A = np.ascontiguousarray(A)
+        inv = np.empty((N, N))
+        ld = np.zeros(1)
+        rc = _load(lib).oracle_spd_inverse(_ptr(A), N, _ptr(inv), _ptr(ld))
+        if rc != 0:
+            info[e] = (rc - 1) // b
+            continue
+        Ab = -(inv @ Gbar @ inv)
+        for v in range(n):
+            blkv = Ab[v * b:(v + 1) * b, v * b:(v + 1) * b]
+            Db[e, v] = np.tril(blkv + blkv.T, -1) + np.diag(np.diag(blkv))
+        for k, (i, j) in enumerate(zip(ei, ej)):
+            Eb[e, k] = Ab[i * b:(i + 1) * b, j * b:(j + 1) * b] + Ab[j * b:(j + 1) * b, i * b:(i + 1) * b].T
+    return {"Db": Db.reshape(lead + (n, b, b)), "Eb": Eb.reshape(lead + (len(ei), b, b)),
+            "info": info.reshape(lead)}
+
+
 def tree(parent, diag, edge, lib=None):
     """Selected inverse of block-tree SPD matrices.
 

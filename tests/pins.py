@@ -732,6 +732,52 @@ def pin_junction_tree_and_order(lib=None):
     return worst
 
 
+def pin_junction_backward_finite_differences(lib=None):
+    """General sparse cotangents against central differences of the (pinned)
+    junction forward oracle on the pages' 3 x 3 grid; the fill blocks of S
+    carry cotangents too."""
+    E = inputs.grid_edges(3, 3)
+    d, e = inputs.graph_inputs(1, 9, 2, E, seed=81, load=1.0)
+    _, S = oracle.junction_symbolic(9, E)
+    rng = np.random.default_rng(81)
+    gd, gl = rng.standard_normal(d.shape), rng.standard_normal((1, S.shape[1], 2, 2))
+    out = oracle.junction_backward(d, E, e, gd, gl, lib=lib)
+    if (out["info"] != -1).any():
+        return float("inf")
+
+    def loss(dd, ee):
+        o = oracle.junction(dd, E, ee, lib=lib)
+        return float((o["G_diag"] * gd).sum() + (o["G_lower"] * gl).sum())
+
+    h = 1e-5
+    scale = max(1.0, float(np.abs(out["Db"]).max()), float(np.abs(out["Eb"]).max()))
+    worst = 0.0
+    for idx in np.ndindex(*d.shape):
+        dp, dm = d.copy(), d.copy()
+        dp[idx] += h
+        dm[idx] -= h
+        worst = max(worst, abs((loss(dp, e) - loss(dm, e)) / (2 * h) - out["Db"][idx]) / scale)
+    for idx in np.ndindex(*e.shape):
+        ep, em = e.copy(), e.copy()
+        ep[idx] += h
+        em[idx] -= h
+        worst = max(worst, abs((loss(d, ep) - loss(d, em)) / (2 * h) - out["Eb"][idx]) / scale)
+    return worst
+
+
+def pin_junction_backward_path_is_chain(lib=None):
+    """On a path pattern (pairs (i + 1, i)) the general sparse cotangents are
+    the (pinned) chain backward's."""
+    L, b = 6, 3
+    cd, cl, _ = inputs.chain_inputs(1, L, b, seed=82, load=1.0, with_rhs=False)
+    rng = np.random.default_rng(82)
+    cgd, cgl = rng.standard_normal(cd.shape), rng.standard_normal(cl.shape)
+    P = np.array([np.arange(1, L), np.arange(L - 1)])
+    jb = oracle.junction_backward(cd, P, cl, cgd, cgl, lib=lib)
+    cb = oracle.chain_backward(cd, cl, cgd, cgl, lib=lib)
+    return max(rel(jb["Db"], cb["Db"]), rel(jb["Eb"], cb["Bb"]))
+
+
 # name -> (function, tolerance)
 PINS = {
     "tiny_chains_dense": (pin_tiny_chains_dense, 1e-12),
@@ -761,4 +807,6 @@ PINS = {
     "junction_dense": (pin_junction_dense, 1e-11),
     "junction_symbolic": (pin_junction_symbolic, 0.5),
     "junction_tree_and_order": (pin_junction_tree_and_order, 1e-12),
+    "junction_backward_finite_differences": (pin_junction_backward_finite_differences, 1e-7),
+    "junction_backward_path_is_chain": (pin_junction_backward_path_is_chain, 1e-12),
 }
