@@ -931,7 +931,7 @@ using namespace selinv;
 
 extern "C" {
 
-selinv_status selinv_tree_plan(const int32_t *parent, int64_t trees, int64_t n, selinv_tree_plan_t **out)
+static selinv_status tree_plan_impl(const int32_t *parent, int64_t trees, int64_t n, selinv_tree_plan_t **out)
 {
     if (!out) return SELINV_ERR_INVALID_ARG;
     *out = nullptr;
@@ -1024,6 +1024,20 @@ selinv_status selinv_tree_plan(const int32_t *parent, int64_t trees, int64_t n, 
     }
     *out = pl;
     return SELINV_OK;
+}
+
+selinv_status selinv_tree_plan(const int32_t *parent, int64_t trees, int64_t n, selinv_tree_plan_t **out)
+{
+    // host tables are C++ containers: no exception may leave the C ABI
+    try {
+        return tree_plan_impl(parent, trees, n, out);
+    } catch (const std::bad_alloc &) {
+        if (out) *out = nullptr;
+        return SELINV_ERR_HOST_MEMORY;
+    } catch (...) {
+        if (out) *out = nullptr;
+        return SELINV_ERR_INVALID_ARG;
+    }
 }
 
 void selinv_tree_plan_free(selinv_tree_plan_t *pl)
