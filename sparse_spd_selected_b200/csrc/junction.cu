@@ -31,6 +31,7 @@
 #include <climits>
 #include <cmath>
 #include <map>
+#include <memory>
 #include <new>
 #include <set>
 #include <unordered_map>
@@ -828,8 +829,12 @@ static selinv_status junction_plan_impl(int64_t n, int64_t m, const int32_t *ei,
                         pair[pair_ptr[v] + a * d + c] = x == y ? -(x + 1) : 2 * slot_of(x, y) + (x < y ? 1 : 0);
                     }
             }
-            auto *pl = new (std::nothrow) selinv_junction_plan_s();
-            if (!pl) return SELINV_ERR_INVALID_ARG;
+            // held by a unique_ptr until handed out, so a host allocation
+            // failure below (caught at the C ABI) releases it and its tables
+            std::unique_ptr<selinv_junction_plan_s, void (*)(selinv_junction_plan_s *)> hold(
+                new (std::nothrow) selinv_junction_plan_s(), selinv_junction_plan_free);
+            if (!hold) return SELINV_ERR_HOST_MEMORY;
+            selinv_junction_plan_s *pl = hold.get();
             pl->n = n;
             pl->m = m;
             pl->nnz = (int64_t)S.size();
@@ -873,11 +878,8 @@ static selinv_status junction_plan_impl(int64_t n, int64_t m, const int32_t *ei,
             up(&pl->d_de_ent, de_ent);
             up(&pl->d_de_node, de_node);
             up(&pl->d_de_a, de_a);
-            if (!ok) {
-                selinv_junction_plan_free(pl);
-                return SELINV_ERR_CUDA;
-            }
-            *out = pl;
+            if (!ok) return SELINV_ERR_CUDA;
+            *out = hold.release();
         }
     }
     return SELINV_OK;

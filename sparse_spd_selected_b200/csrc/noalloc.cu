@@ -90,8 +90,15 @@ selinv_status selinv_chain_noalloc(selinv_dtype dtype, int64_t batch, int64_t L,
         !aligned_to(G_lower, es) || !aligned_to(rhs, es) || !aligned_to(x, es) || !aligned_to(logdet, 8) ||
         !aligned_to(info, 4))
         return SELINV_ERR_INVALID_ARG;
-    const size_t need = (want_g || want_x) ? selinv::chain_small_workspace(es, batch, L) : 0;
-    if (need > NOALLOC_SCRATCH_BYTES) return SELINV_ERR_WORKSPACE;     // beyond the built-in scratch
+    // Scratch is batch * (L-1) slots of 192 elements when G or x is asked for.
+    // Compared by division so that a huge batch or L cannot wrap the product
+    // below the limit.
+    if ((want_g || want_x) && L > 1 && batch > 0) {
+        const size_t per_chain_limit = NOALLOC_SCRATCH_BYTES / (192 * es);     // slots that fit
+        if ((uint64_t)(L - 1) > per_chain_limit || (uint64_t)batch > per_chain_limit / (uint64_t)(L - 1))
+            return SELINV_ERR_WORKSPACE;                                    // beyond the built-in scratch
+        if (selinv::chain_small_workspace(es, batch, L) > NOALLOC_SCRATCH_BYTES) return SELINV_ERR_WORKSPACE;
+    }
     if (batch == 0) return SELINV_OK;
     void *scratch = scratch_for_current_device();
     if (scratch == nullptr) return SELINV_ERR_CUDA;

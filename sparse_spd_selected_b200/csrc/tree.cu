@@ -25,6 +25,7 @@
 // (S_v^-1 E_v^T G_edge[v] = W_v^T G_edge[v]).  Roots get G = S^-1 in collect.
 #include <algorithm>
 #include <climits>
+#include <memory>
 #include <new>
 #include <vector>
 
@@ -982,8 +983,13 @@ static selinv_status tree_plan_impl(const int32_t *parent, int64_t trees, int64_
         H = std::max(H, height[v]);
         Dm = std::max(Dm, depth[v]);
     }
-    auto *pl = new (std::nothrow) selinv_tree_plan_s();
-    if (!pl) return SELINV_ERR_INVALID_ARG;
+    // held by a unique_ptr until handed out, so a host allocation failure
+    // below (caught at the C ABI) releases it and its device tables
+    std::unique_ptr<selinv_tree_plan_s, void (*)(selinv_tree_plan_s *)> hold(new (std::nothrow)
+                                                                                 selinv_tree_plan_s(),
+                                                                             selinv_tree_plan_free);
+    if (!hold) return SELINV_ERR_HOST_MEMORY;
+    selinv_tree_plan_s *pl = hold.get();
     pl->trees = trees;
     pl->n = n;
     cudaGetDevice(&pl->device);
@@ -1018,11 +1024,8 @@ static selinv_status tree_plan_impl(const int32_t *parent, int64_t trees, int64_
     up(&pl->d_child_ptr, cnt);
     up(&pl->d_child_idx, child);
     up(&pl->d_parent, gparent);
-    if (!ok) {
-        selinv_tree_plan_free(pl);
-        return SELINV_ERR_CUDA;
-    }
-    *out = pl;
+    if (!ok) return SELINV_ERR_CUDA;
+    *out = hold.release();
     return SELINV_OK;
 }
 

@@ -196,3 +196,19 @@ def test_junction_plan_rejects_bad_patterns(lib):
     assert plan([1], [0], 3, order=[0, 0, 1]) == selinv.ERR_INVALID_ARG   # not a permutation
     assert lib.selinv_junction(None, 0, 4, 1, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 1 << 30, None) == \
         selinv.ERR_INVALID_ARG
+
+
+def test_noalloc_rejects_oversized_requests_before_any_device_call(lib):
+    """The allocation-free chain entry point checks its request against the
+    built-in scratch by division, so products that wrap 64 bits are refused."""
+    f = lib.selinv_chain_noalloc
+    P = ctypes.c_void_p
+    f.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32] + [P] * 9
+    f.restype = ctypes.c_int
+    # dtype, batch, L, b, diag, lower, G_diag, G_lower, logdet, rhs, x, info, stream
+    assert f(0, 1 << 61, 64, 16, FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE, None) == selinv.ERR_WORKSPACE
+    assert f(0, 3, (1 << 62) + 1, 16, FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE, None) == selinv.ERR_WORKSPACE
+    assert f(1, 1 << 40, 1 << 40, 4, FAKE, FAKE, None, None, None, FAKE, FAKE, FAKE, None) == selinv.ERR_WORKSPACE
+    assert f(0, 1, 4, 17, FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE, None) == selinv.ERR_UNSUPPORTED
+    assert f(0, 1, 4, 4, FAKE, FAKE, FAKE, None, None, None, None, FAKE, None) == selinv.ERR_INVALID_ARG
+    assert f(0, 0, 4, 4, FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE, None) == selinv.OK

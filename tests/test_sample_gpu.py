@@ -7,7 +7,7 @@ import torch
 import oracle
 from sparse_spd_selected_b200 import inputs, selinv
 from tests.dense import chain_dense, rel
-from tests.parity import TOL, host, logdet_err, to_dev, worst
+from tests.parity import TOL, host, logdet_err, to_dev, worst, worst_vec
 
 pytestmark = pytest.mark.gpu
 
@@ -28,7 +28,7 @@ def draw(batch, L, b, seed, with_rhs, dtype, load=1.0):
 @pytest.mark.parametrize("with_rhs", [False, True])
 def test_sample_f64(cuda_ok, b, L, with_rhs):
     out, ref = draw(3, L, b, 8000 + 10 * b + L, with_rhs, torch.float64)
-    assert worst(host(out["eta"]), ref["eta"]) <= TOL[torch.float64]
+    assert worst_vec(host(out["eta"]), ref["eta"]) <= TOL[torch.float64]
     assert logdet_err(host(out["logdet"]), ref["logdet"]) <= TOL[torch.float64]
     assert (host(out["info"]) == -1).all()
 
@@ -36,7 +36,7 @@ def test_sample_f64(cuda_ok, b, L, with_rhs):
 @pytest.mark.parametrize("b,L", [(16, 9), (5, 12)])
 def test_sample_f32(cuda_ok, b, L):
     out, ref = draw(4, L, b, 8100 + b, True, torch.float32)
-    assert worst(host(out["eta"]), ref["eta"]) <= TOL[torch.float32]
+    assert worst_vec(host(out["eta"]), ref["eta"]) <= TOL[torch.float32]
 
 
 def test_sample_standard_basis_is_the_cholesky_factor(cuda_ok):
@@ -72,7 +72,7 @@ def test_sample_full_size_b16(cuda_ok):
     out = selinv.chain_sample(dd, ll, zz, rr)
     pick = [0, 1, 2047, 4095]
     ref = oracle.chain_sample(g["diag"][pick], g["lower"][pick], z[pick], rhs=g["rhs"][pick])
-    assert worst(host(out["eta"][pick]), ref["eta"]) <= TOL[torch.float64]
+    assert worst_vec(host(out["eta"][pick]), ref["eta"]) <= TOL[torch.float64]
     assert logdet_err(host(out["logdet"][pick]), ref["logdet"]) <= TOL[torch.float64]
 
 
@@ -95,7 +95,7 @@ def test_sample_not_spd_and_unsupported(cuda_ok):
 def test_sample_large_blocks_f64(cuda_ok, b, L):
     """Draws through the CTA kernel (R_i z_i met inside its blocked inverse)."""
     out, ref = draw(2, L, b, 8500 + b + L, L != 3, torch.float64)
-    assert worst(host(out["eta"]), ref["eta"]) <= TOL[torch.float64]
+    assert worst_vec(host(out["eta"]), ref["eta"]) <= TOL[torch.float64]
     assert logdet_err(host(out["logdet"]), ref["logdet"]) <= TOL[torch.float64]
 
 
@@ -107,5 +107,5 @@ def test_sample_grid_sampled(cuda_ok):
     out = selinv.chain_sample(d, l, z, r)
     pick = [0, 255]
     ref = oracle.chain_sample(host(d[pick]), host(l[pick]), host(z[pick]), rhs=host(r[pick]))
-    assert worst(host(out["eta"][pick]), ref["eta"]) <= TOL[torch.float64]
+    assert worst_vec(host(out["eta"][pick]), ref["eta"]) <= TOL[torch.float64]
     assert logdet_err(host(out["logdet"][pick]), ref["logdet"]) <= TOL[torch.float64]

@@ -7,7 +7,7 @@ import torch
 import oracle
 from sparse_spd_selected_b200 import inputs, selinv
 from tests.dense import balanced_parent, path_parent, star_parent
-from tests.parity import TOL, host, logdet_err, to_dev, worst
+from tests.parity import TOL, host, logdet_err, to_dev, worst, worst_vec
 
 pytestmark = pytest.mark.gpu
 
@@ -31,7 +31,7 @@ def test_tree_sample_topologies(cuda_ok, b):
     diag, edge = inputs.tree_inputs_from_parent(P, b, seed=200 + b, load=0.5)
     z = rng.standard_normal((5, n, b))
     out, ref = draws(P, diag, edge, z)
-    assert worst(host(out["eta"]), ref["eta"]) <= TOL[torch.float64]
+    assert worst_vec(host(out["eta"]), ref["eta"]) <= TOL[torch.float64]
     assert logdet_err(host(out["logdet"]), ref["logdet"]) <= TOL[torch.float64]
     assert (host(out["info"]) == -1).all()
 
@@ -41,13 +41,13 @@ def test_tree_sample_single_node_and_f32(cuda_ok):
     diag, edge = inputs.tree_inputs_from_parent(P, 16, seed=300, load=1.0)
     z = np.random.default_rng(301).standard_normal((1, 1, 16))
     out, ref = draws(P, diag, edge, z)
-    assert worst(host(out["eta"]), ref["eta"]) <= TOL[torch.float64]
+    assert worst_vec(host(out["eta"]), ref["eta"]) <= TOL[torch.float64]
     rng = np.random.default_rng(302)
     P = np.stack([inputs.random_parent(rng, 50) for _ in range(3)])
     diag, edge = inputs.tree_inputs_from_parent(P, 16, seed=303, load=1.0)
     z = rng.standard_normal((3, 50, 16))
     out, ref = draws(P, diag, edge, z, torch.float32)
-    assert worst(host(out["eta"]), ref["eta"]) <= TOL[torch.float32]
+    assert worst_vec(host(out["eta"]), ref["eta"]) <= TOL[torch.float32]
 
 
 def test_tree_sample_full_size_forest(cuda_ok):
@@ -60,7 +60,7 @@ def test_tree_sample_full_size_forest(cuda_ok):
                              to_dev(z, torch.float64))
     pick = [0, 7]
     ref = oracle.tree_sample(g["parent"][pick], g["diag"][pick], g["edge"][pick], z[pick])
-    assert worst(host(out["eta"][pick]), ref["eta"]) <= TOL[torch.float64]
+    assert worst_vec(host(out["eta"][pick]), ref["eta"]) <= TOL[torch.float64]
     assert logdet_err(host(out["logdet"][pick]), ref["logdet"]) <= TOL[torch.float64]
 
 
