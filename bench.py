@@ -70,6 +70,10 @@ def parse():
                          "cotangents of diag and lower (edge) from those of G_diag and G_lower (G_edge); "
                          "chains and trees, b <= 16; bidiag: the selected inverse of a block "
                          "lower-bidiagonal matrix with general blocks of the chain workload's shape (b <= 16)")
+    ap.add_argument("--configs", default="all", choices=["all", "one"],
+                    help="all (default): with the default workload and op, also measure every other workload "
+                         "of the metric (and the float32 repeat) and report them under per_config; one: the "
+                         "named workload only")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -364,14 +368,33 @@ def job_throughput(world: int, units_per_rank: int, steps: int, max_ms: float) -
 
 # ------------------------------------------------------------------ arms
 
+# The workloads the metric is quoted on, one bench line: the headline
+# (4096 chains of 64 blocks of 16) carries the top-level keys; every workload,
+# the float32 repeat of the long b = 32 chains included, is measured in the
+# same run and reported under "per_config".
+HEADLINE = "chain_4096x64_b16"
+PER_CONFIG = [("chain_1x8_b4", "f64"), ("chain_4096x64_b16", "f64"), ("chain_64x4096_b32", "f64"),
+              ("chain_64x4096_b32", "f32"), ("forest_8x32768_b16", "f64"), ("grid_256x128_b128", "f64")]
+
+
+def config_dict(w, batch, world, op, full_size):
+    """The bench line's `config`: the same dict for both arms of one workload."""
+    l2 = "inputs larger than L2 (no flush)" if w.L * w.batch * w.b * w.b * 8 > 256 << 20 else \
+        "fits in L2 (latency case; device time from a CUDA graph of back-to-back calls)"
+    return {"workload": w.name if full_size else f"{w.name} (batch {batch}, length {w.L} per GPU)",
+            "global_batch": batch * world, "block": w.b, "L_or_n": w.L,
+            "solve": bool(w.solve) and op in ("selinv", "sample"), "op": op,
+            "parallelism": f"dp{world} (independent chains per GPU)", "l2": l2}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = inputs.WORKLOADS[args.workload]
+    w0 = inputs.WORKLOADS[args.workload]
     import oracle
     oracle.build()
-    w, note = oracle_workload(w, args.op)
+    w, note = oracle_workload(w0, args.op)
     n_per_step = {"chain": 64, "tree": 1, "grid": 1, "junction": 4}[w.kind]
     if w.kind == "chain" and w.L * w.b ** 3 > 64 * 16 ** 3 * 64:
         n_per_step = 2
@@ -388,14 +411,15 @@ def run_reference(args):
     blocks = len(elems) * w.L
     value = blocks * len(times) / sum(times)
     sample = f"{len(elems)} of {w.batch} {'trees' if w.kind == 'tree' else 'chains'} per step{note}"
+    full_size = args.length is None and (args.batch is None or args.batch == w0.batch)
     line = {
-        "impl": "reference", "metric": metric_name(args.op, "f64"), "value": value, "unit": "blocks/s",
+        "impl": "reference", "metric": metric_name(args.op, args.dtype), "value": value, "unit": "blocks/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "global_batch": w.batch * args.gpus, "block": w.b, "L": w.L},
+        "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
+        "config": config_dict(w0, args.batch or w0.batch, args.gpus, args.op, full_size),
         "cpu_baseline": {"value": value, "unit": "blocks/s", "cores": oracle.threads(), "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample + " (the oracle computes in float64)"},
         "e2e": {"value": value, "unit": "blocks/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -407,54 +431,43 @@ def metric_name(op, dtype):
     return f"{what} blocks/s ({'fp64' if dtype == 'f64' else 'fp32'})"
 
 
-def run_ours(args):
+_FP64_PEAK = {}
+
+
+def fp64_peak_cached(torch):
+    if "v" not in _FP64_PEAK:
+        _FP64_PEAK["v"] = fp64_peak_tflops(torch)
+    return _FP64_PEAK["v"]
+
+
+def build_step(w, dtype, op, batch, elems):
+    """Inputs, outputs, workspace and the step closure of one workload.
+
+    Returns a dict with step, out, dev_in, host_in, kernel, launches_per_step."""
     import torch
-    import torch.distributed as dist
     from sparse_spd_selected_b200 import selinv
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device")
-    torch.cuda.set_device(local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-
-    w = inputs.WORKLOADS[args.workload]
-    full_size = args.length is None and (args.batch is None or args.batch == w.batch)
-    if args.length is not None:
-        w = dataclasses.replace(w, L=args.length)
-    batch = args.batch or w.batch
-    tdt = torch.float64 if args.dtype == "f64" else torch.float32
-    es = 8 if args.dtype == "f64" else 4
-    # cpu baseline first (host only), so nothing forks after CUDA work starts
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, args.dtype, args.op)
-
-    elems = shard_elements(rank, batch)
-    stream = torch.cuda.current_stream()
+    tdt = torch.float64 if dtype == "f64" else torch.float32
     if w.kind == "grid":
         diag, lower, rhs, _ = inputs.grid_inputs_torch(batch, w.b, w.seed, "cuda", tdt, w.solve)
         host_in = {"diag": diag.cpu().pin_memory(), "lower": lower.cpu().pin_memory()}
         if rhs is not None:
             host_in["rhs"] = rhs.cpu().pin_memory()
-        if args.op == "sample":
+        if op == "sample":
             host_in["z"] = torch.from_numpy(inputs.standard_normals(batch, w.L, w.b, w.seed, elems)).to(
                 tdt).pin_memory()
+        g = None
     else:
         g = inputs.generate(w, elements=elems)   # per-element seeds: rank r owns its own slice
-        if args.op == "bidiag":
+        if op == "bidiag":
             if w.kind != "chain" or w.b > 16:
                 raise SystemExit("--op bidiag runs on chain workload shapes with b <= 16")
             g = dict(zip(("diag", "lower"), inputs.bidiag_inputs(w.batch, w.L, w.b, w.seed, 2.0, elems)))
-        if args.op == "sample":
-            if w.b > 16 and args.dtype != "f64":
+        if op == "sample":
+            if w.b > 16 and dtype != "f64":
                 raise SystemExit("--op sample with b > 16 runs in float64 only")
             g["z"] = inputs.standard_normals(w.batch, w.L, w.b, w.seed, elems)
-        if args.op == "backward":
+        if op == "backward":
             if w.b > 16:
                 raise SystemExit("--op backward runs on workloads with b <= 16")
             g.pop("rhs", None)
@@ -462,8 +475,11 @@ def run_ours(args):
                 g["Gb_diag"], g["Gb_edge"] = inputs.tree_cotangents(w.batch, w.L, w.b, w.seed, elems)
             else:
                 g["Gb_diag"], g["Gb_lower"] = inputs.cotangents(w.batch, w.L, w.b, w.seed, elems)
-        host_in = {k: torch.from_numpy(v).to(tdt).pin_memory() for k, v in g.items()
-                   if v is not None and k not in ("parent", "edge_index")}
+        host_in = {}
+        for k in [k for k, v in g.items() if v is not None and k not in ("parent", "edge_index")]:
+            host_in[k] = torch.from_numpy(g[k]).to(tdt).pin_memory()
+            if k != "tau":
+                g[k] = None                      # free the float64 host copy as we go
         dev_in = {k: v.to("cuda", non_blocking=True) for k, v in host_in.items()}
         torch.cuda.synchronize()
 
@@ -487,13 +503,12 @@ def run_ours(args):
                "logdet": torch.empty(batch, dtype=torch.float64, device="cuda"),
                "info": torch.empty(batch, dtype=torch.int32, device="cuda")}
         ws = torch.empty(plan.workspace_size(tdt, w.b), dtype=torch.uint8, device="cuda")
-        if args.op == "backward":
+        if op == "backward":
             fwd = selinv.selinv_tree(plan, dev_in["diag"], dev_in["edge"])
             for k in ("G_diag", "G_edge"):
                 dev_in[k] = fwd[k]
                 host_in[k] = fwd[k].cpu().pin_memory()
             kernel = "tree_bw_collect_kernel"
-            launches_per_step = 4 if w.L > 1 else 3
             out = {"Db": torch.empty_like(dev_in["diag"]), "Eb": torch.empty_like(dev_in["diag"]),
                    "info": out["info"]}
             ws = torch.empty(plan.backward_workspace_size(tdt, w.b), dtype=torch.uint8, device="cuda")
@@ -501,7 +516,7 @@ def run_ours(args):
             def step():
                 selinv.tree_backward(plan, dev_in["diag"], dev_in["edge"], dev_in["G_diag"], dev_in["G_edge"],
                                      dev_in["Gb_diag"], dev_in["Gb_edge"], check=False, out=out, workspace=ws)
-        elif args.op == "sample":
+        elif op == "sample":
             kernel = "tree_collect_kernel (draw mode)"
             out = {"eta": torch.empty_like(dev_in["z"]), "logdet": out["logdet"], "info": out["info"]}
 
@@ -518,7 +533,7 @@ def run_ours(args):
             dev_in = {"diag": diag, "lower": lower}
             if rhs is not None:
                 dev_in["rhs"] = rhs
-            if args.op == "sample":
+            if op == "sample":
                 dev_in["z"] = host_in["z"].to("cuda")
         L, b = w.L, w.b
         out = {"G_diag": torch.empty((batch, L, b, b), dtype=tdt, device="cuda"),
@@ -531,11 +546,11 @@ def run_ours(args):
                          dtype=torch.uint8, device="cuda")
         launches_per_step = 1
         segments = selinv.chain_segments(batch, L, b, True, "rhs" in dev_in)
-        if args.op == "bidiag":
+        if op == "bidiag":
             kernel = "bidiag_inverse_kernel"
             out = {"G_diag": torch.empty_like(dev_in["diag"]), "G_lower": torch.empty_like(dev_in["lower"]),
                    "info": torch.empty(batch, dtype=torch.int32, device="cuda")}
-        elif args.op == "backward":
+        elif op == "backward":
             # the forward's outputs are the backward's inputs (computed once, outside the timing)
             fwd = selinv.selinv_chain(dev_in["diag"], dev_in["lower"])
             for k in ("G_diag", "G_lower"):
@@ -546,7 +561,7 @@ def run_ours(args):
                    "info": torch.empty(batch, dtype=torch.int32, device="cuda")}
             ws = torch.empty(max(selinv.chain_backward_workspace_size(tdt, batch, L, b), 1), dtype=torch.uint8,
                              device="cuda")
-        elif args.op == "sample":
+        elif op == "sample":
             kernel = "chain_small_kernel (draw mode)" if b <= 16 else "chain_large_kernel (draw mode)"
             out = {"eta": torch.empty((batch, L, b), dtype=tdt, device="cuda"),
                    "logdet": torch.empty(batch, dtype=torch.float64, device="cuda"),
@@ -564,14 +579,14 @@ def run_ours(args):
         else:
             kernel = "chain_large_kernel"
 
-        if args.op == "bidiag":
+        if op == "bidiag":
             def step():
                 selinv.bidiag(dev_in["diag"], dev_in["lower"], check=False, out=out)
-        elif args.op == "backward":
+        elif op == "backward":
             def step():
                 selinv.chain_backward(dev_in["diag"], dev_in["lower"], dev_in["G_diag"], dev_in["G_lower"],
                                       dev_in["Gb_diag"], dev_in["Gb_lower"], check=False, out=out, workspace=ws)
-        elif args.op == "sample":
+        elif op == "sample":
             def step():
                 selinv.chain_sample(dev_in["diag"], dev_in["lower"], dev_in["z"], dev_in.get("rhs"), check=False,
                                     out=out, workspace=ws)
@@ -579,15 +594,60 @@ def run_ours(args):
             def step():
                 selinv.selinv_chain(dev_in["diag"], dev_in["lower"], dev_in.get("rhs"), check=False, out=out,
                                     workspace=ws)
+    return {"step": step, "out": out, "dev_in": dev_in, "host_in": host_in, "kernel": kernel,
+            "launches_per_step": launches_per_step, "keep": (ws,)}
+
+
+def graph_device_us(step, stream, reps=50):
+    """Device time of one call with the host out of the way: `reps` calls captured
+    in one CUDA graph and replayed (the library's calls are stream-ordered and
+    allocate nothing when given outputs and workspace)."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(stream)
+    with torch.cuda.stream(s):
+        step()                                   # warm the capture stream
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=s):
+        for _ in range(reps):
+            step()
+    with torch.cuda.stream(s):                   # replays run on the current stream: time them there
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        for _ in range(5):
+            g.replay()
+        e.record(s)
+    torch.cuda.synchronize()
+    us = a.elapsed_time(e) * 1e3 / (5 * reps)
+    del g
+    return us
+
+
+def measure(w, dtype, op, batch, steps, warmup, rank, world, local, full_size, want_cpu, want_e2e):
+    """One workload, timed as the bench line reports it."""
+    import torch
+    import torch.distributed as dist
+
+    es = 8 if dtype == "f64" else 4
+    cpu = cpu_baseline(w, dtype, op) if want_cpu else None     # host only, before the GPU work
+    elems = shard_elements(rank, batch)
+    stream = torch.cuda.current_stream()
+    S = build_step(w, dtype, op, batch, elems)
+    step, out, dev_in, host_in = S["step"], S["out"], S["dev_in"], S["host_in"]
+    kernel, launches_per_step = S["kernel"], S["launches_per_step"]
 
     # correctness guard: the last warm-up step must report every element SPD
-    for _ in range(max(args.warmup, 3)):
+    for _ in range(max(warmup, 3)):
         step()
     torch.cuda.synchronize()
     if bool((out["info"] != -1).any()):
-        raise SystemExit("bench input reported not SPD")
+        raise SystemExit(f"bench input reported not SPD ({w.name})")
 
-    K = args.steps
+    K = steps
     k_start = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     k_end = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -614,10 +674,12 @@ def run_ours(args):
     elapsed_ms = max_over_ranks(elapsed_ms, world, "cuda")
     nodes_per_rank = batch * w.L
     value = job_throughput(world, nodes_per_rank, K, elapsed_ms)
+    latency_case = w.L * w.batch * w.b * w.b * 8 <= 256 << 20
+    device_us = graph_device_us(step, stream) if latency_case else None
 
     # end to end through the same call, inputs from pinned host memory, outputs read back
     e2e = None
-    if not args.no_e2e and host_in is not None:
+    if want_e2e and host_in is not None:
         host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in out.items()}
         Ke = max(1, min(3, K))
         if world > 1:
@@ -627,7 +689,8 @@ def run_ours(args):
         s.record(stream)
         for _ in range(Ke):
             for k, v in host_in.items():
-                dev_in[k].copy_(v, non_blocking=True)
+                if k in dev_in:
+                    dev_in[k].copy_(v, non_blocking=True)
             step()
             for k, v in out.items():
                 host_out[k].copy_(v, non_blocking=True)
@@ -635,61 +698,116 @@ def run_ours(args):
         torch.cuda.synchronize()
         e2e_ms = s.elapsed_time(e)
         e2e_ms = max_over_ranks(e2e_ms, world, "cuda")
-        h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+        h2d = sum(v.numel() * v.element_size() for k, v in host_in.items() if k in dev_in)
         d2h = sum(v.numel() * v.element_size() for v in out.values())
         e2e = {"value": job_throughput(world, nodes_per_rank, Ke, e2e_ms), "unit": "blocks/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     hbm, src = hbm_peak()
-    byt = algorithmic_bytes(w, es, batch, args.op)
-    hbm_achieved = byt / (kernel_ms / 1e3) / 1e9
-    flops = algorithmic_flops(w, batch, args.op)
-    flop_rate = flops / (kernel_ms / 1e3) / 1e12
+    byt = algorithmic_bytes(w, es, batch, op)
+    t_ms = device_us / 1e3 if device_us is not None else kernel_ms
+    hbm_achieved = byt / (t_ms / 1e3) / 1e9
+    flops = algorithmic_flops(w, batch, op)
+    flop_rate = flops / (t_ms / 1e3) / 1e12
     traffic = profiled_traffic(kernel, w.name) if full_size else None
+    if traffic is not None and dtype != "f64":
+        traffic = None                         # the committed summaries are float64 captures
     hbm_src = f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback 6650 GB/s"
     ridge = 35.5e12 / (hbm * 1e9)                      # FP64 flop per byte where the two roofs meet
     contraction = w.kind == "junction" and flops / byt > ridge
-    if (w.b >= 32 or args.op == "backward" or contraction) and args.dtype == "f64":
+    hbm_side = {"achieved": hbm_achieved, "peak": hbm, "unit": "GB/s", "frac": hbm_achieved / hbm,
+                "peak_source": hbm_src}
+    if (w.b >= 32 or op == "backward" or contraction) and dtype == "f64":
         # arithmetic intensity 7 b^3 / (32 b^2) flop/byte: past the FP64 ridge from b = 32 on
-        peak = fp64_peak_tflops(torch)
+        peak = fp64_peak_cached(torch)
         roof = {"bound": "tensor", "achieved": flop_rate, "peak": peak, "unit": "TFLOP/s",
                 "frac": flop_rate / peak, "traffic": traffic,
                 "peak_source": "measured in this run: cuBLAS DGEMM 8192^3 (FP64 tensor cores)",
-                "algorithmic_flops_per_launch": flops, "kernel": kernel,
-                "hbm": {"achieved": hbm_achieved, "peak": hbm, "unit": "GB/s", "frac": hbm_achieved / hbm,
-                        "peak_source": hbm_src}}
+                "algorithmic_flops_per_launch": flops, "kernel": kernel, "hbm": hbm_side}
     elif w.b >= 32:
         # fp32 runs on the FP32 pipes: 148 SMs x 128 lanes x 2 flop x 1965 MHz
         peak = 148 * 128 * 2 * 1.965e9 / 1e12
         roof = {"bound": "alu", "achieved": flop_rate, "peak": peak, "unit": "TFLOP/s",
                 "frac": flop_rate / peak, "traffic": traffic,
                 "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 flop x 1965 MHz max SM clock",
-                "algorithmic_flops_per_launch": flops, "kernel": kernel,
-                "hbm": {"achieved": hbm_achieved, "peak": hbm, "unit": "GB/s", "frac": hbm_achieved / hbm,
-                        "peak_source": hbm_src}}
+                "algorithmic_flops_per_launch": flops, "kernel": kernel, "hbm": hbm_side}
     else:
         roof = {"bound": "hbm", "achieved": hbm_achieved, "peak": hbm, "unit": "GB/s", "frac": hbm_achieved / hbm,
                 "traffic": traffic, "peak_source": hbm_src, "algorithmic_bytes_per_launch": byt, "kernel": kernel}
+    if latency_case:
+        roof["note"] = ("latency case: one warp works 8 dependent blocks; achieved uses the device time of "
+                        "one call from a CUDA graph, not a bandwidth claim")
+    res = {"value": value, "ms_per_step": elapsed_ms / K, "kernel_ms": kernel_ms, "roofline": roof,
+           "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": K * launches_per_step, "clocks": clk.summary(),
+           "kernel": kernel, "config": config_dict(w, batch, world, op, full_size), "dtype": dtype}
+    if device_us is not None:
+        res["device_us_per_call"] = device_us
+        res["host_us_per_call"] = kernel_ms * 1e3
+    del S, step, out, dev_in, host_in
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    w = inputs.WORKLOADS[args.workload]
+    full_size = args.length is None and (args.batch is None or args.batch == w.batch)
+    if args.length is not None:
+        w = dataclasses.replace(w, L=args.length)
+    batch = args.batch or w.batch
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    head = measure(w, args.dtype, args.op, batch, args.steps, args.warmup, rank, world, local, full_size,
+                   want_cpu, not args.no_e2e)
+    per_config = None
+    if args.configs == "all" and world == 1 and full_size and args.op == "selinv" and w.name == HEADLINE \
+            and args.dtype == "f64":
+        per_config = {}
+        for name, dt in PER_CONFIG:
+            key = name if dt == "f64" else f"{name}_{dt}"
+            if name == w.name and dt == args.dtype:
+                r = head
+            else:
+                wc = inputs.WORKLOADS[name]
+                r = measure(wc, dt, "selinv", wc.batch, args.steps, args.warmup, rank, world, local, True,
+                            want_cpu, not args.no_e2e)
+            per_config[key] = {k: r[k] for k in ("value", "ms_per_step", "kernel_ms", "roofline", "cpu_baseline",
+                                                 "e2e", "clocks", "gpu_launches", "dtype", "config")}
+            for k in ("device_us_per_call", "host_us_per_call"):
+                if k in r:
+                    per_config[key][k] = r[k]
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
         return 0
     line = {
         "metric": metric_name(args.op, args.dtype),
-        "value": value, "unit": "blocks/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
-        "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "value": head["value"], "unit": "blocks/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": args.dtype, "data": "synthetic",
-        "config": {"workload": w.name if full_size else f"{w.name} (batch {batch}, length {w.L} per GPU)",
-                   "global_batch": batch * world, "block": w.b, "L_or_n": w.L,
-                   "solve": bool(w.solve), "op": args.op, "parallelism": f"dp{world} (independent chains per GPU)",
-                   "l2": "inputs larger than L2 (no flush)"},
-        "roofline": roof,
-        "cpu_baseline": cpu,
-        "e2e": e2e,
-        "gpu_launches": K * launches_per_step,
-        "clocks": clk.summary(),
-        "kernel_ms": kernel_ms,
+        "config": head["config"],
+        "roofline": head["roofline"],
+        "cpu_baseline": head["cpu_baseline"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"] + sum(
+            v["gpu_launches"] for k, v in (per_config or {}).items() if k != w.name),
+        "clocks": head["clocks"],
+        "kernel_ms": head["kernel_ms"],
     }
+    if per_config is not None:
+        line["per_config"] = per_config
     print(json.dumps(line), flush=True)
     return 0
 

@@ -38,6 +38,9 @@
  *     halves' first failures.  The outputs of such an element are
  *     unspecified.  Kernels never trap.  A tree distribute step whose wait
  *     for its parent timed out (not expected for a valid plan) reports -2.
+ *     With SELINV_CHECK, an element holding a non-finite input entry
+ *     reports -3 - k instead, k the first block (chain) or node (tree)
+ *     holding one.
  *   - The caller owns every buffer, including the workspace, whose size the
  *     *_workspace_size functions give (0 means none is needed; the pointer
  *     may then be NULL).  Workspace and outputs must not overlap inputs.
@@ -66,7 +69,9 @@ typedef enum {
     SELINV_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
     SELINV_ERR_WORKSPACE = 5,     /* workspace smaller than *_workspace_size */
     SELINV_ERR_UNSUPPORTED = 6,   /* block size beyond selinv_max_block() */
-    SELINV_ERR_HOST_MEMORY = 7    /* a plan's host-side tables could not be allocated */
+    SELINV_ERR_HOST_MEMORY = 7,   /* a plan's host-side tables could not be allocated */
+    SELINV_ERR_TIMEOUT = 8        /* returned by bindings that read info[] back: a bounded
+                                     dependency wait of a tree sweep gave up (info = -2) */
 } selinv_status;
 
 typedef enum { SELINV_F64 = 0, SELINV_F32 = 1 } selinv_dtype;
@@ -103,6 +108,20 @@ size_t selinv_chain_workspace_size(selinv_dtype dtype, int64_t batch, int64_t L,
 int32_t selinv_chain_segments(int64_t batch, int64_t L, int32_t b, int32_t want_g, int32_t want_x);
 
 /*
+ * Flags of selinv_chain and selinv_tree.  The outputs a call computes follow
+ * from which pointers are non-NULL; SELINV_WANT_LOGDET (logdet) and
+ * SELINV_WANT_SOLVE (rhs and x; chains only) make the call reject the
+ * request with SELINV_ERR_INVALID_ARG when those pointers are missing.
+ * SELINV_CHECK (gabp-sparse-inv, "Quickstart": check=True) adds an on-device
+ * pass, after the selected inverse on the same stream, that checks every
+ * entry the call reads -- the lower triangle of each diagonal block, every
+ * entry of each off-diagonal block (trees: non-root edge slots), the
+ * right-hand side -- and writes info = -3 - k for an element whose block k
+ * holds a non-finite value; nothing traps.  Unknown bits are rejected.
+ */
+enum { SELINV_WANT_LOGDET = 1, SELINV_WANT_SOLVE = 2, SELINV_CHECK = 4 };
+
+/*
  * Selected inverse, log-determinant and (optionally) solve of `batch`
  * independent block-tridiagonal SPD chains of L blocks of size b.
  * (gabp-sparse-inv, "Implemented and tested kernels" -> Chain, and the
@@ -116,13 +135,14 @@ int32_t selinv_chain_segments(int64_t batch, int64_t L, int32_t b, int32_t want_
  *   rhs     [batch, L, b]       right-hand side r; NULL for no solve
  *   x       [batch, L, b]       out: A^-1 r; given iff rhs is given
  *   info    [batch] int32       out: see the conventions above (required)
+ *   flags   SELINV_* bits below, or 0
  * Returns SELINV_OK once the work is enqueued.
  */
 selinv_status selinv_chain(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b,
                            const void *diag, const void *lower,
                            void *G_diag, void *G_lower, double *logdet,
                            const void *rhs, void *x, int32_t *info,
-                           void *workspace, size_t workspace_bytes, void *stream);
+                           void *workspace, size_t workspace_bytes, uint32_t flags, void *stream);
 
 /*
  * Solve only: x = A^-1 r for each chain, from the same block LDL^T factor,
@@ -349,6 +369,22 @@ selinv_status selinv_tree_plan(const int32_t *parent, int64_t trees, int64_t n,
 
 void selinv_tree_plan_free(selinv_tree_plan_t *plan);
 
+/*
+ * Dependency waits of the tree sweeps.  A node of the distribute sweep (and
+ * of a draw's and the backward's parents-first pass) waits for its parent's
+ * completion flag with a bounded spin: after spin_limit polls (each at least
+ * 32-64 ns apart) it gives up, writes info = -2 for its tree (outputs of that
+ * tree unspecified) and marks itself failed, so its own descendants give up
+ * at once; the other trees are unaffected and the call returns normally.  A
+ * valid plan never reaches the limit: every parent is handed to a running
+ * warp before its children.  Default spin_limit 4194304 (values < 1 restore
+ * it).  withhold: a node (global index tree * n + v) whose completion the
+ * sweeps never publish, or -1 for none -- a test hook that makes the waits
+ * of that node's children run out.  Host only; applies to later calls with
+ * this plan.
+ */
+selinv_status selinv_tree_plan_set_wait(selinv_tree_plan_t *plan, int32_t spin_limit, int64_t withhold);
+
 /* Levels of a plan: *collect = max height + 1, *distribute = max depth + 1. */
 selinv_status selinv_tree_plan_levels(const selinv_tree_plan_t *plan, int32_t *collect,
                                       int32_t *distribute);
@@ -362,12 +398,15 @@ size_t selinv_tree_workspace_size(const selinv_tree_plan_t *plan, selinv_dtype d
  *   G_diag [trees, n, b, b]  out: (A^-1)_{v,v}
  *   G_edge [trees, n, b, b]  out: (A^-1)_{parent(v), v}; root slot written 0
  *   logdet [trees] float64   out; may be NULL
- *   info   [trees] int32     out: -1, or a node whose pivot failed
+ *   info   [trees] int32     out: -1, or a node whose pivot failed, or -2 when
+ *                            a dependency wait gave up (selinv_tree_plan_set_wait),
+ *                            or -3 - v (SELINV_CHECK: node v holds a non-finite entry)
+ *   flags  SELINV_WANT_LOGDET, SELINV_CHECK, or 0
  */
 selinv_status selinv_tree(const selinv_tree_plan_t *plan, selinv_dtype dtype, int32_t b,
                           const void *diag, const void *edge,
                           void *G_diag, void *G_edge, double *logdet, int32_t *info,
-                          void *workspace, size_t workspace_bytes, void *stream);
+                          void *workspace, size_t workspace_bytes, uint32_t flags, void *stream);
 
 /*
  * Gaussian draw on block trees (gabp-sparse-inv, "Gaussian sampling":

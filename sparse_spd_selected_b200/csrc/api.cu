@@ -66,6 +66,20 @@ selinv_status run_chain(int64_t batch, int64_t L, int32_t b, const void *diag, c
     return from_cuda(chain_large_launch<T>(a, s));
 }
 
+// SELINV_CHECK for a chain call: D_i (lower triangles), B_i and r_i finite.
+template <class T>
+selinv_status check_chain(int64_t batch, int64_t L, int32_t b, const void *diag, const void *lower,
+                          const void *rhs, int32_t *info, cudaStream_t s)
+{
+    cudaError_t e = check_finite_launch<T>(static_cast<const T *>(diag), batch, L, b, 0, nullptr, info, s);
+    if (e == cudaSuccess && L > 1)
+        e = check_finite_launch<T>(static_cast<const T *>(lower), batch, L - 1, b, 1, nullptr, info, s);
+    if (e == cudaSuccess && rhs)
+        e = check_finite_launch<T>(static_cast<const T *>(rhs), batch, L, b, 2, nullptr, info, s);
+    if (e == cudaSuccess) e = check_finalize_launch(info, batch, L, s);
+    return from_cuda(e);
+}
+
 size_t chain_ws(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b, bool want_g, bool want_x)
 {
     if (!want_g && !want_x) return 0;
@@ -94,6 +108,7 @@ const char *selinv_status_string(selinv_status s)
     case SELINV_ERR_WORKSPACE: return "workspace too small";
     case SELINV_ERR_UNSUPPORTED: return "block size not supported";
     case SELINV_ERR_HOST_MEMORY: return "host memory exhausted";
+    case SELINV_ERR_TIMEOUT: return "a dependency wait of a tree sweep gave up";
     }
     return "unknown status";
 }
@@ -118,10 +133,13 @@ size_t selinv_chain_workspace_size(selinv_dtype dtype, int64_t batch, int64_t L,
 selinv_status selinv_chain(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b, const void *diag,
                            const void *lower, void *G_diag, void *G_lower, double *logdet,
                            const void *rhs, void *x, int32_t *info, void *workspace,
-                           size_t workspace_bytes, void *stream)
+                           size_t workspace_bytes, uint32_t flags, void *stream)
 {
     selinv_status st = chain_check(dtype, batch, L, b, diag, lower, info);
     if (st != SELINV_OK) return st;
+    if (flags & ~(uint32_t)(SELINV_WANT_LOGDET | SELINV_WANT_SOLVE | SELINV_CHECK)) return SELINV_ERR_INVALID_ARG;
+    if ((flags & SELINV_WANT_LOGDET) && logdet == nullptr) return SELINV_ERR_INVALID_ARG;
+    if ((flags & SELINV_WANT_SOLVE) && (rhs == nullptr || x == nullptr)) return SELINV_ERR_INVALID_ARG;
     const size_t es = elem_size(dtype);
     const bool want_g = G_diag != nullptr;
     const bool want_x = rhs != nullptr;
@@ -135,11 +153,14 @@ selinv_status selinv_chain(selinv_dtype dtype, int64_t batch, int64_t L, int32_t
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return SELINV_ERR_WORKSPACE;
     if (batch == 0) return SELINV_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (dtype == SELINV_F64)
-        return run_chain<double>(batch, L, b, diag, lower, G_diag, G_lower, logdet, rhs, x, info,
-                                 workspace, s);
-    return run_chain<float>(batch, L, b, diag, lower, G_diag, G_lower, logdet, rhs, x, info,
-                            workspace, s);
+    st = dtype == SELINV_F64 ? run_chain<double>(batch, L, b, diag, lower, G_diag, G_lower, logdet, rhs, x, info,
+                                                 workspace, s)
+                             : run_chain<float>(batch, L, b, diag, lower, G_diag, G_lower, logdet, rhs, x, info,
+                                                workspace, s);
+    if (st != SELINV_OK || !(flags & SELINV_CHECK)) return st;
+    return dtype == SELINV_F64
+               ? check_chain<double>(batch, L, b, diag, lower, rhs, info, s)
+               : check_chain<float>(batch, L, b, diag, lower, rhs, info, s);
 }
 
 selinv_status selinv_chain_sample(selinv_dtype dtype, int64_t batch, int64_t L, int32_t b, const void *diag,
@@ -356,7 +377,7 @@ selinv_status chain_solve(selinv_dtype dtype, int64_t batch, int64_t L, int32_t 
 {
     if (rhs == nullptr || x == nullptr) return batch == 0 ? SELINV_OK : SELINV_ERR_INVALID_ARG;
     return selinv_chain(dtype, batch, L, b, diag, lower, nullptr, nullptr, logdet, rhs, x, info,
-                        workspace, workspace_bytes, stream);
+                        workspace, workspace_bytes, 0u, stream);
 }
 
 }  // extern "C"

@@ -34,19 +34,19 @@ template <int BP> struct Geo {
     static constexpr int NP = BP / 16;       // K panels of width 16
 };
 
-// Shared-memory image of a row-major matrix of pitch P (a multiple of 16).
-//  double: XOR swizzle of 16-byte chunks inside each 128-byte row segment,
-//          chunk ^= f(r), f(r) = ((r & 1) << 2) | ((r >> 1) & 3): conflict-free
-//          tensor-core fragment reads (8 rows x 4 columns, 4 rows x 8 columns).
-//  float:  4-float row padding.
+// Shared-memory image of a row-major matrix of logical pitch P (a multiple
+// of 16), stored with four elements of row padding.
+//  double: rows P + 4 doubles apart put row r at bank offset 8 r (mod 32), so
+//          the tensor-core fragment reads (8 rows x 4 columns, 4 rows x 8
+//          columns) and the accumulator-layout stores are conflict-free, and
+//          every fragment address is a per-row base plus a constant, which
+//          keeps the unrolled product loops' address registers few (an XOR
+//          swizzle needed one precomputed offset per row and k step).
+//  float:  the same 4-float row padding.
 template <class T> struct SW;
 template <> struct SW<double> {
-    static constexpr int PAD = 0;
-    SELINV_DEVINL static int idx(int r, int c, int P)
-    {
-        const int f = ((r & 1) << 2) | ((r >> 1) & 3);
-        return r * P + (c & ~15) + ((((c >> 1) & 7) ^ f) << 1) + (c & 1);
-    }
+    static constexpr int PAD = 4;
+    SELINV_DEVINL static int idx(int r, int c, int P) { return r * (P + 4) + c; }
 };
 template <> struct SW<float> {
     static constexpr int PAD = 4;
@@ -94,7 +94,7 @@ template <class T, int BP> struct Ctx {
 template <class T, int BP> constexpr size_t smem_elems()
 {
     using X = Ctx<T, BP>;
-    return (size_t)X::BIG + 2 * X::PANEL + 2 * BP /*colbuf*/ + 4 * BP /*y, x*/ + 2 * X::RW * BP /*red*/ +
+    return (size_t)X::BIG + 3 * X::PANEL + 2 * BP /*colbuf*/ + 4 * BP /*y, x*/ + 2 * X::RW * BP /*red*/ +
            BP /*z of a draw*/;
 }
 
@@ -154,20 +154,38 @@ SELINV_DEVINL void to_smem_sym(T *S, const Big<T> &a, const Ctx<T, BP> &x)
             }
 }
 
-// diagonal block (row-major b x b, lower triangle read), identity pad
-template <class T, int BP>
+// diagonal block (row-major b x b, lower triangle read), identity pad.
+// FULL (b == BP): every address is one of two per-thread bases -- D[R(0)][C(0)]
+// for entries on or below the diagonal, D[C(0)][R(0)] for their mirrors --
+// plus a constant, so the 32 loads in flight need two address registers
+// (computing each address separately spilled the kernel).
+template <class T, int BP, bool FULL = false>
 SELINV_DEVINL void load_sym(Big<T> &a, const T *D, int b, const Ctx<T, BP> &x)
 {
+    if constexpr (FULL) {
+        const T *Dd = D + x.R(0) * BP + x.C(0, 0);
+        const T *Dm = D + x.C(0, 0) * BP + x.R(0);
 #pragma unroll
-    for (int mi = 0; mi < 4; ++mi)
+        for (int mi = 0; mi < 4; ++mi)
 #pragma unroll
-        for (int ni = 0; ni < 4; ++ni)
+            for (int ni = 0; ni < 4; ++ni)
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int r = x.R(mi), c = x.C(ni, j);
-                const int rr = c <= r ? r : c, cc = c <= r ? c : r;
-                a.v[mi][ni][j] = (r < b && c < b) ? __ldg(D + (int64_t)rr * b + cc) : (r == c ? T(1) : T(0));
-            }
+                for (int j = 0; j < 2; ++j)
+                    a.v[mi][ni][j] = x.C(ni, j) <= x.R(mi) ? __ldg(Dd + (8 * mi) * BP + 8 * ni + j)
+                                                           : __ldg(Dm + (8 * ni + j) * BP + 8 * mi);
+    } else {
+#pragma unroll
+        for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+            for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int r = x.R(mi), c = x.C(ni, j);
+                    const int rr = c <= r ? r : c, cc = c <= r ? c : r;
+                    a.v[mi][ni][j] =
+                        (r < b && c < b) ? __ldg(D + (int64_t)rr * b + cc) : (r == c ? T(1) : T(0));
+                }
+    }
 }
 
 template <class T, int BP, bool FULL>
@@ -261,6 +279,11 @@ enum { OP_BIG = 0, OP_COLPANEL = 1, OP_ROWPANEL = 2 };
 //   A = OP_ROWPANEL: A[m][k] = M[k][m] (row panels of M, i.e. M^T)
 //   B = OP_COLPANEL: B[k][n] = M[n][k] (column panels of M, i.e. M^T)
 //   B = OP_ROWPANEL: B[k][n] = M[k][n] (row panels of M)
+// Panels stream through a ring of three buffers: panel p + 2 is issued right
+// after the barrier that makes panel p visible, which is also the point every
+// warp has finished reading panel p - 1 (the buffer it overwrites), so one
+// barrier per panel suffices (plus one at the end, before the caller reuses
+// the buffers).
 template <class T, int BP, int AOP, int BOP, bool NEG, bool FULL, bool LOWER = false>
 SELINV_DEVINL void gemm(Big<T> &acc, const T *big, T *pbuf, const T *M, int b, const Ctx<T, BP> &x)
 {
@@ -268,21 +291,19 @@ SELINV_DEVINL void gemm(Big<T> &acc, const T *big, T *pbuf, const T *M, int b, c
     constexpr int PANEL = Ctx<T, BP>::PANEL;
     constexpr int STREAM = AOP != OP_BIG ? AOP : BOP;
     auto issue = [&](int p) {
-        T *dst = pbuf + (p & 1) * PANEL;
+        T *dst = pbuf + (p % 3) * PANEL;
         if (STREAM == OP_COLPANEL) load_colpanel<T, BP, FULL>(dst, M, b, 16 * p, x);
         else load_rowpanel<T, BP>(dst, M, 16 * p, x);
         cp_async_commit();
     };
     issue(0);
+    if (NP > 1) issue(1);
     for (int p = 0; p < NP; ++p) {
-        if (p + 1 < NP) {
-            issue(p + 1);
-            cp_async_wait_one();
-        } else {
-            cp_async_wait_all();
-        }
+        if (p + 1 < NP) cp_async_wait_one();          // panel p landed (p + 1 may still be in flight)
+        else cp_async_wait_all();
         __syncthreads();
-        const T *P = pbuf + (p & 1) * PANEL;
+        if (p + 2 < NP) issue(p + 2);
+        const T *P = pbuf + (p % 3) * PANEL;
         const int k0 = 16 * p;
         if (LOWER && x.quad_upper()) {
             // nothing to compute above the diagonal
@@ -344,8 +365,8 @@ SELINV_DEVINL void gemm(Big<T> &acc, const T *big, T *pbuf, const T *M, int b, c
                         for (int j = 0; j < 2; ++j) acc.v[mi][ni][j] = fmaf(a[mi], bf[ni][j], acc.v[mi][ni][j]);
             }
         }
-        __syncthreads();
     }
+    __syncthreads();
 }
 
 // CTA-wide in-register inverse of a symmetric positive definite block by the
@@ -370,9 +391,9 @@ SELINV_DEVINL void spd_inverse(Big<T> &a, T *colbuf, const Ctx<T, BP> &x, LogAcc
             }
             __syncthreads();
             const T d = cb[k];
-            bad |= !(d > T(0));
             if (x.tid == 0) det.mul((double)d);
             const T p = T(1) / d;
+            bad |= bad_pivot(d, p);
             T cr[4], cc[4][2];
 #pragma unroll
             for (int mi = 0; mi < 4; ++mi) cr[mi] = cb[x.R(mi)] * p;
@@ -544,6 +565,145 @@ SELINV_DEVINL void spd_inverse_blocked(Big<double> &a, double *cbuf, double *tbu
         for (int ni = 0; ni < 4; ++ni) a.v[mi][ni][0] = -a.v[mi][ni][0], a.v[mi][ni][1] = -a.v[mi][ni][1];
 }
 
+// The same block steps with look-ahead (float64, no draw): step K's owners
+// of column block K + 1 apply the rank-8 update to those tiles first and
+// publish them, so after the step's single barrier every warp inverts the
+// next pivot block P_{K+1} while it applies the rest of the update: the 8 x 8
+// sweep's shuffle chain overlaps the update's tensor-core work instead of
+// following it behind a barrier, and a step costs one barrier instead of
+// two.  Same pivots in the same order (so the same det), the same products.
+//   step K: T = A_{rows,K} P_K^-1 (P_K^-1 from the previous step); owners of
+//   column K+1: A_{., K+1} -= T A_{K, K+1}, published; barrier; everyone:
+//   P_{K+1}^-1 from the published column and the remaining updates; column K
+//   := T, row K := T^T, A_KK := -P_K^-1.
+// Buffers: the column block K is read before step K's barrier and rewritten
+// (as column K + 2) only after step K + 1's start, so two alternate; T alternates
+// likewise (written before a step's barrier, read after it).
+template <int BP>
+SELINV_DEVINL void spd_inverse_lookahead(Big<double> &a, double *cbuf, double *tbuf, const Ctx<double, BP> &x,
+                                         LogAcc &det, bool &bad)
+{
+    constexpr int NB = BP / 8;
+    if (x.cw == 0) {                                              // publish column block 0
+#pragma unroll
+        for (int mi = 0; mi < 4; ++mi) {
+            double2 u;
+            u.x = a.v[mi][0][0];
+            u.y = a.v[mi][0][1];
+            *reinterpret_cast<double2 *>(cbuf + x.R(mi) * 8 + 2 * x.t) = u;
+        }
+    }
+    __syncthreads();
+    double pv[2];
+    {
+        const double2 u = *reinterpret_cast<const double2 *>(cbuf + x.g * 8 + 2 * x.t);
+        pv[0] = u.x;
+        pv[1] = u.y;
+    }
+    inv8_sweep(pv, x.lane, x.g, x.t, det, bad, x.tid == 0);
+    if (x.tid == 0) det.renorm();
+    for (int K = 0; K < NB; ++K) {
+        const double *cb = cbuf + (K & 1) * BP * 8;               // column block K
+        double *cn = cbuf + ((K + 1) & 1) * BP * 8;               // column block K + 1
+        double *tb = tbuf + (K & 1) * BP * 8;
+        const int qK = K >> 2, tK = K & 3;
+        const int K1 = K + 1, qK1 = K1 >> 2, tK1 = K1 & 3;
+        const bool next = K1 < NB;
+        // T = A_{rows,K} P^-1 for this warp's rows
+        double T[4][2];
+#pragma unroll
+        for (int mi = 0; mi < 4; ++mi) {
+            const double2 arow = *reinterpret_cast<const double2 *>(cb + x.R(mi) * 8 + 2 * x.t);
+            T[mi][0] = T[mi][1] = 0.0;
+            dmma_8x8x4(T[mi][0], T[mi][1], arow.x, pv[0]);
+            dmma_8x8x4(T[mi][0], T[mi][1], arow.y, pv[1]);
+        }
+        if (x.cw == 0) {                                          // publish T (one copy per row)
+#pragma unroll
+            for (int mi = 0; mi < 4; ++mi) {
+                double2 u;
+                u.x = T[mi][0];
+                u.y = T[mi][1];
+                *reinterpret_cast<double2 *>(tb + x.R(mi) * 8 + 2 * x.t) = u;
+            }
+        }
+        // A_Kj = A_jK for this warp's column tile ni (read where it is used)
+        auto bk = [&](int ni) {
+            return *reinterpret_cast<const double2 *>(cb + (32 * x.cw + 8 * ni + x.g) * 8 + 2 * x.t);
+        };
+        const bool own_next = next && x.cw == qK1;
+        if (own_next) {                                           // column block K + 1 first, published
+#pragma unroll
+            for (int n = 0; n < 4; ++n)
+                if (n == tK1) {
+                    const double2 bn = bk(n);
+#pragma unroll
+                    for (int mi = 0; mi < 4; ++mi) {
+                        dmma_8x8x4(a.v[mi][n][0], a.v[mi][n][1], -T[mi][0], bn.x);
+                        dmma_8x8x4(a.v[mi][n][0], a.v[mi][n][1], -T[mi][1], bn.y);
+                        double2 u;
+                        u.x = a.v[mi][n][0];
+                        u.y = a.v[mi][n][1];
+                        *reinterpret_cast<double2 *>(cn + x.R(mi) * 8 + 2 * x.t) = u;
+                    }
+                }
+        }
+        __syncthreads();                                          // T and column block K + 1 published
+        double pn[2] = {0.0, 0.0};
+        if (next) {                                               // P_{K+1}, inverted beside the update below
+            const double2 u = *reinterpret_cast<const double2 *>(cn + (8 * K1 + x.g) * 8 + 2 * x.t);
+            pn[0] = u.x;
+            pn[1] = u.y;
+            inv8_sweep(pn, x.lane, x.g, x.t, det, bad, x.tid == 0);
+        }
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni) {
+            if (own_next && ni == tK1) continue;                  // already updated
+            const double2 bn = bk(ni);
+#pragma unroll
+            for (int mi = 0; mi < 4; ++mi) {
+                dmma_8x8x4(a.v[mi][ni][0], a.v[mi][ni][1], -T[mi][0], bn.x);
+                dmma_8x8x4(a.v[mi][ni][0], a.v[mi][ni][1], -T[mi][1], bn.y);
+            }
+        }
+        if (x.cw == qK) {                                         // column block K: T (rows outside K)
+#pragma unroll
+            for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+                for (int n = 0; n < 4; ++n)
+                    if (n == tK) {
+                        a.v[mi][n][0] = T[mi][0];
+                        a.v[mi][n][1] = T[mi][1];
+                    }
+        }
+        if (x.rw == qK) {                                         // row block K: T_j^T, diagonal block -P^-1
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                if (m == tK) {
+#pragma unroll
+                    for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) a.v[m][ni][j] = tb[x.C(ni, j) * 8 + x.g];
+                    if (x.cw == qK) {
+#pragma unroll
+                        for (int n = 0; n < 4; ++n)
+                            if (n == tK) {
+                                a.v[m][n][0] = -pv[0];
+                                a.v[m][n][1] = -pv[1];
+                            }
+                    }
+                }
+        }
+        pv[0] = pn[0];
+        pv[1] = pn[1];
+        if (x.tid == 0) det.renorm();
+    }
+#pragma unroll
+    for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni) a.v[mi][ni][0] = -a.v[mi][ni][0], a.v[mi][ni][1] = -a.v[mi][ni][1];
+}
+
 // Row sums (over this thread's columns) of a tile times the vector v, reduced
 // over the 4 lanes of a row group: the per-warp partial for rows R(mi).
 template <class T, int BP>
@@ -593,7 +753,7 @@ __global__ void __launch_bounds__(Geo<BP>::NT) chain_large_kernel(ChainArgs<T> p
     extern __shared__ __align__(16) unsigned char smem_raw[];
     T *big = reinterpret_cast<T *>(smem_raw);
     T *pbuf = big + X::BIG;
-    T *colbuf = pbuf + 2 * X::PANEL;
+    T *colbuf = pbuf + 3 * X::PANEL;
     T *ybuf = colbuf + 2 * BP;     // two buffers
     T *xbuf = ybuf + 2 * BP;       // two buffers
     T *red1 = xbuf + 2 * BP;       // [RW][BP]
@@ -621,7 +781,7 @@ __global__ void __launch_bounds__(Geo<BP>::NT) chain_large_kernel(ChainArgs<T> p
         if (x.tid < b) Xv[x.tid] = r0;            // y_0 kept in x until the distribute sweep
     }
     Big<T> a;
-    load_sym<T, BP>(a, D, b, x);
+    load_sym<T, BP, FULL>(a, D, b, x);
     __syncthreads();
 
     // ---------------- collect sweep ----------------
@@ -648,7 +808,7 @@ __global__ void __launch_bounds__(Geo<BP>::NT) chain_large_kernel(ChainArgs<T> p
                 }
             }
         } else if constexpr (sizeof(T) == 8) {
-            spd_inverse_blocked<BP>(a, pbuf, pbuf + 2 * BP * 8, x, det, bad);
+            spd_inverse_lookahead<BP>(a, pbuf, pbuf + 2 * BP * 8, x, det, bad);
         } else {
             spd_inverse<T, BP>(a, colbuf, x, det, bad);
         }
@@ -679,7 +839,7 @@ __global__ void __launch_bounds__(Geo<BP>::NT) chain_large_kernel(ChainArgs<T> p
             ybuf[BP * ((i + 1) & 1) + x.tid] = yv;
             if (x.tid < b) Xv[(i + 1) * b + x.tid] = yv;
         }
-        load_sym<T, BP>(a, D + (i + 1) * bb, b, x);
+        load_sym<T, BP, FULL>(a, D + (i + 1) * bb, b, x);
         gemm<T, BP, OP_BIG, OP_COLPANEL, true, FULL, true>(a, big, pbuf, Bl + i * bb, b, x);   // S_{i+1} = D_{i+1} - W_i B_i^T (lower)
         to_smem_sym<T, BP>(big, a, x);             // complete the upper triangle (big is free after the gemm)
         __syncthreads();

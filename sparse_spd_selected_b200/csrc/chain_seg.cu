@@ -32,6 +32,12 @@
 //   G_jj       = S_j^-1 - W_j^T G_{next,j} - V_j^T G_{s,j}
 // with G_{next,j} = G_lower (upward) or its transpose (downward), and
 // G_{s,lo}^T = G_lower[s_k] at the end of an interior segment.
+//
+// Arithmetic is float64 for both element types: float32 blocks are widened as
+// they are read and rounded as the G blocks are stored, so the float32 run
+// takes the same FP64 tensor-core path as float64 (the scalar float32 path,
+// one pivot per barrier on the FP32 pipes, was slower than float64 here), and
+// the workspace images between the sweeps are float64.
 #include <algorithm>
 
 #include "kernels.h"
@@ -52,7 +58,7 @@ struct SegGeo {
 
 template <class T> struct SegArgs {
     SegGeo geo;
-    T *node;                  // [batch, L, 11 E]: S_j^-1 lower images, W_j images, V_j images
+    double *node;             // [batch, L, 11 E]: S_j^-1 lower images, W_j images, V_j images (float64)
     T *cA, *cB;               // [batch, P-1, b*b]: contribution to separator r from the segment below / above
     T *rdiag, *rlower;        // the separators' chain: [batch, P-1, b*b], [batch, P-2, b*b]
     T *rGd, *rGl;             // its G blocks
@@ -125,8 +131,9 @@ template <class T, bool FULL, bool WANT_G>
 __global__ void __launch_bounds__(GT, 3) seg_collect_kernel(ChainArgs<T> p, SegArgs<T> sa)
 {
     using namespace w16;
-    using Ly = SegLay<T>;
-    constexpr int E = SL<T>::ELEMS;
+    using C = double;                           // arithmetic (T: element type of the inputs and outputs)
+    using Ly = SegLay<C>;
+    constexpr int E = SL<C>::ELEMS;
     const int P = sa.geo.P;
     const int64_t e = blockIdx.x / P;
     const int k = blockIdx.x % P;
@@ -137,12 +144,14 @@ __global__ void __launch_bounds__(GT, 3) seg_collect_kernel(ChainArgs<T> p, SegA
     constexpr int bar = 1;
 
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    T *base = reinterpret_cast<T *>(smem_raw);
-    T *sC = base + Ly::C, *sD = base + Ly::D, *sX = base + Ly::X, *sY = base + Ly::Y;
-    T *sV = base + Ly::V, *sF = base + Ly::F;
-    T *s1 = sizeof(T) == 4 ? base + Ly::CS + wq * 2 * E : nullptr;
-    T *s2 = sizeof(T) == 4 ? s1 + E : nullptr;
-    T *cb = base + Ly::CCB;
+    C *base = reinterpret_cast<C *>(smem_raw);
+    // C_j and D_next arrive by cp.async in the inputs' own element type and
+    // are widened as they are read; every other image is float64
+    T *sC = reinterpret_cast<T *>(base + Ly::C), *sD = reinterpret_cast<T *>(base + Ly::D);
+    C *sX = base + Ly::X, *sY = base + Ly::Y;
+    C *sV = base + Ly::V, *sF = base + Ly::F;
+    C *s1 = nullptr, *s2 = nullptr;             // float64 products need no scratch
+    C *cb = base + Ly::CCB;
 
     const int b = p.b;
     const int64_t L = p.L;
@@ -151,68 +160,74 @@ __global__ void __launch_bounds__(GT, 3) seg_collect_kernel(ChainArgs<T> p, SegA
     const int64_t n = sp.hi - sp.lo + 1;
     const T *Dg = p.diag + e * L * bb;
     const T *Bg = p.lower + e * (L - 1) * bb;
-    T *wsn = WANT_G ? sa.node + e * L * Ly::NODE : nullptr;
+    C *wsn = WANT_G ? sa.node + e * L * Ly::NODE : nullptr;
     auto node = [&](int64_t j) { return sp.down ? sp.hi - j : sp.lo + j; };
     auto cpl = [&](int64_t j) { return sp.down ? sp.hi - j - 1 : sp.lo + j; };   // lower block of C_j
 
     LogAcc det;
     det.init();
     int fail = -1;
-    Tile<T> a, u;
+    Tile<C> a, u;
     zero(u);
 
     load_diag<T, FULL>(sD, Dg + node(0) * bb, b, gtid);
-    if (sp.fill) load_full<T, FULL>(sF, Bg + (sp.lo - 1) * bb, b, gtid);       // F = A_{lo, s} = B_s
+    if (sp.fill) load_full_f64<T, FULL>(sF, Bg + (sp.lo - 1) * bb, b, gtid);   // F = A_{lo, s} = B_s
     cp_async_commit();
     cp_async_wait_all();
     group_bar(bar);
-    sym_quad<T>(a, sD, I, J, g, t);
+    sym_quad<C>(a, sD, I, J, g, t);
     group_bar(bar);
     load_full<T, FULL>(sC, Bg + cpl(0) * bb, b, gtid);
     if (n > 1) load_diag<T, FULL>(sD, Dg + node(1) * bb, b, gtid);
     cp_async_commit();
 
-    Tile<T> fn;
+    Tile<C> fn;
     for (int64_t j = 0; j < n; ++j) {
         bool bad = false;
-        qinverse<T>(a, cb, I, J, g, t, bar, det, bad);              // a = S_j^-1
+        qinverse<C>(a, cb, I, J, g, t, bar, det, bad);              // a = S_j^-1
         if (bad && fail < 0) fail = (int)node(j);
-        to_smem<T>(quad(sX, I, J), a, g, t);
+        to_smem<C>(quad(sX, I, J), a, g, t);
         cp_async_wait_all();
         group_bar(bar);
-        T *slot = WANT_G ? wsn + node(j) * Ly::NODE : nullptr;
+        C *slot = WANT_G ? wsn + node(j) * Ly::NODE : nullptr;
         if (WANT_G) {
-            copy_out<T>(slot, sX, E, gtid);
-            copy_out<T>(slot + E, quad(sX, 1, 0), 2 * E, gtid);
+            copy_out<C>(slot, sX, E, gtid);
+            copy_out<C>(slot + E, quad(sX, 1, 0), 2 * E, gtid);
         }
-        Tile<T> w, v;
+        Tile<C> w, v;
         zero(w);
         if (sp.down) qgemm<false, true, false, false>(w, sC, sX, I, J, s1, s2, g, t);   // W_j = C_j S_j^-1
         else qgemm<false, false, false, false>(w, sC, sX, I, J, s1, s2, g, t);
-        to_smem<T>(quad(sY, I, J), w, g, t);
+        to_smem<C>(quad(sY, I, J), w, g, t);
         if (sp.fill) {
             zero(v);
             qgemm<false, true, false, false>(v, sF, sX, I, J, s1, s2, g, t);        // V_j = F_j^T S_j^-1
-            to_smem<T>(quad(sV, I, J), v, g, t);
+            to_smem<C>(quad(sV, I, J), v, g, t);
         }
         group_bar(bar);
         if (WANT_G) {
-            copy_out<T>(slot + 3 * E, sY, 4 * E, gtid);
-            if (sp.fill) copy_out<T>(slot + 7 * E, sV, 4 * E, gtid);
+            copy_out<C>(slot + 3 * E, sY, 4 * E, gtid);
+            if (sp.fill) copy_out<C>(slot + 7 * E, sV, 4 * E, gtid);
         }
         const bool last = j == n - 1;
-        if (last) zero(a);                                            // the separator's contribution only
-        else sym_quad<T>(a, sD, I, J, g, t);                          // D_next
-        if (sp.down) qgemm<true, false, true, false>(a, sY, sC, I, J, s1, s2, g, t);   // S_next -= W_j C_j^T
-        else qgemm<true, false, false, false>(a, sY, sC, I, J, s1, s2, g, t);
+        // S_next and U_s are symmetric and only their lower quadrants are ever
+        // read (the next inverse starts from quadrants (0,0), (1,0), (1,1); the
+        // separators' D' is read on its lower triangle): warp (0,1) skips them.
+        const bool upper = I == 0 && J == 1;
+        if (last || upper) zero(a);                                   // the separator's contribution only
+        else sym_quad<C>(a, sD, I, J, g, t);                          // D_next
+        if (!upper) {
+            if (sp.down) qgemm<true, false, true, false>(a, sY, sC, I, J, s1, s2, g, t);   // S_next -= W_j C_j^T
+            else qgemm<true, false, false, false>(a, sY, sC, I, J, s1, s2, g, t);
+        }
         if (sp.fill) {
             zero(fn);
             qgemm<true, false, true, false>(fn, sY, sF, I, J, s1, s2, g, t);         // F_next = -W_j F_j
-            qgemm<false, false, true, false>(u, sV, sF, I, J, s1, s2, g, t);         // U_s += V_j F_j
+            if (!upper) qgemm<false, false, true, false>(u, sV, sF, I, J, s1, s2, g, t);   // U_s += V_j F_j
         }
         group_bar(bar);
         if (!last) {
-            if (sp.fill) to_smem<T>(quad(sF, I, J), fn, g, t);
+            if (sp.fill) to_smem<C>(quad(sF, I, J), fn, g, t);
             load_full<T, FULL>(sC, Bg + cpl(j + 1) * bb, b, gtid);
             if (j + 2 < n) load_diag<T, FULL>(sD, Dg + node(j + 2) * bb, b, gtid);
             cp_async_commit();
@@ -230,7 +245,7 @@ __global__ void __launch_bounds__(GT, 3) seg_collect_kernel(ChainArgs<T> p, SegA
         store_quad<T, false>(sa.cB + (e * nsep + (k - 1)) * bb, u, b, I, J, g, t);        // U for s_k
         store_quad<T, false>(sa.rlower + (e * (nsep - 1) + (k - 1)) * bb, fn, b, I, J, g, t);   // A'_{s_{k+1}, s_k}
     }
-    combine_det<T>(sD, det, fail, wq, lane, sa.ld + e * P + k, sa.fail + e * P + k, !sp.down);
+    combine_det<C>(base + Ly::D, det, fail, wq, lane, sa.ld + e * P + k, sa.fail + e * P + k, !sp.down);
 }
 
 // Distribute sweep of one segment per CTA, seeded by the separators' G blocks.
@@ -238,8 +253,9 @@ template <class T, bool FULL>
 __global__ void __launch_bounds__(GT, 3) seg_distribute_kernel(ChainArgs<T> p, SegArgs<T> sa)
 {
     using namespace w16;
-    using Ly = SegLay<T>;
-    constexpr int E = SL<T>::ELEMS;
+    using C = double;                           // arithmetic (T: element type of the inputs and outputs)
+    using Ly = SegLay<C>;
+    constexpr int E = SL<C>::ELEMS;
     const int P = sa.geo.P;
     const int nsep = P - 1;
     const int64_t e = blockIdx.x / P;
@@ -251,32 +267,31 @@ __global__ void __launch_bounds__(GT, 3) seg_distribute_kernel(ChainArgs<T> p, S
     constexpr int bar = 1;
 
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    T *base = reinterpret_cast<T *>(smem_raw);
-    T *sA = base + Ly::A, *sCg = base + Ly::CG;
+    C *base = reinterpret_cast<C *>(smem_raw);
+    C *sA = base + Ly::A, *sCg = base + Ly::CG;
     auto bW = [&](int c) { return base + Ly::W0 + c * Ly::IMG; };
     auto bV = [&](int c) { return base + Ly::V0 + c * Ly::IMG; };
-    T *bS = base + Ly::S0;
-    T *s1 = sizeof(T) == 4 ? base + Ly::DS + wq * 2 * E : nullptr;
-    T *s2 = sizeof(T) == 4 ? s1 + E : nullptr;
+    C *bS = base + Ly::S0;
+    C *s1 = nullptr, *s2 = nullptr;             // float64 products need no scratch
 
     const int b = p.b;
     const int64_t L = p.L;
     const int64_t bb = (int64_t)b * b;
     const SegSpan sp = seg_span(sa.geo, L, k);
     const int64_t n = sp.hi - sp.lo + 1;
-    const T *wsn = sa.node + e * L * Ly::NODE;
+    const C *wsn = sa.node + e * L * Ly::NODE;
     T *Gd = p.G_diag + e * L * bb;
     T *Gl = p.G_lower + e * (L - 1) * bb;
     auto node = [&](int64_t j) { return sp.down ? sp.hi - j : sp.lo + j; };
     auto stage_wv = [&](int64_t j, int c) {
-        const T *slot = wsn + node(j) * Ly::NODE;
-        stage_in<T>(bW(c), slot + 3 * E, 4 * E, gtid);
-        if (sp.fill) stage_in<T>(bV(c), slot + 7 * E, 4 * E, gtid);
+        const C *slot = wsn + node(j) * Ly::NODE;
+        stage_in<C>(bW(c), slot + 3 * E, 4 * E, gtid);
+        if (sp.fill) stage_in<C>(bV(c), slot + 7 * E, 4 * E, gtid);
     };
     auto stage_s = [&](int64_t j) {
-        const T *slot = wsn + node(j) * Ly::NODE;
-        stage_in<T>(bS, slot, E, gtid);
-        stage_in<T>(quad(bS, 1, 0), slot + E, 2 * E, gtid);
+        const C *slot = wsn + node(j) * Ly::NODE;
+        stage_in<C>(bS, slot, E, gtid);
+        stage_in<C>(quad(bS, 1, 0), slot + E, 2 * E, gtid);
     };
 
     if (k == 0) {                                                     // the separators' own G blocks
@@ -286,24 +301,24 @@ __global__ void __launch_bounds__(GT, 3) seg_distribute_kernel(ChainArgs<T> p, S
             for (int64_t i = gtid; i < bb; i += GT) dst[i] = src[i];
         }
     }
-    T *pB = base + Ly::B, *pD = base + Ly::DG;                        // G_{s,next} and the new G_{s,j}
-    load_diag<T, FULL>(sA, sa.rGd + (e * nsep + sp.target) * bb, b, gtid);        // G_next = G of the target
+    C *pB = base + Ly::B, *pD = base + Ly::DG;                        // G_{s,next} and the new G_{s,j}
+    load_diag_f64<T, FULL>(sA, sa.rGd + (e * nsep + sp.target) * bb, b, gtid);    // G_next = G of the target
     if (sp.fill) {
-        load_diag<T, FULL>(pD, sa.rGd + (e * nsep + (k - 1)) * bb, b, gtid);      // G_ss
-        load_full<T, FULL>(sCg, sa.rGl + (e * (nsep - 1) + (k - 1)) * bb, b, gtid);   // G_{target, s}
+        load_diag_f64<T, FULL>(pD, sa.rGd + (e * nsep + (k - 1)) * bb, b, gtid);  // G_ss
+        load_full_f64<T, FULL>(sCg, sa.rGl + (e * (nsep - 1) + (k - 1)) * bb, b, gtid);   // G_{target, s}
     }
     stage_s(n - 1);
     stage_wv(n - 1, 0);
     cp_async_commit();
     cp_async_wait_all();
     group_bar(bar);
-    Tile<T> gss[2];
+    Tile<C> gss[2];
     if (sp.fill) {
-        sym_quad<T>(gss[0], pD, I, 0, g, t);
-        sym_quad<T>(gss[1], pD, I, 1, g, t);
-        Tile<T> x;
-        from_smem_T<T>(x, quad(sCg, J, I), g, t);                     // G_{s,target} = G_{target,s}^T
-        to_smem<T>(quad(pB, I, J), x, g, t);
+        sym_quad<C>(gss[0], pD, I, 0, g, t);
+        sym_quad<C>(gss[1], pD, I, 1, g, t);
+        Tile<C> x;
+        from_smem_T<C>(x, quad(sCg, J, I), g, t);                     // G_{s,target} = G_{target,s}^T
+        to_smem<C>(quad(pB, I, J), x, g, t);
     }
     int cur = 0;
     for (int64_t j = n - 1; j >= 0; --j) {
@@ -313,26 +328,26 @@ __global__ void __launch_bounds__(GT, 3) seg_distribute_kernel(ChainArgs<T> p, S
             stage_wv(j - 1, cur ^ 1);
             cp_async_commit();
         }
-        Tile<T> s, gl, gs;
-        sym_quad<T>(s, bS, I, J, g, t);                               // S_j^-1
+        Tile<C> s, gl, gs;
+        sym_quad<C>(s, bS, I, J, g, t);                               // S_j^-1
         zero(gl);
 #pragma unroll
         for (int K = 0; K < 2; ++K) {                                 // G_{next,j} = -G_next W_j ...
-            Tile<T> x, y;
-            sym_quad<T>(x, sA, I, K, g, t);
-            from_smem_T<T>(y, quad(bW(cur), K, J), g, t);
+            Tile<C> x, y;
+            sym_quad<C>(x, sA, I, K, g, t);
+            from_smem_T<C>(y, quad(bW(cur), K, J), g, t);
             gemm_nt<true>(gl, x, y, s1, s2, g, t);
         }
         if (sp.fill) {
             zero(gs);
 #pragma unroll
             for (int K = 0; K < 2; ++K) {
-                Tile<T> x, y, yv;
-                from_smem_T<T>(yv, quad(bV(cur), K, J), g, t);
-                from_smem_T<T>(x, quad(pB, K, I), g, t);
+                Tile<C> x, y, yv;
+                from_smem_T<C>(yv, quad(bV(cur), K, J), g, t);
+                from_smem_T<C>(x, quad(pB, K, I), g, t);
                 gemm_nt<true>(gl, x, yv, s1, s2, g, t);               // ... - G_{s,next}^T V_j
-                from_smem<T>(x, quad(pB, I, K), g, t);
-                from_smem_T<T>(y, quad(bW(cur), K, J), g, t);
+                from_smem<C>(x, quad(pB, I, K), g, t);
+                from_smem_T<C>(y, quad(bW(cur), K, J), g, t);
                 gemm_nt<true>(gs, x, y, s1, s2, g, t);                // G_{s,j} = -G_{s,next} W_j ...
                 gemm_nt<true>(gs, gss[K], yv, s1, s2, g, t);          // ... - G_ss V_j
             }
@@ -341,21 +356,23 @@ __global__ void __launch_bounds__(GT, 3) seg_distribute_kernel(ChainArgs<T> p, S
         if (sp.down) store_quad<T, true>(Gl + (v - 1) * bb, gl, b, I, J, g, t);   // G_lower[v-1] = G_{v-1,v}^T
         else store_quad<T, false>(Gl + v * bb, gl, b, I, J, g, t);                 // G_lower[v] = G_{v+1,v}
         if (sp.fill && j == 0) store_quad<T, true>(Gl + (sp.lo - 1) * bb, gs, b, I, J, g, t);   // G_{lo,s}
-        to_smem<T>(quad(sCg, I, J), gl, g, t);
-        if (sp.fill) to_smem<T>(quad(pD, I, J), gs, g, t);
+        to_smem<C>(quad(sCg, I, J), gl, g, t);
+        if (sp.fill) to_smem<C>(quad(pD, I, J), gs, g, t);
         group_bar(bar);
         if (j > 0) {
             stage_s(j - 1);
             cp_async_commit();
         }
-        qgemm<true, true, true, false>(s, bW(cur), sCg, I, J, s1, s2, g, t);       // G_jj = S_j^-1 - W_j^T G_{next,j}
-        if (sp.fill) qgemm<true, true, true, false>(s, bV(cur), pD, I, J, s1, s2, g, t);   // - V_j^T G_{s,j}
-        to_smem<T>(quad(sA, I, J), s, g, t);
+        if (!(I == 0 && J == 1)) {                                    // G_jj is read on its lower quadrants
+            qgemm<true, true, true, false>(s, bW(cur), sCg, I, J, s1, s2, g, t);   // G_jj = S_j^-1 - W_j^T G_{next,j}
+            if (sp.fill) qgemm<true, true, true, false>(s, bV(cur), pD, I, J, s1, s2, g, t);   // - V_j^T G_{s,j}
+            to_smem<C>(quad(sA, I, J), s, g, t);
+        }
         group_bar(bar);
-        Tile<T> G;
-        sym_quad<T>(G, sA, I, J, g, t);                               // exactly symmetric G_jj
+        Tile<C> G;
+        sym_quad<C>(G, sA, I, J, g, t);                               // exactly symmetric G_jj
         store_quad<T, false>(Gd + v * bb, G, b, I, J, g, t);
-        T *tmp = pB;
+        C *tmp = pB;
         pB = pD;
         pD = tmp;
         cur ^= 1;
@@ -431,7 +448,7 @@ template <class T> SegWs seg_ws_layout(int64_t batch, int64_t L, int b, int P, b
     SegWs w;
     size_t off = 0;
     const size_t bb = (size_t)b * b, nsep = P - 1;
-    w.node = seg_bytes<T>(off, want_g ? (size_t)batch * L * SegLay<T>::NODE : 0);
+    w.node = seg_bytes<double>(off, want_g ? (size_t)batch * L * SegLay<double>::NODE : 0);
     w.cA = seg_bytes<T>(off, batch * nsep * bb);
     w.cB = seg_bytes<T>(off, batch * nsep * bb);
     w.rdiag = seg_bytes<T>(off, batch * nsep * bb);
@@ -456,19 +473,19 @@ template <class K> cudaError_t set_smem(K k, size_t bytes)
 template <class T, bool FULL>
 cudaError_t seg_run(const ChainArgs<T> &a, const SegArgs<T> &sa, const SegWs &w, cudaStream_t s)
 {
-    using Ly = SegLay<T>;
+    using Ly = SegLay<double>;
     const int P = sa.geo.P;
     const bool G = a.G_diag != nullptr;
     const unsigned grid = (unsigned)(a.batch * P);
     cudaError_t err;
     if (G) {
         auto kc = seg_collect_kernel<T, FULL, true>;
-        if ((err = set_smem(kc, sizeof(T) * Ly::CTOTAL)) != cudaSuccess) return err;
-        kc<<<grid, GT, sizeof(T) * Ly::CTOTAL, s>>>(a, sa);
+        if ((err = set_smem(kc, sizeof(double) * Ly::CTOTAL)) != cudaSuccess) return err;
+        kc<<<grid, GT, sizeof(double) * Ly::CTOTAL, s>>>(a, sa);
     } else {
         auto kc = seg_collect_kernel<T, FULL, false>;
-        if ((err = set_smem(kc, sizeof(T) * Ly::CTOTAL)) != cudaSuccess) return err;
-        kc<<<grid, GT, sizeof(T) * Ly::CTOTAL, s>>>(a, sa);
+        if ((err = set_smem(kc, sizeof(double) * Ly::CTOTAL)) != cudaSuccess) return err;
+        kc<<<grid, GT, sizeof(double) * Ly::CTOTAL, s>>>(a, sa);
     }
     seg_assemble_kernel<T><<<(unsigned)(a.batch * (P - 1)), 256, 0, s>>>(a, sa);
     ChainArgs<T> r{};
@@ -485,8 +502,8 @@ cudaError_t seg_run(const ChainArgs<T> &a, const SegArgs<T> &sa, const SegWs &w,
     if ((err = chain_mid_launch<T>(r, s)) != cudaSuccess) return err;
     if (G) {
         auto kd = seg_distribute_kernel<T, FULL>;
-        if ((err = set_smem(kd, sizeof(T) * Ly::DTOTAL)) != cudaSuccess) return err;
-        kd<<<grid, GT, sizeof(T) * Ly::DTOTAL, s>>>(a, sa);
+        if ((err = set_smem(kd, sizeof(double) * Ly::DTOTAL)) != cudaSuccess) return err;
+        kd<<<grid, GT, sizeof(double) * Ly::DTOTAL, s>>>(a, sa);
     }
     seg_finalize_kernel<T><<<(unsigned)ceil_div(a.batch, 128), 128, 0, s>>>(a, sa);
     return cudaGetLastError();
@@ -526,7 +543,7 @@ template <class T> cudaError_t chain_seg_launch(const ChainArgs<T> &a, int P, cu
     unsigned char *ws = reinterpret_cast<unsigned char *>(a.ws);
     SegArgs<T> sa;
     sa.geo = seg_geometry(a.L, P);
-    sa.node = reinterpret_cast<T *>(ws + w.node);
+    sa.node = reinterpret_cast<double *>(ws + w.node);
     sa.cA = reinterpret_cast<T *>(ws + w.cA);
     sa.cB = reinterpret_cast<T *>(ws + w.cB);
     sa.rdiag = reinterpret_cast<T *>(ws + w.rdiag);

@@ -18,6 +18,45 @@ SELINV_DEVINL void cp_async16(void *smem, const void *gmem)
     unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
 }
+// L2 eviction policies (createpolicy) for cache-hinted copies and stores:
+// data streamed once leaves L2 first, so lines that are read back soon (the
+// workspace slots between the two sweeps) stay resident.
+SELINV_DEVINL uint64_t l2_evict_first()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
+    return p;
+}
+SELINV_DEVINL uint64_t l2_evict_last()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;\n" : "=l"(p));
+    return p;
+}
+// cp_async16 with an L2 eviction policy.
+SELINV_DEVINL void cp_async16_hint(void *smem, const void *gmem, uint64_t pol)
+{
+    unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "l"(pol)
+                 : "memory");
+}
+// 16-byte store of two doubles (or floats) with an L2 eviction policy.
+SELINV_DEVINL void st_hint(double2 *p, double2 v, uint64_t pol)
+{
+    asm volatile("st.global.L2::cache_hint.v2.f64 [%0], {%1, %2}, %3;\n" ::"l"(p), "d"(v.x), "d"(v.y), "l"(pol)
+                 : "memory");
+}
+SELINV_DEVINL void st_hint(float2 *p, float2 v, uint64_t pol)
+{
+    asm volatile("st.global.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;\n" ::"l"(p), "f"(v.x), "f"(v.y), "l"(pol)
+                 : "memory");
+}
+// Drop the 128-byte L2 line at p (128-byte aligned) without writing it back:
+// for scratch lines that are dead once read.
+SELINV_DEVINL void discard_l2_line(const void *p)
+{
+    asm volatile("discard.global.L2 [%0], 128;\n" ::"l"(p) : "memory");
+}
 SELINV_DEVINL void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 SELINV_DEVINL void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
 // Wait until at most one committed group (the most recent) is still in flight.
@@ -45,11 +84,14 @@ SELINV_DEVINL void dmma_8x8x4(double &d0, double &d1, double a, double b)
                  : "d"(a), "d"(b));
 }
 
-// Reciprocal of a positive normal d: the hardware approximation refined by one
-// cubic Newton-Raphson step, r <- r (1 + e + e^2) with e = 1 - d r, which
-// triples the number of correct bits of the estimate (about 20 -> full
-// precision).  Not for zero, negative, subnormal or non-finite d (the callers
-// flag such pivots as failures and do not use the result).
+// Reciprocal of a pivot d in [2^-1022, 2^1022): the hardware approximation
+// refined by one cubic Newton-Raphson step, r <- r (1 + e + e^2) with
+// e = 1 - d r, which triples the number of correct bits of the estimate
+// (about 20 -> full precision).  Outside that range the flush-to-zero
+// estimate is wrong (a subnormal d flushes to zero, a reciprocal below
+// 2^-1022 flushes to zero); bad_pivot reports such pivots as failures (a test
+// off the sweep's dependency chain, unlike a branch to IEEE division here,
+// which lengthened every pivot step).
 SELINV_DEVINL double recip(double d)
 {
     double r;
@@ -58,6 +100,12 @@ SELINV_DEVINL double recip(double d)
     return fma(r, fma(e, e, e), r);
 }
 SELINV_DEVINL float recip(float d) { return __frcp_rn(d); }
+
+// A pivot the sweeps cannot use.  float64: not in [2^-1022, 2^1022) (this
+// covers d <= 0 and NaN, and every pivot whose fast reciprocal would be
+// wrong); float32 (IEEE reciprocal): not > 0, or a reciprocal that overflows.
+SELINV_DEVINL bool bad_pivot(double d, double) { return !(d >= 0x1p-1022 && d < 0x1p1022); }
+SELINV_DEVINL bool bad_pivot(float d, float p) { return !(d > 0.0f) || !(p <= 3.4028234663852886e38f); }
 SELINV_DEVINL double rsqrt_t(double d) { return rsqrt(d); }
 SELINV_DEVINL float rsqrt_t(float d) { return rsqrtf(d); }
 
@@ -104,9 +152,9 @@ SELINV_DEVINL void inv8_sweep(T v[2], int lane, int g, int t, LogAcc &det, bool 
         row[0] = shfl(v[0], (k << 2) | t);                         // P[k][2t]
         row[1] = shfl(v[1], (k << 2) | t);                         // P[k][2t+1]
         const T d = shfl(v[kj], (k << 2) | kt);                    // P[k][k]
-        bad |= !(d > T(0));
         if (count) det.mul((double)d);
         const T p = recip(d);
+        bad |= bad_pivot(d, p);
         if (DRAW) {
             const T zk = shfl(kj ? z1 : z0, (lane & ~3) | kt);
             if (g >= k) *rz = fma(c, zk * rsqrt_t(d), *rz);

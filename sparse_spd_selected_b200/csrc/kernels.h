@@ -24,6 +24,7 @@ template <class T> struct ChainArgs {
     int64_t batch;
     int64_t L;
     int b;
+    bool ws_lines = false;  // workspace starts on a 128-byte boundary (its slots may be dropped from L2)
 };
 
 // b <= 16: one warp per chain.
@@ -87,5 +88,14 @@ template <class T> struct BidiagBwdArgs {
     int b;
 };
 template <class T> cudaError_t bidiag_backward_launch(const BidiagBwdArgs<T> &a, bool aligned16, cudaStream_t s);
+
+// SELINV_CHECK: finiteness of every entry a call reads, reported in info as
+// -3 - k (k = first block with a non-finite entry); runs after the call's
+// kernels.  kind 0: lower triangles of b x b blocks, 1: whole blocks, 2:
+// length-b vectors; a: [batch, nb, ...]; parent (trees): skip root slots.
+template <class T>
+cudaError_t check_finite_launch(const T *a, int64_t batch, int64_t nb, int b, int kind, const int32_t *parent,
+                                int32_t *info, cudaStream_t s);
+cudaError_t check_finalize_launch(int32_t *info, int64_t batch, int64_t nb, cudaStream_t s);
 
 }  // namespace selinv

@@ -35,15 +35,17 @@ template <class T> SELINV_DEVINL T *quad(T *img, int r, int c) { return img + (2
 
 // Quadrant (i, k) of an operand held as four images: TR = false gives
 // M[i][k]; TR = true gives (M^T)[i][k] = M[k][i]^T.
-template <bool TR, class T> SELINV_DEVINL void qget(w16::Tile<T> &o, T *img, int i, int k, int g, int t)
+// The image's element type S may be narrower than the tile's A (a float
+// input image read into float64 tiles).
+template <bool TR, class A, class S> SELINV_DEVINL void qget(w16::Tile<A> &o, S *img, int i, int k, int g, int t)
 {
-    if (TR) w16::from_smem_T<T>(o, quad(img, k, i), g, t);
-    else w16::from_smem<T>(o, quad(img, i, k), g, t);
+    if (TR) w16::from_smem_T_as<A, S>(o, quad(img, k, i), g, t);
+    else w16::from_smem_as<A, S>(o, quad(img, i, k), g, t);
 }
 
 // acc += (NEG ? -1 : 1) (X Y^T)_{IJ} = sum_K X_IK Y_JK^T, operands from images.
-template <bool NEG, bool TX, bool TY, bool LOWER, class T>
-SELINV_DEVINL void qgemm(w16::Tile<T> &acc, T *imgX, T *imgY, int I, int J, T *s1, T *s2, int g, int t)
+template <bool NEG, bool TX, bool TY, bool LOWER, class T, class SX, class SY>
+SELINV_DEVINL void qgemm(w16::Tile<T> &acc, SX *imgX, SY *imgY, int I, int J, T *s1, T *s2, int g, int t)
 {
 #pragma unroll
     for (int K = 0; K < 2; ++K) {
@@ -91,16 +93,47 @@ template <class T, bool FULL> SELINV_DEVINL void load_full(T *img, const T *B, i
     }
 }
 
-// The warp's quadrant of the symmetric block whose lower quadrants are in img.
-template <class T> SELINV_DEVINL void sym_quad(w16::Tile<T> &o, T *img, int I, int J, int g, int t)
+// The same two loads into float64 images from blocks of element type T
+// (plain loads, widened; the caller's barrier makes them visible).  For
+// T = double they are the cp.async loads above (the caller commits / waits).
+template <class T, bool FULL> SELINV_DEVINL void load_diag_f64(double *img, const T *D, int b, int tid)
 {
-    if (I == J) w16::from_smem_lower<T>(o, quad(img, I, J), g, t);
-    else if (I > J) w16::from_smem<T>(o, quad(img, I, J), g, t);
-    else w16::from_smem_T<T>(o, quad(img, J, I), g, t);
+    if constexpr (std::is_same<T, double>::value) {
+        load_diag<double, FULL>(img, D, b, tid);
+    } else {
+        for (int j = tid; j < 1024; j += GT) {
+            const int r = j >> 5, c = j & 31;
+            if (c <= r)
+                quad(img, r >> 4, c >> 4)[w16::SL<double>::idx(r & 15, c & 15)] =
+                    (r < b && c < b) ? (double)__ldg(D + r * b + c) : (r == c ? 1.0 : 0.0);
+        }
+    }
+}
+template <class T, bool FULL> SELINV_DEVINL void load_full_f64(double *img, const T *B, int b, int tid)
+{
+    if constexpr (std::is_same<T, double>::value) {
+        load_full<double, FULL>(img, B, b, tid);
+    } else {
+        for (int j = tid; j < 1024; j += GT) {
+            const int r = j >> 5, c = j & 31;
+            quad(img, r >> 4, c >> 4)[w16::SL<double>::idx(r & 15, c & 15)] =
+                (r < b && c < b) ? (double)__ldg(B + r * b + c) : 0.0;
+        }
+    }
 }
 
-// Store a quadrant tile into a row-major b x b block (TR: transposed position).
-template <class T, bool TR> SELINV_DEVINL void store_quad(T *G, const w16::Tile<T> &a, int b, int I, int J, int g, int t)
+// The warp's quadrant of the symmetric block whose lower quadrants are in img.
+template <class A, class S> SELINV_DEVINL void sym_quad(w16::Tile<A> &o, S *img, int I, int J, int g, int t)
+{
+    if (I == J) w16::from_smem_lower_as<A, S>(o, quad(img, I, J), g, t);
+    else if (I > J) w16::from_smem_as<A, S>(o, quad(img, I, J), g, t);
+    else w16::from_smem_T_as<A, S>(o, quad(img, J, I), g, t);
+}
+
+// Store a quadrant tile into a row-major b x b block (TR: transposed position),
+// rounded to the block's element type T.
+template <class T, bool TR, class A>
+SELINV_DEVINL void store_quad(T *G, const w16::Tile<A> &a, int b, int I, int J, int g, int t)
 {
 #pragma unroll
     for (int h = 0; h < 2; ++h)
@@ -112,7 +145,7 @@ template <class T, bool TR> SELINV_DEVINL void store_quad(T *G, const w16::Tile<
                 r = c;
                 c = tmp;
             }
-            if (r < b && c < b) G[r * b + c] = a.v[h][q];
+            if (r < b && c < b) G[r * b + c] = (T)a.v[h][q];
         }
 }
 
@@ -141,9 +174,9 @@ SELINV_DEVINL void qinverse_scalar(w16::Tile<T> &a, T *cbuf, int I, int J, int g
             const V r01 = *reinterpret_cast<const V *>(cb + 16 * J + 2 * t);
             const V r23 = *reinterpret_cast<const V *>(cb + 16 * J + 2 * t + 8);
             const T row[4] = {r01.x, r01.y, r23.x, r23.y};
-            bad |= !(d > T(0));
             det.mul((double)d);
             const T p = recip(d);
+            bad |= bad_pivot(d, p);
             const T tc[2] = {c0 * p, c1 * p};
 #pragma unroll
             for (int h = 0; h < 2; ++h)

@@ -42,6 +42,8 @@ struct selinv_tree_plan_s {
     int32_t *d_child_ptr = nullptr;        // [trees*n + 1]
     int32_t *d_child_idx = nullptr;        // global ids, ascending per parent
     int32_t *d_parent = nullptr;           // global parent id or -1
+    int32_t spin_limit = 1 << 22;          // polls before a dependency wait gives up (SPIN_LIMIT)
+    int64_t hold = -1;                     // node whose completion is never published (tests)
 };
 
 namespace selinv {
@@ -64,6 +66,8 @@ struct TreeDev {
     const int32_t *child_idx;
     const int32_t *parent;
     int64_t n;
+    int32_t spin_limit;   // polls before a dependency wait gives up
+    int64_t hold;         // a node whose completion flag is never published (tests), or -1
 };
 
 template <class T> struct TreeBufs {
@@ -84,6 +88,11 @@ struct TreeSync {
 };
 
 constexpr int SPIN_LIMIT = 1 << 22;     // x >= 64 ns per poll: well over a second
+
+// Completion flags of the sweeps: 0 = not yet, 1 = the node's data is
+// published, 2 = the node gave up (its own wait ran out, or its parent gave
+// up), so its children give up at once instead of each spinning to the limit.
+constexpr int FLAG_READY = 1, FLAG_FAILED = 2;
 
 SELINV_DEVINL unsigned long long warp_take(unsigned long long *ctr, int lane)
 {
@@ -112,6 +121,36 @@ SELINV_DEVINL int atom_add_acq_rel(int32_t *p, int v)
 SELINV_DEVINL void st_release(int32_t *p, int v)
 {
     asm volatile("st.release.gpu.global.s32 [%0], %1;\n" ::"l"(p), "r"(v) : "memory");
+}
+
+// Bounded wait of lane 0 for a parent's completion flag, broadcast to the
+// warp: 1 when the parent's data may be read, 0 when the parent gave up or
+// the flag stayed unset for td.spin_limit polls.
+SELINV_DEVINL int wait_parent(const int32_t *flag, int limit, int lane, unsigned sleep_ns)
+{
+    int ok = 0;
+    if (lane == 0) {
+        int n = 0, f;
+        while ((f = ld_acquire(flag)) == 0 && ++n <= limit) __nanosleep(sleep_ns);
+        ok = f == FLAG_READY;
+    }
+    return __shfl_sync(FULL_MASK, ok, 0);
+}
+
+// Lane 0 publishes node v's completion (after a warp barrier that orders the
+// warp's stores before it); a node held back for a test stays unpublished.
+SELINV_DEVINL void publish(int32_t *done, const TreeDev &td, int32_t v, int lane)
+{
+    if (lane == 0 && v != td.hold) st_release(done + v, FLAG_READY);
+}
+
+// A wait gave up: the tree reports -2 and v's children (if any) give up too.
+SELINV_DEVINL void give_up(int32_t *info, int32_t *done, const TreeDev &td, int32_t v, int lane)
+{
+    if (lane == 0) {
+        atomicMin(info + v / td.n, -2);
+        if (td.child_ptr[v + 1] > td.child_ptr[v]) st_release(done + v, FLAG_FAILED);
+    }
 }
 
 template <class T> SELINV_DEVINL void load_lower_slot_l2(w16::Tile<T> &a, const T *slot, int lane, int g, int t)
@@ -218,7 +257,7 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leave
                 }
                 if (par < 0) {                        // root: its draw is u_v, published
                     __syncwarp();                     // the warp's stores are ordered before lane 0's release
-                    if (lane == 0) st_release(sy.done + v, 1);
+                    publish(sy.done, td, v, lane);
                     __syncwarp();
                     break;
                 }
@@ -233,7 +272,7 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leave
                 zero(z);
                 store_block<T, FULL>(p.G_edge + v * bb, z, b, g, t);
                 __syncwarp();                         // the warp's stores are ordered before lane 0's release
-                if (lane == 0) st_release(sy.done + v, 1);
+                publish(sy.done, td, v, lane);
                 __syncwarp();
                 break;
             }
@@ -292,15 +331,7 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
         const int32_t v = nodes[k];
         const int32_t par = td.parent[v];
         const unsigned long long kn = warp_take(sy.counters + 1, lane);
-        int ok = 1;                                   // wait for G_pp (bounded)
-        if (lane == 0) {
-            int n = 0;
-            while (ld_acquire(sy.done + par) == 0) {
-                if (++n > SPIN_LIMIT) { ok = 0; break; }
-                __nanosleep(64);
-            }
-        }
-        ok = __shfl_sync(FULL_MASK, ok, 0);
+        const int ok = wait_parent(sy.done + par, td.spin_limit, lane, 64);   // G_pp (bounded wait)
         __syncwarp();                                 // every lane's reads below are ordered after lane 0's acquire
         if (ok) load_lower_async<T, FULL>(sG, p.G_diag + (int64_t)par * bb, b, lane);   // G_pp, from L2
         cp_async_commit();
@@ -314,8 +345,8 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
             cp_async_wait_all();
         }
         __syncwarp();
-        if (!ok) {                                    // cannot happen for a valid plan: report, move on
-            if (lane == 0) atomicMin(p.info + v / td.n, -2);
+        if (!ok) {                                    // the parent never published: report, pass it on
+            give_up(p.info, sy.done, td, v, lane);
             k = kn;
             cur ^= 1;
             continue;
@@ -342,7 +373,7 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
         from_smem_lower<T>(a, sT, g, t);              // exactly symmetric
         store_block<T, FULL>(p.G_diag + v * bb, a, b, g, t);
         __syncwarp();                                 // the warp's stores are ordered before lane 0's release
-        if (lane == 0 && td.child_ptr[v + 1] > td.child_ptr[v]) st_release(sy.done + v, 1);   // only parents are waited for
+        if (td.child_ptr[v + 1] > td.child_ptr[v]) publish(sy.done, td, v, lane);   // only parents are waited for
         __syncwarp();
         k = kn;
         cur ^= 1;
@@ -407,18 +438,10 @@ tree_draw_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *nodes, i
         for (int j = 0; j < DCHUNK; ++j) {
             if (j >= m) break;
             const int32_t v = vs[j], par = ps[j];
-            int ok = 1;                               // wait for w_p (bounded)
-            if (lane == 0) {
-                int n = 0;
-                while (ld_acquire(sy.done + par) == 0) {
-                    if (++n > SPIN_LIMIT) { ok = 0; break; }
-                    __nanosleep(32);
-                }
-            }
-            ok = __shfl_sync(FULL_MASK, ok, 0);
+            const int ok = wait_parent(sy.done + par, td.spin_limit, lane, 32);   // w_p (bounded wait)
             __syncwarp();                             // every lane's reads below follow lane 0's acquire
-            if (!ok) {                                // cannot happen for a valid plan: report, move on
-                if (lane == 0) atomicMin(p.info + v / td.n, -2);
+            if (!ok) {                                // the parent never published: report, pass it on
+                give_up(p.info, sy.done, td, v, lane);
                 continue;
             }
             const T *wp = p.eta + (int64_t)par * b + 8 * hf;
@@ -429,7 +452,7 @@ tree_draw_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *nodes, i
             s2 += shfl_xor(s2, 1);
             if (hf == 0 && r < b) p.eta[(int64_t)v * b + r] = uv[j] - s2;
             __syncwarp();                             // the warp's stores are ordered before lane 0's release
-            if (lane == 0 && td.child_ptr[v + 1] > td.child_ptr[v]) st_release(sy.done + v, 1);
+            if (td.child_ptr[v + 1] > td.child_ptr[v]) publish(sy.done, td, v, lane);
             __syncwarp();
         }
     }
@@ -570,7 +593,7 @@ tree_bw_collect_kernel(TreeBwdBufs<T> p, TreeDev td, TreeSync sy, const int32_t 
                 store_block<T, FULL>(p.Eb + v * bb, z, b, g, t);
                 store_lower_slot<T>(p.ws_U + (int64_t)v * SLOT_ELEMS, sg, lane, g, t);
                 __syncwarp();                         // the warp's stores are ordered before lane 0's release
-                if (lane == 0) st_release(sy.done + v, 1);
+                publish(sy.done, td, v, lane);
                 __syncwarp();
                 break;
             }
@@ -673,18 +696,10 @@ tree_bw_distribute_kernel(TreeBwdBufs<T> p, TreeDev td, TreeSync sy, const int32
         sym_from_slot<T>(Pt, p.ws_Pd + (int64_t)v * SLOT_ELEMS, s0, lane, g, t);
         load_gen<T, FULL>(Ev, p.edge + v * bb, b, g, t, false);
         load_gen<T, FULL>(ed, p.Eb + v * bb, b, g, t, true);
-        int ok = 1;                                   // wait for Sg_p (bounded)
-        if (lane == 0) {
-            int n = 0;
-            while (ld_acquire(sy.done + par) == 0) {
-                if (++n > SPIN_LIMIT) { ok = 0; break; }
-                __nanosleep(64);
-            }
-        }
-        ok = __shfl_sync(FULL_MASK, ok, 0);
+        const int ok = wait_parent(sy.done + par, td.spin_limit, lane, 64);   // Sg_p (bounded wait)
         __syncwarp();                                 // every lane's reads below follow lane 0's acquire
-        if (!ok) {                                    // cannot happen for a valid plan: report, move on
-            if (lane == 0) atomicMin(p.info + v / td.n, -2);
+        if (!ok) {                                    // the parent never published: report, pass it on
+            give_up(p.info, sy.done, td, v, lane);
             continue;
         }
         Tile<T> Sp, ET;
@@ -713,7 +728,7 @@ tree_bw_distribute_kernel(TreeBwdBufs<T> p, TreeDev td, TreeSync sy, const int32
         if (td.child_ptr[v + 1] > td.child_ptr[v]) {
             store_lower_slot<T>(p.ws_U + (int64_t)v * SLOT_ELEMS, sg, lane, g, t);
             __syncwarp();                             // the warp's stores are ordered before lane 0's release
-            if (lane == 0) st_release(sy.done + v, 1);
+            publish(sy.done, td, v, lane);
             __syncwarp();
         }
     }
@@ -803,7 +818,7 @@ cudaError_t run_tree(const selinv_tree_plan_s *pl, int b, const T *diag, const T
     sy.counters = reinterpret_cast<unsigned long long *>(w);
     p.info = info;
     p.b = b;
-    TreeDev td{pl->d_child_ptr, pl->d_child_idx, pl->d_parent, pl->n};
+    TreeDev td{pl->d_child_ptr, pl->d_child_idx, pl->d_parent, pl->n, pl->spin_limit, pl->hold};
 
     const int64_t init_n = std::max<int64_t>(N, pl->trees);
     tree_init<<<(unsigned)ceil_div(init_n, 256), 256, 0, s>>>(pl->d_child_ptr, N, sy.pending, sy.done, sy.counters,
@@ -883,7 +898,7 @@ cudaError_t run_tree_backward(const selinv_tree_plan_s *pl, int b, const T *diag
     sy.counters = reinterpret_cast<unsigned long long *>(w);
     p.info = info;
     p.b = b;
-    TreeDev td{pl->d_child_ptr, pl->d_child_idx, pl->d_parent, pl->n};
+    TreeDev td{pl->d_child_ptr, pl->d_child_idx, pl->d_parent, pl->n, pl->spin_limit, pl->hold};
 
     const int64_t init_n = std::max<int64_t>(N, pl->trees);
     tree_init<<<(unsigned)ceil_div(init_n, 256), 256, 0, s>>>(pl->d_child_ptr, N, sy.pending, sy.done, sy.counters,
@@ -1054,6 +1069,14 @@ void selinv_tree_plan_free(selinv_tree_plan_t *pl)
     delete pl;
 }
 
+selinv_status selinv_tree_plan_set_wait(selinv_tree_plan_t *pl, int32_t spin_limit, int64_t withhold)
+{
+    if (!pl || withhold < -1 || withhold >= pl->trees * pl->n) return SELINV_ERR_INVALID_ARG;
+    pl->spin_limit = spin_limit >= 1 ? spin_limit : selinv::SPIN_LIMIT;
+    pl->hold = withhold;
+    return SELINV_OK;
+}
+
 selinv_status selinv_tree_plan_levels(const selinv_tree_plan_t *pl, int32_t *collect, int32_t *distribute)
 {
     if (!pl || !collect || !distribute) return SELINV_ERR_INVALID_ARG;
@@ -1070,9 +1093,11 @@ size_t selinv_tree_workspace_size(const selinv_tree_plan_t *pl, selinv_dtype dty
 
 selinv_status selinv_tree(const selinv_tree_plan_t *pl, selinv_dtype dtype, int32_t b, const void *diag,
                           const void *edge, void *G_diag, void *G_edge, double *logdet, int32_t *info,
-                          void *workspace, size_t workspace_bytes, void *stream)
+                          void *workspace, size_t workspace_bytes, uint32_t flags, void *stream)
 {
     if (!pl || (dtype != SELINV_F64 && dtype != SELINV_F32) || b < 1) return SELINV_ERR_INVALID_ARG;
+    if (flags & ~(uint32_t)(SELINV_WANT_LOGDET | SELINV_CHECK)) return SELINV_ERR_INVALID_ARG;
+    if ((flags & SELINV_WANT_LOGDET) && logdet == nullptr) return SELINV_ERR_INVALID_ARG;
     if (b > 16) return SELINV_ERR_UNSUPPORTED;
     if (!diag || !edge || !G_diag || !G_edge || !info) return SELINV_ERR_INVALID_ARG;
     const size_t es = dtype == SELINV_F64 ? 8 : 4;
@@ -1096,6 +1121,22 @@ selinv_status selinv_tree(const selinv_tree_plan_t *pl, selinv_dtype dtype, int3
         err = run_tree<float>(pl, b, static_cast<const float *>(diag), static_cast<const float *>(edge),
                               static_cast<float *>(G_diag), static_cast<float *>(G_edge), logdet, info,
                               workspace, full, s);
+    if (err == cudaSuccess && (flags & SELINV_CHECK)) {       // D_v (lower triangles) and non-root edge[v] finite
+        if (dtype == SELINV_F64) {
+            err = check_finite_launch<double>(static_cast<const double *>(diag), pl->trees, pl->n, b, 0, nullptr,
+                                              info, s);
+            if (err == cudaSuccess)
+                err = check_finite_launch<double>(static_cast<const double *>(edge), pl->trees, pl->n, b, 1,
+                                                  pl->d_parent, info, s);
+        } else {
+            err = check_finite_launch<float>(static_cast<const float *>(diag), pl->trees, pl->n, b, 0, nullptr,
+                                             info, s);
+            if (err == cudaSuccess)
+                err = check_finite_launch<float>(static_cast<const float *>(edge), pl->trees, pl->n, b, 1,
+                                                 pl->d_parent, info, s);
+        }
+        if (err == cudaSuccess) err = check_finalize_launch(info, pl->trees, pl->n, s);
+    }
     return err == cudaSuccess ? SELINV_OK : SELINV_ERR_CUDA;
 }
 

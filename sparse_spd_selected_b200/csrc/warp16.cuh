@@ -5,6 +5,8 @@
 // log 1 = 0 to the log-determinant.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace selinv {
@@ -120,7 +122,9 @@ template <class T, bool FULL> SELINV_DEVINL void load_sym(Tile<T> &a, const T *D
 // Lower triangle of a diagonal block D (row-major b x b) into shared memory
 // (entries with c <= r; identity pad beyond b).  FULL: 16-byte cp.async
 // chunks that touch the lower triangle only (caller commits / waits).
-template <class T, bool FULL> SELINV_DEVINL void load_lower_async(T *s, const T *D, int b, int lane)
+// HINT: the copies carry the L2 eviction policy pol.
+template <class T, bool FULL, bool HINT = false>
+SELINV_DEVINL void load_lower_async(T *s, const T *D, int b, int lane, uint64_t pol = 0)
 {
     if (FULL) {
         constexpr int CH = 16 / sizeof(T);
@@ -128,7 +132,10 @@ template <class T, bool FULL> SELINV_DEVINL void load_lower_async(T *s, const T 
 #pragma unroll
         for (int j = lane; j < 16 * PER_ROW; j += 32) {
             const int r = j / PER_ROW, c = (j % PER_ROW) * CH;
-            if (c <= r) cp_async16(s + SL<T>::idx(r, c), D + r * 16 + c);
+            if (c <= r) {
+                if (HINT) cp_async16_hint(s + SL<T>::idx(r, c), D + r * 16 + c, pol);
+                else cp_async16(s + SL<T>::idx(r, c), D + r * 16 + c);
+            }
         }
     } else {
         for (int j = lane; j < 256; j += 32) {
@@ -152,7 +159,9 @@ template <class T> SELINV_DEVINL void from_smem_lower(Tile<T> &a, const T *s, in
 
 // Off-diagonal block (row-major b x b) into shared memory, zero pad beyond b.
 // FULL: 16-byte cp.async chunks (caller commits / waits); else plain loads.
-template <class T, bool FULL> SELINV_DEVINL void load_block_async(T *s, const T *B, int b, int lane)
+// HINT: the copies carry the L2 eviction policy pol.
+template <class T, bool FULL, bool HINT = false>
+SELINV_DEVINL void load_block_async(T *s, const T *B, int b, int lane, uint64_t pol = 0)
 {
     if (FULL) {
         constexpr int CH = 16 / sizeof(T);          // elements per chunk
@@ -160,7 +169,8 @@ template <class T, bool FULL> SELINV_DEVINL void load_block_async(T *s, const T 
 #pragma unroll
         for (int j = lane; j < 16 * PER_ROW; j += 32) {
             const int r = j / PER_ROW, c = (j % PER_ROW) * CH;
-            cp_async16(s + SL<T>::idx(r, c), B + r * 16 + c);
+            if (HINT) cp_async16_hint(s + SL<T>::idx(r, c), B + r * 16 + c, pol);
+            else cp_async16(s + SL<T>::idx(r, c), B + r * 16 + c);
         }
     } else {
         for (int j = lane; j < 256; j += 32) {
@@ -212,22 +222,38 @@ template <class T, bool FULL> SELINV_DEVINL void store_block_T(T *G, const Tile<
 // diagonal pairs) are kept; to_smem_sym rebuilds the full block.
 constexpr int SLOT_ELEMS = 192;
 
-template <class T> SELINV_DEVINL void store_lower_slot(T *slot, const Tile<T> &a, int lane, int g, int t)
+// HINT: the stores carry the L2 eviction policy pol.
+template <class T, bool HINT = false>
+SELINV_DEVINL void store_lower_slot(T *slot, const Tile<T> &a, int lane, int g, int t, uint64_t pol = 0)
 {
     using V = typename Vec2<T>::type;
+    auto put = [&](T *p, V v) {
+        if (HINT) st_hint(reinterpret_cast<V *>(p), v, pol);
+        else *reinterpret_cast<V *>(p) = v;
+    };
     V v;
     v.x = a.v[1][0];
     v.y = a.v[1][1];
-    *reinterpret_cast<V *>(slot + 2 * lane) = v;
+    put(slot + 2 * lane, v);
     if (2 * t <= g) {
         V u, w;
         u.x = a.v[0][0];
         u.y = a.v[0][1];
         w.x = a.v[1][2];
         w.y = a.v[1][3];
-        *reinterpret_cast<V *>(slot + 64 + 4 * lane) = u;
-        *reinterpret_cast<V *>(slot + 64 + 4 * lane + 2) = w;
+        put(slot + 64 + 4 * lane, u);
+        put(slot + 64 + 4 * lane + 2, w);
     }
+}
+
+// Drop a slot's L2 lines without writing them back once the slot has been
+// read (lanes 0.. take one 128-byte line each; the slot must start on a
+// 128-byte boundary, which the launchers check).
+template <class T> SELINV_DEVINL void discard_slot(const T *slot, int lane)
+{
+    constexpr int LINES = SLOT_ELEMS * (int)sizeof(T) / 128;
+    static_assert(SLOT_ELEMS * sizeof(T) % 128 == 0, "slots are whole L2 lines");
+    if (lane < LINES) discard_l2_line(reinterpret_cast<const char *>(slot) + 128 * lane);
 }
 
 template <class T> SELINV_DEVINL void load_lower_slot(Tile<T> &a, const T *slot, int lane, int g, int t)
@@ -251,14 +277,19 @@ template <class T> SELINV_DEVINL void load_lower_slot(Tile<T> &a, const T *slot,
 
 // The same slot copied to shared memory by each lane for itself (cp.async;
 // the caller commits / waits), then read back by the same lane.
-template <class T> SELINV_DEVINL void stage_lower_slot(T *stg, const T *slot, int lane, int g, int t)
+template <class T, bool HINT = false>
+SELINV_DEVINL void stage_lower_slot(T *stg, const T *slot, int lane, int g, int t, uint64_t pol = 0)
 {
     constexpr int CH = 16 / sizeof(T);          // elements per 16-byte chunk
     if (CH == 2) {
-        cp_async16(stg + 2 * lane, slot + 2 * lane);
+        auto cp = [&](T *d, const T *src) {
+            if (HINT) cp_async16_hint(d, src, pol);
+            else cp_async16(d, src);
+        };
+        cp(stg + 2 * lane, slot + 2 * lane);
         if (2 * t <= g) {
-            cp_async16(stg + 64 + 4 * lane, slot + 64 + 4 * lane);
-            cp_async16(stg + 64 + 4 * lane + 2, slot + 64 + 4 * lane + 2);
+            cp(stg + 64 + 4 * lane, slot + 64 + 4 * lane);
+            cp(stg + 64 + 4 * lane + 2, slot + 64 + 4 * lane + 2);
         }
     } else {                                    // float: 8-byte pairs, plain loads
         *reinterpret_cast<typename Vec2<T>::type *>(stg + 2 * lane) =
@@ -301,6 +332,37 @@ template <class T> SELINV_DEVINL void from_smem_T(Tile<T> &a, const T *s, int g,
     for (int h = 0; h < 2; ++h)
 #pragma unroll
         for (int q = 0; q < 4; ++q) a.v[h][q] = s[SL<T>::idx(tcol(t, q), g + 8 * h)];
+}
+
+// Readers of an S-typed shared image into a tile of element type A (a float
+// image widened into a float64 tile; the same reader when A = S).
+template <class A, class S> SELINV_DEVINL void from_smem_as(Tile<A> &a, const S *s, int g, int t)
+{
+    if constexpr (std::is_same<A, S>::value) {
+        from_smem<S>(a, s, g, t);
+    } else {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) a.v[h][q] = (A)s[SL<S>::idx(g + 8 * h, tcol(t, q))];
+    }
+}
+template <class A, class S> SELINV_DEVINL void from_smem_T_as(Tile<A> &a, const S *s, int g, int t)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) a.v[h][q] = (A)s[SL<S>::idx(tcol(t, q), g + 8 * h)];
+}
+template <class A, class S> SELINV_DEVINL void from_smem_lower_as(Tile<A> &a, const S *s, int g, int t)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = g + 8 * h, c = tcol(t, q);
+            a.v[h][q] = (A)(c <= r ? s[SL<S>::idx(r, c)] : s[SL<S>::idx(c, r)]);
+        }
 }
 
 // acc += (NEG ? -1 : 1) X Y^T for register tiles X, Y (16 x 16).
@@ -445,9 +507,9 @@ SELINV_DEVINL void spd_inverse_scalar(Tile<T> &a, T *cbuf, int g, int t, LogAcc 
         const V r01 = *reinterpret_cast<const V *>(cb + 2 * t);
         const V r23 = *reinterpret_cast<const V *>(cb + 2 * t + 8);
         const T row[4] = {r01.x, r01.y, r23.x, r23.y};
-        bad |= !(d > T(0));
         det.mul((double)d);
         const T p = recip(d);
+        bad |= bad_pivot(d, p);
         if (DRAW) {
             const T s = shfl(zc[kq], kt) * rsqrt_t(d);
             if (g >= k) v[0] = fma(c0, s, v[0]);

@@ -22,8 +22,10 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.environ.get("SELINV_LIB") or os.path.join(_HERE, "libselinv.so")
 
-OK, ERR_INVALID_ARG, ERR_NOT_SPD, ERR_BAD_TREE, ERR_CUDA, ERR_WORKSPACE, ERR_UNSUPPORTED, ERR_HOST_MEMORY = range(8)
+(OK, ERR_INVALID_ARG, ERR_NOT_SPD, ERR_BAD_TREE, ERR_CUDA, ERR_WORKSPACE, ERR_UNSUPPORTED, ERR_HOST_MEMORY,
+ ERR_TIMEOUT) = range(9)
 F64, F32 = 0, 1
+WANT_LOGDET, WANT_SOLVE, CHECK = 1, 2, 4          # flags of selinv_chain / selinv_tree
 
 _lib = None
 
@@ -38,6 +40,23 @@ class NotSPDError(SelinvError):
     def __init__(self, info):
         self.info = info
         super().__init__(ERR_NOT_SPD, f"first failing block per batch element: {info}")
+
+
+class WaitTimeoutError(SelinvError):
+    """A bounded dependency wait of a tree sweep gave up (info = -2 for that tree)."""
+
+    def __init__(self, info):
+        self.info = info
+        super().__init__(ERR_TIMEOUT, f"info per tree: {info}")
+
+
+class NonFiniteInputError(SelinvError):
+    """An input entry the call reads is not finite (validate=True: SELINV_CHECK)."""
+
+    def __init__(self, info):
+        self.info = info
+        blocks = [(-3 - v) if v <= -3 else None for v in info]
+        super().__init__(ERR_INVALID_ARG, f"first block with a non-finite entry per batch element: {blocks}")
 
 
 class SingularBlockError(SelinvError):
@@ -65,7 +84,7 @@ def lib():
         L.selinv_chain_workspace_size.restype = SZ
         L.selinv_chain_segments.argtypes = [I64, I64, I32, I32, I32]
         L.selinv_chain_segments.restype = I32
-        L.selinv_chain.argtypes = [ctypes.c_int, I64, I64, I32, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.selinv_chain.argtypes = [ctypes.c_int, I64, I64, I32, P, P, P, P, P, P, P, P, P, SZ, ctypes.c_uint32, P]
         L.selinv_chain.restype = ctypes.c_int
         L.chain_solve_multi.argtypes = [ctypes.c_int, I64, I64, I32, I32, P, P, P, P, P, P, P, SZ, P]
         L.chain_solve_multi.restype = ctypes.c_int
@@ -105,11 +124,13 @@ def lib():
         L.selinv_tree_plan.restype = ctypes.c_int
         L.selinv_tree_plan_free.argtypes = [P]
         L.selinv_tree_plan_free.restype = None
+        L.selinv_tree_plan_set_wait.argtypes = [P, I32, I64]
+        L.selinv_tree_plan_set_wait.restype = ctypes.c_int
         L.selinv_tree_plan_levels.argtypes = [P, ctypes.POINTER(I32), ctypes.POINTER(I32)]
         L.selinv_tree_plan_levels.restype = ctypes.c_int
         L.selinv_tree_workspace_size.argtypes = [P, ctypes.c_int, I32]
         L.selinv_tree_workspace_size.restype = SZ
-        L.selinv_tree.argtypes = [P, ctypes.c_int, I32, P, P, P, P, P, P, P, SZ, P]
+        L.selinv_tree.argtypes = [P, ctypes.c_int, I32, P, P, P, P, P, P, P, SZ, ctypes.c_uint32, P]
         L.selinv_tree_sample.argtypes = [P, ctypes.c_int, I32, P, P, P, P, P, P, P, SZ, P]
         L.selinv_tree_sample.restype = ctypes.c_int
         L.selinv_tree.restype = ctypes.c_int
@@ -179,18 +200,26 @@ def _workspace(nbytes, device, workspace):
 def _raise_on_info(info, check):
     if check:
         host = info.cpu()
+        if bool((host <= -3).any()):
+            raise NonFiniteInputError(host.tolist())
+        if bool((host == -2).any()):
+            raise WaitTimeoutError(host.tolist())
         if bool((host >= 0).any()):
             raise NotSPDError(host.tolist())
 
 
 def selinv_chain(diag: torch.Tensor, lower: Optional[torch.Tensor] = None, rhs: Optional[torch.Tensor] = None,
-                 *, want_g: bool = True, check: bool = True, out=None, workspace=None, stream=None):
+                 *, want_g: bool = True, check: bool = True, validate: bool = False, out=None, workspace=None,
+                 stream=None):
     """Selected inverse (+ log det, + optional solve) of block-tridiagonal SPD chains.
 
     diag [..., L, b, b], lower [..., L-1, b, b] (lower[i] = A_{i+1,i}),
     rhs [..., L, b] optional.  Returns a dict with G_diag, G_lower, logdet
     (float64), x (if rhs) and info (int32, -1 = ok).  With check=True the
     call synchronises once to read info and raises NotSPDError on failure.
+    validate=True adds the library's on-device input check (SELINV_CHECK):
+    an element with a non-finite entry among those read reports info
+    -3 - k, raised as NonFiniteInputError when check=True.
     ``out`` may hold preallocated output tensors under the same keys.
     """
     _cuda_contig("diag", diag)
@@ -240,7 +269,7 @@ def selinv_chain(diag: torch.Tensor, lower: Optional[torch.Tensor] = None, rhs: 
     with torch.cuda.device(dev):
         st = lib().selinv_chain(code, batch, L, b, _ptr(diag), _ptr(lower),
                                 _ptr(G_diag), _ptr(G_lower if L > 1 else None), _ptr(logdet),
-                                _ptr(rhs), _ptr(x), _ptr(info), _ptr(ws), nbytes,
+                                _ptr(rhs), _ptr(x), _ptr(info), _ptr(ws), nbytes, CHECK if validate else 0,
                                 _stream_handle(stream))
     _check(st, "selinv_chain")
     _raise_on_info(info, check)
@@ -687,6 +716,11 @@ class TreePlan:
         _check(lib().selinv_tree_plan_levels(self._h, ctypes.byref(c), ctypes.byref(d)), "levels")
         return c.value, d.value
 
+    def set_wait(self, spin_limit: int = 0, withhold: int = -1):
+        """Bound of the sweeps' dependency waits (polls; 0 = the default) and a
+        node whose completion is never published (-1 = none; a test hook)."""
+        _check(lib().selinv_tree_plan_set_wait(self._h, int(spin_limit), int(withhold)), "selinv_tree_plan_set_wait")
+
     def workspace_size(self, dtype, b) -> int:
         return int(lib().selinv_tree_workspace_size(self._h, _code(dtype), b))
 
@@ -705,13 +739,14 @@ class TreePlan:
             pass
 
 
-def selinv_tree(plan: TreePlan, diag: torch.Tensor, edge: torch.Tensor, *, check=True, out=None,
+def selinv_tree(plan: TreePlan, diag: torch.Tensor, edge: torch.Tensor, *, check=True, validate=False, out=None,
                 workspace=None, stream=None):
     """Selected inverse and log det of block-tree SPD matrices.
 
     diag, edge [trees, n, b, b] (or [n, b, b] for one tree) with
     edge[v] = A_{parent(v), v}.  Returns dict with G_diag, G_edge (root slot
-    zero), logdet [trees] float64 and info [trees].
+    zero), logdet [trees] float64 and info [trees].  check and validate as in
+    selinv_chain (info -3 - v: node v holds a non-finite entry).
     """
     _cuda_contig("diag", diag)
     dt = diag.dtype
@@ -743,7 +778,8 @@ def selinv_tree(plan: TreePlan, diag: torch.Tensor, edge: torch.Tensor, *, check
     ws = _workspace(nbytes, dev, workspace)
     with torch.cuda.device(dev):
         st = lib().selinv_tree(plan.handle, code, b, _ptr(d4), _ptr(e4), _ptr(G_diag), _ptr(G_edge),
-                               _ptr(logdet), _ptr(info), _ptr(ws), nbytes, _stream_handle(stream))
+                               _ptr(logdet), _ptr(info), _ptr(ws), nbytes, CHECK if validate else 0,
+                               _stream_handle(stream))
     _check(st, "selinv_tree")
     _raise_on_info(info, check)
     if single:

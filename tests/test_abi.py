@@ -34,7 +34,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_limits(lib):
-    for code in range(8):
+    for code in range(9):
         assert selinv.status_string(code) and selinv.status_string(code) != "unknown status"
     assert selinv.max_block() == 128
     assert lib.selinv_version() >= 100
@@ -44,8 +44,8 @@ FAKE = ctypes.c_void_p(1 << 20)     # never dereferenced: validation fails first
 
 
 def call_chain(lib, dtype=0, batch=1, L=4, b=4, diag=FAKE, lower=FAKE, G=FAKE, Gl=FAKE, ld=None,
-               rhs=None, x=None, info=FAKE, ws=FAKE, ws_bytes=1 << 30):
-    return lib.selinv_chain(dtype, batch, L, b, diag, lower, G, Gl, ld, rhs, x, info, ws, ws_bytes, None)
+               rhs=None, x=None, info=FAKE, ws=FAKE, ws_bytes=1 << 30, flags=0):
+    return lib.selinv_chain(dtype, batch, L, b, diag, lower, G, Gl, ld, rhs, x, info, ws, ws_bytes, flags, None)
 
 
 def test_chain_argument_errors(lib):
@@ -212,3 +212,20 @@ def test_noalloc_rejects_oversized_requests_before_any_device_call(lib):
     assert f(0, 1, 4, 17, FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE, None) == selinv.ERR_UNSUPPORTED
     assert f(0, 1, 4, 4, FAKE, FAKE, FAKE, None, None, None, None, FAKE, None) == selinv.ERR_INVALID_ARG
     assert f(0, 0, 4, 4, FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE, None) == selinv.OK
+
+
+def test_tree_set_wait_argument_errors(lib):
+    assert lib.selinv_tree_plan_set_wait(None, 10, -1) == selinv.ERR_INVALID_ARG
+    assert selinv.status_string(selinv.ERR_TIMEOUT) != "unknown status"
+
+
+def test_flags_are_validated_before_any_launch(lib):
+    """SELINV_WANT_LOGDET / SELINV_WANT_SOLVE insist on their pointers; unknown bits are refused."""
+    assert call_chain(lib, batch=0, flags=selinv.CHECK) == selinv.OK
+    assert call_chain(lib, flags=1 << 7) == selinv.ERR_INVALID_ARG
+    assert call_chain(lib, flags=selinv.WANT_LOGDET) == selinv.ERR_INVALID_ARG          # logdet NULL
+    assert call_chain(lib, flags=selinv.WANT_SOLVE) == selinv.ERR_INVALID_ARG           # rhs, x NULL
+    assert call_chain(lib, batch=0, ld=FAKE, rhs=FAKE, x=FAKE,
+                      flags=selinv.WANT_LOGDET | selinv.WANT_SOLVE | selinv.CHECK) == selinv.OK
+    f = lib.selinv_tree
+    assert f(None, 0, 4, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 1 << 30, 0, None) == selinv.ERR_INVALID_ARG

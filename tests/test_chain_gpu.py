@@ -221,6 +221,34 @@ def test_pivot_reciprocal_against_cuda_division(cuda_ok):
     assert float(torch.max(torch.abs(out["logdet"] - torch.log(dev.reshape(-1))))) <= 1e-12
 
 
+def test_pivot_reciprocal_at_the_ends_of_the_range(cuda_ok):
+    """Pivots near the ends of the float64 range: in [2^-1022, 2^1022) the
+    kernel's Newton-refined reciprocal agrees with CUDA's 1/d to a few ulp;
+    outside it (subnormal pivots, pivots whose reciprocal would be subnormal,
+    pivots whose reciprocal overflows) the fast reciprocal would flush, so the
+    block is reported in info like a non-positive pivot."""
+    rng = np.random.default_rng(321)
+    small = 2.0 ** rng.uniform(-1022.0, -1000.0, 4000)
+    large = 2.0 ** rng.uniform(1000.0, 1021.9, 4000)
+    out_of_range = np.concatenate([
+        2.0 ** rng.uniform(1022.0, 1023.9, 100),                 # reciprocal below 2^-1022
+        2.0 ** np.array([-1022.25, -1023.0, -1030.0, -1060.0]),  # subnormal pivots
+        np.array([5e-324])])
+    d = np.concatenate([small, large, out_of_range])
+    dev = torch.from_numpy(d).cuda().reshape(-1, 1, 1, 1)
+    out = selinv.selinv_chain(dev, None, check=False)
+    G = out["G_diag"].reshape(-1)
+    ref = 1.0 / dev.reshape(-1)
+    info = host(out["info"])
+    n1 = small.size + large.size
+    ulp = torch.abs(G[:n1] - ref[:n1]) / (torch.finfo(torch.float64).eps * torch.abs(ref[:n1]))
+    assert float(ulp.max()) <= 4.0
+    assert (info[:n1] == -1).all()
+    assert (info[n1:] == 0).all()
+    with pytest.raises(selinv.NotSPDError):
+        selinv.selinv_chain(dev[n1:], None)
+
+
 # ---------------- 16 < b <= 32 without a right-hand side: two-ended kernel ----------------
 
 @pytest.mark.parametrize("b", [17, 20, 24, 31, 32])
@@ -307,3 +335,27 @@ def test_segmented_deterministic_and_leading_dims(cuda_ok):
                          torch.float64, lead_ndim=2)
     assert out["G_diag"].shape == (2, 2, 160, 32, 32) and out["logdet"].shape == (2, 2)
     assert max(errs.values()) <= TOL[torch.float64], errs
+
+
+@pytest.mark.parametrize("b", [5, 16, 32, 64])
+def test_validate_reports_non_finite_inputs(cuda_ok, b):
+    """validate=True (SELINV_CHECK): an element whose read entries hold a NaN or
+    an infinity reports info = -3 - k for the first such block k; entries the
+    call does not read (the upper triangle of D) are not checked; clean
+    elements are untouched; check=True raises NonFiniteInputError."""
+    diag, lower, rhs = inputs.chain_inputs(5, 7, b, seed=3500 + b, load=1.0)
+    diag[1, 3, b - 1, 0] = np.nan            # lower triangle of D_3
+    lower[2, 2, 0, b - 1] = np.inf           # B_2
+    rhs[3, 5, 0] = np.nan                    # r_5
+    diag[4, 1, 0, b - 1] = np.nan            # upper triangle of D_1: not read
+    d, l, r = (to_dev(a, torch.float64) for a in (diag, lower, rhs))
+    out = selinv.selinv_chain(d, l, r, check=False, validate=True)
+    info = host(out["info"]).tolist()
+    assert info[0] == -1 and info[4] == -1
+    assert info[1] == -3 - 3 and info[2] == -3 - 2 and info[3] == -3 - 5
+    ref = oracle.chain(diag[[0]], lower[[0]], rhs[[0]])
+    assert worst(host(out["G_diag"])[[0]], ref["G_diag"]) <= 1e-9
+    with pytest.raises(selinv.NonFiniteInputError):
+        selinv.selinv_chain(d, l, r, validate=True)
+    clean = selinv.selinv_chain(d[[0, 4]], l[[0, 4]], r[[0, 4]], validate=True)
+    assert (host(clean["info"]) == -1).all()

@@ -87,3 +87,46 @@ def test_junction_not_spd(cuda_ok):
     assert info[0] == -1 and info[1] >= 0
     with pytest.raises(selinv.NotSPDError):
         selinv.junction(plan, to_dev(d, torch.float64), to_dev(e, torch.float64))
+
+
+def test_junction_lattice_benchmark_size(cuda_ok):
+    """The benchmarked launch: 64 matrices on a 32 x 32 lattice of 8 x 8 blocks
+    (N = 8192 each).  Every matrix: the diagonal block rows of A G = I, which
+    use only blocks on S (the pattern is inside S), sum_u A_vu G_uv = I.  One
+    sampled matrix: every block on S and log det against the dense inverse
+    (numpy's LAPACK on the same matrix, read on S)."""
+    w = inputs.WORKLOADS["lattice_64x1024_b8"]
+    g = inputs.generate(w)
+    E = g["edge_index"]
+    n, b = w.L, w.b
+    plan = selinv.JunctionPlan(n, E)
+    out = selinv.junction(plan, to_dev(g["diag"], torch.float64), to_dev(g["edge_val"], torch.float64))
+    Gd, Gl = host(out["G_diag"]), host(out["G_lower"])
+    Si, Sj = plan.S_index
+    slot = {(int(i), int(j)): k for k, (i, j) in enumerate(zip(Si, Sj))}
+    ei, ej = E
+    sym = lambda D: np.tril(D) + np.swapaxes(np.tril(D, -1), -1, -2)
+    # block row v of A G, diagonal block: D_v G_vv + sum over pattern neighbours u of A_vu G_uv
+    ki = np.array([slot[(int(i), int(j))] for i, j in zip(ei, ej)])
+    for e in range(w.batch):
+        R = np.einsum("vab,vbc->vac", sym(g["diag"][e]), Gd[e]) - np.eye(b)
+        Aij = g["edge_val"][e]                       # A_{i,j}, i > j
+        Gij = Gl[e][ki]                              # (A^-1)_{i,j}
+        np.add.at(R, ei, Aij @ np.swapaxes(Gij, -1, -2))       # row i: A_ij G_ji = A_ij G_ij^T
+        np.add.at(R, ej, np.swapaxes(Aij, -1, -2) @ Gij)       # row j: A_ji G_ij = A_ij^T G_ij
+        assert float(np.abs(R).max()) <= 1e-9, e
+    # one matrix against the dense inverse
+    e = 17
+    N = n * b
+    A = np.zeros((N, N))
+    for v in range(n):
+        A[v * b:(v + 1) * b, v * b:(v + 1) * b] = sym(g["diag"][e, v])
+    for k, (i, j) in enumerate(zip(ei, ej)):
+        A[i * b:(i + 1) * b, j * b:(j + 1) * b] = g["edge_val"][e, k]
+        A[j * b:(j + 1) * b, i * b:(i + 1) * b] = g["edge_val"][e, k].T
+    inv = np.linalg.inv(A)
+    ref_d = np.stack([inv[v * b:(v + 1) * b, v * b:(v + 1) * b] for v in range(n)])
+    ref_l = np.stack([inv[i * b:(i + 1) * b, j * b:(j + 1) * b] for i, j in zip(Si, Sj)])
+    assert worst(Gd[e][None], ref_d[None]) <= 1e-9
+    assert worst(Gl[e][None], ref_l[None]) <= 1e-9
+    assert logdet_err(host(out["logdet"])[e], np.linalg.slogdet(A)[1]) <= 1e-9

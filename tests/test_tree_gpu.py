@@ -91,3 +91,75 @@ def test_tree_not_spd_and_determinism(cuda_ok):
     b = selinv.selinv_tree(plan, to_dev(diag, torch.float64), to_dev(edge, torch.float64))
     for k in ("G_diag", "G_edge", "logdet"):
         assert torch.equal(a[k], b[k])
+
+
+def _held_node(P, tree):
+    """A non-root node of `tree` with children (its children wait on its flag)."""
+    par = P[tree]
+    kids = np.bincount(par[par >= 0], minlength=P.shape[1])
+    cand = [v for v in range(P.shape[1]) if par[v] >= 0 and kids[v] > 0]
+    return tree * P.shape[1] + cand[len(cand) // 2]
+
+
+@pytest.mark.parametrize("b", [16, 5])
+def test_bounded_wait_gives_up_on_an_unpublished_parent(cuda_ok, b):
+    """A node whose completion flag is never published (the plan's test hook):
+    its children give up after the spin limit, its tree reports info = -2
+    (WaitTimeoutError with check=True), the failure reaches the descendants at
+    once, the other trees are exact, and the next call on the same plan and
+    context is correct.  Forward sweep, draw and backward (all three waits)."""
+    import time
+    P, diag, edge = inputs.tree_inputs(3, 300, b, seed=41 + b, load=1.0)
+    plan = selinv.TreePlan(P)
+    dd, ee = to_dev(diag, torch.float64), to_dev(edge, torch.float64)
+    ref = oracle.tree(P, diag, edge)
+    plan.set_wait(spin_limit=4096, withhold=_held_node(P, 1))
+    t0 = time.perf_counter()
+    out = selinv.selinv_tree(plan, dd, ee, check=False)
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 < 10.0
+    assert host(out["info"]).tolist() == [-1, -2, -1]
+    ok = [0, 2]
+    assert worst(host(out["G_diag"])[ok], ref["G_diag"][ok]) <= 1e-9
+    assert worst(host(out["G_edge"])[ok], ref["G_edge"][ok]) <= 1e-9
+    with pytest.raises(selinv.WaitTimeoutError):
+        selinv.selinv_tree(plan, dd, ee)
+    # draw: the vector recurrence waits on the same flags
+    z = to_dev(np.random.default_rng(5).standard_normal((3, 300, b)), torch.float64)
+    dr = selinv.tree_sample(plan, dd, ee, z, check=False)
+    torch.cuda.synchronize()
+    assert host(dr["info"]).tolist() == [-1, -2, -1]
+    # backward: its parents-first pass waits on the same flags
+    plan.set_wait()
+    fwd = selinv.selinv_tree(plan, dd, ee)
+    gd = to_dev(np.random.default_rng(6).standard_normal(diag.shape), torch.float64)
+    bw_ok = selinv.tree_backward(plan, dd, ee, fwd["G_diag"], fwd["G_edge"], gd, None)
+    plan.set_wait(spin_limit=4096, withhold=_held_node(P, 1))
+    bw = selinv.tree_backward(plan, dd, ee, fwd["G_diag"], fwd["G_edge"], gd, None, check=False)
+    torch.cuda.synchronize()
+    assert host(bw["info"]).tolist() == [-1, -2, -1]
+    assert torch.equal(bw["Db"][ok], bw_ok["Db"][ok]) and torch.equal(bw["Eb"][ok], bw_ok["Eb"][ok])
+    # the hook off again: the same plan and context give the exact answer
+    plan.set_wait()
+    again = selinv.selinv_tree(plan, dd, ee)
+    assert (host(again["info"]) == -1).all()
+    assert worst(host(again["G_diag"]), ref["G_diag"]) <= 1e-9
+    assert worst(host(again["G_edge"]), ref["G_edge"]) <= 1e-9
+
+
+def test_tree_validate_reports_non_finite_inputs(cuda_ok):
+    """validate=True on trees: info = -3 - v for the first node v whose D_v
+    (lower triangle) or edge slot holds a non-finite entry; root edge slots and
+    upper triangles are not read, hence not checked."""
+    P, diag, edge = inputs.tree_inputs(4, 60, 16, seed=77, load=1.0)
+    diag[1, 40, 5, 2] = np.nan
+    v2 = int(np.nonzero(P[2] >= 0)[0][10])
+    edge[2, v2, 3, 3] = -np.inf
+    edge[3, 0] = np.nan                      # root slot of tree 3 (root is node 0): not read
+    diag[3, 7, 0, 9] = np.nan                # upper triangle: not read
+    plan = selinv.TreePlan(P)
+    out = selinv.selinv_tree(plan, to_dev(diag, torch.float64), to_dev(edge, torch.float64), check=False,
+                             validate=True)
+    assert host(out["info"]).tolist() == [-1, -3 - 40, -3 - v2, -1]
+    with pytest.raises(selinv.NonFiniteInputError):
+        selinv.selinv_tree(plan, to_dev(diag, torch.float64), to_dev(edge, torch.float64), validate=True)
