@@ -444,16 +444,23 @@ SELINV_DEVINL void spd_inverse(Big<T> &a, T *colbuf, const Ctx<T, BP> &x, LogAcc
 // R_KK = chol(P), P being the Schur complement the step pivots on, and
 // R_iK = T_i R_KK for the rows below, so v_K += R_KK z_K and v_i += T_i (R_KK z_K).
 template <int BP, bool DRAW = false>
-SELINV_DEVINL void spd_inverse_blocked(Big<double> &a, double *cbuf, double *tbuf, const Ctx<double, BP> &x,
-                                       LogAcc &det, bool &bad, const double *zs = nullptr, double *vacc = nullptr)
+SELINV_DEVINL void spd_inverse_blocked(Big<double> &a, double *cbuf, double *tbuf, double *big_scratch,
+                                       const Ctx<double, BP> &x, LogAcc &det, bool &bad, const double *zs = nullptr,
+                                       double *vacc = nullptr)
 {
     constexpr int NB = BP / 8;
+    // The matrix stays symmetric through the sweep, so the warps holding a
+    // quadrant strictly above the diagonal (rw < cw) do no updates at all:
+    // their entries are read from the mirrored lower quadrants (the column
+    // block K for rows above quadrant row qK is published, transposed, from
+    // row block K), and their tiles are rebuilt from the lower ones at the end.
+    const bool upper = x.rw < x.cw;
     if (DRAW) vacc[0] = vacc[1] = vacc[2] = vacc[3] = 0.0;
     for (int K = 0; K < NB; ++K) {
         double *cb = cbuf + (K & 1) * BP * 8;                     // cb[r * 8 + c] = A[r][8K + c]
         double *tb = tbuf + (K & 1) * BP * 8;                     // tb[r * 8 + c] = T[r][c]
         const int qK = K >> 2, tK = K & 3;                        // quadrant and tile holding block K
-        if (x.cw == qK) {                                         // publish column block K
+        if (x.cw == qK && !upper) {                               // publish column block K (rows >= 32 qK)
 #pragma unroll
             for (int mi = 0; mi < 4; ++mi) {
 #pragma unroll
@@ -465,6 +472,16 @@ SELINV_DEVINL void spd_inverse_blocked(Big<double> &a, double *cbuf, double *tbu
                         *reinterpret_cast<double2 *>(cb + x.R(mi) * 8 + 2 * x.t) = u;
                     }
             }
+        }
+        if (x.rw == qK && x.cw < qK) {                            // rows above: A[c][8K + r] = A[8K + r][c]
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                if (m == tK) {
+#pragma unroll
+                    for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) cb[x.C(ni, j) * 8 + x.g] = a.v[m][ni][j];
+                }
         }
         __syncthreads();
         // P^-1 in registers (accumulator layout of one 8 x 8 tile; symmetric)
@@ -514,21 +531,19 @@ SELINV_DEVINL void spd_inverse_blocked(Big<double> &a, double *cbuf, double *tbu
             }
         }
         // rank-8 update A_ij -= T_i A_Kj, A_Kj = A_jK (symmetric): B fragments from cb
-        double bk[4][2];
-#pragma unroll
-        for (int ni = 0; ni < 4; ++ni) {
-            const double2 u = *reinterpret_cast<const double2 *>(cb + (32 * x.cw + 8 * ni + x.g) * 8 + 2 * x.t);
-            bk[ni][0] = u.x;
-            bk[ni][1] = u.y;
-        }
-#pragma unroll
-        for (int mi = 0; mi < 4; ++mi)
+        if (!upper) {
 #pragma unroll
             for (int ni = 0; ni < 4; ++ni) {
-                dmma_8x8x4(a.v[mi][ni][0], a.v[mi][ni][1], -T[mi][0], bk[ni][0]);
-                dmma_8x8x4(a.v[mi][ni][0], a.v[mi][ni][1], -T[mi][1], bk[ni][1]);
+                const double2 u =
+                    *reinterpret_cast<const double2 *>(cb + (32 * x.cw + 8 * ni + x.g) * 8 + 2 * x.t);
+#pragma unroll
+                for (int mi = 0; mi < 4; ++mi) {
+                    dmma_8x8x4(a.v[mi][ni][0], a.v[mi][ni][1], -T[mi][0], u.x);
+                    dmma_8x8x4(a.v[mi][ni][0], a.v[mi][ni][1], -T[mi][1], u.y);
+                }
             }
-        if (x.cw == qK) {                                         // column block K: T (rows outside K)
+        }
+        if (x.cw == qK && !upper) {                               // column block K: T (rows outside K)
 #pragma unroll
             for (int mi = 0; mi < 4; ++mi)
 #pragma unroll
@@ -539,7 +554,7 @@ SELINV_DEVINL void spd_inverse_blocked(Big<double> &a, double *cbuf, double *tbu
                     }
         }
         __syncthreads();                                          // T published
-        if (x.rw == qK) {                                         // row block K: T_j^T, diagonal block -P^-1
+        if (x.rw == qK && !upper) {                               // row block K: T_j^T, diagonal block -P^-1
 #pragma unroll
             for (int m = 0; m < 4; ++m)
                 if (m == tK) {
@@ -563,145 +578,18 @@ SELINV_DEVINL void spd_inverse_blocked(Big<double> &a, double *cbuf, double *tbu
     for (int mi = 0; mi < 4; ++mi)
 #pragma unroll
         for (int ni = 0; ni < 4; ++ni) a.v[mi][ni][0] = -a.v[mi][ni][0], a.v[mi][ni][1] = -a.v[mi][ni][1];
-}
-
-// The same block steps with look-ahead (float64, no draw): step K's owners
-// of column block K + 1 apply the rank-8 update to those tiles first and
-// publish them, so after the step's single barrier every warp inverts the
-// next pivot block P_{K+1} while it applies the rest of the update: the 8 x 8
-// sweep's shuffle chain overlaps the update's tensor-core work instead of
-// following it behind a barrier, and a step costs one barrier instead of
-// two.  Same pivots in the same order (so the same det), the same products.
-//   step K: T = A_{rows,K} P_K^-1 (P_K^-1 from the previous step); owners of
-//   column K+1: A_{., K+1} -= T A_{K, K+1}, published; barrier; everyone:
-//   P_{K+1}^-1 from the published column and the remaining updates; column K
-//   := T, row K := T^T, A_KK := -P_K^-1.
-// Buffers: the column block K is read before step K's barrier and rewritten
-// (as column K + 2) only after step K + 1's start, so two alternate; T alternates
-// likewise (written before a step's barrier, read after it).
-template <int BP>
-SELINV_DEVINL void spd_inverse_lookahead(Big<double> &a, double *cbuf, double *tbuf, const Ctx<double, BP> &x,
-                                         LogAcc &det, bool &bad)
-{
-    constexpr int NB = BP / 8;
-    if (x.cw == 0) {                                              // publish column block 0
+    // the upper quadrants from their mirrors, through the free resident image
+    if (!upper) to_smem<double, BP>(big_scratch, a, x);
+    __syncthreads();
+    if (upper) {
 #pragma unroll
-        for (int mi = 0; mi < 4; ++mi) {
-            double2 u;
-            u.x = a.v[mi][0][0];
-            u.y = a.v[mi][0][1];
-            *reinterpret_cast<double2 *>(cbuf + x.R(mi) * 8 + 2 * x.t) = u;
-        }
+        for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+            for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) a.v[mi][ni][j] = big_scratch[SW<double>::idx(x.C(ni, j), x.R(mi), BP)];
     }
     __syncthreads();
-    double pv[2];
-    {
-        const double2 u = *reinterpret_cast<const double2 *>(cbuf + x.g * 8 + 2 * x.t);
-        pv[0] = u.x;
-        pv[1] = u.y;
-    }
-    inv8_sweep(pv, x.lane, x.g, x.t, det, bad, x.tid == 0);
-    if (x.tid == 0) det.renorm();
-    for (int K = 0; K < NB; ++K) {
-        const double *cb = cbuf + (K & 1) * BP * 8;               // column block K
-        double *cn = cbuf + ((K + 1) & 1) * BP * 8;               // column block K + 1
-        double *tb = tbuf + (K & 1) * BP * 8;
-        const int qK = K >> 2, tK = K & 3;
-        const int K1 = K + 1, qK1 = K1 >> 2, tK1 = K1 & 3;
-        const bool next = K1 < NB;
-        // T = A_{rows,K} P^-1 for this warp's rows
-        double T[4][2];
-#pragma unroll
-        for (int mi = 0; mi < 4; ++mi) {
-            const double2 arow = *reinterpret_cast<const double2 *>(cb + x.R(mi) * 8 + 2 * x.t);
-            T[mi][0] = T[mi][1] = 0.0;
-            dmma_8x8x4(T[mi][0], T[mi][1], arow.x, pv[0]);
-            dmma_8x8x4(T[mi][0], T[mi][1], arow.y, pv[1]);
-        }
-        if (x.cw == 0) {                                          // publish T (one copy per row)
-#pragma unroll
-            for (int mi = 0; mi < 4; ++mi) {
-                double2 u;
-                u.x = T[mi][0];
-                u.y = T[mi][1];
-                *reinterpret_cast<double2 *>(tb + x.R(mi) * 8 + 2 * x.t) = u;
-            }
-        }
-        // A_Kj = A_jK for this warp's column tile ni (read where it is used)
-        auto bk = [&](int ni) {
-            return *reinterpret_cast<const double2 *>(cb + (32 * x.cw + 8 * ni + x.g) * 8 + 2 * x.t);
-        };
-        const bool own_next = next && x.cw == qK1;
-        if (own_next) {                                           // column block K + 1 first, published
-#pragma unroll
-            for (int n = 0; n < 4; ++n)
-                if (n == tK1) {
-                    const double2 bn = bk(n);
-#pragma unroll
-                    for (int mi = 0; mi < 4; ++mi) {
-                        dmma_8x8x4(a.v[mi][n][0], a.v[mi][n][1], -T[mi][0], bn.x);
-                        dmma_8x8x4(a.v[mi][n][0], a.v[mi][n][1], -T[mi][1], bn.y);
-                        double2 u;
-                        u.x = a.v[mi][n][0];
-                        u.y = a.v[mi][n][1];
-                        *reinterpret_cast<double2 *>(cn + x.R(mi) * 8 + 2 * x.t) = u;
-                    }
-                }
-        }
-        __syncthreads();                                          // T and column block K + 1 published
-        double pn[2] = {0.0, 0.0};
-        if (next) {                                               // P_{K+1}, inverted beside the update below
-            const double2 u = *reinterpret_cast<const double2 *>(cn + (8 * K1 + x.g) * 8 + 2 * x.t);
-            pn[0] = u.x;
-            pn[1] = u.y;
-            inv8_sweep(pn, x.lane, x.g, x.t, det, bad, x.tid == 0);
-        }
-#pragma unroll
-        for (int ni = 0; ni < 4; ++ni) {
-            if (own_next && ni == tK1) continue;                  // already updated
-            const double2 bn = bk(ni);
-#pragma unroll
-            for (int mi = 0; mi < 4; ++mi) {
-                dmma_8x8x4(a.v[mi][ni][0], a.v[mi][ni][1], -T[mi][0], bn.x);
-                dmma_8x8x4(a.v[mi][ni][0], a.v[mi][ni][1], -T[mi][1], bn.y);
-            }
-        }
-        if (x.cw == qK) {                                         // column block K: T (rows outside K)
-#pragma unroll
-            for (int mi = 0; mi < 4; ++mi)
-#pragma unroll
-                for (int n = 0; n < 4; ++n)
-                    if (n == tK) {
-                        a.v[mi][n][0] = T[mi][0];
-                        a.v[mi][n][1] = T[mi][1];
-                    }
-        }
-        if (x.rw == qK) {                                         // row block K: T_j^T, diagonal block -P^-1
-#pragma unroll
-            for (int m = 0; m < 4; ++m)
-                if (m == tK) {
-#pragma unroll
-                    for (int ni = 0; ni < 4; ++ni)
-#pragma unroll
-                        for (int j = 0; j < 2; ++j) a.v[m][ni][j] = tb[x.C(ni, j) * 8 + x.g];
-                    if (x.cw == qK) {
-#pragma unroll
-                        for (int n = 0; n < 4; ++n)
-                            if (n == tK) {
-                                a.v[m][n][0] = -pv[0];
-                                a.v[m][n][1] = -pv[1];
-                            }
-                    }
-                }
-        }
-        pv[0] = pn[0];
-        pv[1] = pn[1];
-        if (x.tid == 0) det.renorm();
-    }
-#pragma unroll
-    for (int mi = 0; mi < 4; ++mi)
-#pragma unroll
-        for (int ni = 0; ni < 4; ++ni) a.v[mi][ni][0] = -a.v[mi][ni][0], a.v[mi][ni][1] = -a.v[mi][ni][1];
 }
 
 // Row sums (over this thread's columns) of a tile times the vector v, reduced
@@ -797,7 +685,7 @@ __global__ void __launch_bounds__(Geo<BP>::NT) chain_large_kernel(ChainArgs<T> p
             // eta = A^-1 r + L^-T z.  R_i z_i comes out of the blocked inverse.
             if (x.tid < BP) zs[x.tid] = x.tid < b ? Zv[i * b + x.tid] : T(0);   // visible after its first barrier
             double vacc[4];
-            spd_inverse_blocked<BP, true>(a, pbuf, pbuf + 2 * BP * 8, x, det, bad, zs, vacc);
+            spd_inverse_blocked<BP, true>(a, pbuf, pbuf + 2 * BP * 8, big, x, det, bad, zs, vacc);
             if (x.cw == 0 && x.t == 0) {
 #pragma unroll
                 for (int mi = 0; mi < 4; ++mi) {
@@ -808,7 +696,7 @@ __global__ void __launch_bounds__(Geo<BP>::NT) chain_large_kernel(ChainArgs<T> p
                 }
             }
         } else if constexpr (sizeof(T) == 8) {
-            spd_inverse_lookahead<BP>(a, pbuf, pbuf + 2 * BP * 8, x, det, bad);
+            spd_inverse_blocked<BP>(a, pbuf, pbuf + 2 * BP * 8, big, x, det, bad);
         } else {
             spd_inverse<T, BP>(a, colbuf, x, det, bad);
         }

@@ -46,6 +46,8 @@ constexpr int WARPS = 4;
 #ifndef SELINV_L2MODE
 #define SELINV_L2MODE 3
 #endif
+
+constexpr int WS_ELEMS = w16::SLOT_ELEMS;   // workspace per block: the S_i^-1 slot
 #ifndef SELINV_L2KEEP
 #define SELINV_L2KEEP 64
 #endif
@@ -82,7 +84,7 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
     const int64_t bb = (int64_t)b * b;
     const T *D = p.diag + e * L * bb;
     const T *Bl = p.lower + e * (L - 1) * bb;
-    T *ws = (WANT_G || WANT_X) ? p.ws + e * (L - 1) * SLOT_ELEMS : nullptr;
+    T *ws = (WANT_G || WANT_X) ? p.ws + e * (L - 1) * WS_ELEMS : nullptr;
     const T *R = (WANT_X && p.rhs) ? p.rhs + e * L * b : nullptr;   // a draw may come without a mean
     T *X = WANT_X ? p.x + e * L * b : nullptr;
     const T *Zv = SAMPLE ? p.z + e * L * b : nullptr;
@@ -165,10 +167,10 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
 
         if (WANT_G || WANT_X) {
             if (HINT && SELINV_L2MODE == 2)
-                store_lower_slot<T, true>(ws + i * SLOT_ELEMS, a, lane, g, t,
+                store_lower_slot<T, true>(ws + i * WS_ELEMS, a, lane, g, t,
                                           L - 1 - i <= SELINV_L2KEEP ? pol_keep : pol_first);
             else
-                store_lower_slot<T>(ws + i * SLOT_ELEMS, a, lane, g, t);
+                store_lower_slot<T>(ws + i * WS_ELEMS, a, lane, g, t);
         }
         cp_async_wait_all();
         __syncwarp();
@@ -249,7 +251,7 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
     __syncwarp();
     if (L > 1) {
         load_block_async<T, FULL, HINT>(sB, Bl + (L - 2) * bb, b, lane, pol_first);
-        stage_lower_slot<T, HINT>(stg, ws + (L - 2) * SLOT_ELEMS, lane, g, t, pol_first);
+        stage_lower_slot<T, HINT>(stg, ws + (L - 2) * WS_ELEMS, lane, g, t, pol_first);
         cp_async_commit();
     }
 
@@ -262,7 +264,7 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
         for (int q = 0; q < 4; ++q) yi[q] = yc[q];
         cp_async_wait_all();
         unstage_lower_slot<T>(a, stg, lane, g, t);
-        if (drop) discard_slot<T>(ws + i * SLOT_ELEMS, lane);   // dead once staged
+        if (drop) discard_slot<T>(ws + i * WS_ELEMS, lane);   // dead once staged
         to_smem<T>(sT, a, g, t);                      // lower entries valid
         __syncwarp();
         from_smem_lower<T>(a, sT, g, t);              // S_i^-1, full and symmetric
@@ -270,7 +272,7 @@ __global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_ker
         __syncwarp();
         if (i > 0) {
             load_block_async<T, FULL, HINT>(sB, Bl + (i - 1) * bb, b, lane, pol_first);
-            stage_lower_slot<T, HINT>(stg, ws + (i - 1) * SLOT_ELEMS, lane, g, t, pol_first);
+            stage_lower_slot<T, HINT>(stg, ws + (i - 1) * WS_ELEMS, lane, g, t, pol_first);
             cp_async_commit();
             if (WANT_X) {
 #pragma unroll
@@ -496,7 +498,7 @@ cudaError_t launch_full(const ChainArgs<T> &a, cudaStream_t s)
 
 size_t chain_small_workspace(size_t elem, int64_t batch, int64_t L)
 {
-    return (size_t)batch * (size_t)(L > 1 ? L - 1 : 0) * w16::SLOT_ELEMS * elem;
+    return (size_t)batch * (size_t)(L > 1 ? L - 1 : 0) * WS_ELEMS * elem;
 }
 
 template <class T> cudaError_t chain_small_launch(const ChainArgs<T> &a, bool aligned16, cudaStream_t s)

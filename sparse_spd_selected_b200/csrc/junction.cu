@@ -32,6 +32,7 @@
 #include <cmath>
 #include <map>
 #include <memory>
+#include <mutex>
 #include <new>
 #include <set>
 #include <unordered_map>
@@ -59,6 +60,21 @@ struct selinv_junction_plan_s {
     std::vector<int64_t> ct_off, ce_off, de_off;
     int32_t *d_ct_node = nullptr, *d_ct_t = nullptr, *d_ce_ent = nullptr, *d_ce_node = nullptr;
     int32_t *d_de_ent = nullptr, *d_de_node = nullptr, *d_de_a = nullptr;
+    // One call is a few launches per elimination level (thousands on a lattice),
+    // each doing little work, so the sequence is recorded once as a CUDA graph
+    // per set of arguments and replayed: the graph's kernel nodes carry the
+    // pointers, so a call with the same buffers (new values in them) replays it.
+    struct Graph {
+        int dtype = -1, b = 0;
+        int64_t batch = 0;
+        const void *ptr[7] = {};           // diag, edge, G_diag, G_lower, logdet, info, workspace
+        cudaGraphExec_t exec = nullptr;
+        uint64_t used = 0;
+    };
+    std::vector<Graph> graphs;                  // at most GRAPH_CACHE entries, least recently used replaced
+    cudaStream_t capture = nullptr;             // non-blocking stream the graphs are recorded on
+    uint64_t calls = 0;
+    std::mutex mu;
 };
 
 namespace selinv {
@@ -537,16 +553,9 @@ cudaError_t run_junction(const selinv_junction_plan_s *pl, int b, int64_t batch,
     JDev jd{pl->d_col_ptr, pl->d_ent_slot, pl->d_ent_trans, pl->d_ent_src, pl->d_con_ptr, pl->d_con_w,
             pl->d_con_a, pl->d_pair_ptr, pl->d_pair, pl->n, pl->m, pl->nnz, pl->E};
     const unsigned ib = (unsigned)ceil_div(batch, 256);
-    junction_init<<<ib, 256, 0, s>>>(info, batch);
     const size_t smem_r = sizeof(T) * j_smem_elems<T, Pol>();      // CTA-per-item kernels
     const size_t smem_w = sizeof(T) * JWARPS * 2 * Pol::IMG, smem_i = sizeof(T) * JWARPS * 32;
-    cudaError_t err = cudaSuccess;
-    for (auto k : {(const void *)jn_target_kernel<T, Pol>, (const void *)jn_gcol_kernel<T, Pol>,
-                   (const void *)jn_gdiag_kernel<T, Pol>})
-        if (err == cudaSuccess) err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_r);
-    if (err == cudaSuccess)
-        err = cudaFuncSetAttribute(jn_w_kernel<T, Pol>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_w);
-    if (err != cudaSuccess) return err;
+    junction_init<<<ib, 256, 0, s>>>(info, batch);
     for (size_t l = 0; l + 1 < pl->c_off.size(); ++l) {
         const int64_t nt = pl->ct_off[l + 1] - pl->ct_off[l];
         const int64_t nn = pl->c_off[l + 1] - pl->c_off[l];
@@ -572,6 +581,77 @@ cudaError_t run_junction(const selinv_junction_plan_s *pl, int b, int64_t batch,
     return cudaGetLastError();
 }
 
+// Shared-memory limits of the kernels run_junction launches (set before a
+// capture: attribute calls are not stream work).
+template <class T, class Pol> cudaError_t junction_attributes()
+{
+    const size_t smem_r = sizeof(T) * j_smem_elems<T, Pol>();
+    const size_t smem_w = sizeof(T) * JWARPS * 2 * Pol::IMG;
+    cudaError_t err = cudaSuccess;
+    for (auto k : {(const void *)jn_target_kernel<T, Pol>, (const void *)jn_gcol_kernel<T, Pol>,
+                   (const void *)jn_gdiag_kernel<T, Pol>})
+        if (err == cudaSuccess) err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_r);
+    if (err == cudaSuccess)
+        err = cudaFuncSetAttribute(jn_w_kernel<T, Pol>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_w);
+    return err;
+}
+
+constexpr size_t GRAPH_CACHE = 4;
+
+// Launch one call through the plan's graph cache: replay the graph recorded
+// for these arguments, or record it (on the plan's own capture stream, so the
+// caller's stream may be any stream, the legacy default one included) and
+// replay it.  A caller whose stream is itself being captured gets the
+// launches directly, inside its own graph.
+template <class T, class Pol>
+cudaError_t junction_call(selinv_junction_plan_s *pl, int dtype, int b, int64_t batch, const T *diag, const T *edge,
+                          T *G_diag, T *G_lower, double *logdet, int32_t *info, void *ws, cudaStream_t s)
+{
+    cudaError_t err = junction_attributes<T, Pol>();
+    if (err != cudaSuccess) return err;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone)
+        return run_junction<T, Pol>(pl, b, batch, diag, edge, G_diag, G_lower, logdet, info, ws, s);
+    const void *key[7] = {diag, edge, G_diag, G_lower, logdet, info, ws};
+    std::lock_guard<std::mutex> lock(pl->mu);
+    ++pl->calls;
+    for (auto &g : pl->graphs)
+        if (g.dtype == dtype && g.b == b && g.batch == batch && std::equal(key, key + 7, g.ptr)) {
+            g.used = pl->calls;
+            return cudaGraphLaunch(g.exec, s);
+        }
+    if (!pl->capture && (err = cudaStreamCreateWithFlags(&pl->capture, cudaStreamNonBlocking)) != cudaSuccess)
+        return err;
+    if ((err = cudaStreamBeginCapture(pl->capture, cudaStreamCaptureModeThreadLocal)) != cudaSuccess) return err;
+    cudaError_t run = run_junction<T, Pol>(pl, b, batch, diag, edge, G_diag, G_lower, logdet, info, ws, pl->capture);
+    cudaGraph_t graph = nullptr;
+    err = cudaStreamEndCapture(pl->capture, &graph);
+    if (run != cudaSuccess || err != cudaSuccess) {
+        if (graph) cudaGraphDestroy(graph);
+        cudaGetLastError();
+        return run != cudaSuccess ? run : err;
+    }
+    cudaGraphExec_t exec = nullptr;
+    err = cudaGraphInstantiate(&exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (err != cudaSuccess) return err;
+    if (pl->graphs.size() >= GRAPH_CACHE) {                 // replace the least recently used
+        auto old = std::min_element(pl->graphs.begin(), pl->graphs.end(),
+                                    [](const auto &x, const auto &y) { return x.used < y.used; });
+        cudaGraphExecDestroy(old->exec);
+        pl->graphs.erase(old);
+    }
+    selinv_junction_plan_s::Graph g;
+    g.dtype = dtype;
+    g.b = b;
+    g.batch = batch;
+    std::copy(key, key + 7, g.ptr);
+    g.exec = exec;
+    g.used = pl->calls;
+    pl->graphs.push_back(g);
+    return cudaGraphLaunch(exec, s);
+}
+
 bool is_aligned(const void *q, size_t a) { return (reinterpret_cast<uintptr_t>(q) % a) == 0; }
 
 }  // namespace
@@ -588,6 +668,8 @@ void selinv_junction_plan_free(selinv_junction_plan_t *pl)
     int32_t *arrs[] = {pl->d_c_nodes, pl->d_d_nodes, pl->d_col_ptr, pl->d_ent_slot, pl->d_ent_trans, pl->d_ent_src,
                        pl->d_con_ptr, pl->d_con_w, pl->d_con_a, pl->d_pair_ptr, pl->d_pair, pl->d_ct_node,
                        pl->d_ct_t, pl->d_ce_ent, pl->d_ce_node, pl->d_de_ent, pl->d_de_node, pl->d_de_a};
+    for (auto &g : pl->graphs) cudaGraphExecDestroy(g.exec);   // a launch in flight is freed on completion
+    if (pl->capture) cudaStreamDestroy(pl->capture);
     for (int32_t *a : arrs) cudaFree(a);
     delete pl;
 }
@@ -982,12 +1064,14 @@ selinv_status selinv_junction(const selinv_junction_plan_t *pl, selinv_dtype dty
     const float *fd = static_cast<const float *>(diag), *fe = static_cast<const float *>(edge_val);
     double *dg = static_cast<double *>(G_diag), *dl = static_cast<double *>(G_lower);
     float *fg = static_cast<float *>(G_diag), *fl = static_cast<float *>(G_lower);
+    auto *mp = const_cast<selinv_junction_plan_s *>(pl);      // the graph cache is the plan's own mutable state
+    const int dt = (int)dtype;
     if (dtype == SELINV_F64)
-        err = b <= 8 ? run_junction<double, Pol8<double>>(pl, b, batch, dd, de, dg, dl, logdet, info, workspace, s)
-                     : run_junction<double, Pol16<double>>(pl, b, batch, dd, de, dg, dl, logdet, info, workspace, s);
+        err = b <= 8 ? junction_call<double, Pol8<double>>(mp, dt, b, batch, dd, de, dg, dl, logdet, info, workspace, s)
+                     : junction_call<double, Pol16<double>>(mp, dt, b, batch, dd, de, dg, dl, logdet, info, workspace, s);
     else
-        err = b <= 8 ? run_junction<float, Pol8<float>>(pl, b, batch, fd, fe, fg, fl, logdet, info, workspace, s)
-                     : run_junction<float, Pol16<float>>(pl, b, batch, fd, fe, fg, fl, logdet, info, workspace, s);
+        err = b <= 8 ? junction_call<float, Pol8<float>>(mp, dt, b, batch, fd, fe, fg, fl, logdet, info, workspace, s)
+                     : junction_call<float, Pol16<float>>(mp, dt, b, batch, fd, fe, fg, fl, logdet, info, workspace, s);
     return err == cudaSuccess ? SELINV_OK : SELINV_ERR_CUDA;
 }
 

@@ -130,3 +130,49 @@ def test_junction_lattice_benchmark_size(cuda_ok):
     assert worst(Gd[e][None], ref_d[None]) <= 1e-9
     assert worst(Gl[e][None], ref_l[None]) <= 1e-9
     assert logdet_err(host(out["logdet"])[e], np.linalg.slogdet(A)[1]) <= 1e-9
+
+
+def test_junction_graph_replay_reads_new_values(cuda_ok):
+    """Calls with the same buffers replay the launch sequence recorded by the
+    first one (the plan's graph cache): new values written into those buffers
+    give the new matrices' results; other buffers, another batch size or
+    another block size record their own; a replay inside the caller's own
+    stream capture still works."""
+    E = inputs.grid_edges(6, 6)
+    n, b = 36, 8
+    plan = selinv.JunctionPlan(n, E)
+    d1, e1 = inputs.graph_inputs(3, n, b, E, seed=11700, load=1.0)
+    d2, e2 = inputs.graph_inputs(3, n, b, E, seed=11701, load=1.0)
+    dd, ee = to_dev(d1, torch.float64), to_dev(e1, torch.float64)
+    out = {"G_diag": torch.empty_like(dd), "G_lower": torch.empty((3, plan.nnz, b, b), dtype=torch.float64, device="cuda"),
+           "logdet": torch.empty(3, dtype=torch.float64, device="cuda"),
+           "info": torch.empty(3, dtype=torch.int32, device="cuda")}
+    ws = torch.empty(plan.workspace_size(torch.float64, b, 3), dtype=torch.uint8, device="cuda")
+    for d, e in ((d1, e1), (d2, e2), (d1, e1)):
+        dd.copy_(to_dev(d, torch.float64))
+        ee.copy_(to_dev(e, torch.float64))
+        r = selinv.junction(plan, dd, ee, out=out, workspace=ws)
+        ref = oracle.junction(d, E, e)
+        assert worst(host(r["G_diag"]), ref["G_diag"]) <= 1e-9
+        assert worst(host(r["G_lower"]), ref["G_lower"]) <= 1e-9
+        assert logdet_err(host(r["logdet"]), ref["logdet"]) <= 1e-9
+    fresh = selinv.junction(plan, dd, ee)                          # other buffers: its own recording
+    assert torch.equal(fresh["G_diag"], out["G_diag"]) and torch.equal(fresh["G_lower"], out["G_lower"])
+    one = selinv.junction(plan, dd[:1].contiguous(), ee[:1].contiguous())   # another batch size
+    assert torch.equal(one["G_diag"], out["G_diag"][:1])
+    d5, e5 = inputs.graph_inputs(2, n, 5, E, seed=11702, load=1.0)  # another block size
+    r5 = selinv.junction(plan, to_dev(d5, torch.float64), to_dev(e5, torch.float64))
+    assert worst(host(r5["G_diag"]), oracle.junction(d5, E, e5)["G_diag"]) <= 1e-9
+    # inside the caller's own capture the launches go straight into that graph
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        selinv.junction(plan, dd, ee, check=False, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=s):
+        selinv.junction(plan, dd, ee, check=False, out=out, workspace=ws)
+    out["G_diag"].zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out["G_diag"], fresh["G_diag"])
