@@ -14,7 +14,8 @@ selected inverse ("Differentiable selected inverse", written from the dense
 definition Ab = -A^-1 Gbar A^-1), the block lower-bidiagonal non-symmetric
 case and its cotangents ("Non-symmetric selected inverse"), and general
 block-sparse SPD patterns ("General sparse selected inverse": its own
-minimum-degree symbolic elimination, then the dense inverse read on the fill).
+minimum-degree symbolic elimination, then the dense inverse read on the fill,
+and its solve x = A^-1 r).
 The C file states each recursion or definition and every reading taken where
 the pages are silent.
 """
@@ -349,6 +350,47 @@ def junction(diag, edge_index, edge_val, order=None, lib=None):
     return {"G_diag": G_diag.reshape(lead + (n, b, b)), "S_index": S,
             "G_lower": G_lower.reshape(lead + (S.shape[1], b, b)), "logdet": logdet.reshape(lead),
             "info": info.reshape(lead)}
+
+
+def junction_solve(diag, edge_index, edge_val, rhs, lib=None):
+    """x = A^-1 r for general block-sparse SPD matrices (gabp-sparse-inv,
+    "General sparse selected inverse": junction_solve from the same
+    factorisation), written from the definition: the dense matrix assembled
+    as in ``junction`` (D_v read on its lower triangle, A_{i,j} = edge_val[k]
+    at (i, j) and transposed at (j, i)), its dense inverse by the textbook
+    Cholesky route, times r.  diag [..., n, b, b], edge_val [..., m, b, b],
+    rhs [..., n, b].  Returns dict with x [..., n, b], logdet, info (-1, or
+    the node holding the first failing pivot in natural order)."""
+    diag, edge_val, rhs = _f64(diag), _f64(edge_val), _f64(rhs)
+    lead = diag.shape[:-3]
+    n, b = diag.shape[-3], diag.shape[-1]
+    ei = np.asarray(edge_index[0], dtype=np.int64)
+    ej = np.asarray(edge_index[1], dtype=np.int64)
+    batch = int(np.prod(lead)) if lead else 1
+    d2 = diag.reshape(batch, n, b, b)
+    e2 = edge_val.reshape(batch, len(ei), b, b)
+    r2 = rhs.reshape(batch, n * b)
+    x = np.zeros((batch, n * b))
+    logdet = np.zeros(batch)
+    info = np.full(batch, -1, dtype=np.int32)
+    N = n * b
+    for e in range(batch):
+        A = np.zeros((N, N))
+        for v in range(n):
+            A[v * b:(v + 1) * b, v * b:(v + 1) * b] = np.tril(d2[e, v]) + np.tril(d2[e, v], -1).T
+        for k, (i, j) in enumerate(zip(ei, ej)):
+            A[i * b:(i + 1) * b, j * b:(j + 1) * b] = e2[e, k]
+            A[j * b:(j + 1) * b, i * b:(i + 1) * b] = e2[e, k].T
+        A = np.ascontiguousarray(A)
+        inv = np.empty((N, N))
+        ld = np.zeros(1)
+        rc = _load(lib).oracle_spd_inverse(_ptr(A), N, _ptr(inv), _ptr(ld))
+        if rc != 0:
+            info[e] = (rc - 1) // b
+            continue
+        logdet[e] = ld[0]
+        x[e] = inv @ r2[e]
+    return {"x": x.reshape(lead + (n, b)), "logdet": logdet.reshape(lead), "info": info.reshape(lead)}
 
 
 def junction_backward(diag, edge_index, edge_val, Gb_diag, Gb_lower, order=None, lib=None):

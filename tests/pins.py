@@ -778,6 +778,43 @@ def pin_junction_backward_path_is_chain(lib=None):
     return max(rel(jb["Db"], cb["Db"]), rel(jb["Eb"], cb["Bb"]))
 
 
+def pin_junction_solve(lib=None):
+    """The general sparse solve x = A^-1 r: on a path pattern (pairs (i + 1,
+    i)) it is the (pinned) chain oracle's solve; without edges each block row
+    is its own system, x_v = D_v^-1 r_v (numpy's solve of each symmetric
+    D_v); on a random pattern the block residual sum_u A_vu x_u - r_v
+    vanishes and log det equals the (pinned) selected inverse's."""
+    worst = 0.0
+    L, b = 7, 3
+    cd, cl, cr = inputs.chain_inputs(2, L, b, seed=83, load=1.0)
+    P = np.array([np.arange(1, L), np.arange(L - 1)])
+    js = oracle.junction_solve(cd, P, cl, cr, lib=lib)
+    ch = oracle.chain(cd, cl, cr, want_g=False, lib=lib)
+    worst = max(worst, rel(js["x"], ch["x"]), float(np.max(np.abs(js["logdet"] - ch["logdet"]))))
+    n = 5
+    d, e = inputs.graph_inputs(1, n, b, np.zeros((2, 0), dtype=np.int64), seed=84, load=1.0)
+    r = np.random.default_rng(84).standard_normal((1, n, b))
+    js = oracle.junction_solve(d, np.zeros((2, 0), dtype=np.int64), e, r, lib=lib)
+    for v in range(n):
+        Dv = np.tril(d[0, v]) + np.tril(d[0, v], -1).T
+        worst = max(worst, rel(js["x"][0, v], np.linalg.solve(Dv, r[0, v])))
+    n, m = 12, 25
+    rng = np.random.default_rng(85)
+    pairs = sorted({(max(a, c), min(a, c)) for a, c in rng.integers(0, n, (m, 2)) if a != c})
+    E = np.array(pairs, dtype=np.int64).T
+    d, e = inputs.graph_inputs(2, n, b, E, seed=85, load=1.0)
+    r = rng.standard_normal((2, n, b))
+    js = oracle.junction_solve(d, E, e, r, lib=lib)
+    full = oracle.junction(d, E, e, lib=lib)
+    for k in range(2):
+        res = np.einsum("vab,vb->va", np.tril(d[k]) + np.swapaxes(np.tril(d[k], -1), -1, -2), js["x"][k]) - r[k]
+        np.add.at(res, E[0], np.einsum("kab,kb->ka", e[k], js["x"][k][E[1]]))
+        np.add.at(res, E[1], np.einsum("kba,kb->ka", e[k], js["x"][k][E[0]]))
+        worst = max(worst, float(np.linalg.norm(res) / np.linalg.norm(r[k])))
+    worst = max(worst, float(np.max(np.abs(js["logdet"] - full["logdet"]))))
+    return worst
+
+
 # name -> (function, tolerance)
 PINS = {
     "tiny_chains_dense": (pin_tiny_chains_dense, 1e-12),
@@ -809,4 +846,5 @@ PINS = {
     "junction_tree_and_order": (pin_junction_tree_and_order, 1e-12),
     "junction_backward_finite_differences": (pin_junction_backward_finite_differences, 1e-7),
     "junction_backward_path_is_chain": (pin_junction_backward_path_is_chain, 1e-12),
+    "junction_solve": (pin_junction_solve, 1e-11),
 }
