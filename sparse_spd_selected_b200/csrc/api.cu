@@ -53,6 +53,9 @@ selinv_status run_chain(int64_t batch, int64_t L, int32_t b, const void *diag, c
     a.batch = batch;
     a.L = L;
     a.b = b;
+    if constexpr (std::is_same<T, double>::value) {
+        if (chain_tiny_fits(L, b)) return from_cuda(chain_tiny_launch(a, s));
+    }
     if (b <= 16) {
         const bool al = aligned(diag, 16) && aligned(lower, 16) && aligned(G_diag, 16) &&
                         aligned(G_lower, 16) && aligned(ws, 16);

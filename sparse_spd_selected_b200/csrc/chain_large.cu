@@ -485,26 +485,28 @@ SELINV_DEVINL void spd_inverse_blocked(Big<double> &a, double *cbuf, double *tbu
         }
         __syncthreads();
         // P^-1 in registers (accumulator layout of one 8 x 8 tile; symmetric)
-        double pv[2];
-        {
-            const double2 u = *reinterpret_cast<const double2 *>(cb + (8 * K + x.g) * 8 + 2 * x.t);
-            pv[0] = u.x;
-            pv[1] = u.y;
-        }
+        // the warps above the diagonal need neither P^-1 nor T: only the barriers
+        double pv[2] = {0.0, 0.0};
+        double T[4][2] = {};
         double wk = 0.0;                                          // (R_KK z_K) at row 8K + g
-        if (DRAW && x.cw == 0)
-            inv8_sweep<true>(pv, x.lane, x.g, x.t, det, bad, x.tid == 0, zs[8 * K + 2 * x.t],
-                             zs[8 * K + 2 * x.t + 1], &wk);
-        else
-            inv8_sweep(pv, x.lane, x.g, x.t, det, bad, x.tid == 0);
-        // T = A_{rows,K} P^-1 for this warp's rows: 4 m-tiles x 2 k-steps
-        double T[4][2];
+        if (!upper) {
+            {
+                const double2 u = *reinterpret_cast<const double2 *>(cb + (8 * K + x.g) * 8 + 2 * x.t);
+                pv[0] = u.x;
+                pv[1] = u.y;
+            }
+            if (DRAW && x.cw == 0)
+                inv8_sweep<true>(pv, x.lane, x.g, x.t, det, bad, x.tid == 0, zs[8 * K + 2 * x.t],
+                                 zs[8 * K + 2 * x.t + 1], &wk);
+            else
+                inv8_sweep(pv, x.lane, x.g, x.t, det, bad, x.tid == 0);
+            // T = A_{rows,K} P^-1 for this warp's rows: 4 m-tiles x 2 k-steps
 #pragma unroll
-        for (int mi = 0; mi < 4; ++mi) {
-            const double2 arow = *reinterpret_cast<const double2 *>(cb + x.R(mi) * 8 + 2 * x.t);
-            T[mi][0] = T[mi][1] = 0.0;
-            dmma_8x8x4(T[mi][0], T[mi][1], arow.x, pv[0]);
-            dmma_8x8x4(T[mi][0], T[mi][1], arow.y, pv[1]);
+            for (int mi = 0; mi < 4; ++mi) {
+                const double2 arow = *reinterpret_cast<const double2 *>(cb + x.R(mi) * 8 + 2 * x.t);
+                dmma_8x8x4(T[mi][0], T[mi][1], arow.x, pv[0]);
+                dmma_8x8x4(T[mi][0], T[mi][1], arow.y, pv[1]);
+            }
         }
         if (DRAW && x.cw == 0) {                                  // v at this warp's rows
             const double w0 = shfl(wk, (2 * x.t) << 2), w1 = shfl(wk, (2 * x.t + 1) << 2);

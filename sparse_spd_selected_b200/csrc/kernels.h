@@ -35,6 +35,11 @@ template <class T> cudaError_t chain_small_multi_launch(const ChainArgs<T> &a, b
 // The same kernel drawing eta = A^-1 rhs + L^-T z into a.x (rhs may be null; no G).
 template <class T> cudaError_t chain_small_sample_launch(const ChainArgs<T> &a, bool aligned16, cudaStream_t s);
 
+// Short chains with small blocks (float64, b <= 8, L <= 16): one warp per
+// chain, the chain held in shared memory, 8 x 8 tiles; no workspace.
+bool chain_tiny_fits(int64_t L, int b);
+cudaError_t chain_tiny_launch(const ChainArgs<double> &a, cudaStream_t s);
+
 // 16 < b <= 32, no right-hand side: one CTA of two 4-warp groups per chain,
 // eliminating from both ends toward the middle block.
 size_t chain_mid_workspace(size_t elem, int64_t batch, int64_t L);

@@ -359,3 +359,31 @@ def test_validate_reports_non_finite_inputs(cuda_ok, b):
         selinv.selinv_chain(d, l, r, validate=True)
     clean = selinv.selinv_chain(d[[0, 4]], l[[0, 4]], r[[0, 4]], validate=True)
     assert (host(clean["info"]) == -1).all()
+
+
+@pytest.mark.parametrize("b", [1, 3, 4, 7, 8])
+@pytest.mark.parametrize("L", [1, 2, 8, 16])
+def test_short_chains_of_small_blocks(cuda_ok, b, L):
+    """float64, b <= 8, L <= 16: the shared-memory kernel with 8 x 8 tiles.
+    Against the oracle; the solve-only and log-det-only calls agree with the
+    full one; the upper triangle of D is not read; a failing block is named."""
+    diag, lower, rhs = inputs.chain_inputs(6, L, b, seed=3600 + 10 * b + L, load=0.5)
+    errs, full = run_both(diag, lower, rhs, torch.float64)
+    assert max(errs.values()) <= TOL[torch.float64], errs
+    d, l, r = (to_dev(a, torch.float64) for a in (diag, lower, rhs))
+    x, ld, _ = selinv.chain_solve(d, l, r)
+    assert torch.equal(x, full["x"]) and torch.equal(ld, full["logdet"])
+    only = selinv.selinv_chain(d, l, None, want_g=False)
+    assert torch.equal(only["logdet"], full["logdet"])
+    junk = d.clone()
+    if b > 1:
+        iu = torch.triu_indices(b, b, 1)
+        junk[..., iu[0], iu[1]] = float("nan")
+    again = selinv.selinv_chain(junk, l, r)
+    for k in ("G_diag", "G_lower", "logdet", "x"):
+        assert torch.equal(again[k], full[k]), k
+    bad = diag.copy()
+    bad[2, L - 1] = -np.eye(b)
+    out = selinv.selinv_chain(to_dev(bad, torch.float64), l, check=False)
+    info = host(out["info"]).tolist()
+    assert info[2] == L - 1 and all(v == -1 for k, v in enumerate(info) if k != 2)
