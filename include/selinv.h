@@ -323,6 +323,13 @@ selinv_status selinv_chain_noalloc(selinv_dtype dtype, int64_t batch, int64_t L,
  * Workspace: selinv_junction_workspace_size(plan, dtype, b, batch) bytes.
  * Each level of the collect is three launches (target blocks, inverses,
  * W products), each level of the distribute two (clique columns, diagonals).
+ * The first call with a given set of arguments (pointers, batch, b, dtype)
+ * records that launch sequence as a CUDA graph held by the plan (up to four,
+ * least recently used replaced, on a stream the plan creates for recording)
+ * and every call replays it on `stream`, so a call whose buffers hold new
+ * values replays the same graph; a call made while `stream` is itself being
+ * captured launches the kernels directly into that capture.  The plan's
+ * lock serialises the host side of concurrent calls on one plan.
  */
 typedef struct selinv_junction_plan_s selinv_junction_plan_t;
 
@@ -349,6 +356,24 @@ selinv_status selinv_junction(const selinv_junction_plan_t *plan, selinv_dtype d
                               const void *diag, const void *edge_val, void *G_diag, void *G_lower,
                               double *logdet, int32_t *info, void *workspace, size_t workspace_bytes,
                               void *stream);
+
+/*
+ * Solve x = A^-1 r for `batch` general block-sparse SPD matrices on the
+ * plan's pattern, from the same factorisation (gabp-sparse-inv, "General
+ * sparse selected inverse": junction_solve).  With W_{u,v} = A'_{u,v} S_v^-1
+ * for u in N(v), the factor is unit lower in elimination order and
+ *   z_v = r_v - sum_{k: v in N(k)} W_{v,k} z_k      (children first)
+ *   x_v = S_v^-1 z_v - sum_{u in N(v)} W_{u,v}^T x_u  (parents first).
+ *   diag, edge_val  as in selinv_junction
+ *   rhs [batch, n, b]  r;  x [batch, n, b] out (must not alias rhs)
+ *   logdet [batch] (may be NULL), info [batch] as in selinv_junction
+ * Workspace: selinv_junction_workspace_size(plan, dtype, b, batch) bytes.
+ * Same launch sequence caching as selinv_junction (keyed on rhs and x too).
+ */
+selinv_status selinv_junction_solve(const selinv_junction_plan_t *plan, selinv_dtype dtype, int32_t b,
+                                    int64_t batch, const void *diag, const void *edge_val, const void *rhs,
+                                    void *x, double *logdet, int32_t *info, void *workspace,
+                                    size_t workspace_bytes, void *stream);
 
 /*
  * Tree plan: validates `trees` parent arrays of n nodes each (HOST memory,

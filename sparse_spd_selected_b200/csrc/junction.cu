@@ -60,6 +60,7 @@ struct selinv_junction_plan_s {
     std::vector<int64_t> ct_off, ce_off, de_off;
     int32_t *d_ct_node = nullptr, *d_ct_t = nullptr, *d_ce_ent = nullptr, *d_ce_node = nullptr;
     int32_t *d_de_ent = nullptr, *d_de_node = nullptr, *d_de_a = nullptr;
+    int32_t *d_ent_owner = nullptr, *d_ent_u = nullptr;   // [E] node v of entry (u, v) and its u (solve)
     // One call is a few launches per elimination level (thousands on a lattice),
     // each doing little work, so the sequence is recorded once as a CUDA graph
     // per set of arguments and replayed: the graph's kernel nodes carry the
@@ -67,7 +68,7 @@ struct selinv_junction_plan_s {
     struct Graph {
         int dtype = -1, b = 0;
         int64_t batch = 0;
-        const void *ptr[7] = {};           // diag, edge, G_diag, G_lower, logdet, info, workspace
+        const void *ptr[9] = {};           // diag, edge, G_diag, G_lower, logdet, info, workspace, rhs, x
         cudaGraphExec_t exec = nullptr;
         uint64_t used = 0;
     };
@@ -505,6 +506,121 @@ jn_gdiag_kernel(JBufs<T> p, JDev jd, const int32_t *nodes, int64_t count)
     Pol::st_blk(p.G_diag + (e * jd.n + v) * bb, acc, b, g, t, false);
 }
 
+// The solve x = A^-1 r from the same factorisation (gabp-sparse-inv, "General
+// sparse selected inverse": junction_solve).  With L_{u,v} = W_{u,v} for u in
+// N(v) (unit lower in elimination order) and S_v the pivots, A = L diag(S) L^T:
+//   forward, children first:  z_v = r_v - sum_{k : v in N(k)} W_{v,k} z_k
+//   backward, parents first:  x_v = S_v^-1 z_v - sum_{u in N(v)} W_{u,v}^T x_u
+// The k with v in N(k) are exactly the contributions of v's diagonal target
+// in the collect, and N(v) its clique entries; z lives in x until the
+// backward pass overwrites it.  One warp per node and matrix.
+template <class T, class Pol> struct VecOps {
+    static constexpr int RH = Pol::DIM == 16 ? 2 : 1;       // rows per lane
+    static constexpr int CQ = Pol::DIM == 16 ? 4 : 2;       // columns per lane
+    static SELINV_DEVINL int col(int t, int q) { return Pol::DIM == 16 ? w16::tcol(t, q) : 2 * t + q; }
+    static SELINV_DEVINL T at(const typename Pol::Tile &a, int h, int q)
+    {
+        if constexpr (Pol::DIM == 16) return a.v[h][q];
+        else return a.v[q];
+    }
+    static SELINV_DEVINL void gather(T xv[CQ], const T *x, int b, int t)
+    {
+#pragma unroll
+        for (int q = 0; q < CQ; ++q) xv[q] = col(t, q) < b ? __ldcg(x + col(t, q)) : T(0);
+    }
+    // part[h] += (NEG ? -1 : 1) sum over the lane's columns of a[row][col] x[col]
+    template <bool NEG> static SELINV_DEVINL void madd(T part[RH], const typename Pol::Tile &a, const T xv[CQ])
+    {
+#pragma unroll
+        for (int h = 0; h < RH; ++h)
+#pragma unroll
+            for (int q = 0; q < CQ; ++q) part[h] = fma(NEG ? -at(a, h, q) : at(a, h, q), xv[q], part[h]);
+    }
+    static SELINV_DEVINL void reduce(T part[RH])
+    {
+#pragma unroll
+        for (int h = 0; h < RH; ++h) {
+            part[h] += shfl_xor(part[h], 1);
+            part[h] += shfl_xor(part[h], 2);
+        }
+    }
+};
+
+template <class T, class Pol>
+__global__ void __launch_bounds__(JWARPS * 32)
+jn_solve_fwd_kernel(JBufs<T> p, JDev jd, const int32_t *ent_owner, const int32_t *nodes, int64_t count,
+                    int64_t batch, const T *rhs, T *x)
+{
+    using V = VecOps<T, Pol>;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int64_t item = (int64_t)blockIdx.x * JWARPS + wid;
+    if (item >= count * batch) return;
+    const int32_t v = nodes[item % count];
+    const int64_t e = item / count;
+    const int b = p.b;
+    const T *W = p.W + e * jd.E * Pol::SLOT;
+    T *xe = x + e * jd.n * b;
+    const int64_t tau = (int64_t)jd.col_ptr[v] + v;            // v's diagonal target
+    T part[V::RH] = {};
+    for (int32_t c = jd.con_ptr[tau]; c < jd.con_ptr[tau + 1]; ++c) {
+        const int32_t ent = jd.con_w[c];                        // W_{v,k}
+        typename Pol::Tile w;
+        Pol::ld_ws(w, W + (int64_t)ent * Pol::SLOT, g, t, false);
+        T zk[V::CQ];
+        V::gather(zk, xe + (int64_t)ent_owner[ent] * b, b, t);
+        V::template madd<false>(part, w, zk);
+    }
+    V::reduce(part);
+    if (t == 0) {
+#pragma unroll
+        for (int h = 0; h < V::RH; ++h) {
+            const int r = g + 8 * h;
+            if (r < b) xe[(int64_t)v * b + r] = rhs[(e * jd.n + v) * b + r] - part[h];
+        }
+    }
+}
+
+template <class T, class Pol>
+__global__ void __launch_bounds__(JWARPS * 32)
+jn_solve_bwd_kernel(JBufs<T> p, JDev jd, const int32_t *ent_u, const int32_t *nodes, int64_t count, int64_t batch,
+                    T *x)
+{
+    using V = VecOps<T, Pol>;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int64_t item = (int64_t)blockIdx.x * JWARPS + wid;
+    if (item >= count * batch) return;
+    const int32_t v = nodes[item % count];
+    const int64_t e = item / count;
+    const int b = p.b;
+    const T *W = p.W + e * jd.E * Pol::SLOT;
+    T *xe = x + e * jd.n * b;
+    T part[V::RH] = {};
+    {
+        typename Pol::Tile sinv;
+        Pol::ld_ws(sinv, p.Sinv + (e * jd.n + v) * Pol::SLOT, g, t, false);
+        T zv[V::CQ];
+        V::gather(zv, xe + (int64_t)v * b, b, t);
+        V::template madd<false>(part, sinv, zv);                // S_v^-1 z_v
+    }
+    for (int32_t ent = jd.col_ptr[v]; ent < jd.col_ptr[v + 1]; ++ent) {
+        typename Pol::Tile wt;
+        Pol::ld_ws(wt, W + (int64_t)ent * Pol::SLOT, g, t, true);   // W_{u,v}^T
+        T xu[V::CQ];
+        V::gather(xu, xe + (int64_t)ent_u[ent] * b, b, t);
+        V::template madd<true>(part, wt, xu);
+    }
+    V::reduce(part);
+    if (t == 0) {
+#pragma unroll
+        for (int h = 0; h < V::RH; ++h) {
+            const int r = g + 8 * h;
+            if (r < b) xe[(int64_t)v * b + r] = part[h];
+        }
+    }
+}
+
 __global__ void junction_init(int32_t *info, int64_t batch)
 {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -530,9 +646,11 @@ template <class T, int SLOT> size_t ws_bytes(const selinv_junction_plan_s *pl, i
            2 * align256(sizeof(T) * SLOT * (size_t)(batch * pl->E)) + align256(sizeof(double) * (size_t)(batch * pl->n));
 }
 
+// G_diag == nullptr: the solve (rhs -> x) instead of the selected inverse.
 template <class T, class Pol>
 cudaError_t run_junction(const selinv_junction_plan_s *pl, int b, int64_t batch, const T *diag, const T *edge,
-                         T *G_diag, T *G_lower, double *logdet, int32_t *info, void *ws, cudaStream_t s)
+                         T *G_diag, T *G_lower, double *logdet, int32_t *info, void *ws, cudaStream_t s,
+                         const T *rhs = nullptr, T *x = nullptr)
 {
     constexpr int S = Pol::SLOT;
     char *w = static_cast<char *>(ws);
@@ -567,6 +685,20 @@ cudaError_t run_junction(const selinv_junction_plan_s *pl, int b, int64_t batch,
         if (ne > 0)
             jn_w_kernel<T, Pol><<<(unsigned)ceil_div(ne * batch, JWARPS), JWARPS * 32, smem_w, s>>>(
                 p, jd, pl->d_ce_ent + pl->ce_off[l], pl->d_ce_node + pl->ce_off[l], ne, batch);
+    }
+    if (G_diag == nullptr) {                                    // solve: forward, then backward
+        for (size_t l = 0; l + 1 < pl->c_off.size(); ++l) {
+            const int64_t nn = pl->c_off[l + 1] - pl->c_off[l];
+            jn_solve_fwd_kernel<T, Pol><<<(unsigned)ceil_div(nn * batch, JWARPS), JWARPS * 32, 0, s>>>(
+                p, jd, pl->d_ent_owner, pl->d_c_nodes + pl->c_off[l], nn, batch, rhs, x);
+        }
+        for (size_t l = 0; l + 1 < pl->d_off.size(); ++l) {
+            const int64_t nn = pl->d_off[l + 1] - pl->d_off[l];
+            jn_solve_bwd_kernel<T, Pol><<<(unsigned)ceil_div(nn * batch, JWARPS), JWARPS * 32, 0, s>>>(
+                p, jd, pl->d_ent_u, pl->d_d_nodes + pl->d_off[l], nn, batch, x);
+        }
+        junction_finalize<<<ib, 256, 0, s>>>(p.ld, pl->n, batch, logdet, info);
+        return cudaGetLastError();
     }
     for (size_t l = 0; l + 1 < pl->d_off.size(); ++l) {
         const int64_t nn = pl->d_off[l + 1] - pl->d_off[l];
@@ -605,25 +737,27 @@ constexpr size_t GRAPH_CACHE = 4;
 // launches directly, inside its own graph.
 template <class T, class Pol>
 cudaError_t junction_call(selinv_junction_plan_s *pl, int dtype, int b, int64_t batch, const T *diag, const T *edge,
-                          T *G_diag, T *G_lower, double *logdet, int32_t *info, void *ws, cudaStream_t s)
+                          T *G_diag, T *G_lower, double *logdet, int32_t *info, void *ws, cudaStream_t s,
+                          const T *rhs = nullptr, T *x = nullptr)
 {
     cudaError_t err = junction_attributes<T, Pol>();
     if (err != cudaSuccess) return err;
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone)
-        return run_junction<T, Pol>(pl, b, batch, diag, edge, G_diag, G_lower, logdet, info, ws, s);
-    const void *key[7] = {diag, edge, G_diag, G_lower, logdet, info, ws};
+        return run_junction<T, Pol>(pl, b, batch, diag, edge, G_diag, G_lower, logdet, info, ws, s, rhs, x);
+    const void *key[9] = {diag, edge, G_diag, G_lower, logdet, info, ws, rhs, x};
     std::lock_guard<std::mutex> lock(pl->mu);
     ++pl->calls;
     for (auto &g : pl->graphs)
-        if (g.dtype == dtype && g.b == b && g.batch == batch && std::equal(key, key + 7, g.ptr)) {
+        if (g.dtype == dtype && g.b == b && g.batch == batch && std::equal(key, key + 9, g.ptr)) {
             g.used = pl->calls;
             return cudaGraphLaunch(g.exec, s);
         }
     if (!pl->capture && (err = cudaStreamCreateWithFlags(&pl->capture, cudaStreamNonBlocking)) != cudaSuccess)
         return err;
     if ((err = cudaStreamBeginCapture(pl->capture, cudaStreamCaptureModeThreadLocal)) != cudaSuccess) return err;
-    cudaError_t run = run_junction<T, Pol>(pl, b, batch, diag, edge, G_diag, G_lower, logdet, info, ws, pl->capture);
+    cudaError_t run =
+        run_junction<T, Pol>(pl, b, batch, diag, edge, G_diag, G_lower, logdet, info, ws, pl->capture, rhs, x);
     cudaGraph_t graph = nullptr;
     err = cudaStreamEndCapture(pl->capture, &graph);
     if (run != cudaSuccess || err != cudaSuccess) {
@@ -645,7 +779,7 @@ cudaError_t junction_call(selinv_junction_plan_s *pl, int dtype, int b, int64_t 
     g.dtype = dtype;
     g.b = b;
     g.batch = batch;
-    std::copy(key, key + 7, g.ptr);
+    std::copy(key, key + 9, g.ptr);
     g.exec = exec;
     g.used = pl->calls;
     pl->graphs.push_back(g);
@@ -667,7 +801,8 @@ void selinv_junction_plan_free(selinv_junction_plan_t *pl)
     if (!pl) return;
     int32_t *arrs[] = {pl->d_c_nodes, pl->d_d_nodes, pl->d_col_ptr, pl->d_ent_slot, pl->d_ent_trans, pl->d_ent_src,
                        pl->d_con_ptr, pl->d_con_w, pl->d_con_a, pl->d_pair_ptr, pl->d_pair, pl->d_ct_node,
-                       pl->d_ct_t, pl->d_ce_ent, pl->d_ce_node, pl->d_de_ent, pl->d_de_node, pl->d_de_a};
+                       pl->d_ct_t, pl->d_ce_ent, pl->d_ce_node, pl->d_de_ent, pl->d_de_node, pl->d_de_a,
+                       pl->d_ent_owner, pl->d_ent_u};
     for (auto &g : pl->graphs) cudaGraphExecDestroy(g.exec);   // a launch in flight is freed on completion
     if (pl->capture) cudaStreamDestroy(pl->capture);
     for (int32_t *a : arrs) cudaFree(a);
@@ -960,6 +1095,16 @@ static selinv_status junction_plan_impl(int64_t n, int64_t m, const int32_t *ei,
             up(&pl->d_de_ent, de_ent);
             up(&pl->d_de_node, de_node);
             up(&pl->d_de_a, de_a);
+            {
+                std::vector<int32_t> owner(std::max<int64_t>(E, 1), 0), uu(std::max<int64_t>(E, 1), 0);
+                for (int32_t v = 0; v < n; ++v)
+                    for (int32_t a = 0; a < (int32_t)nbr[v].size(); ++a) {
+                        owner[col_ptr[v] + a] = v;
+                        uu[col_ptr[v] + a] = nbr[v][a];
+                    }
+                up(&pl->d_ent_owner, owner);
+                up(&pl->d_ent_u, uu);
+            }
             if (!ok) return SELINV_ERR_CUDA;
             *out = hold.release();
         }
@@ -1072,6 +1217,48 @@ selinv_status selinv_junction(const selinv_junction_plan_t *pl, selinv_dtype dty
     else
         err = b <= 8 ? junction_call<float, Pol8<float>>(mp, dt, b, batch, fd, fe, fg, fl, logdet, info, workspace, s)
                      : junction_call<float, Pol16<float>>(mp, dt, b, batch, fd, fe, fg, fl, logdet, info, workspace, s);
+    return err == cudaSuccess ? SELINV_OK : SELINV_ERR_CUDA;
+}
+
+selinv_status selinv_junction_solve(const selinv_junction_plan_t *pl, selinv_dtype dtype, int32_t b, int64_t batch,
+                                    const void *diag, const void *edge_val, const void *rhs, void *x, double *logdet,
+                                    int32_t *info, void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!pl || (dtype != SELINV_F64 && dtype != SELINV_F32) || b < 1 || batch < 0) return SELINV_ERR_INVALID_ARG;
+    if (b > 16) return SELINV_ERR_UNSUPPORTED;
+    if (batch == 0) return SELINV_OK;
+    if (!diag || (pl->m > 0 && !edge_val) || !rhs || !x || !info) return SELINV_ERR_INVALID_ARG;
+    if (rhs == x) return SELINV_ERR_INVALID_ARG;
+    const size_t es = dtype == SELINV_F64 ? 8 : 4;
+    if (!is_aligned(diag, es) || !is_aligned(edge_val, es) || !is_aligned(rhs, es) || !is_aligned(x, es) ||
+        !is_aligned(logdet, 8) || !is_aligned(info, 4) || !is_aligned(workspace, 256))
+        return SELINV_ERR_INVALID_ARG;
+    const size_t need = selinv_junction_workspace_size(pl, dtype, b, batch);
+    if (!workspace || workspace_bytes < need) return SELINV_ERR_WORKSPACE;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev != pl->device) return SELINV_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    auto *mp = const_cast<selinv_junction_plan_s *>(pl);
+    const int dt = (int)dtype;
+    cudaError_t err;
+    if (dtype == SELINV_F64) {
+        const double *dd = static_cast<const double *>(diag), *de = static_cast<const double *>(edge_val);
+        const double *r = static_cast<const double *>(rhs);
+        double *xx = static_cast<double *>(x);
+        err = b <= 8 ? junction_call<double, Pol8<double>>(mp, dt, b, batch, dd, de, nullptr, nullptr, logdet, info,
+                                                           workspace, s, r, xx)
+                     : junction_call<double, Pol16<double>>(mp, dt, b, batch, dd, de, nullptr, nullptr, logdet, info,
+                                                            workspace, s, r, xx);
+    } else {
+        const float *fd = static_cast<const float *>(diag), *fe = static_cast<const float *>(edge_val);
+        const float *r = static_cast<const float *>(rhs);
+        float *xx = static_cast<float *>(x);
+        err = b <= 8 ? junction_call<float, Pol8<float>>(mp, dt, b, batch, fd, fe, nullptr, nullptr, logdet, info,
+                                                         workspace, s, r, xx)
+                     : junction_call<float, Pol16<float>>(mp, dt, b, batch, fd, fe, nullptr, nullptr, logdet, info,
+                                                          workspace, s, r, xx);
+    }
     return err == cudaSuccess ? SELINV_OK : SELINV_ERR_CUDA;
 }
 

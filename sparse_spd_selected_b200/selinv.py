@@ -120,6 +120,8 @@ def lib():
         L.selinv_junction_workspace_size.restype = SZ
         L.selinv_junction.argtypes = [P, ctypes.c_int, I32, I64, P, P, P, P, P, P, P, SZ, P]
         L.selinv_junction.restype = ctypes.c_int
+        L.selinv_junction_solve.argtypes = [P, ctypes.c_int, I32, I64, P, P, P, P, P, P, P, SZ, P]
+        L.selinv_junction_solve.restype = ctypes.c_int
         L.selinv_tree_plan.argtypes = [P, I64, I64, ctypes.POINTER(P)]
         L.selinv_tree_plan.restype = ctypes.c_int
         L.selinv_tree_plan_free.argtypes = [P]
@@ -648,6 +650,46 @@ class JunctionPlan:
             self.close()
         except Exception:
             pass
+
+
+def junction_solve(plan: JunctionPlan, diag, edge_val, rhs, *, check=True, out=None, workspace=None, stream=None):
+    """x = A^-1 r for general block-sparse SPD matrices on the plan's pattern
+    (b <= 16), from the same factorisation: diag [..., n, b, b], edge_val
+    [..., m, b, b], rhs [..., n, b].  Returns (x, logdet, info)."""
+    _cuda_contig("diag", diag)
+    dt = diag.dtype
+    if diag.dim() < 3 or diag.shape[-1] != diag.shape[-2] or int(diag.shape[-3]) != plan.n:
+        raise ValueError(f"diag must be [..., {plan.n}, b, b]")
+    lead = tuple(diag.shape[:-3])
+    b = int(diag.shape[-1])
+    batch = 1
+    for d in lead:
+        batch *= int(d)
+    _cuda_contig("edge_val", edge_val, dt)
+    if tuple(edge_val.shape) != lead + (plan.m, b, b):
+        raise ValueError(f"edge_val must be {lead + (plan.m, b, b)}")
+    _cuda_contig("rhs", rhs, dt)
+    if tuple(rhs.shape) != lead + (plan.n, b):
+        raise ValueError(f"rhs must be {lead + (plan.n, b)}")
+    dev = diag.device
+    out = dict(out or {})
+    x = out.get("x")
+    if x is None:
+        x = torch.empty_like(rhs)
+    logdet = out.get("logdet")
+    if logdet is None:
+        logdet = torch.empty(lead, dtype=torch.float64, device=dev)
+    info = out.get("info")
+    if info is None:
+        info = torch.empty(lead, dtype=torch.int32, device=dev)
+    nbytes = plan.workspace_size(dt, b, batch)
+    ws = _workspace(nbytes, dev, workspace)
+    with torch.cuda.device(dev):
+        st = lib().selinv_junction_solve(plan.handle, _code(dt), b, batch, _ptr(diag), _ptr(edge_val), _ptr(rhs),
+                                         _ptr(x), _ptr(logdet), _ptr(info), _ptr(ws), nbytes, _stream_handle(stream))
+    _check(st, "selinv_junction_solve")
+    _raise_on_info(info, check)
+    return x, logdet, info
 
 
 def junction(plan: JunctionPlan, diag, edge_val, *, check=True, out=None, workspace=None, stream=None):

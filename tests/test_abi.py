@@ -229,3 +229,9 @@ def test_flags_are_validated_before_any_launch(lib):
                       flags=selinv.WANT_LOGDET | selinv.WANT_SOLVE | selinv.CHECK) == selinv.OK
     f = lib.selinv_tree
     assert f(None, 0, 4, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 1 << 30, 0, None) == selinv.ERR_INVALID_ARG
+
+
+def test_junction_solve_argument_errors(lib):
+    f = lib.selinv_junction_solve
+    # plan, dtype, b, batch, diag, edge_val, rhs, x, logdet, info, workspace, ws_bytes, stream
+    assert f(None, 0, 4, 1, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 1 << 30, None) == selinv.ERR_INVALID_ARG

@@ -176,3 +176,70 @@ def test_junction_graph_replay_reads_new_values(cuda_ok):
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(out["G_diag"], fresh["G_diag"])
+
+
+def solve_both(n, E, b, seed, dtype, lead=(2,), load=1.0):
+    batch = int(np.prod(lead))
+    d, e = inputs.graph_inputs(batch, n, b, E, seed=seed, load=load)
+    r = np.random.default_rng([seed, 7]).standard_normal((batch, n, b))
+    d, e, r = d.reshape(lead + (n, b, b)), e.reshape(lead + (E.shape[1], b, b)), r.reshape(lead + (n, b))
+    plan = selinv.JunctionPlan(n, E)
+    dd, ee, rr = to_dev(d, dtype), to_dev(e, dtype), to_dev(r, dtype)
+    x, ld, info = selinv.junction_solve(plan, dd, ee, rr)
+    ref = oracle.junction_solve(host(dd), E, host(ee), host(rr))
+    nl = len(lead)
+    assert (host(info) == -1).all()
+    assert worst(host(x), ref["x"], nl, block_ndim=1) <= TOL[dtype]
+    assert logdet_err(host(ld), ref["logdet"]) <= TOL[dtype]
+    return plan, dd, ee, rr, x
+
+
+@pytest.mark.parametrize("b", [1, 3, 8, 16])
+def test_junction_solve_matches_oracle(cuda_ok, b):
+    """x = A^-1 r on the pages' 3 x 3 grid and on random patterns (fill)."""
+    solve_both(9, inputs.grid_edges(3, 3), b, 11800 + b, torch.float64)
+    solve_both(30, random_pattern(30, 70, 11810 + b), b, 11820 + b, torch.float64)
+
+
+def test_junction_solve_f32_leading_dims_and_selinv_consistency(cuda_ok):
+    solve_both(16, inputs.grid_edges(4, 4), 8, 11900, torch.float32, lead=(3,), load=2.0)
+    solve_both(16, inputs.grid_edges(4, 4), 16, 11901, torch.float32, lead=(2, 2), load=2.0)
+    plan, dd, ee, rr, x = solve_both(20, inputs.grid_edges(4, 5), 5, 11902, torch.float64, lead=(3,))
+    # the same factorisation: the log det of the selected-inverse call is identical
+    full = selinv.junction(plan, dd, ee)
+    _, ld, _ = selinv.junction_solve(plan, dd, ee, rr)
+    assert torch.equal(ld, full["logdet"])
+
+
+def test_junction_solve_lattice_benchmark_size(cuda_ok):
+    """64 matrices on the 32 x 32 lattice of 8 x 8 blocks: the block residual
+    sum_u A_vu x_u - r_v of every matrix, against the right-hand side."""
+    w = inputs.WORKLOADS["lattice_64x1024_b8"]
+    g = inputs.generate(w)
+    E = g["edge_index"]
+    n, b = w.L, w.b
+    r = np.random.default_rng(11950).standard_normal((w.batch, n, b))
+    plan = selinv.JunctionPlan(n, E)
+    x, _, info = selinv.junction_solve(plan, to_dev(g["diag"], torch.float64), to_dev(g["edge_val"], torch.float64),
+                                       to_dev(r, torch.float64))
+    x = host(x)
+    assert (host(info) == -1).all()
+    ei, ej = E
+    sym = lambda D: np.tril(D) + np.swapaxes(np.tril(D, -1), -1, -2)
+    for e in range(w.batch):
+        res = np.einsum("vab,vb->va", sym(g["diag"][e]), x[e]) - r[e]
+        np.add.at(res, ei, np.einsum("kab,kb->ka", g["edge_val"][e], x[e][ej]))
+        np.add.at(res, ej, np.einsum("kba,kb->ka", g["edge_val"][e], x[e][ei]))
+        assert float(np.linalg.norm(res) / np.linalg.norm(r[e])) <= 1e-12, e
+
+
+def test_junction_solve_not_spd(cuda_ok):
+    E = inputs.grid_edges(3, 4)
+    d, e = inputs.graph_inputs(2, 12, 3, E, seed=11960, load=1.0)
+    d[1, 5] = -np.eye(3)
+    plan = selinv.JunctionPlan(12, E)
+    r = to_dev(np.ones((2, 12, 3)), torch.float64)
+    _, _, info = selinv.junction_solve(plan, to_dev(d, torch.float64), to_dev(e, torch.float64), r, check=False)
+    assert host(info)[0] == -1 and host(info)[1] >= 0
+    with pytest.raises(selinv.NotSPDError):
+        selinv.junction_solve(plan, to_dev(d, torch.float64), to_dev(e, torch.float64), r)
