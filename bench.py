@@ -12,7 +12,10 @@ The metric is b x b blocks per second (value = all ranks' blocks / time).
 Under torchrun each rank owns its own slice of chains (batch elements are
 independent, so there is no data-path collective: weak scaling); a barrier and
 a max-over-ranks of the device-timed region are the only cross-rank steps.
-Inputs (> 2 GB) are larger than L2, so no flush is needed between steps.
+The default workload's inputs (> 2 GB) are larger than L2, so no flush is
+needed between its steps; workloads whose inputs fit in L2 (126 MB) get a
+256 MB device write before every timed step, outside the step's own events,
+and are timed by those per-step events.
 
 ``--impl reference`` times the CPU oracle (the plain C implementation the
 tests check against) on a bounded sample of the same workload instead.
@@ -40,6 +43,7 @@ from sparse_spd_selected_b200 import inputs  # noqa: E402
 
 PROFILES = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = {
+    "chain_tiny_kernel": ["chain_tiny.cu", "common.cuh"],
     "chain_small_kernel": ["chain_small.cu", "warp16.cuh", "common.cuh"],
     "chain_mid_kernel": ["chain_mid.cu", "quad32.cuh", "warp16.cuh", "common.cuh"],
     "seg_collect_kernel": ["chain_seg.cu", "quad32.cuh", "warp16.cuh", "common.cuh"],
@@ -377,10 +381,19 @@ PER_CONFIG = [("chain_1x8_b4", "f64"), ("chain_4096x64_b16", "f64"), ("chain_64x
               ("chain_64x4096_b32", "f32"), ("forest_8x32768_b16", "f64"), ("grid_256x128_b128", "f64")]
 
 
+L2_FLUSH_BYTES = 256 << 20      # more than twice the B200's 126 MB L2
+
+
+def fits_l2(w):
+    """Inputs small enough to stay in L2 between steps (then flushed before each timed step)."""
+    return w.L * w.batch * w.b * w.b * 8 <= L2_FLUSH_BYTES
+
+
 def config_dict(w, batch, world, op, full_size):
     """The bench line's `config`: the same dict for both arms of one workload."""
-    l2 = "inputs larger than L2 (no flush)" if w.L * w.batch * w.b * w.b * 8 > 256 << 20 else \
-        "fits in L2 (latency case; device time from a CUDA graph of back-to-back calls)"
+    l2 = "inputs larger than L2 (no flush)" if not fits_l2(w) else \
+        ("inputs fit in L2: a 256 MB device write flushes L2 before every timed step, outside the "
+         "step's own CUDA events; time = sum of the per-step event times")
     return {"workload": w.name if full_size else f"{w.name} (batch {batch}, length {w.L} per GPU)",
             "global_batch": batch * world, "block": w.b, "L_or_n": w.L,
             "solve": bool(w.solve) and op in ("selinv", "sample"), "op": op,
@@ -568,6 +581,8 @@ def build_step(w, dtype, op, batch, elems):
                    "info": torch.empty(batch, dtype=torch.int32, device="cuda")}
             ws = torch.empty(max(selinv.chain_workspace_size(tdt, batch, L, b, False, True), 1),
                              dtype=torch.uint8, device="cuda")
+        elif b <= 8 and L <= 16 and tdt == torch.float64:
+            kernel = "chain_tiny_kernel"
         elif b <= 16:
             kernel = "chain_small_kernel"
         elif segments > 0:
@@ -659,9 +674,13 @@ def measure(w, dtype, op, batch, steps, warmup, rank, world, local, full_size, w
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    small = fits_l2(w)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda") if small else None
     with ClockSampler(dev_index) as clk:
         t_start.record(stream)
         for i in range(K):
+            if flush is not None:
+                flush.fill_(i & 0xFF)            # evicts this step's inputs and outputs from L2
             k_start[i].record(stream)
             step()
             k_end[i].record(stream)
@@ -671,11 +690,13 @@ def measure(w, dtype, op, batch, steps, warmup, rank, world, local, full_size, w
         dist.barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
     kernel_ms = sum(a.elapsed_time(b_) for a, b_ in zip(k_start, k_end)) / K
+    if small:
+        elapsed_ms = kernel_ms * K               # the flushes between steps are not the workload's time
+    del flush
     elapsed_ms = max_over_ranks(elapsed_ms, world, "cuda")
     nodes_per_rank = batch * w.L
     value = job_throughput(world, nodes_per_rank, K, elapsed_ms)
-    latency_case = w.L * w.batch * w.b * w.b * 8 <= 256 << 20
-    device_us = graph_device_us(step, stream) if latency_case else None
+    device_us = graph_device_us(step, stream) if small else None
 
     # end to end through the same call, inputs from pinned host memory, outputs read back
     e2e = None
@@ -705,7 +726,7 @@ def measure(w, dtype, op, batch, steps, warmup, rank, world, local, full_size, w
 
     hbm, src = hbm_peak()
     byt = algorithmic_bytes(w, es, batch, op)
-    t_ms = device_us / 1e3 if device_us is not None else kernel_ms
+    t_ms = kernel_ms
     hbm_achieved = byt / (t_ms / 1e3) / 1e9
     flops = algorithmic_flops(w, batch, op)
     flop_rate = flops / (t_ms / 1e3) / 1e12
@@ -734,15 +755,15 @@ def measure(w, dtype, op, batch, steps, warmup, rank, world, local, full_size, w
     else:
         roof = {"bound": "hbm", "achieved": hbm_achieved, "peak": hbm, "unit": "GB/s", "frac": hbm_achieved / hbm,
                 "traffic": traffic, "peak_source": hbm_src, "algorithmic_bytes_per_launch": byt, "kernel": kernel}
-    if latency_case:
-        roof["note"] = ("latency case: one warp works 8 dependent blocks; achieved uses the device time of "
-                        "one call from a CUDA graph, not a bandwidth claim")
+    if small:
+        roof["note"] = ("inputs fit in L2: achieved uses the per-step device time with L2 flushed before "
+                        "each step; device_us_per_call is one call's time inside a CUDA graph of "
+                        "back-to-back calls (warm L2)")
     res = {"value": value, "ms_per_step": elapsed_ms / K, "kernel_ms": kernel_ms, "roofline": roof,
            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": K * launches_per_step, "clocks": clk.summary(),
            "kernel": kernel, "config": config_dict(w, batch, world, op, full_size), "dtype": dtype}
     if device_us is not None:
         res["device_us_per_call"] = device_us
-        res["host_us_per_call"] = kernel_ms * 1e3
     del S, step, out, dev_in, host_in
     torch.cuda.synchronize()
     torch.cuda.empty_cache()

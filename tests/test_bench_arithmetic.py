@@ -50,3 +50,17 @@ def test_oracle_stand_ins_stay_small():
     w, note = bench.oracle_workload(W["chain_4096x64_b16"], "selinv")
     assert w == W["chain_4096x64_b16"] and note == ""
     assert dataclasses.replace(W["chain_1x8_b4"]) == W["chain_1x8_b4"]
+
+
+def test_l2_rule_per_workload():
+    # workloads whose inputs stay in L2 are flushed before every timed step; the rest
+    # are larger than L2 (126 MB) by more than twice
+    small = {n for n, w in inputs.WORKLOADS.items() if bench.fits_l2(w)}
+    assert "chain_1x8_b4" in small and "lattice_64x1024_b8" in small
+    for n, w in inputs.WORKLOADS.items():
+        cfg = bench.config_dict(w, w.batch, 1, "selinv", True)
+        if n in small:
+            assert "flushes L2" in cfg["l2"]
+        else:
+            assert w.L * w.batch * w.b * w.b * 8 > 2 * 126e6
+            assert cfg["l2"].startswith("inputs larger than L2")
