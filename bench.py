@@ -806,7 +806,7 @@ def run_ours(args):
                             want_cpu, not args.no_e2e)
             per_config[key] = {k: r[k] for k in ("value", "ms_per_step", "kernel_ms", "roofline", "cpu_baseline",
                                                  "e2e", "clocks", "gpu_launches", "dtype", "config")}
-            for k in ("device_us_per_call", "host_us_per_call"):
+            for k in ("device_us_per_call",):
                 if k in r:
                     per_config[key][k] = r[k]
     if world > 1:
@@ -827,6 +827,8 @@ def run_ours(args):
         "clocks": head["clocks"],
         "kernel_ms": head["kernel_ms"],
     }
+    if "device_us_per_call" in head:
+        line["device_us_per_call"] = head["device_us_per_call"]
     if per_config is not None:
         line["per_config"] = per_config
     print(json.dumps(line), flush=True)
