@@ -25,12 +25,17 @@ namespace selinv {
 
 namespace {
 
-constexpr int WARPS = 4;
+constexpr int WARPS = 4;                 // chains per CTA of the several-right-hand-side kernel
 
-// Resident CTAs per SM the register allocation is sized for (4 warps each).
-#ifndef SELINV_CHAIN_MINB
-#define SELINV_CHAIN_MINB 4
+// Chains (warps) per CTA of the selected-inverse kernel, and the resident CTAs
+// per SM its register allocation is sized for.
+#ifndef SELINV_CHAIN_WARPS
+#define SELINV_CHAIN_WARPS 1
 #endif
+#ifndef SELINV_CHAIN_MINB
+#define SELINV_CHAIN_MINB 16
+#endif
+constexpr int CWARPS = SELINV_CHAIN_WARPS;
 
 // L2 use between the sweeps.  The distribute sweep reads the S_i^-1 slots
 // and the B_i back in reverse order, so those of a chain's last blocks are
@@ -58,14 +63,14 @@ template <class T> __host__ __device__ constexpr int warp_smem_elems()
 }
 
 template <class T, bool FULL, bool WANT_G, bool WANT_X, bool SAMPLE = false>
-__global__ void __launch_bounds__(WARPS * 32, SELINV_CHAIN_MINB) chain_small_kernel(ChainArgs<T> p)
+__global__ void __launch_bounds__(CWARPS * 32, SELINV_CHAIN_MINB) chain_small_kernel(ChainArgs<T> p)
 {
     using namespace w16;
     constexpr int E = SL<T>::ELEMS;
     const int lane = threadIdx.x & 31;
     const int wid = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
-    const int64_t e = (int64_t)blockIdx.x * WARPS + wid;
+    const int64_t e = (int64_t)blockIdx.x * CWARPS + wid;
     if (e >= p.batch) return;
 
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -473,14 +478,14 @@ __global__ void __launch_bounds__(WARPS * 32, 3) chain_multi_kernel(ChainArgs<T>
 template <class T, bool FULL, bool G, bool X, bool SAMPLE = false>
 cudaError_t launch_t(const ChainArgs<T> &a, cudaStream_t s)
 {
-    const size_t smem = sizeof(T) * warp_smem_elems<T>() * WARPS;
+    const size_t smem = sizeof(T) * warp_smem_elems<T>() * CWARPS;
     auto k = chain_small_kernel<T, FULL, G, X, SAMPLE>;
     cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    const int64_t blocks = ceil_div(a.batch, WARPS);
+    const int64_t blocks = ceil_div(a.batch, CWARPS);
     ChainArgs<T> c = a;
     c.ws_lines = (reinterpret_cast<uintptr_t>(a.ws) & 127) == 0;
-    k<<<(unsigned)blocks, WARPS * 32, smem, s>>>(c);
+    k<<<(unsigned)blocks, CWARPS * 32, smem, s>>>(c);
     return cudaGetLastError();
 }
 
