@@ -387,3 +387,45 @@ def test_short_chains_of_small_blocks(cuda_ok, b, L):
     out = selinv.selinv_chain(to_dev(bad, torch.float64), l, check=False)
     info = host(out["info"]).tolist()
     assert info[2] == L - 1 and all(v == -1 for k, v in enumerate(info) if k != 2)
+
+
+# ---------------- b <= 16, more chains than the GPU holds at once ----------------
+
+BIG_BATCH = 5000      # above the 2368 chains a B200 holds at once (one per CTA, 16 per SM)
+
+
+@pytest.mark.parametrize("b,L,dtype", [(16, 8, torch.float64), (16, 9, torch.float64), (5, 12, torch.float64),
+                                       (16, 10, torch.float32)])
+def test_batch_beyond_one_round(cuda_ok, b, L, dtype):
+    """Chains started in the first round and in the last one, sampled against
+    the oracle; G, x and log det the same from every entry point."""
+    diag, lower, rhs = inputs.chain_inputs(BIG_BATCH, L, b, seed=8100 + 7 * b + L, load=1.0)
+    d, l, r = to_dev(diag, dtype), to_dev(lower, dtype), to_dev(rhs, dtype)
+    out = selinv.selinv_chain(d, l, r)
+    assert bool((out["info"] == -1).all())
+    pick = [0, 1, 2500, 3900, 4300, 4998, 4999]
+    ref = oracle.chain(host(d)[pick], host(l)[pick], host(r)[pick])
+    tol = TOL[dtype]
+    assert worst(host(out["G_diag"][pick]), ref["G_diag"]) <= tol
+    assert worst(host(out["G_lower"][pick]), ref["G_lower"]) <= tol
+    assert worst_vec(host(out["x"][pick]), ref["x"]) <= tol
+    assert logdet_err(host(out["logdet"][pick]), ref["logdet"]) <= tol
+    Gd = out["G_diag"]
+    assert torch.equal(Gd, Gd.transpose(-1, -2))
+    again = selinv.selinv_chain(d, l, r)
+    for k in ("G_diag", "G_lower", "x", "logdet"):
+        assert torch.equal(again[k], out[k]), k
+    g_only = selinv.selinv_chain(d, l)
+    assert torch.equal(g_only["G_diag"], out["G_diag"]) and torch.equal(g_only["G_lower"], out["G_lower"])
+    x, ld, info = selinv.chain_solve(d, l, r)
+    assert torch.equal(x, out["x"]) and torch.equal(ld, out["logdet"])
+
+
+def test_batch_beyond_one_round_not_spd(cuda_ok):
+    diag, lower, _ = inputs.chain_inputs(BIG_BATCH, 8, 16, seed=8200, load=1.0, with_rhs=False)
+    diag[BIG_BATCH - 1, 2] = -np.eye(16)
+    diag[BIG_BATCH - 2, 6] = -np.eye(16)
+    out = selinv.selinv_chain(to_dev(diag, torch.float64), to_dev(lower, torch.float64), check=False)
+    info = host(out["info"])
+    assert (info[:BIG_BATCH - 2] == -1).all()
+    assert info[BIG_BATCH - 1] == 2 and info[BIG_BATCH - 2] == 6
