@@ -41,6 +41,7 @@ struct selinv_tree_plan_s {
     int32_t *d_dist_nodes = nullptr;       // non-root global ids by (depth, id)
     int32_t *d_child_ptr = nullptr;        // [trees*n + 1]
     int32_t *d_child_idx = nullptr;        // global ids, ascending per parent
+    int32_t *d_cpos = nullptr;             // [trees*n] position of each node in its parent's list, -1 roots
     int32_t *d_parent = nullptr;           // global parent id or -1
     int32_t spin_limit = 1 << 22;          // polls before a dependency wait gives up (SPIN_LIMIT)
     int64_t hold = -1;                     // node whose completion is never published (tests)
@@ -68,6 +69,7 @@ struct TreeDev {
     int64_t n;
     int32_t spin_limit;   // polls before a dependency wait gives up
     int64_t hold;         // a node whose completion flag is never published (tests), or -1
+    const int32_t *cpos;  // position of each node in its parent's child list (-1 for roots)
 };
 
 template <class T> struct TreeBufs {
@@ -75,7 +77,7 @@ template <class T> struct TreeBufs {
     T *G_diag, *G_edge;
     const T *z;              // draws: standard normals [N, b]
     T *eta;                  // draws: R_v z_v after the collect sweep, the draw after the distribute sweep
-    T *ws_sinv, *ws_u;       // per node lower slots
+    T *ws_sinv, *ws_u;       // lower slots: S_v^-1 per node, U_v at v's position in its parent's child list
     double *ws_ld;           // per node log det S_v
     int32_t *info;           // per tree, INT_MAX = ok until finalised
     int b;
@@ -203,10 +205,10 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leave
             Tile<T> acc;                              // sum of the children's U_c (lower slots), two
             zero(acc);                                // children's loads in flight at a time
             const int32_t c0 = td.child_ptr[v], c1 = td.child_ptr[v + 1];
-            for (int32_t c = c0; c < c1; c += 2) {
+            for (int32_t c = c0; c < c1; c += 2) {    // children's slots sit at their list positions
                 Tile<T> u, u2;
-                load_lower_slot_l2<T>(u, p.ws_u + (int64_t)td.child_idx[c] * SLOT_ELEMS, lane, g, t);
-                if (c + 1 < c1) load_lower_slot_l2<T>(u2, p.ws_u + (int64_t)td.child_idx[c + 1] * SLOT_ELEMS, lane, g, t);
+                load_lower_slot_l2<T>(u, p.ws_u + (int64_t)c * SLOT_ELEMS, lane, g, t);
+                if (c + 1 < c1) load_lower_slot_l2<T>(u2, p.ws_u + (int64_t)(c + 1) * SLOT_ELEMS, lane, g, t);
                 else zero(u2);
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
@@ -284,7 +286,7 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leave
             if (DRAW) store_block_T<T, true>(p.ws_sinv + (int64_t)v * DRAW_SLOT, w, 16, g, t);   // W_v^T, 16 x 16
             zero(u);
             gemm_nt<false, true>(u, w, et, sT, sT2, g, t);   // U_v = W_v E_v^T (lower tiles)
-            store_lower_slot<T>(p.ws_u + (int64_t)v * SLOT_ELEMS, u, lane, g, t);
+            store_lower_slot<T>(p.ws_u + (int64_t)td.cpos[v] * SLOT_ELEMS, u, lane, g, t);
             __syncwarp();                             // the warp's stores are ordered before lane 0's release
             int old = 0;
             if (lane == 0) old = atom_add_acq_rel(sy.pending + par, -1);   // release U_v; the last child acquires all siblings'
@@ -818,7 +820,7 @@ cudaError_t run_tree(const selinv_tree_plan_s *pl, int b, const T *diag, const T
     sy.counters = reinterpret_cast<unsigned long long *>(w);
     p.info = info;
     p.b = b;
-    TreeDev td{pl->d_child_ptr, pl->d_child_idx, pl->d_parent, pl->n, pl->spin_limit, pl->hold};
+    TreeDev td{pl->d_child_ptr, pl->d_child_idx, pl->d_parent, pl->n, pl->spin_limit, pl->hold, pl->d_cpos};
 
     const int64_t init_n = std::max<int64_t>(N, pl->trees);
     tree_init<<<(unsigned)ceil_div(init_n, 256), 256, 0, s>>>(pl->d_child_ptr, N, sy.pending, sy.done, sy.counters,
@@ -898,7 +900,7 @@ cudaError_t run_tree_backward(const selinv_tree_plan_s *pl, int b, const T *diag
     sy.counters = reinterpret_cast<unsigned long long *>(w);
     p.info = info;
     p.b = b;
-    TreeDev td{pl->d_child_ptr, pl->d_child_idx, pl->d_parent, pl->n, pl->spin_limit, pl->hold};
+    TreeDev td{pl->d_child_ptr, pl->d_child_idx, pl->d_parent, pl->n, pl->spin_limit, pl->hold, pl->d_cpos};
 
     const int64_t init_n = std::max<int64_t>(N, pl->trees);
     tree_init<<<(unsigned)ceil_div(init_n, 256), 256, 0, s>>>(pl->d_child_ptr, N, sy.pending, sy.done, sy.counters,
@@ -1038,6 +1040,12 @@ static selinv_status tree_plan_impl(const int32_t *parent, int64_t trees, int64_
     up(&pl->d_dist_nodes, dnodes);
     up(&pl->d_child_ptr, cnt);
     up(&pl->d_child_idx, child);
+    {
+        std::vector<int32_t> cpos(N, -1);
+        for (int64_t v = 0; v < N; ++v)
+            for (int32_t c = cnt[v]; c < cnt[v + 1]; ++c) cpos[child[c]] = c;
+        up(&pl->d_cpos, cpos);
+    }
     up(&pl->d_parent, gparent);
     if (!ok) return SELINV_ERR_CUDA;
     *out = hold.release();
@@ -1065,6 +1073,7 @@ void selinv_tree_plan_free(selinv_tree_plan_t *pl)
     cudaFree(pl->d_dist_nodes);
     cudaFree(pl->d_child_ptr);
     cudaFree(pl->d_child_idx);
+    cudaFree(pl->d_cpos);
     cudaFree(pl->d_parent);
     delete pl;
 }
