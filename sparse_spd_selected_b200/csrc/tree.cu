@@ -42,6 +42,9 @@ struct selinv_tree_plan_s {
     int32_t *d_child_ptr = nullptr;        // [trees*n + 1]
     int32_t *d_child_idx = nullptr;        // global ids, ascending per parent
     int32_t *d_cpos = nullptr;             // [trees*n] position of each node in its parent's list, -1 roots
+    int32_t *d_cont = nullptr;             // [trees*n] first child of a non-root node, else -1
+    int32_t *d_heads = nullptr;            // distribute chain heads by (depth, id)
+    int64_t nheads = 0;
     int32_t *d_parent = nullptr;           // global parent id or -1
     int32_t spin_limit = 1 << 22;          // polls before a dependency wait gives up (SPIN_LIMIT)
     int64_t hold = -1;                     // node whose completion is never published (tests)
@@ -70,6 +73,7 @@ struct TreeDev {
     int32_t spin_limit;   // polls before a dependency wait gives up
     int64_t hold;         // a node whose completion flag is never published (tests), or -1
     const int32_t *cpos;  // position of each node in its parent's child list (-1 for roots)
+    const int32_t *cont;  // first child of a non-root node (its chain goes on there), else -1
 };
 
 template <class T> struct TreeBufs {
@@ -300,7 +304,7 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leave
 
 template <class T, bool FULL>
 __global__ void __launch_bounds__(TWARPS * 32)
-tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *nodes, int64_t count)
+tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *heads, int64_t count)
 {
     using namespace w16;
     constexpr int E = SL<T>::ELEMS;
@@ -316,32 +320,52 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
     const int b = p.b;
     const int64_t bb = (int64_t)b * b;
     const unsigned long long cnt = (unsigned long long)count;
+    auto prefetch = [&](int32_t u, int c) {
+        load_block_async<T, FULL>(sBuf(c), p.edge + u * bb, b, lane);
+        stage_lower_slot<T>(stg(c), p.ws_sinv + (int64_t)u * SLOT_ELEMS, lane, g, t);
+        cp_async_commit();
+    };
 
-    // Nodes are taken one ahead: the next node's edge block and S^-1 slot
-    // stream in while the current one is computed (its loads are issued after
-    // the current G_pp load, so waiting for "all but the newest group" waits
-    // for exactly the current node's data).
-    unsigned long long k = warp_take(sy.counters + 1, lane);
-    int cur = 0;
-    if (k < cnt) {
-        const int32_t v0 = nodes[k];
-        load_block_async<T, FULL>(sBuf(0), p.edge + v0 * bb, b, lane);
-        stage_lower_slot<T>(stg(0), p.ws_sinv + (int64_t)v0 * SLOT_ELEMS, lane, g, t);
-        cp_async_commit();
+    // A warp takes a chain head from the depth-ordered list (every non-root
+    // node except the first child of a non-root parent), waits for its parent's
+    // flag and reads G_pp, then runs down the chain of first children: each
+    // one's G_pp is the G_vv the warp has just formed, in registers, so it
+    // neither waits nor loads it.  The next node (the first child, or the next
+    // head) is known before the current one is computed, and its edge block
+    // and S^-1 slot stream in meanwhile (waiting for "all but the newest group"
+    // waits for exactly the current node's data and G_pp).
+    int32_t v;
+    {
+        const unsigned long long k = warp_take(sy.counters + 1, lane);
+        v = k < cnt ? heads[k] : -1;
     }
-    while (k < cnt) {
-        const int32_t v = nodes[k];
+    int cur = 0;
+    if (v >= 0) prefetch(v, 0);
+    bool head = true;                                 // v came from the list
+    bool failed = false;                              // the chain's head gave up
+    Tile<T> G;                                        // G_vv of the node before v in its chain
+    zero(G);
+    while (v >= 0) {
         const int32_t par = td.parent[v];
-        const unsigned long long kn = warp_take(sy.counters + 1, lane);
-        const int ok = wait_parent(sy.done + par, td.spin_limit, lane, 64);   // G_pp (bounded wait)
-        __syncwarp();                                 // every lane's reads below are ordered after lane 0's acquire
-        if (ok) load_lower_async<T, FULL>(sG, p.G_diag + (int64_t)par * bb, b, lane);   // G_pp, from L2
-        cp_async_commit();
-        if (kn < cnt) {
-            const int32_t vn = nodes[kn];
-            load_block_async<T, FULL>(sBuf(cur ^ 1), p.edge + vn * bb, b, lane);
-            stage_lower_slot<T>(stg(cur ^ 1), p.ws_sinv + (int64_t)vn * SLOT_ELEMS, lane, g, t);
+        const int32_t c = td.cont[v];
+        int ok;
+        if (head) {
+            ok = wait_parent(sy.done + par, td.spin_limit, lane, 64);   // G_pp (bounded wait)
+            __syncwarp();                             // every lane's reads below are ordered after lane 0's acquire
+            if (ok) load_lower_async<T, FULL>(sG, p.G_diag + (int64_t)par * bb, b, lane);   // G_pp, from L2
             cp_async_commit();
+            failed = !ok;
+        } else {
+            failed = failed || par == td.hold;        // a withheld node's flag would never have come
+            ok = !failed;
+        }
+        int32_t nxt = c;
+        if (c < 0) {
+            const unsigned long long kn = warp_take(sy.counters + 1, lane);
+            nxt = kn < cnt ? heads[kn] : -1;
+        }
+        if (nxt >= 0) {
+            prefetch(nxt, cur ^ 1);
             cp_async_wait_one();
         } else {
             cp_async_wait_all();
@@ -349,35 +373,35 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *no
         __syncwarp();
         if (!ok) {                                    // the parent never published: report, pass it on
             give_up(p.info, sy.done, td, v, lane);
-            k = kn;
-            cur ^= 1;
-            continue;
+        } else {
+            Tile<T> a;
+            unstage_lower_slot<T>(a, stg(cur), lane, g, t);
+            to_smem<T>(sT, a, g, t);                  // lower entries of S_v^-1 valid
+            __syncwarp();
+            from_smem_lower<T>(a, sT, g, t);          // S_v^-1, full
+            Tile<T> gp, et, wt, get;
+            if (head) from_smem_lower<T>(gp, sG, g, t);   // G_pp, full
+            else gp = G;
+            from_smem<T>(et, sBuf(cur), g, t);        // E_v
+            // W_v^T = S_v^-1 E_v^T and G_edge[v]^T = -W_v^T G_pp are X Y^T products of
+            // register tiles (S_v^-1, G_pp symmetric): nothing is transposed.
+            zero(wt);
+            gemm_nt<false>(wt, a, et, sT, sT2, g, t); // W_v^T = S_v^-1 E_v^T
+            zero(get);
+            gemm_nt<true>(get, wt, gp, sT, sT2, g, t);   // G_edge[v]^T = -W_v^T G_pp
+            store_block_T<T, FULL>(p.G_edge + v * bb, get, b, g, t);
+            gemm_nt<true, true>(a, wt, get, sT, sT2, g, t);   // G_vv = S_v^-1 - W_v^T G_edge[v] (lower tiles)
+            __syncwarp();
+            to_smem<T>(sT, a, g, t);
+            __syncwarp();
+            from_smem_lower<T>(G, sT, g, t);          // exactly symmetric
+            store_block<T, FULL>(p.G_diag + v * bb, G, b, g, t);
+            __syncwarp();                             // the warp's stores are ordered before lane 0's release
+            if (td.child_ptr[v + 1] - td.child_ptr[v] >= 2) publish(sy.done, td, v, lane);   // heads wait on it
+            __syncwarp();
         }
-        Tile<T> a;
-        unstage_lower_slot<T>(a, stg(cur), lane, g, t);
-        to_smem<T>(sT, a, g, t);                      // lower entries of S_v^-1 valid
-        __syncwarp();
-        from_smem_lower<T>(a, sT, g, t);              // S_v^-1, full
-        Tile<T> gp, et, wt, get;
-        from_smem_lower<T>(gp, sG, g, t);             // G_pp, full
-        from_smem<T>(et, sBuf(cur), g, t);            // E_v
-        // W_v^T = S_v^-1 E_v^T and G_edge[v]^T = -W_v^T G_pp are X Y^T products of
-        // register tiles (S_v^-1, G_pp symmetric): nothing is transposed.
-        zero(wt);
-        gemm_nt<false>(wt, a, et, sT, sT2, g, t);     // W_v^T = S_v^-1 E_v^T
-        zero(get);
-        gemm_nt<true>(get, wt, gp, sT, sT2, g, t);    // G_edge[v]^T = -W_v^T G_pp
-        store_block_T<T, FULL>(p.G_edge + v * bb, get, b, g, t);
-        gemm_nt<true, true>(a, wt, get, sT, sT2, g, t);   // G_vv = S_v^-1 - W_v^T G_edge[v] (lower tiles)
-        __syncwarp();
-        to_smem<T>(sT, a, g, t);
-        __syncwarp();
-        from_smem_lower<T>(a, sT, g, t);              // exactly symmetric
-        store_block<T, FULL>(p.G_diag + v * bb, a, b, g, t);
-        __syncwarp();                                 // the warp's stores are ordered before lane 0's release
-        if (td.child_ptr[v + 1] > td.child_ptr[v]) publish(sy.done, td, v, lane);   // only parents are waited for
-        __syncwarp();
-        k = kn;
+        head = c < 0;
+        v = nxt;
         cur ^= 1;
     }
 }
@@ -820,7 +844,8 @@ cudaError_t run_tree(const selinv_tree_plan_s *pl, int b, const T *diag, const T
     sy.counters = reinterpret_cast<unsigned long long *>(w);
     p.info = info;
     p.b = b;
-    TreeDev td{pl->d_child_ptr, pl->d_child_idx, pl->d_parent, pl->n, pl->spin_limit, pl->hold, pl->d_cpos};
+    TreeDev td{pl->d_child_ptr, pl->d_child_idx, pl->d_parent, pl->n, pl->spin_limit, pl->hold, pl->d_cpos,
+                pl->d_cont};
 
     const int64_t init_n = std::max<int64_t>(N, pl->trees);
     tree_init<<<(unsigned)ceil_div(init_n, 256), 256, 0, s>>>(pl->d_child_ptr, N, sy.pending, sy.done, sy.counters,
@@ -854,8 +879,8 @@ cudaError_t run_tree(const selinv_tree_plan_s *pl, int b, const T *diag, const T
         const int64_t bw = std::min<int64_t>((int64_t)sms * 4, ceil_div(ceil_div(ndist, DCHUNK), wpb));
         kw<<<(unsigned)bw, DRAW_THREADS, 0, s>>>(p, td, sy, pl->d_dist_nodes, ndist);
     } else if (ndist > 0) {
-        const int64_t bd = std::min<int64_t>((int64_t)sms * occ_d, ceil_div(ndist, TWARPS));
-        kd<<<(unsigned)bd, TWARPS * 32, smem_d, s>>>(p, td, sy, pl->d_dist_nodes, ndist);
+        const int64_t bd = std::min<int64_t>((int64_t)sms * occ_d, ceil_div(pl->nheads, TWARPS));
+        kd<<<(unsigned)bd, TWARPS * 32, smem_d, s>>>(p, td, sy, pl->d_heads, pl->nheads);
     }
     tree_finalize<<<(unsigned)pl->trees, FIN_THREADS, 0, s>>>(p.ws_ld, pl->n, logdet, info);
     return cudaGetLastError();
@@ -900,7 +925,8 @@ cudaError_t run_tree_backward(const selinv_tree_plan_s *pl, int b, const T *diag
     sy.counters = reinterpret_cast<unsigned long long *>(w);
     p.info = info;
     p.b = b;
-    TreeDev td{pl->d_child_ptr, pl->d_child_idx, pl->d_parent, pl->n, pl->spin_limit, pl->hold, pl->d_cpos};
+    TreeDev td{pl->d_child_ptr, pl->d_child_idx, pl->d_parent, pl->n, pl->spin_limit, pl->hold, pl->d_cpos,
+                pl->d_cont};
 
     const int64_t init_n = std::max<int64_t>(N, pl->trees);
     tree_init<<<(unsigned)ceil_div(init_n, 256), 256, 0, s>>>(pl->d_child_ptr, N, sy.pending, sy.done, sy.counters,
@@ -1041,10 +1067,21 @@ static selinv_status tree_plan_impl(const int32_t *parent, int64_t trees, int64_
     up(&pl->d_child_ptr, cnt);
     up(&pl->d_child_idx, child);
     {
-        std::vector<int32_t> cpos(N, -1);
+        std::vector<int32_t> cpos(N, -1), cont(N, -1), heads;
         for (int64_t v = 0; v < N; ++v)
             for (int32_t c = cnt[v]; c < cnt[v + 1]; ++c) cpos[child[c]] = c;
+        for (int64_t v = 0; v < N; ++v)
+            if (gparent[v] >= 0 && cnt[v + 1] > cnt[v]) cont[v] = child[cnt[v]];
+        heads.reserve(dnodes.size());
+        for (int64_t i = 0; i < pl->dist_off[Dm]; ++i) {   // depth order, ascending ids within a depth
+            const int32_t v = dnodes[i];
+            if (cont[gparent[v]] != v) heads.push_back(v);
+        }
+        pl->nheads = (int64_t)heads.size();
+        if (heads.empty()) heads.push_back(0);
         up(&pl->d_cpos, cpos);
+        up(&pl->d_cont, cont);
+        up(&pl->d_heads, heads);
     }
     up(&pl->d_parent, gparent);
     if (!ok) return SELINV_ERR_CUDA;
@@ -1074,6 +1111,8 @@ void selinv_tree_plan_free(selinv_tree_plan_t *pl)
     cudaFree(pl->d_child_ptr);
     cudaFree(pl->d_child_idx);
     cudaFree(pl->d_cpos);
+    cudaFree(pl->d_cont);
+    cudaFree(pl->d_heads);
     cudaFree(pl->d_parent);
     delete pl;
 }
