@@ -530,7 +530,7 @@ def build_step(w, dtype, op, batch, elems):
                 selinv.tree_backward(plan, dev_in["diag"], dev_in["edge"], dev_in["G_diag"], dev_in["G_edge"],
                                      dev_in["Gb_diag"], dev_in["Gb_edge"], check=False, out=out, workspace=ws)
         elif op == "sample":
-            kernel = "tree_collect_kernel (draw mode)"
+            kernel = "tree_collect_draw_kernel"
             out = {"eta": torch.empty_like(dev_in["z"]), "logdet": out["logdet"], "info": out["info"]}
 
             def step():

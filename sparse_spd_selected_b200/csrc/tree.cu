@@ -178,9 +178,9 @@ template <class T> SELINV_DEVINL void load_lower_slot_l2(w16::Tile<T> &a, const 
     }
 }
 
-template <class T, bool FULL, bool DRAW = false>
-__global__ void __launch_bounds__(TWARPS * 32)
-tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leaves, int64_t nleaves)
+template <class T, bool FULL, bool DRAW>
+SELINV_DEVINL void collect_sweep(const TreeBufs<T> &p, const TreeDev &td, const TreeSync &sy, const int32_t *leaves,
+                                 int64_t nleaves)
 {
     using namespace w16;
     constexpr int E = SL<T>::ELEMS;
@@ -300,6 +300,22 @@ tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leave
             v = par;
         }
     }
+}
+
+// The collect sweep without and with the draws' extra state; the draw
+// variant is held to 96 registers so that five CTAs fit an SM, as for the
+// plain sweep.
+template <class T, bool FULL>
+__global__ void __launch_bounds__(TWARPS * 32)
+tree_collect_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leaves, int64_t nleaves)
+{
+    collect_sweep<T, FULL, false>(p, td, sy, leaves, nleaves);
+}
+template <class T, bool FULL>
+__global__ void __launch_bounds__(TWARPS * 32, 5)
+tree_collect_draw_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *leaves, int64_t nleaves)
+{
+    collect_sweep<T, FULL, true>(p, td, sy, leaves, nleaves);
 }
 
 template <class T, bool FULL>
@@ -852,7 +868,7 @@ cudaError_t run_tree(const selinv_tree_plan_s *pl, int b, const T *diag, const T
                                                                info, pl->trees);
     const size_t smem = sizeof(T) * tree_smem_elems<T>() * TWARPS;
     const size_t smem_d = sizeof(T) * dist_smem_elems<T>() * TWARPS;
-    auto kc = draw ? (full ? tree_collect_kernel<T, true, true> : tree_collect_kernel<T, false, true>)
+    auto kc = draw ? (full ? tree_collect_draw_kernel<T, true> : tree_collect_draw_kernel<T, false>)
                    : (full ? tree_collect_kernel<T, true> : tree_collect_kernel<T, false>);
     auto kd = full ? tree_distribute_kernel<T, true> : tree_distribute_kernel<T, false>;
     auto kw = full ? tree_draw_kernel<T, true> : tree_draw_kernel<T, false>;
