@@ -714,38 +714,62 @@ tree_bw_distribute_kernel(TreeBwdBufs<T> p, TreeDev td, TreeSync sy, const int32
     const int b = p.b;
     const int64_t bb = (int64_t)b * b;
     const unsigned long long cnt = (unsigned long long)count;
-    // Nodes are taken one ahead and the next node's operands sent toward L2
-    // while the current one waits and computes.  Every wait still ends: the
-    // smallest unfinished node is always some warp's current node (a node
-    // held as "next" comes after its warp's current one), and its parent,
-    // earlier in the depth order, is finished.
-    unsigned long long k = warp_take(sy.counters + 1, lane);
-    while (k < cnt) {
-        const unsigned long long kn = warp_take(sy.counters + 1, lane);
-        if (kn < cnt) {
-            const int32_t vn = nodes[kn];
-            prefetch_range_l2(p.ws_P + (int64_t)vn * SLOT_ELEMS, SLOT_ELEMS, lane, 32);
-            prefetch_range_l2(p.ws_Pd + (int64_t)vn * SLOT_ELEMS, SLOT_ELEMS, lane, 32);
-            prefetch_range_l2(p.edge + vn * bb, bb, lane, 32);
-            prefetch_range_l2(p.Eb + vn * bb, bb, lane, 32);
-        }
-        const int32_t v = nodes[k];
+    // The distribute sweep's chains, reversed: a warp takes a chain head (every
+    // non-root node except the first child of a non-root parent) in depth order,
+    // waits for its parent's flag and reads Sg_p, then runs down the chain of
+    // first children, each one's Sg_p being the Sg_v the warp has just formed.
+    // The next node (first child, or next head) is known before the current one
+    // is computed, and its operands are sent toward L2 meanwhile.  Every wait
+    // still ends: the smallest unfinished head is some warp's current node, and
+    // its parent, earlier in the depth order or earlier in a running chain, is
+    // finished or being finished by a warp that waits on nothing later.
+    int32_t v;
+    {
+        const unsigned long long k = warp_take(sy.counters + 1, lane);
+        v = k < cnt ? nodes[k] : -1;
+    }
+    bool head = true, failed = false;
+    Tile<T> Sn;                                       // Sg_v of the node before v in its chain
+    zero(Sn);
+    while (v >= 0) {
         const int32_t par = td.parent[v];
-        k = kn;
+        const int32_t c = td.cont[v];
+        int32_t nxt = c;
+        if (c < 0) {
+            const unsigned long long kn = warp_take(sy.counters + 1, lane);
+            nxt = kn < cnt ? nodes[kn] : -1;
+        }
+        if (nxt >= 0) {
+            prefetch_range_l2(p.ws_P + (int64_t)nxt * SLOT_ELEMS, SLOT_ELEMS, lane, 32);
+            prefetch_range_l2(p.ws_Pd + (int64_t)nxt * SLOT_ELEMS, SLOT_ELEMS, lane, 32);
+            prefetch_range_l2(p.edge + nxt * bb, bb, lane, 32);
+            prefetch_range_l2(p.Eb + nxt * bb, bb, lane, 32);
+        }
         // operands that do not depend on the parent first
         Tile<T> P, Pt, Ev, ed;
         sym_from_slot<T>(P, p.ws_P + (int64_t)v * SLOT_ELEMS, s0, lane, g, t);
         sym_from_slot<T>(Pt, p.ws_Pd + (int64_t)v * SLOT_ELEMS, s0, lane, g, t);
         load_gen<T, FULL>(Ev, p.edge + v * bb, b, g, t, false);
         load_gen<T, FULL>(ed, p.Eb + v * bb, b, g, t, true);
-        const int ok = wait_parent(sy.done + par, td.spin_limit, lane, 64);   // Sg_p (bounded wait)
-        __syncwarp();                                 // every lane's reads below follow lane 0's acquire
+        int ok;
+        if (head) {
+            ok = wait_parent(sy.done + par, td.spin_limit, lane, 64);   // Sg_p (bounded wait)
+            __syncwarp();                             // every lane's reads below follow lane 0's acquire
+            failed = !ok;
+        } else {
+            failed = failed || par == td.hold;        // a withheld node's flag would never have come
+            ok = !failed;
+        }
+        const bool was_head = head;
+        head = c < 0;
         if (!ok) {                                    // the parent never published: report, pass it on
             give_up(p.info, sy.done, td, v, lane);
+            v = nxt;
             continue;
         }
         Tile<T> Sp, ET;
-        sym_from_slot<T>(Sp, p.ws_U + (int64_t)par * SLOT_ELEMS, s0, lane, g, t);
+        if (was_head) sym_from_slot<T>(Sp, p.ws_U + (int64_t)par * SLOT_ELEMS, s0, lane, g, t);
+        else Sp = Sn;
         transpose_t<T>(ET, Ev, s0, g, t);
         {
             Tile<T> zt;
@@ -767,12 +791,20 @@ tree_bw_distribute_kernel(TreeBwdBufs<T> p, TreeDev td, TreeSync sy, const int32
         gemm_nt<true, true>(sg, q, P, s1, s2, g, t);              // Sg_v = -P Pt P (lower tiles)
         mirror_upper(sg, g, t);
         store_db<T, FULL>(p.Db + v * bb, sg, b, g, t);
-        if (td.child_ptr[v + 1] > td.child_ptr[v]) {
+        if (td.child_ptr[v + 1] - td.child_ptr[v] >= 2) {          // chain heads below wait for it
             store_lower_slot<T>(p.ws_U + (int64_t)v * SLOT_ELEMS, sg, lane, g, t);
             __syncwarp();                             // the warp's stores are ordered before lane 0's release
             publish(sy.done, td, v, lane);
             __syncwarp();
         }
+        if (c >= 0) {                                 // the first child's Sg_p: exactly symmetric, as read back
+            __syncwarp();
+            to_smem<T>(s0, sg, g, t);
+            __syncwarp();
+            from_smem_lower<T>(Sn, s0, g, t);
+            __syncwarp();
+        }
+        v = nxt;
     }
 }
 
@@ -966,8 +998,8 @@ cudaError_t run_tree_backward(const selinv_tree_plan_s *pl, int b, const T *diag
     const int64_t bc = std::min<int64_t>((int64_t)sms * occ_c, std::max<int64_t>(1, ceil_div(nleaves, TWARPS)));
     kc<<<(unsigned)bc, TWARPS * 32, smem, s>>>(p, td, sy, pl->d_collect_nodes, nleaves);
     if (ndist > 0) {
-        const int64_t bd = std::min<int64_t>((int64_t)sms * occ_d, ceil_div(ndist, TWARPS));
-        kd<<<(unsigned)bd, TWARPS * 32, smem, s>>>(p, td, sy, pl->d_dist_nodes, ndist);
+        const int64_t bd = std::min<int64_t>((int64_t)sms * occ_d, ceil_div(pl->nheads, TWARPS));
+        kd<<<(unsigned)bd, TWARPS * 32, smem, s>>>(p, td, sy, pl->d_heads, pl->nheads);
     }
     tree_info_finalize<<<(unsigned)ceil_div(pl->trees, 256), 256, 0, s>>>(info, pl->trees);
     return cudaGetLastError();
