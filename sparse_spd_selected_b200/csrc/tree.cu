@@ -424,78 +424,99 @@ tree_distribute_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *he
 
 // Draws, top-down: w_v = u_v - W_v^T w_p with u_v = R_v^-T z_v and W_v^T
 // left by the collect sweep (W_v^T as a 16 x 16 row-major slot, zero outside
-// b x b) and w_p published by the parent.  A warp takes DCHUNK consecutive
-// nodes of the depth order per atomic and loads all their W_v^T rows and u_v
-// before it waits for the first parent.  Lane (r, hf) = (lane / 2, lane % 2)
-// holds row r, columns 8 hf .. 8 hf + 7.  Every wait ends: a node's parent
-// comes earlier in the order, in an earlier chunk (taken by a running warp) or
-// earlier in the same chunk.
-constexpr int DCHUNK = 4;
+// b x b) and w_p published by the parent (or, along a chain, just formed by
+// the same warp).  Lane (r, hf) = (lane / 2, lane % 2) holds row r, columns
+// 8 hf .. 8 hf + 7.  Every wait ends: a head's parent was handed out earlier,
+// to a warp that is running and waits on nothing later.
 constexpr int DRAW_THREADS = 256;
 
 template <class T, bool FULL>
 __global__ void __launch_bounds__(DRAW_THREADS)
-tree_draw_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *nodes, int64_t count)
+tree_draw_kernel(TreeBufs<T> p, TreeDev td, TreeSync sy, const int32_t *heads, int64_t count)
 {
     const int lane = threadIdx.x & 31;
     const int r = lane >> 1, hf = lane & 1;
     const int b = p.b;
-    for (;;) {
-        const int64_t k0 = (int64_t)warp_take(sy.counters + 1, lane) * DCHUNK;
-        if (k0 >= count) break;
-        const int m = (int)(count - k0 < DCHUNK ? count - k0 : DCHUNK);
-        T wr[DCHUNK][8], uv[DCHUNK];
-        int32_t vs[DCHUNK], ps[DCHUNK];
+    // W_v^T row r (the lane's eight columns) and u_v[r] of node u
+    auto load_node = [&](int32_t u, T w[8], T &uu) {
+        const T *row = p.ws_sinv + (int64_t)u * DRAW_SLOT + r * 16 + 8 * hf;
+        if constexpr (sizeof(T) == 8) {
 #pragma unroll
-        for (int j = 0; j < DCHUNK; ++j) {
-            vs[j] = j < m ? nodes[k0 + j] : 0;
-            ps[j] = j < m ? td.parent[vs[j]] : 0;
-            const T *row = p.ws_sinv + (int64_t)vs[j] * DRAW_SLOT + r * 16 + 8 * hf;
-            if (j < m) {
-                if constexpr (sizeof(T) == 8) {
+            for (int c = 0; c < 8; c += 2) {
+                const double2 x = __ldcs(reinterpret_cast<const double2 *>(row + c));
+                w[c] = x.x;
+                w[c + 1] = x.y;
+            }
+        } else {
 #pragma unroll
-                    for (int c = 0; c < 8; c += 2) {
-                        const double2 x = __ldcs(reinterpret_cast<const double2 *>(row + c));
-                        wr[j][c] = x.x;
-                        wr[j][c + 1] = x.y;
-                    }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 8; c += 4) {
-                        const float4 x = __ldcs(reinterpret_cast<const float4 *>(row + c));
-                        wr[j][c] = x.x;
-                        wr[j][c + 1] = x.y;
-                        wr[j][c + 2] = x.z;
-                        wr[j][c + 3] = x.w;
-                    }
-                }
-                uv[j] = r < b ? p.eta[(int64_t)vs[j] * b + r] : T(0);
-            } else {
-#pragma unroll
-                for (int c = 0; c < 8; ++c) wr[j][c] = T(0);
-                uv[j] = T(0);
+            for (int c = 0; c < 8; c += 4) {
+                const float4 x = __ldcs(reinterpret_cast<const float4 *>(row + c));
+                w[c] = x.x;
+                w[c + 1] = x.y;
+                w[c + 2] = x.z;
+                w[c + 3] = x.w;
             }
         }
+        uu = r < b ? p.eta[(int64_t)u * b + r] : T(0);
+    };
+    // The distribute sweep's chains: a warp takes a chain head, waits for its
+    // parent's w_p, and runs down the chain of first children, each one's w_p
+    // being the w_v it has just formed (moved to the lanes' columns by
+    // shuffles); the next node's W^T row and u are loaded before the current
+    // one's wait.  A warp holds no other node while it waits, so a wait that
+    // runs out in one tree delays no other tree.
+    for (;;) {
+        const unsigned long long k = warp_take(sy.counters + 1, lane);
+        if (k >= (unsigned long long)count) break;
+        int32_t v = heads[k];
+        T w[8], u;
+        load_node(v, w, u);
+        bool head = true, failed = false;
+        T wp[8];                                      // w_p at the lane's columns 8 hf .. 8 hf + 7
 #pragma unroll
-        for (int j = 0; j < DCHUNK; ++j) {
-            if (j >= m) break;
-            const int32_t v = vs[j], par = ps[j];
-            const int ok = wait_parent(sy.done + par, td.spin_limit, lane, 32);   // w_p (bounded wait)
-            __syncwarp();                             // every lane's reads below follow lane 0's acquire
+        for (int c = 0; c < 8; ++c) wp[c] = T(0);
+        while (v >= 0) {
+            const int32_t par = td.parent[v];
+            const int32_t cn = td.cont[v];
+            T wn[8], un = T(0);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) wn[c] = T(0);
+            if (cn >= 0) load_node(cn, wn, un);
+            int ok;
+            if (head) {
+                ok = wait_parent(sy.done + par, td.spin_limit, lane, 32);   // w_p (bounded wait)
+                __syncwarp();                         // every lane's reads below follow lane 0's acquire
+                failed = !ok;
+                if (ok) {
+                    const T *src = p.eta + (int64_t)par * b + 8 * hf;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) wp[c] = (FULL || 8 * hf + c < b) ? __ldcg(src + c) : T(0);
+                }
+            } else {
+                failed = failed || par == td.hold;    // a withheld node's flag would never have come
+                ok = !failed;
+            }
             if (!ok) {                                // the parent never published: report, pass it on
                 give_up(p.info, sy.done, td, v, lane);
-                continue;
-            }
-            const T *wp = p.eta + (int64_t)par * b + 8 * hf;
-            T s2 = T(0);
+            } else {
+                T s2 = T(0);
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                if (FULL || 8 * hf + c < b) s2 = fma(wr[j][c], __ldcg(wp + c), s2);
-            s2 += shfl_xor(s2, 1);
-            if (hf == 0 && r < b) p.eta[(int64_t)v * b + r] = uv[j] - s2;
-            __syncwarp();                             // the warp's stores are ordered before lane 0's release
-            if (td.child_ptr[v + 1] > td.child_ptr[v]) publish(sy.done, td, v, lane);
-            __syncwarp();
+                for (int c = 0; c < 8; ++c)
+                    if (FULL || 8 * hf + c < b) s2 = fma(w[c], wp[c], s2);
+                s2 += shfl_xor(s2, 1);
+                const T wv = u - s2;                  // w_v[r] (zero for r >= b)
+                if (hf == 0 && r < b) p.eta[(int64_t)v * b + r] = wv;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) wp[c] = __shfl_sync(FULL_MASK, wv, 2 * (8 * hf + c));
+                __syncwarp();                         // the warp's stores are ordered before lane 0's release
+                if (td.child_ptr[v + 1] - td.child_ptr[v] >= 2) publish(sy.done, td, v, lane);   // heads wait on it
+                __syncwarp();
+            }
+            head = cn < 0;
+            v = cn;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) w[c] = wn[c];
+            u = un;
         }
     }
 }
@@ -924,8 +945,8 @@ cudaError_t run_tree(const selinv_tree_plan_s *pl, int b, const T *diag, const T
     kc<<<(unsigned)bc, TWARPS * 32, smem, s>>>(p, td, sy, pl->d_collect_nodes, nleaves);
     if (ndist > 0 && draw) {
         const int64_t wpb = DRAW_THREADS / 32;
-        const int64_t bw = std::min<int64_t>((int64_t)sms * 4, ceil_div(ceil_div(ndist, DCHUNK), wpb));
-        kw<<<(unsigned)bw, DRAW_THREADS, 0, s>>>(p, td, sy, pl->d_dist_nodes, ndist);
+        const int64_t bw = std::min<int64_t>((int64_t)sms * 4, ceil_div(pl->nheads, wpb));
+        kw<<<(unsigned)bw, DRAW_THREADS, 0, s>>>(p, td, sy, pl->d_heads, pl->nheads);
     } else if (ndist > 0) {
         const int64_t bd = std::min<int64_t>((int64_t)sms * occ_d, ceil_div(pl->nheads, TWARPS));
         kd<<<(unsigned)bd, TWARPS * 32, smem_d, s>>>(p, td, sy, pl->d_heads, pl->nheads);
