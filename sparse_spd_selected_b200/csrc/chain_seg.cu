@@ -93,9 +93,9 @@ template <class T> struct SegLay {
     static constexpr int IMG = 4 * E;
     static constexpr int SCR = sizeof(T) == 4 ? 2 * E * GW : 0;
     static constexpr int CBN = sizeof(T) == 8 ? QSCHUR : 64;
-    // collect: C, D, X (S^-1), Y (W), V, F
-    static constexpr int C = 0, D = IMG, X = 2 * IMG, Y = 3 * IMG, V = 4 * IMG, F = 5 * IMG;
-    static constexpr int CS = 6 * IMG, CCB = CS + SCR, CTOTAL = CCB + CBN;
+    // collect: C, D, X (S^-1), Y (W), V, F (two buffers)
+    static constexpr int C = 0, D = IMG, X = 2 * IMG, Y = 3 * IMG, V = 4 * IMG, F = 5 * IMG, F2 = 6 * IMG;
+    static constexpr int CS = 7 * IMG, CCB = CS + SCR, CTOTAL = CCB + CBN;
     // distribute: A (G_next), B (G_{s,next}), Cg (G_{next,j}), Dg (G_{s,j}), W x 2, V x 2, S
     // (S: quadrant image slots (0,0), (1,0), (1,1) of a four-quadrant image)
     static constexpr int A = 0, B = IMG, CG = 2 * IMG, DG = 3 * IMG, W0 = 4 * IMG, V0 = 6 * IMG, S0 = 8 * IMG;
@@ -149,7 +149,8 @@ __global__ void __launch_bounds__(GT, 3) seg_collect_kernel(ChainArgs<T> p, SegA
     // are widened as they are read; every other image is float64
     T *sC = reinterpret_cast<T *>(base + Ly::C), *sD = reinterpret_cast<T *>(base + Ly::D);
     C *sX = base + Ly::X, *sY = base + Ly::Y;
-    C *sV = base + Ly::V, *sF = base + Ly::F;
+    C *sV = base + Ly::V;
+    auto sFb = [&](int64_t j) { return base + ((j & 1) ? Ly::F2 : Ly::F); };   // F_j
     C *s1 = nullptr, *s2 = nullptr;             // float64 products need no scratch
     C *cb = base + Ly::CCB;
 
@@ -171,7 +172,7 @@ __global__ void __launch_bounds__(GT, 3) seg_collect_kernel(ChainArgs<T> p, SegA
     zero(u);
 
     load_diag<T, FULL>(sD, Dg + node(0) * bb, b, gtid);
-    if (sp.fill) load_full_f64<T, FULL>(sF, Bg + (sp.lo - 1) * bb, b, gtid);   // F = A_{lo, s} = B_s
+    if (sp.fill) load_full_f64<T, FULL>(sFb(0), Bg + (sp.lo - 1) * bb, b, gtid);   // F = A_{lo, s} = B_s
     cp_async_commit();
     cp_async_wait_all();
     group_bar(bar);
@@ -182,9 +183,22 @@ __global__ void __launch_bounds__(GT, 3) seg_collect_kernel(ChainArgs<T> p, SegA
     cp_async_commit();
 
     Tile<C> fn;
+    const bool upper = I == 0 && J == 1;
+    // Interior segments: F_{j+1} = -W_j F_j and U_s += V_j F_j do not feed
+    // S_{j+1}, so they run while block j+1's inverse keeps the group waiting
+    // (warp (0,0) while (1,1) inverts S, the others while (0,0) inverts A).
+    bool pend = false;
     for (int64_t j = 0; j < n; ++j) {
         bool bad = false;
-        qinverse<C>(a, cb, I, J, g, t, bar, det, bad);              // a = S_j^-1
+        auto idle = [&](int phase) {
+            if (!pend || phase != ((I == 0 && J == 0) ? 3 : 1)) return;
+            Tile<C> f;
+            zero(f);
+            qgemm<true, false, true, false>(f, sY, sFb(j - 1), I, J, s1, s2, g, t);   // F_j = -W_{j-1} F_{j-1}
+            to_smem<C>(quad(sFb(j), I, J), f, g, t);
+            if (!upper) qgemm<false, false, true, false>(u, sV, sFb(j - 1), I, J, s1, s2, g, t);   // U_s += V F
+        };
+        qinverse<C>(a, cb, I, J, g, t, bar, det, bad, idle);        // a = S_j^-1
         if (bad && fail < 0) fail = (int)node(j);
         to_smem<C>(quad(sX, I, J), a, g, t);
         cp_async_wait_all();
@@ -201,7 +215,7 @@ __global__ void __launch_bounds__(GT, 3) seg_collect_kernel(ChainArgs<T> p, SegA
         to_smem<C>(quad(sY, I, J), w, g, t);
         if (sp.fill) {
             zero(v);
-            qgemm<false, true, false, false>(v, sF, sX, I, J, s1, s2, g, t);        // V_j = F_j^T S_j^-1
+            qgemm<false, true, false, false>(v, sFb(j), sX, I, J, s1, s2, g, t);    // V_j = F_j^T S_j^-1
             to_smem<C>(quad(sV, I, J), v, g, t);
         }
         group_bar(bar);
@@ -213,21 +227,20 @@ __global__ void __launch_bounds__(GT, 3) seg_collect_kernel(ChainArgs<T> p, SegA
         // S_next and U_s are symmetric and only their lower quadrants are ever
         // read (the next inverse starts from quadrants (0,0), (1,0), (1,1); the
         // separators' D' is read on its lower triangle): warp (0,1) skips them.
-        const bool upper = I == 0 && J == 1;
         if (last || upper) zero(a);                                   // the separator's contribution only
         else sym_quad<C>(a, sD, I, J, g, t);                          // D_next
         if (!upper) {
             if (sp.down) qgemm<true, false, true, false>(a, sY, sC, I, J, s1, s2, g, t);   // S_next -= W_j C_j^T
             else qgemm<true, false, false, false>(a, sY, sC, I, J, s1, s2, g, t);
         }
-        if (sp.fill) {
+        if (sp.fill && last) {                                        // the last block's, at once
             zero(fn);
-            qgemm<true, false, true, false>(fn, sY, sF, I, J, s1, s2, g, t);         // F_next = -W_j F_j
-            if (!upper) qgemm<false, false, true, false>(u, sV, sF, I, J, s1, s2, g, t);   // U_s += V_j F_j
+            qgemm<true, false, true, false>(fn, sY, sFb(j), I, J, s1, s2, g, t);     // F_next = -W_j F_j
+            if (!upper) qgemm<false, false, true, false>(u, sV, sFb(j), I, J, s1, s2, g, t);   // U_s += V_j F_j
         }
+        pend = sp.fill && !last;
         group_bar(bar);
         if (!last) {
-            if (sp.fill) to_smem<C>(quad(sF, I, J), fn, g, t);
             load_full<T, FULL>(sC, Bg + cpl(j + 1) * bb, b, gtid);
             if (j + 2 < n) load_diag<T, FULL>(sD, Dg + node(j + 2) * bb, b, gtid);
             cp_async_commit();

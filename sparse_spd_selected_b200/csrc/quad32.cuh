@@ -208,10 +208,18 @@ SELINV_DEVINL void qinverse_scalar(w16::Tile<T> &a, T *cbuf, int I, int J, int g
 // (two 8-pivot block steps, warp16.cuh; pivots -> det, bad), so the group
 // meets at three barriers only; every product is a register-register FP64
 // tensor-core product with operands from four 16 x 16 images in buf.
+// `idle(phase)` is called by every warp in phases 1 (while warp (0,0) inverts
+// A) and 3 (while warp (1,1) inverts S), so that a caller can give the warps
+// that wait there independent work; it must not touch `buf`.
 constexpr int QSCHUR = 4 * w16::SL<double>::ELEMS;
 
+struct NoIdle {
+    SELINV_DEVINL void operator()(int) const {}
+};
+
+template <class Idle = NoIdle>
 SELINV_DEVINL void qinverse_schur(w16::Tile<double> &a, double *buf, int I, int J, int g, int t, int bar,
-                                  LogAcc &det, bool &bad)
+                                  LogAcc &det, bool &bad, const Idle &idle = Idle())
 {
     using namespace w16;
     constexpr int E = SL<double>::ELEMS;
@@ -223,6 +231,7 @@ SELINV_DEVINL void qinverse_schur(w16::Tile<double> &a, double *buf, int I, int 
     } else if (I == 1 && J == 0) {
         to_smem<double>(sB, a, g, t);
     }
+    idle(1);
     group_bar(bar);
     if (I == 1 && J == 0) {                                          // T = B A^-1
         Tile<double> ai, tt;
@@ -242,6 +251,7 @@ SELINV_DEVINL void qinverse_schur(w16::Tile<double> &a, double *buf, int I, int 
         det.renorm();
         to_smem<double>(sSi, a, g, t);
     }
+    idle(3);
     group_bar(bar);
     if (!(I == 1 && J == 1)) {
         Tile<double> si, tT;
@@ -262,11 +272,17 @@ SELINV_DEVINL void qinverse_schur(w16::Tile<double> &a, double *buf, int I, int 
     }
 }
 
-template <class T>
-SELINV_DEVINL void qinverse(w16::Tile<T> &a, T *cbuf, int I, int J, int g, int t, int bar, LogAcc &det, bool &bad)
+template <class T, class Idle = NoIdle>
+SELINV_DEVINL void qinverse(w16::Tile<T> &a, T *cbuf, int I, int J, int g, int t, int bar, LogAcc &det, bool &bad,
+                            const Idle &idle = Idle())
 {
-    if constexpr (sizeof(T) == 8) qinverse_schur(a, cbuf, I, J, g, t, bar, det, bad);
-    else qinverse_scalar(a, cbuf, I, J, g, t, bar, det, bad);
+    if constexpr (sizeof(T) == 8) {
+        qinverse_schur(a, cbuf, I, J, g, t, bar, det, bad, idle);
+    } else {
+        idle(1);
+        idle(3);
+        qinverse_scalar(a, cbuf, I, J, g, t, bar, det, bad);
+    }
 }
 
 // Copy n elements (a multiple of 16 bytes) from shared to global memory, or
