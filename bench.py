@@ -93,9 +93,10 @@ def source_hash(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged since."""
-    path = os.path.join(PROFILES, f"{kernel}__{workload}.md")
+def profiled_traffic(kernel: str, workload: str, dtype: str = "f64"):
+    """DRAM bytes per launch from the committed ncu summary of this dtype, if the kernel is unchanged since."""
+    suffix = "" if dtype == "f64" else f"_{dtype}"
+    path = os.path.join(PROFILES, f"{kernel}__{workload}{suffix}.md")
     if not os.path.exists(path):
         return None
     txt = open(path).read()
@@ -730,21 +731,24 @@ def measure(w, dtype, op, batch, steps, warmup, rank, world, local, full_size, w
     hbm_achieved = byt / (t_ms / 1e3) / 1e9
     flops = algorithmic_flops(w, batch, op)
     flop_rate = flops / (t_ms / 1e3) / 1e12
-    traffic = profiled_traffic(kernel, w.name) if full_size else None
-    if traffic is not None and dtype != "f64":
-        traffic = None                         # the committed summaries are float64 captures
+    traffic = profiled_traffic(kernel, w.name, dtype) if full_size else None
     hbm_src = f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback 6650 GB/s"
     ridge = 35.5e12 / (hbm * 1e9)                      # FP64 flop per byte where the two roofs meet
     contraction = w.kind == "junction" and flops / byt > ridge
     hbm_side = {"achieved": hbm_achieved, "peak": hbm, "unit": "GB/s", "frac": hbm_achieved / hbm,
                 "peak_source": hbm_src}
-    if (w.b >= 32 or op == "backward" or contraction) and dtype == "f64":
+    # the segmented b = 32 path reads and writes float32 but computes in float64
+    # (operands widened in registers, the FP64 tensor-core products and inverse)
+    arith = "f64" if dtype == "f64" or kernel == "seg_collect_kernel" else dtype
+    if (w.b >= 32 or op == "backward" or contraction) and arith == "f64":
         # arithmetic intensity 7 b^3 / (32 b^2) flop/byte: past the FP64 ridge from b = 32 on
         peak = fp64_peak_cached(torch)
         roof = {"bound": "tensor", "achieved": flop_rate, "peak": peak, "unit": "TFLOP/s",
                 "frac": flop_rate / peak, "traffic": traffic,
                 "peak_source": "measured in this run: cuBLAS DGEMM 8192^3 (FP64 tensor cores)",
                 "algorithmic_flops_per_launch": flops, "kernel": kernel, "hbm": hbm_side}
+        if arith != dtype:
+            roof["note"] = f"{dtype} inputs and outputs, float64 arithmetic on the FP64 tensor cores"
     elif w.b >= 32:
         # fp32 runs on the FP32 pipes: 148 SMs x 128 lanes x 2 flop x 1965 MHz
         peak = 148 * 128 * 2 * 1.965e9 / 1e12
@@ -761,7 +765,9 @@ def measure(w, dtype, op, batch, steps, warmup, rank, world, local, full_size, w
                         "back-to-back calls (warm L2)")
     res = {"value": value, "ms_per_step": elapsed_ms / K, "kernel_ms": kernel_ms, "roofline": roof,
            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": K * launches_per_step, "clocks": clk.summary(),
-           "kernel": kernel, "config": config_dict(w, batch, world, op, full_size), "dtype": dtype}
+           "kernel": kernel, "config": config_dict(w, batch, world, op, full_size), "dtype": arith}
+    if arith != dtype:
+        res["data_dtype"] = dtype
     if device_us is not None:
         res["device_us_per_call"] = device_us
     del S, step, out, dev_in, host_in
@@ -806,7 +812,7 @@ def run_ours(args):
                             want_cpu, not args.no_e2e)
             per_config[key] = {k: r[k] for k in ("value", "ms_per_step", "kernel_ms", "roofline", "cpu_baseline",
                                                  "e2e", "clocks", "gpu_launches", "dtype", "config")}
-            for k in ("device_us_per_call",):
+            for k in ("device_us_per_call", "data_dtype"):
                 if k in r:
                     per_config[key][k] = r[k]
     if world > 1:
@@ -817,7 +823,7 @@ def run_ours(args):
         "metric": metric_name(args.op, args.dtype),
         "value": head["value"], "unit": "blocks/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": args.dtype, "data": "synthetic",
+        "dtype": head["dtype"], "data": "synthetic",
         "config": head["config"],
         "roofline": head["roofline"],
         "cpu_baseline": head["cpu_baseline"],
@@ -827,8 +833,9 @@ def run_ours(args):
         "clocks": head["clocks"],
         "kernel_ms": head["kernel_ms"],
     }
-    if "device_us_per_call" in head:
-        line["device_us_per_call"] = head["device_us_per_call"]
+    for k in ("device_us_per_call", "data_dtype"):
+        if k in head:
+            line[k] = head[k]
     if per_config is not None:
         line["per_config"] = per_config
     print(json.dumps(line), flush=True)
