@@ -380,7 +380,10 @@ selinv_status selinv_junction_solve(const selinv_junction_plan_t *plan, selinv_d
  * parent [trees, n] int32, exactly one root per tree with parent = -1, no
  * cycles, indices in [0, n)), builds the level-set schedule -- nodes grouped
  * by height for the collect sweep and by depth for the distribute sweep,
- * children in ascending index -- and copies it to the current device.
+ * children in ascending index, each node's position in its parent's child
+ * list, and the chains of first children whose heads the distribute sweep,
+ * a draw's and the backward's parents-first pass take in depth order -- and
+ * copies it to the current device.
  * (gabp-sparse-inv, "Implemented and tested kernels" -> Tree, and the
  * level-set batched path of "General sparse selected inverse": one batched
  * step per elimination level.)  The plan is owned by the library until
@@ -395,18 +398,19 @@ selinv_status selinv_tree_plan(const int32_t *parent, int64_t trees, int64_t n,
 void selinv_tree_plan_free(selinv_tree_plan_t *plan);
 
 /*
- * Dependency waits of the tree sweeps.  A node of the distribute sweep (and
- * of a draw's and the backward's parents-first pass) waits for its parent's
- * completion flag with a bounded spin: after spin_limit polls (each at least
+ * Dependency waits of the tree sweeps.  A chain head of the distribute sweep
+ * (and of a draw's and the backward's parents-first pass) waits for its
+ * parent's completion flag with a bounded spin: after spin_limit polls (each at least
  * 32-64 ns apart) it gives up, writes info = -2 for its tree (outputs of that
  * tree unspecified) and marks itself failed, so its own descendants give up
  * at once; the other trees are unaffected and the call returns normally.  A
  * valid plan never reaches the limit: every parent is handed to a running
  * warp before its children.  Default spin_limit 4194304 (values < 1 restore
  * it).  withhold: a node (global index tree * n + v) whose completion the
- * sweeps never publish, or -1 for none -- a test hook that makes the waits
- * of that node's children run out.  Host only; applies to later calls with
- * this plan.
+ * sweeps never publish, or -1 for none -- a test hook that makes that
+ * node's children give up (those that wait run out their bound; its first
+ * child, which follows it in a chain without waiting, gives up at once).
+ * Host only; applies to later calls with this plan.
  */
 selinv_status selinv_tree_plan_set_wait(selinv_tree_plan_t *plan, int32_t spin_limit, int64_t withhold);
 
